@@ -1,0 +1,400 @@
+"""Float64 CPU oracle of the tiered-KV decode path (TEST INFRASTRUCTURE ONLY).
+
+Imported only by tests, ``__graft_entry__.smoke()`` and the CPU legs of
+``bench.py``. It shares no code with the CUDA path and imports nothing from the
+product package.
+
+Everything is float64 except where floating point decides an integer: the INT2
+code of an element and the fp16 scale/zero are decided in float32 with
+round-to-nearest-even, exactly as written below, so that the CUDA path can take
+the same decisions in the same precision.
+
+Pins (tests that tie each function to something other than itself):
+
+* attend -- brute force with scalar ``math.exp`` loops; uniform-key and
+  single-token closed forms; G=1 reduces to plain multi-head attention.
+* int2_quantize -- inputs already on the grid {z, z+s, z+2s, z+3s} round-trip
+  exactly; a constant group gives s = 0 and all codes 0; hand-worked groups in
+  ``tests/golden/int2_groups.txt``.
+* vwo_l1norm -- W_O = identity reduces to ||V_i||_1; permutation/sign
+  invariance; hand-worked case.
+* two_stage -- exhaustive enumeration of subsets on small sets; hand-worked
+  routing fixture in ``tests/golden/two_stage.txt``.
+* QEvictUnit -- per-step mass invariant (sum over live windows = G);
+  write-once ledger (demote -> promote -> demote yields identical codes);
+  with budgets covering every window it reduces to plain attention.
+* observation_mass -- brute force; sum over keys of A = G * n_obs.
+* trim_global_topm -- closed forms: constant beta keeps the most recent
+  entries, equal age keeps the larger beta, beta = 1 everywhere ties and keeps
+  the lowest flat indices; compared with ``np.argsort`` on tiny sets.
+* output_perturbation -- diagnostic only (parity unpinned: the pages give no
+  value for it and the bound theta is not printed).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+EVICTED, INT2, FULL, TAIL = 0, 1, 2, 3
+GROUP = 16  # INT2 group: 16 consecutive head-dim elements of one token
+
+# ---------------------------------------------------------------------------
+# dtype helpers (oracle-private; not shared with any other module)
+# ---------------------------------------------------------------------------
+
+
+def _f32_to_bf16(x32: np.ndarray) -> np.ndarray:
+    """float32 -> bfloat16 round-to-nearest-even, returned as float64 values."""
+    u = np.ascontiguousarray(x32, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    r = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
+    return r.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def round_to_cache_dtype(x32: np.ndarray, dtype: str) -> np.ndarray:
+    """Round float32 values once to the cache dtype; float64 result."""
+    x32 = np.asarray(x32, dtype=np.float32)
+    if dtype == "bf16":
+        return _f32_to_bf16(x32)
+    if dtype == "fp16":
+        return x32.astype(np.float16).astype(np.float64)
+    raise ValueError(dtype)
+
+
+# ---------------------------------------------------------------------------
+# attention ("Resumo Técnico: QEvict", Implementação: GQA decode path)
+# ---------------------------------------------------------------------------
+
+
+def attend(q: np.ndarray, K: np.ndarray, V: np.ndarray):
+    """Softmax attention of one query head over n keys.
+
+    s_i = q.K_i / sqrt(D); p = softmax(s) (max-subtracted); o = sum_i p_i V_i.
+    Returns (o [D], p [n]).
+    """
+    D = q.shape[-1]
+    s = (K @ q) / math.sqrt(D)
+    s = s - s.max()
+    e = np.exp(s)
+    p = e / e.sum()
+    return p @ V, p
+
+
+# ---------------------------------------------------------------------------
+# INT2 recoverable tier ("Resumo Técnico: QEvict", Metodologia 2)
+# ---------------------------------------------------------------------------
+
+
+def int2_quantize(x: np.ndarray):
+    """Asymmetric INT2 quantisation of [T][D] values in groups of 16 elements.
+
+    Per group (16 consecutive head-dim elements of one token):
+      mn, mx = min, max                          (exact)
+      s = fp16( f32(mx - mn) / 3 )               (float32 ops, RNE to fp16)
+      z = fp16( mn )
+      code = clamp( rint( f32(x - z) / s ), 0, 3 ), code = 0 where s == 0
+    All operations are float32 with round-to-nearest-even (rint: half to even).
+    Returns (codes uint8 [T][D], s float16 [T][D/16], z float16 [T][D/16]).
+    """
+    T, D = x.shape
+    g = np.asarray(x, dtype=np.float32).reshape(T, D // GROUP, GROUP)
+    mn = g.min(axis=-1)
+    mx = g.max(axis=-1)
+    s16 = ((mx - mn) / np.float32(3.0)).astype(np.float16)
+    z16 = mn.astype(np.float16)
+    s32 = s16.astype(np.float32)[..., None]
+    z32 = z16.astype(np.float32)[..., None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        t = (g - z32) / s32
+    codes = np.clip(np.rint(t), 0, 3)
+    codes = np.where(s32 == 0, 0, codes).astype(np.uint8)
+    return codes.reshape(T, D), s16, z16
+
+
+def int2_dequantize(codes: np.ndarray, s16: np.ndarray, z16: np.ndarray) -> np.ndarray:
+    """x_hat = code * s + z, exact in float64. Shapes as returned by int2_quantize."""
+    T, D = codes.shape
+    c = codes.reshape(T, D // GROUP, GROUP).astype(np.float64)
+    x = c * s16.astype(np.float64)[..., None] + z16.astype(np.float64)[..., None]
+    return x.reshape(T, D)
+
+
+def int2_promote_values(codes, s16, z16, dtype: str) -> np.ndarray:
+    """Values a promoted window holds in the full-precision tier.
+
+    The full tier stores the cache dtype, so dequant(code) is rounded to it:
+    first to float32 (one rounding of the exact code*s+z), then to fp16/bf16.
+    """
+    x32 = int2_dequantize(codes, s16, z16).astype(np.float32)
+    return round_to_cache_dtype(x32, dtype)
+
+
+# ---------------------------------------------------------------------------
+# projected-value norms ("Resumo Técnico: CriticalKV", Framework Teórico)
+# ---------------------------------------------------------------------------
+
+
+def vwo_l1norm(V: np.ndarray, W_O: np.ndarray, heads, D: int, chunk: int = 4096) -> np.ndarray:
+    """N[i, j] = || V_i @ W_O[h_j*D:(h_j+1)*D, :] ||_1 for each query head h_j.
+
+    V: [n][D]; W_O: [Hq*D][hidden] with y = concat_h(o_h) @ W_O, so W_O^h is the
+    row block h*D .. h*D+D-1. Returns [n][len(heads)] float64.
+    """
+    V = np.asarray(V, dtype=np.float64)
+    out = np.empty((V.shape[0], len(heads)))
+    for j, h in enumerate(heads):
+        Wh = np.asarray(W_O[h * D:(h + 1) * D, :], dtype=np.float64)
+        for a in range(0, V.shape[0], chunk):
+            out[a:a + chunk, j] = np.abs(V[a:a + chunk] @ Wh).sum(axis=1)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# two-stage selection ("Resumo Técnico: CriticalKV", Algoritmo, Etapas 1 e 2)
+# ---------------------------------------------------------------------------
+
+
+def top_b(ids: np.ndarray, score: np.ndarray, b: int) -> np.ndarray:
+    """The b ids with the highest score; ties go to the lower id."""
+    ids = np.asarray(ids)
+    if b <= 0 or ids.size == 0:
+        return ids[:0]
+    order = np.lexsort((ids, -score[ids]))
+    return ids[order[:b]]
+
+
+def two_stage(ids: np.ndarray, attn: np.ndarray, pert: np.ndarray, b: int, alpha: float):
+    """Two-stage greedy selection of b items out of ``ids``.
+
+    If |ids| <= b every item is kept. Otherwise b' = floor(alpha*b) items with
+    the highest attention score are taken first, then b - b' items with the
+    highest perturbation score among the rest. ``attn`` and ``pert`` are indexed
+    by id. Returns (stage1 ids, stage2 ids).
+    """
+    ids = np.asarray(ids)
+    if ids.size <= b:
+        return ids.copy(), ids[:0]
+    b1 = int(math.floor(alpha * b))
+    s1 = top_b(ids, attn, b1)
+    rest = np.setdiff1d(ids, s1, assume_unique=True)
+    s2 = top_b(rest, pert, b - b1)
+    return s1, s2
+
+
+# ---------------------------------------------------------------------------
+# QEvict unit ("Resumo Técnico: QEvict", Metodologia / Mecanismos Principais)
+# ---------------------------------------------------------------------------
+
+
+class QEvictUnit:
+    """One (batch, kv-head) unit of the window-routed three-tier cache.
+
+    State per window: tier (FULL / INT2 / EVICTED / TAIL), cumulative attention
+    mass and cumulative perturbation score, and the write-once INT2 ledger entry.
+    Per token: the values attention uses (``Keff``/``Veff``), the values the
+    full tier stores (``Kst``/``Vst``) and the projected-value norms n[h].
+
+    Readings where the pages are silent (each listed in the design doc):
+    the tail (newest, incomplete) window is always full precision, outside the
+    budget and not routed; scores accumulate undecayed from step 0; evicted
+    windows never return; routing runs after attention on steps s % R == 0;
+    per-kv-head scores are sums over the G query heads of the group.
+    """
+
+    def __init__(self, K0, V0, W_O, kvh: int, G: int, window: int, full_windows: int,
+                 int2_windows: int, alpha: float, dtype: str, max_tokens: int):
+        K0 = np.asarray(K0, dtype=np.float64)
+        V0 = np.asarray(V0, dtype=np.float64)
+        n0, D = K0.shape
+        self.D, self.G, self.w = D, G, window
+        self.F, self.Q, self.alpha, self.dtype = full_windows, int2_windows, alpha, dtype
+        self.heads = [kvh * G + j for j in range(G)]
+        self.W_O = W_O
+        nw = (max_tokens + window - 1) // window
+        self.Kst = np.zeros((max_tokens, D))
+        self.Vst = np.zeros((max_tokens, D))
+        self.Keff = np.zeros((max_tokens, D))
+        self.Veff = np.zeros((max_tokens, D))
+        self.norms = np.zeros((max_tokens, G))
+        self.tier = np.full(nw, EVICTED, dtype=np.int8)
+        self.mass = np.zeros(nw)
+        self.pert = np.zeros(nw)
+        self.ledger = {}
+        self.n = n0
+        self.Kst[:n0], self.Vst[:n0] = K0, V0
+        self.Keff[:n0], self.Veff[:n0] = K0, V0
+        self.norms[:n0] = vwo_l1norm(V0, W_O, self.heads, D)
+        self.tier[: n0 // window] = FULL
+        if n0 % window:
+            self.tier[n0 // window] = TAIL
+        self.last_route = None
+
+    # -- helpers --------------------------------------------------------------
+    def tokens(self, w: int) -> slice:
+        return slice(w * self.w, min((w + 1) * self.w, self.n))
+
+    def live_windows(self) -> np.ndarray:
+        # windows past the newest token are initialised EVICTED and become TAIL on append
+        return np.nonzero(self.tier != EVICTED)[0]
+
+    def live_tokens(self) -> np.ndarray:
+        return np.concatenate([np.arange(self.tokens(w).start, self.tokens(w).stop)
+                               for w in self.live_windows()])
+
+    # -- one decode step ------------------------------------------------------
+    def append(self, k, v):
+        """Write the new token's K/V at position n and compute its norms n_h."""
+        i = self.n
+        self.Kst[i], self.Vst[i] = k, v
+        self.Keff[i], self.Veff[i] = k, v
+        self.norms[i] = vwo_l1norm(np.asarray(v, dtype=np.float64)[None, :], self.W_O,
+                                   self.heads, self.D)[0]
+        self.n += 1
+        w = i // self.w
+        self.tier[w] = FULL if self.n % self.w == 0 else TAIL
+
+    def attend_and_score(self, qG):
+        """Attention of the G query heads over every live token, plus scoring.
+
+        mass_w += sum_h sum_{i in w} p_{h,i};  pert_w += sum_h sum_{i in w} p_{h,i} n_{h,i}.
+        Returns o [G][D] and the per-window mass added at this step.
+        """
+        idx = self.live_tokens()
+        K, V = self.Keff[idx], self.Veff[idx]
+        win = idx // self.w
+        o = np.empty((self.G, self.D))
+        step_mass = np.zeros_like(self.mass)
+        for j in range(self.G):
+            o[j], p = attend(np.asarray(qG[j], dtype=np.float64), K, V)
+            np.add.at(step_mass, win, p)
+            np.add.at(self.pert, win, p * self.norms[idx, j])
+        self.mass += step_mass
+        return o, step_mass
+
+    def route(self):
+        """Full = TwoStage(L, F); INT2 = TwoStage(L minus Full, Q); the rest is evicted."""
+        L = np.nonzero((self.tier == FULL) | (self.tier == INT2))[0]
+        f1, f2 = two_stage(L, self.mass, self.pert, self.F, self.alpha)
+        full = np.concatenate([f1, f2])
+        rest = np.setdiff1d(L, full, assume_unique=True)
+        q1, q2 = two_stage(rest, self.mass, self.pert, self.Q, self.alpha)
+        int2 = np.concatenate([q1, q2])
+        new = {int(w): EVICTED for w in L}
+        new.update({int(w): FULL for w in full})
+        new.update({int(w): INT2 for w in int2})
+        self.last_route = dict(L=L, full=(f1, f2), int2=(q1, q2))
+        self.apply(new)
+        return new
+
+    def apply(self, new: dict):
+        """Tier transitions with the write-once ledger.
+
+        FULL->INT2 quantises the stored values only if the window has no ledger
+        entry yet; otherwise the entry is reused. INT2->FULL writes
+        dequant(ledger) rounded to the cache dtype into the full tier and keeps
+        the entry. ->EVICTED drops the data and the entry for good.
+        """
+        for w, t in sorted(new.items()):
+            old = self.tier[w]
+            sl = self.tokens(w)
+            if old == FULL and t == INT2:
+                if w not in self.ledger:
+                    self.ledger[w] = (int2_quantize(self.Kst[sl]), int2_quantize(self.Vst[sl]))
+                (ck, sk, zk), (cv, sv, zv) = self.ledger[w]
+                self.Keff[sl] = int2_dequantize(ck, sk, zk)
+                self.Veff[sl] = int2_dequantize(cv, sv, zv)
+            elif old == INT2 and t == FULL:
+                (ck, sk, zk), (cv, sv, zv) = self.ledger[w]
+                self.Kst[sl] = int2_promote_values(ck, sk, zk, self.dtype)
+                self.Vst[sl] = int2_promote_values(cv, sv, zv, self.dtype)
+                self.Keff[sl], self.Veff[sl] = self.Kst[sl], self.Vst[sl]
+            elif t == EVICTED:
+                self.ledger.pop(w, None)
+            self.tier[w] = t
+
+    def step(self, s: int, qG, k, v, route_every: int):
+        self.append(k, v)
+        o, _ = self.attend_and_score(qG)
+        routed = None
+        if s % route_every == 0:
+            routed = self.route()
+        return o, routed
+
+
+# ---------------------------------------------------------------------------
+# CriticalKV with an observation window ("Resumo Técnico: CriticalKV", Algoritmo)
+# ---------------------------------------------------------------------------
+
+
+def observation_mass(q_obs: np.ndarray, K: np.ndarray) -> np.ndarray:
+    """A[h, i] = sum_j softmax_j(q_{h,j}.K / sqrt(D))_i over the observation queries.
+
+    q_obs [G][n_obs][D]: the queries at the last n_obs context positions; query j
+    sits at position n - n_obs + j and attends causally to keys 0..n-n_obs+j.
+    Returns A [G][n].
+    """
+    G, n_obs, D = q_obs.shape
+    n = K.shape[0]
+    K = np.asarray(K, dtype=np.float64)
+    A = np.zeros((G, n))
+    for h in range(G):
+        for j in range(n_obs):
+            last = n - n_obs + j + 1
+            s = (K[:last] @ np.asarray(q_obs[h, j], dtype=np.float64)) / math.sqrt(D)
+            e = np.exp(s - s.max())
+            A[h, :last] += e / e.sum()
+    return A
+
+
+def criticalkv_select(A: np.ndarray, N: np.ndarray, b: int, alpha: float):
+    """Stage 1 on sum_h A[h,i]; stage 2 on sum_h A[h,i] * N[i,h]. Returns (s1, s2, a, p)."""
+    a = A.sum(axis=0)
+    p = (A * N.T).sum(axis=0)
+    ids = np.arange(a.size)
+    s1, s2 = two_stage(ids, a, p, b, alpha)
+    return s1, s2, a, p
+
+
+# ---------------------------------------------------------------------------
+# DBTrimKV global top-M ("Make Each Token Count", Metodologia 2-4)
+# ---------------------------------------------------------------------------
+
+
+def retention_log(beta: np.ndarray, pos: np.ndarray, t: int) -> np.ndarray:
+    """log r_{t,i} = (t - i) * ln(beta_i), float64."""
+    return (t - np.asarray(pos, dtype=np.float64)) * np.log(np.asarray(beta, dtype=np.float64))
+
+
+def trim_global_topm(betas, poss, t: int, M: int):
+    """Keep the M entries with the highest log r over all heads (ties: lower flat index).
+
+    betas/poss: per-head arrays in head order; the flat index runs over heads
+    first, then entries. Returns (keep masks per head, new lengths, all keys).
+    """
+    keys = np.concatenate([retention_log(b, p, t) for b, p in zip(betas, poss)])
+    flat = np.arange(keys.size)
+    order = np.lexsort((flat, -keys))
+    keep = np.zeros(keys.size, dtype=bool)
+    keep[order[:M]] = True
+    masks, lens, a = [], [], 0
+    for b in betas:
+        m = keep[a:a + b.size]
+        masks.append(m)
+        lens.append(int(m.sum()))
+        a += b.size
+    return masks, np.array(lens, dtype=np.int64), keys
+
+
+# ---------------------------------------------------------------------------
+# output perturbation ("Resumo Técnico: CriticalKV", Definição de Perturbação)
+# ---------------------------------------------------------------------------
+
+
+def output_perturbation(q, K, V, subset, W_O_h=None) -> float:
+    """L = ||o - o_hat||_1 between full-cache and subset attention (optionally projected)."""
+    o, _ = attend(q, K, V)
+    oh, _ = attend(q, K[subset], V[subset])
+    d = o - oh
+    if W_O_h is not None:
+        d = d @ np.asarray(W_O_h, dtype=np.float64)
+    return float(np.abs(d).sum())
