@@ -1,0 +1,256 @@
+/*
+ * qevict.h - C ABI of the tiered KV-cache decode library (libqevict.so, sm_100a).
+ *
+ * One decode step of grouped-query attention over a window-partitioned paged KV
+ * cache that holds a full-precision tier (fp16/bf16) and a recoverable INT2 tier,
+ * fused with cumulative window scoring, budgeted two-stage routing of every window
+ * to full / INT2 / evicted, and a write-once INT2 ledger. Sources:
+ *   "Resumo Técnico: QEvict"  - Metodologia (three tiers under a fixed budget),
+ *       Mecanismos Principais (window-level routing, cumulative scoring, demotion,
+ *       promotion, write-once quantisation ledger, GQA decode path).
+ *   "Resumo Técnico: CriticalKV" - Framework Teórico (perturbation L = ||o - o_hat||_1,
+ *       projected values V W_O), Algoritmo (two-stage greedy, b' = alpha*b, alpha = 0.5,
+ *       then A_i * ||V_i W_O||_1 on the remaining budget).
+ *   "Make Each Token Count" (DBTrimKV) - Metodologia 2 (retention r = beta^(t-i)),
+ *       3 (one global budget M over layers and heads), 4 (paged variable-length heads).
+ *
+ * Conventions (every entry point):
+ *   - Pointers marked [dev] are device pointers, [host] are host pointers. The caller
+ *     owns every buffer; the library never allocates device memory (cudaMalloc) itself.
+ *   - Every call that takes a cudaStream_t is asynchronous on that stream and returns
+ *     after enqueueing. Arguments are validated on the host before anything is enqueued.
+ *   - Return value: QE_OK (0) or a negative QE_ERR_*. Errors found by a kernel (pool
+ *     exhausted, an index out of range, a bounded wait that gave up) are recorded in the
+ *     context's device status word; read them with qe_status() after synchronising.
+ *     No kernel traps or asserts; a failing kernel records the error and returns.
+ *   - Row-major layouts. The cache dtype (fp16 or bf16) is fixed at qe_create.
+ *   - No C++ exception crosses this boundary.
+ */
+#ifndef QEVICT_H
+#define QEVICT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define QE_API __attribute__((visibility("default")))
+
+typedef struct CUstream_st* qe_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+enum {
+  QE_OK = 0,
+  QE_ERR_INVALID_ARG = -1,      /* NULL pointer, bad size, misaligned buffer        */
+  QE_ERR_UNSUPPORTED_SHAPE = -2,/* D not in {64,128}, G > 8, window not in {16..64} */
+  QE_ERR_POOL_EXHAUSTED = -3,   /* a unit's page free list ran empty (device)       */
+  QE_ERR_LEDGER_FULL = -4,      /* a unit's INT2 ledger ran out of slots (device)   */
+  QE_ERR_CUDA = -5,             /* a CUDA runtime call failed                        */
+  QE_ERR_TIMEOUT = -6,          /* a bounded device wait gave up (device)            */
+  QE_ERR_DEVICE_FAULT = -7,     /* an index read from device state was out of range  */
+  QE_ERR_WORKSPACE = -8,        /* workspace smaller than qe_workspace_bytes()       */
+  QE_ERR_STATE = -9             /* call out of order (e.g. decode before prefill)    */
+};
+
+enum { QE_FP16 = 0, QE_BF16 = 1 };
+
+/* Window tiers as stored in the tier map (one byte per window). */
+enum { QE_TIER_EVICTED = 0, QE_TIER_INT2 = 1, QE_TIER_FULL = 2, QE_TIER_TAIL = 3 };
+
+/*
+ * qe_config - shape and budgets of one decode context (one attention layer).
+ * A "unit" is one (batch b, kv-head g) pair; units are independent and numbered
+ * u = b*Hkv + g. Budgets are per unit and counted in windows.
+ */
+typedef struct {
+  int B, Hq, Hkv, D;          /* batch, query heads, KV heads, head dim (64 or 128)      */
+  int dtype;                  /* QE_FP16 or QE_BF16: cache, query and W_O element type   */
+  int page;                   /* tokens per page; must be 16                              */
+  int window;                 /* tokens per routing window: 16, 32 or 64                  */
+  int full_windows;           /* F: full-precision budget per unit (windows)              */
+  int int2_windows;           /* Q: INT2 budget per unit (windows)                        */
+  float alpha;                /* stage-1 share of each budget (0.5 on the pages)          */
+  int route_every;            /* R: route after attention on decode steps s % R == 0      */
+  int hidden;                 /* columns of W_O                                           */
+  int max_ctx;                /* capacity in tokens per unit (prefill + decode)           */
+  int pages_per_unit;         /* page-pool capacity per unit (>= ceil(prefill/16) + margin)*/
+  int slots_per_unit;         /* INT2 ledger capacity per unit (>= F + Q)                 */
+  int max_splits;             /* upper bound on split-K blocks per unit (1..64)           */
+} qe_config;
+
+/* Byte offsets of the state arrays inside the caller's workspace (see qe_layout). */
+typedef struct {
+  size_t total;               /* bytes the workspace must hold                            */
+  size_t pages;               /* [U][pages_per_unit][2][16][D] cache dtype: K rows, V rows */
+  size_t page_free;           /* [U][pages_per_unit] int32 free-page stack per unit       */
+  size_t win_pages;           /* [U][max_windows][window/16] int32 page of each window    */
+  size_t win_tier;            /* [U][max_windows] uint8 QE_TIER_*                          */
+  size_t win_slot;            /* [U][max_windows] int32 ledger slot or -1                 */
+  size_t slots;               /* [U][slots_per_unit][window*D] bytes: INT2 ledger entries  */
+  size_t slot_free;           /* [U][slots_per_unit] int32 free-slot stack per unit       */
+  size_t mass;                /* [U][max_windows] float cumulative attention mass         */
+  size_t pert;                /* [U][max_windows] float cumulative perturbation score     */
+  size_t norms;               /* [U][max_ctx][G] float ||V_i W_O^h||_1 per token and head */
+  size_t full_list;           /* [U][max_windows] int32 windows in the full tier          */
+  size_t int2_list;           /* [U][max_windows] int32 windows in the INT2 tier          */
+  size_t tail_p;              /* [U][window][G] float cumulative attention of tail tokens */
+  size_t stacks;              /* [U][4] int32: page-stack top, slot-stack top, -, -       */
+  size_t route_stats;         /* [U][8] int32: promotions, new demotions, reused demotions,
+                                 evictions, full kept, int2 kept, -, stage-1 mass x 1e6    */
+  size_t status;              /* [4] int32 device status word (first error, detail)       */
+  size_t scratch;             /* split-K partials, window partials, transition lists       */
+  size_t scratch_bytes;
+  int max_windows;            /* ceil(max_ctx / window)                                    */
+  int units;                  /* B * Hkv                                                   */
+} qe_layout;
+
+typedef struct qe_ctx qe_ctx; /* opaque host object; owns no device memory */
+
+/* Per-call statistics of the most recent routing event, summed over units. */
+typedef struct {
+  long long promotions, demotions_new, demotions_reused, evictions;
+} qe_route_totals;
+
+/* qe_plan - fill *out with the workspace size and state-array offsets for *cfg.
+ * [host] cfg, out. Returns QE_ERR_UNSUPPORTED_SHAPE / QE_ERR_INVALID_ARG on a bad config. */
+QE_API int qe_plan(const qe_config* cfg, qe_layout* out);
+
+/* qe_workspace_bytes - bytes of device workspace qe_create needs (0 on a bad config). */
+QE_API size_t qe_workspace_bytes(const qe_config* cfg);
+
+/* qe_create - bind a context to a caller-allocated device workspace.
+ *   workspace [dev]: at least qe_workspace_bytes(cfg) bytes, 256-byte aligned; the
+ *                    library keeps every piece of state in it and never frees it.
+ *   W_O [dev]:       [Hq*D][hidden] in the cache dtype; y = concat_h(o_h) @ W_O, so the
+ *                    rows h*D..h*D+D-1 are W_O^h. Must outlive the context.
+ *   out [host]:      receives the context.
+ * The context is host-only state (shape, step counter, pointers into the workspace). */
+QE_API int qe_create(const qe_config* cfg, void* workspace, size_t workspace_bytes,
+                     const void* W_O, qe_ctx** out);
+
+/* qe_destroy - free the host context. The workspace stays the caller's. */
+QE_API int qe_destroy(qe_ctx* ctx);
+
+/* qe_load_prefill - reset the context and load a prefill cache of ctx_len tokens.
+ *   K, V [dev]: [B][Hkv][ctx_len][D] cache dtype. Every complete window goes to the
+ *   full tier; an incomplete last window becomes the tail. Computes ||V_i W_O^h||_1 for
+ *   every prefill token on tensor cores. Scores start at 0. (QEvict, Metodologia.) */
+QE_API int qe_load_prefill(qe_ctx* ctx, const void* K, const void* V, int ctx_len,
+                           qe_stream_t stream);
+
+/* qe_kv_append - append one token per unit at position n (the current length).
+ *   k_new, v_new [dev]: [B][Hkv][D] cache dtype. Takes a fresh page from the unit's free
+ *   list at every 16th token. (QEvict, Metodologia: states appended during decoding.) */
+QE_API int qe_kv_append(qe_ctx* ctx, const void* k_new, const void* v_new, qe_stream_t stream);
+
+/* qe_decode_attend_and_score - GQA decode attention over every live token of both tiers.
+ *   q [dev]: [B][Hq][D] cache dtype; query head h uses kv head h / (Hq/Hkv).
+ *   out [dev]: [B][Hq][D] float32 attention output o_h = sum_i p_{h,i} V_i.
+ *   INT2 tokens are dequantised in registers (code*s + z). Fused with the scoring of
+ *   "Resumo Técnico: QEvict" (Pontuação Cumulativa) and "Resumo Técnico: CriticalKV"
+ *   (Etapa 2): for every live window w of unit (b,g),
+ *     mass[w] += sum_{h in g} sum_{i in w} p_{h,i}
+ *     pert[w] += sum_{h in g} sum_{i in w} p_{h,i} * ||V_i W_O^h||_1.
+ *   When this step completes the tail window, its norms are computed (tensor cores) and it
+ *   joins the full tier as a routing candidate. */
+QE_API int qe_decode_attend_and_score(qe_ctx* ctx, const void* q, float* out,
+                                      qe_stream_t stream);
+
+/* qe_route_windows - two-stage budgeted routing of every live complete window, then the
+ * tier transitions (QEvict Metodologia + CriticalKV Algoritmo):
+ *   Full = TwoStage(L, F); INT2 = TwoStage(L \ Full, Q); the rest is evicted for good.
+ *   TwoStage(S, b): all of S if |S| <= b, else the floor(alpha*b) highest mass, then the
+ *   b - floor(alpha*b) highest pert among the rest; ties go to the lower window index.
+ * Demotions quantise only windows with no ledger entry yet (write-once); promotions write
+ * dequant(ledger) rounded to the cache dtype into fresh pages and keep the entry.
+ *   totals [host, may be NULL]: not filled asynchronously; pass NULL and read the
+ *   route_stats array of the layout instead. */
+QE_API int qe_route_windows(qe_ctx* ctx, qe_stream_t stream);
+
+/* qe_decode_step - one whole decode step: kv_append, decode_attend_and_score and, on steps
+ * s % R == 0 (s counted from the prefill), route_windows. Arguments as above. */
+QE_API int qe_decode_step(qe_ctx* ctx, const void* q, const void* k_new, const void* v_new,
+                          float* out, qe_stream_t stream);
+
+/* qe_quantize_once - demote the listed windows of one unit to the INT2 tier.
+ *   win_ids [host]: n window indices of unit `unit`, each currently in the full tier.
+ *   A window that already has a ledger entry reuses it (no re-quantisation).
+ * (QEvict, Hierarquia Recuperável: Rebaixamento + write-once ledger.) */
+QE_API int qe_quantize_once(qe_ctx* ctx, int unit, const int32_t* win_ids, int n,
+                            qe_stream_t stream);
+
+/* qe_promote - promote the listed INT2 windows of one unit back to the full tier; their
+ * pages receive dequant(ledger) rounded to the cache dtype; the ledger entry is kept.
+ * (QEvict, Hierarquia Recuperável: Promoção.) */
+QE_API int qe_promote(qe_ctx* ctx, int unit, const int32_t* win_ids, int n,
+                      qe_stream_t stream);
+
+/* qe_int2_quantize - standalone INT2 group quantiser (the one the ledger uses).
+ *   x [dev]: [T][D] cache dtype, D a multiple of 16. codes [dev]: [T][D/4] bytes, byte j of
+ *   a token holds elements 4j..4j+3, element 4j+e in bits 2e..2e+1. meta [dev]: [T][D/16]
+ *   pairs of fp16 (scale s, zero z), s in the low half. Per 16-element group:
+ *   s = fp16(f32(max-min)/3), z = fp16(min), code = clamp(rint(f32(x-z)/s), 0, 3), 0 if s==0. */
+QE_API int qe_int2_quantize(const void* x, int T, int D, int dtype, uint8_t* codes,
+                            uint32_t* meta, qe_stream_t stream);
+
+/* qe_vwo_l1norm - N[g][r][j] = || V[g][r][:] @ W_O^{h} ||_1 with h = (g % Hkv)*G + j, on
+ * tensor cores (tcgen05, accumulators in TMEM).
+ *   V [dev]: [n_groups][rows][D] dtype. W_O [dev]: [Hq*D][hidden] dtype.
+ *   out [dev]: float, element (g, r, j) at out[g*out_group_stride + r*G + j].
+ * ("Resumo Técnico: CriticalKV", Framework Teórico: projected values V W_O.) */
+QE_API int qe_vwo_l1norm(const void* V, int n_groups, int rows, int D, int dtype,
+                         const void* W_O, int Hq, int Hkv, int hidden, float* out,
+                         long long out_group_stride, qe_stream_t stream);
+
+/* qe_criticalkv_select - CriticalKV two-stage selection per (batch, kv head) with a
+ * SnapKV-style observation window ("Resumo Técnico: CriticalKV", Algoritmo).
+ *   q_obs [dev]: [B][Hq][n_obs][D] queries of the last n_obs positions (causal).
+ *   K, V [dev]: [B][Hkv][n][D]. W_O [dev]: [Hq*D][hidden].
+ *   A_out [dev, float]: [B][Hkv][G][n] observation attention mass per query head.
+ *   N_out [dev, float]: [B][Hkv][n][G] ||V_i W_O^h||_1.
+ *   idx_out [dev, int32]: [B][Hkv][budget] selected token indices: stage-1 picks in
+ *   descending score order, then stage-2 picks in descending score order.
+ *   scratch [dev]: qe_criticalkv_scratch_bytes() bytes. */
+QE_API size_t qe_criticalkv_scratch_bytes(int B, int Hq, int Hkv, int n, int n_obs);
+QE_API int qe_criticalkv_select(const void* q_obs, int n_obs, const void* K, const void* V,
+                                const void* W_O, int B, int Hq, int Hkv, int n, int D,
+                                int hidden, int dtype, int budget, float alpha,
+                                float* A_out, float* N_out, int32_t* idx_out,
+                                void* scratch, size_t scratch_bytes, qe_stream_t stream);
+
+/* qe_trim_global_topm - DBTrimKV global top-M over log r = (t - pos) * ln(beta) in float64
+ * across every (layer, head) of a paged variable-length cache ("Make Each Token Count",
+ * Metodologia 2-4). Ties go to the lower flat index (head-major, then entry).
+ *   beta [dev, float], pos [dev, int32]: [n_pages_total][16] per physical page.
+ *   page_table [dev, int32]: [n_heads][max_pages_per_head] physical page of each logical page.
+ *   lengths [dev, int32]: [n_heads].  kv_in [dev]: [n_pages_total][2][16][D] dtype.
+ *   kv_out, beta_out, pos_out [dev]: same shapes as the inputs; head h's survivors are
+ *   written in their original order to its logical pages 0.. through the same page table.
+ *   new_lengths [dev, int32]: [n_heads]. scratch [dev]: qe_trim_scratch_bytes() bytes. */
+QE_API size_t qe_trim_scratch_bytes(int n_heads, int max_pages_per_head);
+QE_API int qe_trim_global_topm(const float* beta, const int32_t* pos, const int32_t* page_table,
+                               const int32_t* lengths, int n_heads, int max_pages_per_head,
+                               int D, int dtype, int t, long long M, const void* kv_in,
+                               void* kv_out, float* beta_out, int32_t* pos_out,
+                               int32_t* new_lengths, void* scratch, size_t scratch_bytes,
+                               qe_stream_t stream);
+
+/* qe_status - copy the device status word to the host (synchronises the context's last
+ * stream) and return the first recorded error, or QE_OK. *detail (may be NULL) receives the
+ * failing index or unit. */
+QE_API int qe_status(qe_ctx* ctx, int* detail);
+
+/* qe_step_index - decode steps taken since the last prefill; qe_length - tokens per unit. */
+QE_API int qe_step_index(const qe_ctx* ctx);
+QE_API int qe_length(const qe_ctx* ctx);
+/* qe_list_counts - full-tier and INT2-tier window counts (identical for every unit). */
+QE_API int qe_list_counts(const qe_ctx* ctx, int* n_full, int* n_int2);
+
+/* qe_strerror - static message for a QE_* code. */
+QE_API const char* qe_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QEVICT_H */

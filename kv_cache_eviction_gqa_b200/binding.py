@@ -1,0 +1,310 @@
+"""Python binding of libqevict (argument marshalling only).
+
+Every function here forwards to the C ABI declared in ``include/qevict.h``; all
+computation runs in the library's CUDA kernels. PyTorch supplies device memory
+(the context workspace and the inputs/outputs) and the current CUDA stream.
+If the shared library is missing, every call raises RuntimeError: there is no
+fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from dataclasses import dataclass
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqevict.so")
+_lib = None
+
+QE_FP16, QE_BF16 = 0, 1
+TIER_EVICTED, TIER_INT2, TIER_FULL, TIER_TAIL = 0, 1, 2, 3
+
+
+class QeConfig(C.Structure):
+    _fields_ = [(n, C.c_int) for n in ("B", "Hq", "Hkv", "D", "dtype", "page", "window",
+                                        "full_windows", "int2_windows")] + \
+               [("alpha", C.c_float)] + \
+               [(n, C.c_int) for n in ("route_every", "hidden", "max_ctx", "pages_per_unit",
+                                        "slots_per_unit", "max_splits")]
+
+
+class QeLayout(C.Structure):
+    _fields_ = [(n, C.c_size_t) for n in ("total", "pages", "page_free", "win_pages", "win_tier",
+                                           "win_slot", "slots", "slot_free", "mass", "pert", "norms",
+                                           "full_list", "int2_list", "tail_p", "stacks", "route_stats",
+                                           "status", "scratch", "scratch_bytes")] + \
+               [("max_windows", C.c_int), ("units", C.c_int)]
+
+
+def lib():
+    """Load libqevict.so (raises RuntimeError if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"libqevict.so not found at {_LIB_PATH}; build it with "
+                               "`python -m kv_cache_eviction_gqa_b200.build`")
+        L = C.CDLL(_LIB_PATH)
+        vp, i, sz, f, ll = C.c_void_p, C.c_int, C.c_size_t, C.c_float, C.c_longlong
+        sig = {
+            "qe_plan": (i, [C.POINTER(QeConfig), C.POINTER(QeLayout)]),
+            "qe_workspace_bytes": (sz, [C.POINTER(QeConfig)]),
+            "qe_create": (i, [C.POINTER(QeConfig), vp, sz, vp, C.POINTER(vp)]),
+            "qe_destroy": (i, [vp]),
+            "qe_load_prefill": (i, [vp, vp, vp, i, vp]),
+            "qe_kv_append": (i, [vp, vp, vp, vp]),
+            "qe_decode_attend_and_score": (i, [vp, vp, vp, vp]),
+            "qe_route_windows": (i, [vp, vp]),
+            "qe_decode_step": (i, [vp, vp, vp, vp, vp, vp]),
+            "qe_quantize_once": (i, [vp, i, vp, i, vp]),
+            "qe_promote": (i, [vp, i, vp, i, vp]),
+            "qe_int2_quantize": (i, [vp, i, i, i, vp, vp, vp]),
+            "qe_vwo_l1norm": (i, [vp, i, i, i, i, vp, i, i, i, vp, ll, vp]),
+            "qe_criticalkv_scratch_bytes": (sz, [i, i, i, i, i]),
+            "qe_criticalkv_select": (i, [vp, i, vp, vp, vp, i, i, i, i, i, i, i, i, f, vp, vp, vp,
+                                         vp, sz, vp]),
+            "qe_trim_scratch_bytes": (sz, [i, i]),
+            "qe_trim_global_topm": (i, [vp, vp, vp, vp, i, i, i, i, i, ll, vp, vp, vp, vp, vp, vp,
+                                        sz, vp]),
+            "qe_status": (i, [vp, C.POINTER(C.c_int)]),
+            "qe_step_index": (i, [vp]),
+            "qe_length": (i, [vp]),
+            "qe_list_counts": (i, [vp, C.POINTER(C.c_int), C.POINTER(C.c_int)]),
+            "qe_strerror": (C.c_char_p, [i]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name, None)
+            if fn is None:
+                continue
+            fn.restype, fn.argtypes = res, args
+        _lib = L
+    return _lib
+
+
+def strerror(code: int) -> str:
+    return lib().qe_strerror(code).decode()
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise RuntimeError(f"{what} failed: {strerror(rc)} ({rc})")
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return C.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: torch.Tensor):
+    return C.c_void_p(t.data_ptr())
+
+
+def dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return QE_BF16
+    if dt == torch.float16:
+        return QE_FP16
+    raise ValueError(f"unsupported cache dtype {dt}")
+
+
+def _need(t: torch.Tensor, name: str, dtype=None, shape=None):
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+@dataclass
+class ContextShape:
+    B: int
+    Hq: int
+    Hkv: int
+    D: int
+    window: int
+    full_windows: int
+    int2_windows: int
+    route_every: int
+    hidden: int
+    max_ctx: int
+    alpha: float = 0.5
+    pages_per_unit: int = 0  # 0: ceil(max_ctx / 16) + 2 * window / 16
+    slots_per_unit: int = 0  # 0: full_windows + int2_windows
+    max_splits: int = 32
+
+
+class QEvictContext:
+    """One decode context (one attention layer) bound to a torch-allocated workspace."""
+
+    def __init__(self, shape: ContextShape, W_O: torch.Tensor):
+        self.shape = shape
+        self.dtype = W_O.dtype
+        _need(W_O, "W_O", shape=(shape.Hq * shape.D, shape.hidden))
+        ppu = shape.pages_per_unit or (-(-shape.max_ctx // 16) + 2 * shape.window // 16)
+        spu = shape.slots_per_unit or (shape.full_windows + shape.int2_windows)
+        self.cfg = QeConfig(shape.B, shape.Hq, shape.Hkv, shape.D, dtype_code(W_O.dtype), 16,
+                            shape.window, shape.full_windows, shape.int2_windows, shape.alpha,
+                            shape.route_every, shape.hidden, shape.max_ctx, ppu, spu, shape.max_splits)
+        self.layout = QeLayout()
+        _check(lib().qe_plan(C.byref(self.cfg), C.byref(self.layout)), "qe_plan")
+        self.W_O = W_O
+        self.workspace = torch.empty(self.layout.total, dtype=torch.uint8, device=W_O.device)
+        h = C.c_void_p()
+        _check(lib().qe_create(C.byref(self.cfg), _ptr(self.workspace), self.layout.total, _ptr(W_O),
+                               C.byref(h)), "qe_create")
+        self._h = h
+        self.G = shape.Hq // shape.Hkv
+        self.units = shape.B * shape.Hkv
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and _lib is not None:
+            _lib.qe_destroy(h)
+            self._h = None
+
+    # -- the hot path -------------------------------------------------------------
+    def load_prefill(self, K: torch.Tensor, V: torch.Tensor, stream=None):
+        s = self.shape
+        _need(K, "K", self.dtype)
+        _need(V, "V", self.dtype, K.shape)
+        if K.dim() != 4 or K.shape[:2] != (s.B, s.Hkv) or K.shape[3] != s.D:
+            raise ValueError("K, V must be [B][Hkv][ctx][D]")
+        _check(lib().qe_load_prefill(self._h, _ptr(K), _ptr(V), K.shape[2], _stream(stream)),
+               "qe_load_prefill")
+
+    def kv_append(self, k: torch.Tensor, v: torch.Tensor, stream=None):
+        s = self.shape
+        _need(k, "k_new", self.dtype, (s.B, s.Hkv, s.D))
+        _need(v, "v_new", self.dtype, (s.B, s.Hkv, s.D))
+        _check(lib().qe_kv_append(self._h, _ptr(k), _ptr(v), _stream(stream)), "qe_kv_append")
+
+    def decode_attend_and_score(self, q: torch.Tensor, out: torch.Tensor = None, stream=None):
+        s = self.shape
+        _need(q, "q", self.dtype, (s.B, s.Hq, s.D))
+        if out is None:
+            out = torch.empty((s.B, s.Hq, s.D), dtype=torch.float32, device=q.device)
+        _need(out, "out", torch.float32, (s.B, s.Hq, s.D))
+        _check(lib().qe_decode_attend_and_score(self._h, _ptr(q), _ptr(out), _stream(stream)),
+               "qe_decode_attend_and_score")
+        return out
+
+    def route_windows(self, stream=None):
+        _check(lib().qe_route_windows(self._h, _stream(stream)), "qe_route_windows")
+
+    def decode_step(self, q, k, v, out=None, stream=None):
+        s = self.shape
+        _need(q, "q", self.dtype, (s.B, s.Hq, s.D))
+        _need(k, "k_new", self.dtype, (s.B, s.Hkv, s.D))
+        _need(v, "v_new", self.dtype, (s.B, s.Hkv, s.D))
+        if out is None:
+            out = torch.empty((s.B, s.Hq, s.D), dtype=torch.float32, device=q.device)
+        _need(out, "out", torch.float32, (s.B, s.Hq, s.D))
+        _check(lib().qe_decode_step(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _stream(stream)),
+               "qe_decode_step")
+        return out
+
+    def quantize_once(self, unit: int, win_ids, stream=None):
+        ids = (C.c_int32 * len(win_ids))(*[int(x) for x in win_ids])
+        _check(lib().qe_quantize_once(self._h, unit, ids, len(win_ids), _stream(stream)),
+               "qe_quantize_once")
+
+    def promote(self, unit: int, win_ids, stream=None):
+        ids = (C.c_int32 * len(win_ids))(*[int(x) for x in win_ids])
+        _check(lib().qe_promote(self._h, unit, ids, len(win_ids), _stream(stream)), "qe_promote")
+
+    # -- status and state -----------------------------------------------------------
+    def status(self):
+        d = C.c_int()
+        rc = lib().qe_status(self._h, C.byref(d))
+        return rc, d.value
+
+    @property
+    def step_index(self) -> int:
+        return lib().qe_step_index(self._h)
+
+    @property
+    def length(self) -> int:
+        return lib().qe_length(self._h)
+
+    def _view(self, off: int, count: int, dtype, shape):
+        nbytes = count * torch.tensor([], dtype=dtype).element_size()
+        return self.workspace[off:off + nbytes].view(dtype).view(*shape)
+
+    def state(self) -> dict:
+        """Views (no copies) of the context's state arrays inside the workspace."""
+        L, s, U, W = self.layout, self.shape, self.units, self.layout.max_windows
+        ppu, spu = self.cfg.pages_per_unit, self.cfg.slots_per_unit
+        pitch = -(-s.max_ctx // 16) * 16
+        return {
+            "pages": self._view(L.pages, U * ppu * 2 * 16 * s.D, self.dtype, (U, ppu, 2, 16, s.D)),
+            "win_pages": self._view(L.win_pages, U * W * (s.window // 16), torch.int32,
+                                    (U, W, s.window // 16)),
+            "win_tier": self._view(L.win_tier, U * W, torch.uint8, (U, W)),
+            "win_slot": self._view(L.win_slot, U * W, torch.int32, (U, W)),
+            "slots": self._view(L.slots, U * spu * s.window * s.D, torch.uint8, (U, spu, s.window * s.D)),
+            "mass": self._view(L.mass, U * W, torch.float32, (U, W)),
+            "pert": self._view(L.pert, U * W, torch.float32, (U, W)),
+            "norms": self._view(L.norms, U * pitch * self.G, torch.float32, (U, pitch, self.G)),
+            "full_list": self._view(L.full_list, U * W, torch.int32, (U, W)),
+            "int2_list": self._view(L.int2_list, U * W, torch.int32, (U, W)),
+            "tail_p": self._view(L.tail_p, U * s.window * self.G, torch.float32, (U, s.window, self.G)),
+            "stacks": self._view(L.stacks, U * 4, torch.int32, (U, 4)),
+            "route_stats": self._view(L.route_stats, U * 8, torch.int32, (U, 8)),
+        }
+
+    def ledger_entry(self, unit: int, win: int):
+        """Decode one window's INT2 ledger entry into (codes_K, s_K, z_K, codes_V, s_V, z_V).
+
+        Layout of an entry (window w, head dim D): codes K [w][D/4] bytes | codes V | meta K
+        [w][D/16] u32 (fp16 scale low, fp16 zero high) | meta V.
+        """
+        st = self.state()
+        slot = int(st["win_slot"][unit, win])
+        if slot < 0:
+            return None
+        w, D = self.shape.window, self.shape.D
+        raw = st["slots"][unit, slot].cpu().numpy()
+        import numpy as np
+        def codes(b):
+            b = b.reshape(w, D // 4)
+            return np.stack([(b >> (2 * e)) & 3 for e in range(4)], -1).reshape(w, D)
+        def meta(b):
+            m = b.view(np.uint32).reshape(w, D // 16)
+            return ((m & 0xFFFF).astype(np.uint16).view(np.float16),
+                    (m >> 16).astype(np.uint16).view(np.float16))
+        n = w * D // 4
+        ck, cv = codes(raw[:n]), codes(raw[n:2 * n])
+        sk, zk = meta(raw[2 * n:3 * n])
+        sv, zv = meta(raw[3 * n:4 * n])
+        return ck, sk, zk, cv, sv, zv
+
+
+# ---------------------------------------------------------------------------------
+# standalone kernels
+# ---------------------------------------------------------------------------------
+
+
+def int2_quantize(x: torch.Tensor, stream=None):
+    """INT2 group quantiser: x [T][D] -> (codes uint8 [T][D/4], meta int32 [T][D/16])."""
+    _need(x, "x")
+    T, D = x.shape
+    codes = torch.empty((T, D // 4), dtype=torch.uint8, device=x.device)
+    meta = torch.empty((T, D // 16), dtype=torch.int32, device=x.device)
+    _check(lib().qe_int2_quantize(_ptr(x), T, D, dtype_code(x.dtype), _ptr(codes), _ptr(meta),
+                                  _stream(stream)), "qe_int2_quantize")
+    return codes, meta
+
+
+def vwo_l1norm(V: torch.Tensor, W_O: torch.Tensor, Hq: int, Hkv: int, out=None, stream=None):
+    """N[g][r][j] = ||V[g][r] @ W_O^{(g % Hkv)*G + j}||_1 for V [n_groups][rows][D]."""
+    _need(V, "V")
+    _need(W_O, "W_O", V.dtype)
+    n_groups, rows, D = V.shape
+    G = Hq // Hkv
+    if out is None:
+        out = torch.empty((n_groups, rows, G), dtype=torch.float32, device=V.device)
+    _need(out, "out", torch.float32)
+    _check(lib().qe_vwo_l1norm(_ptr(V), n_groups, rows, D, dtype_code(V.dtype), _ptr(W_O), Hq, Hkv,
+                               W_O.shape[1], _ptr(out), rows * G, _stream(stream)), "qe_vwo_l1norm")
+    return out

@@ -1,0 +1,70 @@
+// INT2 group quantiser and dequantiser used by the ledger ("Resumo Técnico: QEvict",
+// Metodologia: recoverable INT2 tier; Hierarquia Recuperável: write-once ledger).
+//
+// One row of D elements is held by a warp, DPL = D/32 consecutive elements per lane, so a
+// 16-element group spans LPG = 16/DPL consecutive lanes. Per group, in float32 with
+// round-to-nearest-even:
+//   s = fp16((max - min) / 3), z = fp16(min), code = clamp(rint((x - z) / s), 0, 3), 0 if s == 0.
+// Row layout in a ledger entry: codes [D/4] bytes (element 4j+e in bits 2e..2e+1 of byte j),
+// meta [D/16] u32 = fp16 s (low half) | fp16 z (high half).
+#pragma once
+#include "qe_internal.cuh"
+
+template <int DPL>
+struct Int2Row {
+  static constexpr int LPG = 16 / DPL;  // lanes per 16-element group
+
+  // Quantise the lane's DPL values. Returns the lane's codes packed at bits 2e, and the
+  // group's (s, z) as a u32 in *meta (valid in every lane).
+  static __device__ __forceinline__ uint32_t quantize(const float (&x)[DPL], uint32_t* meta) {
+    float mn = x[0], mx = x[0];
+#pragma unroll
+    for (int e = 1; e < DPL; ++e) {
+      mn = fminf(mn, x[e]);
+      mx = fmaxf(mx, x[e]);
+    }
+#pragma unroll
+    for (int o = 1; o < LPG; o <<= 1) {
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    const __half sh = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), 3.0f));
+    const __half zh = __float2half_rn(mn);
+    const float s = __half2float(sh), z = __half2float(zh);
+    uint32_t bits = 0;
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) {
+      float c = 0.f;
+      if (s != 0.f) c = fminf(fmaxf(rintf(__fdiv_rn(__fsub_rn(x[e], z), s)), 0.f), 3.f);
+      bits |= static_cast<uint32_t>(c) << (2 * e);
+    }
+    *meta = static_cast<uint32_t>(__half_as_ushort(sh)) |
+            (static_cast<uint32_t>(__half_as_ushort(zh)) << 16);
+    return bits;
+  }
+
+  // Write the lane's codes (from quantize) into a row of D/4 bytes. All lanes must call.
+  static __device__ __forceinline__ void store_codes(uint8_t* row, uint32_t bits, int lane) {
+    if (DPL == 4) {
+      row[lane] = static_cast<uint8_t>(bits);
+    } else {  // DPL == 2: two lanes share a byte
+      const uint32_t other = __shfl_down_sync(0xffffffffu, bits, 1);
+      if ((lane & 1) == 0) row[lane >> 1] = static_cast<uint8_t>(bits | (other << 4));
+    }
+  }
+
+  // The lane's DPL codes from a row of D/4 bytes, packed at bits 2e.
+  static __device__ __forceinline__ uint32_t load_codes(const uint8_t* row, int lane) {
+    if (DPL == 4) return row[lane];
+    return (row[lane >> 1] >> (4 * (lane & 1))) & 0xFu;
+  }
+
+  static __device__ __forceinline__ int group_of(int lane) { return lane / LPG; }
+};
+
+__device__ __forceinline__ float meta_scale(uint32_t m) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(m & 0xffffu)));
+}
+__device__ __forceinline__ float meta_zero(uint32_t m) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(m >> 16)));
+}

@@ -1,0 +1,185 @@
+// Internal declarations shared by the CUDA translation units of libqevict.
+// Device helpers (bulk copies, mbarriers, bounded waits, dtype conversion) and the
+// host-side context. Nothing here is part of the C ABI (see include/qevict.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "../../include/qevict.h"
+
+#define QE_PAGE 16
+#define QE_MAX_G 8
+#define QE_MAX_SPLITS 64
+
+// status word slots
+#define QE_ST_CODE 0
+#define QE_ST_DETAIL 1
+
+// ----------------------------------------------------------------------------
+// host context
+// ----------------------------------------------------------------------------
+struct qe_ctx {
+  qe_config cfg;
+  qe_layout lay;
+  int G;
+  uint8_t* ws;          // workspace base [dev]
+  const void* W_O;      // [Hq*D][hidden] [dev]
+  // host mirror of the length / step (identical for every unit)
+  int n;                // tokens per unit
+  int step;             // decode steps since prefill
+  int complete;         // windows complete and in the tier lists (the tail is window `complete`)
+  int loaded;           // prefill done
+  int n_full_max;       // upper bound of full-tier windows over units
+  int n_int2_max;       // upper bound of INT2-tier windows over units
+  cudaStream_t last_stream;
+  // scratch sub-buffers [dev]
+  float* split_part;    // [U][max_splits][G][2 + D]
+  float* win_part;      // [U][max_windows][G][4]
+  float* tail_s;        // [U][window][G]
+  uint32_t* tickets;    // [U]
+  int32_t* xlist;       // [U][max_windows] transition lists (quantise) [win]
+  int32_t* plist;       // [U][max_windows] transition lists (promote)  [win]
+  int32_t* xcount;      // [U][4] counts: quantise, promote
+  int32_t* host_ids;    // [max_windows] staging for host-given window ids
+  uint8_t* tailV;       // [Hkv][B][window][D] dtype: V of the tail window (for its norms)
+  float* tail_norm;     // [Hkv][B*window][G] norms of a just-completed window
+  // typed views of the state arrays
+  template <typename T> T* at(size_t off) const { return reinterpret_cast<T*>(ws + off); }
+};
+
+// ----------------------------------------------------------------------------
+// device state view passed by value to kernels
+// ----------------------------------------------------------------------------
+struct DevState {
+  uint8_t* pages;       // [U][P][2][16][D] T
+  int32_t* page_free;   // [U][P]
+  int32_t* win_pages;   // [U][Wmax][ppw]
+  uint8_t* win_tier;    // [U][Wmax]
+  int32_t* win_slot;    // [U][Wmax]
+  uint8_t* slots;       // [U][S][window*D]
+  int32_t* slot_free;   // [U][S]
+  float* mass;          // [U][Wmax]
+  float* pert;          // [U][Wmax]
+  float* norms;         // [U][max_ctx][G]
+  int32_t* full_list;   // [U][Wmax]
+  int32_t* int2_list;   // [U][Wmax]
+  float* tail_p;        // [U][window][G]
+  int32_t* stacks;      // [U][4] page top, slot top, n_full, n_int2
+  int32_t* route_stats; // [U][8]
+  int32_t* status;      // [4]
+  int P, S, Wmax, ppw, window, D, G, max_ctx, norm_pitch, U, B, Hkv, Hq;
+  size_t page_bytes, slot_bytes;
+};
+
+DevState make_state(const qe_ctx* c);
+
+// ----------------------------------------------------------------------------
+// device helpers
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void qe_record_error(int32_t* status, int code, int detail) {
+  if (atomicCAS(&status[QE_ST_CODE], 0, code) == 0) status[QE_ST_DETAIL] = detail;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+// 1-D bulk copy global -> shared, completion signalled on an mbarrier (no multicast).
+// src, dst 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait on an mbarrier phase: gives up after ~2^31 clock cycles (about a
+// second), records QE_ERR_TIMEOUT and returns false.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int32_t* status,
+                                                  int where) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > (1ll << 31)) {
+      qe_record_error(status, QE_ERR_TIMEOUT, where);
+      return false;
+    }
+  }
+  return true;
+}
+
+// dtype traits: 16-bit element -> float
+template <typename T> struct Elem;
+template <> struct Elem<__nv_bfloat16> {
+  static __device__ __forceinline__ float lo(uint32_t w) { return __uint_as_float(w << 16); }
+  static __device__ __forceinline__ float hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+  static __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+  static __device__ __forceinline__ __nv_bfloat16 from_f(float x) { return __float2bfloat16_rn(x); }
+};
+template <> struct Elem<__half> {
+  static __device__ __forceinline__ float lo(uint32_t w) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xffffu)));
+  }
+  static __device__ __forceinline__ float hi(uint32_t w) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16)));
+  }
+  static __device__ __forceinline__ float to_f(__half x) { return __half2float(x); }
+  static __device__ __forceinline__ __half from_f(float x) { return __float2half_rn(x); }
+};
+
+// ----------------------------------------------------------------------------
+// host helpers
+// ----------------------------------------------------------------------------
+#define QE_CUDA_TRY(expr)                         \
+  do {                                            \
+    cudaError_t _e = (expr);                      \
+    if (_e != cudaSuccess) return QE_ERR_CUDA;    \
+  } while (0)
+
+static inline bool qe_aligned(const void* p, size_t a) {
+  return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+// launchers (defined in the .cu files)
+int launch_prefill(qe_ctx* c, const void* K, const void* V, int ctx_len, cudaStream_t st);
+int launch_append(qe_ctx* c, const void* k, const void* v, cudaStream_t st);
+int launch_decode(qe_ctx* c, const void* q, float* out, cudaStream_t st);
+int launch_finalize(qe_ctx* c, int tail_win, cudaStream_t st);
+int launch_route(qe_ctx* c, cudaStream_t st);
+int launch_set_tier(qe_ctx* c, int unit, const int32_t* ids_host, int n, int tier, cudaStream_t st);
+int launch_vwo(const void* V, int n_groups, int rows, int D, int dtype, const void* W_O, int Hq,
+               int Hkv, int hidden, float* out, long long out_group_stride, cudaStream_t st);
+int launch_int2_quantize(const void* x, int T, int D, int dtype, uint8_t* codes, uint32_t* meta,
+                         cudaStream_t st);

@@ -1,0 +1,661 @@
+// Cache-state kernels: prefill load, token append, tail-window finalisation, two-stage
+// routing with its tier transitions, and the write-once quantise / promote pass.
+//
+// "Resumo Técnico: QEvict" - Metodologia (three tiers: full precision, recoverable INT2,
+// evicted, under a fixed budget) and Mecanismos Principais (window-level routing,
+// cumulative scores, Rebaixamento / Promoção, write-once quantisation ledger).
+// "Resumo Técnico: CriticalKV" - Algoritmo (two-stage selection: b' = alpha*b by
+// attention mass, b - b' by the perturbation score).
+//
+// Every unit (batch, kv-head) owns a private slice of the page pool and of the ledger,
+// with its own free stacks; one CTA per unit does that unit's bookkeeping, so no
+// cross-unit atomics are needed and allocation is deterministic.
+#include <math.h>
+
+#include "int2.cuh"
+#include "qe_internal.cuh"
+
+namespace {
+
+constexpr int kRouteThreads = 512;
+
+// ---------------------------------------------------------------------------
+// block helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int t = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += t;
+  }
+  return v;
+}
+
+// Exclusive scan of one int per thread over the block; returns the block total in *total.
+// `buf` needs 33 ints of shared memory.
+__device__ int block_excl_scan(int v, int* buf, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int inc = warp_incl_scan(v, lane);
+  if (lane == 31) buf[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int x = lane < nw ? buf[lane] : 0;
+    int xi = warp_incl_scan(x, lane);
+    if (lane < nw) buf[lane] = xi - x;
+    if (lane == 31) buf[32] = xi;
+  }
+  __syncthreads();
+  const int r = buf[warp] + inc - v;
+  *total = buf[32];
+  __syncthreads();
+  return r;
+}
+
+__device__ float block_sum(float v, float* buf) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (lane == 0) buf[warp] = v;
+  __syncthreads();
+  float r = 0.f;
+  if (threadIdx.x == 0)
+    for (int i = 0; i < nw; ++i) r += buf[i];
+  __syncthreads();
+  return r;  // valid in thread 0
+}
+
+// float -> uint32 whose unsigned order is the float order
+__device__ __forceinline__ uint32_t ordered_bits(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// ---------------------------------------------------------------------------
+// prefill
+// ---------------------------------------------------------------------------
+// K, V: [U][ctx][D]. Page p of unit u receives tokens 16p..16p+15 (zero past ctx).
+__global__ void prefill_pages_kernel(DevState st, const uint4* K, const uint4* V, int ctx) {
+  const int p = blockIdx.x, u = blockIdx.y;
+  const int vec_per_row = st.D * 2 / 16;  // 16-byte vectors per row
+  uint4* page = reinterpret_cast<uint4*>(st.pages + ((size_t)u * st.P + p) * st.page_bytes);
+  for (int i = threadIdx.x; i < 2 * QE_PAGE * vec_per_row; i += blockDim.x) {
+    const int kv = i / (QE_PAGE * vec_per_row), rem = i % (QE_PAGE * vec_per_row);
+    const int r = rem / vec_per_row, c = rem % vec_per_row;
+    const int tok = p * QE_PAGE + r;
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (tok < ctx) val = (kv ? V : K)[((size_t)u * ctx + tok) * vec_per_row + c];
+    page[i] = val;
+  }
+}
+
+__global__ void prefill_meta_kernel(DevState st, const uint4* V, int ctx, uint4* tailV) {
+  const int u = blockIdx.x, b = u / st.Hkv, kvh = u % st.Hkv;
+  const int w = st.window, complete = ctx / w, n_pages = (ctx + QE_PAGE - 1) / QE_PAGE;
+  const int n_win = (ctx + w - 1) / w;
+  for (int i = threadIdx.x; i < n_win; i += blockDim.x) {
+    st.win_tier[(size_t)u * st.Wmax + i] = i < complete ? QE_TIER_FULL : QE_TIER_TAIL;
+    for (int k = 0; k < st.ppw; ++k) {
+      const int pg = i * st.ppw + k;
+      st.win_pages[((size_t)u * st.Wmax + i) * st.ppw + k] = pg < n_pages ? pg : -1;
+    }
+    if (i < complete) st.full_list[(size_t)u * st.Wmax + i] = i;
+  }
+  for (int i = threadIdx.x; i < st.P - n_pages; i += blockDim.x)
+    st.page_free[(size_t)u * st.P + i] = st.P - 1 - i;
+  for (int i = threadIdx.x; i < st.S; i += blockDim.x) st.slot_free[(size_t)u * st.S + i] = st.S - 1 - i;
+  if (threadIdx.x == 0) {
+    st.stacks[u * 4 + 0] = st.P - n_pages;
+    st.stacks[u * 4 + 1] = st.S;
+    st.stacks[u * 4 + 2] = complete;
+    st.stacks[u * 4 + 3] = 0;
+  }
+  // V of an incomplete last window, staged for its norms when it completes
+  const int vec_per_row = st.D * 2 / 16, tail = ctx - complete * w;
+  for (int i = threadIdx.x; i < tail * vec_per_row; i += blockDim.x) {
+    const int t = i / vec_per_row, c = i % vec_per_row;
+    tailV[(((size_t)kvh * st.B + b) * w + t) * vec_per_row + c] =
+        V[((size_t)u * ctx + complete * w + t) * vec_per_row + c];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// append one token per unit at position pos
+// ---------------------------------------------------------------------------
+__global__ void append_kernel(DevState st, const uint4* k_new, const uint4* v_new, int pos,
+                              uint4* tailV) {
+  const int u = blockIdx.x, b = u / st.Hkv, kvh = u % st.Hkv;
+  const int w = st.window, tw = pos / w, t = pos % w, pg = t / QE_PAGE, r = pos % QE_PAGE;
+  __shared__ int s_page;
+  if (threadIdx.x == 0) {
+    const size_t wi = (size_t)u * st.Wmax + tw;
+    int page = -1;
+    if (t == 0) {
+      st.win_tier[wi] = QE_TIER_TAIL;
+      st.win_slot[wi] = -1;
+      st.mass[wi] = 0.f;
+      st.pert[wi] = 0.f;
+    }
+    if (r == 0) {
+      const int top = st.stacks[u * 4 + 0];
+      if (top <= 0) {
+        qe_record_error(st.status, QE_ERR_POOL_EXHAUSTED, u);
+      } else {
+        page = st.page_free[(size_t)u * st.P + top - 1];
+        st.stacks[u * 4 + 0] = top - 1;
+        st.win_pages[wi * st.ppw + pg] = page;
+      }
+    } else {
+      page = st.win_pages[wi * st.ppw + pg];
+    }
+    if (page >= st.P) {
+      qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
+      page = -1;
+    }
+    s_page = page;
+  }
+  __syncthreads();
+  if (t == 0)
+    for (int i = threadIdx.x; i < w * st.G; i += blockDim.x) st.tail_p[(size_t)u * w * st.G + i] = 0.f;
+  const int page = s_page;
+  if (page < 0) return;
+  const int vpr = st.D * 2 / 16;
+  uint4* base = reinterpret_cast<uint4*>(st.pages + ((size_t)u * st.P + page) * st.page_bytes);
+  for (int c = threadIdx.x; c < vpr; c += blockDim.x) {
+    const uint4 kv = k_new[(size_t)u * vpr + c], vv = v_new[(size_t)u * vpr + c];
+    base[r * vpr + c] = kv;
+    base[(QE_PAGE + r) * vpr + c] = vv;
+    tailV[(((size_t)kvh * st.B + b) * w + t) * vpr + c] = vv;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// the tail window completed: store its norms, fold the deferred perturbation score,
+// and move it into the full tier as a routing candidate
+// ---------------------------------------------------------------------------
+__global__ void finalize_kernel(DevState st, const float* tail_norm, int tw) {
+  const int u = blockIdx.x, b = u / st.Hkv, kvh = u % st.Hkv, w = st.window, G = st.G;
+  __shared__ float red[32];
+  float acc = 0.f;
+  for (int i = threadIdx.x; i < w * G; i += blockDim.x) {
+    const int t = i / G, h = i % G;
+    const float nrm = tail_norm[(((size_t)kvh * st.B + b) * w + t) * G + h];
+    st.norms[((size_t)u * st.norm_pitch + (size_t)tw * w + t) * G + h] = nrm;
+    float* tp = st.tail_p + (size_t)u * w * G + i;
+    acc += *tp * nrm;
+    *tp = 0.f;
+  }
+  const float sum = block_sum(acc, red);
+  if (threadIdx.x == 0) {
+    const size_t wi = (size_t)u * st.Wmax + tw;
+    st.pert[wi] += sum;
+    st.win_tier[wi] = QE_TIER_FULL;
+    const int nf = st.stacks[u * 4 + 2];
+    if (nf >= st.Wmax) {
+      qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
+    } else {
+      st.full_list[(size_t)u * st.Wmax + nf] = tw;
+      st.stacks[u * 4 + 2] = nf + 1;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// routing
+// ---------------------------------------------------------------------------
+struct RouteArgs {
+  DevState st;
+  int32_t* xlist;   // [U][Wmax] windows to quantise
+  int32_t* plist;   // [U][Wmax] windows to promote
+  int32_t* xcount;  // [U][4]
+  int F, Q, F1, Q1; // budgets and their stage-1 shares floor(alpha*b)
+  int mode;         // 0: two-stage routing; 1: explicit targets for one unit
+  int unit;         // mode 1
+  const int32_t* ids;  // mode 1: window ids
+  int n_ids;           // mode 1
+  int target;          // mode 1: QE_TIER_INT2 or QE_TIER_FULL
+};
+
+// Two-stage selection among candidates with inset[i]; selected ones get sel[i] = 1.
+// Ranks use 64-bit keys (ordered score, ~window) so ties go to the lower window index.
+__device__ void two_stage_select(int n, const int32_t* cand, const float* k1, const float* k2,
+                                 const uint8_t* inset, uint8_t* sel, uint8_t* s1mark, int b, int b1,
+                                 int* ibuf) {
+  int cnt_local = 0;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) cnt_local += inset[i];
+  int cnt;
+  block_excl_scan(cnt_local, ibuf, &cnt);
+  if (cnt <= b) {
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      sel[i] = inset[i];
+      s1mark[i] = inset[i];
+    }
+    __syncthreads();
+    return;
+  }
+  // stage 1: rank by k1 among inset
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    uint8_t s = 0;
+    if (inset[i]) {
+      const unsigned long long ki =
+          ((unsigned long long)ordered_bits(k1[i]) << 32) | (0xffffffffu - (uint32_t)cand[i]);
+      int rank = 0;
+      for (int j = 0; j < n; ++j) {
+        const unsigned long long kj =
+            ((unsigned long long)ordered_bits(k1[j]) << 32) | (0xffffffffu - (uint32_t)cand[j]);
+        rank += (inset[j] && kj > ki);
+      }
+      s = rank < b1;
+    }
+    s1mark[i] = s;
+  }
+  __syncthreads();
+  // stage 2: rank by k2 among inset minus stage 1
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    uint8_t s = s1mark[i];
+    if (inset[i] && !s1mark[i]) {
+      const unsigned long long ki =
+          ((unsigned long long)ordered_bits(k2[i]) << 32) | (0xffffffffu - (uint32_t)cand[i]);
+      int rank = 0;
+      for (int j = 0; j < n; ++j) {
+        const unsigned long long kj =
+            ((unsigned long long)ordered_bits(k2[j]) << 32) | (0xffffffffu - (uint32_t)cand[j]);
+        rank += (inset[j] && !s1mark[j] && kj > ki);
+      }
+      s = rank < b - b1;
+    }
+    sel[i] = s;
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
+  const DevState& st = a.st;
+  const int u = a.mode == 1 ? a.unit : blockIdx.x;
+  extern __shared__ __align__(16) uint8_t sm[];
+  const int nf = st.stacks[u * 4 + 2], nq = st.stacks[u * 4 + 3], n = nf + nq;
+  int32_t* cand = reinterpret_cast<int32_t*>(sm);
+  float* km = reinterpret_cast<float*>(cand + st.Wmax);
+  float* kp = km + st.Wmax;
+  uint8_t* oldt = reinterpret_cast<uint8_t*>(kp + st.Wmax);
+  uint8_t* newt = oldt + st.Wmax;
+  uint8_t* inset = newt + st.Wmax;
+  uint8_t* sel = inset + st.Wmax;
+  uint8_t* s1 = sel + st.Wmax;
+  __shared__ int ibuf[33];
+  __shared__ float fbuf[32];
+  __shared__ int s_abort;
+  if (threadIdx.x == 0) s_abort = 0;
+  if (n > st.Wmax) {
+    if (threadIdx.x == 0) qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
+    return;
+  }
+  const size_t ub = (size_t)u * st.Wmax;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int win = i < nf ? st.full_list[ub + i] : st.int2_list[ub + i - nf];
+    cand[i] = win;
+    km[i] = st.mass[ub + win];
+    kp[i] = st.pert[ub + win];
+    oldt[i] = i < nf ? QE_TIER_FULL : QE_TIER_INT2;
+    newt[i] = QE_TIER_EVICTED;
+  }
+  __syncthreads();
+
+  float stage1_mass = 0.f, all_mass = 0.f;
+  if (a.mode == 0) {
+    for (int i = threadIdx.x; i < n; i += blockDim.x) inset[i] = 1;
+    __syncthreads();
+    two_stage_select(n, cand, km, kp, inset, sel, s1, a.F, a.F1, ibuf);
+    float s1m = 0.f, am = 0.f;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      if (sel[i]) newt[i] = QE_TIER_FULL;
+      if (s1[i]) s1m += km[i];
+      am += km[i];
+      inset[i] = !sel[i];
+    }
+    stage1_mass = block_sum(s1m, fbuf);
+    all_mass = block_sum(am, fbuf);
+    two_stage_select(n, cand, km, kp, inset, sel, s1, a.Q, a.Q1, ibuf);
+    for (int i = threadIdx.x; i < n; i += blockDim.x)
+      if (sel[i]) newt[i] = QE_TIER_INT2;
+  } else {
+    for (int i = threadIdx.x; i < n; i += blockDim.x) newt[i] = oldt[i];
+    __syncthreads();
+    for (int k = threadIdx.x; k < a.n_ids; k += blockDim.x) {
+      const int id = a.ids[k];
+      int found = -1;
+      for (int i = 0; i < n; ++i)
+        if (cand[i] == id) found = i;
+      const int want_old = a.target == QE_TIER_INT2 ? QE_TIER_FULL : QE_TIER_INT2;
+      if (found < 0 || oldt[found] != want_old)
+        qe_record_error(st.status, QE_ERR_INVALID_ARG, id);
+      else
+        newt[found] = (uint8_t)a.target;
+    }
+  }
+  __syncthreads();
+
+  // ---- transitions: counts, then allocation (pops), then frees (pushes) ----
+  // each thread owns a contiguous run of candidates so prefix sums stay in candidate order
+  const int per = (n + blockDim.x - 1) / blockDim.x;
+  const int i0 = threadIdx.x * per, i1 = min(n, i0 + per);
+  int c_tp = 0, c_ts = 0, c_gp = 0, c_gs = 0, c_pr = 0, c_nf = 0, c_nq = 0;
+  for (int i = i0; i < i1; ++i) {
+    const int o = oldt[i], t = newt[i];
+    const int slot = st.win_slot[ub + cand[i]];
+    c_tp += (o == QE_TIER_INT2 && t == QE_TIER_FULL) ? st.ppw : 0;
+    c_ts += (o == QE_TIER_FULL && t == QE_TIER_INT2 && slot < 0);
+    c_gp += (o == QE_TIER_FULL && t != QE_TIER_FULL) ? st.ppw : 0;
+    c_gs += (t == QE_TIER_EVICTED && slot >= 0);
+    c_pr += (o == QE_TIER_INT2 && t == QE_TIER_FULL);
+    c_nf += (t == QE_TIER_FULL);
+    c_nq += (t == QE_TIER_INT2);
+  }
+  int T_tp, T_ts, T_gp, T_gs, T_pr, T_nf, T_nq;
+  int o_tp = block_excl_scan(c_tp, ibuf, &T_tp);
+  int o_ts = block_excl_scan(c_ts, ibuf, &T_ts);
+  int o_gp = block_excl_scan(c_gp, ibuf, &T_gp);
+  int o_gs = block_excl_scan(c_gs, ibuf, &T_gs);
+  int o_pr = block_excl_scan(c_pr, ibuf, &T_pr);
+  int o_nf = block_excl_scan(c_nf, ibuf, &T_nf);
+  int o_nq = block_excl_scan(c_nq, ibuf, &T_nq);
+  const int ptop = st.stacks[u * 4 + 0], stop = st.stacks[u * 4 + 1];
+  if (threadIdx.x == 0) {
+    if (T_tp > ptop) {
+      qe_record_error(st.status, QE_ERR_POOL_EXHAUSTED, u);
+      s_abort = 1;
+    } else if (T_ts > stop) {
+      qe_record_error(st.status, QE_ERR_LEDGER_FULL, u);
+      s_abort = 1;
+    }
+  }
+  __syncthreads();
+  if (s_abort) return;  // nothing was modified yet
+
+  // pops
+  {
+    int tp = o_tp, ts = o_ts, pr = o_pr;
+    for (int i = i0; i < i1; ++i) {
+      const int o = oldt[i], t = newt[i], win = cand[i];
+      if (o == QE_TIER_INT2 && t == QE_TIER_FULL) {
+        for (int k = 0; k < st.ppw; ++k) {
+          const int page = st.page_free[(size_t)u * st.P + ptop - 1 - (tp + k)];
+          st.win_pages[(ub + win) * st.ppw + k] = page;
+        }
+        tp += st.ppw;
+        a.plist[ub + pr++] = win;
+      }
+      if (o == QE_TIER_FULL && t == QE_TIER_INT2 && st.win_slot[ub + win] < 0) {
+        const int slot = st.slot_free[(size_t)u * st.S + stop - 1 - ts];
+        st.win_slot[ub + win] = slot;
+        a.xlist[ub + ts] = win;
+        ++ts;
+      }
+    }
+  }
+  __syncthreads();
+  // pushes (freed pages and slots) on top of the shrunken stacks
+  {
+    const int ntop = ptop - T_tp, nstop = stop - T_ts;
+    int gp = o_gp, gs = o_gs, f = o_nf, q = o_nq;
+    for (int i = i0; i < i1; ++i) {
+      const int o = oldt[i], t = newt[i], win = cand[i];
+      if (o == QE_TIER_FULL && t != QE_TIER_FULL) {
+        for (int k = 0; k < st.ppw; ++k)
+          st.page_free[(size_t)u * st.P + ntop + gp + k] = st.win_pages[(ub + win) * st.ppw + k];
+        gp += st.ppw;
+      }
+      if (t == QE_TIER_EVICTED) {
+        const int slot = st.win_slot[ub + win];
+        if (slot >= 0) {
+          st.slot_free[(size_t)u * st.S + nstop + gs++] = slot;
+          st.win_slot[ub + win] = -1;
+        }
+      }
+      if (t == QE_TIER_FULL) st.full_list[ub + f++] = win;
+      if (t == QE_TIER_INT2) st.int2_list[ub + q++] = win;
+      st.win_tier[ub + win] = (uint8_t)t;
+    }
+  }
+  if (threadIdx.x == 0) {
+    st.stacks[u * 4 + 0] = ptop - T_tp + T_gp;
+    st.stacks[u * 4 + 1] = stop - T_ts + T_gs;
+    st.stacks[u * 4 + 2] = T_nf;
+    st.stacks[u * 4 + 3] = T_nq;
+    a.xcount[u * 4 + 0] = T_ts;
+    a.xcount[u * 4 + 1] = T_pr;
+    int32_t* rs = st.route_stats + u * 8;
+    rs[0] = T_pr;
+    rs[1] = T_ts;
+    rs[2] = 0;  // filled below (demotions that reused a ledger entry)
+    rs[4] = T_nf;
+    rs[5] = T_nq;
+    rs[7] = all_mass > 0.f ? (int)llrintf(1e6f * stage1_mass / all_mass) : 0;
+  }
+  // demotions that reused an entry, evictions
+  int c_re = 0, c_ev = 0;
+  for (int i = i0; i < i1; ++i) {
+    c_re += (oldt[i] == QE_TIER_FULL && newt[i] == QE_TIER_INT2);
+    c_ev += (newt[i] == QE_TIER_EVICTED);
+  }
+  int T_re, T_ev;
+  block_excl_scan(c_re, ibuf, &T_re);
+  block_excl_scan(c_ev, ibuf, &T_ev);
+  if (threadIdx.x == 0) {
+    st.route_stats[u * 8 + 2] = T_re - T_ts;
+    st.route_stats[u * 8 + 3] = T_ev;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// quantise (first demotion only) and promote, one warp per window
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void apply_kernel(DevState st, const int32_t* xlist, const int32_t* plist,
+                             const int32_t* xcount, int unit_only) {
+  constexpr int DPL = D / 32;
+  using R = Int2Row<DPL>;
+  const int u = unit_only >= 0 ? unit_only : blockIdx.x;
+  const int lane = threadIdx.x & 31;
+  const int warps = blockDim.x >> 5, gw = blockIdx.y * warps + (threadIdx.x >> 5);
+  const int nx = xcount[u * 4 + 0], np = xcount[u * 4 + 1];
+  const size_t ub = (size_t)u * st.Wmax;
+  const int w = st.window;
+  for (int item = gw; item < nx + np; item += gridDim.y * warps) {
+    const bool quant = item < nx;
+    const int win = quant ? xlist[ub + item] : plist[ub + item - nx];
+    const int slot = st.win_slot[ub + win];
+    if (win < 0 || win >= st.Wmax || slot < 0 || slot >= st.S) {
+      if (lane == 0) qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
+      continue;
+    }
+    uint8_t* sl = st.slots + ((size_t)u * st.S + slot) * st.slot_bytes;
+    uint8_t* kc = sl;
+    uint8_t* vc = sl + (size_t)w * D / 4;
+    uint32_t* km = reinterpret_cast<uint32_t*>(sl + (size_t)w * D / 2);
+    uint32_t* vm = km + (size_t)w * D / 16;
+    for (int t = 0; t < w; ++t) {
+      const int page = st.win_pages[(ub + win) * st.ppw + t / QE_PAGE];
+      if (page < 0 || page >= st.P) {
+        if (lane == 0) qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
+        break;
+      }
+      T* prow = reinterpret_cast<T*>(st.pages + ((size_t)u * st.P + page) * st.page_bytes);
+      T* krow = prow + (size_t)(t % QE_PAGE) * D;
+      T* vrow = prow + (size_t)(QE_PAGE + t % QE_PAGE) * D;
+      if (quant) {
+        float xk[DPL], xv[DPL];
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) {
+          xk[e] = Elem<T>::to_f(krow[lane * DPL + e]);
+          xv[e] = Elem<T>::to_f(vrow[lane * DPL + e]);
+        }
+        uint32_t mk, mv;
+        const uint32_t bk = R::quantize(xk, &mk);
+        const uint32_t bv = R::quantize(xv, &mv);
+        R::store_codes(kc + (size_t)t * D / 4, bk, lane);
+        R::store_codes(vc + (size_t)t * D / 4, bv, lane);
+        if (lane % R::LPG == 0) {
+          km[(size_t)t * D / 16 + R::group_of(lane)] = mk;
+          vm[(size_t)t * D / 16 + R::group_of(lane)] = mv;
+        }
+      } else {
+        const uint32_t bk = R::load_codes(kc + (size_t)t * D / 4, lane);
+        const uint32_t bv = R::load_codes(vc + (size_t)t * D / 4, lane);
+        const uint32_t mk = km[(size_t)t * D / 16 + R::group_of(lane)];
+        const uint32_t mv = vm[(size_t)t * D / 16 + R::group_of(lane)];
+        const float sk = meta_scale(mk), zk = meta_zero(mk), sv = meta_scale(mv), zv = meta_zero(mv);
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) {
+          krow[lane * DPL + e] = Elem<T>::from_f(fmaf((float)((bk >> (2 * e)) & 3u), sk, zk));
+          vrow[lane * DPL + e] = Elem<T>::from_f(fmaf((float)((bv >> (2 * e)) & 3u), sv, zv));
+        }
+      }
+    }
+  }
+}
+
+// standalone quantiser: one warp per row
+template <typename T, int D>
+__global__ void int2_quantize_kernel(const T* x, int rows, uint8_t* codes, uint32_t* meta) {
+  constexpr int DPL = D / 32;
+  using R = Int2Row<DPL>;
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  float xv[DPL];
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) xv[e] = Elem<T>::to_f(x[(size_t)row * D + lane * DPL + e]);
+  uint32_t m;
+  const uint32_t bits = R::quantize(xv, &m);
+  R::store_codes(codes + (size_t)row * D / 4, bits, lane);
+  if (lane % R::LPG == 0) meta[(size_t)row * D / 16 + R::group_of(lane)] = m;
+}
+
+template <typename T, int D>
+void launch_apply(const DevState& st, const qe_ctx* c, int unit_only, cudaStream_t s) {
+  const int units = unit_only >= 0 ? 1 : st.U;
+  // enough warps to give every window of the largest possible transition list its own warp
+  int per_unit = (st.Wmax + 7) / 8;
+  if (per_unit > 64) per_unit = 64;
+  apply_kernel<T, D><<<dim3(units, per_unit), 256, 0, s>>>(st, c->xlist, c->plist, c->xcount,
+                                                            unit_only);
+}
+
+int apply_dispatch(const qe_ctx* c, const DevState& st, int unit_only, cudaStream_t s) {
+  const bool bf = c->cfg.dtype == QE_BF16;
+  if (c->cfg.D == 128) {
+    if (bf) launch_apply<__nv_bfloat16, 128>(st, c, unit_only, s);
+    else launch_apply<__half, 128>(st, c, unit_only, s);
+  } else {
+    if (bf) launch_apply<__nv_bfloat16, 64>(st, c, unit_only, s);
+    else launch_apply<__half, 64>(st, c, unit_only, s);
+  }
+  return cudaGetLastError() == cudaSuccess ? QE_OK : QE_ERR_CUDA;
+}
+
+size_t route_smem(const DevState& st) { return (size_t)st.Wmax * (4 + 4 + 4 + 5) + 64; }
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// launchers
+// ---------------------------------------------------------------------------
+int launch_prefill(qe_ctx* c, const void* K, const void* V, int ctx, cudaStream_t s) {
+  DevState st = make_state(c);
+  const qe_layout& L = c->lay;
+  const size_t U = L.units, W = L.max_windows;
+  QE_CUDA_TRY(cudaMemsetAsync(st.win_tier, 0, U * W, s));
+  QE_CUDA_TRY(cudaMemsetAsync(st.win_slot, 0xff, U * W * 4, s));
+  QE_CUDA_TRY(cudaMemsetAsync(st.win_pages, 0xff, U * W * st.ppw * 4, s));
+  QE_CUDA_TRY(cudaMemsetAsync(st.mass, 0, U * W * 4, s));
+  QE_CUDA_TRY(cudaMemsetAsync(st.pert, 0, U * W * 4, s));
+  QE_CUDA_TRY(cudaMemsetAsync(st.tail_p, 0, U * st.window * st.G * 4, s));
+  QE_CUDA_TRY(cudaMemsetAsync(st.route_stats, 0, U * 8 * 4, s));
+  QE_CUDA_TRY(cudaMemsetAsync(st.status, 0, 16, s));
+  QE_CUDA_TRY(cudaMemsetAsync(c->tickets, 0, U * 4, s));
+  QE_CUDA_TRY(cudaMemsetAsync(c->xcount, 0, U * 16, s));
+  const int n_pages = (ctx + QE_PAGE - 1) / QE_PAGE;
+  prefill_pages_kernel<<<dim3(n_pages, (unsigned)U), 256, 0, s>>>(st, (const uint4*)K, (const uint4*)V,
+                                                                  ctx);
+  prefill_meta_kernel<<<(unsigned)U, 256, 0, s>>>(st, (const uint4*)V, ctx, (uint4*)c->tailV);
+  QE_CUDA_TRY(cudaGetLastError());
+  return launch_vwo(V, (int)U, ctx, c->cfg.D, c->cfg.dtype, c->W_O, c->cfg.Hq, c->cfg.Hkv,
+                    c->cfg.hidden, st.norms, (long long)st.norm_pitch * c->G, s);
+}
+
+int launch_append(qe_ctx* c, const void* k, const void* v, cudaStream_t s) {
+  DevState st = make_state(c);
+  append_kernel<<<st.U, 64, 0, s>>>(st, (const uint4*)k, (const uint4*)v, c->n, (uint4*)c->tailV);
+  return cudaGetLastError() == cudaSuccess ? QE_OK : QE_ERR_CUDA;
+}
+
+int launch_finalize(qe_ctx* c, int tw, cudaStream_t s) {
+  DevState st = make_state(c);
+  const int rows = c->cfg.B * c->cfg.window;
+  int e = launch_vwo(c->tailV, c->cfg.Hkv, rows, c->cfg.D, c->cfg.dtype, c->W_O, c->cfg.Hq,
+                     c->cfg.Hkv, c->cfg.hidden, c->tail_norm, (long long)rows * c->G, s);
+  if (e) return e;
+  finalize_kernel<<<st.U, 128, 0, s>>>(st, c->tail_norm, tw);
+  return cudaGetLastError() == cudaSuccess ? QE_OK : QE_ERR_CUDA;
+}
+
+int launch_route(qe_ctx* c, cudaStream_t s) {
+  DevState st = make_state(c);
+  RouteArgs a{};
+  a.st = st;
+  a.xlist = c->xlist;
+  a.plist = c->plist;
+  a.xcount = c->xcount;
+  a.F = c->cfg.full_windows;
+  a.Q = c->cfg.int2_windows;
+  a.F1 = (int)floor((double)c->cfg.alpha * a.F);
+  a.Q1 = (int)floor((double)c->cfg.alpha * a.Q);
+  a.mode = 0;
+  a.unit = -1;
+  const size_t smem = route_smem(st);
+  if (smem > 200 * 1024) return QE_ERR_UNSUPPORTED_SHAPE;
+  QE_CUDA_TRY(cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  route_kernel<<<st.U, kRouteThreads, smem, s>>>(a);
+  QE_CUDA_TRY(cudaGetLastError());
+  return apply_dispatch(c, st, -1, s);
+}
+
+int launch_set_tier(qe_ctx* c, int unit, const int32_t* ids, int n, int tier, cudaStream_t s) {
+  DevState st = make_state(c);
+  QE_CUDA_TRY(cudaMemcpyAsync(c->host_ids, ids, (size_t)n * 4, cudaMemcpyHostToDevice, s));
+  RouteArgs a{};
+  a.st = st;
+  a.xlist = c->xlist;
+  a.plist = c->plist;
+  a.xcount = c->xcount;
+  a.mode = 1;
+  a.unit = unit;
+  a.ids = c->host_ids;
+  a.n_ids = n;
+  a.target = tier;
+  const size_t smem = route_smem(st);
+  if (smem > 200 * 1024) return QE_ERR_UNSUPPORTED_SHAPE;
+  QE_CUDA_TRY(cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  route_kernel<<<1, kRouteThreads, smem, s>>>(a);
+  QE_CUDA_TRY(cudaGetLastError());
+  return apply_dispatch(c, st, unit, s);
+}
+
+int launch_int2_quantize(const void* x, int T, int D, int dtype, uint8_t* codes, uint32_t* meta,
+                         cudaStream_t s) {
+  const int blocks = (T + 7) / 8;
+  if (D == 128) {
+    if (dtype == QE_BF16)
+      int2_quantize_kernel<__nv_bfloat16, 128><<<blocks, 256, 0, s>>>((const __nv_bfloat16*)x, T, codes, meta);
+    else
+      int2_quantize_kernel<__half, 128><<<blocks, 256, 0, s>>>((const __half*)x, T, codes, meta);
+  } else if (D == 64) {
+    if (dtype == QE_BF16)
+      int2_quantize_kernel<__nv_bfloat16, 64><<<blocks, 256, 0, s>>>((const __nv_bfloat16*)x, T, codes, meta);
+    else
+      int2_quantize_kernel<__half, 64><<<blocks, 256, 0, s>>>((const __half*)x, T, codes, meta);
+  } else {
+    return QE_ERR_UNSUPPORTED_SHAPE;
+  }
+  return cudaGetLastError() == cudaSuccess ? QE_OK : QE_ERR_CUDA;
+}

@@ -1,0 +1,215 @@
+"""Lock-step comparison of the CUDA decode path with the CPU oracle.
+
+Both sides take the same seeded inputs (kv_cache_eviction_gqa_b200.workloads). After
+every decode step the checked units are compared:
+
+* attention output: max |o_gpu - o_ref| / max |o_ref| per (batch, query head) <= 2e-3;
+* cumulative window mass and perturbation: |d| / max(|ref|, 1e-30) <= 1e-4 per window
+  (the tail window's perturbation is folded in when it completes, so it is compared then);
+* routing: tier decisions must match, except items whose score lies within 1e-4 relative
+  of a selection boundary (near-ties: counted and reported). When every mismatch is a
+  near-tie the oracle adopts the GPU's tiers for those windows so histories stay aligned;
+  the GPU's decision is also checked to be exactly the two-stage selection of its own
+  scores (a property of the selection, independent of the oracle);
+* INT2 ledger codes and fp16 scale/zero of every newly demoted window: bit-exact;
+* promoted pages: bit-exact dequant(ledger) in the cache dtype.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+import torch
+
+import oracle as O
+from kv_cache_eviction_gqa_b200 import workloads as W
+from kv_cache_eviction_gqa_b200.binding import (TIER_EVICTED, TIER_FULL, TIER_INT2, TIER_TAIL,
+                                                ContextShape, QEvictContext)
+
+OUT_TOL = 2e-3
+SCORE_TOL = 1e-4
+TIE_TOL = 1e-4
+
+
+def torch_dtype(name):
+    return torch.bfloat16 if name == "bf16" else torch.float16
+
+
+@dataclass
+class ParityReport:
+    steps: int = 0
+    max_out_err: float = 0.0
+    max_mass_err: float = 0.0
+    max_pert_err: float = 0.0
+    route_events: int = 0
+    route_mismatch: int = 0
+    near_ties: int = 0
+    codes_checked: int = 0
+    promoted_checked: int = 0
+    notes: list = field(default_factory=list)
+
+
+def _select_two_stage(ids, k1, k2, b, b1):
+    """Independent restatement for the property check (lexsort on score desc, id asc)."""
+    ids = np.asarray(ids)
+    if ids.size <= b:
+        return set(ids.tolist())
+    o1 = np.lexsort((ids, -k1[ids]))
+    s1 = ids[o1[:b1]]
+    rest = np.setdiff1d(ids, s1)
+    o2 = np.lexsort((rest, -k2[rest]))
+    return set(s1.tolist()) | set(rest[o2[:b - b1]].tolist())
+
+
+def _near_tie(unit: O.QEvictUnit, w: int) -> bool:
+    """Is window w within TIE_TOL of any of the four selection boundaries of the last route?"""
+    r = unit.last_route
+    L = r["L"]
+    mass, pert = unit.mass, unit.pert
+    full = np.concatenate(r["full"])
+    rest = np.setdiff1d(L, full)
+    checks = [(L, mass, int(math.floor(unit.alpha * unit.F))),
+              (np.setdiff1d(L, r["full"][0]), pert, unit.F - int(math.floor(unit.alpha * unit.F))),
+              (rest, mass, int(math.floor(unit.alpha * unit.Q))),
+              (np.setdiff1d(rest, r["int2"][0]), pert, unit.Q - int(math.floor(unit.alpha * unit.Q)))]
+    for ids, key, k in checks:
+        if ids.size == 0 or k <= 0 or k >= ids.size:
+            continue
+        srt = np.sort(key[ids])[::-1]
+        for bnd in (srt[k - 1], srt[k]):
+            if abs(key[w] - bnd) <= TIE_TOL * max(abs(bnd), 1e-30):
+                return True
+    return False
+
+
+def run_decode_parity(cfg: W.DecodeConfig, check_units=None, steps=None, max_splits=32,
+                      check_every=1, verbose=False) -> ParityReport:
+    dev = "cuda"
+    tdt = torch_dtype(cfg.dtype)
+    steps = cfg.steps if steps is None else steps
+    all_units = [(b, h) for b in range(cfg.B) for h in range(cfg.Hkv)]
+    if check_units is None:
+        check_units = list(range(len(all_units)))
+    inp = W.draw_decode_inputs(cfg)
+    K = torch.from_numpy(inp.K).view(cfg.B, cfg.Hkv, cfg.ctx, cfg.D).to(dev, tdt)
+    V = torch.from_numpy(inp.V).view(cfg.B, cfg.Hkv, cfg.ctx, cfg.D).to(dev, tdt)
+    W_O = torch.from_numpy(inp.W_O).to(dev, tdt)
+    max_ctx = cfg.ctx + steps
+    shape = ContextShape(cfg.B, cfg.Hq, cfg.Hkv, cfg.D, cfg.window, cfg.full_windows,
+                         cfg.int2_windows, cfg.route_every, cfg.hidden, max_ctx, cfg.alpha,
+                         max_splits=max_splits)
+    ctx = QEvictContext(shape, W_O)
+    ctx.load_prefill(K, V)
+    G = cfg.G
+    units = {}
+    for u in check_units:
+        b, h = all_units[u]
+        units[u] = O.QEvictUnit(inp.K[u], inp.V[u], inp.W_O, h, G, cfg.window, cfg.full_windows,
+                                cfg.int2_windows, cfg.alpha, cfg.dtype, max_ctx)
+    rep = ParityReport()
+    st = ctx.state()
+    b1F = int(math.floor(cfg.alpha * cfg.full_windows))
+    b1Q = int(math.floor(cfg.alpha * cfg.int2_windows))
+    for s in range(steps):
+        q = torch.from_numpy(inp.q[s]).to(dev, tdt)
+        k = torch.from_numpy(inp.k_new[s]).to(dev, tdt)
+        v = torch.from_numpy(inp.v_new[s]).to(dev, tdt)
+        # scores before routing, for the selection-property check
+        ctx.kv_append(k, v)
+        out = ctx.decode_attend_and_score(q)
+        torch.cuda.synchronize()
+        routing = s % cfg.route_every == 0
+        g_mass = st["mass"].cpu().numpy().copy()
+        g_pert = st["pert"].cpu().numpy().copy()
+        g_tier_before = st["win_tier"].cpu().numpy().copy()
+        if routing:
+            ctx.route_windows()
+        torch.cuda.synchronize()
+        rc, det = ctx.status()
+        assert rc == 0, f"device status {rc} detail {det} at step {s}"
+        o_gpu = out.cpu().numpy()
+        g_tier = st["win_tier"].cpu().numpy()
+        for u, unit in units.items():
+            b, h = all_units[u]
+            unit.append(inp.k_new[s, b, h].astype(np.float64), inp.v_new[s, b, h].astype(np.float64))
+            o_ref, _ = unit.attend_and_score(inp.q[s, b, h * G:(h + 1) * G].astype(np.float64))
+            for j in range(G):
+                og = o_gpu[b, h * G + j]
+                err = np.abs(og - o_ref[j]).max() / np.abs(o_ref[j]).max()
+                rep.max_out_err = max(rep.max_out_err, err)
+                assert err <= OUT_TOL, f"step {s} unit {u} head {j}: output rel err {err:.3e}"
+            if s % check_every == 0 or routing:
+                live = np.nonzero(unit.tier != O.EVICTED)[0]
+                tail = unit.n // cfg.window if unit.n % cfg.window else -1
+                rm = np.abs(g_mass[u, live] - unit.mass[live]) / np.maximum(np.abs(unit.mass[live]), 1e-30)
+                rep.max_mass_err = max(rep.max_mass_err, rm.max())
+                assert rm.max() <= SCORE_TOL, f"step {s} unit {u}: mass rel err {rm.max():.3e} " \
+                    f"at window {live[rm.argmax()]}"
+                lp = live[live != tail]
+                rp = np.abs(g_pert[u, lp] - unit.pert[lp]) / np.maximum(np.abs(unit.pert[lp]), 1e-30)
+                if rp.size:
+                    rep.max_pert_err = max(rep.max_pert_err, rp.max())
+                    assert rp.max() <= SCORE_TOL, f"step {s} unit {u}: pert rel err {rp.max():.3e} " \
+                        f"at window {lp[rp.argmax()]}"
+            if routing:
+                rep.route_events += 1
+                cands = np.nonzero((g_tier_before[u] == TIER_FULL) | (g_tier_before[u] == TIER_INT2))[0]
+                # property: the GPU decision is the two-stage selection of its own scores
+                full_g = _select_two_stage(cands, g_mass[u].astype(np.float64),
+                                           g_pert[u].astype(np.float64), cfg.full_windows, b1F)
+                rest = np.array(sorted(set(cands.tolist()) - full_g), dtype=np.int64)
+                int2_g = _select_two_stage(rest, g_mass[u].astype(np.float64),
+                                           g_pert[u].astype(np.float64), cfg.int2_windows, b1Q)
+                got_full = set(np.nonzero(g_tier[u] == TIER_FULL)[0].tolist())
+                got_int2 = set(np.nonzero(g_tier[u] == TIER_INT2)[0].tolist())
+                assert got_full == full_g, f"step {s} unit {u}: full tier is not the two-stage pick"
+                assert got_int2 == int2_g, f"step {s} unit {u}: INT2 tier is not the two-stage pick"
+                ledger_before = set(unit.ledger.keys())
+                new = unit.route()
+                mism = [w for w, t in new.items() if int(g_tier[u, w]) != t]
+                if mism:
+                    ties = [w for w in mism if _near_tie(unit, w)]
+                    rep.route_mismatch += len(mism)
+                    rep.near_ties += len(ties)
+                    assert len(ties) == len(mism), (
+                        f"step {s} unit {u}: routing mismatch on windows "
+                        f"{sorted(set(mism) - set(ties))} not near a selection boundary")
+                    # replay: adopt the GPU's tiers for the near-tie windows
+                    unit.apply({w: int(g_tier[u, w]) for w in mism})
+                # INT2 codes of windows quantised at this event: bit-exact
+                for w in sorted(set(unit.ledger.keys()) - ledger_before):
+                    e = ctx.ledger_entry(u, w)
+                    assert e is not None, f"unit {u} window {w}: no ledger slot on the GPU"
+                    (ck, sk, zk), (cv, sv, zv) = unit.ledger[w]
+                    gk, gsk, gzk, gv, gsv, gzv = e
+                    for a_, b_, nm in ((gk, ck, "K codes"), (gv, cv, "V codes")):
+                        np.testing.assert_array_equal(a_, b_, err_msg=f"unit {u} win {w} {nm}")
+                    for a_, b_, nm in ((gsk, sk, "K scale"), (gzk, zk, "K zero"), (gsv, sv, "V scale"),
+                                       (gzv, zv, "V zero")):
+                        np.testing.assert_array_equal(a_.view(np.uint16), b_.view(np.uint16),
+                                                      err_msg=f"unit {u} win {w} {nm}")
+                    rep.codes_checked += 1
+                # promoted windows: their pages hold dequant(ledger) in the cache dtype
+                promoted = [w for w, t in new.items() if t == O.FULL and g_tier_before[u, w] == TIER_INT2]
+                if promoted:
+                    pages = st["pages"][u].float().cpu().numpy()
+                    wp = st["win_pages"][u].cpu().numpy()
+                    for w in promoted:
+                        for t in range(cfg.window):
+                            pg = wp[w, t // 16]
+                            np.testing.assert_array_equal(pages[pg, 0, t % 16], unit.Kst[w * cfg.window + t])
+                            np.testing.assert_array_equal(pages[pg, 1, t % 16], unit.Vst[w * cfg.window + t])
+                        rep.promoted_checked += 1
+                # tiers agree after replay
+                live_o = {int(w): int(unit.tier[w]) for w in np.nonzero(unit.tier != O.EVICTED)[0]}
+                for w, t in live_o.items():
+                    gt = int(g_tier[u, w])
+                    assert gt == t or (t in (O.TAIL, O.FULL) and gt in (TIER_TAIL, TIER_FULL)), \
+                        f"unit {u} window {w}: tier {gt} vs oracle {t}"
+        ctx._steps_done = s + 1
+        rep.steps += 1
+        if verbose and (s % 8 == 0):
+            print(f"step {s}: out {rep.max_out_err:.2e} mass {rep.max_mass_err:.2e} "
+                  f"pert {rep.max_pert_err:.2e} ties {rep.near_ties}")
+    return rep
