@@ -1,0 +1,472 @@
+#!/usr/bin/env python
+"""Benchmark of the tiered-KV decode step (attention + scoring + routing) on B200.
+
+Workload: one attention layer shaped like Llama-3-8B (32 query / 8 KV heads, head dim
+128), batch 8, 32K-token prefill, windows of 32 tokens, 2048 full-precision + 4096 INT2
+tokens per head, 64 decode steps with scoring every step and routing every 16 steps
+(bf16, seeded synthetic data: K/V N(0,1) with 4 outlier channels x8).
+
+A bench step is one decode step of that sequence: kv_append, decode attention with the
+fused window scoring, and (on steps s % 16 == 0) two-stage routing with its INT2
+quantise / promote pass. Timed steps start at decode step 0 of a fresh prefill and cycle
+through the 64-step sequence (the prefill state is restored, untimed, between
+sequences). Each step runs from its CUDA graph, timed with CUDA events on its stream;
+L2 is flushed (512 MiB write) before every step, outside the timed region.
+
+--impl reference times the CPU oracle (float64 NumPy) on a bounded sample of the same
+workload and prints the same JSON line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import copy
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from kv_cache_eviction_gqa_b200 import workloads as W  # noqa: E402
+
+METRIC = "decode attn+routing steps/sec; achieved HBM GB/s vs peak at 32K ctx, batch 8"
+CFG = W.C2
+FALLBACK_HBM_GBS = 6650.0
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs", FALLBACK_HBM_GBS), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def workload_config(cfg):
+    return {
+        "workload": f"{cfg.name}: 1 layer, B={cfg.B}, Hq={cfg.Hq}, Hkv={cfg.Hkv}, D={cfg.D}, "
+                    f"prefill {cfg.ctx}, window {cfg.window}, {cfg.full_windows * cfg.window} full + "
+                    f"{cfg.int2_windows * cfg.window} INT2 tokens per head, {cfg.steps} decode steps, "
+                    f"route every {cfg.route_every}",
+        "global_batch": cfg.B, "seq_len": cfg.ctx, "window": cfg.window,
+        "budget_full_tokens": cfg.full_windows * cfg.window,
+        "budget_int2_tokens": cfg.int2_windows * cfg.window,
+        "route_every": cfg.route_every, "decode_steps_per_sequence": cfg.steps,
+        "accumulate": "f32", "l2": "flushed before every step (512 MiB write), outside the timed region",
+        "parallelism": "replicas (one independent context per GPU, no collective)",
+    }
+
+
+def decode_bytes(cfg, nf, nq, tail_len):
+    """Algorithmic HBM bytes of one decode launch (every unit).
+
+    Per unit: full tokens read K+V (2*D*2 B) and their norms (G*4 B); INT2 tokens read
+    2-bit K+V codes (D/2 B), fp16 scale/zero per 16-element group (D/2 B) and norms; tail
+    tokens read K+V; q read, o written (fp32); mass and pert read and written per live window.
+    """
+    D, G, w = cfg.D, cfg.G, cfg.window
+    per_unit = (nf * w * (4 * D + 4 * G) + nq * w * (D + 4 * G) + tail_len * 4 * D
+                + G * D * 2 + G * D * 4 + (nf + nq + 1) * 16)
+    return per_unit * cfg.units
+
+
+# ---------------------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) >= 9:
+                    rows.append(p)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------------------
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:  # noqa: BLE001
+        return 1
+
+
+def oracle_units(cfg, units):
+    import oracle as O
+    Wo = W.draw_w_o(cfg)
+    q, k, v = W.draw_step_inputs(cfg)
+    out = []
+    for (b, h) in units:
+        K, V = W.draw_unit_cache(cfg, b, h)
+        u = O.QEvictUnit(K, V, Wo, h, cfg.G, cfg.window, cfg.full_windows, cfg.int2_windows,
+                         cfg.alpha, cfg.dtype, cfg.ctx + cfg.steps)
+        out.append(((b, h), u))
+    return out, (q, k, v)
+
+
+def oracle_step(cfg, unit, s, b, h, q, k, v):
+    G = cfg.G
+    unit.step(s, q[s, b, h * G:(h + 1) * G].astype(np.float64), k[s, b, h].astype(np.float64),
+              v[s, b, h].astype(np.float64), cfg.route_every)
+
+
+def cpu_baseline(cfg, target_s=10.0):
+    """Time the oracle's decode steps on 2 sampled units, repeating the 64-step sequence
+    from the post-prefill state until about target_s seconds of CPU work; scale to the
+    whole batch (every unit)."""
+    units, (q, k, v) = oracle_units(cfg, [(0, 0), (cfg.B - 1, cfg.Hkv - 1)])
+    done, t = 0, 0.0
+    reps = 0
+    while t < target_s:
+        for (b, h), u0 in units:
+            u = copy.deepcopy(u0)
+            t0 = time.perf_counter()
+            for s in range(cfg.steps):
+                oracle_step(cfg, u, s, b, h, q, k, v)
+            t += time.perf_counter() - t0
+            done += cfg.steps
+        reps += 1
+    unit_steps_per_s = done / t
+    return {"value": unit_steps_per_s / cfg.units, "unit": "steps/s", "kind": "oracle",
+            "cores": len(os.sched_getaffinity(0)), "blas_threads": blas_threads(),
+            "sample": f"float64 NumPy oracle, {len(units)} of {cfg.units} (batch, kv-head) units x "
+                      f"{cfg.steps} decode steps x {reps} repeats ({t:.1f} s of decode work; prefill "
+                      f"norms untimed); steps/s scaled to all {cfg.units} units"}
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    cfg = CFG
+    units, (q, k, v) = oracle_units(cfg, [(0, 0)])
+    (b, h), u0 = units[0]
+    u = copy.deepcopy(u0)
+    for i in range(args.warmup):
+        s = i % cfg.steps
+        if s == 0 and i:
+            u = copy.deepcopy(u0)
+        oracle_step(cfg, u, s, b, h, q, k, v)
+    u = copy.deepcopy(u0)
+    t = 0.0
+    for i in range(args.steps):
+        s = i % cfg.steps
+        if s == 0 and i:
+            u = copy.deepcopy(u0)
+        t0 = time.perf_counter()
+        oracle_step(cfg, u, s, b, h, q, k, v)
+        t += time.perf_counter() - t0
+    per_step_full = t / args.steps * cfg.units  # one decode step of the whole batch
+    value = 1.0 / per_step_full
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": per_step_full * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": workload_config(cfg),
+            "cpu_baseline": {"value": value, "unit": "steps/s", "kind": "oracle",
+                             "cores": len(os.sched_getaffinity(0)), "blas_threads": blas_threads(),
+                             "sample": f"each step: 1 of {cfg.units} units (b=0, kv-head 0) of the "
+                                       f"decode step, scaled to the whole batch"},
+            "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------------------
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from kv_cache_eviction_gqa_b200.binding import ContextShape, QEvictContext, vwo_l1norm
+
+    cfg = CFG
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    tdt = torch.bfloat16
+    peak, peak_kind = measured_peaks()
+
+    # cpu baseline first (rank 0, single GPU only), before any GPU work
+    cpu = cpu_baseline(cfg) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
+
+    inp = W.draw_decode_inputs(cfg)
+    K = torch.from_numpy(inp.K).view(cfg.B, cfg.Hkv, cfg.ctx, cfg.D).to(dev, tdt)
+    V = torch.from_numpy(inp.V).view(cfg.B, cfg.Hkv, cfg.ctx, cfg.D).to(dev, tdt)
+    W_O = torch.from_numpy(inp.W_O).to(dev, tdt)
+    qs = torch.from_numpy(inp.q).to(dev, tdt)
+    ks = torch.from_numpy(inp.k_new).to(dev, tdt)
+    vs = torch.from_numpy(inp.v_new).to(dev, tdt)
+    del inp
+    S, R = cfg.steps, cfg.route_every
+    shape = ContextShape(cfg.B, cfg.Hq, cfg.Hkv, cfg.D, cfg.window, cfg.full_windows, cfg.int2_windows,
+                         R, cfg.hidden, cfg.ctx + S, cfg.alpha, max_splits=args.max_splits)
+    ctx = QEvictContext(shape, W_O)
+    norms = vwo_l1norm(V.view(cfg.units, cfg.ctx, cfg.D), W_O, cfg.Hq, cfg.Hkv)
+    norms = norms.view(cfg.B, cfg.Hkv, cfg.ctx, cfg.G)
+    out = torch.empty((cfg.B, cfg.Hq, cfg.D), dtype=torch.float32, device=dev)
+
+    # one eager pass through the public API (also validates the device status)
+    ctx.load_prefill(K, V, norms)
+    for s in range(args.profile_steps or S):
+        ctx.decode_step(qs[s], ks[s], vs[s], out)
+    rc, det = ctx.status()
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} ({det}) after the eager pass")
+    if args.profile_steps:
+        # profiling mode: only the eager decode steps above (for ncu -k ... -s ... -c ...)
+        return
+
+    # capture one CUDA graph per step part, and record the per-step list sizes
+    ctx.load_prefill(K, V, norms)
+    torch.cuda.synchronize()
+    snapshot = ctx.workspace.clone()
+    from kv_cache_eviction_gqa_b200.binding import lib
+    import ctypes as C
+    g_app, g_dec, g_route, meta = [], [], [], []
+    cap_stream = torch.cuda.Stream()
+    for s in range(S):
+        nf, nq = C.c_int(), C.c_int()
+        ga, gd, gr = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), None
+        with torch.cuda.graph(ga, stream=cap_stream):
+            ctx.kv_append(ks[s], vs[s])
+        lib().qe_list_counts(ctx._h, C.byref(nf), C.byref(nq))
+        n = ctx.length
+        tail_len = (n - 1) % cfg.window + 1
+        with torch.cuda.graph(gd, stream=cap_stream):
+            ctx.decode_attend_and_score(qs[s], out)
+        finalize = n % cfg.window == 0
+        if s % R == 0:
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=cap_stream):
+                ctx.route_windows()
+        g_app.append(ga)
+        g_dec.append(gd)
+        g_route.append(gr)
+        launches = 2 + (2 if finalize else 0) + (2 if s % R == 0 else 0)
+        meta.append((nf.value, nq.value, tail_len, finalize, launches))
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def restore():
+        ctx.workspace.copy_(snapshot)
+
+    # warm-up
+    restore()
+    for i in range(args.warmup):
+        s = i % S
+        if s == 0 and i:
+            restore()
+        g_app[s].replay()
+        g_dec[s].replay()
+        if g_route[s] is not None:
+            g_route[s].replay()
+    torch.cuda.synchronize()
+    restore()
+
+    K_steps = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K_steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for i in range(K_steps):
+            s = i % S
+            if s == 0 and i:
+                restore()
+            flush.zero_()
+            e = ev[i]
+            e[0].record(stream)
+            g_app[s].replay()
+            e[1].record(stream)
+            g_dec[s].replay()
+            e[2].record(stream)
+            if g_route[s] is not None:
+                g_route[s].replay()
+            e[3].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = clk.summary()
+    step_ms = [ev[i][0].elapsed_time(ev[i][3]) for i in range(K_steps)]
+    dec_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K_steps)]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    value = world * K_steps / (total_ms / 1e3)
+
+    # roofline of the decode kernel (steps without a tail-window completion)
+    b_sum, t_sum, n_l = 0.0, 0.0, 0
+    all_bytes = 0.0
+    for i in range(K_steps):
+        nf, nq, tl, fin, _ = meta[i % S]
+        by = decode_bytes(cfg, nf, nq, tl)
+        all_bytes += by
+        if not fin:
+            b_sum += by
+            t_sum += dec_ms[i] / 1e3
+            n_l += 1
+    achieved = b_sum / t_sum / 1e9
+    steady = [i for i in range(K_steps) if (i % S) % R != 0 and not meta[i % S][3]]
+    st_ms = sum(step_ms[i] for i in steady)
+    st_bytes = sum(decode_bytes(cfg, *meta[i % S][:3]) for i in steady)
+    st_dec_ms = sum(dec_ms[i] for i in steady)
+
+    # end to end through the public API with host buffers (H2D inputs, D2H output)
+    q_h = torch.empty((S, cfg.B, cfg.Hq, cfg.D), dtype=tdt, pin_memory=True)
+    k_h = torch.empty((S, cfg.B, cfg.Hkv, cfg.D), dtype=tdt, pin_memory=True)
+    v_h = torch.empty_like(k_h, pin_memory=True)
+    q_h.copy_(qs.cpu())
+    k_h.copy_(ks.cpu())
+    v_h.copy_(vs.cpu())
+    out_h = torch.empty((cfg.B, cfg.Hq, cfg.D), dtype=torch.float32, pin_memory=True)
+    q_d, k_d, v_d = torch.empty_like(qs[0]), torch.empty_like(ks[0]), torch.empty_like(vs[0])
+    h2d = q_d.numel() * 2 + k_d.numel() * 2 + v_d.numel() * 2
+    d2h = out.numel() * 4
+    e2e_steps = min(K_steps, args.e2e_steps)
+    e2e_ms = 0.0
+    ctx.load_prefill(K, V, norms)
+    a, bvt = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for i in range(e2e_steps):
+        s = i % S
+        if s == 0 and i:
+            ctx.load_prefill(K, V, norms)
+        flush.zero_()
+        torch.cuda.synchronize()  # the host starts each step idle: its launch cost is timed
+        a.record(stream)
+        q_d.copy_(q_h[s], non_blocking=True)
+        k_d.copy_(k_h[s], non_blocking=True)
+        v_d.copy_(v_h[s], non_blocking=True)
+        ctx.decode_step(q_d, k_d, v_d, out)
+        out_h.copy_(out, non_blocking=True)
+        bvt.record(stream)
+        bvt.synchronize()
+        e2e_ms += a.elapsed_time(bvt)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * e2e_steps / (e2e_ms / 1e3)
+    rc, det = ctx.status()
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} ({det}) after the timed run")
+
+    if rank == 0:
+        launches = sum(meta[i % S][4] for i in range(K_steps))
+        line = {
+            "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": K_steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / K_steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(cfg),
+            "tokens_per_s": value * cfg.B,
+            "hbm_gbs_step": all_bytes / (sum(step_ms) / 1e3) / 1e9,
+            "hbm_frac_step": all_bytes / (sum(step_ms) / 1e3) / 1e9 / peak,
+            "steady_state": {"steps_per_s": len(steady) / (st_ms / 1e3) if st_ms else None,
+                             "decode_kernel_gbs": st_bytes / (st_dec_ms / 1e3) / 1e9 if st_dec_ms else None,
+                             "note": "decode steps with no routing and no window completion"},
+            "per_step_first_sequence": [
+                {"s": i, "step_us": round(step_ms[i] * 1e3, 2), "decode_us": round(dec_ms[i] * 1e3, 2),
+                 "decode_gbs": round(decode_bytes(cfg, *meta[i][:3]) / (dec_ms[i] / 1e3) / 1e9, 1)}
+                for i in range(min(K_steps, S)) if i < 3 or i % 16 in (0, 1) or meta[i][3]],
+            "roofline": {"kernel": "decode_kernel (split-K GQA decode + window scoring)",
+                         "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
+                         "traffic": None, "launches_counted": n_l,
+                         "bytes_per_launch_avg": b_sum / max(n_l, 1)},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                    "path": "qe_decode_step through the Python binding, pinned host buffers, "
+                            "host waits for each step's output"},
+            "clocks": clocks,
+            "gpu_launches": launches,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=640)
+    ap.add_argument("--warmup", type=int, default=64)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--max-splits", type=int, default=32)
+    ap.add_argument("--e2e-steps", type=int, default=640)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-steps", type=int, default=0,
+                    help="run only this many eager decode steps after the prefill, then exit")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    run_ours(args, rank, world, local_rank)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

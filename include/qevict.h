@@ -107,11 +107,6 @@ typedef struct {
 
 typedef struct qe_ctx qe_ctx; /* opaque host object; owns no device memory */
 
-/* Per-call statistics of the most recent routing event, summed over units. */
-typedef struct {
-  long long promotions, demotions_new, demotions_reused, evictions;
-} qe_route_totals;
-
 /* qe_plan - fill *out with the workspace size and state-array offsets for *cfg.
  * [host] cfg, out. Returns QE_ERR_UNSUPPORTED_SHAPE / QE_ERR_INVALID_ARG on a bad config. */
 QE_API int qe_plan(const qe_config* cfg, qe_layout* out);
@@ -134,10 +129,12 @@ QE_API int qe_destroy(qe_ctx* ctx);
 
 /* qe_load_prefill - reset the context and load a prefill cache of ctx_len tokens.
  *   K, V [dev]: [B][Hkv][ctx_len][D] cache dtype. Every complete window goes to the
- *   full tier; an incomplete last window becomes the tail. Computes ||V_i W_O^h||_1 for
- *   every prefill token on tensor cores. Scores start at 0. (QEvict, Metodologia.) */
+ *   full tier; an incomplete last window becomes the tail. Scores start at 0.
+ *   norms [dev, may be NULL]: [B][Hkv][ctx_len][G] float ||V_i W_O^h||_1 of the prefill
+ *   tokens (e.g. from qe_vwo_l1norm); NULL computes them here on tensor cores.
+ * (QEvict, Metodologia: the cache before decoding starts.) */
 QE_API int qe_load_prefill(qe_ctx* ctx, const void* K, const void* V, int ctx_len,
-                           qe_stream_t stream);
+                           const float* norms, qe_stream_t stream);
 
 /* qe_kv_append - append one token per unit at position n (the current length).
  *   k_new, v_new [dev]: [B][Hkv][D] cache dtype. Takes a fresh page from the unit's free
@@ -164,8 +161,7 @@ QE_API int qe_decode_attend_and_score(qe_ctx* ctx, const void* q, float* out,
  *   b - floor(alpha*b) highest pert among the rest; ties go to the lower window index.
  * Demotions quantise only windows with no ledger entry yet (write-once); promotions write
  * dequant(ledger) rounded to the cache dtype into fresh pages and keep the entry.
- *   totals [host, may be NULL]: not filled asynchronously; pass NULL and read the
- *   route_stats array of the layout instead. */
+ * Per-unit counts of the event land in the layout's route_stats array. */
 QE_API int qe_route_windows(qe_ctx* ctx, qe_stream_t stream);
 
 /* qe_decode_step - one whole decode step: kv_append, decode_attend_and_score and, on steps

@@ -51,7 +51,7 @@ def lib():
             "qe_workspace_bytes": (sz, [C.POINTER(QeConfig)]),
             "qe_create": (i, [C.POINTER(QeConfig), vp, sz, vp, C.POINTER(vp)]),
             "qe_destroy": (i, [vp]),
-            "qe_load_prefill": (i, [vp, vp, vp, i, vp]),
+            "qe_load_prefill": (i, [vp, vp, vp, i, vp, vp]),
             "qe_kv_append": (i, [vp, vp, vp, vp]),
             "qe_decode_attend_and_score": (i, [vp, vp, vp, vp]),
             "qe_route_windows": (i, [vp, vp]),
@@ -164,13 +164,17 @@ class QEvictContext:
             self._h = None
 
     # -- the hot path -------------------------------------------------------------
-    def load_prefill(self, K: torch.Tensor, V: torch.Tensor, stream=None):
+    def load_prefill(self, K: torch.Tensor, V: torch.Tensor, norms: torch.Tensor = None, stream=None):
+        """Load a prefill cache K, V [B][Hkv][ctx][D]; norms [B][Hkv][ctx][G] float32 or None."""
         s = self.shape
         _need(K, "K", self.dtype)
         _need(V, "V", self.dtype, K.shape)
         if K.dim() != 4 or K.shape[:2] != (s.B, s.Hkv) or K.shape[3] != s.D:
             raise ValueError("K, V must be [B][Hkv][ctx][D]")
-        _check(lib().qe_load_prefill(self._h, _ptr(K), _ptr(V), K.shape[2], _stream(stream)),
+        if norms is not None:
+            _need(norms, "norms", torch.float32, (s.B, s.Hkv, K.shape[2], self.G))
+        _check(lib().qe_load_prefill(self._h, _ptr(K), _ptr(V), K.shape[2],
+                                     _ptr(norms) if norms is not None else None, _stream(stream)),
                "qe_load_prefill")
 
     def kv_append(self, k: torch.Tensor, v: torch.Tensor, stream=None):

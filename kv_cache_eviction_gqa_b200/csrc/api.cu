@@ -136,13 +136,14 @@ QE_API int qe_destroy(qe_ctx* c) {
   return QE_OK;
 }
 
-QE_API int qe_load_prefill(qe_ctx* c, const void* K, const void* V, int ctx_len, qe_stream_t s) {
+QE_API int qe_load_prefill(qe_ctx* c, const void* K, const void* V, int ctx_len, const float* norms,
+                           qe_stream_t s) {
   if (!c || !K || !V) return QE_ERR_INVALID_ARG;
-  if (!qe_aligned(K, 16) || !qe_aligned(V, 16)) return QE_ERR_INVALID_ARG;
+  if (!qe_aligned(K, 16) || !qe_aligned(V, 16) || !qe_aligned(norms, 4)) return QE_ERR_INVALID_ARG;
   if (ctx_len < 1 || ctx_len > c->cfg.max_ctx) return QE_ERR_INVALID_ARG;
   if ((ctx_len + QE_PAGE - 1) / QE_PAGE > c->cfg.pages_per_unit) return QE_ERR_POOL_EXHAUSTED;
   cudaStream_t st = (cudaStream_t)s;
-  int e = launch_prefill(c, K, V, ctx_len, st);
+  int e = launch_prefill(c, K, V, ctx_len, norms, st);
   if (e) return e;
   c->n = ctx_len;
   c->complete = ctx_len / c->cfg.window;

@@ -2,25 +2,41 @@
 // cumulative window scores.
 //
 // "Resumo Técnico: QEvict" - Mecanismos Principais: window-level routing driven by
-// attention accumulated over time (Pontuação Cumulativa); recoverable INT2 tier that
-// attention still reads (Metodologia 2); GQA decode path (Implementação).
+// attention accumulated over time (Pontuação Cumulativa); the recoverable INT2 tier stays
+// readable by attention (Metodologia 2); GQA decode path (Implementação).
 // "Resumo Técnico: CriticalKV" - Etapa 2: the perturbation score A_i * ||V_i W_O||_1.
 //
-// Per unit u = (b, g) the live windows form a list [full windows | INT2 windows | tail].
-// The list is cut into `splits` contiguous, cost-balanced ranges, one CTA each. Inside a
-// CTA every warp takes whole windows round-robin and streams them through its own ring of
-// shared-memory stages with 1-D bulk copies (cp.async.bulk, completion on an mbarrier):
-// one 16-token page (K rows then V rows) per stage for full windows, one ledger entry per
-// stage for INT2 windows, each with the window's norms. Lanes split the head dimension
-// (D/32 elements each); a token's G query-head dot products are reduced across the warp
-// in batches of 8 tokens. Softmax runs online in the log2 domain.
+// Work split. Per unit u = (b, g) the live windows are [full windows | INT2 windows | tail].
+// Split s of S takes the s-th S-th of the full windows and the s-th S-th of the INT2
+// windows (the last split also takes the tail), so every CTA - and every SM - streams the
+// same mix of bandwidth-heavy full pages and arithmetic-heavy INT2 entries. Inside a CTA
+// each warp takes whole windows round-robin and streams them through its own ring of
+// shared-memory stages with 1-D bulk copies (cp.async.bulk, completion on an mbarrier, no
+// multicast): one 16-token page (K rows then V rows) per stage for a full window, the whole
+// ledger entry for an INT2 window, each with the tokens' projected-value norms.
 //
-// Scoring without a second pass: every warp records, per window and head, the partial
-// (m, sum_i 2^(s_i-m), sum_i 2^(s_i-m) n_i) relative to its running max m. The last CTA of
-// the unit to finish (atomic ticket, no spinning) combines the splits into the output and
-// the per-head log-sum-exp, then adds each window's exact attention mass and perturbation
-// to the cumulative scores. The tail window's norms are not known yet, so its per-token
-// attention is accumulated instead (tail_p) and folded in when it completes.
+// Lane mapping. A token is handled by LPT = D / DPL lanes; lane `sub` owns the DPL
+// contiguous head-dim elements [DPL*sub, DPL*sub + DPL), i.e. one INT2 group (DPL = 16) or
+// half of one (DPL = 8), so it needs one scale/zero per token. With DPL = 16 the two 8-element
+// chunks of a lane are loaded in a lane-dependent order (register chunk c holds memory chunk
+// c ^ sw) so that every 16-byte shared-memory load instruction of the warp touches each bank
+// once. A warp works on TPS = 32 / LPT tokens at a time; q and the accumulators of the G
+// query heads stay in registers as float pairs and all multiply-adds are packed (f32x2).
+// A token's G dot products are summed over its lanes with a butterfly, so every lane of the
+// group holds the scores and no weight broadcast is needed. Each lane group keeps its own
+// online-softmax state (log2 domain); the accumulators are rescaled only when the running
+// maximum grows by more than 2^8, and the groups are merged once per warp at the end.
+//
+// INT2 decoding without float conversions: a 2-bit code c is placed in the two top
+// mantissa bits of 1.0, x = 1 + c/4 (two integer ops), and the affine map is folded into
+// the per-token scale: k = c*s + z = 4s*x + (z - 4s).
+//
+// Scoring without a second pass: every warp records per window and head the partial
+// (m, sum_i 2^(s_i-m), sum_i 2^(s_i-m) n_i). The last CTA of the unit to finish (atomic
+// ticket, no spinning) merges the splits into the output and the per-head log-sum-exp and
+// adds each window's exact attention mass and perturbation to the cumulative scores. The
+// tail window's norms are not known yet; its per-token attention is accumulated instead
+// (tail_p) and folded in when the window completes.
 #include <math.h>
 
 #include "int2.cuh"
@@ -28,8 +44,24 @@
 
 namespace {
 
-constexpr int kNW = 4;   // warps per CTA
-constexpr int kNST = 3;  // stages per warp
+#ifndef QE_DECODE_NW
+#define QE_DECODE_NW 4
+#endif
+#ifndef QE_DECODE_NST
+#define QE_DECODE_NST 3
+#endif
+#ifndef QE_DECODE_MINB
+#define QE_DECODE_MINB 2
+#endif
+#ifndef QE_DECODE_SB
+#define QE_DECODE_SB 4
+#endif
+#ifndef QE_DECODE_WAVES
+#define QE_DECODE_WAVES 1
+#endif
+constexpr int kNW = QE_DECODE_NW;    // warps per CTA
+constexpr int kNST = QE_DECODE_NST;  // stages per warp
+constexpr float kRescale = 8.f;  // rescale the accumulators when the max grows by > 2^8
 
 struct DecodeArgs {
   DevState st;
@@ -44,31 +76,15 @@ struct DecodeArgs {
   float scale_log2;  // log2(e) / sqrt(D)
 };
 
-// Sum a value per token over the warp, for 8 tokens at once. Lane l ends with the
-// total of token (l >> 2) & 7 (each token replicated in 4 lanes).
-__device__ __forceinline__ float reduce8(const float (&v)[8], int lane) {
-  const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
-  float r4[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float send = b4 ? v[i] : v[i + 4];
-    const float keep = b4 ? v[i + 4] : v[i];
-    r4[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-  }
-  float r2[2];
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const float send = b3 ? r4[i] : r4[i + 2];
-    const float keep = b3 ? r4[i + 2] : r4[i];
-    r2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-  }
-  const float send = b2 ? r2[0] : r2[1];
-  const float keep = b2 ? r2[1] : r2[0];
-  float r = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-  r += __shfl_xor_sync(0xffffffffu, r, 2);
-  r += __shfl_xor_sync(0xffffffffu, r, 1);
-  return r;
-}
+template <int D, int G>
+struct Map {
+  static constexpr int DPL = G <= 4 ? 16 : 8;  // head-dim elements per lane
+  static constexpr int LPT = D / DPL;          // lanes per token
+  static constexpr int TPS = 32 / LPT;         // tokens per warp step
+  static constexpr int SB = (16 / TPS) < QE_DECODE_SB ? (16 / TPS) : QE_DECODE_SB;  // tokens per group per batch
+  static constexpr int SBT = SB * TPS;         // tokens per batch (divides 16)
+  static constexpr int NP = DPL / 2;           // float pairs per lane
+};
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -76,51 +92,96 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// First list index of split s: windows are weighted 4 (full, tail) and 1 (INT2).
-__device__ __forceinline__ int split_begin(int s, int S, int nf, int nq, int has_tail) {
-  const long long W = 4ll * nf + nq + 4ll * has_tail;
-  const long long t = (s * W + S - 1) / S;
-  if (t <= 4ll * nf) return (int)((t + 3) / 4);
-  if (t <= 4ll * nf + nq) return nf + (int)(t - 4ll * nf);
-  return nf + nq + 1;
+// Chunk order of a lane (DPL = 16): register chunk c holds memory chunk c ^ sw. It may
+// depend on `sub` only: lanes with the same `sub` in different token groups must hold the
+// same elements in the same registers, since the groups are summed register by register.
+// At D = 64 a row is one bank cycle and no lane-only order helps; those loads stay 2-way.
+template <int D, int DPL>
+__device__ __forceinline__ int chunk_swap(int sub, int grp) {
+  (void)grp;
+  if constexpr (DPL == 16 && D == 128) return (sub >> 2) & 1;
+  else return 0;
 }
 
-template <typename T, int D>
-__device__ __forceinline__ void load_row(const T* row, int lane, float (&x)[D / 32]) {
-  constexpr int DPL = D / 32;
-  if constexpr (DPL == 4) {
-    const uint2 w = *reinterpret_cast<const uint2*>(row + lane * 4);
-    x[0] = Elem<T>::lo(w.x);
-    x[1] = Elem<T>::hi(w.x);
-    x[2] = Elem<T>::lo(w.y);
-    x[3] = Elem<T>::hi(w.y);
+template <typename T>
+__device__ __forceinline__ void cvt8(const uint4 w, float2* x) {
+  x[0] = make_float2(Elem<T>::lo(w.x), Elem<T>::hi(w.x));
+  x[1] = make_float2(Elem<T>::lo(w.y), Elem<T>::hi(w.y));
+  x[2] = make_float2(Elem<T>::lo(w.z), Elem<T>::hi(w.z));
+  x[3] = make_float2(Elem<T>::lo(w.w), Elem<T>::hi(w.w));
+}
+
+// the lane's DPL elements of a row as float pairs
+template <typename T, int DPL>
+__device__ __forceinline__ void load_row(const T* row, int sub, int sw, float2 (&x)[DPL / 2]) {
+  const uint4* p = reinterpret_cast<const uint4*>(row + DPL * sub);
+  if constexpr (DPL == 16) {
+    cvt8<T>(p[sw], x);
+    cvt8<T>(p[sw ^ 1], x + 4);
   } else {
-    const uint32_t w = *reinterpret_cast<const uint32_t*>(row + lane * 2);
-    x[0] = Elem<T>::lo(w);
-    x[1] = Elem<T>::hi(w);
+    cvt8<T>(p[0], x);
   }
 }
 
+// x = 1 + c/4 for the 2-bit code c in bits 2E..2E+1 of `bits`
+template <int E>
+__device__ __forceinline__ float code_x(uint32_t bits) {
+  constexpr int sh = 21 - 2 * E;
+  const uint32_t v = sh >= 0 ? (bits << (sh >= 0 ? sh : 0)) : (bits >> (sh < 0 ? -sh : 0));
+  return __uint_as_float((v & 0x00600000u) | 0x3f800000u);
+}
+
+template <int NP>
+__device__ __forceinline__ void decode_codes(uint32_t bits, float2 (&x)[NP]) {
+  x[0] = make_float2(code_x<0>(bits), code_x<1>(bits));
+  x[1] = make_float2(code_x<2>(bits), code_x<3>(bits));
+  x[2] = make_float2(code_x<4>(bits), code_x<5>(bits));
+  x[3] = make_float2(code_x<6>(bits), code_x<7>(bits));
+  if constexpr (NP == 8) {
+    x[4] = make_float2(code_x<8>(bits), code_x<9>(bits));
+    x[5] = make_float2(code_x<10>(bits), code_x<11>(bits));
+    x[6] = make_float2(code_x<12>(bits), code_x<13>(bits));
+    x[7] = make_float2(code_x<14>(bits), code_x<15>(bits));
+  }
+}
+
+// the lane's codes of one row, with register chunk c = memory chunk c ^ sw in bits 16c..
+template <int DPL>
+__device__ __forceinline__ uint32_t load_codes(const uint8_t* row, int sub, int sw) {
+  if constexpr (DPL == 16) {
+    const uint32_t b = reinterpret_cast<const uint32_t*>(row)[sub];
+    return sw ? __funnelshift_l(b, b, 16) : b;
+  } else {
+    return reinterpret_cast<const uint16_t*>(row)[sub];
+  }
+}
+
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kNW * 32) decode_kernel(DecodeArgs a) {
-  constexpr int DPL = D / 32;
-  using R = Int2Row<DPL>;
-  constexpr int PAGE_BYTES = 2 * QE_PAGE * D * 2;   // K rows then V rows
-  constexpr int NORM_BYTES = 64 * G * 4;            // up to a 64-token window
+__global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB) decode_kernel(DecodeArgs a) {
+  using M = Map<D, G>;
+  constexpr int DPL = M::DPL, LPT = M::LPT, TPS = M::TPS, SB = M::SB, SBT = M::SBT, NP = M::NP;
+  constexpr int PAGE_BYTES = 2 * QE_PAGE * D * 2;  // K rows then V rows
+  constexpr int NORM_BYTES = 64 * G * 4;           // up to a 64-token window
   constexpr int STAGE = PAGE_BYTES + NORM_BYTES;
   extern __shared__ __align__(128) uint8_t smem[];
   const DevState& st = a.st;
   const int u = blockIdx.x / a.splits, split = blockIdx.x % a.splits;
   const int b = u / st.Hkv, kvh = u % st.Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp = lane / LPT, sub = lane % LPT;
+  const int sw = chunk_swap<D, DPL>(sub, grp);
   const int w = st.window, ppw = st.ppw;
   const size_t ub = (size_t)u * st.Wmax;
+  const int gi = DPL * sub / 16;  // this lane's INT2 group within a row
 
+  // this split's share of each tier
   const int nf = st.stacks[u * 4 + 2], nq = st.stacks[u * 4 + 3];
-  const int has_tail = a.tail_len > 0;
-  const int nwin = nf + nq + has_tail;
-  const int j0 = split_begin(split, a.splits, nf, nq, has_tail);
-  const int j1 = split + 1 == a.splits ? nwin : split_begin(split + 1, a.splits, nf, nq, has_tail);
+  const int f0 = (int)((long long)nf * split / a.splits), f1 = (int)((long long)nf * (split + 1) / a.splits);
+  const int q0 = (int)((long long)nq * split / a.splits), q1 = (int)((long long)nq * (split + 1) / a.splits);
+  const int has_tail = (a.tail_len > 0 && split == a.splits - 1) ? 1 : 0;
+  const int nF = f1 - f0, nQ = q1 - q0, nJ = nF + nQ + has_tail;
 
   uint8_t* ring = smem + warp * kNST * STAGE;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kNW * kNST * STAGE) + warp * kNST;
@@ -130,35 +191,41 @@ __global__ void __launch_bounds__(kNW * 32) decode_kernel(DecodeArgs a) {
   }
   __syncwarp();
 
-  // query heads of this group, pre-scaled into the log2 domain
-  float q[G][DPL], qsum[G];
+  // the G query heads of this group, this lane's DPL elements, in the log2 domain
+  float2 q[G][NP];
+  float qsum[G];
   {
     const T* qb = reinterpret_cast<const T*>(a.q) + ((size_t)b * st.Hq + (size_t)kvh * G) * D;
+    const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      load_row<T, D>(qb + (size_t)h * D, lane, q[h]);
-      qsum[h] = 0.f;
+      load_row<T, DPL>(qb + (size_t)h * D, sub, sw, q[h]);
+      float2 s2 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int e = 0; e < DPL; ++e) {
-        q[h][e] *= a.scale_log2;
-        qsum[h] += q[h][e];
+      for (int e = 0; e < NP; ++e) {
+        q[h][e] = __fmul2_rn(q[h][e], sc2);
+        s2 = __fadd2_rn(s2, q[h][e]);
       }
+      qsum[h] = s2.x + s2.y;
     }
   }
-  float acc[G][DPL], zacc[G], m[G], lsum[G], lw[G], nw[G];
+  // per lane-group online-softmax state; lw/nw: sums of the current window
+  float2 acc[G][NP];
+  float zacc[G], m[G], lsum[G], lw[G], nw[G];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
     zacc[h] = 0.f;
-    m[h] = -INFINITY;
+    m[h] = -1e30f;
     lsum[h] = 0.f;
     lw[h] = 0.f;
     nw[h] = 0.f;
 #pragma unroll
-    for (int e = 0; e < DPL; ++e) acc[h][e] = 0.f;
+    for (int e = 0; e < NP; ++e) acc[h][e] = make_float2(0.f, 0.f);
   }
 
-  // ---- task iteration: (window list index j, page index pg) ----
-  auto kind_of = [&](int j) { return j < nf ? 0 : (j < nf + nq ? 1 : 2); };  // full, int2, tail
+  // virtual index j of this split -> (kind, list index)
+  auto kind_of = [&](int j) { return j < nF ? 0 : (j < nF + nQ ? 1 : 2); };  // full, int2, tail
+  auto list_idx = [&](int j) { return j < nF ? f0 + j : nf + q0 + (j - nF); };
   auto n_tasks = [&](int j) {
     const int k = kind_of(j);
     return k == 0 ? ppw : (k == 1 ? 1 : (a.tail_len + QE_PAGE - 1) / QE_PAGE);
@@ -169,95 +236,181 @@ __global__ void __launch_bounds__(kNW * 32) decode_kernel(DecodeArgs a) {
       j += kNW;
     }
   };
-  // issue the bulk copies of task (j, pg) into stage s (lane 0 only)
+  // Index prefetch: lane l holds the window id and the page ids (full, tail) or the ledger
+  // slot (INT2) of this warp's window r = rb + l, j = warp + kNW * r, so issuing a copy
+  // never waits on a dependent global load. Reloaded every 32 windows.
+  int e_win = -1, e_id[4] = {-1, -1, -1, -1}, rb = -32;
+  auto load_ids = [&](int base) {
+    rb = base;
+    const int jj = warp + kNW * (base + lane);
+    e_win = -1;
+#pragma unroll
+    for (int p = 0; p < 4; ++p) e_id[p] = -1;
+    if (jj < nJ) {
+      const int kd = kind_of(jj);
+      const int win = kd == 0 ? st.full_list[ub + f0 + jj]
+                              : (kd == 1 ? st.int2_list[ub + q0 + (jj - nF)] : a.tail_win);
+      if (win >= 0 && win < st.Wmax) {
+        e_win = win;
+        if (kd == 1) {
+          e_id[0] = st.win_slot[ub + win];
+        } else {
+#pragma unroll
+          for (int p = 0; p < 4; ++p)
+            if (p < ppw) e_id[p] = st.win_pages[(ub + win) * ppw + p];
+        }
+      }
+    }
+  };
+  // issue the bulk copies of task (j, pg) into stage s (all lanes call; lane 0 copies)
   auto issue = [&](int j, int pg, int s) {
+    const int r = (j - warp) / kNW;
+    if (r - rb >= 32) load_ids(r - r % 32);
+    const int src = r - rb;
+    const int win = __shfl_sync(0xffffffffu, e_win, src);
+    const int sel = pg == 0 ? e_id[0] : (pg == 1 ? e_id[1] : (pg == 2 ? e_id[2] : e_id[3]));
+    const int id = __shfl_sync(0xffffffffu, sel, src);
+    if (lane != 0) return;
+    fence_proxy_async_smem();
     uint8_t* dst = ring + s * STAGE;
     uint64_t* bar = &bars[s];
     const int k = kind_of(j);
     if (k == 1) {
-      const int win = st.int2_list[ub + j - nf];
-      const int slot = (win >= 0 && win < st.Wmax) ? st.win_slot[ub + win] : -1;
-      if (slot < 0 || slot >= st.S) {
+      if (win < 0 || id < 0 || id >= st.S) {
         qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
         mbar_arrive_expect_tx(bar, 0);
         return;
       }
       const uint32_t nb = (uint32_t)(w * G * 4);
       mbar_arrive_expect_tx(bar, (uint32_t)st.slot_bytes + nb);
-      bulk_g2s(dst, st.slots + ((size_t)u * st.S + slot) * st.slot_bytes, (uint32_t)st.slot_bytes, bar);
+      bulk_g2s(dst, st.slots + ((size_t)u * st.S + id) * st.slot_bytes, (uint32_t)st.slot_bytes, bar);
       bulk_g2s(dst + PAGE_BYTES, st.norms + ((size_t)u * st.norm_pitch + (size_t)win * w) * G, nb, bar);
     } else {
-      const int win = k == 0 ? st.full_list[ub + j] : a.tail_win;
-      const int page = (win >= 0 && win < st.Wmax) ? st.win_pages[(ub + win) * ppw + pg] : -1;
-      if (page < 0 || page >= st.P) {
+      if (win < 0 || id < 0 || id >= st.P) {
         qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
         mbar_arrive_expect_tx(bar, 0);
         return;
       }
-      const uint8_t* src = st.pages + ((size_t)u * st.P + page) * st.page_bytes;
+      const uint8_t* src_p = st.pages + ((size_t)u * st.P + id) * st.page_bytes;
       if (k == 0) {
         const uint32_t nb = QE_PAGE * G * 4;
         mbar_arrive_expect_tx(bar, PAGE_BYTES + nb);
-        bulk_g2s(dst, src, PAGE_BYTES, bar);
+        bulk_g2s(dst, src_p, PAGE_BYTES, bar);
         bulk_g2s(dst + PAGE_BYTES,
                  st.norms + ((size_t)u * st.norm_pitch + (size_t)win * w + pg * QE_PAGE) * G, nb, bar);
       } else {
         mbar_arrive_expect_tx(bar, PAGE_BYTES);
-        bulk_g2s(dst, src, PAGE_BYTES, bar);
+        bulk_g2s(dst, src_p, PAGE_BYTES, bar);
       }
     }
   };
 
-  // online-softmax update with one batch of 8 scores (lane holds token (lane>>2)&7)
-  auto online = [&](float (&s)[G], float (&p)[G]) {
+  // softmax bookkeeping for one batch: s[i][h] are the scores of the group's SB tokens
+  // (-inf where invalid); on return they hold the weights 2^(s - m). The running max m
+  // starts at a finite -1e30 so that 2^(-inf - m) = 0 needs no guard. One rarely taken
+  // branch per batch covers every head.
+  auto online = [&](float (&s)[SB][G]) {
+    float mb[G];
+    bool grow = false;
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      float mb = s[h];
-      mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 4));
-      mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 8));
-      mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 16));
-      const float mn = fmaxf(m[h], mb);
-      if (mn == -INFINITY) {
-        p[h] = 0.f;
-        continue;
-      }
-      if (mn > m[h]) {
-        const float sc = exp2f(m[h] - mn);
+      mb[h] = s[0][h];
 #pragma unroll
-        for (int e = 0; e < DPL; ++e) acc[h][e] *= sc;
-        zacc[h] *= sc;
-        lsum[h] *= sc;
-        lw[h] *= sc;
-        nw[h] *= sc;
+      for (int i = 1; i < SB; ++i) mb[h] = fmaxf(mb[h], s[i][h]);
+      grow |= mb[h] > m[h] + kRescale;
+    }
+    if (grow) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float mn = mb[h] > m[h] + kRescale ? mb[h] : m[h];
+        const float f = exp2f(m[h] - mn);
+        const float2 f2 = make_float2(f, f);
+#pragma unroll
+        for (int e = 0; e < NP; ++e) acc[h][e] = __fmul2_rn(acc[h][e], f2);
+        zacc[h] *= f;
+        lsum[h] *= f;
+        lw[h] *= f;
+        nw[h] *= f;
         m[h] = mn;
       }
-      p[h] = exp2f(s[h] - mn);
+    }
+#pragma unroll
+    for (int i = 0; i < SB; ++i)
+#pragma unroll
+      for (int h = 0; h < G; ++h) s[i][h] = exp2f(s[i][h] - m[h]);
+  };
+
+  // sum every score over the LPT lanes of its token (pairs of heads added as f32x2)
+  auto butterfly = [&](float (&s)[SB][G]) {
+#pragma unroll
+    for (int o = LPT / 2; o; o >>= 1)
+#pragma unroll
+      for (int i = 0; i < SB; ++i) {
+#pragma unroll
+        for (int h = 0; h + 1 < G; h += 2) {
+          const float2 r = make_float2(__shfl_xor_sync(0xffffffffu, s[i][h], o),
+                                       __shfl_xor_sync(0xffffffffu, s[i][h + 1], o));
+          const float2 v = __fadd2_rn(make_float2(s[i][h], s[i][h + 1]), r);
+          s[i][h] = v.x;
+          s[i][h + 1] = v.y;
+        }
+        if constexpr (G % 2) s[i][G - 1] += __shfl_xor_sync(0xffffffffu, s[i][G - 1], o);
+      }
+  };
+
+  // window sums of one token: lw += p, nw += p * n (pairs of heads as f32x2)
+  auto window_sums = [&](const float (&p)[G], const float* n) {
+#pragma unroll
+    for (int h = 0; h + 1 < G; h += 2) {
+      const float2 pp = make_float2(p[h], p[h + 1]);
+      const float2 l2 = __fadd2_rn(make_float2(lw[h], lw[h + 1]), pp);
+      // n + h is 8-byte aligned only when G is even (n = norms + t * G)
+      const float2 nn = G % 2 == 0 ? *reinterpret_cast<const float2*>(n + h) : make_float2(n[h], n[h + 1]);
+      const float2 n2 = ffma2(pp, nn, make_float2(nw[h], nw[h + 1]));
+      lw[h] = l2.x;
+      lw[h + 1] = l2.y;
+      nw[h] = n2.x;
+      nw[h + 1] = n2.y;
+    }
+    if constexpr (G % 2) {
+      lw[G - 1] += p[G - 1];
+      nw[G - 1] = fmaf(p[G - 1], n[G - 1], nw[G - 1]);
     }
   };
 
-  int j = j0 + warp, pg = 0;
-  const bool any = j < j1;
-  // prologue: fill kNST - 1 stages
-  int ij = j, ipg = pg, issued = 0;
-  if (lane == 0) {
-    for (int s = 0; s < kNST - 1 && ij < j1; ++s) {
-      issue(ij, ipg, s);
-      advance(ij, ipg);
-      ++issued;
+  // QK of one row of K for every head
+  auto qk_row = [&](const float2 (&kx)[NP], float (&out)[G]) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float2 d2 = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int e = 0; e < NP; ++e) d2 = ffma2(q[h][e], kx[e], d2);
+      out[h] = d2.x + d2.y;
     }
+  };
+
+  // PV of one row of V for every head: acc[h] += p[h] * v
+  auto pv_row = [&](const float2 (&vx)[NP], const float (&p)[G]) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float2 p2 = make_float2(p[h], p[h]);
+#pragma unroll
+      for (int e = 0; e < NP; ++e) acc[h][e] = ffma2(p2, vx[e], acc[h][e]);
+    }
+  };
+
+  int j = warp, pg = 0;
+  int ij = j, ipg = 0, issued = 0;
+  for (int s = 0; s < kNST - 1 && ij < nJ; ++s) {
+    issue(ij, ipg, s);
+    advance(ij, ipg);
+    ++issued;
   }
-  ij = __shfl_sync(0xffffffffu, ij, 0);
-  ipg = __shfl_sync(0xffffffffu, ipg, 0);
-  issued = __shfl_sync(0xffffffffu, issued, 0);
-  int k = 0;  // tasks consumed
+  int k = 0;
   bool ok = true;
-  while (any && j < j1) {
-    // keep kNST - 1 tasks in flight
-    if (ij < j1) {
-      if (lane == 0) {
-        fence_proxy_async_smem();
-        issue(ij, ipg, issued % kNST);
-      }
+  while (j < nJ) {
+    if (ij < nJ) {
+      issue(ij, ipg, issued % kNST);
       advance(ij, ipg);
       ++issued;
     }
@@ -267,124 +420,143 @@ __global__ void __launch_bounds__(kNW * 32) decode_kernel(DecodeArgs a) {
     const uint8_t* stage = ring + s * STAGE;
     const int kind = kind_of(j);
     const float* nrm = reinterpret_cast<const float*>(stage + PAGE_BYTES);
-    if (kind != 1) {
-      // ---- full-precision page (K rows then V rows) ----
+    if (kind == 0) {
+      // ---- full-precision page of a complete window: K rows [16][D], V rows [16][D] ----
       const T* Ks = reinterpret_cast<const T*>(stage);
       const T* Vs = Ks + QE_PAGE * D;
-      const int valid = kind == 2 ? min(QE_PAGE, a.tail_len - pg * QE_PAGE) : QE_PAGE;
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        if (half * 8 >= valid) break;
-        float part[G][8];
+      for (int t0 = 0; t0 < QE_PAGE; t0 += SBT) {
+        float sc[SB][G];
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          float kx[DPL];
-          load_row<T, D>(Ks + (size_t)(half * 8 + t) * D, lane, kx);
+        for (int i = 0; i < SB; ++i) {
+          float2 kx[NP];
+          load_row<T, DPL>(Ks + (size_t)(t0 + i * TPS + grp) * D, sub, sw, kx);
+          qk_row(kx, sc[i]);
+        }
+        butterfly(sc);
+        online(sc);
 #pragma unroll
-          for (int h = 0; h < G; ++h) {
-            float d0 = 0.f;
+        for (int i = 0; i < SB; ++i) {
+          const int t = t0 + i * TPS + grp;
+          window_sums(sc[i], nrm + t * G);
+          float2 vx[NP];
+          load_row<T, DPL>(Vs + (size_t)t * D, sub, sw, vx);
+          pv_row(vx, sc[i]);
+        }
+      }
+    } else if (kind == 2) {
+      // ---- a page of the tail window: mask tokens past its length, keep raw scores ----
+      const T* Ks = reinterpret_cast<const T*>(stage);
+      const T* Vs = Ks + QE_PAGE * D;
+      const int valid = min(QE_PAGE, a.tail_len - pg * QE_PAGE);
+      for (int t0 = 0; t0 < valid; t0 += SBT) {
+        float sc[SB][G];
 #pragma unroll
-            for (int e = 0; e < DPL; ++e) d0 = fmaf(q[h][e], kx[e], d0);
-            part[h][t] = d0;
+        for (int i = 0; i < SB; ++i) {
+          float2 kx[NP];
+          load_row<T, DPL>(Ks + (size_t)(t0 + i * TPS + grp) * D, sub, sw, kx);
+          qk_row(kx, sc[i]);
+        }
+        butterfly(sc);
+#pragma unroll
+        for (int i = 0; i < SB; ++i) {
+          const int t = t0 + i * TPS + grp;
+          if (t >= valid) {
+#pragma unroll
+            for (int h = 0; h < G; ++h) sc[i][h] = -INFINITY;
+          } else if (sub == 0) {
+#pragma unroll
+            for (int h = 0; h < G; ++h) a.tail_s[((size_t)u * w + pg * QE_PAGE + t) * G + h] = sc[i][h];
           }
         }
-        const int tl = half * 8 + ((lane >> 2) & 7);
-        const bool vt = tl < valid;
-        float sc[G], p[G];
+        online(sc);
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          sc[h] = reduce8(part[h], lane);
-          if (!vt) sc[h] = -INFINITY;
-        }
-        online(sc, p);
-        if ((lane & 3) == 0 && vt) {
+        for (int i = 0; i < SB; ++i) {
+          const int t = t0 + i * TPS + grp;
 #pragma unroll
-          for (int h = 0; h < G; ++h) {
-            lsum[h] += p[h];
-            if (kind == 0) {
-              lw[h] += p[h];
-              nw[h] = fmaf(p[h], nrm[tl * G + h], nw[h]);  // this page's 16 tokens
-            } else {
-              a.tail_s[((size_t)u * w + pg * QE_PAGE + tl) * G + h] = sc[h];
-            }
-          }
-        }
-        const int nt = min(8, valid - half * 8);
-        for (int t = 0; t < nt; ++t) {
-          float vx[DPL];
-          load_row<T, D>(Vs + (size_t)(half * 8 + t) * D, lane, vx);
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const float pt = __shfl_sync(0xffffffffu, p[h], t * 4);
-#pragma unroll
-            for (int e = 0; e < DPL; ++e) acc[h][e] = fmaf(pt, vx[e], acc[h][e]);
+          for (int h = 0; h < G; ++h) lw[h] += sc[i][h];
+          if (t < valid) {
+            float2 vx[NP];
+            load_row<T, DPL>(Vs + (size_t)t * D, sub, sw, vx);
+            pv_row(vx, sc[i]);
           }
         }
       }
     } else {
-      // ---- INT2 ledger entry of a whole window: codes K | codes V | meta K | meta V ----
+      // ---- INT2 ledger entry: codes K [w][D/4] | codes V | meta K [w][D/16] | meta V ----
       const uint8_t* kc = stage;
       const uint8_t* vc = stage + w * D / 4;
       const uint32_t* km = reinterpret_cast<const uint32_t*>(stage + w * D / 2);
       const uint32_t* vm = km + w * D / 16;
-      const int grp = R::group_of(lane);
-      for (int t0 = 0; t0 < w; t0 += 8) {
-        float part[G][8];
+      for (int t0 = 0; t0 < w; t0 += SBT) {
+        float sc[SB][G];
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          const uint32_t bits = R::load_codes(kc + (t0 + t) * (D / 4), lane);
-          const uint32_t mt = km[(t0 + t) * (D / 16) + grp];
-          const float sk = meta_scale(mt), zk = meta_zero(mt);
+        for (int i = 0; i < SB; ++i) {
+          const int t = t0 + i * TPS + grp;
+          float2 x[NP];
+          decode_codes<NP>(load_codes<DPL>(kc + t * (D / 4), sub, sw), x);
+          const uint32_t mt = km[t * (D / 16) + gi];
+          const float s4 = 4.f * meta_scale(mt), zz = meta_zero(mt) - s4;
+          float d[G];
+          qk_row(x, d);
+          // score = 4s * (q . x) + (z - 4s) * sum(q)
 #pragma unroll
-          for (int h = 0; h < G; ++h) {
-            float dc = 0.f;
-#pragma unroll
-            for (int e = 0; e < DPL; ++e) dc = fmaf(q[h][e], (float)((bits >> (2 * e)) & 3u), dc);
-            part[h][t] = fmaf(sk, dc, zk * qsum[h]);
+          for (int h = 0; h + 1 < G; h += 2) {
+            const float2 r = ffma2(make_float2(s4, s4), make_float2(d[h], d[h + 1]),
+                                   __fmul2_rn(make_float2(zz, zz), make_float2(qsum[h], qsum[h + 1])));
+            sc[i][h] = r.x;
+            sc[i][h + 1] = r.y;
           }
+          if constexpr (G % 2) sc[i][G - 1] = fmaf(s4, d[G - 1], zz * qsum[G - 1]);
         }
-        const int tl = t0 + ((lane >> 2) & 7);
-        float sc[G], p[G];
+        butterfly(sc);
+        online(sc);
 #pragma unroll
-        for (int h = 0; h < G; ++h) sc[h] = reduce8(part[h], lane);
-        online(sc, p);
-        if ((lane & 3) == 0) {
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            lsum[h] += p[h];
-            lw[h] += p[h];
-            nw[h] = fmaf(p[h], nrm[tl * G + h], nw[h]);
-          }
-        }
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          const uint32_t bits = R::load_codes(vc + (t0 + t) * (D / 4), lane);
-          const uint32_t mt = vm[(t0 + t) * (D / 16) + grp];
-          const float sv = meta_scale(mt), zv = meta_zero(mt);
+        for (int i = 0; i < SB; ++i) {
+          const int t = t0 + i * TPS + grp;
+          window_sums(sc[i], nrm + t * G);
+          float2 x[NP];
+          decode_codes<NP>(load_codes<DPL>(vc + t * (D / 4), sub, sw), x);
+          const uint32_t mt = vm[t * (D / 16) + gi];
+          const float s4 = 4.f * meta_scale(mt), zz = meta_zero(mt) - s4;
+          // v = 4s * x + (z - 4s): acc += (p*4s) * x, zacc += p * (z - 4s)
+          float ps[G];
 #pragma unroll
           for (int h = 0; h < G; ++h) {
-            const float pt = __shfl_sync(0xffffffffu, p[h], t * 4);
-            const float ps = pt * sv;
-#pragma unroll
-            for (int e = 0; e < DPL; ++e) acc[h][e] = fmaf(ps, (float)((bits >> (2 * e)) & 3u), acc[h][e]);
-            zacc[h] = fmaf(pt, zv, zacc[h]);
+            ps[h] = sc[i][h] * s4;
+            zacc[h] = fmaf(sc[i][h], zz, zacc[h]);
           }
+          pv_row(x, ps);
         }
       }
     }
     __syncwarp();
-    // end of a window: record its partial scores
-    const bool last_task = pg + 1 >= n_tasks(j);
-    if (last_task && kind != 2) {
+    if (pg + 1 >= n_tasks(j)) {
+      // end of a window: fold its sums into the total; record full/INT2 window partials
+      if (kind != 2) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          float mx = m[h];
+#pragma unroll
+          for (int o = LPT; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          const float f = exp2f(m[h] - mx);
+          float l2 = lw[h] * f, n2 = nw[h] * f;
+#pragma unroll
+          for (int o = LPT; o < 32; o <<= 1) {
+            l2 += __shfl_xor_sync(0xffffffffu, l2, o);
+            n2 += __shfl_xor_sync(0xffffffffu, n2, o);
+          }
+          if (lane == 0) {
+            float* wp = a.win_part + ((ub + list_idx(j)) * G + h) * 4;
+            wp[0] = mx;
+            wp[1] = l2;
+            wp[2] = n2;
+          }
+        }
+      }
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float l2 = warp_sum(lw[h]), n2 = warp_sum(nw[h]);
-        if (lane == 0) {
-          float* wp = a.win_part + ((ub + j) * G + h) * 4;
-          wp[0] = m[h];
-          wp[1] = l2;
-          wp[2] = n2;
-        }
+        lsum[h] += lw[h];
         lw[h] = 0.f;
         nw[h] = 0.f;
       }
@@ -392,43 +564,70 @@ __global__ void __launch_bounds__(kNW * 32) decode_kernel(DecodeArgs a) {
     advance(j, pg);
     ++k;
   }
-  // drain copies still in flight if a wait gave up
-  if (!ok) {
+  if (!ok) {  // drain copies still in flight if a wait gave up
     for (; k < issued; ++k) mbar_wait_bounded(&bars[k % kNST], (k / kNST) & 1, st.status, 2000 + u);
   }
 
-  // ---- merge the warps of this CTA into one split partial ----
-  __syncthreads();
-  float* mw = reinterpret_cast<float*>(smem);             // [kNW][G]
-  float* lwv = mw + kNW * G;                              // [kNW][G]
-  float* aw = lwv + kNW * G;                              // [kNW][G][D]
+  // ---- merge lane groups, then warps, into one split partial ----
 #pragma unroll
   for (int h = 0; h < G; ++h) {
-    const float l2 = warp_sum(lsum[h]);
-    if (lane == 0) {
-      mw[warp * G + h] = m[h];
-      lwv[warp * G + h] = l2;
-    }
+    float mx = m[h];
 #pragma unroll
-    for (int e = 0; e < DPL; ++e) aw[((size_t)warp * G + h) * D + lane * DPL + e] = acc[h][e] + zacc[h];
+    for (int o = LPT; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float f = exp2f(m[h] - mx);
+    lsum[h] *= f;
+    const float2 z2 = make_float2(zacc[h], zacc[h]), f2 = make_float2(f, f);
+#pragma unroll
+    for (int e = 0; e < NP; ++e) acc[h][e] = __fmul2_rn(__fadd2_rn(acc[h][e], z2), f2);
+#pragma unroll
+    for (int o = LPT; o < 32; o <<= 1) {
+      lsum[h] += __shfl_xor_sync(0xffffffffu, lsum[h], o);
+#pragma unroll
+      for (int e = 0; e < NP; ++e) {
+        acc[h][e].x += __shfl_xor_sync(0xffffffffu, acc[h][e].x, o);
+        acc[h][e].y += __shfl_xor_sync(0xffffffffu, acc[h][e].y, o);
+      }
+    }
+    m[h] = mx;
+  }
+  __syncthreads();
+  float* mw = reinterpret_cast<float*>(smem);  // [kNW][G]
+  float* lwv = mw + kNW * G;                   // [kNW][G]
+  float* aw = lwv + kNW * G;                   // [kNW][G][D]
+  if (lane < LPT) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      if (lane == 0) {
+        mw[warp * G + h] = m[h];
+        lwv[warp * G + h] = lsum[h];
+      }
+#pragma unroll
+      for (int e = 0; e < NP; ++e) {
+        // register pair e of chunk c = e / 4 sits in memory chunk c ^ sw
+        const int d = DPL * sub + 8 * ((e / 4) ^ sw) + 2 * (e % 4);
+        aw[((size_t)warp * G + h) * D + d] = acc[h][e].x;
+        aw[((size_t)warp * G + h) * D + d + 1] = acc[h][e].y;
+      }
+    }
   }
   __syncthreads();
   float* sp = a.split_part + ((size_t)u * a.max_splits + split) * G * (D + 2);
   for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
     const int h = i / D, d = i % D;
-    float M = -INFINITY;
-    for (int x = 0; x < kNW; ++x) M = fmaxf(M, mw[x * G + h]);
+    float Mx = -INFINITY;
+    for (int x = 0; x < kNW; ++x) Mx = fmaxf(Mx, mw[x * G + h]);
     float L = 0.f, A = 0.f;
-    if (M != -INFINITY) {
+    if (Mx != -INFINITY) {
       for (int x = 0; x < kNW; ++x) {
-        const float f = exp2f(mw[x * G + h] - M);
+        const float mm = mw[x * G + h];
+        const float f = mm == -INFINITY ? 0.f : exp2f(mm - Mx);
         L += lwv[x * G + h] * f;
         A += aw[((size_t)x * G + h) * D + d] * f;
       }
     }
     sp[h * (D + 2) + 2 + d] = A;
     if (d == 0) {
-      sp[h * (D + 2) + 0] = M;
+      sp[h * (D + 2) + 0] = Mx;
       sp[h * (D + 2) + 1] = L;
     }
   }
@@ -441,34 +640,34 @@ __global__ void __launch_bounds__(kNW * 32) decode_kernel(DecodeArgs a) {
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  float* lse = reinterpret_cast<float*>(smem);  // [G]
+  float* lse = reinterpret_cast<float*>(smem);  // [8]
   float* red = lse + QE_MAX_G;                  // [32]
   const float* sp0 = a.split_part + (size_t)u * a.max_splits * G * (D + 2);
   if (threadIdx.x < G) {
     const int h = threadIdx.x;
-    float M = -INFINITY;
-    for (int x = 0; x < a.splits; ++x) M = fmaxf(M, __ldcg(sp0 + (x * G + h) * (D + 2)));
+    float Mx = -INFINITY;
+    for (int x = 0; x < a.splits; ++x) Mx = fmaxf(Mx, __ldcg(sp0 + (x * G + h) * (D + 2)));
     float L = 0.f;
     for (int x = 0; x < a.splits; ++x) {
       const float mx = __ldcg(sp0 + (x * G + h) * (D + 2));
-      if (mx != -INFINITY) L += __ldcg(sp0 + (x * G + h) * (D + 2) + 1) * exp2f(mx - M);
+      if (mx != -INFINITY) L += __ldcg(sp0 + (x * G + h) * (D + 2) + 1) * exp2f(mx - Mx);
     }
-    lse[h] = M + log2f(L);
-    red[h] = M;
+    lse[h] = Mx + log2f(L);
+    red[h] = Mx;
     red[8 + h] = L;
   }
   __syncthreads();
   for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
     const int h = i / D, d = i % D;
-    const float M = red[h], L = red[8 + h];
+    const float Mx = red[h], L = red[8 + h];
     float A = 0.f;
     for (int x = 0; x < a.splits; ++x) {
       const float mx = __ldcg(sp0 + (x * G + h) * (D + 2));
-      if (mx != -INFINITY) A += __ldcg(sp0 + (x * G + h) * (D + 2) + 2 + d) * exp2f(mx - M);
+      if (mx != -INFINITY) A += __ldcg(sp0 + (x * G + h) * (D + 2) + 2 + d) * exp2f(mx - Mx);
     }
     a.out[((size_t)b * st.Hq + (size_t)kvh * G + h) * D + d] = A / L;
   }
-  // exact per-window mass and perturbation of this step
+  // exact per-window attention mass and perturbation of this step
   for (int jj = threadIdx.x; jj < nf + nq; jj += blockDim.x) {
     const int win = jj < nf ? st.full_list[ub + jj] : st.int2_list[ub + jj - nf];
     if (win < 0 || win >= st.Wmax) continue;
@@ -483,7 +682,7 @@ __global__ void __launch_bounds__(kNW * 32) decode_kernel(DecodeArgs a) {
     st.mass[ub + win] += dm;
     st.pert[ub + win] += dp;
   }
-  // tail tokens: cumulative per-token attention, window mass
+  // tail tokens: cumulative per-token attention and the window's mass
   float tm = 0.f;
   for (int i = threadIdx.x; i < a.tail_len * G; i += blockDim.x) {
     const int h = i % G;
@@ -492,13 +691,12 @@ __global__ void __launch_bounds__(kNW * 32) decode_kernel(DecodeArgs a) {
     tm += pv;
   }
   tm = warp_sum(tm);
-  __syncthreads();
   if (lane == 0) red[16 + warp] = tm;
   __syncthreads();
   if (threadIdx.x == 0) {
     float s = 0.f;
     for (int x = 0; x < kNW; ++x) s += red[16 + x];
-    if (has_tail) st.mass[ub + a.tail_win] += s;
+    if (a.tail_len > 0) st.mass[ub + a.tail_win] += s;
     a.tickets[u] = 0;
   }
 }
@@ -510,12 +708,16 @@ int launch_decode_t(qe_ctx* c, const void* q, float* out, cudaStream_t s) {
   const size_t smem = (size_t)kNW * kNST * STAGE + kNW * kNST * 8;
   static_assert((size_t)kNW * G * (D + 2) * 4 <= (size_t)kNW * kNST * STAGE, "merge area");
   auto kern = decode_kernel<T, D, G>;
-  QE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  int per_sm = 1, sms = 148, dev = 0;
-  QE_CUDA_TRY(cudaGetDevice(&dev));
-  QE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-  QE_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kNW * 32, smem));
-  if (per_sm < 1) per_sm = 1;
+  // one-time set-up per instantiation (kept out of the per-step path and of graph capture)
+  static int per_sm = 0, sms = 0;
+  if (per_sm == 0) {
+    int dev = 0;
+    QE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    QE_CUDA_TRY(cudaGetDevice(&dev));
+    QE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    QE_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kNW * 32, smem));
+    if (per_sm < 1) per_sm = 1;
+  }
   DecodeArgs a{};
   a.st = make_state(c);
   a.q = q;
@@ -529,8 +731,9 @@ int launch_decode_t(qe_ctx* c, const void* q, float* out, cudaStream_t s) {
   a.tail_len = c->n - c->complete * c->cfg.window;
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
   const int U = c->lay.units;
-  const int nwin = c->n_full_max + c->n_int2_max + 1;
-  int S = (2 * per_sm * sms + U - 1) / U;
+  // one wave of resident CTAs; never more splits than windows per tier
+  const int nwin = c->n_full_max > c->n_int2_max ? c->n_full_max : c->n_int2_max;
+  int S = QE_DECODE_WAVES * per_sm * sms / U;
   if (S > nwin) S = nwin;
   if (S > c->cfg.max_splits) S = c->cfg.max_splits;
   if (S < 1) S = 1;

@@ -173,7 +173,8 @@ static inline bool qe_aligned(const void* p, size_t a) {
 }
 
 // launchers (defined in the .cu files)
-int launch_prefill(qe_ctx* c, const void* K, const void* V, int ctx_len, cudaStream_t st);
+int launch_prefill(qe_ctx* c, const void* K, const void* V, int ctx_len, const float* norms,
+                   cudaStream_t st);
 int launch_append(qe_ctx* c, const void* k, const void* v, cudaStream_t st);
 int launch_decode(qe_ctx* c, const void* q, float* out, cudaStream_t st);
 int launch_finalize(qe_ctx* c, int tail_win, cudaStream_t st);

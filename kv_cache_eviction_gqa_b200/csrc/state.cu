@@ -555,12 +555,24 @@ int apply_dispatch(const qe_ctx* c, const DevState& st, int unit_only, cudaStrea
 
 size_t route_smem(const DevState& st) { return (size_t)st.Wmax * (4 + 4 + 4 + 5) + 64; }
 
+// Raise the route kernel's dynamic shared-memory limit once (outside any graph capture).
+int route_smem_attr(size_t smem) {
+  static size_t granted = 0;
+  if (smem > 200 * 1024) return QE_ERR_UNSUPPORTED_SHAPE;
+  if (smem > granted) {
+    QE_CUDA_TRY(cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
+    granted = 200 * 1024;
+  }
+  return QE_OK;
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------
-int launch_prefill(qe_ctx* c, const void* K, const void* V, int ctx, cudaStream_t s) {
+int launch_prefill(qe_ctx* c, const void* K, const void* V, int ctx, const float* norms,
+                   cudaStream_t s) {
   DevState st = make_state(c);
   const qe_layout& L = c->lay;
   const size_t U = L.units, W = L.max_windows;
@@ -579,6 +591,11 @@ int launch_prefill(qe_ctx* c, const void* K, const void* V, int ctx, cudaStream_
                                                                   ctx);
   prefill_meta_kernel<<<(unsigned)U, 256, 0, s>>>(st, (const uint4*)V, ctx, (uint4*)c->tailV);
   QE_CUDA_TRY(cudaGetLastError());
+  if (norms) {
+    const size_t row = (size_t)ctx * c->G * 4, pitch = (size_t)st.norm_pitch * c->G * 4;
+    QE_CUDA_TRY(cudaMemcpy2DAsync(st.norms, pitch, norms, row, row, U, cudaMemcpyDeviceToDevice, s));
+    return QE_OK;
+  }
   return launch_vwo(V, (int)U, ctx, c->cfg.D, c->cfg.dtype, c->W_O, c->cfg.Hq, c->cfg.Hkv,
                     c->cfg.hidden, st.norms, (long long)st.norm_pitch * c->G, s);
 }
@@ -613,8 +630,7 @@ int launch_route(qe_ctx* c, cudaStream_t s) {
   a.mode = 0;
   a.unit = -1;
   const size_t smem = route_smem(st);
-  if (smem > 200 * 1024) return QE_ERR_UNSUPPORTED_SHAPE;
-  QE_CUDA_TRY(cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  if (int e = route_smem_attr(smem)) return e;
   route_kernel<<<st.U, kRouteThreads, smem, s>>>(a);
   QE_CUDA_TRY(cudaGetLastError());
   return apply_dispatch(c, st, -1, s);
@@ -634,8 +650,7 @@ int launch_set_tier(qe_ctx* c, int unit, const int32_t* ids, int n, int tier, cu
   a.n_ids = n;
   a.target = tier;
   const size_t smem = route_smem(st);
-  if (smem > 200 * 1024) return QE_ERR_UNSUPPORTED_SHAPE;
-  QE_CUDA_TRY(cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  if (int e = route_smem_attr(smem)) return e;
   route_kernel<<<1, kRouteThreads, smem, s>>>(a);
   QE_CUDA_TRY(cudaGetLastError());
   return apply_dispatch(c, st, unit, s);
