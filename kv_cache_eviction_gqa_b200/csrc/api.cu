@@ -259,7 +259,7 @@ QE_API int qe_vwo_l1norm(const void* V, int n_groups, int rows, int D, int dtype
   if (!qe_aligned(V, 16) || !qe_aligned(W_O, 16)) return QE_ERR_INVALID_ARG;
   if (out_group_stride < (long long)rows * (Hq / Hkv)) return QE_ERR_INVALID_ARG;
   if (rows == 0) return QE_OK;
-  return launch_vwo(V, n_groups, rows, D, dtype, W_O, Hq, Hkv, hidden, out, out_group_stride,
+  return launch_vwo(V, n_groups, rows, D, dtype, W_O, Hq, Hkv, hidden, out, out_group_stride, nullptr,
                     (cudaStream_t)s);
 }
 

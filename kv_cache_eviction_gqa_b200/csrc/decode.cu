@@ -11,8 +11,8 @@
 // windows (the last split also takes the tail), so every CTA - and every SM - streams the
 // same mix of bandwidth-heavy full pages and arithmetic-heavy INT2 entries. Inside a CTA
 // each warp takes whole windows round-robin and streams them through its own ring of
-// shared-memory stages with 1-D bulk copies (cp.async.bulk, completion on an mbarrier, no
-// multicast): one 16-token page (K rows then V rows) per stage for a full window, the whole
+// shared-memory stages with 1-D bulk copies (cp.async.bulk, completion on an mbarrier,
+// one CTA only): one 16-token page (K rows then V rows) per stage for a full window, the whole
 // ledger entry for an INT2 window, each with the tokens' projected-value norms.
 //
 // Lane mapping. A token is handled by LPT = D / DPL lanes; lane `sub` owns the DPL

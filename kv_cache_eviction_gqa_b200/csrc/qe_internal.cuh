@@ -105,7 +105,7 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
-// 1-D bulk copy global -> shared, completion signalled on an mbarrier (no multicast).
+// 1-D bulk copy global -> shared of this CTA, completion signalled on an mbarrier.
 // src, dst 16-byte aligned; bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
@@ -181,6 +181,10 @@ int launch_finalize(qe_ctx* c, int tail_win, cudaStream_t st);
 int launch_route(qe_ctx* c, cudaStream_t st);
 int launch_set_tier(qe_ctx* c, int unit, const int32_t* ids_host, int n, int tier, cudaStream_t st);
 int launch_vwo(const void* V, int n_groups, int rows, int D, int dtype, const void* W_O, int Hq,
-               int Hkv, int hidden, float* out, long long out_group_stride, cudaStream_t st);
+               int Hkv, int hidden, float* out, long long out_group_stride, int32_t* status,
+               cudaStream_t st);
+int launch_vwo_tc(const void* V, int n_groups, int rows, int D, int dtype, const void* W_O, int Hq,
+                  int Hkv, int hidden, float* out, long long out_group_stride, int32_t* status,
+                  cudaStream_t st);
 int launch_int2_quantize(const void* x, int T, int D, int dtype, uint8_t* codes, uint32_t* meta,
                          cudaStream_t st);

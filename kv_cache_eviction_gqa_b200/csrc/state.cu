@@ -597,7 +597,7 @@ int launch_prefill(qe_ctx* c, const void* K, const void* V, int ctx, const float
     return QE_OK;
   }
   return launch_vwo(V, (int)U, ctx, c->cfg.D, c->cfg.dtype, c->W_O, c->cfg.Hq, c->cfg.Hkv,
-                    c->cfg.hidden, st.norms, (long long)st.norm_pitch * c->G, s);
+                    c->cfg.hidden, st.norms, (long long)st.norm_pitch * c->G, st.status, s);
 }
 
 int launch_append(qe_ctx* c, const void* k, const void* v, cudaStream_t s) {
@@ -610,7 +610,7 @@ int launch_finalize(qe_ctx* c, int tw, cudaStream_t s) {
   DevState st = make_state(c);
   const int rows = c->cfg.B * c->cfg.window;
   int e = launch_vwo(c->tailV, c->cfg.Hkv, rows, c->cfg.D, c->cfg.dtype, c->W_O, c->cfg.Hq,
-                     c->cfg.Hkv, c->cfg.hidden, c->tail_norm, (long long)rows * c->G, s);
+                     c->cfg.Hkv, c->cfg.hidden, c->tail_norm, (long long)rows * c->G, st.status, s);
   if (e) return e;
   finalize_kernel<<<st.U, 128, 0, s>>>(st, c->tail_norm, tw);
   return cudaGetLastError() == cudaSuccess ? QE_OK : QE_ERR_CUDA;

@@ -3,7 +3,8 @@
 // projected values V W_O; Algoritmo, Etapa 2: A_i * ||V_i W_O||_1).
 //
 // out[g][r][j] = sum_c | sum_d V[g][r][d] * W_O[(kvh*G + j)*D + d][c] |, kvh = g % Hkv.
-// This file holds the dispatcher; the tensor-core kernel lives in vwo_tc.cu.
+// This file holds the dispatcher and a CUDA-core kernel for widths the tensor-core kernel
+// (vwo_tc.cu) does not tile (hidden not a multiple of 128).
 #include "qe_internal.cuh"
 
 namespace {
@@ -83,6 +84,8 @@ int launch_vwo_simt(const void* V, int n_groups, int rows, int D, int dtype, con
 }
 
 int launch_vwo(const void* V, int n_groups, int rows, int D, int dtype, const void* W_O, int Hq,
-               int Hkv, int hidden, float* out, long long ogs, cudaStream_t s) {
+               int Hkv, int hidden, float* out, long long ogs, int32_t* status, cudaStream_t s) {
+  if (hidden % 128 == 0)
+    return launch_vwo_tc(V, n_groups, rows, D, dtype, W_O, Hq, Hkv, hidden, out, ogs, status, s);
   return launch_vwo_simt(V, n_groups, rows, D, dtype, W_O, Hq, Hkv, hidden, out, ogs, s);
 }

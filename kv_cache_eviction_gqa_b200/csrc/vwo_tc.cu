@@ -1,0 +1,331 @@
+// ||V_i W_O^h||_1 on the 5th-generation tensor cores (tcgen05, accumulators in TMEM).
+//
+// "Resumo Técnico: CriticalKV", Framework Teórico: the perturbation bound depends on the
+// projected values V W_O; Algoritmo, Etapa 2 scores an entry by A_i * ||V_i W_O||_1.
+//
+// out[g][r][j] = sum_c | sum_d V[g][r][d] * W_O[(kvh*G + j)*D + d][c] |,  kvh = g % Hkv.
+//
+// One CTA owns 256 rows (two 128-row M-tiles) of one group and a range of N-tiles of
+// 128 columns over (query head j, hidden tile). Warp roles:
+//   warp 0     one elected thread issues TMA loads: the 256 x D block of V once (K-major,
+//              128-byte swizzle), then W_O^h tiles [D rows][128 columns] through a 4-stage
+//              ring. W_O is read in its natural row-major layout as an MN-major operand.
+//   warp 1     allocates 512 TMEM columns; one elected thread issues tcgen05.mma
+//              (kind::f16, M = 128, N = 128, K = 16) into one of two accumulator buffers
+//              (2 M-tiles x 128 columns each) and commits to mbarriers.
+//   warps 2-9  epilogue: each thread owns one accumulator row (TMEM lane), reads 128 fp32
+//              columns with tcgen05.ld, adds their absolute values to a running row sum and
+//              releases the buffer; at the end of a head's columns the row sum is written.
+// The product V W_O (rows x G*hidden) is never stored. All waits are bounded: a wait that
+// gives up records QE_ERR_TIMEOUT, raises a CTA-wide abort flag and the CTA winds down.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "qe_internal.cuh"
+
+namespace {
+
+constexpr int kMT = 2;          // 128-row M-tiles per CTA
+constexpr int kBM = 128;
+constexpr int kBN = 128;        // N tile = TMEM columns per accumulator
+constexpr int kNST = 4;         // W_O stages
+constexpr int kEpiWarps = 4 * kMT;
+constexpr int kThreads = (2 + kEpiWarps) * 32;
+constexpr int kTmemCols = 2 * kMT * kBN;  // two accumulator buffers = 512 columns
+
+struct VwoArgs {
+  float* out;
+  long long ogs;
+  int rows, G, Hkv;
+  int ntiles_per_head;  // hidden / kBN
+  int mpairs;           // ceil(rows / 256)
+  int nsplit;           // N-tile ranges per (group, row block)
+  int ntot;             // G * ntiles_per_head
+  int atomic;           // several CTAs add into one output element
+  int32_t* status;
+};
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                              int32_t* status, int where) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > (1ll << 31)) {
+      *abort_flag = 1;
+      if (status) qe_record_error(status, QE_ERR_TIMEOUT, where);
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// shared-memory matrix descriptor: 128-byte swizzle, sm_100 descriptor version 1
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane -> sum of absolute values
+__device__ __forceinline__ float tmem_abs_sum32(uint32_t taddr) {
+  uint32_t v[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+        "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+        "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+  float2 s = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int i = 0; i < 32; i += 2)
+    s = __fadd2_rn(s, make_float2(fabsf(__uint_as_float(v[i])), fabsf(__uint_as_float(v[i + 1]))));
+  return s.x + s.y;
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+    vwo_tc_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmW, VwoArgs a) {
+  constexpr int KB = D / 64;               // 64-element (128-byte) K boxes
+  constexpr int A_BOX = kBM * 128;         // one box: 128 rows x 128 bytes
+  constexpr int A_BYTES = kMT * KB * A_BOX;
+  constexpr int B_BOX = D * 128;           // one box: D rows x 64 columns x 2 bytes
+  constexpr int B_STAGE = (kBN / 64) * B_BOX;
+  constexpr uint32_t FMT = BF16 ? 1u : 0u;
+  // kind::f16 instruction descriptor: D fp32, A/B fp16|bf16, A K-major, B MN-major, M=128, N=128
+  constexpr uint32_t IDESC = (1u << 4) | (FMT << 7) | (FMT << 10) | (1u << 16) | ((uint32_t)(kBN >> 3) << 17) |
+                             ((uint32_t)(kBM >> 4) << 24);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kNST * B_STAGE);
+  uint64_t* empty = full + kNST;
+  uint64_t* accf = empty + kNST;
+  uint64_t* acce = accf + 2;
+  uint64_t* afull = acce + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(afull + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int item = blockIdx.x;
+  const int split = item % a.nsplit;
+  item /= a.nsplit;
+  const int p = item % a.mpairs, g = item / a.mpairs, kvh = g % a.Hkv;
+  const int n0 = (int)((long long)a.ntot * split / a.nsplit), n1 = (int)((long long)a.ntot * (split + 1) / a.nsplit);
+  const int NT = n1 - n0;
+  const int row0 = p * kMT * kBM;
+  const int grow0 = g * a.rows + row0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kNST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accf[b], 1);
+      mbar_init(&acce[b], kEpiWarps);
+    }
+    mbar_init(afull, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---- producer ----
+      mbar_arrive_expect_tx(afull, A_BYTES);
+      for (int mt = 0; mt < kMT; ++mt)
+        for (int kb = 0; kb < KB; ++kb) tma_load_2d(sA + (mt * KB + kb) * A_BOX, &tmV, kb * 64, grow0 + mt * kBM, afull);
+      for (int i = 0; i < NT; ++i) {
+        const int s = i % kNST;
+        if (!wait_or_abort(&empty[s], ((i / kNST) & 1) ^ 1, abort_flag, a.status, 3001)) break;
+        const int n = n0 + i, j = n / a.ntiles_per_head, nt = n % a.ntiles_per_head;
+        const int hrow = (kvh * a.G + j) * D, col = nt * kBN;
+        mbar_arrive_expect_tx(&full[s], B_STAGE);
+        for (int c = 0; c < kBN / 64; ++c) tma_load_2d(sB + s * B_STAGE + c * B_BOX, &tmW, col + c * 64, hrow, &full[s]);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---- MMA issuer ----
+      if (wait_or_abort(afull, 0, abort_flag, a.status, 3002)) {
+        tc_fence_after();
+        for (int i = 0; i < NT; ++i) {
+          const int s = i % kNST, b = i & 1;
+          if (!wait_or_abort(&full[s], (i / kNST) & 1, abort_flag, a.status, 3003)) break;
+          if (!wait_or_abort(&acce[b], ((i >> 1) & 1) ^ 1, abort_flag, a.status, 3004)) break;
+          tc_fence_after();
+#pragma unroll
+          for (int mt = 0; mt < kMT; ++mt) {
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+              const uint64_t ad = sdesc(smem_u32(sA + (mt * KB + k / 4) * A_BOX + (k % 4) * 32), 16, 1024);
+              const uint64_t bd = sdesc(smem_u32(sB + s * B_STAGE + k * 16 * 128), B_BOX, 1024);
+              mma_f16(tmem + (uint32_t)(b * kMT * kBN + mt * kBN), ad, bd, IDESC, k > 0 ? 1u : 0u);
+            }
+          }
+          mma_commit(&empty[s]);
+          mma_commit(&accf[b]);
+        }
+      }
+    }
+  } else {
+    // ---- epilogue ----
+    const int ew = warp - 2, mt = ew / 4, q = warp & 3;
+    const int r = row0 + mt * kBM + q * 32 + lane;
+    float rowsum = 0.f;
+    for (int i = 0; i < NT; ++i) {
+      const int b = i & 1;
+      if (!__all_sync(0xffffffffu, wait_or_abort(&accf[b], (i >> 1) & 1, abort_flag, a.status, 3005))) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * kMT * kBN + mt * kBN);
+#pragma unroll
+      for (int c = 0; c < kBN / 32; ++c) rowsum += tmem_abs_sum32(taddr + c * 32);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acce[b]);
+      const int n = n0 + i;
+      if (n % a.ntiles_per_head == a.ntiles_per_head - 1 || i == NT - 1) {
+        const int j = n / a.ntiles_per_head;
+        if (r < a.rows) {
+          float* o = a.out + (size_t)g * a.ogs + (size_t)r * a.G + j;
+          if (a.atomic) atomicAdd(o, rowsum);
+          else *o = rowsum;
+        }
+        rowsum = 0.f;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+int make_map(CUtensorMap* m, const void* base, bool bf16, uint64_t inner, uint64_t outer, uint32_t box_inner,
+             uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (!fn) return QE_ERR_CUDA;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner * 2};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? QE_OK : QE_ERR_CUDA;
+}
+
+template <int D, bool BF16>
+int launch_tc(const void* V, int n_groups, int rows, const void* W, int Hq, int Hkv, int hidden, float* out,
+              long long ogs, int32_t* status, cudaStream_t s) {
+  constexpr int KB = D / 64;
+  // at least 120 KB so that two CTAs never share an SM (each holds all 512 TMEM columns)
+  constexpr size_t SMEM_USE = 1024 + (size_t)kMT * KB * kBM * 128 + (size_t)kNST * (kBN / 64) * D * 128 + 256;
+  constexpr size_t SMEM = SMEM_USE > 120 * 1024 ? SMEM_USE : 120 * 1024;
+  auto kern = vwo_tc_kernel<D, BF16>;
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    QE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM));
+    QE_CUDA_TRY(cudaGetDevice(&dev));
+    QE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  }
+  CUtensorMap tmV, tmW;
+  int e = make_map(&tmV, V, BF16, D, (uint64_t)n_groups * rows, 64, kBM);
+  if (e) return e;
+  e = make_map(&tmW, W, BF16, hidden, (uint64_t)Hq * D, 64, D);
+  if (e) return e;
+  VwoArgs a{};
+  a.out = out;
+  a.ogs = ogs;
+  a.rows = rows;
+  a.G = Hq / Hkv;
+  a.Hkv = Hkv;
+  a.ntiles_per_head = hidden / kBN;
+  a.mpairs = (rows + kMT * kBM - 1) / (kMT * kBM);
+  a.ntot = a.G * a.ntiles_per_head;
+  const long long items = (long long)n_groups * a.mpairs;
+  int nsplit = 1;
+  if (items < 2ll * sms) nsplit = (int)((2ll * sms + items - 1) / items);
+  if (nsplit > a.ntot) nsplit = a.ntot;
+  a.nsplit = nsplit;
+  a.atomic = nsplit > 1;
+  a.status = status;
+  if (a.atomic)
+    QE_CUDA_TRY(cudaMemset2DAsync(out, (size_t)ogs * 4, 0, (size_t)rows * a.G * 4, n_groups, s));
+  kern<<<(unsigned)(items * nsplit), kThreads, SMEM, s>>>(tmV, tmW, a);
+  return cudaGetLastError() == cudaSuccess ? QE_OK : QE_ERR_CUDA;
+}
+
+}  // namespace
+
+// Tensor-core path for hidden % 128 == 0; status may be NULL (errors then go nowhere).
+int launch_vwo_tc(const void* V, int n_groups, int rows, int D, int dtype, const void* W_O, int Hq, int Hkv,
+                  int hidden, float* out, long long ogs, int32_t* status, cudaStream_t s) {
+  if (hidden % kBN) return QE_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)n_groups * rows > 0x7fffffffll) return QE_ERR_UNSUPPORTED_SHAPE;
+  const bool bf = dtype == QE_BF16;
+  if (D == 128)
+    return bf ? launch_tc<128, true>(V, n_groups, rows, W_O, Hq, Hkv, hidden, out, ogs, status, s)
+              : launch_tc<128, false>(V, n_groups, rows, W_O, Hq, Hkv, hidden, out, ogs, status, s);
+  return bf ? launch_tc<64, true>(V, n_groups, rows, W_O, Hq, Hkv, hidden, out, ogs, status, s)
+            : launch_tc<64, false>(V, n_groups, rows, W_O, Hq, Hkv, hidden, out, ogs, status, s);
+}
