@@ -154,6 +154,21 @@ QE_API int qe_kv_append(qe_ctx* ctx, const void* k_new, const void* v_new, qe_st
 QE_API int qe_decode_attend_and_score(qe_ctx* ctx, const void* q, float* out,
                                       qe_stream_t stream);
 
+/* qe_decode_attend_and_score_noalloc - the same computation, arguments and results as
+ * qe_decode_attend_and_score, for callers that cannot provide device memory beyond their
+ * inputs and outputs while a step runs (an engine that gives a plugin only its buffers and
+ * forbids allocation during execution, or a process whose memory belongs to another
+ * allocator). The pages have no counterpart to this entry point: it only changes where the
+ * decode kernel keeps its per-call scratch (split and window partials, tail scores, tickets):
+ * in a fixed 16 MiB array inside the library image instead of the workspace scratch region.
+ * It calls no cudaMalloc/cudaFree. Every GPU that loads the library keeps that array until
+ * exit; all calls on one GPU share it, so calls whose kernels overlap on that GPU race and
+ * must be serialised. Returns QE_ERR_INVALID_ARG if the context's scratch would exceed
+ * 16 MiB. The first call on a device resolves the array's address (cudaGetSymbolAddress);
+ * make it before any stream capture. */
+QE_API int qe_decode_attend_and_score_noalloc(qe_ctx* ctx, const void* q, float* out,
+                                              qe_stream_t stream);
+
 /* qe_route_windows - two-stage budgeted routing of every live complete window, then the
  * tier transitions (QEvict Metodologia + CriticalKV Algoritmo):
  *   Full = TwoStage(L, F); INT2 = TwoStage(L \ Full, Q); the rest is evicted for good.

@@ -54,6 +54,7 @@ def lib():
             "qe_load_prefill": (i, [vp, vp, vp, i, vp, vp]),
             "qe_kv_append": (i, [vp, vp, vp, vp]),
             "qe_decode_attend_and_score": (i, [vp, vp, vp, vp]),
+            "qe_decode_attend_and_score_noalloc": (i, [vp, vp, vp, vp]),
             "qe_route_windows": (i, [vp, vp]),
             "qe_decode_step": (i, [vp, vp, vp, vp, vp, vp]),
             "qe_quantize_once": (i, [vp, i, vp, i, vp]),

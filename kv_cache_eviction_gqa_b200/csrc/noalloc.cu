@@ -1,0 +1,80 @@
+// Allocation-free variant of qe_decode_attend_and_score.
+//
+// Some callers cannot give this library extra device memory at run time: for example an
+// inference engine that hands a plugin only its input and output buffers and forbids any
+// allocation while a request executes, or a process whose device memory is entirely owned
+// by another allocator. For them this entry point runs the split-K decode kernel with its
+// per-call scratch (split partials, per-window partials, tail-token scores and the
+// per-unit completion tickets) in a fixed array that is part of the library image, instead
+// of the scratch region of the context workspace. The cache state itself still lives in the
+// caller's workspace, and q / out are the caller's buffers.
+//
+// The array is a file-scope __device__ object of kStaticScratchBytes: every GPU that loads
+// this library holds that much memory until the process exits. All calls on one GPU share
+// it and it keeps the previous call's contents, so the tickets are cleared on every call,
+// and two calls whose kernels overlap on the same GPU (for example two contexts on two
+// streams) race on it: issue them one after the other. A config whose scratch needs more
+// than kStaticScratchBytes is rejected with QE_ERR_INVALID_ARG before anything is enqueued.
+// The first call on a device looks up the array's device address (cudaGetSymbolAddress with
+// that device current) and caches it; make that first call before any stream capture.
+#include "qe_internal.cuh"
+
+namespace {
+
+constexpr size_t kStaticScratchBytes = 16u << 20;  // 16 MiB
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+uint8_t* g_scratch_ptr[kMaxDevices];  // device address of g_static_scratch per device
+
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Device address of the static scratch on the current device. The first call on a device
+// resolves it with cudaGetSymbolAddress (with that device current) and caches it.
+int static_scratch(uint8_t** out) {
+  int dev = 0;
+  QE_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return QE_ERR_INVALID_ARG;
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return QE_ERR_CUDA;
+    g_scratch_ptr[dev] = static_cast<uint8_t*>(p);
+  }
+  *out = g_scratch_ptr[dev];
+  return QE_OK;
+}
+
+}  // namespace
+
+extern "C" QE_API int qe_decode_attend_and_score_noalloc(qe_ctx* c, const void* q, float* out,
+                                                         qe_stream_t s) {
+  if (!c || !q || !out) return QE_ERR_INVALID_ARG;
+  // the decode kernel's per-call scratch, laid out like the workspace scratch
+  const size_t U = c->lay.units, G = c->G, D = c->cfg.D, w = c->cfg.window, W = c->lay.max_windows;
+  const size_t b_split = round256(U * c->cfg.max_splits * G * (2 + D) * 4);
+  const size_t b_win = round256(U * W * G * 4 * 4);
+  const size_t b_tail = round256(U * w * G * 4);
+  const size_t b_tick = round256(U * 4);
+  if (b_split + b_win + b_tail + b_tick > kStaticScratchBytes) return QE_ERR_INVALID_ARG;
+  uint8_t* base = nullptr;
+  int e = static_scratch(&base);
+  if (e) return e;
+  cudaStream_t st = (cudaStream_t)s;
+  uint32_t* tickets = reinterpret_cast<uint32_t*>(base + b_split + b_win + b_tail);
+  QE_CUDA_TRY(cudaMemsetAsync(tickets, 0, U * 4, st));
+  // run the regular entry point with the context's scratch pointers aimed at the array
+  float* sp = c->split_part;
+  float* wp = c->win_part;
+  float* ts = c->tail_s;
+  uint32_t* tk = c->tickets;
+  c->split_part = reinterpret_cast<float*>(base);
+  c->win_part = reinterpret_cast<float*>(base + b_split);
+  c->tail_s = reinterpret_cast<float*>(base + b_split + b_win);
+  c->tickets = tickets;
+  e = qe_decode_attend_and_score(c, q, out, s);
+  c->split_part = sp;
+  c->win_part = wp;
+  c->tail_s = ts;
+  c->tickets = tk;
+  return e;
+}
