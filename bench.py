@@ -417,6 +417,8 @@ def run_ours(args, rank, world, local_rank):
                              "note": "decode steps with no routing and no window completion"},
             "per_step_first_sequence": [
                 {"s": i, "step_us": round(step_ms[i] * 1e3, 2), "decode_us": round(dec_ms[i] * 1e3, 2),
+                 "append_us": round(ev[i][0].elapsed_time(ev[i][1]) * 1e3, 2),
+                 "route_us": round(ev[i][2].elapsed_time(ev[i][3]) * 1e3, 2),
                  "decode_gbs": round(decode_bytes(cfg, *meta[i][:3]) / (dec_ms[i] / 1e3) / 1e9, 1)}
                 for i in range(min(K_steps, S)) if i < 3 or i % 16 in (0, 1) or meta[i][3]],
             "roofline": {"kernel": "decode_kernel (split-K GQA decode + window scoring)",

@@ -31,11 +31,21 @@ struct Int2Row {
     const __half sh = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), 3.0f));
     const __half zh = __float2half_rn(mn);
     const float s = __half2float(sh), z = __half2float(zh);
+    // code = rint(f32(x - z) / s): the quotient is formed with a reciprocal, whose error
+    // (a few ulp, < 1e-6 here) can only change rint() next to a half-integer; within 1e-3 of
+    // one the correctly rounded division decides instead, so the result is that of rint of
+    // the IEEE quotient in every case.
+    const float rs = s != 0.f ? __frcp_rn(s) : 0.f;
     uint32_t bits = 0;
 #pragma unroll
     for (int e = 0; e < DPL; ++e) {
       float c = 0.f;
-      if (s != 0.f) c = fminf(fmaxf(rintf(__fdiv_rn(__fsub_rn(x[e], z), s)), 0.f), 3.f);
+      if (s != 0.f) {
+        const float d = __fsub_rn(x[e], z);
+        float qv = __fmul_rn(d, rs);
+        if (fabsf(qv - floorf(qv) - 0.5f) < 1e-3f) qv = __fdiv_rn(d, s);
+        c = fminf(fmaxf(rintf(qv), 0.f), 3.f);
+      }
       bits |= static_cast<uint32_t>(c) << (2 * e);
     }
     *meta = static_cast<uint32_t>(__half_as_ushort(sh)) |

@@ -215,11 +215,36 @@ struct RouteArgs {
   int target;          // mode 1: QE_TIER_INT2 or QE_TIER_FULL
 };
 
-// Two-stage selection among candidates with inset[i]; selected ones get sel[i] = 1.
-// Ranks use 64-bit keys (ordered score, ~window) so ties go to the lower window index.
-__device__ void two_stage_select(int n, const int32_t* cand, const float* k1, const float* k2,
+// Sort N 64-bit keys in shared memory in descending order (bitonic network, N a power of 2).
+__device__ void bitonic_desc(unsigned long long* key, int N) {
+  for (int k = 2; k <= N; k <<= 1)
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < N; i += blockDim.x) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const unsigned long long x = key[i], y = key[ixj];
+          if (((i & k) == 0) ? (x < y) : (x > y)) {
+            key[i] = y;
+            key[ixj] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+}
+
+// Selection key: higher score first, then the lower window id; the candidate index rides in
+// the low 12 bits (window ids < 2^20, candidates < 4096). Every real key is non-zero.
+__device__ __forceinline__ unsigned long long sel_key(float score, int win, int idx) {
+  return ((unsigned long long)ordered_bits(score) << 32) |
+         ((unsigned long long)(0xFFFFFu - (uint32_t)win) << 12) | (uint32_t)idx;
+}
+
+// Two-stage selection among candidates with inset[i]; selected ones get sel[i] = 1 and the
+// stage-1 picks s1mark[i] = 1. `key` holds N >= n 64-bit keys (N a power of two).
+__device__ void two_stage_select(int n, int N, const int32_t* cand, const float* k1, const float* k2,
                                  const uint8_t* inset, uint8_t* sel, uint8_t* s1mark, int b, int b1,
-                                 int* ibuf) {
+                                 int* ibuf, unsigned long long* key) {
   int cnt_local = 0;
   for (int i = threadIdx.x; i < n; i += blockDim.x) cnt_local += inset[i];
   int cnt;
@@ -232,39 +257,23 @@ __device__ void two_stage_select(int n, const int32_t* cand, const float* k1, co
     __syncthreads();
     return;
   }
-  // stage 1: rank by k1 among inset
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    uint8_t s = 0;
-    if (inset[i]) {
-      const unsigned long long ki =
-          ((unsigned long long)ordered_bits(k1[i]) << 32) | (0xffffffffu - (uint32_t)cand[i]);
-      int rank = 0;
-      for (int j = 0; j < n; ++j) {
-        const unsigned long long kj =
-            ((unsigned long long)ordered_bits(k1[j]) << 32) | (0xffffffffu - (uint32_t)cand[j]);
-        rank += (inset[j] && kj > ki);
-      }
-      s = rank < b1;
-    }
-    s1mark[i] = s;
+  // stage 1: the b1 largest k1 among inset
+  for (int i = threadIdx.x; i < N; i += blockDim.x) {
+    key[i] = (i < n && inset[i]) ? sel_key(k1[i], cand[i], i) : 0ull;
+    if (i < n) s1mark[i] = 0;
   }
   __syncthreads();
-  // stage 2: rank by k2 among inset minus stage 1
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    uint8_t s = s1mark[i];
-    if (inset[i] && !s1mark[i]) {
-      const unsigned long long ki =
-          ((unsigned long long)ordered_bits(k2[i]) << 32) | (0xffffffffu - (uint32_t)cand[i]);
-      int rank = 0;
-      for (int j = 0; j < n; ++j) {
-        const unsigned long long kj =
-            ((unsigned long long)ordered_bits(k2[j]) << 32) | (0xffffffffu - (uint32_t)cand[j]);
-        rank += (inset[j] && !s1mark[j] && kj > ki);
-      }
-      s = rank < b - b1;
-    }
-    sel[i] = s;
+  bitonic_desc(key, N);
+  for (int r = threadIdx.x; r < b1; r += blockDim.x) s1mark[key[r] & 0xFFFu] = 1;
+  __syncthreads();
+  // stage 2: the b - b1 largest k2 among inset minus stage 1
+  for (int i = threadIdx.x; i < N; i += blockDim.x) {
+    key[i] = (i < n && inset[i] && !s1mark[i]) ? sel_key(k2[i], cand[i], i) : 0ull;
+    if (i < n) sel[i] = s1mark[i];
   }
+  __syncthreads();
+  bitonic_desc(key, N);
+  for (int r = threadIdx.x; r < b - b1; r += blockDim.x) sel[key[r] & 0xFFFu] = 1;
   __syncthreads();
 }
 
@@ -273,7 +282,12 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
   const int u = a.mode == 1 ? a.unit : blockIdx.x;
   extern __shared__ __align__(16) uint8_t sm[];
   const int nf = st.stacks[u * 4 + 2], nq = st.stacks[u * 4 + 3], n = nf + nq;
-  int32_t* cand = reinterpret_cast<int32_t*>(sm);
+  int NW = 1;  // key buffer capacity (power of two >= Wmax)
+  while (NW < st.Wmax) NW <<= 1;
+  int N = 1;   // sort size: power of two >= the candidate count
+  while (N < n) N <<= 1;
+  unsigned long long* key = reinterpret_cast<unsigned long long*>(sm);
+  int32_t* cand = reinterpret_cast<int32_t*>(key + NW);
   float* km = reinterpret_cast<float*>(cand + st.Wmax);
   float* kp = km + st.Wmax;
   uint8_t* oldt = reinterpret_cast<uint8_t*>(kp + st.Wmax);
@@ -304,7 +318,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
   if (a.mode == 0) {
     for (int i = threadIdx.x; i < n; i += blockDim.x) inset[i] = 1;
     __syncthreads();
-    two_stage_select(n, cand, km, kp, inset, sel, s1, a.F, a.F1, ibuf);
+    two_stage_select(n, N, cand, km, kp, inset, sel, s1, a.F, a.F1, ibuf, key);
     float s1m = 0.f, am = 0.f;
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
       if (sel[i]) newt[i] = QE_TIER_FULL;
@@ -314,7 +328,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
     }
     stage1_mass = block_sum(s1m, fbuf);
     all_mass = block_sum(am, fbuf);
-    two_stage_select(n, cand, km, kp, inset, sel, s1, a.Q, a.Q1, ibuf);
+    two_stage_select(n, N, cand, km, kp, inset, sel, s1, a.Q, a.Q1, ibuf, key);
     for (int i = threadIdx.x; i < n; i += blockDim.x)
       if (sel[i]) newt[i] = QE_TIER_INT2;
   } else {
@@ -460,7 +474,9 @@ __global__ void apply_kernel(DevState st, const int32_t* xlist, const int32_t* p
   const int nx = xcount[u * 4 + 0], np = xcount[u * 4 + 1];
   const size_t ub = (size_t)u * st.Wmax;
   const int w = st.window;
-  for (int item = gw; item < nx + np; item += gridDim.y * warps) {
+  // one warp per (window, token): the K row and the V row of that token
+  for (int it = gw; it < (nx + np) * w; it += gridDim.y * warps) {
+    const int item = it / w, t = it % w;
     const bool quant = item < nx;
     const int win = quant ? xlist[ub + item] : plist[ub + item - nx];
     const int slot = st.win_slot[ub + win];
@@ -473,11 +489,11 @@ __global__ void apply_kernel(DevState st, const int32_t* xlist, const int32_t* p
     uint8_t* vc = sl + (size_t)w * D / 4;
     uint32_t* km = reinterpret_cast<uint32_t*>(sl + (size_t)w * D / 2);
     uint32_t* vm = km + (size_t)w * D / 16;
-    for (int t = 0; t < w; ++t) {
+    {
       const int page = st.win_pages[(ub + win) * st.ppw + t / QE_PAGE];
       if (page < 0 || page >= st.P) {
         if (lane == 0) qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
-        break;
+        continue;
       }
       T* prow = reinterpret_cast<T*>(st.pages + ((size_t)u * st.P + page) * st.page_bytes);
       T* krow = prow + (size_t)(t % QE_PAGE) * D;
@@ -534,8 +550,8 @@ __global__ void int2_quantize_kernel(const T* x, int rows, uint8_t* codes, uint3
 template <typename T, int D>
 void launch_apply(const DevState& st, const qe_ctx* c, int unit_only, cudaStream_t s) {
   const int units = unit_only >= 0 ? 1 : st.U;
-  // enough warps to give every window of the largest possible transition list its own warp
-  int per_unit = (st.Wmax + 7) / 8;
+  // 8 warps per block, up to 64 blocks per unit, each warp one (window, token) at a time
+  int per_unit = (st.Wmax * st.window + 7) / 8;
   if (per_unit > 64) per_unit = 64;
   apply_kernel<T, D><<<dim3(units, per_unit), 256, 0, s>>>(st, c->xlist, c->plist, c->xcount,
                                                             unit_only);
@@ -553,12 +569,16 @@ int apply_dispatch(const qe_ctx* c, const DevState& st, int unit_only, cudaStrea
   return cudaGetLastError() == cudaSuccess ? QE_OK : QE_ERR_CUDA;
 }
 
-size_t route_smem(const DevState& st) { return (size_t)st.Wmax * (4 + 4 + 4 + 5) + 64; }
+size_t route_smem(const DevState& st) {
+  size_t N = 1;
+  while (N < (size_t)st.Wmax) N <<= 1;
+  return N * 8 + (size_t)st.Wmax * (4 + 4 + 4 + 5) + 64;
+}
 
 // Raise the route kernel's dynamic shared-memory limit once (outside any graph capture).
-int route_smem_attr(size_t smem) {
+int route_smem_attr(size_t smem, int Wmax) {
   static size_t granted = 0;
-  if (smem > 200 * 1024) return QE_ERR_UNSUPPORTED_SHAPE;
+  if (smem > 200 * 1024 || Wmax > 4096) return QE_ERR_UNSUPPORTED_SHAPE;
   if (smem > granted) {
     QE_CUDA_TRY(cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
     granted = 200 * 1024;
@@ -630,7 +650,7 @@ int launch_route(qe_ctx* c, cudaStream_t s) {
   a.mode = 0;
   a.unit = -1;
   const size_t smem = route_smem(st);
-  if (int e = route_smem_attr(smem)) return e;
+  if (int e = route_smem_attr(smem, st.Wmax)) return e;
   route_kernel<<<st.U, kRouteThreads, smem, s>>>(a);
   QE_CUDA_TRY(cudaGetLastError());
   return apply_dispatch(c, st, -1, s);
@@ -650,7 +670,7 @@ int launch_set_tier(qe_ctx* c, int unit, const int32_t* ids, int n, int tier, cu
   a.n_ids = n;
   a.target = tier;
   const size_t smem = route_smem(st);
-  if (int e = route_smem_attr(smem)) return e;
+  if (int e = route_smem_attr(smem, st.Wmax)) return e;
   route_kernel<<<1, kRouteThreads, smem, s>>>(a);
   QE_CUDA_TRY(cudaGetLastError());
   return apply_dispatch(c, st, unit, s);
