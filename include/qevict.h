@@ -230,20 +230,38 @@ QE_API int qe_criticalkv_select(const void* q_obs, int n_obs, const void* K, con
                                 float* A_out, float* N_out, int32_t* idx_out,
                                 void* scratch, size_t scratch_bytes, qe_stream_t stream);
 
-/* qe_trim_global_topm - DBTrimKV global top-M over log r = (t - pos) * ln(beta) in float64
- * across every (layer, head) of a paged variable-length cache ("Make Each Token Count",
- * Metodologia 2-4). Ties go to the lower flat index (head-major, then entry).
- *   beta [dev, float], pos [dev, int32]: [n_pages_total][16] per physical page.
- *   page_table [dev, int32]: [n_heads][max_pages_per_head] physical page of each logical page.
- *   lengths [dev, int32]: [n_heads].  kv_in [dev]: [n_pages_total][2][16][D] dtype.
- *   kv_out, beta_out, pos_out [dev]: same shapes as the inputs; head h's survivors are
- *   written in their original order to its logical pages 0.. through the same page table.
- *   new_lengths [dev, int32]: [n_heads]. scratch [dev]: qe_trim_scratch_bytes() bytes. */
+/* qe_trim_global_topm - DBTrimKV global trim of a paged, variable-length cache ("Make Each
+ * Token Count", Metodologia 2-4: the retention of entry i at step t is beta_i^(t - pos_i); the
+ * cache keeps the M entries of highest retention over every (layer, head) and drops the rest).
+ * Each entry's key is log r = (t - pos) * ln(beta), computed in float64 (beta widened from
+ * float32 exactly, ln in float64). Entries are ranked by key, descending; equal keys go to the
+ * lower flat index, where the flat index runs over heads first (head 0's entries, then head 1's,
+ * ...) and then over a head's entries in logical order. The first M are kept (all of them when
+ * M is at least the total; none when M == 0).
+ *   beta [dev, float], pos [dev, int32]: [n_pages_total][16], indexed by physical page and slot.
+ *     beta is expected in (0, 1]; a key that is NaN ranks below every other key.
+ *   page_table [dev, int32]: [n_heads][max_pages_per_head]; entry (h, p) is the physical page of
+ *     head h's logical page p. Entry e of head h lives in logical page e/16, slot e%16.
+ *   lengths [dev, int32]: [n_heads] entries per head, each in [0, 16*max_pages_per_head].
+ *   kv_in [dev]: [n_pages_total][2][16][D] dtype (K rows of a page, then its V rows).
+ *   kv_out, beta_out, pos_out [dev]: same shapes as kv_in, beta, pos, and must not overlap them.
+ *     Head h's survivors are written in their original order to its logical entries 0..L_h-1,
+ *     through the same page table. Nothing else in the outputs is written.
+ *   new_lengths [dev, int32]: [n_heads] survivor count L_h of each head.
+ *   scratch [dev]: qe_trim_scratch_bytes(n_heads, max_pages_per_head) bytes, 256-byte aligned,
+ *     owned by the caller and not shared by concurrent calls. Its first 8 bytes receive a status
+ *     word {int32 code, int32 detail}: 0 after a clean run, otherwise the first device-side error
+ *     (QE_ERR_INVALID_ARG for a length out of range, QE_ERR_DEVICE_FAULT for a page-table entry
+ *     outside [0, n_pages_total); detail = the head). The caller reads it after synchronising.
+ * Host-side errors (returned, nothing launched): QE_ERR_INVALID_ARG for a null or misaligned
+ * pointer (kv 16-byte aligned), M < 0, overlapping in/out buffers or a small scratch;
+ * QE_ERR_UNSUPPORTED_SHAPE for D not in {64, 128, 256} or n_heads * 16 * max_pages_per_head
+ * at or above 2^31. Asynchronous on `stream`; allocates nothing. */
 QE_API size_t qe_trim_scratch_bytes(int n_heads, int max_pages_per_head);
 QE_API int qe_trim_global_topm(const float* beta, const int32_t* pos, const int32_t* page_table,
                                const int32_t* lengths, int n_heads, int max_pages_per_head,
-                               int D, int dtype, int t, long long M, const void* kv_in,
-                               void* kv_out, float* beta_out, int32_t* pos_out,
+                               int n_pages_total, int D, int dtype, int t, long long M,
+                               const void* kv_in, void* kv_out, float* beta_out, int32_t* pos_out,
                                int32_t* new_lengths, void* scratch, size_t scratch_bytes,
                                qe_stream_t stream);
 

@@ -18,6 +18,8 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqevict.
 _lib = None
 
 QE_FP16, QE_BF16 = 0, 1
+(QE_OK, QE_ERR_INVALID_ARG, QE_ERR_UNSUPPORTED_SHAPE, QE_ERR_POOL_EXHAUSTED, QE_ERR_LEDGER_FULL,
+ QE_ERR_CUDA, QE_ERR_TIMEOUT, QE_ERR_DEVICE_FAULT, QE_ERR_WORKSPACE, QE_ERR_STATE) = range(0, -10, -1)
 TIER_EVICTED, TIER_INT2, TIER_FULL, TIER_TAIL = 0, 1, 2, 3
 
 
@@ -65,8 +67,8 @@ def lib():
             "qe_criticalkv_select": (i, [vp, i, vp, vp, vp, i, i, i, i, i, i, i, i, f, vp, vp, vp,
                                          vp, sz, vp]),
             "qe_trim_scratch_bytes": (sz, [i, i]),
-            "qe_trim_global_topm": (i, [vp, vp, vp, vp, i, i, i, i, i, ll, vp, vp, vp, vp, vp, vp,
-                                        sz, vp]),
+            "qe_trim_global_topm": (i, [vp, vp, vp, vp, i, i, i, i, i, i, ll, vp, vp, vp, vp, vp,
+                                        vp, sz, vp]),
             "qe_status": (i, [vp, C.POINTER(C.c_int)]),
             "qe_step_index": (i, [vp]),
             "qe_length": (i, [vp]),
@@ -313,3 +315,48 @@ def vwo_l1norm(V: torch.Tensor, W_O: torch.Tensor, Hq: int, Hkv: int, out=None, 
     _check(lib().qe_vwo_l1norm(_ptr(V), n_groups, rows, D, dtype_code(V.dtype), _ptr(W_O), Hq, Hkv,
                                W_O.shape[1], _ptr(out), rows * G, _stream(stream)), "qe_vwo_l1norm")
     return out
+
+
+def trim_scratch_bytes(n_heads: int, max_pages_per_head: int) -> int:
+    return int(lib().qe_trim_scratch_bytes(n_heads, max_pages_per_head))
+
+
+def trim_global_topm(beta: torch.Tensor, pos: torch.Tensor, page_table: torch.Tensor,
+                     lengths: torch.Tensor, t: int, M: int, kv_in: torch.Tensor, kv_out=None,
+                     beta_out=None, pos_out=None, new_lengths=None, scratch=None, stream=None):
+    """DBTrimKV global top-M trim with stable per-head compaction (qe_trim_global_topm).
+
+    beta [P][16] float32, pos [P][16] int32, page_table [H][max_pages] int32, lengths [H] int32,
+    kv_in [P][2][16][D] fp16/bf16. Returns (kv_out, beta_out, pos_out, new_lengths, scratch);
+    the device status word is scratch[:8] (see trim_status).
+    """
+    _need(beta, "beta", torch.float32)
+    P = beta.shape[0]
+    _need(pos, "pos", torch.int32, beta.shape)
+    _need(page_table, "page_table", torch.int32)
+    H, max_pages = page_table.shape
+    _need(lengths, "lengths", torch.int32, (H,))
+    _need(kv_in, "kv_in")
+    D = kv_in.shape[-1]
+    dev = kv_in.device
+    kv_out = torch.empty_like(kv_in) if kv_out is None else kv_out
+    beta_out = torch.empty_like(beta) if beta_out is None else beta_out
+    pos_out = torch.empty_like(pos) if pos_out is None else pos_out
+    new_lengths = torch.empty(H, dtype=torch.int32, device=dev) if new_lengths is None else new_lengths
+    for name, x, y in (("kv_out", kv_out, kv_in), ("beta_out", beta_out, beta), ("pos_out", pos_out, pos)):
+        _need(x, name, y.dtype, y.shape)
+    nbytes = trim_scratch_bytes(H, max_pages)
+    if scratch is None:
+        scratch = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    _check(lib().qe_trim_global_topm(_ptr(beta), _ptr(pos), _ptr(page_table), _ptr(lengths), H,
+                                     max_pages, P, D, dtype_code(kv_in.dtype), int(t), int(M),
+                                     _ptr(kv_in), _ptr(kv_out), _ptr(beta_out), _ptr(pos_out),
+                                     _ptr(new_lengths), _ptr(scratch), scratch.numel(),
+                                     _stream(stream)), "qe_trim_global_topm")
+    return kv_out, beta_out, pos_out, new_lengths, scratch
+
+
+def trim_status(scratch: torch.Tensor):
+    """(code, detail) of the device status word a trim call left in its scratch."""
+    w = scratch[:8].view(torch.int32).cpu()
+    return int(w[0]), int(w[1])

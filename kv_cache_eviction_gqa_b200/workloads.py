@@ -312,3 +312,66 @@ def draw_trim_kv_page(cfg: TrimConfig, head: int, page: int):
     r = _rng(cfg.seed, 0x7A6E, head, page)
     kv = r.standard_normal((2, cfg.page, cfg.D), dtype=np.float32)
     return to_dtype_values(kv, cfg.dtype)
+
+
+@dataclass
+class TrimLayout:
+    """A paged cache for the trim: per-head entries scattered over physical pages.
+
+    lengths [H] int32; page_table [H][max_pages] int32 (-1 past a head's pages);
+    beta_pages [P][page] float32 and pos_pages [P][page] int32 by physical page and slot
+    (slots past a head's length hold beta 1, pos 0); betas/poss the per-head arrays in
+    logical order (the same values).
+    """
+    lengths: np.ndarray
+    page_table: np.ndarray
+    beta_pages: np.ndarray
+    pos_pages: np.ndarray
+    betas: list
+    poss: list
+
+    @property
+    def n_pages(self) -> int:
+        return self.beta_pages.shape[0]
+
+
+def trim_layout(cfg: TrimConfig, lengths=None, betas=None, poss=None) -> TrimLayout:
+    """Lay the (drawn or given) per-head metadata out over a seeded permutation of pages."""
+    if lengths is None:
+        lengths, betas, poss = draw_trim_meta(cfg)
+    lengths = np.asarray(lengths, dtype=np.int32)
+    pg = cfg.page
+    max_pages = max(1, -(-cfg.len_hi // pg))
+    n_pages = [-(-int(n) // pg) for n in lengths]
+    P = max(1, sum(n_pages))
+    perm = _rng(cfg.seed, 0x9A6E).permutation(P).astype(np.int32)
+    table = np.full((len(lengths), max_pages), -1, dtype=np.int32)
+    beta_pages = np.ones((P, pg), dtype=np.float32)
+    pos_pages = np.zeros((P, pg), dtype=np.int32)
+    a = 0
+    for h, n in enumerate(lengths):
+        k = n_pages[h]
+        phys = perm[a:a + k]
+        a += k
+        table[h, :k] = phys
+        pad = k * pg - int(n)
+        b = np.concatenate([np.asarray(betas[h], dtype=np.float32), np.ones(pad, np.float32)])
+        q = np.concatenate([np.asarray(poss[h], dtype=np.int32), np.zeros(pad, np.int32)])
+        beta_pages[phys] = b.reshape(k, pg)
+        pos_pages[phys] = q.reshape(k, pg)
+    return TrimLayout(lengths, table, beta_pages, pos_pages, list(betas), list(poss))
+
+
+def draw_trim_kv_pool(cfg: TrimConfig, n_pages: int, device, dtype):
+    """K/V of the whole page pool [P][2][page][D], N(0, 1) drawn with a seeded torch generator
+    on `device` (1M-row slabs, so that no float32 copy of the pool is held at once)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(cfg.seed * 7919 + 0x7A6E)
+    out = torch.empty((n_pages, 2, cfg.page, cfg.D), dtype=dtype, device=device)
+    flat = out.view(-1, cfg.D)
+    step = 1 << 20
+    for a in range(0, flat.shape[0], step):
+        b = min(a + step, flat.shape[0])
+        flat[a:b] = torch.randn((b - a, cfg.D), generator=g, device=device, dtype=torch.float32).to(dtype)
+    return out

@@ -1,0 +1,61 @@
+"""The C-ABI library loads without a GPU and exports exactly the entry points that
+include/qevict.h declares (no compute calls: nothing here needs a device)."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import shutil
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qevict.h")
+
+
+def declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    return sorted(set(re.findall(r"QE_API\s+[\w\s\*]*?\b(qe_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def libpath():
+    from kv_cache_eviction_gqa_b200 import build
+    return build.build()
+
+
+def test_header_declares_the_boundary():
+    names = declared()
+    for must in ("qe_create", "qe_kv_append", "qe_decode_attend_and_score", "qe_route_windows",
+                 "qe_quantize_once", "qe_promote", "qe_vwo_l1norm", "qe_criticalkv_select",
+                 "qe_trim_global_topm", "qe_decode_attend_and_score_noalloc"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(libpath):
+    L = ctypes.CDLL(libpath)
+    missing = [n for n in declared() if not hasattr(L, n)]
+    assert not missing, f"declared but not exported: {missing}"
+
+
+@pytest.mark.skipif(shutil.which("nm") is None, reason="nm not available")
+def test_no_undeclared_exports(libpath):
+    out = subprocess.run(["nm", "-D", "--defined-only", libpath], capture_output=True, text=True,
+                         check=True).stdout
+    exported = sorted({l.split()[-1] for l in out.splitlines() if l.split()[-1].startswith("qe_")})
+    extra = sorted(set(exported) - set(declared()))
+    assert not extra, f"exported but not declared: {extra}"
+
+
+def test_host_side_argument_errors_need_no_device(libpath):
+    from kv_cache_eviction_gqa_b200 import binding as B
+    L = B.lib()
+    assert L.qe_trim_scratch_bytes(0, 10) == 0
+    assert L.qe_trim_scratch_bytes(256, 1536) > 256 * 1536 * 16 * 8
+    # null pointers are rejected before anything touches the device
+    rc = L.qe_trim_global_topm(None, None, None, None, 1, 1, 1, 128, B.QE_BF16, 10, 1, None, None,
+                               None, None, None, None, 0, None)
+    assert rc == B.QE_ERR_INVALID_ARG
+    assert L.qe_strerror(B.QE_ERR_WORKSPACE).decode() == "workspace too small"
