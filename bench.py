@@ -437,6 +437,212 @@ def run_ours(args, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------------------------------
+# secondary rows: CriticalKV selection (c3) and DBTrimKV trim (c4)
+# ---------------------------------------------------------------------------------------
+def measured_tflops():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("bf16_tflops", 1590.0), d.get("bf16_tflops_sustained", 1400.0), "measured"
+    return 1590.0, 1400.0, "fallback"
+
+
+def _timed(fn, steps, flush, stream):
+    """CUDA-event time of each call of fn (L2 flushed before each, outside the event pair)."""
+    import torch
+    ms = []
+    for _ in range(steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        b.synchronize()
+        ms.append(a.elapsed_time(b))
+    return ms
+
+
+def run_c3(args):
+    import torch
+
+    from kv_cache_eviction_gqa_b200 import binding as Bd
+    import oracle as O
+    cfg = W.C3
+    dev = torch.device("cuda", 0)
+    t = torch.bfloat16
+    hbm, _ = measured_peaks()
+    tf_burst, tf_sus, tf_kind = measured_tflops()
+    cpu = None
+    if not args.no_cpu_baseline:
+        K0, V0, q0 = W.draw_critical_unit(cfg, 0, 0)
+        Wo0 = W.draw_critical_w_o(cfg)
+        t0 = time.perf_counter()
+        A0 = O.observation_mass(q0, K0)
+        N0 = O.vwo_l1norm(V0, Wo0, list(range(cfg.G)), cfg.D)
+        O.criticalkv_select(A0, N0, cfg.budget, cfg.alpha)
+        dt = time.perf_counter() - t0
+        per = dt * cfg.B * cfg.Hkv
+        cpu = {"value": 1.0 / per, "unit": "selections/s", "kind": "oracle",
+               "cores": len(os.sched_getaffinity(0)), "blas_threads": blas_threads(),
+               "sample": f"float64 oracle on 1 of {cfg.B * cfg.Hkv} units ({dt:.1f} s), scaled to all units"}
+        del K0, V0, q0, A0, N0
+    Ks, Vs, Qs = [], [], []
+    for b in range(cfg.B):
+        for h in range(cfg.Hkv):
+            K, V, q = W.draw_critical_unit(cfg, b, h)
+            Ks.append(torch.from_numpy(K).to(t))
+            Vs.append(torch.from_numpy(V).to(t))
+            Qs.append(torch.from_numpy(q).to(t))
+    K = torch.stack(Ks).view(cfg.B, cfg.Hkv, cfg.n, cfg.D).to(dev)
+    V = torch.stack(Vs).view(cfg.B, cfg.Hkv, cfg.n, cfg.D).to(dev)
+    q = torch.stack(Qs).view(cfg.B, cfg.Hq, cfg.n_obs, cfg.D).to(dev)
+    Wo = torch.from_numpy(W.draw_critical_w_o(cfg)).to(dev, t)
+    del Ks, Vs, Qs
+    A, N, idx, scratch = Bd.criticalkv_select(q, K, V, Wo, cfg.budget, cfg.alpha)
+    torch.cuda.synchronize()
+    if Bd.trim_status(scratch) != (0, 0):
+        raise RuntimeError("device status after the eager pass")
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    st = torch.cuda.current_stream()
+    call = lambda: Bd.criticalkv_select(q, K, V, Wo, cfg.budget, cfg.alpha, A, N, idx, scratch)
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    with ClockSampler(0) as clk:
+        ms = _timed(call, args.steps, flush, st)
+        vw = _timed(lambda: Bd.vwo_l1norm(V.view(-1, cfg.n, cfg.D), Wo, cfg.Hq, cfg.Hkv, out=N.view(-1, cfg.n, cfg.G)),
+                    args.steps, flush, st)
+    total = sum(ms) / 1e3
+    flops = 2.0 * cfg.B * cfg.Hkv * cfg.n * cfg.D * cfg.G * cfg.hidden
+    vw_s = statistics.mean(vw) / 1e3
+    obs_bytes = 2 * K.numel() * 2 + A.numel() * 4  # K read by both passes, A written
+    # e2e: host K/V/q in pinned memory, copied in; idx copied out
+    Kh, Vh, qh = K.cpu().pin_memory(), V.cpu().pin_memory(), q.cpu().pin_memory()
+    idx_h = torch.empty(idx.shape, dtype=idx.dtype, pin_memory=True)
+    e2e_ms = []
+    for _ in range(min(args.steps, 3)):
+        flush.zero_()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        K.copy_(Kh, non_blocking=True)
+        V.copy_(Vh, non_blocking=True)
+        q.copy_(qh, non_blocking=True)
+        call()
+        idx_h.copy_(idx, non_blocking=True)
+        b.record(st)
+        b.synchronize()
+        e2e_ms.append(a.elapsed_time(b))
+    line = {
+        "metric": "CriticalKV observation-window selections/sec (64K ctx, batch 4, b=2048)",
+        "value": args.steps / total, "unit": "selections/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": sum(ms) / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{cfg.name}: B={cfg.B}, Hq={cfg.Hq}, Hkv={cfg.Hkv}, D={cfg.D}, n={cfg.n}, "
+                               f"n_obs={cfg.n_obs}, budget={cfg.budget}, alpha={cfg.alpha}, hidden={cfg.hidden}, "
+                               "Zipf(1.1) keys",
+                   "l2": "flushed before every step (512 MiB write), outside the timed region"},
+        "roofline": {"kernel": "vwo_tc_kernel (V W_O L1 norms, tcgen05), timed alone through qe_vwo_l1norm",
+                     "bound": "tensor", "achieved": flops / vw_s / 1e12, "peak": tf_burst, "unit": "TFLOP/s",
+                     "frac": flops / vw_s / 1e12 / tf_burst,
+                     "peak_kind": f"{tf_kind} bf16 burst (MEASURED_PEAKS.json bf16_tflops)", "traffic": None,
+                     "flops_per_launch": flops},
+        "secondary": {"vwo_share_of_step": vw_s / (total / args.steps),
+                      "observation_passes_and_selection_ms": (total / args.steps - vw_s) * 1e3,
+                      "observation_pass_hbm_bytes": obs_bytes,
+                      "frac_of_sustained_tensor_peak": flops / vw_s / 1e12 / tf_sus},
+        "cpu_baseline": cpu,
+        "e2e": {"value": len(e2e_ms) / (sum(e2e_ms) / 1e3), "unit": "selections/s",
+                "h2d_bytes_per_step": (K.numel() + V.numel() + q.numel()) * 2,
+                "d2h_bytes_per_step": idx.numel() * 4, "steps": len(e2e_ms)},
+        "clocks": clk.summary(),
+        "gpu_launches": args.steps * 5 + args.steps,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_c4(args):
+    import torch
+
+    from kv_cache_eviction_gqa_b200 import binding as Bd
+    import oracle as O
+    cfg = W.C4
+    dev = torch.device("cuda", 0)
+    hbm, hbm_kind = measured_peaks()
+    lay = W.trim_layout(cfg)
+    cpu = None
+    if not args.no_cpu_baseline:
+        t0 = time.perf_counter()
+        O.trim_global_topm(lay.betas, lay.poss, cfg.t, cfg.M)
+        dt = time.perf_counter() - t0
+        cpu = {"value": 1.0 / dt, "unit": "trims/s", "kind": "oracle", "cores": len(os.sched_getaffinity(0)),
+               "blas_threads": blas_threads(),
+               "sample": f"float64 oracle, one full trim ({dt:.1f} s; selection only, no K/V movement)"}
+    total = int(lay.lengths.sum())
+    beta = torch.from_numpy(lay.beta_pages).to(dev)
+    pos = torch.from_numpy(lay.pos_pages).to(dev)
+    table = torch.from_numpy(lay.page_table).to(dev)
+    lengths = torch.from_numpy(lay.lengths).to(dev)
+    kv = W.draw_trim_kv_pool(cfg, lay.n_pages, dev, torch.bfloat16)
+    kv_out, beta_out, pos_out, new_len, scratch = Bd.trim_global_topm(beta, pos, table, lengths, cfg.t, cfg.M, kv)
+    torch.cuda.synchronize()
+    if Bd.trim_status(scratch) != (0, 0) or int(new_len.sum()) != cfg.M:
+        raise RuntimeError("trim eager pass failed")
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    st = torch.cuda.current_stream()
+    call = lambda: Bd.trim_global_topm(beta, pos, table, lengths, cfg.t, cfg.M, kv, kv_out, beta_out, pos_out,
+                                       new_len, scratch)
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    with ClockSampler(0) as clk:
+        ms = _timed(call, args.steps, flush, st)
+    step_s = sum(ms) / 1e3 / args.steps
+    move = cfg.M * (2 * cfg.D * 2 + 8) * 2  # survivors' K/V rows + beta/pos, read once and written once
+    meta = total * 8  # beta + pos read for the keys
+    alg = move + meta
+    # e2e: inputs from pinned host memory, compacted cache and lengths back
+    hb = [x.cpu().pin_memory() for x in (beta, pos, table, lengths, kv)]
+    ho = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in (kv_out, beta_out, pos_out, new_len)]
+    e2e_ms = []
+    for _ in range(min(args.steps, 3)):
+        flush.zero_()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        for d, h in zip((beta, pos, table, lengths, kv), hb):
+            d.copy_(h, non_blocking=True)
+        call()
+        for h, d in zip(ho, (kv_out, beta_out, pos_out, new_len)):
+            h.copy_(d, non_blocking=True)
+        b.record(st)
+        b.synchronize()
+        e2e_ms.append(a.elapsed_time(b))
+    line = {
+        "metric": "DBTrimKV global top-M trims/sec (256 heads, 4.2M entries, M=1M)",
+        "value": 1.0 / step_s, "unit": "trims/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64 keys, bf16 K/V", "data": "synthetic",
+        "config": {"workload": f"{cfg.name}: {cfg.layers} layers x {cfg.Hkv} heads, lengths U[{cfg.len_lo}, "
+                               f"{cfg.len_hi}] ({total} entries), pages of {cfg.page}, D={cfg.D}, t={cfg.t}, "
+                               f"M={cfg.M}, beta ~ Beta(8, 1)",
+                   "l2": "flushed before every step (512 MiB write), outside the timed region"},
+        "roofline": {"kernel": "whole trim call (init, keygen + 6 radix passes, count, scan, move)",
+                     "bound": "hbm", "achieved": alg / step_s / 1e9, "peak": hbm, "unit": "GB/s",
+                     "frac": alg / step_s / 1e9 / hbm, "peak_kind": f"{hbm_kind} (MEASURED_PEAKS.json hbm_gbs)",
+                     "traffic": None, "algorithmic_bytes": alg},
+        "cpu_baseline": cpu,
+        "e2e": {"value": len(e2e_ms) / (sum(e2e_ms) / 1e3), "unit": "trims/s",
+                "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in hb),
+                "d2h_bytes_per_step": sum(x.numel() * x.element_size() for x in ho), "steps": len(e2e_ms)},
+        "clocks": clk.summary(),
+        "gpu_launches": args.steps * 10,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
@@ -446,6 +652,8 @@ def main():
     ap.add_argument("--max-splits", type=int, default=32)
     ap.add_argument("--e2e-steps", type=int, default=640)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=["c2", "c3", "c4"], default="c2",
+                    help="c2: tiered decode (the default bench); c3: CriticalKV selection; c4: DBTrimKV trim")
     ap.add_argument("--profile-steps", type=int, default=0,
                     help="run only this many eager decode steps after the prefill, then exit")
     args = ap.parse_args()
@@ -456,6 +664,10 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank)
+        return
+    if args.workload != "c2":
+        if rank == 0:
+            (run_c3 if args.workload == "c3" else run_c4)(args)
         return
     if world > 1:
         import datetime

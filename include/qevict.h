@@ -215,14 +215,27 @@ QE_API int qe_vwo_l1norm(const void* V, int n_groups, int rows, int D, int dtype
                          long long out_group_stride, qe_stream_t stream);
 
 /* qe_criticalkv_select - CriticalKV two-stage selection per (batch, kv head) with a
- * SnapKV-style observation window ("Resumo Técnico: CriticalKV", Algoritmo).
- *   q_obs [dev]: [B][Hq][n_obs][D] queries of the last n_obs positions (causal).
- *   K, V [dev]: [B][Hkv][n][D]. W_O [dev]: [Hq*D][hidden].
- *   A_out [dev, float]: [B][Hkv][G][n] observation attention mass per query head.
- *   N_out [dev, float]: [B][Hkv][n][G] ||V_i W_O^h||_1.
- *   idx_out [dev, int32]: [B][Hkv][budget] selected token indices: stage-1 picks in
- *   descending score order, then stage-2 picks in descending score order.
- *   scratch [dev]: qe_criticalkv_scratch_bytes() bytes. */
+ * SnapKV-style observation window ("Resumo Técnico: CriticalKV", Algoritmo, Etapas 1 e 2;
+ * Framework Teórico for the projected values V W_O).
+ * Per unit (b, kvh) with query heads h = kvh*G .. kvh*G+G-1 (G = Hq/Hkv):
+ *   A[h][i] = sum_j softmax_i(q_(h,j) . K_i / sqrt(D)), query j at position n - n_obs + j seeing
+ *             keys 0 .. n - n_obs + j (causal);
+ *   N[i][h] = || V_i W_O^h ||_1, W_O^h = rows h*D .. h*D+D-1 of W_O;
+ *   a_i = sum_h A[h][i], p_i = sum_h A[h][i] N[i][h] (float32);
+ *   stage 1 keeps floor(alpha * budget) entries of highest a, stage 2 the remaining budget
+ *   entries of highest p among the rest; equal scores go to the lower index.
+ *   q_obs [dev]: [B][Hq][n_obs][D] queries of the last n_obs positions.
+ *   K, V [dev]: [B][Hkv][n][D]. W_O [dev]: [Hq*D][hidden]. All of one dtype, 16-byte aligned.
+ *   A_out [dev, float]: [B][Hkv][G][n].  N_out [dev, float]: [B][Hkv][n][G].
+ *   idx_out [dev, int32]: [B][Hkv][budget]: stage-1 picks in descending a, then stage-2 picks in
+ *   descending p. When n <= budget every entry is kept: idx_out = 0..n-1, then -1.
+ *   scratch [dev]: qe_criticalkv_scratch_bytes() bytes, 256-byte aligned, owned by the caller;
+ *   its first 8 bytes receive a status word {int32 code, int32 detail}: 0, or QE_ERR_TIMEOUT if a
+ *   bounded wait inside a tensor-core kernel gave up. Read it after synchronising.
+ * Supported: D in {64, 128}; n_obs in {32, 64} with G * n_obs <= 128 and n_obs <= n;
+ * budget <= 8192; hidden a multiple of 64 (tensor cores when a multiple of 128); alpha in
+ * [0, 1]. Otherwise QE_ERR_UNSUPPORTED_SHAPE / QE_ERR_INVALID_ARG, nothing launched.
+ * Asynchronous on `stream`; allocates nothing. */
 QE_API size_t qe_criticalkv_scratch_bytes(int B, int Hq, int Hkv, int n, int n_obs);
 QE_API int qe_criticalkv_select(const void* q_obs, int n_obs, const void* K, const void* V,
                                 const void* W_O, int B, int Hq, int Hkv, int n, int D,

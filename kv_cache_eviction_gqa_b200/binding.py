@@ -360,3 +360,36 @@ def trim_status(scratch: torch.Tensor):
     """(code, detail) of the device status word a trim call left in its scratch."""
     w = scratch[:8].view(torch.int32).cpu()
     return int(w[0]), int(w[1])
+
+
+def criticalkv_select(q_obs: torch.Tensor, K: torch.Tensor, V: torch.Tensor, W_O: torch.Tensor,
+                      budget: int, alpha: float = 0.5, A=None, N=None, idx=None, scratch=None,
+                      stream=None):
+    """CriticalKV two-stage selection with an observation window (qe_criticalkv_select).
+
+    q_obs [B][Hq][n_obs][D], K and V [B][Hkv][n][D], W_O [Hq*D][hidden], all one cache dtype.
+    Returns (A [B][Hkv][G][n] fp32, N [B][Hkv][n][G] fp32, idx [B][Hkv][budget] int32, scratch);
+    the device status word is scratch[:8] (see trim_status).
+    """
+    _need(q_obs, "q_obs")
+    B, Hq, n_obs, D = q_obs.shape
+    _need(K, "K", q_obs.dtype)
+    _, Hkv, n, _ = K.shape
+    _need(V, "V", q_obs.dtype, K.shape)
+    _need(W_O, "W_O", q_obs.dtype)
+    G = Hq // Hkv
+    dev = K.device
+    A = torch.empty((B, Hkv, G, n), dtype=torch.float32, device=dev) if A is None else A
+    N = torch.empty((B, Hkv, n, G), dtype=torch.float32, device=dev) if N is None else N
+    idx = torch.empty((B, Hkv, budget), dtype=torch.int32, device=dev) if idx is None else idx
+    _need(A, "A", torch.float32, (B, Hkv, G, n))
+    _need(N, "N", torch.float32, (B, Hkv, n, G))
+    _need(idx, "idx", torch.int32, (B, Hkv, budget))
+    nbytes = int(lib().qe_criticalkv_scratch_bytes(B, Hq, Hkv, n, n_obs))
+    if scratch is None:
+        scratch = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    _check(lib().qe_criticalkv_select(_ptr(q_obs), n_obs, _ptr(K), _ptr(V), _ptr(W_O), B, Hq, Hkv, n, D,
+                                      W_O.shape[1], dtype_code(K.dtype), budget, float(alpha), _ptr(A),
+                                      _ptr(N), _ptr(idx), _ptr(scratch), scratch.numel(),
+                                      _stream(stream)), "qe_criticalkv_select")
+    return A, N, idx, scratch
