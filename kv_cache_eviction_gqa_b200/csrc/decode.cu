@@ -45,21 +45,22 @@
 namespace {
 
 #ifndef QE_DECODE_NW
-#define QE_DECODE_NW 4
+#define QE_DECODE_NW 2
 #endif
 #ifndef QE_DECODE_NST
 #define QE_DECODE_NST 3
 #endif
 #ifndef QE_DECODE_MINB
-#define QE_DECODE_MINB 2
+#define QE_DECODE_MINB 4
+#endif
+#ifndef QE_DECODE_DPL4
+#define QE_DECODE_DPL4 16
 #endif
 #ifndef QE_DECODE_SB
 #define QE_DECODE_SB 4
 #endif
-#ifndef QE_DECODE_WAVES
-#define QE_DECODE_WAVES 1
-#endif
 constexpr int kNW = QE_DECODE_NW;    // warps per CTA
+#define QE_MAX_SPLITS_CLUSTER 16          // CTAs per unit (one cluster, non-portable size)
 constexpr int kNST = QE_DECODE_NST;  // stages per warp
 constexpr float kRescale = 8.f;  // rescale the accumulators when the max grows by > 2^8
 
@@ -67,24 +68,43 @@ struct DecodeArgs {
   DevState st;
   const void* q;     // [B][Hq][D]
   float* out;        // [B][Hq][D]
-  float* split_part; // [U][max_splits][G][D + 2]
   float* win_part;   // [U][Wmax][G][4]
   float* tail_s;     // [U][window][G]
-  uint32_t* tickets; // [U]
-  int splits, max_splits;
+  int splits;        // CTAs per unit = cluster size
   int tail_win, tail_len;
   float scale_log2;  // log2(e) / sqrt(D)
 };
 
 template <int D, int G>
 struct Map {
-  static constexpr int DPL = G <= 4 ? 16 : 8;  // head-dim elements per lane
+  static constexpr int DPL = G <= 4 ? QE_DECODE_DPL4 : 8;  // head-dim elements per lane
   static constexpr int LPT = D / DPL;          // lanes per token
   static constexpr int TPS = 32 / LPT;         // tokens per warp step
   static constexpr int SB = (16 / TPS) < QE_DECODE_SB ? (16 / TPS) : QE_DECODE_SB;  // tokens per group per batch
   static constexpr int SBT = SB * TPS;         // tokens per batch (divides 16)
   static constexpr int NP = DPL / 2;           // float pairs per lane
 };
+
+// 2^x with the hardware approximation (relative error about 2^-22; results below 2^-126
+// flush to zero, which no sum here can notice).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// thread-block cluster helpers: barrier over the cluster's CTAs, and a load from the shared
+// memory of CTA `rank` of the cluster at the address of a local shared variable
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ float ld_cluster(const float* local, uint32_t rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(local)), "r"(rank));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+  return v;
+}
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -123,25 +143,29 @@ __device__ __forceinline__ void load_row(const T* row, int sub, int sw, float2 (
   }
 }
 
-// x = 1 + c/4 for the 2-bit code c in bits 2E..2E+1 of `bits`
+// Codes E (even) and E+1 from one shift: the pair {4 + c_E/4, 1 + c_(E+1)/4}. Code E lands in
+// mantissa bits 19-20 of 4.0 (4 * (1 + c/16)) and code E+1 in bits 21-22 of 1.0, so both
+// values are exact and the code's contribution is c/4 in either case; only the constant part
+// differs (4 for even elements, 1 for odd ones).
 template <int E>
-__device__ __forceinline__ float code_x(uint32_t bits) {
-  constexpr int sh = 21 - 2 * E;
+__device__ __forceinline__ float2 code_pair(uint32_t bits) {
+  constexpr int sh = 19 - 2 * E;
   const uint32_t v = sh >= 0 ? (bits << (sh >= 0 ? sh : 0)) : (bits >> (sh < 0 ? -sh : 0));
-  return __uint_as_float((v & 0x00600000u) | 0x3f800000u);
+  return make_float2(__uint_as_float((v & 0x00180000u) | 0x40800000u),
+                     __uint_as_float((v & 0x00600000u) | 0x3f800000u));
 }
 
 template <int NP>
 __device__ __forceinline__ void decode_codes(uint32_t bits, float2 (&x)[NP]) {
-  x[0] = make_float2(code_x<0>(bits), code_x<1>(bits));
-  x[1] = make_float2(code_x<2>(bits), code_x<3>(bits));
-  x[2] = make_float2(code_x<4>(bits), code_x<5>(bits));
-  x[3] = make_float2(code_x<6>(bits), code_x<7>(bits));
+  x[0] = code_pair<0>(bits);
+  x[1] = code_pair<2>(bits);
+  x[2] = code_pair<4>(bits);
+  x[3] = code_pair<6>(bits);
   if constexpr (NP == 8) {
-    x[4] = make_float2(code_x<8>(bits), code_x<9>(bits));
-    x[5] = make_float2(code_x<10>(bits), code_x<11>(bits));
-    x[6] = make_float2(code_x<12>(bits), code_x<13>(bits));
-    x[7] = make_float2(code_x<14>(bits), code_x<15>(bits));
+    x[4] = code_pair<8>(bits);
+    x[5] = code_pair<10>(bits);
+    x[6] = code_pair<12>(bits);
+    x[7] = code_pair<14>(bits);
   }
 }
 
@@ -193,7 +217,8 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB) decode_kernel(Decode
 
   // the G query heads of this group, this lane's DPL elements, in the log2 domain
   float2 q[G][NP];
-  float qsum[G];
+  float qsum[G];   // sum of the lane's q elements
+  float qsum2[G];  // 4 * (sum over even elements) + (sum over odd elements): the constant part of q . x
   {
     const T* qb = reinterpret_cast<const T*>(a.q) + ((size_t)b * st.Hq + (size_t)kvh * G) * D;
     const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
@@ -207,14 +232,16 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB) decode_kernel(Decode
         s2 = __fadd2_rn(s2, q[h][e]);
       }
       qsum[h] = s2.x + s2.y;
+      qsum2[h] = fmaf(4.f, s2.x, s2.y);
     }
   }
   // per lane-group online-softmax state; lw/nw: sums of the current window
   float2 acc[G][NP];
-  float zacc[G], m[G], lsum[G], lw[G], nw[G];
+  float2 zacc[G];  // INT2 value offsets (even, odd element) weighted by p * ...
+  float m[G], lsum[G], lw[G], nw[G];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
-    zacc[h] = 0.f;
+    zacc[h] = make_float2(0.f, 0.f);
     m[h] = -1e30f;
     lsum[h] = 0.f;
     lw[h] = 0.f;
@@ -323,11 +350,11 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB) decode_kernel(Decode
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         const float mn = mb[h] > m[h] + kRescale ? mb[h] : m[h];
-        const float f = exp2f(m[h] - mn);
+        const float f = ex2(m[h] - mn);
         const float2 f2 = make_float2(f, f);
 #pragma unroll
         for (int e = 0; e < NP; ++e) acc[h][e] = __fmul2_rn(acc[h][e], f2);
-        zacc[h] *= f;
+        zacc[h] = __fmul2_rn(zacc[h], f2);
         lsum[h] *= f;
         lw[h] *= f;
         nw[h] *= f;
@@ -337,7 +364,7 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB) decode_kernel(Decode
 #pragma unroll
     for (int i = 0; i < SB; ++i)
 #pragma unroll
-      for (int h = 0; h < G; ++h) s[i][h] = exp2f(s[i][h] - m[h]);
+      for (int h = 0; h < G; ++h) s[i][h] = ex2(s[i][h] - m[h]);
   };
 
   // sum every score over the LPT lanes of its token (pairs of heads added as f32x2)
@@ -496,18 +523,20 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB) decode_kernel(Decode
           float2 x[NP];
           decode_codes<NP>(load_codes<DPL>(kc + t * (D / 4), sub, sw), x);
           const uint32_t mt = km[t * (D / 16) + gi];
-          const float s4 = 4.f * meta_scale(mt), zz = meta_zero(mt) - s4;
+          const float s4 = 4.f * meta_scale(mt), z = meta_zero(mt);
           float d[G];
           qk_row(x, d);
-          // score = 4s * (q . x) + (z - 4s) * sum(q)
+          // q . x = qsum2 + (q . c) / 4, so q . k = s (q . c) + z qsum = 4s (q . x) + z qsum - 4s qsum2
 #pragma unroll
           for (int h = 0; h + 1 < G; h += 2) {
-            const float2 r = ffma2(make_float2(s4, s4), make_float2(d[h], d[h + 1]),
-                                   __fmul2_rn(make_float2(zz, zz), make_float2(qsum[h], qsum[h + 1])));
+            const float2 c0 = ffma2(make_float2(z, z), make_float2(qsum[h], qsum[h + 1]),
+                                    __fmul2_rn(make_float2(-s4, -s4), make_float2(qsum2[h], qsum2[h + 1])));
+            const float2 r = ffma2(make_float2(s4, s4), make_float2(d[h], d[h + 1]), c0);
             sc[i][h] = r.x;
             sc[i][h + 1] = r.y;
           }
-          if constexpr (G % 2) sc[i][G - 1] = fmaf(s4, d[G - 1], zz * qsum[G - 1]);
+          if constexpr (G % 2)
+            sc[i][G - 1] = fmaf(s4, d[G - 1], fmaf(z, qsum[G - 1], -s4 * qsum2[G - 1]));
         }
         butterfly(sc);
         online(sc);
@@ -518,13 +547,15 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB) decode_kernel(Decode
           float2 x[NP];
           decode_codes<NP>(load_codes<DPL>(vc + t * (D / 4), sub, sw), x);
           const uint32_t mt = vm[t * (D / 16) + gi];
-          const float s4 = 4.f * meta_scale(mt), zz = meta_zero(mt) - s4;
-          // v = 4s * x + (z - 4s): acc += (p*4s) * x, zacc += p * (z - 4s)
+          const float s4 = 4.f * meta_scale(mt), z = meta_zero(mt);
+          // v = 4s * x + (z - 16s) for even elements (x = 4 + c/4), 4s * x + (z - 4s) for odd
+          // ones (x = 1 + c/4): acc += (p * 4s) * x, zacc += p * (z - 16s, z - 4s)
+          const float2 zz = make_float2(fmaf(-4.f, s4, z), z - s4);
           float ps[G];
 #pragma unroll
           for (int h = 0; h < G; ++h) {
             ps[h] = sc[i][h] * s4;
-            zacc[h] = fmaf(sc[i][h], zz, zacc[h]);
+            zacc[h] = ffma2(make_float2(sc[i][h], sc[i][h]), zz, zacc[h]);
           }
           pv_row(x, ps);
         }
@@ -539,7 +570,7 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB) decode_kernel(Decode
           float mx = m[h];
 #pragma unroll
           for (int o = LPT; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-          const float f = exp2f(m[h] - mx);
+          const float f = ex2(m[h] - mx);
           float l2 = lw[h] * f, n2 = nw[h] * f;
 #pragma unroll
           for (int o = LPT; o < 32; o <<= 1) {
@@ -568,17 +599,17 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB) decode_kernel(Decode
     for (; k < issued; ++k) mbar_wait_bounded(&bars[k % kNST], (k / kNST) & 1, st.status, 2000 + u);
   }
 
-  // ---- merge lane groups, then warps, into one split partial ----
+  // ---- merge lane groups, then warps, into the CTA's partial ----
 #pragma unroll
   for (int h = 0; h < G; ++h) {
     float mx = m[h];
 #pragma unroll
     for (int o = LPT; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    const float f = exp2f(m[h] - mx);
+    const float f = ex2(m[h] - mx);
     lsum[h] *= f;
-    const float2 z2 = make_float2(zacc[h], zacc[h]), f2 = make_float2(f, f);
+    const float2 f2 = make_float2(f, f);
 #pragma unroll
-    for (int e = 0; e < NP; ++e) acc[h][e] = __fmul2_rn(__fadd2_rn(acc[h][e], z2), f2);
+    for (int e = 0; e < NP; ++e) acc[h][e] = __fmul2_rn(__fadd2_rn(acc[h][e], zacc[h]), f2);
 #pragma unroll
     for (int o = LPT; o < 32; o <<= 1) {
       lsum[h] += __shfl_xor_sync(0xffffffffu, lsum[h], o);
@@ -594,6 +625,15 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB) decode_kernel(Decode
   float* mw = reinterpret_cast<float*>(smem);  // [kNW][G]
   float* lwv = mw + kNW * G;                   // [kNW][G]
   float* aw = lwv + kNW * G;                   // [kNW][G][D]
+  float* cm = aw + kNW * G * D;                // [G]     CTA partial: max,
+  float* cl = cm + QE_MAX_G;                   // [G]     sum of weights,
+  float* ca = cl + QE_MAX_G;                   // [G][D]  weighted values (read by the cluster)
+  float* pm = ca + G * D;                      // [S][G]  every CTA's max,
+  float* pl = pm + QE_MAX_SPLITS_CLUSTER * QE_MAX_G;  // [S][G] sum of weights,
+  float* pf = pl + QE_MAX_SPLITS_CLUSTER * QE_MAX_G;  // [S][G] and rescale factor
+  float* gl = pf + QE_MAX_SPLITS_CLUSTER * QE_MAX_G;  // [G] unit sum of weights
+  float* lse = gl + QE_MAX_G;                         // [G] unit log2-sum-exp
+  float* red = lse + QE_MAX_G;                        // [kNW]
   if (lane < LPT) {
 #pragma unroll
     for (int h = 0; h < G; ++h) {
@@ -611,94 +651,93 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB) decode_kernel(Decode
     }
   }
   __syncthreads();
-  float* sp = a.split_part + ((size_t)u * a.max_splits + split) * G * (D + 2);
   for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
-    const int h = i / D, d = i % D;
-    float Mx = -INFINITY;
-    for (int x = 0; x < kNW; ++x) Mx = fmaxf(Mx, mw[x * G + h]);
+    const int h = i / D;
+    float Mx = mw[h];
+#pragma unroll
+    for (int x = 1; x < kNW; ++x) Mx = fmaxf(Mx, mw[x * G + h]);
     float L = 0.f, A = 0.f;
-    if (Mx != -INFINITY) {
-      for (int x = 0; x < kNW; ++x) {
-        const float mm = mw[x * G + h];
-        const float f = mm == -INFINITY ? 0.f : exp2f(mm - Mx);
-        L += lwv[x * G + h] * f;
-        A += aw[((size_t)x * G + h) * D + d] * f;
-      }
+#pragma unroll
+    for (int x = 0; x < kNW; ++x) {
+      const float f = ex2(mw[x * G + h] - Mx);
+      L = fmaf(lwv[x * G + h], f, L);
+      A = fmaf(aw[((size_t)x * G + h) * D + i % D], f, A);
     }
-    sp[h * (D + 2) + 2 + d] = A;
-    if (d == 0) {
-      sp[h * (D + 2) + 0] = Mx;
-      sp[h * (D + 2) + 1] = L;
+    ca[i] = A;
+    if (i % D == 0) {
+      cm[h] = Mx;
+      cl[h] = L;
     }
   }
 
-  // ---- the last CTA of the unit combines ----
-  __shared__ int s_last;
-  __threadfence();
+  // ---- the unit's S CTAs form one cluster: merge the partials through distributed
+  // shared memory; each CTA writes its share of the output and the scores of its windows ----
+  const int S = a.splits;
+  cluster_sync();
+  for (int i = threadIdx.x; i < S * G; i += blockDim.x) {
+    pm[i] = ld_cluster(cm + i % G, (uint32_t)(i / G));
+    pl[i] = ld_cluster(cl + i % G, (uint32_t)(i / G));
+  }
   __syncthreads();
-  if (threadIdx.x == 0) s_last = atomicAdd(&a.tickets[u], 1u) == (unsigned)(a.splits - 1);
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  float* lse = reinterpret_cast<float*>(smem);  // [8]
-  float* red = lse + QE_MAX_G;                  // [32]
-  const float* sp0 = a.split_part + (size_t)u * a.max_splits * G * (D + 2);
   if (threadIdx.x < G) {
     const int h = threadIdx.x;
-    float Mx = -INFINITY;
-    for (int x = 0; x < a.splits; ++x) Mx = fmaxf(Mx, __ldcg(sp0 + (x * G + h) * (D + 2)));
+    float M = pm[h];
+    for (int r = 1; r < S; ++r) M = fmaxf(M, pm[r * G + h]);
     float L = 0.f;
-    for (int x = 0; x < a.splits; ++x) {
-      const float mx = __ldcg(sp0 + (x * G + h) * (D + 2));
-      if (mx != -INFINITY) L += __ldcg(sp0 + (x * G + h) * (D + 2) + 1) * exp2f(mx - Mx);
+    for (int r = 0; r < S; ++r) {
+      const float f = ex2(pm[r * G + h] - M);
+      pf[r * G + h] = f;
+      L = fmaf(pl[r * G + h], f, L);
     }
-    lse[h] = Mx + log2f(L);
-    red[h] = Mx;
-    red[8 + h] = L;
+    gl[h] = L;
+    lse[h] = M + log2f(L);
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
-    const int h = i / D, d = i % D;
-    const float Mx = red[h], L = red[8 + h];
-    float A = 0.f;
-    for (int x = 0; x < a.splits; ++x) {
-      const float mx = __ldcg(sp0 + (x * G + h) * (D + 2));
-      if (mx != -INFINITY) A += __ldcg(sp0 + (x * G + h) * (D + 2) + 2 + d) * exp2f(mx - Mx);
+  {
+    const int per = (G * D + S - 1) / S;
+    const int i1 = min((split + 1) * per, G * D);
+    for (int i = split * per + threadIdx.x; i < i1; i += blockDim.x) {
+      const int h = i / D;
+      float A = 0.f;
+      for (int r = 0; r < S; ++r) A = fmaf(ld_cluster(ca + i, (uint32_t)r), pf[r * G + h], A);
+      a.out[((size_t)b * st.Hq + (size_t)kvh * G + h) * D + i % D] = A / gl[h];
     }
-    a.out[((size_t)b * st.Hq + (size_t)kvh * G + h) * D + d] = A / L;
   }
-  // exact per-window attention mass and perturbation of this step
-  for (int jj = threadIdx.x; jj < nf + nq; jj += blockDim.x) {
-    const int win = jj < nf ? st.full_list[ub + jj] : st.int2_list[ub + jj - nf];
+  // exact attention mass and perturbation of this step for the windows this CTA streamed
+  for (int jj = threadIdx.x; jj < nF + nQ; jj += blockDim.x) {
+    const int li = list_idx(jj);
+    const int win = jj < nF ? st.full_list[ub + li] : st.int2_list[ub + li - nf];
     if (win < 0 || win >= st.Wmax) continue;
     float dm = 0.f, dp = 0.f;
-    const float* wp = a.win_part + (ub + jj) * G * 4;
+    const float* wp = a.win_part + (ub + li) * G * 4;
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      const float f = exp2f(__ldcg(wp + h * 4 + 0) - lse[h]);
-      dm = fmaf(__ldcg(wp + h * 4 + 1), f, dm);
-      dp = fmaf(__ldcg(wp + h * 4 + 2), f, dp);
+      const float f = ex2(wp[h * 4 + 0] - lse[h]);
+      dm = fmaf(wp[h * 4 + 1], f, dm);
+      dp = fmaf(wp[h * 4 + 2], f, dp);
     }
     st.mass[ub + win] += dm;
     st.pert[ub + win] += dp;
   }
-  // tail tokens: cumulative per-token attention and the window's mass
-  float tm = 0.f;
-  for (int i = threadIdx.x; i < a.tail_len * G; i += blockDim.x) {
-    const int h = i % G;
-    const float pv = exp2f(__ldcg(a.tail_s + (size_t)u * w * G + i) - lse[h]);
-    st.tail_p[(size_t)u * w * G + i] += pv;
-    tm += pv;
+  // tail tokens (last CTA of the cluster): cumulative per-token attention and window mass
+  if (has_tail) {
+    float tm = 0.f;
+    for (int i = threadIdx.x; i < a.tail_len * G; i += blockDim.x) {
+      const int h = i % G;
+      const float pv = ex2(a.tail_s[(size_t)u * w * G + i] - lse[h]);
+      st.tail_p[(size_t)u * w * G + i] += pv;
+      tm += pv;
+    }
+    tm = warp_sum(tm);
+    if (lane == 0) red[warp] = tm;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float s2 = 0.f;
+      for (int x = 0; x < kNW; ++x) s2 += red[x];
+      st.mass[ub + a.tail_win] += s2;
+    }
   }
-  tm = warp_sum(tm);
-  if (lane == 0) red[16 + warp] = tm;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float s = 0.f;
-    for (int x = 0; x < kNW; ++x) s += red[16 + x];
-    if (a.tail_len > 0) st.mass[ub + a.tail_win] += s;
-    a.tickets[u] = 0;
-  }
+  cluster_sync();  // keep this CTA's partial alive until every CTA of the cluster has read it
 }
 
 template <typename T, int D, int G>
@@ -706,40 +745,72 @@ int launch_decode_t(qe_ctx* c, const void* q, float* out, cudaStream_t s) {
   constexpr int PAGE_BYTES = 2 * QE_PAGE * D * 2;
   constexpr int STAGE = PAGE_BYTES + 64 * G * 4;
   const size_t smem = (size_t)kNW * kNST * STAGE + kNW * kNST * 8;
-  static_assert((size_t)kNW * G * (D + 2) * 4 <= (size_t)kNW * kNST * STAGE, "merge area");
+  static_assert((size_t)(kNW * G * (D + 2) + 2 * QE_MAX_G + G * D + 3 * QE_MAX_SPLITS_CLUSTER * QE_MAX_G +
+                         2 * QE_MAX_G + kNW) * 4 <= (size_t)kNW * kNST * STAGE,
+                "merge area");
   auto kern = decode_kernel<T, D, G>;
-  // one-time set-up per instantiation (kept out of the per-step path and of graph capture)
-  static int per_sm = 0, sms = 0;
-  if (per_sm == 0) {
-    int dev = 0;
+  // One-time set-up per instantiation (kept out of the per-step path and of graph capture):
+  // clusters[S] = how many clusters of S CTAs can be resident at once.
+  static int clusters[QE_MAX_SPLITS_CLUSTER + 1] = {0};
+  static bool ready = false;
+  if (!ready) {
     QE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    QE_CUDA_TRY(cudaGetDevice(&dev));
-    QE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-    QE_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kNW * 32, smem));
-    if (per_sm < 1) per_sm = 1;
+    QE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+    for (int S = 1; S <= QE_MAX_SPLITS_CLUSTER; ++S) {
+      cudaLaunchConfig_t qc = {};
+      cudaLaunchAttribute qa[1];
+      qa[0].id = cudaLaunchAttributeClusterDimension;
+      qa[0].val.clusterDim.x = S;
+      qa[0].val.clusterDim.y = 1;
+      qa[0].val.clusterDim.z = 1;
+      qc.gridDim = dim3(S);
+      qc.blockDim = dim3(kNW * 32);
+      qc.dynamicSmemBytes = smem;
+      qc.attrs = qa;
+      qc.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &qc) != cudaSuccess) {
+        (void)cudaGetLastError();
+        n = 0;
+      }
+      clusters[S] = n;
+    }
+    ready = true;
   }
   DecodeArgs a{};
   a.st = make_state(c);
   a.q = q;
   a.out = out;
-  a.split_part = c->split_part;
   a.win_part = c->win_part;
   a.tail_s = c->tail_s;
-  a.tickets = c->tickets;
-  a.max_splits = c->cfg.max_splits;
   a.tail_win = c->complete;
   a.tail_len = c->n - c->complete * c->cfg.window;
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
   const int U = c->lay.units;
-  // one wave of resident CTAs; never more splits than windows per tier
+  // The largest split count whose U clusters are all resident in one wave, never more splits
+  // than windows per tier nor than the configured maximum.
   const int nwin = c->n_full_max > c->n_int2_max ? c->n_full_max : c->n_int2_max;
-  int S = QE_DECODE_WAVES * per_sm * sms / U;
-  if (S > nwin) S = nwin;
-  if (S > c->cfg.max_splits) S = c->cfg.max_splits;
-  if (S < 1) S = 1;
+  int S = 1;
+  for (int t = QE_MAX_SPLITS_CLUSTER; t >= 1; --t)
+    if (clusters[t] >= U && t <= nwin && t <= c->cfg.max_splits) {
+      S = t;
+      break;
+    }
   a.splits = S;
-  kern<<<U * S, kNW * 32, smem, s>>>(a);
-  return cudaGetLastError() == cudaSuccess ? QE_OK : QE_ERR_CUDA;
+  cudaLaunchConfig_t lc = {};
+  cudaLaunchAttribute la[1];
+  la[0].id = cudaLaunchAttributeClusterDimension;
+  la[0].val.clusterDim.x = S;
+  la[0].val.clusterDim.y = 1;
+  la[0].val.clusterDim.z = 1;
+  lc.gridDim = dim3(U * S);
+  lc.blockDim = dim3(kNW * 32);
+  lc.dynamicSmemBytes = smem;
+  lc.stream = s;
+  lc.attrs = la;
+  lc.numAttrs = 1;
+  QE_CUDA_TRY(cudaLaunchKernelEx(&lc, kern, a));
+  return QE_OK;
 }
 
 template <typename T, int D>

@@ -125,6 +125,13 @@ __global__ void append_kernel(DevState st, const uint4* k_new, const uint4* v_ne
                               uint4* tailV) {
   const int u = blockIdx.x, b = u / st.Hkv, kvh = u % st.Hkv;
   const int w = st.window, tw = pos / w, t = pos % w, pg = t / QE_PAGE, r = pos % QE_PAGE;
+  const int vpr = st.D * 2 / 16;
+  // the new rows do not depend on the page lookup: load them first
+  uint4 kv = make_uint4(0, 0, 0, 0), vv = kv;
+  if (threadIdx.x < vpr) {
+    kv = k_new[(size_t)u * vpr + threadIdx.x];
+    vv = v_new[(size_t)u * vpr + threadIdx.x];
+  }
   __shared__ int s_page;
   if (threadIdx.x == 0) {
     const size_t wi = (size_t)u * st.Wmax + tw;
@@ -158,10 +165,9 @@ __global__ void append_kernel(DevState st, const uint4* k_new, const uint4* v_ne
     for (int i = threadIdx.x; i < w * st.G; i += blockDim.x) st.tail_p[(size_t)u * w * st.G + i] = 0.f;
   const int page = s_page;
   if (page < 0) return;
-  const int vpr = st.D * 2 / 16;
   uint4* base = reinterpret_cast<uint4*>(st.pages + ((size_t)u * st.P + page) * st.page_bytes);
-  for (int c = threadIdx.x; c < vpr; c += blockDim.x) {
-    const uint4 kv = k_new[(size_t)u * vpr + c], vv = v_new[(size_t)u * vpr + c];
+  if (threadIdx.x < vpr) {
+    const int c = threadIdx.x;
     base[r * vpr + c] = kv;
     base[(QE_PAGE + r) * vpr + c] = vv;
     tailV[(((size_t)kvh * st.B + b) * w + t) * vpr + c] = vv;
