@@ -39,6 +39,10 @@ from kv_cache_eviction_gqa_b200 import workloads as W  # noqa: E402
 METRIC = "decode attn+routing steps/sec; achieved HBM GB/s vs peak at 32K ctx, batch 8"
 CFG = W.C2
 FALLBACK_HBM_GBS = 6650.0
+# DRAM read + write of one steady decode launch (decode step 2 of the sequence) from an ncu
+# capture of the current decode kernel (profiles/decode_kernel_c2_llama8b_32k_b8.md); set to
+# None whenever the kernel changes until it is captured again.
+DECODE_TRAFFIC_BYTES = 109.679872e6 + 3.514368e6
 
 
 def measured_peaks():
@@ -458,7 +462,9 @@ def run_ours(args, rank, world, local_rank):
             "roofline": {"kernel": "decode_kernel (split-K GQA decode + window scoring)",
                          "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
-                         "traffic": None, "launches_counted": n_l,
+                         "traffic": DECODE_TRAFFIC_BYTES, "launches_counted": n_l,
+                         "traffic_launch": "decode step 2 (steady), ncu dram__bytes_read.sum + write.sum",
+                         "algorithmic_bytes_traffic_launch": decode_bytes(cfg, *meta[2 % S][:3]),
                          "bytes_per_launch_avg": b_sum / max(n_l, 1)},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": h2d,
