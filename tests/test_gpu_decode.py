@@ -40,6 +40,24 @@ def test_small_sequences(cfg):
     print(rep)
 
 
+# full sizes, in the launch configuration the bench uses; the oracle follows sampled units
+@pytest.mark.slow
+def test_c2_full_size_sampled_units():
+    cfg = W.C2
+    units = [0, cfg.units - 1]
+    rep = run_decode_parity(cfg, check_units=units)
+    assert rep.steps == cfg.steps and rep.route_events == 4 * len(units) and rep.codes_checked > 0
+    print(rep)
+
+
+@pytest.mark.slow
+def test_c5_full_size_sampled_unit():
+    cfg = W.C5
+    rep = run_decode_parity(cfg, check_units=[3], steps=80)
+    assert rep.steps == 80 and rep.route_events == 5 and rep.codes_checked > 0
+    print(rep)
+
+
 @pytest.mark.parametrize("splits", [1, 3, 64])
 def test_split_counts_agree(splits):
     cfg = SMALL[0].scaled(steps=9)
