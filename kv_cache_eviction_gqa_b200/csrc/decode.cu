@@ -41,6 +41,7 @@
 
 #include "int2.cuh"
 #include "qe_internal.cuh"
+#include "tc_common.cuh"
 
 namespace {
 
@@ -52,6 +53,9 @@ namespace {
 #endif
 #ifndef QE_DECODE_MINB
 #define QE_DECODE_MINB 4
+#endif
+#ifndef QE_DECODE_FULL_LAST
+#define QE_DECODE_FULL_LAST 0  // 1: odd warps stream their full-precision windows last
 #endif
 #ifndef QE_DECODE_DPL4
 #define QE_DECODE_DPL4 16
@@ -182,14 +186,80 @@ __device__ __forceinline__ uint32_t load_codes(const uint8_t* row, int sub, int 
 
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
+// ---- warp-level tensor-core helpers (m16n8k16, 16-bit inputs, f32 accumulate) ----
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(p)));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(p)));
+}
+template <typename T> struct MmaOp;
+template <> struct MmaOp<__nv_bfloat16> {
+  static __device__ __forceinline__ void run(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                             uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  }
+  // {lo, hi} 16-bit pair of (x, y) (x in the low half), and the residual pair
+  static __device__ __forceinline__ void split(float x, float y, uint32_t& hi, uint32_t& lo) {
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(hi) : "f"(y), "f"(x));
+    const float xr = x - __uint_as_float(hi << 16), yr = y - __uint_as_float(hi & 0xffff0000u);
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(lo) : "f"(yr), "f"(xr));
+  }
+};
+template <> struct MmaOp<__half> {
+  static __device__ __forceinline__ void run(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                             uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  }
+  static __device__ __forceinline__ void split(float x, float y, uint32_t& hi, uint32_t& lo) {
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(hi) : "f"(y), "f"(x));
+    const float xr = x - __half2float(__ushort_as_half(static_cast<unsigned short>(hi & 0xffffu)));
+    const float yr = y - __half2float(__ushort_as_half(static_cast<unsigned short>(hi >> 16)));
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(lo) : "f"(yr), "f"(xr));
+  }
+};
+
+// Shared-memory stage of one task (1024-byte aligned). A full-precision page arrives as TMA
+// boxes of 16 rows x 64 elements with the 128-byte swizzle (box (part, x) at
+// (part * D/64 + x) * 2048, part 0 = K rows, 1 = V rows), so the 8 rows of every ldmatrix
+// tile sit in distinct banks; tail pages and INT2 ledger entries are 1-D bulk copies in their
+// contiguous layout. Up to 64 tokens' norms follow at PAGE_BYTES.
+template <int D, int G>
+struct StageLayout {
+  static constexpr int PAGE_BYTES = 2 * QE_PAGE * D * 2;            // K rows then V rows
+  static constexpr int RAW = PAGE_BYTES + 64 * G * 4;
+  static constexpr int BYTES = (RAW + 1023) / 1024 * 1024;
+};
+
+// byte offset of the 16-byte chunk holding element (row r, column c), c % 8 == 0, of part
+// `part` of a swizzled full-precision page
+template <int D>
+__device__ __forceinline__ int swz(int part, int r, int c) {
+  return (part * (D / 64) + c / 64) * 2048 + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4);
+}
+
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB) decode_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
+    decode_kernel(const __grid_constant__ CUtensorMap tmP, DecodeArgs a) {
   using M = Map<D, G>;
   constexpr int DPL = M::DPL, LPT = M::LPT, TPS = M::TPS, SB = M::SB, SBT = M::SBT, NP = M::NP;
-  constexpr int PAGE_BYTES = 2 * QE_PAGE * D * 2;  // K rows then V rows
-  constexpr int NORM_BYTES = 64 * G * 4;           // up to a 64-token window
-  constexpr int STAGE = PAGE_BYTES + NORM_BYTES;
-  extern __shared__ __align__(128) uint8_t smem[];
+  using SL = StageLayout<D, G>;
+  constexpr int PAGE_BYTES = SL::PAGE_BYTES;
+  constexpr int STAGE = SL::BYTES;
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const DevState& st = a.st;
   const int u = blockIdx.x / a.splits, split = blockIdx.x % a.splits;
   const int b = u / st.Hkv, kvh = u % st.Hkv;
@@ -215,40 +285,15 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB) decode_kernel(Decode
   }
   __syncwarp();
 
-  // the G query heads of this group, this lane's DPL elements, in the log2 domain
+  // SIMT state for the INT2 and tail windows (set up after the full-precision phase): the G
+  // query heads of this group, this lane's DPL elements, in the log2 domain; per lane-group
+  // online-softmax state; lw/nw: sums of the current window
   float2 q[G][NP];
   float qsum[G];   // sum of the lane's q elements
   float qsum2[G];  // 4 * (sum over even elements) + (sum over odd elements): the constant part of q . x
-  {
-    const T* qb = reinterpret_cast<const T*>(a.q) + ((size_t)b * st.Hq + (size_t)kvh * G) * D;
-    const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      load_row<T, DPL>(qb + (size_t)h * D, sub, sw, q[h]);
-      float2 s2 = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int e = 0; e < NP; ++e) {
-        q[h][e] = __fmul2_rn(q[h][e], sc2);
-        s2 = __fadd2_rn(s2, q[h][e]);
-      }
-      qsum[h] = s2.x + s2.y;
-      qsum2[h] = fmaf(4.f, s2.x, s2.y);
-    }
-  }
-  // per lane-group online-softmax state; lw/nw: sums of the current window
   float2 acc[G][NP];
   float2 zacc[G];  // INT2 value offsets (even, odd element) weighted by p * ...
   float m[G], lsum[G], lw[G], nw[G];
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    zacc[h] = make_float2(0.f, 0.f);
-    m[h] = -1e30f;
-    lsum[h] = 0.f;
-    lw[h] = 0.f;
-    nw[h] = 0.f;
-#pragma unroll
-    for (int e = 0; e < NP; ++e) acc[h][e] = make_float2(0.f, 0.f);
-  }
 
   // virtual index j of this split -> (kind, list index)
   auto kind_of = [&](int j) { return j < nF ? 0 : (j < nF + nQ ? 1 : 2); };  // full, int2, tail
@@ -257,19 +302,30 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB) decode_kernel(Decode
     const int k = kind_of(j);
     return k == 0 ? ppw : (k == 1 ? 1 : (a.tail_len + QE_PAGE - 1) / QE_PAGE);
   };
-  auto advance = [&](int& j, int& pg) {
-    if (++pg >= n_tasks(j)) {
+  // This warp's windows are j = warp + kNW * r, r < n_own; the first n_own_full are
+  // full-precision. With QE_DECODE_FULL_LAST, odd warps stream their full-precision windows
+  // last (measured: no gain at c2, so off). Tasks are addressed by the ordinal o of the window
+  // in this warp's order.
+  const int n_own = nJ > warp ? (nJ - warp + kNW - 1) / kNW : 0;
+  const int n_own_full = nF > warp ? (nF - warp + kNW - 1) / kNW : 0;
+  const bool full_last = QE_DECODE_FULL_LAST && (warp & 1) && n_own_full > 0 && n_own_full < n_own;
+  auto jmap = [&](int o) {
+    const int r = !full_last ? o : (o < n_own - n_own_full ? n_own_full + o : o - (n_own - n_own_full));
+    return warp + kNW * r;
+  };
+  auto advance = [&](int& o, int& pg) {
+    if (++pg >= n_tasks(jmap(o))) {
       pg = 0;
-      j += kNW;
+      ++o;
     }
   };
   // Index prefetch: lane l holds the window id and the page ids (full, tail) or the ledger
-  // slot (INT2) of this warp's window r = rb + l, j = warp + kNW * r, so issuing a copy
-  // never waits on a dependent global load. Reloaded every 32 windows.
+  // slot (INT2) of this warp's window of ordinal rb + l, so issuing a copy never waits on a
+  // dependent global load. Reloaded every 32 windows.
   int e_win = -1, e_id[4] = {-1, -1, -1, -1}, rb = -32;
   auto load_ids = [&](int base) {
     rb = base;
-    const int jj = warp + kNW * (base + lane);
+    const int jj = base + lane < n_own ? jmap(base + lane) : nJ;
     e_win = -1;
 #pragma unroll
     for (int p = 0; p < 4; ++p) e_id[p] = -1;
@@ -289,19 +345,39 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB) decode_kernel(Decode
       }
     }
   };
-  // issue the bulk copies of task (j, pg) into stage s (all lanes call; lane 0 copies)
-  auto issue = [&](int j, int pg, int s) {
-    const int r = (j - warp) / kNW;
+  // issue the copies of task (window ordinal r, page pg) into stage s (all lanes call)
+  auto issue = [&](int r, int pg, int s) {
+    const int j = jmap(r);
     if (r - rb >= 32) load_ids(r - r % 32);
     const int src = r - rb;
     const int win = __shfl_sync(0xffffffffu, e_win, src);
     const int sel = pg == 0 ? e_id[0] : (pg == 1 ? e_id[1] : (pg == 2 ? e_id[2] : e_id[3]));
     const int id = __shfl_sync(0xffffffffu, sel, src);
-    if (lane != 0) return;
-    fence_proxy_async_smem();
     uint8_t* dst = ring + s * STAGE;
     uint64_t* bar = &bars[s];
     const int k = kind_of(j);
+    fence_proxy_async_smem();
+    if (lane != 0) return;
+    if (k == 0) {
+      // full-precision page: 2 * D/64 swizzled TMA boxes, then the page's norms
+      if (win < 0 || id < 0 || id >= st.P) {
+        qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
+        mbar_arrive_expect_tx(bar, 0);
+        return;
+      }
+      const uint32_t nb = QE_PAGE * G * 4;
+      mbar_arrive_expect_tx(bar, PAGE_BYTES + nb);
+      const int row0 = (u * st.P + id) * 2 * QE_PAGE;
+#pragma unroll
+      for (int part = 0; part < 2; ++part)
+#pragma unroll
+        for (int xb = 0; xb < D / 64; ++xb)
+          tc::tma_load_2d(dst + (part * (D / 64) + xb) * 2048, &tmP, xb * 64, row0 + part * QE_PAGE, bar);
+      bulk_g2s(dst + PAGE_BYTES, st.norms + ((size_t)u * st.norm_pitch + (size_t)win * w + pg * QE_PAGE) * G, nb,
+               bar);
+      return;
+    }
+    if (lane != 0) return;
     if (k == 1) {
       if (win < 0 || id < 0 || id >= st.S) {
         qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
@@ -319,13 +395,7 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB) decode_kernel(Decode
         return;
       }
       const uint8_t* src_p = st.pages + ((size_t)u * st.P + id) * st.page_bytes;
-      if (k == 0) {
-        const uint32_t nb = QE_PAGE * G * 4;
-        mbar_arrive_expect_tx(bar, PAGE_BYTES + nb);
-        bulk_g2s(dst, src_p, PAGE_BYTES, bar);
-        bulk_g2s(dst + PAGE_BYTES,
-                 st.norms + ((size_t)u * st.norm_pitch + (size_t)win * w + pg * QE_PAGE) * G, nb, bar);
-      } else {
+      {
         mbar_arrive_expect_tx(bar, PAGE_BYTES);
         bulk_g2s(dst, src_p, PAGE_BYTES, bar);
       }
@@ -426,174 +496,351 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB) decode_kernel(Decode
     }
   };
 
-  int j = warp, pg = 0;
-  int ij = j, ipg = 0, issued = 0;
-  for (int s = 0; s < kNST - 1 && ij < nJ; ++s) {
-    issue(ij, ipg, s);
-    advance(ij, ipg);
+  int o = 0, pg = 0;                  // window ordinal and page being computed
+  int io = 0, ipg = 0, issued = 0;    // next task to copy
+  for (int s = 0; s < kNST - 1 && io < n_own; ++s) {
+    issue(io, ipg, s);
+    advance(io, ipg);
     ++issued;
   }
   int k = 0;
   bool ok = true;
-  while (j < nJ) {
-    if (ij < nJ) {
-      issue(ij, ipg, issued % kNST);
-      advance(ij, ipg);
-      ++issued;
-    }
-    const int s = k % kNST;
-    ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[s], (k / kNST) & 1, st.status, 1000 + u));
-    if (!ok) break;
-    const uint8_t* stage = ring + s * STAGE;
-    const int kind = kind_of(j);
-    const float* nrm = reinterpret_cast<const float*>(stage + PAGE_BYTES);
-    if (kind == 0) {
-      // ---- full-precision page of a complete window: K rows [16][D], V rows [16][D] ----
-      const T* Ks = reinterpret_cast<const T*>(stage);
-      const T* Vs = Ks + QE_PAGE * D;
-#pragma unroll
-      for (int t0 = 0; t0 < QE_PAGE; t0 += SBT) {
-        float sc[SB][G];
-#pragma unroll
-        for (int i = 0; i < SB; ++i) {
-          float2 kx[NP];
-          load_row<T, DPL>(Ks + (size_t)(t0 + i * TPS + grp) * D, sub, sw, kx);
-          qk_row(kx, sc[i]);
-        }
-        butterfly(sc);
-        online(sc);
-#pragma unroll
-        for (int i = 0; i < SB; ++i) {
-          const int t = t0 + i * TPS + grp;
-          window_sums(sc[i], nrm + t * G);
-          float2 vx[NP];
-          load_row<T, DPL>(Vs + (size_t)t * D, sub, sw, vx);
-          pv_row(vx, sc[i]);
+  const int g8 = lane >> 2, t4 = lane & 3;
+
+  // ---- full-precision pages on the tensor cores ----
+  // S = Q K^T with A = the G query rows (padded to 16, raw q), B = 8-token tiles of K
+  // (ldmatrix); lane (g8, t4) then holds head g8's scores of tokens 2t4, 2t4+1, 8+2t4, 9+2t4.
+  // O^T = V^T P^T with A = V^T (ldmatrix.trans) and B = P^T taken straight from those
+  // registers, split into two 16-bit parts so the product keeps float32 accuracy. At the end
+  // the partial (per head: max, sum of weights, O as [G][D]) goes to the stage consumed last
+  // (the next copy targets it only after the merge below).
+  auto mma_phase = [&]() -> const float* {
+      uint32_t qa[D / 16][2];
+      {
+        const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+            reinterpret_cast<const T*>(a.q) + ((size_t)b * st.Hq + (size_t)kvh * G + (g8 < G ? g8 : 0)) * D);
+  #pragma unroll
+        for (int kc = 0; kc < D / 16; ++kc) {
+          qa[kc][0] = g8 < G ? qrow[kc * 8 + t4] : 0u;
+          qa[kc][1] = g8 < G ? qrow[kc * 8 + 4 + t4] : 0u;
         }
       }
-    } else if (kind == 2) {
-      // ---- a page of the tail window: mask tokens past its length, keep raw scores ----
-      const T* Ks = reinterpret_cast<const T*>(stage);
-      const T* Vs = Ks + QE_PAGE * D;
-      const int valid = min(QE_PAGE, a.tail_len - pg * QE_PAGE);
-      for (int t0 = 0; t0 < valid; t0 += SBT) {
-        float sc[SB][G];
-#pragma unroll
-        for (int i = 0; i < SB; ++i) {
-          float2 kx[NP];
-          load_row<T, DPL>(Ks + (size_t)(t0 + i * TPS + grp) * D, sub, sw, kx);
-          qk_row(kx, sc[i]);
+      float oacc[D / 16][4];
+  #pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) oacc[mt][0] = oacc[mt][1] = oacc[mt][2] = oacc[mt][3] = 0.f;
+      float mh = -1e30f, lh = 0.f, lwh = 0.f, nwh = 0.f;  // head g8: running max, sums
+      const float hmask = g8 < G ? 1.f : 0.f;
+      while (o < n_own && kind_of(jmap(o)) == 0) {
+        if (io < n_own) {
+          issue(io, ipg, issued % kNST);
+          advance(io, ipg);
+          ++issued;
         }
-        butterfly(sc);
-#pragma unroll
-        for (int i = 0; i < SB; ++i) {
-          const int t = t0 + i * TPS + grp;
-          if (t >= valid) {
-#pragma unroll
-            for (int h = 0; h < G; ++h) sc[i][h] = -INFINITY;
-          } else if (sub == 0) {
-#pragma unroll
-            for (int h = 0; h < G; ++h) a.tail_s[((size_t)u * w + pg * QE_PAGE + t) * G + h] = sc[i][h];
+        const int s = k % kNST;
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[s], (k / kNST) & 1, st.status, 1000 + u));
+        if (!ok) break;
+        const uint8_t* stage = ring + s * STAGE;
+        const float* nrm = reinterpret_cast<const float*>(stage + PAGE_BYTES);
+        float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+  #pragma unroll
+        for (int kc2 = 0; kc2 < D / 32; ++kc2) {
+          uint32_t kb[4];
+          ldsm_x4(kb, stage + swz<D>(0, lane & 7, kc2 * 32 + (lane >> 3) * 8));
+          MmaOp<T>::run(c0, qa[2 * kc2][0], 0u, qa[2 * kc2][1], 0u, kb[0], kb[1]);
+          MmaOp<T>::run(c0, qa[2 * kc2 + 1][0], 0u, qa[2 * kc2 + 1][1], 0u, kb[2], kb[3]);
+          ldsm_x4(kb, stage + swz<D>(0, 8 + (lane & 7), kc2 * 32 + (lane >> 3) * 8));
+          MmaOp<T>::run(c1, qa[2 * kc2][0], 0u, qa[2 * kc2][1], 0u, kb[0], kb[1]);
+          MmaOp<T>::run(c1, qa[2 * kc2 + 1][0], 0u, qa[2 * kc2 + 1][1], 0u, kb[2], kb[3]);
+        }
+        float mx = fmaxf(fmaxf(c0[0], c0[1]), fmaxf(c1[0], c1[1]));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        const float ms = mx * a.scale_log2;
+        const bool grow = ms > mh + kRescale;
+        if (__any_sync(0xffffffffu, grow)) {
+          const float mn = grow ? ms : mh;
+          const float f = ex2(mh - mn);
+          lh *= f;
+          lwh *= f;
+          nwh *= f;
+          mh = mn;
+          // O^T column pair (2 t4, 2 t4 + 1) belongs to heads held by lanes 8 t4 and 8 t4 + 4
+          const float fa = __shfl_sync(0xffffffffu, f, 8 * t4);
+          const float fb = __shfl_sync(0xffffffffu, f, 8 * t4 + 4);
+  #pragma unroll
+          for (int mt = 0; mt < D / 16; ++mt) {
+            oacc[mt][0] *= fa;
+            oacc[mt][1] *= fb;
+            oacc[mt][2] *= fa;
+            oacc[mt][3] *= fb;
           }
         }
-        online(sc);
-#pragma unroll
-        for (int i = 0; i < SB; ++i) {
-          const int t = t0 + i * TPS + grp;
-#pragma unroll
-          for (int h = 0; h < G; ++h) lw[h] += sc[i][h];
-          if (t < valid) {
-            float2 vx[NP];
-            load_row<T, DPL>(Vs + (size_t)t * D, sub, sw, vx);
-            pv_row(vx, sc[i]);
-          }
+        const float p0 = hmask * ex2(fmaf(c0[0], a.scale_log2, -mh));
+        const float p1 = hmask * ex2(fmaf(c0[1], a.scale_log2, -mh));
+        const float p2 = hmask * ex2(fmaf(c1[0], a.scale_log2, -mh));
+        const float p3 = hmask * ex2(fmaf(c1[1], a.scale_log2, -mh));
+        const float psum = (p0 + p1) + (p2 + p3);
+        lh += psum;
+        lwh += psum;
+        if (g8 < G) {
+          nwh = fmaf(p0, nrm[(2 * t4) * G + g8], nwh);
+          nwh = fmaf(p1, nrm[(2 * t4 + 1) * G + g8], nwh);
+          nwh = fmaf(p2, nrm[(8 + 2 * t4) * G + g8], nwh);
+          nwh = fmaf(p3, nrm[(9 + 2 * t4) * G + g8], nwh);
         }
-      }
-    } else {
-      // ---- INT2 ledger entry: codes K [w][D/4] | codes V | meta K [w][D/16] | meta V ----
-      const uint8_t* kc = stage;
-      const uint8_t* vc = stage + w * D / 4;
-      const uint32_t* km = reinterpret_cast<const uint32_t*>(stage + w * D / 2);
-      const uint32_t* vm = km + w * D / 16;
-      for (int t0 = 0; t0 < w; t0 += SBT) {
-        float sc[SB][G];
-#pragma unroll
-        for (int i = 0; i < SB; ++i) {
-          const int t = t0 + i * TPS + grp;
-          float2 x[NP];
-          decode_codes<NP>(load_codes<DPL>(kc + t * (D / 4), sub, sw), x);
-          const uint32_t mt = km[t * (D / 16) + gi];
-          const float s4 = 4.f * meta_scale(mt), z = meta_zero(mt);
-          float d[G];
-          qk_row(x, d);
-          // q . x = qsum2 + (q . c) / 4, so q . k = s (q . c) + z qsum = 4s (q . x) + z qsum - 4s qsum2
-#pragma unroll
-          for (int h = 0; h + 1 < G; h += 2) {
-            const float2 c0 = ffma2(make_float2(z, z), make_float2(qsum[h], qsum[h + 1]),
-                                    __fmul2_rn(make_float2(-s4, -s4), make_float2(qsum2[h], qsum2[h + 1])));
-            const float2 r = ffma2(make_float2(s4, s4), make_float2(d[h], d[h + 1]), c0);
-            sc[i][h] = r.x;
-            sc[i][h + 1] = r.y;
-          }
-          if constexpr (G % 2)
-            sc[i][G - 1] = fmaf(s4, d[G - 1], fmaf(z, qsum[G - 1], -s4 * qsum2[G - 1]));
+        uint32_t ph0, pl0, ph1, pl1;
+        MmaOp<T>::split(p0, p1, ph0, pl0);
+        MmaOp<T>::split(p2, p3, ph1, pl1);
+  #pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+          uint32_t va[4];
+          ldsm_x4_t(va, stage + swz<D>(1, ((lane >> 4) << 3) + (lane & 7), mt * 16 + ((lane >> 3) & 1) * 8));
+          MmaOp<T>::run(oacc[mt], va[0], va[1], va[2], va[3], ph0, ph1);
+          MmaOp<T>::run(oacc[mt], va[0], va[1], va[2], va[3], pl0, pl1);
         }
-        butterfly(sc);
-        online(sc);
-#pragma unroll
-        for (int i = 0; i < SB; ++i) {
-          const int t = t0 + i * TPS + grp;
-          window_sums(sc[i], nrm + t * G);
-          float2 x[NP];
-          decode_codes<NP>(load_codes<DPL>(vc + t * (D / 4), sub, sw), x);
-          const uint32_t mt = vm[t * (D / 16) + gi];
-          const float s4 = 4.f * meta_scale(mt), z = meta_zero(mt);
-          // v = 4s * x + (z - 16s) for even elements (x = 4 + c/4), 4s * x + (z - 4s) for odd
-          // ones (x = 1 + c/4): acc += (p * 4s) * x, zacc += p * (z - 16s, z - 4s)
-          const float2 zz = make_float2(fmaf(-4.f, s4, z), z - s4);
-          float ps[G];
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            ps[h] = sc[i][h] * s4;
-            zacc[h] = ffma2(make_float2(sc[i][h], sc[i][h]), zz, zacc[h]);
-          }
-          pv_row(x, ps);
-        }
-      }
-    }
-    __syncwarp();
-    if (pg + 1 >= n_tasks(j)) {
-      // end of a window: fold its sums into the total; record full/INT2 window partials
-      if (kind != 2) {
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          float mx = m[h];
-#pragma unroll
-          for (int o = LPT; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-          const float f = ex2(m[h] - mx);
-          float l2 = lw[h] * f, n2 = nw[h] * f;
-#pragma unroll
-          for (int o = LPT; o < 32; o <<= 1) {
-            l2 += __shfl_xor_sync(0xffffffffu, l2, o);
-            n2 += __shfl_xor_sync(0xffffffffu, n2, o);
-          }
-          if (lane == 0) {
-            float* wp = a.win_part + ((ub + list_idx(j)) * G + h) * 4;
-            wp[0] = mx;
+        __syncwarp();
+        if (pg + 1 >= ppw) {
+          // end of a window: its partial (m, sum p, sum p n) per head
+          float l2 = lwh + __shfl_xor_sync(0xffffffffu, lwh, 1);
+          l2 += __shfl_xor_sync(0xffffffffu, l2, 2);
+          float n2 = nwh + __shfl_xor_sync(0xffffffffu, nwh, 1);
+          n2 += __shfl_xor_sync(0xffffffffu, n2, 2);
+          if (t4 == 0 && g8 < G) {
+            float* wp = a.win_part + ((ub + list_idx(jmap(o))) * G + g8) * 4;
+            wp[0] = mh;
             wp[1] = l2;
             wp[2] = n2;
           }
+          lwh = 0.f;
+          nwh = 0.f;
         }
+        advance(o, pg);
+        ++k;
       }
+    lh += __shfl_xor_sync(0xffffffffu, lh, 1);
+    lh += __shfl_xor_sync(0xffffffffu, lh, 2);
+    float* fo = reinterpret_cast<float*>(ring + ((k + kNST - 1) % kNST) * STAGE);
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        lsum[h] += lw[h];
-        lw[h] = 0.f;
-        nw[h] = 0.f;
+    for (int mt = 0; mt < D / 16; ++mt) {
+      if (2 * t4 < G) {
+        fo[(2 * t4) * D + mt * 16 + g8] = oacc[mt][0];
+        fo[(2 * t4) * D + mt * 16 + g8 + 8] = oacc[mt][2];
+      }
+      if (2 * t4 + 1 < G) {
+        fo[(2 * t4 + 1) * D + mt * 16 + g8] = oacc[mt][1];
+        fo[(2 * t4 + 1) * D + mt * 16 + g8 + 8] = oacc[mt][3];
       }
     }
-    advance(j, pg);
-    ++k;
+    if (t4 == 0 && g8 < G) {
+      fo[G * D + g8] = mh;
+      fo[G * D + G + g8] = lh;
+    }
+    __syncwarp();
+    return fo;
+  };
+
+  // ---- SIMT state for the INT2 and tail windows ----
+  auto load_q = [&]() {
+    const T* qb = reinterpret_cast<const T*>(a.q) + ((size_t)b * st.Hq + (size_t)kvh * G) * D;
+    const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      load_row<T, DPL>(qb + (size_t)h * D, sub, sw, q[h]);
+      float2 s2 = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int e = 0; e < NP; ++e) {
+        q[h][e] = __fmul2_rn(q[h][e], sc2);
+        s2 = __fadd2_rn(s2, q[h][e]);
+      }
+      qsum[h] = s2.x + s2.y;
+      qsum2[h] = fmaf(4.f, s2.x, s2.y);
+    }
+  };
+  auto simt_empty = [&]() {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      zacc[h] = make_float2(0.f, 0.f);
+      m[h] = -1e30f;
+      lsum[h] = 0.f;
+      lw[h] = 0.f;
+      nw[h] = 0.f;
+#pragma unroll
+      for (int e = 0; e < NP; ++e) acc[h][e] = make_float2(0.f, 0.f);
+    }
+  };
+  // merge a tensor-core partial (at a window boundary) into the SIMT state; lane group 0
+  // takes its values, every lane group rescales to the common maximum
+  auto merge = [&](const float* fo) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float mf = fo[G * D + h], lf = fo[G * D + G + h];
+      const float M = fmaxf(m[h], mf);
+      const float fs = ex2(m[h] - M), ff = grp == 0 ? ex2(mf - M) : 0.f;
+      const float2 fs2 = make_float2(fs, fs), ff2 = make_float2(ff, ff);
+      lsum[h] = fmaf(lsum[h], fs, lf * ff);
+      zacc[h] = __fmul2_rn(zacc[h], fs2);
+#pragma unroll
+      for (int e = 0; e < NP; ++e) {
+        // register pair e of chunk c = e / 4 sits in memory chunk c ^ sw
+        const int d = DPL * sub + 8 * ((e / 4) ^ sw) + 2 * (e % 4);
+        acc[h][e] = ffma2(make_float2(fo[h * D + d], fo[h * D + d + 1]), ff2, __fmul2_rn(acc[h][e], fs2));
+      }
+      m[h] = M;
+    }
+    __syncwarp();
+  };
+
+  // ---- INT2 ledger entries and the tail window on the CUDA cores ----
+  auto simt_phase = [&]() {
+    while (ok && o < n_own && kind_of(jmap(o)) != 0) {
+      if (io < n_own) {
+        issue(io, ipg, issued % kNST);
+        advance(io, ipg);
+        ++issued;
+      }
+      const int s = k % kNST;
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[s], (k / kNST) & 1, st.status, 1000 + u));
+      if (!ok) break;
+      const uint8_t* stage = ring + s * STAGE;
+      const int j = jmap(o);
+      const int kind = kind_of(j);
+      const float* nrm = reinterpret_cast<const float*>(stage + PAGE_BYTES);
+      if (kind == 2) {
+        // ---- a page of the tail window: mask tokens past its length, keep raw scores ----
+        const T* Ks = reinterpret_cast<const T*>(stage);
+        const T* Vs = Ks + QE_PAGE * D;
+        const int valid = min(QE_PAGE, a.tail_len - pg * QE_PAGE);
+        for (int t0 = 0; t0 < valid; t0 += SBT) {
+          float sc[SB][G];
+  #pragma unroll
+          for (int i = 0; i < SB; ++i) {
+            float2 kx[NP];
+            load_row<T, DPL>(Ks + (size_t)(t0 + i * TPS + grp) * D, sub, sw, kx);
+            qk_row(kx, sc[i]);
+          }
+          butterfly(sc);
+  #pragma unroll
+          for (int i = 0; i < SB; ++i) {
+            const int t = t0 + i * TPS + grp;
+            if (t >= valid) {
+  #pragma unroll
+              for (int h = 0; h < G; ++h) sc[i][h] = -INFINITY;
+            } else if (sub == 0) {
+  #pragma unroll
+              for (int h = 0; h < G; ++h) a.tail_s[((size_t)u * w + pg * QE_PAGE + t) * G + h] = sc[i][h];
+            }
+          }
+          online(sc);
+  #pragma unroll
+          for (int i = 0; i < SB; ++i) {
+            const int t = t0 + i * TPS + grp;
+  #pragma unroll
+            for (int h = 0; h < G; ++h) lw[h] += sc[i][h];
+            if (t < valid) {
+              float2 vx[NP];
+              load_row<T, DPL>(Vs + (size_t)t * D, sub, sw, vx);
+              pv_row(vx, sc[i]);
+            }
+          }
+        }
+      } else {
+        // ---- INT2 ledger entry: codes K [w][D/4] | codes V | meta K [w][D/16] | meta V ----
+        const uint8_t* kc = stage;
+        const uint8_t* vc = stage + w * D / 4;
+        const uint32_t* km = reinterpret_cast<const uint32_t*>(stage + w * D / 2);
+        const uint32_t* vm = km + w * D / 16;
+        for (int t0 = 0; t0 < w; t0 += SBT) {
+          float sc[SB][G];
+  #pragma unroll
+          for (int i = 0; i < SB; ++i) {
+            const int t = t0 + i * TPS + grp;
+            float2 x[NP];
+            decode_codes<NP>(load_codes<DPL>(kc + t * (D / 4), sub, sw), x);
+            const uint32_t mt = km[t * (D / 16) + gi];
+            const float s4 = 4.f * meta_scale(mt), z = meta_zero(mt);
+            float d[G];
+            qk_row(x, d);
+            // q . x = qsum2 + (q . c) / 4, so q . k = s (q . c) + z qsum = 4s (q . x) + z qsum - 4s qsum2
+  #pragma unroll
+            for (int h = 0; h + 1 < G; h += 2) {
+              const float2 c0 = ffma2(make_float2(z, z), make_float2(qsum[h], qsum[h + 1]),
+                                      __fmul2_rn(make_float2(-s4, -s4), make_float2(qsum2[h], qsum2[h + 1])));
+              const float2 r = ffma2(make_float2(s4, s4), make_float2(d[h], d[h + 1]), c0);
+              sc[i][h] = r.x;
+              sc[i][h + 1] = r.y;
+            }
+            if constexpr (G % 2)
+              sc[i][G - 1] = fmaf(s4, d[G - 1], fmaf(z, qsum[G - 1], -s4 * qsum2[G - 1]));
+          }
+          butterfly(sc);
+          online(sc);
+  #pragma unroll
+          for (int i = 0; i < SB; ++i) {
+            const int t = t0 + i * TPS + grp;
+            window_sums(sc[i], nrm + t * G);
+            float2 x[NP];
+            decode_codes<NP>(load_codes<DPL>(vc + t * (D / 4), sub, sw), x);
+            const uint32_t mt = vm[t * (D / 16) + gi];
+            const float s4 = 4.f * meta_scale(mt), z = meta_zero(mt);
+            // v = 4s * x + (z - 16s) for even elements (x = 4 + c/4), 4s * x + (z - 4s) for odd
+            // ones (x = 1 + c/4): acc += (p * 4s) * x, zacc += p * (z - 16s, z - 4s)
+            const float2 zz = make_float2(fmaf(-4.f, s4, z), z - s4);
+            float ps[G];
+  #pragma unroll
+            for (int h = 0; h < G; ++h) {
+              ps[h] = sc[i][h] * s4;
+              zacc[h] = ffma2(make_float2(sc[i][h], sc[i][h]), zz, zacc[h]);
+            }
+            pv_row(x, ps);
+          }
+        }
+      }
+      __syncwarp();
+      if (pg + 1 >= n_tasks(j)) {
+        // end of a window: fold its sums into the total; record full/INT2 window partials
+        if (kind != 2) {
+  #pragma unroll
+          for (int h = 0; h < G; ++h) {
+            float mx = m[h];
+  #pragma unroll
+            for (int o = LPT; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            const float f = ex2(m[h] - mx);
+            float l2 = lw[h] * f, n2 = nw[h] * f;
+  #pragma unroll
+            for (int o = LPT; o < 32; o <<= 1) {
+              l2 += __shfl_xor_sync(0xffffffffu, l2, o);
+              n2 += __shfl_xor_sync(0xffffffffu, n2, o);
+            }
+            if (lane == 0) {
+              float* wp = a.win_part + ((ub + list_idx(j)) * G + h) * 4;
+              wp[0] = mx;
+              wp[1] = l2;
+              wp[2] = n2;
+            }
+          }
+        }
+  #pragma unroll
+        for (int h = 0; h < G; ++h) {
+          lsum[h] += lw[h];
+          lw[h] = 0.f;
+          nw[h] = 0.f;
+        }
+      }
+      advance(o, pg);
+      ++k;
+    }
+  };
+
+  // at most two segments (full then the rest, or the rest then full); each phase has one call
+  // site so that it is inlined and its state stays in registers
+  simt_empty();
+  for (int seg = 0; seg < 2 && ok && o < n_own; ++seg) {
+    if (kind_of(jmap(o)) == 0) {
+      merge(mma_phase());
+    } else {
+      load_q();
+      simt_phase();
+    }
   }
   if (!ok) {  // drain copies still in flight if a wait gave up
     for (; k < issued; ++k) mbar_wait_bounded(&bars[k % kNST], (k / kNST) & 1, st.status, 2000 + u);
@@ -742,9 +989,8 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB) decode_kernel(Decode
 
 template <typename T, int D, int G>
 int launch_decode_t(qe_ctx* c, const void* q, float* out, cudaStream_t s) {
-  constexpr int PAGE_BYTES = 2 * QE_PAGE * D * 2;
-  constexpr int STAGE = PAGE_BYTES + 64 * G * 4;
-  const size_t smem = (size_t)kNW * kNST * STAGE + kNW * kNST * 8;
+  constexpr int STAGE = StageLayout<D, G>::BYTES;
+  const size_t smem = 1024 + (size_t)kNW * kNST * STAGE + kNW * kNST * 8;  // + alignment slack
   static_assert((size_t)(kNW * G * (D + 2) + 2 * QE_MAX_G + G * D + 3 * QE_MAX_SPLITS_CLUSTER * QE_MAX_G +
                          2 * QE_MAX_G + kNW) * 4 <= (size_t)kNW * kNST * STAGE,
                 "merge area");
@@ -779,6 +1025,14 @@ int launch_decode_t(qe_ctx* c, const void* q, float* out, cudaStream_t s) {
   }
   DecodeArgs a{};
   a.st = make_state(c);
+  // the page pool as a 2-D tensor [units * P * 32 rows][D] for the swizzled TMA page loads
+  CUtensorMap tmP;
+  {
+    const unsigned long long rows = (unsigned long long)a.st.U * a.st.P * 2 * QE_PAGE;
+    if (rows >= (1ull << 31)) return QE_ERR_UNSUPPORTED_SHAPE;
+    const int e = tc::make_map(&tmP, a.st.pages, c->cfg.dtype == QE_BF16, D, rows, 64, QE_PAGE);
+    if (e) return e;
+  }
   a.q = q;
   a.out = out;
   a.win_part = c->win_part;
@@ -809,7 +1063,7 @@ int launch_decode_t(qe_ctx* c, const void* q, float* out, cudaStream_t s) {
   lc.stream = s;
   lc.attrs = la;
   lc.numAttrs = 1;
-  QE_CUDA_TRY(cudaLaunchKernelEx(&lc, kern, a));
+  QE_CUDA_TRY(cudaLaunchKernelEx(&lc, kern, tmP, a));
   return QE_OK;
 }
 

@@ -467,26 +467,66 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// quantise (first demotion only) and promote, one warp per window
+// quantise (first demotion only) and promote, one warp per (window, page)
 // ---------------------------------------------------------------------------
+// A lane owns DPL = D/32 consecutive elements of a row (one 4- or 8-byte word). The window's
+// ledger slot and the page are looked up once per 16 tokens; every row load of the page is
+// issued before the first one is used.
+template <int DPL> struct RowWord;
+template <> struct RowWord<4> { using type = uint2; };
+template <> struct RowWord<2> { using type = uint32_t; };
+
+template <typename T>
+__device__ __forceinline__ void word_to_f(uint2 w, float (&x)[4]) {
+  x[0] = Elem<T>::lo(w.x);
+  x[1] = Elem<T>::hi(w.x);
+  x[2] = Elem<T>::lo(w.y);
+  x[3] = Elem<T>::hi(w.y);
+}
+template <typename T>
+__device__ __forceinline__ void word_to_f(uint32_t w, float (&x)[2]) {
+  x[0] = Elem<T>::lo(w);
+  x[1] = Elem<T>::hi(w);
+}
+template <typename T>
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+  const T lo = Elem<T>::from_f(a), hi = Elem<T>::from_f(b);
+  return static_cast<uint32_t>(*reinterpret_cast<const unsigned short*>(&lo)) |
+         (static_cast<uint32_t>(*reinterpret_cast<const unsigned short*>(&hi)) << 16);
+}
+template <typename T>
+__device__ __forceinline__ void f_to_word(const float (&x)[4], uint2& w) {
+  w.x = pack2<T>(x[0], x[1]);
+  w.y = pack2<T>(x[2], x[3]);
+}
+template <typename T>
+__device__ __forceinline__ void f_to_word(const float (&x)[2], uint32_t& w) {
+  w = pack2<T>(x[0], x[1]);
+}
+
 template <typename T, int D>
-__global__ void apply_kernel(DevState st, const int32_t* xlist, const int32_t* plist,
-                             const int32_t* xcount, int unit_only) {
+__global__ void __launch_bounds__(256) apply_kernel(DevState st, const int32_t* xlist, const int32_t* plist,
+                                                    const int32_t* xcount, int unit_only) {
   constexpr int DPL = D / 32;
   using R = Int2Row<DPL>;
+  using Wd = typename RowWord<DPL>::type;
   const int u = unit_only >= 0 ? unit_only : blockIdx.x;
   const int lane = threadIdx.x & 31;
   const int warps = blockDim.x >> 5, gw = blockIdx.y * warps + (threadIdx.x >> 5);
   const int nx = xcount[u * 4 + 0], np = xcount[u * 4 + 1];
   const size_t ub = (size_t)u * st.Wmax;
-  const int w = st.window;
-  // one warp per (window, token): the K row and the V row of that token
-  for (int it = gw; it < (nx + np) * w; it += gridDim.y * warps) {
-    const int item = it / w, t = it % w;
+  const int w = st.window, ppw = st.ppw;
+  for (int it = gw; it < (nx + np) * ppw; it += gridDim.y * warps) {
+    const int item = it / ppw, pg = it % ppw;
     const bool quant = item < nx;
     const int win = quant ? xlist[ub + item] : plist[ub + item - nx];
+    if (win < 0 || win >= st.Wmax) {
+      if (lane == 0) qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
+      continue;
+    }
     const int slot = st.win_slot[ub + win];
-    if (win < 0 || win >= st.Wmax || slot < 0 || slot >= st.S) {
+    const int page = st.win_pages[(ub + win) * ppw + pg];
+    if (slot < 0 || slot >= st.S || page < 0 || page >= st.P) {
       if (lane == 0) qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
       continue;
     }
@@ -495,22 +535,22 @@ __global__ void apply_kernel(DevState st, const int32_t* xlist, const int32_t* p
     uint8_t* vc = sl + (size_t)w * D / 4;
     uint32_t* km = reinterpret_cast<uint32_t*>(sl + (size_t)w * D / 2);
     uint32_t* vm = km + (size_t)w * D / 16;
-    {
-      const int page = st.win_pages[(ub + win) * st.ppw + t / QE_PAGE];
-      if (page < 0 || page >= st.P) {
-        if (lane == 0) qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
-        continue;
-      }
-      T* prow = reinterpret_cast<T*>(st.pages + ((size_t)u * st.P + page) * st.page_bytes);
-      T* krow = prow + (size_t)(t % QE_PAGE) * D;
-      T* vrow = prow + (size_t)(QE_PAGE + t % QE_PAGE) * D;
-      if (quant) {
-        float xk[DPL], xv[DPL];
+    Wd* krows = reinterpret_cast<Wd*>(st.pages + ((size_t)u * st.P + page) * st.page_bytes);
+    Wd* vrows = krows + QE_PAGE * 32;  // 32 words per row
+    const int t0 = pg * QE_PAGE;       // first token of the page in its window
+    if (quant) {
+      Wd kw[QE_PAGE], vw[QE_PAGE];
 #pragma unroll
-        for (int e = 0; e < DPL; ++e) {
-          xk[e] = Elem<T>::to_f(krow[lane * DPL + e]);
-          xv[e] = Elem<T>::to_f(vrow[lane * DPL + e]);
-        }
+      for (int r = 0; r < QE_PAGE; ++r) {
+        kw[r] = krows[r * 32 + lane];
+        vw[r] = vrows[r * 32 + lane];
+      }
+#pragma unroll
+      for (int r = 0; r < QE_PAGE; ++r) {
+        const int t = t0 + r;
+        float xk[DPL], xv[DPL];
+        word_to_f<T>(kw[r], xk);
+        word_to_f<T>(vw[r], xv);
         uint32_t mk, mv;
         const uint32_t bk = R::quantize(xk, &mk);
         const uint32_t bv = R::quantize(xv, &mv);
@@ -520,17 +560,32 @@ __global__ void apply_kernel(DevState st, const int32_t* xlist, const int32_t* p
           km[(size_t)t * D / 16 + R::group_of(lane)] = mk;
           vm[(size_t)t * D / 16 + R::group_of(lane)] = mv;
         }
-      } else {
-        const uint32_t bk = R::load_codes(kc + (size_t)t * D / 4, lane);
-        const uint32_t bv = R::load_codes(vc + (size_t)t * D / 4, lane);
-        const uint32_t mk = km[(size_t)t * D / 16 + R::group_of(lane)];
-        const uint32_t mv = vm[(size_t)t * D / 16 + R::group_of(lane)];
-        const float sk = meta_scale(mk), zk = meta_zero(mk), sv = meta_scale(mv), zv = meta_zero(mv);
+      }
+    } else {
+      uint32_t bk[QE_PAGE], bv[QE_PAGE], mk[QE_PAGE], mv[QE_PAGE];
+#pragma unroll
+      for (int r = 0; r < QE_PAGE; ++r) {
+        const int t = t0 + r;
+        bk[r] = R::load_codes(kc + (size_t)t * D / 4, lane);
+        bv[r] = R::load_codes(vc + (size_t)t * D / 4, lane);
+        mk[r] = km[(size_t)t * D / 16 + R::group_of(lane)];
+        mv[r] = vm[(size_t)t * D / 16 + R::group_of(lane)];
+      }
+#pragma unroll
+      for (int r = 0; r < QE_PAGE; ++r) {
+        const float sk = meta_scale(mk[r]), zk = meta_zero(mk[r]);
+        const float sv = meta_scale(mv[r]), zv = meta_zero(mv[r]);
+        float xk[DPL], xv[DPL];
 #pragma unroll
         for (int e = 0; e < DPL; ++e) {
-          krow[lane * DPL + e] = Elem<T>::from_f(fmaf((float)((bk >> (2 * e)) & 3u), sk, zk));
-          vrow[lane * DPL + e] = Elem<T>::from_f(fmaf((float)((bv >> (2 * e)) & 3u), sv, zv));
+          xk[e] = fmaf((float)((bk[r] >> (2 * e)) & 3u), sk, zk);
+          xv[e] = fmaf((float)((bv[r] >> (2 * e)) & 3u), sv, zv);
         }
+        Wd ok, ov;
+        f_to_word<T>(xk, ok);
+        f_to_word<T>(xv, ov);
+        krows[r * 32 + lane] = ok;
+        vrows[r * 32 + lane] = ov;
       }
     }
   }
@@ -556,9 +611,13 @@ __global__ void int2_quantize_kernel(const T* x, int rows, uint8_t* codes, uint3
 template <typename T, int D>
 void launch_apply(const DevState& st, const qe_ctx* c, int unit_only, cudaStream_t s) {
   const int units = unit_only >= 0 ? 1 : st.U;
-  // 8 warps per block, up to 64 blocks per unit, each warp one (window, token) at a time
-  int per_unit = (st.Wmax * st.window + 7) / 8;
-  if (per_unit > 64) per_unit = 64;
+  // 8 warps per block, one warp per (window, page); a routing event moves at most F + Q
+  // windows into a new tier (host-given transitions at most Wmax)
+  int wins = unit_only >= 0 ? st.Wmax : c->cfg.full_windows + c->cfg.int2_windows;
+  if (wins > st.Wmax) wins = st.Wmax;
+  int per_unit = (wins * st.ppw + 7) / 8;
+  if (per_unit < 1) per_unit = 1;
+  if (per_unit > 1024) per_unit = 1024;
   apply_kernel<T, D><<<dim3(units, per_unit), 256, 0, s>>>(st, c->xlist, c->plist, c->xcount,
                                                             unit_only);
 }
