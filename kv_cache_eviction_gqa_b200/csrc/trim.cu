@@ -119,12 +119,10 @@ __device__ __forceinline__ int block_excl_scan(int v, int* total, int* sm) {
   return before + x - v;
 }
 
-// Adds one to bin `digit` of a shared histogram, aggregating equal digits of a warp.
+// Adds one to bin `digit` of a shared histogram (plain shared-memory atomics: aggregating
+// equal digits with a warp match vote cost more than the contention it saves).
 __device__ __forceinline__ void hist_add(uint32_t* sh, uint32_t digit, bool valid) {
-  const uint32_t act = __ballot_sync(0xffffffffu, valid);
-  if (!valid) return;
-  const uint32_t peers = __match_any_sync(act, digit);
-  if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&sh[digit], __popc(peers));
+  if (valid) atomicAdd(&sh[digit], 1u);
 }
 
 // Run by the last CTA of pass p once every CTA's counts are in `hist`: find the digit whose
@@ -219,19 +217,35 @@ __global__ void __launch_bounds__(kCT) trim_keygen(const float* __restrict__ bet
   if (e0 < len) {
     const int32_t* pt = page_table + static_cast<size_t>(h) * max_pages;
     unsigned long long* kout = s.keys + s.off[h];
-#pragma unroll 2
+    // every load of the thread's entries is issued before any is used: page ids, then the
+    // entries' beta and pos
+    int pgv[kEPT];
+#pragma unroll
     for (int j = 0; j < kEPT; ++j) {
       const int e = e0 + j * kCT + tid;
-      bool valid = e < len;
+      pgv[j] = e < len ? pt[e >> 4] : -1;
+    }
+    float bv[kEPT];
+    int32_t pv[kEPT];
+#pragma unroll
+    for (int j = 0; j < kEPT; ++j) {
+      const int e = e0 + j * kCT + tid;
+      const bool good = pgv[j] >= 0 && pgv[j] < n_pages_total;
+      const size_t at = good ? static_cast<size_t>(pgv[j]) * QE_PAGE + (e & 15) : 0;
+      bv[j] = good ? beta[at] : 1.f;
+      pv[j] = good ? pos[at] : 0;
+    }
+#pragma unroll
+    for (int j = 0; j < kEPT; ++j) {
+      const int e = e0 + j * kCT + tid;
+      const bool valid = e < len;
       unsigned long long ok = 0;
       if (valid) {
-        const int pg = pt[e >> 4];
-        if (pg < 0 || pg >= n_pages_total) {
+        if (pgv[j] < 0 || pgv[j] >= n_pages_total) {
           trim_error(s.st, QE_ERR_DEVICE_FAULT, h);
         } else {
-          const size_t at = static_cast<size_t>(pg) * QE_PAGE + (e & 15);
-          const double age = static_cast<double>(t) - static_cast<double>(pos[at]);
-          ok = ordered_key(age * log(static_cast<double>(beta[at])));
+          const double age = static_cast<double>(t) - static_cast<double>(pv[j]);
+          ok = ordered_key(age * log(static_cast<double>(bv[j])));
         }
         kout[e] = ok;
       }
@@ -268,21 +282,29 @@ __global__ void __launch_bounds__(kHT) trim_hist(TrimScratch s, int p) {
   const uint32_t mask = (1u << pass_width(p)) - 1u;
   for (int b = tid; b < kBins; b += kHT) sh[b] = 0;
   __syncthreads();
-  // each warp takes 64 consecutive keys per step (2 per lane); the bound is warp-uniform so
-  // every lane reaches the warp-wide votes in hist_add
+  // each warp takes 256 consecutive keys per step (8 per lane, four 16-byte loads issued
+  // together); the bound is warp-uniform so every lane reaches the warp-wide votes in hist_add
   const int lane = tid & 31;
-  const int stride = gridDim.x * kHT * 2;
-  for (int wb = (blockIdx.x * kHT + (tid & ~31)) * 2; wb < total; wb += stride) {
-    const int i0 = wb + lane * 2;
-    ulonglong2 v = make_ulonglong2(0ull, 0ull);
-    if (i0 + 1 < total)
-      v = __ldcg(reinterpret_cast<const ulonglong2*>(s.keys + i0));
-    else if (i0 < total)
-      v.x = __ldcg(s.keys + i0);
-    const bool m0 = i0 < total && (v.x >> cmp) == want;
-    const bool m1 = i0 + 1 < total && (v.y >> cmp) == want;
-    hist_add(sh, static_cast<uint32_t>(v.x >> sft) & mask, m0);
-    hist_add(sh, static_cast<uint32_t>(v.y >> sft) & mask, m1);
+  const int stride = gridDim.x * kHT * 8;
+  for (int wb = (blockIdx.x * kHT + (tid & ~31)) * 8; wb < total; wb += stride) {
+    ulonglong2 v[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int i0 = wb + c * 64 + lane * 2;
+      v[c] = make_ulonglong2(0ull, 0ull);
+      if (i0 + 1 < total)
+        v[c] = __ldcg(reinterpret_cast<const ulonglong2*>(s.keys + i0));
+      else if (i0 < total)
+        v[c].x = __ldcg(s.keys + i0);
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int i0 = wb + c * 64 + lane * 2;
+      const bool m0 = i0 < total && (v[c].x >> cmp) == want;
+      const bool m1 = i0 + 1 < total && (v[c].y >> cmp) == want;
+      hist_add(sh, static_cast<uint32_t>(v[c].x >> sft) & mask, m0);
+      hist_add(sh, static_cast<uint32_t>(v[c].y >> sft) & mask, m1);
+    }
   }
   __syncthreads();
   for (int b = tid; b < kBins; b += kHT)
