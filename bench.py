@@ -45,6 +45,22 @@ FALLBACK_HBM_GBS = 6650.0
 DECODE_TRAFFIC_BYTES = 109.682944e6 + 3.082752e6
 
 
+def max_over_ranks(value: float, device) -> float:
+    """The maximum of `value` over all ranks (the value itself without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: int, world: int, max_ms: float) -> float:
+    """Units per second of the whole job: every rank's units over the slowest rank's time."""
+    return world * units_per_rank / (max_ms / 1e3)
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -348,12 +364,8 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     clocks = clk.summary()
     step_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K_steps)]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-    value = world * K_steps / (total_ms / 1e3)
+    total_ms = max_over_ranks(sum(step_ms), dev)
+    value = whole_job_rate(K_steps, world, total_ms)
 
     # per-part breakdown (untimed for the value): one pass over the sequence with events
     # between the parts; the decode-kernel roofline comes from these decode timings
@@ -430,11 +442,8 @@ def run_ours(args, rank, world, local_rank):
         bvt.record(stream)
         bvt.synchronize()
         e2e_ms += a.elapsed_time(bvt)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * e2e_steps / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(e2e_ms, dev)
+    e2e_value = whole_job_rate(e2e_steps, world, e2e_ms)
     rc, det = ctx.status()
     if rc != 0:
         raise RuntimeError(f"device status {rc} ({det}) after the timed run")
