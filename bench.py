@@ -286,8 +286,9 @@ def run_ours(args, rank, world, local_rank):
         # profiling mode: only the eager decode steps above (for ncu -k ... -s ... -c ...)
         return
 
-    # capture one CUDA graph per decode step (append, decode, routing on s % R == 0) for the
-    # timed run, and one per step part for the per-part breakdown of the first sequence
+    # capture one CUDA graph per decode step (qe_decode_step: append fused into the decode
+    # launch, routing on s % R == 0) for the timed run, and one per step part for the per-part
+    # breakdown of the first sequence
     ctx.load_prefill(K, V, norms)
     torch.cuda.synchronize()
     snapshot = ctx.workspace.clone()
@@ -297,18 +298,15 @@ def run_ours(args, rank, world, local_rank):
     cap_stream = torch.cuda.Stream()
     for s in range(S):
         g = torch.cuda.CUDAGraph()
+        nf, nq = C.c_int(), C.c_int()
+        lib().qe_list_counts(ctx._h, C.byref(nf), C.byref(nq))
         with torch.cuda.graph(g, stream=cap_stream):
-            ctx.kv_append(ks[s], vs[s])
-            nf, nq = C.c_int(), C.c_int()
-            lib().qe_list_counts(ctx._h, C.byref(nf), C.byref(nq))
-            n = ctx.length
-            ctx.decode_attend_and_score(qs[s], out)
-            if s % R == 0:
-                ctx.route_windows()
+            ctx.decode_step(qs[s], ks[s], vs[s], out)
+        n = ctx.length
         tail_len = (n - 1) % cfg.window + 1
         finalize = n % cfg.window == 0
         g_step.append(g)
-        launches = 2 + (2 if finalize else 0) + (2 if s % R == 0 else 0)
+        launches = 1 + (2 if finalize else 0) + (2 if s % R == 0 else 0)
         meta.append((nf.value, nq.value, tail_len, finalize, launches))
     # the captures advanced the host-side step counter: start the per-part captures from a
     # fresh prefill (same device state as the snapshot)

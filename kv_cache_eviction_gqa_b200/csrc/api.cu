@@ -200,10 +200,24 @@ QE_API int qe_route_windows(qe_ctx* c, qe_stream_t s) {
 
 QE_API int qe_decode_step(qe_ctx* c, const void* q, const void* k, const void* v, float* out,
                           qe_stream_t s) {
-  int e = qe_kv_append(c, k, v, s);
-  if (e) return e;
-  e = qe_decode_attend_and_score(c, q, out, s);
-  if (e) return e;
+  // append + decode in one launch: the CTA that streams a unit's tail window first writes the
+  // new token (same results as qe_kv_append followed by qe_decode_attend_and_score)
+  if (!c || !q || !out || !k || !v) return QE_ERR_INVALID_ARG;
+  if (!c->loaded) return QE_ERR_STATE;
+  if (!qe_aligned(q, 16) || !qe_aligned(out, 16) || !qe_aligned(k, 16) || !qe_aligned(v, 16))
+    return QE_ERR_INVALID_ARG;
+  if (c->n >= c->cfg.max_ctx) return QE_ERR_POOL_EXHAUSTED;
+  cudaStream_t st = (cudaStream_t)s;
+  int e;
+  if (c->n - c->complete * c->cfg.window == c->cfg.window && (e = finalize_tail(c, st))) return e;
+  c->n += 1;
+  e = launch_decode(c, q, out, st, k, v);
+  if (e) {
+    c->n -= 1;
+    return e;
+  }
+  c->last_stream = st;
+  if (c->n - c->complete * c->cfg.window == c->cfg.window && (e = finalize_tail(c, st))) return e;
   if (c->step % c->cfg.route_every == 0) {
     e = qe_route_windows(c, s);
     if (e) return e;

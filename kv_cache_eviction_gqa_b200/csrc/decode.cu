@@ -39,6 +39,7 @@
 // (tail_p) and folded in when the window completes.
 #include <math.h>
 
+#include "append.cuh"
 #include "int2.cuh"
 #include "qe_internal.cuh"
 #include "tc_common.cuh"
@@ -77,6 +78,12 @@ struct DecodeArgs {
   int splits;        // CTAs per unit = cluster size
   int tail_win, tail_len;
   float scale_log2;  // log2(e) / sqrt(D)
+  // optional fused append of the step's token at position append_pos (k_new != nullptr): the
+  // CTA that streams the tail window writes it before its first copy
+  const uint4* k_new;
+  const uint4* v_new;
+  uint4* tailV;
+  int append_pos;
 };
 
 template <int D, int G>
@@ -276,6 +283,10 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
   const int q0 = (int)((long long)nq * split / a.splits), q1 = (int)((long long)nq * (split + 1) / a.splits);
   const int has_tail = (a.tail_len > 0 && split == a.splits - 1) ? 1 : 0;
   const int nF = f1 - f0, nQ = q1 - q0, nJ = nF + nQ + has_tail;
+  // fused append: the warp that streams the tail window writes the new token first (its tail
+  // task comes last, after this warp's own fence); the other warp starts at once
+  if (a.k_new != nullptr && has_tail && warp == (nJ - 1) % kNW)
+    append_token_warp(st, u, a.append_pos, a.k_new, a.v_new, a.tailV);
 
   uint8_t* ring = smem + warp * kNST * STAGE;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kNW * kNST * STAGE) + warp * kNST;
@@ -988,7 +999,8 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
 }
 
 template <typename T, int D, int G>
-int launch_decode_t(qe_ctx* c, const void* q, float* out, cudaStream_t s) {
+int launch_decode_t(qe_ctx* c, const void* q, float* out, cudaStream_t s, const void* k_new,
+                    const void* v_new) {
   constexpr int STAGE = StageLayout<D, G>::BYTES;
   const size_t smem = 1024 + (size_t)kNW * kNST * STAGE + kNW * kNST * 8;  // + alignment slack
   static_assert((size_t)(kNW * G * (D + 2) + 2 * QE_MAX_G + G * D + 3 * QE_MAX_SPLITS_CLUSTER * QE_MAX_G +
@@ -1040,6 +1052,10 @@ int launch_decode_t(qe_ctx* c, const void* q, float* out, cudaStream_t s) {
   a.tail_win = c->complete;
   a.tail_len = c->n - c->complete * c->cfg.window;
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
+  a.k_new = static_cast<const uint4*>(k_new);
+  a.v_new = static_cast<const uint4*>(v_new);
+  a.tailV = reinterpret_cast<uint4*>(c->tailV);
+  a.append_pos = c->n - 1;
   const int U = c->lay.units;
   // The largest split count whose U clusters are all resident in one wave, never more splits
   // than windows per tier nor than the configured maximum.
@@ -1068,22 +1084,25 @@ int launch_decode_t(qe_ctx* c, const void* q, float* out, cudaStream_t s) {
 }
 
 template <typename T, int D>
-int launch_decode_g(qe_ctx* c, const void* q, float* out, cudaStream_t s) {
+int launch_decode_g(qe_ctx* c, const void* q, float* out, cudaStream_t s, const void* k, const void* v) {
   switch (c->G) {
-    case 1: return launch_decode_t<T, D, 1>(c, q, out, s);
-    case 2: return launch_decode_t<T, D, 2>(c, q, out, s);
-    case 4: return launch_decode_t<T, D, 4>(c, q, out, s);
-    case 5: return launch_decode_t<T, D, 5>(c, q, out, s);
-    case 8: return launch_decode_t<T, D, 8>(c, q, out, s);
+    case 1: return launch_decode_t<T, D, 1>(c, q, out, s, k, v);
+    case 2: return launch_decode_t<T, D, 2>(c, q, out, s, k, v);
+    case 4: return launch_decode_t<T, D, 4>(c, q, out, s, k, v);
+    case 5: return launch_decode_t<T, D, 5>(c, q, out, s, k, v);
+    case 8: return launch_decode_t<T, D, 8>(c, q, out, s, k, v);
     default: return QE_ERR_UNSUPPORTED_SHAPE;
   }
 }
 
 }  // namespace
 
-int launch_decode(qe_ctx* c, const void* q, float* out, cudaStream_t s) {
+int launch_decode(qe_ctx* c, const void* q, float* out, cudaStream_t s, const void* k_new,
+                  const void* v_new) {
   const bool bf = c->cfg.dtype == QE_BF16;
   if (c->cfg.D == 128)
-    return bf ? launch_decode_g<__nv_bfloat16, 128>(c, q, out, s) : launch_decode_g<__half, 128>(c, q, out, s);
-  return bf ? launch_decode_g<__nv_bfloat16, 64>(c, q, out, s) : launch_decode_g<__half, 64>(c, q, out, s);
+    return bf ? launch_decode_g<__nv_bfloat16, 128>(c, q, out, s, k_new, v_new)
+              : launch_decode_g<__half, 128>(c, q, out, s, k_new, v_new);
+  return bf ? launch_decode_g<__nv_bfloat16, 64>(c, q, out, s, k_new, v_new)
+            : launch_decode_g<__half, 64>(c, q, out, s, k_new, v_new);
 }

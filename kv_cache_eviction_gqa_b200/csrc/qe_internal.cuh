@@ -176,7 +176,10 @@ static inline bool qe_aligned(const void* p, size_t a) {
 int launch_prefill(qe_ctx* c, const void* K, const void* V, int ctx_len, const float* norms,
                    cudaStream_t st);
 int launch_append(qe_ctx* c, const void* k, const void* v, cudaStream_t st);
-int launch_decode(qe_ctx* c, const void* q, float* out, cudaStream_t st);
+// k_new / v_new non-null: the decode launch also appends the step's token (position c->n - 1,
+// c->n already advanced by the caller)
+int launch_decode(qe_ctx* c, const void* q, float* out, cudaStream_t st, const void* k_new = nullptr,
+                  const void* v_new = nullptr);
 int launch_finalize(qe_ctx* c, int tail_win, cudaStream_t st);
 int launch_route(qe_ctx* c, cudaStream_t st);
 int launch_set_tier(qe_ctx* c, int unit, const int32_t* ids_host, int n, int tier, cudaStream_t st);

@@ -12,6 +12,7 @@
 // cross-unit atomics are needed and allocation is deterministic.
 #include <math.h>
 
+#include "append.cuh"
 #include "int2.cuh"
 #include "qe_internal.cuh"
 
@@ -123,55 +124,8 @@ __global__ void prefill_meta_kernel(DevState st, const uint4* V, int ctx, uint4*
 // ---------------------------------------------------------------------------
 __global__ void append_kernel(DevState st, const uint4* k_new, const uint4* v_new, int pos,
                               uint4* tailV) {
-  const int u = blockIdx.x, b = u / st.Hkv, kvh = u % st.Hkv;
-  const int w = st.window, tw = pos / w, t = pos % w, pg = t / QE_PAGE, r = pos % QE_PAGE;
-  const int vpr = st.D * 2 / 16;
-  // the new rows do not depend on the page lookup: load them first
-  uint4 kv = make_uint4(0, 0, 0, 0), vv = kv;
-  if (threadIdx.x < vpr) {
-    kv = k_new[(size_t)u * vpr + threadIdx.x];
-    vv = v_new[(size_t)u * vpr + threadIdx.x];
-  }
   __shared__ int s_page;
-  if (threadIdx.x == 0) {
-    const size_t wi = (size_t)u * st.Wmax + tw;
-    int page = -1;
-    if (t == 0) {
-      st.win_tier[wi] = QE_TIER_TAIL;
-      st.win_slot[wi] = -1;
-      st.mass[wi] = 0.f;
-      st.pert[wi] = 0.f;
-    }
-    if (r == 0) {
-      const int top = st.stacks[u * 4 + 0];
-      if (top <= 0) {
-        qe_record_error(st.status, QE_ERR_POOL_EXHAUSTED, u);
-      } else {
-        page = st.page_free[(size_t)u * st.P + top - 1];
-        st.stacks[u * 4 + 0] = top - 1;
-        st.win_pages[wi * st.ppw + pg] = page;
-      }
-    } else {
-      page = st.win_pages[wi * st.ppw + pg];
-    }
-    if (page >= st.P) {
-      qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
-      page = -1;
-    }
-    s_page = page;
-  }
-  __syncthreads();
-  if (t == 0)
-    for (int i = threadIdx.x; i < w * st.G; i += blockDim.x) st.tail_p[(size_t)u * w * st.G + i] = 0.f;
-  const int page = s_page;
-  if (page < 0) return;
-  uint4* base = reinterpret_cast<uint4*>(st.pages + ((size_t)u * st.P + page) * st.page_bytes);
-  if (threadIdx.x < vpr) {
-    const int c = threadIdx.x;
-    base[r * vpr + c] = kv;
-    base[(QE_PAGE + r) * vpr + c] = vv;
-    tailV[(((size_t)kvh * st.B + b) * w + t) * vpr + c] = vv;
-  }
+  append_token(st, blockIdx.x, pos, k_new, v_new, tailV, &s_page);
 }
 
 // ---------------------------------------------------------------------------
