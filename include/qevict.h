@@ -76,7 +76,8 @@ typedef struct {
   int max_ctx;                /* capacity in tokens per unit (prefill + decode)           */
   int pages_per_unit;         /* page-pool capacity per unit (>= ceil(prefill/16) + margin)*/
   int slots_per_unit;         /* INT2 ledger capacity per unit (>= F + Q)                 */
-  int max_splits;             /* upper bound on split-K blocks per unit (1..64)           */
+  int max_splits;             /* upper bound on split-K CTAs per unit (1..64; the kernel uses
+                                 at most 16, one thread-block cluster per unit)             */
 } qe_config;
 
 /* Byte offsets of the state arrays inside the caller's workspace (see qe_layout). */
@@ -159,8 +160,8 @@ QE_API int qe_decode_attend_and_score(qe_ctx* ctx, const void* q, float* out,
  * inputs and outputs while a step runs (an engine that gives a plugin only its buffers and
  * forbids allocation during execution, or a process whose memory belongs to another
  * allocator). The pages have no counterpart to this entry point: it only changes where the
- * decode kernel keeps its per-call scratch (split and window partials, tail scores, tickets):
- * in a fixed 16 MiB array inside the library image instead of the workspace scratch region.
+ * decode kernel keeps its per-call scratch (per-window score partials, tail scores): in a
+ * fixed 16 MiB array inside the library image instead of the workspace scratch region.
  * It calls no cudaMalloc/cudaFree. Every GPU that loads the library keeps that array until
  * exit; all calls on one GPU share it, so calls whose kernels overlap on that GPU race and
  * must be serialised. Returns QE_ERR_INVALID_ARG if the context's scratch would exceed

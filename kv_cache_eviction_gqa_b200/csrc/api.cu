@@ -29,6 +29,25 @@ int check_config(const qe_config* c) {
   return QE_OK;
 }
 
+// Sizes of the scratch buffers, in workspace order (qe_plan reserves them, qe_create points
+// into them): window partials (win_part_floats per window),
+// tail scores, quantise list, promote list, list counts, host-given ids, tail-window V rows,
+// tail-window norms.
+constexpr int kScratchParts = 8;
+void scratch_sizes(const qe_config* c, size_t (&sz)[kScratchParts]) {
+  const size_t G = c->Hq / c->Hkv, D = c->D, w = c->window;
+  const size_t U = (size_t)c->B * c->Hkv;
+  const size_t Wmax = (c->max_ctx + w - 1) / w;
+  sz[0] = U * Wmax * win_part_floats((int)D, (int)G) * 4;
+  sz[1] = U * w * G * 4;
+  sz[2] = U * Wmax * 4;
+  sz[3] = U * Wmax * 4;
+  sz[4] = U * 4 * 4;
+  sz[5] = Wmax * 4;
+  sz[6] = (size_t)c->Hkv * c->B * w * D * 2;
+  sz[7] = (size_t)c->Hkv * c->B * w * G * 4;
+}
+
 int finalize_tail(qe_ctx* c, cudaStream_t st) {
   int e = launch_finalize(c, c->complete, st);
   if (e) return e;
@@ -73,16 +92,9 @@ QE_API int qe_plan(const qe_config* c, qe_layout* L) {
   L->status = take(16);
   const size_t s0 = off;
   L->scratch = s0;
-  take(U * c->max_splits * G * (2 + D) * 4);  // split partials
-  take(U * Wmax * G * 4 * 4);                 // window partials
-  take(U * w * G * 4);                        // tail scores
-  take(U * 4);                                // tickets
-  take(U * Wmax * 4);                         // quantise list
-  take(U * Wmax * 4);                         // promote list
-  take(U * 4 * 4);                            // list counts
-  take(Wmax * 4);                             // host-given ids
-  take((size_t)c->Hkv * c->B * w * D * 2);    // tail V
-  take((size_t)c->Hkv * c->B * w * G * 4);    // tail norms
+  size_t sz[kScratchParts];
+  scratch_sizes(c, sz);
+  for (int i = 0; i < kScratchParts; ++i) take(sz[i]);
   L->scratch_bytes = off - s0;
   L->total = off;
   L->max_windows = (int)Wmax;
@@ -116,16 +128,16 @@ QE_API int qe_create(const qe_config* cfg, void* ws, size_t bytes, const void* W
     off = align_up(off + b, 256);
     return c->ws + o;
   };
-  c->split_part = (float*)take(U * cfg->max_splits * G * (2 + D) * 4);
-  c->win_part = (float*)take(U * Wmax * G * 4 * 4);
-  c->tail_s = (float*)take(U * w * G * 4);
-  c->tickets = (uint32_t*)take(U * 4);
-  c->xlist = (int32_t*)take(U * Wmax * 4);
-  c->plist = (int32_t*)take(U * Wmax * 4);
-  c->xcount = (int32_t*)take(U * 4 * 4);
-  c->host_ids = (int32_t*)take(Wmax * 4);
-  c->tailV = (uint8_t*)take((size_t)cfg->Hkv * cfg->B * w * D * 2);
-  c->tail_norm = (float*)take((size_t)cfg->Hkv * cfg->B * w * G * 4);
+  size_t sz[kScratchParts];
+  scratch_sizes(cfg, sz);
+  c->win_part = (float*)take(sz[0]);
+  c->tail_s = (float*)take(sz[1]);
+  c->xlist = (int32_t*)take(sz[2]);
+  c->plist = (int32_t*)take(sz[3]);
+  c->xcount = (int32_t*)take(sz[4]);
+  c->host_ids = (int32_t*)take(sz[5]);
+  c->tailV = (uint8_t*)take(sz[6]);
+  c->tail_norm = (float*)take(sz[7]);
   *out = c;
   return QE_OK;
 }

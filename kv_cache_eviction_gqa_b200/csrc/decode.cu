@@ -58,9 +58,6 @@ namespace {
 #ifndef QE_DECODE_FULL_LAST
 #define QE_DECODE_FULL_LAST 0  // 1: odd warps stream their full-precision windows last
 #endif
-#ifndef QE_DECODE_DPL4
-#define QE_DECODE_DPL4 16
-#endif
 #ifndef QE_DECODE_SB
 #define QE_DECODE_SB 4
 #endif
@@ -69,11 +66,13 @@ constexpr int kNW = QE_DECODE_NW;    // warps per CTA
 constexpr int kNST = QE_DECODE_NST;  // stages per warp
 constexpr float kRescale = 8.f;  // rescale the accumulators when the max grows by > 2^8
 
+// Per-window score partials: one slot per lane group of {max, sum p, sum p n} x G heads,
+// weights 2^(s - max) relative to the slot's max; an unused slot holds max -1e30 and zeros.
 struct DecodeArgs {
   DevState st;
   const void* q;     // [B][Hq][D]
   float* out;        // [B][Hq][D]
-  float* win_part;   // [U][Wmax][G][4]
+  float* win_part;   // [U][Wmax][win_part_floats(D, G)]
   float* tail_s;     // [U][window][G]
   int splits;        // CTAs per unit = cluster size
   int tail_win, tail_len;
@@ -88,7 +87,7 @@ struct DecodeArgs {
 
 template <int D, int G>
 struct Map {
-  static constexpr int DPL = G <= 4 ? QE_DECODE_DPL4 : 8;  // head-dim elements per lane
+  static constexpr int DPL = decode_dpl(G);    // head-dim elements per lane
   static constexpr int LPT = D / DPL;          // lanes per token
   static constexpr int TPS = 32 / LPT;         // tokens per warp step
   static constexpr int SB = (16 / TPS) < QE_DECODE_SB ? (16 / TPS) : QE_DECODE_SB;  // tokens per group per batch
@@ -616,11 +615,15 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
           l2 += __shfl_xor_sync(0xffffffffu, l2, 2);
           float n2 = nwh + __shfl_xor_sync(0xffffffffu, nwh, 1);
           n2 += __shfl_xor_sync(0xffffffffu, n2, 2);
-          if (t4 == 0 && g8 < G) {
-            float* wp = a.win_part + ((ub + list_idx(jmap(o))) * G + g8) * 4;
-            wp[0] = mh;
-            wp[1] = l2;
-            wp[2] = n2;
+          if (g8 < G) {
+            // slot 0 holds the window's partial, the other lanes mark the remaining slots unused
+            float* wp = a.win_part + (ub + list_idx(jmap(o))) * win_part_floats(D, G) + g8;
+#pragma unroll
+            for (int slot = t4; slot < TPS; slot += 4) {
+              wp[slot * 3 * G] = slot == 0 ? mh : -1e30f;
+              wp[slot * 3 * G + G] = slot == 0 ? l2 : 0.f;
+              wp[slot * 3 * G + 2 * G] = slot == 0 ? n2 : 0.f;
+            }
           }
           lwh = 0.f;
           nwh = 0.f;
@@ -808,25 +811,20 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
       }
       __syncwarp();
       if (pg + 1 >= n_tasks(j)) {
-        // end of a window: fold its sums into the total; record full/INT2 window partials
-        if (kind != 2) {
-  #pragma unroll
-          for (int h = 0; h < G; ++h) {
-            float mx = m[h];
-  #pragma unroll
-            for (int o = LPT; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            const float f = ex2(m[h] - mx);
-            float l2 = lw[h] * f, n2 = nw[h] * f;
-  #pragma unroll
-            for (int o = LPT; o < 32; o <<= 1) {
-              l2 += __shfl_xor_sync(0xffffffffu, l2, o);
-              n2 += __shfl_xor_sync(0xffffffffu, n2, o);
-            }
-            if (lane == 0) {
-              float* wp = a.win_part + ((ub + list_idx(j)) * G + h) * 4;
-              wp[0] = mx;
-              wp[1] = l2;
-              wp[2] = n2;
+        // end of a window: each lane group's leader records its (max, sum p, sum p n) per head
+        // in its own slot (no cross-group reduction here: the score update folds the slots)
+        if (kind != 2 && sub == 0) {
+          float* ws = a.win_part + (ub + list_idx(j)) * win_part_floats(D, G) + grp * 3 * G;
+          if constexpr (G == 4) {
+            reinterpret_cast<float4*>(ws)[0] = make_float4(m[0], m[1], m[2], m[3]);
+            reinterpret_cast<float4*>(ws + G)[0] = make_float4(lw[0], lw[1], lw[2], lw[3]);
+            reinterpret_cast<float4*>(ws + 2 * G)[0] = make_float4(nw[0], nw[1], nw[2], nw[3]);
+          } else {
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+              ws[h] = m[h];
+              ws[G + h] = lw[h];
+              ws[2 * G + h] = nw[h];
             }
           }
         }
@@ -967,12 +965,16 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
     const int win = jj < nF ? st.full_list[ub + li] : st.int2_list[ub + li - nf];
     if (win < 0 || win >= st.Wmax) continue;
     float dm = 0.f, dp = 0.f;
-    const float* wp = a.win_part + (ub + li) * G * 4;
+    const float* wp = a.win_part + (ub + li) * win_part_floats(D, G);
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float f = ex2(wp[h * 4 + 0] - lse[h]);
-      dm = fmaf(wp[h * 4 + 1], f, dm);
-      dp = fmaf(wp[h * 4 + 2], f, dp);
+    for (int slot = 0; slot < TPS; ++slot) {
+      const float* ws = wp + slot * 3 * G;
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float f = ex2(ws[h] - lse[h]);
+        dm = fmaf(ws[G + h], f, dm);
+        dp = fmaf(ws[2 * G + h], f, dp);
+      }
     }
     st.mass[ub + win] += dm;
     st.pert[ub + win] += dp;

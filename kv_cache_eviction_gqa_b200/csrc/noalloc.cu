@@ -4,16 +4,17 @@
 // inference engine that hands a plugin only its input and output buffers and forbids any
 // allocation while a request executes, or a process whose device memory is entirely owned
 // by another allocator. For them this entry point runs the split-K decode kernel with its
-// per-call scratch (split partials, per-window partials, tail-token scores and the
-// per-unit completion tickets) in a fixed array that is part of the library image, instead
-// of the scratch region of the context workspace. The cache state itself still lives in the
-// caller's workspace, and q / out are the caller's buffers.
+// per-call scratch (per-window score partials and tail-token scores) in a fixed array that is
+// part of the library image, instead of the scratch region of the context workspace. The
+// cache state itself still lives in the caller's workspace, and q / out are the caller's
+// buffers. (The splits of a unit merge through distributed shared memory, so no split
+// partials or completion counters are needed.)
 //
 // The array is a file-scope __device__ object of kStaticScratchBytes: every GPU that loads
 // this library holds that much memory until the process exits. All calls on one GPU share
-// it and it keeps the previous call's contents, so the tickets are cleared on every call,
-// and two calls whose kernels overlap on the same GPU (for example two contexts on two
-// streams) race on it: issue them one after the other. A config whose scratch needs more
+// it; every value a call reads from it was written earlier in the same call, so nothing needs
+// clearing, but two calls whose kernels overlap on the same GPU (for example two contexts on
+// two streams) race on it: issue them one after the other. A config whose scratch needs more
 // than kStaticScratchBytes is rejected with QE_ERR_INVALID_ARG before anything is enqueued.
 // The first call on a device looks up the array's device address (cudaGetSymbolAddress with
 // that device current) and caches it; make that first call before any stream capture.
@@ -50,31 +51,20 @@ extern "C" QE_API int qe_decode_attend_and_score_noalloc(qe_ctx* c, const void* 
                                                          qe_stream_t s) {
   if (!c || !q || !out) return QE_ERR_INVALID_ARG;
   // the decode kernel's per-call scratch, laid out like the workspace scratch
-  const size_t U = c->lay.units, G = c->G, D = c->cfg.D, w = c->cfg.window, W = c->lay.max_windows;
-  const size_t b_split = round256(U * c->cfg.max_splits * G * (2 + D) * 4);
-  const size_t b_win = round256(U * W * G * 4 * 4);
+  const size_t U = c->lay.units, G = c->G, w = c->cfg.window, W = c->lay.max_windows;
+  const size_t b_win = round256(U * W * win_part_floats(c->cfg.D, c->G) * 4);
   const size_t b_tail = round256(U * w * G * 4);
-  const size_t b_tick = round256(U * 4);
-  if (b_split + b_win + b_tail + b_tick > kStaticScratchBytes) return QE_ERR_INVALID_ARG;
+  if (b_win + b_tail > kStaticScratchBytes) return QE_ERR_INVALID_ARG;
   uint8_t* base = nullptr;
   int e = static_scratch(&base);
   if (e) return e;
-  cudaStream_t st = (cudaStream_t)s;
-  uint32_t* tickets = reinterpret_cast<uint32_t*>(base + b_split + b_win + b_tail);
-  QE_CUDA_TRY(cudaMemsetAsync(tickets, 0, U * 4, st));
   // run the regular entry point with the context's scratch pointers aimed at the array
-  float* sp = c->split_part;
   float* wp = c->win_part;
   float* ts = c->tail_s;
-  uint32_t* tk = c->tickets;
-  c->split_part = reinterpret_cast<float*>(base);
-  c->win_part = reinterpret_cast<float*>(base + b_split);
-  c->tail_s = reinterpret_cast<float*>(base + b_split + b_win);
-  c->tickets = tickets;
+  c->win_part = reinterpret_cast<float*>(base);
+  c->tail_s = reinterpret_cast<float*>(base + b_win);
   e = qe_decode_attend_and_score(c, q, out, s);
-  c->split_part = sp;
   c->win_part = wp;
   c->tail_s = ts;
-  c->tickets = tk;
   return e;
 }

@@ -11,6 +11,17 @@
 #include "../../include/qevict.h"
 
 #define QE_PAGE 16
+
+// Lane mapping of the decode kernel's CUDA-core path: head-dim elements per lane, and lane
+// groups (tokens processed side by side) per warp. The per-window score partials keep one
+// slot per lane group.
+#ifndef QE_DECODE_DPL4
+#define QE_DECODE_DPL4 16
+#endif
+__host__ __device__ constexpr int decode_dpl(int G) { return G <= 4 ? QE_DECODE_DPL4 : 8; }
+__host__ __device__ constexpr int decode_groups(int D, int G) { return 32 / (D / decode_dpl(G)); }
+// floats of one window's score partials: [lane-group slot][max, sum p, sum p n][G]
+__host__ __device__ constexpr int win_part_floats(int D, int G) { return decode_groups(D, G) * 3 * G; }
 #define QE_MAX_G 8
 #define QE_MAX_SPLITS 64
 
@@ -36,10 +47,8 @@ struct qe_ctx {
   int n_int2_max;       // upper bound of INT2-tier windows over units
   cudaStream_t last_stream;
   // scratch sub-buffers [dev]
-  float* split_part;    // [U][max_splits][G][2 + D]
-  float* win_part;      // [U][max_windows][G][4]
+  float* win_part;      // [U][max_windows][win_part_floats(D, G)]
   float* tail_s;        // [U][window][G]
-  uint32_t* tickets;    // [U]
   int32_t* xlist;       // [U][max_windows] transition lists (quantise) [win]
   int32_t* plist;       // [U][max_windows] transition lists (promote)  [win]
   int32_t* xcount;      // [U][4] counts: quantise, promote

@@ -623,7 +623,6 @@ int launch_prefill(qe_ctx* c, const void* K, const void* V, int ctx, const float
   QE_CUDA_TRY(cudaMemsetAsync(st.tail_p, 0, U * st.window * st.G * 4, s));
   QE_CUDA_TRY(cudaMemsetAsync(st.route_stats, 0, U * 8 * 4, s));
   QE_CUDA_TRY(cudaMemsetAsync(st.status, 0, 16, s));
-  QE_CUDA_TRY(cudaMemsetAsync(c->tickets, 0, U * 4, s));
   QE_CUDA_TRY(cudaMemsetAsync(c->xcount, 0, U * 16, s));
   const int n_pages = (ctx + QE_PAGE - 1) / QE_PAGE;
   prefill_pages_kernel<<<dim3(n_pages, (unsigned)U), 256, 0, s>>>(st, (const uint4*)K, (const uint4*)V,
