@@ -28,25 +28,32 @@ struct Int2Row {
       mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     }
-    const __half sh = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), 3.0f));
+    // (max - min) / 3 correctly rounded in float32, by the correction for division by a
+    // known constant (Markstein; Brisebarre, Muller and Raina): q0 = RN(d * RN(1/3)),
+    // r = d - 3 q0 (exact with an FMA), q = RN(q0 + r * RN(1/3)). Checked against IEEE
+    // division for every non-negative finite float32 and +inf (which passes through).
+    const float d3 = __fsub_rn(mx, mn);
+    const float third = 0.333333343267440796f;  // RN(1/3)
+    float q3 = __fmul_rn(d3, third);
+    q3 = __fmaf_rn(__fmaf_rn(-3.f, q3, d3), third, q3);
+    if (isinf(d3)) q3 = d3;
+    const __half sh = __float2half_rn(q3);
     const __half zh = __float2half_rn(mn);
     const float s = __half2float(sh), z = __half2float(zh);
-    // code = rint(f32(x - z) / s): the quotient is formed with a reciprocal, whose error
-    // (a few ulp, < 1e-6 here) can only change rint() next to a half-integer; within 1e-3 of
-    // one the correctly rounded division decides instead, so the result is that of rint of
-    // the IEEE quotient in every case.
-    const float rs = s != 0.f ? __frcp_rn(s) : 0.f;
+    // code = rint(f32(x - z) / s): the quotient is formed with an approximate reciprocal
+    // (relative error about 2^-23, far below 1e-3); within 1e-3 of a half-integer the correctly
+    // rounded division decides instead, so the result is that of rint of the IEEE quotient in
+    // every case. s == 0 gives 0 for every element; negative values and NaN convert to 0.
+    float rs = 0.f;
+    if (s != 0.f) asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rs) : "f"(s));
     uint32_t bits = 0;
 #pragma unroll
     for (int e = 0; e < DPL; ++e) {
-      float c = 0.f;
-      if (s != 0.f) {
-        const float d = __fsub_rn(x[e], z);
-        float qv = __fmul_rn(d, rs);
-        if (fabsf(qv - floorf(qv) - 0.5f) < 1e-3f) qv = __fdiv_rn(d, s);
-        c = fminf(fmaxf(rintf(qv), 0.f), 3.f);
-      }
-      bits |= static_cast<uint32_t>(c) << (2 * e);
+      const float d = __fsub_rn(x[e], z);
+      float qv = __fmul_rn(d, rs);
+      if (fabsf(qv - rintf(qv)) > 0.499f) qv = __fdiv_rn(d, s);
+      const uint32_t c = min(__float2uint_rn(qv), 3u);
+      bits |= c << (2 * e);
     }
     *meta = static_cast<uint32_t>(__half_as_ushort(sh)) |
             (static_cast<uint32_t>(__half_as_ushort(zh)) << 16);
