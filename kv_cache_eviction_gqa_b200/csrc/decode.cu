@@ -279,7 +279,11 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
   // this split's share of each tier
   const int nf = st.stacks[u * 4 + 2], nq = st.stacks[u * 4 + 3];
   const int f0 = (int)((long long)nf * split / a.splits), f1 = (int)((long long)nf * (split + 1) / a.splits);
-  const int q0 = (int)((long long)nq * split / a.splits), q1 = (int)((long long)nq * (split + 1) / a.splits);
+  // the last split also streams the tail window (and appends the new token): it counts as one
+  // INT2 window of that split's share
+  const int nqv = a.tail_len > 0 ? nq + 1 : nq;
+  const int q0 = (int)((long long)nqv * split / a.splits);
+  const int q1 = min(nq, (int)((long long)nqv * (split + 1) / a.splits));
   const int has_tail = (a.tail_len > 0 && split == a.splits - 1) ? 1 : 0;
   const int nF = f1 - f0, nQ = q1 - q0, nJ = nF + nQ + has_tail;
   // fused append: the warp that streams the tail window writes the new token first (its tail
