@@ -42,7 +42,7 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM read + write of one steady decode launch (decode step 2 of the sequence) from an ncu
 # capture of the current decode kernel (profiles/decode_kernel_c2_llama8b_32k_b8.md); set to
 # None whenever the kernel changes until it is captured again.
-DECODE_TRAFFIC_BYTES = 109.713408e6 + 5.631232e6
+DECODE_TRAFFIC_BYTES = 108.958464e6 + 4.140032e6
 
 
 def max_over_ranks(value: float, device) -> float:
