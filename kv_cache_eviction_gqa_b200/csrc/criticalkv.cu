@@ -424,16 +424,19 @@ int launch_obs(const void* q_obs, const void* K, int units, int B, int Hq, int H
   using S = ObsSmem<D>;
   auto k1 = obs_kernel<D, BF16, 1>;
   auto k2 = obs_kernel<D, BF16, 2>;
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
+  static QeOnce once;
+  static int sms_of[QE_MAX_DEVICES];
+  int dev = 0;
+  int e = qe_once_per_device(once, &dev, [&](int d) {
     QE_CUDA_TRY(cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, S::BYTES));
     QE_CUDA_TRY(cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, S::BYTES));
-    QE_CUDA_TRY(cudaGetDevice(&dev));
-    QE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-  }
+    QE_CUDA_TRY(cudaDeviceGetAttribute(&sms_of[d], cudaDevAttrMultiProcessorCount, d));
+    return QE_OK;
+  });
+  if (e) return e;
+  const int sms = sms_of[dev];
   CUtensorMap tmQ, tmK;
-  int e = make_map(&tmQ, q_obs, BF16, D, (uint64_t)B * Hq * n_obs, 64, kRows);
+  e = make_map(&tmQ, q_obs, BF16, D, (uint64_t)B * Hq * n_obs, 64, kRows);
   if (e) return e;
   e = make_map(&tmK, K, BF16, D, (uint64_t)units * n, 64, kTile);
   if (e) return e;
@@ -521,11 +524,13 @@ QE_API int qe_criticalkv_select(const void* q_obs, int n_obs, const void* K, con
   if (e) return e;
   const int b1 = (int)floor((double)alpha * (double)budget);
   const size_t smem = sizeof(SelShared);
-  static bool attr = false;
-  if (!attr) {
+  static QeOnce once;
+  int dev = 0;
+  e = qe_once_per_device(once, &dev, [&](int) {
     QE_CUDA_TRY(cudaFuncSetAttribute(ckv_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    attr = true;
-  }
+    return QE_OK;
+  });
+  if (e) return e;
   ckv_select<<<units, kSelThreads, smem, st>>>(A_out, N_out, n, G, budget, b1,
                                                reinterpret_cast<float*>(base + L.sa),
                                                reinterpret_cast<float*>(base + L.sp), idx_out);

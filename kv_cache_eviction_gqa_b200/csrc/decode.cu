@@ -1,5 +1,5 @@
 // Split-K GQA decode attention over the full-precision and INT2 tiers, fused with the
-// cumulative window scores.
+// cumulative window scores and (optionally) the append of the step's token.
 //
 // "Resumo Técnico: QEvict" - Mecanismos Principais: window-level routing driven by
 // attention accumulated over time (Pontuação Cumulativa); the recoverable INT2 tier stays
@@ -7,36 +7,44 @@
 // "Resumo Técnico: CriticalKV" - Etapa 2: the perturbation score A_i * ||V_i W_O||_1.
 //
 // Work split. Per unit u = (b, g) the live windows are [full windows | INT2 windows | tail].
-// Split s of S takes the s-th S-th of the full windows and the s-th S-th of the INT2
-// windows (the last split also takes the tail), so every CTA - and every SM - streams the
-// same mix of bandwidth-heavy full pages and arithmetic-heavy INT2 entries. Inside a CTA
-// each warp takes whole windows round-robin and streams them through its own ring of
-// shared-memory stages with 1-D bulk copies (cp.async.bulk, completion on an mbarrier,
-// one CTA only): one 16-token page (K rows then V rows) per stage for a full window, the whole
-// ledger entry for an INT2 window, each with the tokens' projected-value norms.
+// The unit's S CTAs form one thread-block cluster; CTA s takes the s-th S-th of the full
+// windows and of the INT2 windows (the tail counts as one more INT2 window of the last CTA),
+// so every SM streams the same mix of bandwidth-heavy full pages and arithmetic-heavy INT2
+// entries. Inside a CTA each warp takes whole windows round-robin and streams them through
+// its own ring of shared-memory stages (completion on an mbarrier per stage): a full page
+// arrives as 128-byte-swizzled TMA boxes from a tensor map over the page pool, an INT2
+// ledger entry or a tail page as one 1-D bulk copy, each with its tokens' projected-value norms.
 //
-// Lane mapping. A token is handled by LPT = D / DPL lanes; lane `sub` owns the DPL
-// contiguous head-dim elements [DPL*sub, DPL*sub + DPL), i.e. one INT2 group (DPL = 16) or
-// half of one (DPL = 8), so it needs one scale/zero per token. With DPL = 16 the two 8-element
-// chunks of a lane are loaded in a lane-dependent order (register chunk c holds memory chunk
-// c ^ sw) so that every 16-byte shared-memory load instruction of the warp touches each bank
-// once. A warp works on TPS = 32 / LPT tokens at a time; q and the accumulators of the G
-// query heads stay in registers as float pairs and all multiply-adds are packed (f32x2).
-// A token's G dot products are summed over its lanes with a butterfly, so every lane of the
-// group holds the scores and no weight broadcast is needed. Each lane group keeps its own
-// online-softmax state (log2 domain); the accumulators are rescaled only when the running
-// maximum grows by more than 2^8, and the groups are merged once per warp at the end.
+// Full-precision windows run on the warp-level tensor cores (m16n8k16, f32 accumulate):
+// S = Q K^T with the G query rows padded to 16, then O^T = V^T P^T with P split into two
+// 16-bit parts so the product keeps float32 accuracy. A decode step has G <= 8 query rows per
+// KV head; a tcgen05 tile (M >= 64) would be mostly padding and its TMEM round trip buys
+// nothing on a path that HBM bounds, so these pages stay on mma.sync.
 //
-// INT2 decoding without float conversions: a 2-bit code c is placed in the two top
-// mantissa bits of 1.0, x = 1 + c/4 (two integer ops), and the affine map is folded into
-// the per-token scale: k = c*s + z = 4s*x + (z - 4s).
+// INT2 and tail windows run on the CUDA cores. A token is handled by LPT = D / DPL lanes; lane
+// `sub` owns the DPL contiguous head-dim elements [DPL*sub, DPL*sub + DPL), i.e. one INT2
+// group (DPL = 16) or half of one (DPL = 8), so it needs one scale/zero per token. With
+// DPL = 16 the two 8-element chunks of a lane are loaded in a lane-dependent order (register
+// chunk c holds memory chunk c ^ sw) so that every 16-byte shared-memory load instruction of
+// the warp touches each bank once. A warp works on TPS = 32 / LPT tokens at a time; q and the
+// accumulators of the G query heads stay in registers as float pairs and all multiply-adds
+// are packed (f32x2). A token's G dot products are summed over its lanes with a butterfly, so
+// every lane of the group holds the scores and no weight broadcast is needed. Each lane group
+// keeps its own online-softmax state (log2 domain); the accumulators are rescaled only when
+// the running maximum grows by more than 2^8.
 //
-// Scoring without a second pass: every warp records per window and head the partial
-// (m, sum_i 2^(s_i-m), sum_i 2^(s_i-m) n_i). The last CTA of the unit to finish (atomic
-// ticket, no spinning) merges the splits into the output and the per-head log-sum-exp and
-// adds each window's exact attention mass and perturbation to the cumulative scores. The
-// tail window's norms are not known yet; its per-token attention is accumulated instead
-// (tail_p) and folded in when the window completes.
+// INT2 decoding without float conversions: a pair of 2-bit codes (even element E, odd E+1)
+// is shifted once into the mantissas of 4.0 and 1.0, giving x = 4 + c_E/4 and 1 + c_(E+1)/4
+// exactly; the affine map k = c*s + z is folded into the per-token scale (4s) and a per-pair
+// offset, so a score is 4s (q . x) + z sum(q) - 4s (4 sum(q_even) + sum(q_odd)).
+//
+// Scoring without a second pass: at the end of each window every lane group records its
+// (max, sum_i 2^(s_i-max), sum_i 2^(s_i-max) n_i) per head in its own slot. After the pass the
+// cluster merges the CTA partials through distributed shared memory into the unit's log-sum-
+// exp; each CTA writes its share of the output and adds the exact attention mass and
+// perturbation of the windows it streamed to the cumulative scores. The tail window's norms
+// are not known yet; its per-token attention is accumulated instead (tail_p) and folded in
+// when the window completes.
 #include <math.h>
 
 #include "append.cuh"
@@ -391,7 +399,6 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
                bar);
       return;
     }
-    if (lane != 0) return;
     if (k == 1) {
       if (win < 0 || id < 0 || id >= st.S) {
         qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
@@ -1013,11 +1020,12 @@ int launch_decode_t(qe_ctx* c, const void* q, float* out, cudaStream_t s, const 
                          2 * QE_MAX_G + kNW) * 4 <= (size_t)kNW * kNST * STAGE,
                 "merge area");
   auto kern = decode_kernel<T, D, G>;
-  // One-time set-up per instantiation (kept out of the per-step path and of graph capture):
-  // clusters[S] = how many clusters of S CTAs can be resident at once.
-  static int clusters[QE_MAX_SPLITS_CLUSTER + 1] = {0};
-  static bool ready = false;
-  if (!ready) {
+  // One-time set-up per instantiation and device (kept out of the per-step path and of graph
+  // capture): clusters[S] = how many clusters of S CTAs can be resident at once.
+  static QeOnce once;
+  static int clusters_of[QE_MAX_DEVICES][QE_MAX_SPLITS_CLUSTER + 1];
+  int dev = 0;
+  const int se = qe_once_per_device(once, &dev, [&](int d) {
     QE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     QE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
     for (int S = 1; S <= QE_MAX_SPLITS_CLUSTER; ++S) {
@@ -1037,10 +1045,12 @@ int launch_decode_t(qe_ctx* c, const void* q, float* out, cudaStream_t s, const 
         (void)cudaGetLastError();
         n = 0;
       }
-      clusters[S] = n;
+      clusters_of[d][S] = n;
     }
-    ready = true;
-  }
+    return QE_OK;
+  });
+  if (se) return se;
+  const int* clusters = clusters_of[dev];
   DecodeArgs a{};
   a.st = make_state(c);
   // the page pool as a 2-D tensor [units * P * 32 rows][D] for the swizzled TMA page loads

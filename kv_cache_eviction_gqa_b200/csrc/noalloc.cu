@@ -25,22 +25,22 @@ namespace {
 constexpr size_t kStaticScratchBytes = 16u << 20;  // 16 MiB
 static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
-constexpr int kMaxDevices = 64;
-uint8_t* g_scratch_ptr[kMaxDevices];  // device address of g_static_scratch per device
+uint8_t* g_scratch_ptr[QE_MAX_DEVICES];  // device address of g_static_scratch per device
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
 // Device address of the static scratch on the current device. The first call on a device
 // resolves it with cudaGetSymbolAddress (with that device current) and caches it.
 int static_scratch(uint8_t** out) {
+  static QeOnce once;
   int dev = 0;
-  QE_CUDA_TRY(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= kMaxDevices) return QE_ERR_INVALID_ARG;
-  if (!g_scratch_ptr[dev]) {
+  const int e = qe_once_per_device(once, &dev, [](int d) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return QE_ERR_CUDA;
-    g_scratch_ptr[dev] = static_cast<uint8_t*>(p);
-  }
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return (int)QE_ERR_CUDA;
+    g_scratch_ptr[d] = static_cast<uint8_t*>(p);
+    return (int)QE_OK;
+  });
+  if (e) return e;
   *out = g_scratch_ptr[dev];
   return QE_OK;
 }

@@ -8,6 +8,8 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/qevict.h"
 
 #define QE_PAGE 16
@@ -176,6 +178,28 @@ template <> struct Elem<__half> {
     cudaError_t _e = (expr);                      \
     if (_e != cudaSuccess) return QE_ERR_CUDA;    \
   } while (0)
+
+// One-time host set-up of a kernel (attributes, occupancy queries) for each device this
+// process launches on. setup(dev) runs under a lock on the first call for that device and is
+// retried on the next call if it failed; results it stores per device are visible to every
+// thread once this returns QE_OK.
+#define QE_MAX_DEVICES 64
+struct QeOnce {
+  std::mutex mu;
+  bool done[QE_MAX_DEVICES] = {};
+};
+template <typename F>
+int qe_once_per_device(QeOnce& once, int* dev_out, F&& setup) {
+  int dev = 0;
+  QE_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= QE_MAX_DEVICES) return QE_ERR_UNSUPPORTED_SHAPE;
+  *dev_out = dev;
+  std::lock_guard<std::mutex> g(once.mu);
+  if (once.done[dev]) return QE_OK;
+  const int e = setup(dev);
+  if (e == QE_OK) once.done[dev] = true;
+  return e;
+}
 
 static inline bool qe_aligned(const void* p, size_t a) {
   return (reinterpret_cast<uintptr_t>(p) % a) == 0;

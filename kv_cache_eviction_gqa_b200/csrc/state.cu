@@ -594,15 +594,16 @@ size_t route_smem(const DevState& st) {
   return N * 8 + (size_t)st.Wmax * (4 + 4 + 4 + 5) + 64;
 }
 
-// Raise the route kernel's dynamic shared-memory limit once (outside any graph capture).
+// Raise the route kernel's dynamic shared-memory limit once per device (outside any graph
+// capture).
 int route_smem_attr(size_t smem, int Wmax) {
-  static size_t granted = 0;
   if (smem > 200 * 1024 || Wmax > 4096) return QE_ERR_UNSUPPORTED_SHAPE;
-  if (smem > granted) {
+  static QeOnce once;
+  int dev = 0;
+  return qe_once_per_device(once, &dev, [](int) {
     QE_CUDA_TRY(cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
-    granted = 200 * 1024;
-  }
-  return QE_OK;
+    return QE_OK;
+  });
 }
 
 }  // namespace

@@ -184,15 +184,18 @@ int launch_tc(const void* V, int n_groups, int rows, const void* W, int Hq, int 
   constexpr size_t SMEM_USE = 1024 + (size_t)kMT * KB * kBM * 128 + (size_t)kNST * (kBN / 64) * D * 128 + 256;
   constexpr size_t SMEM = SMEM_USE > 120 * 1024 ? SMEM_USE : 120 * 1024;
   auto kern = vwo_tc_kernel<D, BF16>;
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
+  static QeOnce once;
+  static int sms_of[QE_MAX_DEVICES];
+  int dev = 0;
+  int e = qe_once_per_device(once, &dev, [&](int d) {
     QE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM));
-    QE_CUDA_TRY(cudaGetDevice(&dev));
-    QE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-  }
+    QE_CUDA_TRY(cudaDeviceGetAttribute(&sms_of[d], cudaDevAttrMultiProcessorCount, d));
+    return QE_OK;
+  });
+  if (e) return e;
+  const int sms = sms_of[dev];
   CUtensorMap tmV, tmW;
-  int e = make_map(&tmV, V, BF16, D, (uint64_t)n_groups * rows, 64, kBM);
+  e = make_map(&tmV, V, BF16, D, (uint64_t)n_groups * rows, 64, kBM);
   if (e) return e;
   e = make_map(&tmW, W, BF16, hidden, (uint64_t)Hq * D, 64, D);
   if (e) return e;
