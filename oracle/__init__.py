@@ -25,6 +25,9 @@ Functions and where they come from (page title, section):
   (Orçamento Global), 4 (Implementação, paged variable-length heads).
 * ``output_perturbation`` -- L = ||o - o_hat||_1; "Resumo Técnico: CriticalKV",
   Framework Teórico (Definição de Perturbação). Diagnostic only.
+* ``tier_diagnostics`` / ``future_missed_mass`` -- selection churn, global
+  latent importance reactivation and future missed mass; "Resumo Técnico:
+  QEvict", Principais Contribuições 1.
 
 Parity status of each function is listed in ``oracle/qevict_oracle.py``.
 """

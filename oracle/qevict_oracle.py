@@ -29,6 +29,13 @@ Pins (tests that tie each function to something other than itself):
   the lowest flat indices; compared with ``np.argsort`` on tiny sets.
 * output_perturbation -- diagnostic only (parity unpinned: the pages give no
   value for it and the bound theta is not printed).
+* tier_diagnostics -- hand-worked two-unit event sequence in
+  ``tests/golden/diag_tiers.txt``; a constant sequence has no change and no exit;
+  a window alternating FULL/INT2 counts every exit and re-entry once per event and
+  once per window; TAIL->FULL and first entries are not re-entries.
+* future_missed_mass -- brute force with scalar ``math.exp`` loops; q = 0 gives
+  the evicted share of tokens; no evicted window gives 0 and all evicted gives 1;
+  a hand-worked four-token case with p proportional to 1:2:3:4.
 """
 from __future__ import annotations
 
@@ -398,3 +405,78 @@ def output_perturbation(q, K, V, subset, W_O_h=None) -> float:
     if W_O_h is not None:
         d = d @ np.asarray(W_O_h, dtype=np.float64)
     return float(np.abs(d).sum())
+
+
+# ---------------------------------------------------------------------------
+# QEvict diagnostics ("Resumo Técnico: QEvict", Principais Contribuições 1:
+# Massa Perdida Futura, LIR Global, Churn de Seleção)
+# ---------------------------------------------------------------------------
+
+# per-unit counter order shared by the tier diagnostics' results
+DIAG_COUNTERS = ("live_prev", "changed", "exits", "reentries", "windows_exited", "windows_reentered")
+
+
+def tier_diagnostics(tier_maps) -> dict:
+    """Selection churn and latent importance reactivation over consecutive routing events.
+
+    tier_maps: sequence of E integer arrays [U][W] (or [W]), the tier of every window
+    after routing events 0..E-1 (EVICTED also marks windows that do not exist yet).
+    Between events e-1 and e, per unit:
+      live_prev  += #windows live (FULL or INT2) at e-1
+      changed    += #of those whose tier at e differs from their tier at e-1
+      exits      += #windows FULL at e-1 and not FULL at e  (leaving the active set)
+      reentries  += #windows not FULL at e-1, FULL at e, that exited at an earlier event
+      windows_exited / windows_reentered: windows whose first exit / first re-entry this is.
+    churn = changed / live_prev and lir = windows_reentered / windows_exited, both pooled
+    over every unit (nan when the denominator is 0). Returns {"per_unit": int64 [U][6] in
+    DIAG_COUNTERS order, "churn": float, "lir": float}.
+    """
+    maps = [np.atleast_2d(np.asarray(m, dtype=np.int64)) for m in tier_maps]
+    U, W = maps[0].shape
+    counts = np.zeros((U, len(DIAG_COUNTERS)), dtype=np.int64)
+    for u in range(U):
+        exited = [False] * W
+        reentered = [False] * W
+        for e in range(1, len(maps)):
+            for w in range(W):
+                before, now = int(maps[e - 1][u, w]), int(maps[e][u, w])
+                if before in (FULL, INT2):
+                    counts[u, 0] += 1
+                    if now != before:
+                        counts[u, 1] += 1
+                if before == FULL and now != FULL:
+                    counts[u, 2] += 1
+                    if not exited[w]:
+                        exited[w] = True
+                        counts[u, 4] += 1
+                elif before != FULL and now == FULL and exited[w]:
+                    counts[u, 3] += 1
+                    if not reentered[w]:
+                        reentered[w] = True
+                        counts[u, 5] += 1
+    tot = counts.sum(axis=0)
+    churn = tot[1] / tot[0] if tot[0] else float("nan")
+    lir = tot[5] / tot[4] if tot[4] else float("nan")
+    return {"per_unit": counts, "churn": float(churn), "lir": float(lir)}
+
+
+def future_missed_mass(qG: np.ndarray, K: np.ndarray, tiers: np.ndarray, window: int) -> float:
+    """Share of the ghost attention that falls on evicted windows, averaged over the G heads.
+
+    qG [G][D]: the step's query heads of one kv head; K [n][D]: the keys of every token so far
+    at their original precision (the ghost cache: evicted windows included); tiers [W]: the
+    tier of each window, token i lying in window i // window. For each head the ghost
+    attention is the softmax of q.K_i / sqrt(D) over all n tokens; the result is
+    (1/G) sum_h sum_{i in an EVICTED window} p_{h,i}, and 0 when n = 0.
+    """
+    K = np.asarray(K, dtype=np.float64)
+    n = K.shape[0]
+    if n == 0:
+        return 0.0
+    evicted = np.asarray(tiers)[np.arange(n) // window] == EVICTED
+    G = len(qG)
+    total = 0.0
+    for h in range(G):
+        _, p = attend(np.asarray(qG[h], dtype=np.float64), K, K)
+        total += p[evicted].sum()
+    return total / G

@@ -404,3 +404,106 @@ def test_output_perturbation_full_subset_is_zero():
     q, K, V = r.standard_normal(8), r.standard_normal((6, 8)), r.standard_normal((6, 8))
     assert O.output_perturbation(q, K, V, np.arange(6)) < 1e-14
     assert O.output_perturbation(q, K, V, np.arange(3)) > 0
+
+
+# ---------------------------------------------------------------------------
+# QEvict diagnostics ("Resumo Técnico: QEvict", Principais Contribuições 1)
+# ---------------------------------------------------------------------------
+
+_LETTER = {"E": O.EVICTED, "Q": O.INT2, "F": O.FULL, "T": O.TAIL}
+
+
+def _golden_diag(golden_dir):
+    units, counts, vals = {}, {}, {}
+    for line in open(os.path.join(golden_dir, "diag_tiers.txt")):
+        if line.startswith("#") or "|" not in line:
+            continue
+        key, val = (x.strip() for x in line.split("|"))
+        if key.startswith("unit"):
+            units[int(key.split()[1])] = [[_LETTER[c] for c in ev] for ev in val.split()]
+        elif key.startswith("counts"):
+            counts[int(key.split()[1])] = [int(x) for x in val.split()]
+        else:
+            vals[key] = float(val)
+    return units, counts, vals
+
+
+def test_tier_diagnostics_golden(golden_dir):
+    units, counts, vals = _golden_diag(golden_dir)
+    per = []
+    for u in sorted(units):
+        r = O.tier_diagnostics([np.array(ev) for ev in units[u]])
+        assert r["per_unit"][0].tolist() == counts[u]
+        per.append(r["per_unit"][0])
+    # pooled over the two units
+    tot = np.sum(per, axis=0)
+    assert tot[1] / tot[0] == vals["churn"]
+    assert abs(tot[5] / tot[4] - vals["lir"]) < 1e-15
+
+
+def test_tier_diagnostics_invariants():
+    F, Q, E, T = O.FULL, O.INT2, O.EVICTED, O.TAIL
+    # a constant sequence: live windows counted every event, nothing changes or exits
+    m = np.array([[F, Q, E, T]])
+    r = O.tier_diagnostics([m, m, m])
+    assert r["per_unit"][0].tolist() == [4, 0, 0, 0, 0, 0] and r["churn"] == 0.0
+    assert np.isnan(r["lir"])
+    # one window alternating F/Q over 5 events: 4 changes, 2 exits, 2 re-entries, 1 window each
+    seq = [np.array([x]) for x in (F, Q, F, Q, F)]
+    r = O.tier_diagnostics(seq)
+    assert r["per_unit"][0].tolist() == [4, 4, 2, 2, 1, 1] and r["lir"] == 1.0
+    # eviction is final: F -> E -> E counts one exit and nothing after it
+    r = O.tier_diagnostics([np.array([F]), np.array([E]), np.array([E])])
+    assert r["per_unit"][0].tolist() == [1, 1, 1, 0, 1, 0] and r["lir"] == 0.0
+    # tail and not-yet-existing windows are not live; their first F is not a re-entry
+    r = O.tier_diagnostics([np.array([E, T]), np.array([T, F]), np.array([F, F])])
+    assert r["per_unit"][0].tolist() == [1, 0, 0, 0, 0, 0]
+    # units are independent: stacking two units adds their counts
+    a = [np.array([F, Q]), np.array([Q, F]), np.array([F, F])]
+    b = [np.array([Q, F]), np.array([F, E]), np.array([E, E])]
+    ra, rb = O.tier_diagnostics(a)["per_unit"][0], O.tier_diagnostics(b)["per_unit"][0]
+    rab = O.tier_diagnostics([np.stack([x, y]) for x, y in zip(a, b)])["per_unit"]
+    assert rab[0].tolist() == ra.tolist() and rab[1].tolist() == rb.tolist()
+
+
+def _fmm_brute(qG, K, tiers, window):
+    n, D = len(K), len(K[0])
+    acc = 0.0
+    for q in qG:
+        s = [sum(float(q[d]) * float(K[i][d]) for d in range(D)) / math.sqrt(D) for i in range(n)]
+        mx = max(s)
+        e = [math.exp(x - mx) for x in s]
+        tot = sum(e)
+        acc += sum(e[i] for i in range(n) if tiers[i // window] == O.EVICTED) / tot
+    return acc / len(qG)
+
+
+def test_future_missed_mass_brute_force():
+    rng = np.random.default_rng(91)
+    for n, G, D, w in [(37, 3, 8, 8), (16, 1, 4, 16), (50, 5, 16, 4)]:
+        qG = rng.normal(size=(G, D)) * 2
+        K = rng.normal(size=(n, D))
+        tiers = rng.choice([O.EVICTED, O.INT2, O.FULL], size=(n + w - 1) // w)
+        tiers[-1] = O.TAIL
+        assert abs(O.future_missed_mass(qG, K, tiers, w) - _fmm_brute(qG, K, tiers, w)) < 1e-12
+
+
+def test_future_missed_mass_closed_forms():
+    rng = np.random.default_rng(92)
+    n, D, w = 40, 8, 8
+    K = rng.normal(size=(n, D))
+    tiers = np.array([O.EVICTED, O.FULL, O.EVICTED, O.INT2, O.TAIL])
+    # q = 0: uniform attention, so the missed mass is the evicted share of the tokens
+    assert abs(O.future_missed_mass(np.zeros((3, D)), K, tiers, w) - 16 / 40) < 1e-15
+    # nothing evicted -> 0; everything evicted -> 1; no tokens -> 0
+    q = rng.normal(size=(2, D))
+    assert O.future_missed_mass(q, K, np.full(5, O.FULL), w) == 0.0
+    assert abs(O.future_missed_mass(q, K, np.full(5, O.EVICTED), w) - 1.0) < 1e-15
+    assert O.future_missed_mass(q, K[:0], tiers, w) == 0.0
+    # hand-worked: D = 4 (sqrt D = 2), q = (2, 0, 0, 0), K_i = (ln a_i, 0, 0, 0) gives
+    # scores ln a_i and p proportional to a = 1:2:3:4; window 2 with window 0 evicted -> 3/10
+    a = np.array([1.0, 2.0, 3.0, 4.0])
+    Kh = np.zeros((4, 4))
+    Kh[:, 0] = np.log(a)
+    fmm = O.future_missed_mass(np.array([[2.0, 0, 0, 0]]), Kh, np.array([O.EVICTED, O.FULL]), 2)
+    assert abs(fmm - 0.3) < 1e-15
