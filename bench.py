@@ -690,6 +690,114 @@ def run_c4(args):
     print(json.dumps(line), flush=True)
 
 
+def run_diag(args):
+    import torch
+
+    from kv_cache_eviction_gqa_b200 import binding as Bd
+    import oracle as O
+    cfg = W.DIAG_C2
+    b = cfg.base
+    dev = torch.device("cuda", 0)
+    t = torch.bfloat16
+    hbm, hbm_kind = measured_peaks()
+    hist = W.draw_tier_history(cfg)
+    qn = W.draw_diag_queries(cfg)
+    U, Wn, E = b.units, cfg.W, cfg.events
+    cpu = None
+    if not args.no_cpu_baseline:
+        K0 = W.draw_ghost_keys(cfg, 0, 0)
+        t0 = time.perf_counter()
+        reps = 0
+        while True:
+            O.future_missed_mass(qn[0, :b.G], K0, hist[-1][0], b.window)
+            O.tier_diagnostics([h[0] for h in hist[:2]])
+            reps += 1
+            if time.perf_counter() - t0 > 10.0:
+                break
+        per_unit = (time.perf_counter() - t0) / reps
+        cpu = {"value": 1.0 / (per_unit * U), "unit": "diagnostic updates/s", "kind": "oracle",
+               "cores": len(os.sched_getaffinity(0)), "blas_threads": blas_threads(),
+               "sample": f"float64 oracle on 1 of {U} units ({reps} updates: FMM over {cfg.n} keys + one "
+                         "tier-map comparison), scaled to all units"}
+    K = torch.empty((b.B, b.Hkv, cfg.n_stride, b.D), dtype=t, device=dev)
+    for bb in range(b.B):
+        for h in range(b.Hkv):
+            K[bb, h, :cfg.n] = torch.from_numpy(W.draw_ghost_keys(cfg, bb, h)).to(dev, t)
+    q = torch.from_numpy(qn).to(dev, t)
+    maps = torch.from_numpy(hist).to(dev)
+    diag = Bd.TierDiagnostics(U, Wn, dev)
+    fmm, scratch = Bd.diag_fmm(q, K, cfg.n, maps[-1], b.window)
+    torch.cuda.synchronize()
+    if Bd.trim_status(scratch) != (0, 0):
+        raise RuntimeError("device status after the eager pass")
+    st = torch.cuda.current_stream()
+    L = Bd.lib()
+    state = {"i": 0}
+
+    def step():
+        e = state["i"] % E
+        state["i"] += 1
+        Bd._check(L.qe_diag_tiers(Bd._ptr(maps[e]), Bd._ptr(diag.prev), Bd._ptr(diag.flags), U, Wn,
+                                  1 if e == 0 else 0, Bd._ptr(diag.counters), Bd._stream()), "qe_diag_tiers")
+        Bd.diag_fmm(q, K, cfg.n, maps[e], b.window, fmm, scratch)
+
+    fmm_only = lambda: Bd.diag_fmm(q, K, cfg.n, maps[-1], b.window, fmm, scratch)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    with ClockSampler(0) as clk:
+        ms = _timed(step, args.steps, flush, st)
+        fm = _timed(fmm_only, args.steps, flush, st)
+    step_s = sum(ms) / 1e3 / args.steps
+    fmm_s = statistics.mean(fm) / 1e3
+    alg = U * cfg.n * b.D * 2 + q.numel() * 2 + U * Wn + U * 4  # ghost keys, q, tier map, result
+    # e2e: each step's q and tier map from pinned host memory, FMM and counters back
+    qh, mh = q.cpu().pin_memory(), maps.cpu().pin_memory()
+    fh = torch.empty(fmm.shape, dtype=fmm.dtype, pin_memory=True)
+    ch = torch.empty(diag.counters.shape, dtype=diag.counters.dtype, pin_memory=True)
+    e2e_ms = []
+    for i in range(min(args.steps, 64)):
+        flush.zero_()
+        torch.cuda.synchronize()
+        ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ea.record(st)
+        e = state["i"] % E
+        q.copy_(qh, non_blocking=True)
+        maps[e].copy_(mh[e], non_blocking=True)
+        step()
+        fh.copy_(fmm, non_blocking=True)
+        ch.copy_(diag.counters, non_blocking=True)
+        eb.record(st)
+        eb.synchronize()
+        e2e_ms.append(ea.elapsed_time(eb))
+    summary = diag.summary()
+    line = {
+        "metric": "QEvict diagnostic updates/sec (future missed mass over a 32K ghost cache + churn/LIR, batch 8)",
+        "value": 1.0 / step_s, "unit": "diagnostic updates/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{cfg.name}: B={b.B}, Hq={b.Hq}, Hkv={b.Hkv}, D={b.D}, ghost cache of {cfg.n} "
+                               f"keys per kv head, window {b.window}, {E}-event routing-like tier history "
+                               f"({b.full_windows} full / {b.int2_windows} INT2 windows, rest evicted)",
+                   "l2": "flushed before every step (512 MiB write), outside the timed region"},
+        "roofline": {"kernel": "fmm_partial_kernel + fmm_combine_kernel, timed alone through qe_diag_fmm",
+                     "bound": "hbm", "achieved": alg / fmm_s / 1e9, "peak": hbm, "unit": "GB/s",
+                     "frac": alg / fmm_s / 1e9 / hbm, "peak_kind": f"{hbm_kind} (MEASURED_PEAKS.json hbm_gbs)",
+                     "traffic": None, "algorithmic_bytes": alg},
+        "secondary": {"fmm_ms": fmm_s * 1e3, "fmm_share_of_step": fmm_s / step_s,
+                      "fmm_mean_over_units_last_event": float(fmm.mean()),
+                      "churn": summary["churn"], "lir": summary["lir"]},
+        "cpu_baseline": cpu,
+        "e2e": {"value": len(e2e_ms) / (sum(e2e_ms) / 1e3), "unit": "diagnostic updates/s",
+                "h2d_bytes_per_step": q.numel() * 2 + U * Wn,
+                "d2h_bytes_per_step": fmm.numel() * 4 + diag.counters.numel() * 8, "steps": len(e2e_ms)},
+        "clocks": clk.summary(),
+        "gpu_launches": args.steps * 3 + args.steps * 2,  # step: tiers + FMM partial + combine; FMM alone
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
@@ -699,8 +807,9 @@ def main():
     ap.add_argument("--max-splits", type=int, default=32)
     ap.add_argument("--e2e-steps", type=int, default=640)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["c2", "c3", "c4"], default="c2",
-                    help="c2: tiered decode (the default bench); c3: CriticalKV selection; c4: DBTrimKV trim")
+    ap.add_argument("--workload", choices=["c2", "c3", "c4", "diag"], default="c2",
+                    help="c2: tiered decode (the default bench); c3: CriticalKV selection; c4: DBTrimKV trim; "
+                         "diag: QEvict diagnostics (future missed mass, churn, LIR) at the c2 shape")
     ap.add_argument("--profile-steps", type=int, default=0,
                     help="run only this many eager decode steps after the prefill, then exit")
     args = ap.parse_args()
@@ -714,7 +823,7 @@ def main():
         return
     if args.workload != "c2":
         if rank == 0:
-            (run_c3 if args.workload == "c3" else run_c4)(args)
+            {"c3": run_c3, "c4": run_c4, "diag": run_diag}[args.workload](args)
         return
     if world > 1:
         import datetime

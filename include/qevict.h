@@ -279,6 +279,53 @@ QE_API int qe_trim_global_topm(const float* beta, const int32_t* pos, const int3
                                int32_t* new_lengths, void* scratch, size_t scratch_bytes,
                                qe_stream_t stream);
 
+/* qe_diag_tiers - selection churn and global latent importance reactivation between two
+ * consecutive routing events ("Resumo Técnico: QEvict", Principais Contribuições 1: Churn de
+ * Seleção, LIR Global). The active set is the full-precision tier.
+ *   tiers [dev, uint8]: [units][W] QE_TIER_* of every window after this event (a context's
+ *     win_tier array, or any map in that encoding; EVICTED also marks windows not created yet).
+ *   prev [dev, uint8]: [units][W] the map at the previous event; overwritten with `tiers`.
+ *   flags [dev, uint8]: [units][W] per-window history (bit 0: has left the full tier, bit 1:
+ *     has re-entered it); owned by the caller, kept across calls.
+ *   first: nonzero on the first event of a run: copies tiers to prev, zeroes flags, counts
+ *     nothing (counters may then be NULL).
+ *   counters [dev, int64]: [units][6], ADDED to (the caller zeroes them once):
+ *     0 live_prev  windows FULL or INT2 at the previous event
+ *     1 changed    of those, windows whose tier differs now
+ *     2 exits      windows FULL before and not FULL now
+ *     3 reentries  windows not FULL before, FULL now, that had exited at an earlier event
+ *     4 windows_exited, 5 windows_reentered: first exit / first re-entry of a window
+ *   churn = sum(changed) / sum(live_prev); LIR = sum(windows_reentered) / sum(windows_exited),
+ *   pooled over units and events.
+ * QE_ERR_INVALID_ARG for a null pointer or a non-positive size. Asynchronous on `stream`;
+ * allocates nothing. */
+QE_API int qe_diag_tiers(const uint8_t* tiers, uint8_t* prev, uint8_t* flags, int units, int W,
+                         int first, long long* counters, qe_stream_t stream);
+
+/* qe_diag_fmm - future missed mass of one decode step ("Resumo Técnico: QEvict", Principais
+ * Contribuições 1: Massa Perdida Futura): for each (b, kvh) unit, the share of the ghost
+ * attention that falls on tokens of evicted windows, averaged over the unit's G query heads:
+ *   fmm[u] = (1/G) sum_h sum_{i < n, tiers[u][i / window] == EVICTED} p_{h,i},
+ *   p_{h,.} = softmax_i(q_h . K_i / sqrt(D)) over all n tokens of the ghost cache; 0 if n == 0.
+ *   q [dev]: [B][Hq][D] dtype, query head h = kvh * G + g of unit (b, kvh).
+ *   K_ghost [dev]: [B][Hkv][n_stride][D] dtype, 16-byte aligned: every token's key at its
+ *     original precision (the caller appends each step's key; evicted windows stay in it).
+ *   tiers [dev, uint8]: [B*Hkv][W] QE_TIER_*; token i lies in window i / window.
+ *   fmm_out [dev, float]: [B*Hkv].
+ *   scratch [dev]: qe_diag_fmm_scratch_bytes(B*Hkv, G) bytes, 16-byte aligned, not shared by
+ *     concurrent calls; its first 8 bytes receive a status word {int32 code, int32 detail}: 0,
+ *     or QE_ERR_TIMEOUT if a bounded wait gave up (detail = where and the unit).
+ * Host-side errors (returned, nothing launched): QE_ERR_INVALID_ARG for a null or misaligned
+ * pointer, Hq not a multiple of Hkv, n < 0, n_stride < n, ceil(n / window) > W or a bad dtype;
+ * QE_ERR_UNSUPPORTED_SHAPE for D not in {64, 128}, G not in {1, 2, 4, 5, 8} or
+ * B * Hkv * n_stride + 16 >= 2^31; QE_ERR_WORKSPACE for a small scratch. Asynchronous on `stream`;
+ * allocates nothing. */
+QE_API size_t qe_diag_fmm_scratch_bytes(int units, int G);
+QE_API int qe_diag_fmm(const void* q, const void* K_ghost, long long n_stride, int n,
+                       const uint8_t* tiers, int W, int window, int B, int Hq, int Hkv, int D,
+                       int dtype, float* fmm_out, void* scratch, size_t scratch_bytes,
+                       qe_stream_t stream);
+
 /* qe_status - copy the device status word to the host (synchronises the context's last
  * stream) and return the first recorded error, or QE_OK. *detail (may be NULL) receives the
  * failing index or unit. */

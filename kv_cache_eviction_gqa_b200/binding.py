@@ -69,6 +69,9 @@ def lib():
             "qe_trim_scratch_bytes": (sz, [i, i]),
             "qe_trim_global_topm": (i, [vp, vp, vp, vp, i, i, i, i, i, i, ll, vp, vp, vp, vp, vp,
                                         vp, sz, vp]),
+            "qe_diag_tiers": (i, [vp, vp, vp, i, i, i, vp, vp]),
+            "qe_diag_fmm_scratch_bytes": (sz, [i, i]),
+            "qe_diag_fmm": (i, [vp, vp, ll, i, vp, i, i, i, i, i, i, i, vp, vp, sz, vp]),
             "qe_status": (i, [vp, C.POINTER(C.c_int)]),
             "qe_step_index": (i, [vp]),
             "qe_length": (i, [vp]),
@@ -393,3 +396,67 @@ def criticalkv_select(q_obs: torch.Tensor, K: torch.Tensor, V: torch.Tensor, W_O
                                       _ptr(N), _ptr(idx), _ptr(scratch), scratch.numel(),
                                       _stream(stream)), "qe_criticalkv_select")
     return A, N, idx, scratch
+
+
+class TierDiagnostics:
+    """Selection churn and global LIR over the routing events of a run (qe_diag_tiers).
+
+    Holds the previous tier map, the per-window history flags and the int64 counters
+    [units][6] (live_prev, changed, exits, reentries, windows_exited, windows_reentered) on the
+    device. Call ``update(tiers)`` after every routing event with the [units][W] uint8 tier map
+    (e.g. ``QEvictContext.state()["win_tier"]``); the first call only records the map.
+    """
+
+    def __init__(self, units: int, W: int, device):
+        self.units, self.W = units, W
+        self.prev = torch.zeros((units, W), dtype=torch.uint8, device=device)
+        self.flags = torch.zeros((units, W), dtype=torch.uint8, device=device)
+        self.counters = torch.zeros((units, 6), dtype=torch.int64, device=device)
+        self.events = 0
+
+    def update(self, tiers: torch.Tensor, stream=None):
+        _need(tiers, "tiers", torch.uint8, (self.units, self.W))
+        _check(lib().qe_diag_tiers(_ptr(tiers), _ptr(self.prev), _ptr(self.flags), self.units, self.W,
+                                   1 if self.events == 0 else 0, _ptr(self.counters), _stream(stream)),
+               "qe_diag_tiers")
+        self.events += 1
+
+    def summary(self) -> dict:
+        """Pooled counts and the two ratios (nan when a denominator is 0); synchronises."""
+        c = self.counters.sum(dim=0).cpu().tolist()
+        keys = ("live_prev", "changed", "exits", "reentries", "windows_exited", "windows_reentered")
+        out = dict(zip(keys, c))
+        out["churn"] = c[1] / c[0] if c[0] else float("nan")
+        out["lir"] = c[5] / c[4] if c[4] else float("nan")
+        return out
+
+
+def diag_fmm_scratch_bytes(units: int, G: int) -> int:
+    return int(lib().qe_diag_fmm_scratch_bytes(units, G))
+
+
+def diag_fmm(q: torch.Tensor, K_ghost: torch.Tensor, n: int, tiers: torch.Tensor, window: int,
+             out=None, scratch=None, stream=None):
+    """Future missed mass of one step (qe_diag_fmm).
+
+    q [B][Hq][D], K_ghost [B][Hkv][n_stride][D] (same dtype; the first n rows of each unit are
+    used), tiers [B*Hkv][W] uint8. Returns (fmm [B*Hkv] float32, scratch); the device status
+    word is scratch[:8] (see trim_status).
+    """
+    _need(q, "q")
+    B, Hq, D = q.shape
+    _need(K_ghost, "K_ghost", q.dtype)
+    _, Hkv, n_stride, _ = K_ghost.shape
+    _need(tiers, "tiers", torch.uint8)
+    U, W = tiers.shape
+    if U != B * Hkv:
+        raise ValueError(f"tiers must have {B * Hkv} rows, got {U}")
+    dev = q.device
+    out = torch.empty(U, dtype=torch.float32, device=dev) if out is None else out
+    _need(out, "out", torch.float32, (U,))
+    if scratch is None:
+        scratch = torch.empty(diag_fmm_scratch_bytes(U, Hq // Hkv), dtype=torch.uint8, device=dev)
+    _check(lib().qe_diag_fmm(_ptr(q), _ptr(K_ghost), n_stride, int(n), _ptr(tiers), W, int(window), B, Hq,
+                             Hkv, D, dtype_code(q.dtype), _ptr(out), _ptr(scratch), scratch.numel(),
+                             _stream(stream)), "qe_diag_fmm")
+    return out, scratch

@@ -375,3 +375,90 @@ def draw_trim_kv_pool(cfg: TrimConfig, n_pages: int, device, dtype):
         b = min(a + step, flat.shape[0])
         flat[a:b] = torch.randn((b - a, cfg.D), generator=g, device=device, dtype=torch.float32).to(dtype)
     return out
+
+
+# --------------------------------------------------------------------------
+# QEvict diagnostics workloads (routing histories and ghost caches)
+# --------------------------------------------------------------------------
+
+# tier encoding of a window (the library's QE_TIER_* values)
+TIER_EVICTED, TIER_INT2, TIER_FULL, TIER_TAIL = 0, 1, 2, 3
+
+
+@dataclass(frozen=True)
+class DiagConfig:
+    """Inputs of the QEvict diagnostics: a history of tier maps over ``events`` routing events
+    and, at the last event, one decode step's queries over a ghost cache that holds every one
+    of the ``n`` tokens' keys at their original precision. Shapes, dtype, key distribution
+    and tier budgets come from ``base``."""
+
+    name: str
+    base: DecodeConfig
+    n: int  # tokens at the last event (the tail window may be incomplete)
+    events: int
+    extra_windows: int = 3  # trailing windows never created: the map row is longer than needed
+    n_pad: int = 0  # ghost-cache rows per unit beyond n (capacity for later tokens)
+
+    @property
+    def W(self) -> int:
+        return -(-self.n // self.base.window) + self.extra_windows
+
+    @property
+    def n_stride(self) -> int:
+        return self.n + self.n_pad
+
+    def scaled(self, **kw) -> "DiagConfig":
+        return dataclasses.replace(self, **kw)
+
+
+# the c2 layer after 20 decode steps: 1024 complete windows of 32 plus a 20-token tail
+DIAG_C2 = DiagConfig("diag_c2_llama8b_32k_b8", C2, n=32768 + 20, events=8)
+
+
+def draw_tier_history(cfg: DiagConfig) -> np.ndarray:
+    """Tier maps [events][B*Hkv][W] uint8 with the structure of a routing history.
+
+    This draws data; it ranks windows by a random priority, not by any attention score. One
+    window completes per event: at event e the first c_e = n // window - (events-1-e) windows
+    are complete, window c_e is the tail (TAIL; at the last event only if n is not a multiple
+    of the window) and later windows do not exist yet (EVICTED). Among the complete windows not
+    evicted at an earlier event, the full_windows of highest priority are FULL, the next
+    int2_windows INT2 and the rest EVICTED for good. A window's priority starts N(0, 1) and
+    moves as p <- 0.8 p + 0.6 N(0, 1) between events, so windows leave and re-enter the full
+    tier.
+    """
+    b = cfg.base
+    U, W, w = b.units, cfg.W, b.window
+    out = np.zeros((cfg.events, U, W), dtype=np.uint8)
+    last_complete = cfg.n // w
+    for u in range(U):
+        r = _rng(b.seed, 0xD1A6, u)
+        prio = r.standard_normal(W)
+        gone = np.zeros(W, dtype=bool)
+        for e in range(cfg.events):
+            if e:
+                prio = 0.8 * prio + 0.6 * r.standard_normal(W)
+            c = max(0, last_complete - (cfg.events - 1 - e))
+            cand = np.nonzero(~gone[:c])[0]
+            order = cand[np.argsort(-prio[cand], kind="stable")]
+            row = out[e, u]
+            row[order[:b.full_windows]] = TIER_FULL
+            row[order[b.full_windows:b.full_windows + b.int2_windows]] = TIER_INT2
+            ev = order[b.full_windows + b.int2_windows:]
+            row[ev] = TIER_EVICTED
+            gone[ev] = True
+            if c < W and (e < cfg.events - 1 or cfg.n % w):
+                row[c] = TIER_TAIL
+    return out
+
+
+def draw_ghost_keys(cfg: DiagConfig, b: int, kvh: int) -> np.ndarray:
+    """Ghost cache of one unit: the keys of all n tokens [n][D] (dtype-exact float32), drawn
+    like the decode prefill cache of ``base`` at context n."""
+    K, _ = draw_unit_cache(cfg.base.scaled(ctx=cfg.n), b, kvh)
+    return K
+
+
+def draw_diag_queries(cfg: DiagConfig) -> np.ndarray:
+    """The step's queries [B][Hq][D]: the first decode step's q of ``base``."""
+    return draw_step_inputs(cfg.base.scaled(steps=1))[0][0]

@@ -30,7 +30,8 @@ def test_header_declares_the_boundary():
     names = declared()
     for must in ("qe_create", "qe_kv_append", "qe_decode_attend_and_score", "qe_route_windows",
                  "qe_quantize_once", "qe_promote", "qe_vwo_l1norm", "qe_criticalkv_select",
-                 "qe_trim_global_topm", "qe_decode_attend_and_score_noalloc"):
+                 "qe_trim_global_topm", "qe_decode_attend_and_score_noalloc", "qe_diag_tiers",
+                 "qe_diag_fmm"):
         assert must in names
 
 
@@ -59,3 +60,9 @@ def test_host_side_argument_errors_need_no_device(libpath):
                                None, None, None, None, 0, None)
     assert rc == B.QE_ERR_INVALID_ARG
     assert L.qe_strerror(B.QE_ERR_WORKSPACE).decode() == "workspace too small"
+    # diagnostics: sizes and argument checks on the host
+    assert L.qe_diag_fmm_scratch_bytes(64, 4) >= 64 * 64 * 4 * 16
+    assert L.qe_diag_fmm_scratch_bytes(0, 4) == 0 and L.qe_diag_fmm_scratch_bytes(1, 9) == 0
+    assert L.qe_diag_tiers(None, None, None, 1, 1, 0, None, None) == B.QE_ERR_INVALID_ARG
+    assert L.qe_diag_fmm(None, None, 1, 0, None, 1, 1, 1, 1, 1, 128, B.QE_BF16, None, None, 0,
+                         None) == B.QE_ERR_INVALID_ARG
