@@ -47,6 +47,8 @@ class ParityReport:
     near_ties: int = 0
     codes_checked: int = 0
     promoted_checked: int = 0
+    max_fmm: float = 0.0
+    diag: dict = field(default_factory=dict)
     notes: list = field(default_factory=list)
 
 
@@ -84,7 +86,15 @@ def _near_tie(unit: O.QEvictUnit, w: int) -> bool:
 
 
 def run_decode_parity(cfg: W.DecodeConfig, check_units=None, steps=None, max_splits=32,
-                      check_every=1, verbose=False) -> ParityReport:
+                      check_every=1, verbose=False, diag=False) -> ParityReport:
+    """Decode sequence on the GPU and in the oracle, compared step by step.
+
+    With diag=True the QEvict diagnostics ride along: after every routing event the context's
+    tier map goes to qe_diag_tiers (the oracle's own tier history to tier_diagnostics, counts
+    compared exactly at the end), and at every step qe_diag_fmm over a ghost cache of the
+    seeded keys, with the tier map in force during that step's attention, is compared with
+    future_missed_mass.
+    """
     dev = "cuda"
     tdt = torch_dtype(cfg.dtype)
     steps = cfg.steps if steps is None else steps
@@ -109,6 +119,15 @@ def run_decode_parity(cfg: W.DecodeConfig, check_units=None, steps=None, max_spl
                                 cfg.int2_windows, cfg.alpha, cfg.dtype, max_ctx)
     rep = ParityReport()
     st = ctx.state()
+    if diag:
+        from kv_cache_eviction_gqa_b200.binding import TierDiagnostics, diag_fmm, trim_status
+        Wn = st["win_tier"].shape[1]
+        tdiag = TierDiagnostics(len(all_units), Wn, dev)
+        tdiag.update(st["win_tier"])
+        o_hist = {u: [unit.tier.copy()] for u, unit in units.items()}
+        ghost = torch.zeros((cfg.B, cfg.Hkv, max_ctx, cfg.D), dtype=tdt, device=dev)
+        ghost[:, :, :cfg.ctx] = K
+        ghost_np = {u: np.concatenate([inp.K[u], np.zeros((steps, cfg.D), np.float32)]) for u in units}
     b1F = int(math.floor(cfg.alpha * cfg.full_windows))
     b1Q = int(math.floor(cfg.alpha * cfg.int2_windows))
     for s in range(steps):
@@ -118,7 +137,13 @@ def run_decode_parity(cfg: W.DecodeConfig, check_units=None, steps=None, max_spl
         # scores before routing, for the selection-property check
         ctx.kv_append(k, v)
         out = ctx.decode_attend_and_score(q)
+        if diag:
+            ghost[:, :, cfg.ctx + s] = k
+            fmm_g, fscr = diag_fmm(q, ghost, cfg.ctx + s + 1, st["win_tier"], cfg.window)
         torch.cuda.synchronize()
+        if diag:
+            assert trim_status(fscr) == (0, 0)
+            fmm_g = fmm_g.cpu().numpy()
         routing = s % cfg.route_every == 0
         g_mass = st["mass"].cpu().numpy().copy()
         g_pert = st["pert"].cpu().numpy().copy()
@@ -139,6 +164,12 @@ def run_decode_parity(cfg: W.DecodeConfig, check_units=None, steps=None, max_spl
                 err = np.abs(og - o_ref[j]).max() / np.abs(o_ref[j]).max()
                 rep.max_out_err = max(rep.max_out_err, err)
                 assert err <= OUT_TOL, f"step {s} unit {u} head {j}: output rel err {err:.3e}"
+            if diag:
+                ghost_np[u][cfg.ctx + s] = inp.k_new[s, b, h]
+                ref = O.future_missed_mass(inp.q[s, b, h * G:(h + 1) * G], ghost_np[u][:cfg.ctx + s + 1],
+                                           unit.tier, cfg.window)
+                assert abs(fmm_g[u] - ref) <= 1e-6 + 1e-4 * ref, f"step {s} unit {u}: fmm {fmm_g[u]} vs {ref}"
+                rep.max_fmm = max(rep.max_fmm, ref)
             if s % check_every == 0 or routing:
                 live = np.nonzero(unit.tier != O.EVICTED)[0]
                 tail = unit.n // cfg.window if unit.n % cfg.window else -1
@@ -201,15 +232,25 @@ def run_decode_parity(cfg: W.DecodeConfig, check_units=None, steps=None, max_spl
                             np.testing.assert_array_equal(pages[pg, 0, t % 16], unit.Kst[w * cfg.window + t])
                             np.testing.assert_array_equal(pages[pg, 1, t % 16], unit.Vst[w * cfg.window + t])
                         rep.promoted_checked += 1
+                if diag:
+                    o_hist[u].append(unit.tier.copy())
                 # tiers agree after replay
                 live_o = {int(w): int(unit.tier[w]) for w in np.nonzero(unit.tier != O.EVICTED)[0]}
                 for w, t in live_o.items():
                     gt = int(g_tier[u, w])
                     assert gt == t or (t in (O.TAIL, O.FULL) and gt in (TIER_TAIL, TIER_FULL)), \
                         f"unit {u} window {w}: tier {gt} vs oracle {t}"
+        if diag and routing:
+            tdiag.update(st["win_tier"])
         ctx._steps_done = s + 1
         rep.steps += 1
         if verbose and (s % 8 == 0):
             print(f"step {s}: out {rep.max_out_err:.2e} mass {rep.max_mass_err:.2e} "
                   f"pert {rep.max_pert_err:.2e} ties {rep.near_ties}")
+    if diag:
+        got = tdiag.counters.cpu().numpy()
+        for u in units:
+            ref = O.tier_diagnostics(o_hist[u])["per_unit"][0]
+            np.testing.assert_array_equal(got[u], ref, err_msg=f"unit {u}: tier diagnostics")
+        rep.diag = tdiag.summary()
     return rep

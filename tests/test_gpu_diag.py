@@ -168,3 +168,19 @@ def test_fmm_full_c2_sampled_units():
     assert np.all((got >= 0) & (got <= 1))
     vals = [_check_unit(cfg, q, Ks, tiers, got, bb, h) for (bb, h) in [(0, 0), (3, 5), (7, 7)]]
     print("c2 fmm sampled", vals, "mean over units", float(got.mean()))
+
+
+ROUTED = [
+    W.C1,
+    W.C5.scaled(name="c5_small", B=1, Hkv=2, Hq=10, ctx=3000, full_windows=5, int2_windows=20,
+                route_every=8, steps=70, hidden=1280),
+]
+
+
+@pytest.mark.parametrize("cfg", ROUTED, ids=[c.name for c in ROUTED])
+def test_diagnostics_over_a_routed_decode_run(cfg):
+    """The diagnostics fed by a context's own routing history (oracle: by its own history)."""
+    from tests.parity_helpers import run_decode_parity
+    rep = run_decode_parity(cfg, diag=True)
+    assert rep.route_events > 0 and rep.max_fmm > 0
+    print(cfg.name, rep.diag, "max fmm", rep.max_fmm, "near-ties", rep.near_ties)
