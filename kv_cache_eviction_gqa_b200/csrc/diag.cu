@@ -291,9 +291,10 @@ int launch_fmm(const void* q, const void* K, long long n_stride, int n, const ui
   CUtensorMap tm;
   e = tc::make_map(&tm, K, std::is_same<T, __nv_bfloat16>::value, D, (uint64_t)(rows > 0 ? rows : 1), 64, 16);
   if (e) return e;
-  // enough splits to fill every resident slot once, never more than the unit's tiles allow
+  // as many splits as keep every CTA in one wave of resident slots (a second, partial wave
+  // would double the pass), never more than the unit's tiles allow
   const int tiles = (n + 15) / 16;
-  int S = (slots_of[dev] + U - 1) / U;
+  int S = slots_of[dev] / U;
   const int cap = (tiles + kFmmWarps - 1) / kFmmWarps;
   if (S > cap) S = cap;
   if (S > kFmmMaxSplits) S = kFmmMaxSplits;
