@@ -185,8 +185,19 @@ __global__ void __launch_bounds__(kFmmWarps * 32)
       MmaOp<T>::run(c1, qa[2 * kc2 + 1][0], 0u, qa[2 * kc2 + 1][1], 0u, kb[2], kb[3]);
     }
     __syncwarp();
-    // lane (g8, t4) holds head g8's scores of tokens 2t4, 2t4+1, 8+2t4, 9+2t4 of the tile
-    const int tok0 = (t0 + warp + kFmmWarps * r) * 16 + 2 * t4;
+    // lane (g8, t4) holds head g8's scores of tokens 2t4, 2t4+1, 8+2t4, 9+2t4 of the tile.
+    // With windows of at least 16 tokens a tile meets at most two windows: one division and
+    // two tier loads per tile (shorter windows take one division per token).
+    const int tile0 = (t0 + warp + kFmmWarps * r) * 16;
+    const int tok0 = tile0 + 2 * t4;
+    int w0 = 0, wb = 0;
+    bool e0 = false, e1 = false;
+    if (a.window >= 16) {
+      w0 = tile0 / a.window;
+      wb = (w0 + 1) * a.window;  // first token of the next window
+      e0 = tier_u[w0] == QE_TIER_EVICTED;
+      e1 = wb < a.n && tier_u[w0 + 1] == QE_TIER_EVICTED;
+    }
     float sc[4] = {c0[0], c0[1], c1[0], c1[1]};
     bool ev[4];
     float mx = -1e30f;
@@ -195,7 +206,10 @@ __global__ void __launch_bounds__(kFmmWarps * 32)
       const int tok = tok0 + (i & 1) + (i >> 1) * 8;
       const bool valid = tok < a.n;
       sc[i] = valid ? sc[i] * a.scale_log2 : -INFINITY;
-      ev[i] = valid && tier_u[tok / a.window] == QE_TIER_EVICTED;
+      if (a.window >= 16)
+        ev[i] = valid && (tok < wb ? e0 : e1);
+      else
+        ev[i] = valid && tier_u[tok / a.window] == QE_TIER_EVICTED;
       mx = fmaxf(mx, sc[i]);
     }
     if (mx > mh) {

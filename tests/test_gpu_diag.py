@@ -118,6 +118,12 @@ FMM_CASES = [
                      n=999, events=7),
     W.DIAG_C2.scaled(name="fmm_tiny_n7", base=W.C1.scaled(full_windows=1, int2_windows=1), n=7, events=1),
     W.DIAG_C2.scaled(name="fmm_one_tile", base=W.C1.scaled(full_windows=1, int2_windows=0), n=48, events=3),
+    # windows that are not a multiple of the 16-key tile: tiles that straddle two windows
+    W.DIAG_C2.scaled(name="fmm_window24", base=W.C1.scaled(window=24, full_windows=6, int2_windows=10),
+                     n=1001, events=5),
+    # windows shorter than a tile: one tier lookup per key
+    W.DIAG_C2.scaled(name="fmm_window7", base=W.C1.scaled(window=7, full_windows=20, int2_windows=30),
+                     n=500, events=4),
 ]
 
 

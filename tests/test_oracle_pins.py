@@ -204,6 +204,30 @@ def test_two_stage_exhaustive(seed):
     assert sorted(best2) == sorted(s2.tolist())
 
 
+def test_two_stage_true_perturbation_rank_informative():
+    """Informative ("Resumo Técnico: CriticalKV", Framework Teórico): over every size-b subset
+    of a small attention problem, the rank of the TwoStage pick by the true perturbation
+    L = ||(o - o_hat) W_O||_1. Nothing is asserted about the rank: the pages bound L from above
+    and give no value for it; the test only prints where the pick falls."""
+    r = _rng(55)
+    n, D, b = 10, 8, 4
+    q = r.standard_normal(D) * 2
+    K = r.standard_normal((n, D))
+    V = r.standard_normal((n, D))
+    Wo = r.standard_normal((D, 16)) / 4
+    _, p = O.attend(q, K, V)
+    norms = O.vwo_l1norm(V, Wo, [0], D)[:, 0]
+    s1, s2 = O.two_stage(np.arange(n), p, p * norms, b, 0.5)
+    pick = sorted(np.concatenate([s1, s2]).tolist())
+    Ls = sorted((O.output_perturbation(q, K, V, list(c), Wo), list(c))
+                for c in itertools.combinations(range(n), b))
+    rank = [c for _, c in Ls].index(pick) + 1
+    L_pick = O.output_perturbation(q, K, V, pick, Wo)
+    assert L_pick >= Ls[0][0] - 1e-12
+    print(f"TwoStage pick ranks {rank} of {len(Ls)} subsets by true L "
+          f"(L = {L_pick:.4f}, best {Ls[0][0]:.4f}, worst {Ls[-1][0]:.4f})")
+
+
 def test_two_stage_small_set_and_ties():
     ids = np.array([3, 1, 2])
     s1, s2 = O.two_stage(ids, np.zeros(4), np.zeros(4), 5, 0.5)
