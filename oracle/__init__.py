@@ -18,6 +18,9 @@ Functions and where they come from (page title, section):
   the perturbation score; "Resumo Técnico: CriticalKV", Algoritmo, Etapas 1-2.
 * ``QEvictUnit`` -- one (batch, kv-head) unit of the window-routed three-tier
   cache; "Resumo Técnico: QEvict", Metodologia and Mecanismos Principais.
+* ``route_global`` -- one routing event under budgets shared by every layer and kv
+  head of a sequence; "Make Each Token Count", Metodologia 3 (Orçamento Global)
+  applied to the window tiers of "Resumo Técnico: QEvict", Metodologia.
 * ``observation_mass`` / ``criticalkv_select`` -- CriticalKV selection with a
   SnapKV-style observation window; "Resumo Técnico: CriticalKV", Algoritmo.
 * ``trim_global_topm`` -- DBTrimKV global budget over r = beta^(t-i);

@@ -29,6 +29,9 @@ Pins (tests that tie each function to something other than itself):
   the lowest flat indices; compared with ``np.argsort`` on tiny sets.
 * output_perturbation -- diagnostic only (parity unpinned: the pages give no
   value for it and the bound theta is not printed).
+* route_global -- one unit reduces to the unit's own routing; budgets covering
+  every window evict nothing; equal scores across units go to the earlier unit;
+  a hand-worked two-unit case (``tests/golden/route_global.txt``).
 * tier_diagnostics -- hand-worked two-unit event sequence in
   ``tests/golden/diag_tiers.txt``; a constant sequence has no change and no exit;
   a window alternating FULL/INT2 counts every exit and re-entry once per event and
@@ -326,6 +329,37 @@ class QEvictUnit:
         if s % route_every == 0:
             routed = self.route()
         return o, routed
+
+
+def route_global(units, full_windows: int, int2_windows: int, alpha: float):
+    """One routing event of a sequence under global budgets across layers and kv heads.
+
+    "Make Each Token Count", Metodologia 3 (Orçamento Global: one budget over every layer and
+    head instead of a fixed share per head) applied to the window tiers of "Resumo Técnico:
+    QEvict", Metodologia: the live (FULL or INT2) windows of all ``units`` compete together,
+    Full = TwoStage(L, F); INT2 = TwoStage(L minus Full, Q); the rest is evicted, and each unit
+    applies its part with the write-once ledger. ``units`` are the QEvictUnit of one sequence
+    in flat order (layer-major, then kv head); window w of unit k has the flat id k * W + w
+    (W windows per unit), and ties go to the lower flat id. Returns the per-unit assignments.
+    """
+    W = len(units[0].tier)
+    mass = np.concatenate([u.mass for u in units])
+    pert = np.concatenate([u.pert for u in units])
+    tiers = np.concatenate([u.tier for u in units])
+    L = np.nonzero((tiers == FULL) | (tiers == INT2))[0]
+    f1, f2 = two_stage(L, mass, pert, full_windows, alpha)
+    full = np.concatenate([f1, f2])
+    rest = np.setdiff1d(L, full, assume_unique=True)
+    q1, q2 = two_stage(rest, mass, pert, int2_windows, alpha)
+    new = {int(j): EVICTED for j in L}
+    new.update({int(j): FULL for j in full})
+    new.update({int(j): INT2 for j in np.concatenate([q1, q2])})
+    per_unit = [dict() for _ in units]
+    for j, t in new.items():
+        per_unit[j // W][j % W] = t
+    for k, u in enumerate(units):
+        u.apply(per_unit[k])
+    return per_unit
 
 
 # ---------------------------------------------------------------------------

@@ -531,3 +531,67 @@ def test_future_missed_mass_closed_forms():
     Kh[:, 0] = np.log(a)
     fmm = O.future_missed_mass(np.array([[2.0, 0, 0, 0]]), Kh, np.array([O.EVICTED, O.FULL]), 2)
     assert abs(fmm - 0.3) < 1e-15
+
+
+# ---------------------------------------------------------------------------
+# global routing across layers ("Make Each Token Count", Metodologia 3, on QEvict's tiers)
+# ---------------------------------------------------------------------------
+
+
+def _scored_units(n_units, seed, n0=48, w=16):
+    units = []
+    for k in range(n_units):
+        u, _ = _unit(seed + k, n0=n0, w=w)
+        units.append(u)
+    return units
+
+
+def test_route_global_golden(golden_dir):
+    vals = {}
+    for line in open(os.path.join(golden_dir, "route_global.txt")):
+        if line.startswith("#") or "|" not in line:
+            continue
+        key, val = (x.strip() for x in line.split("|"))
+        vals[key] = val.split()
+    units = _scored_units(2, 300)  # 3 complete windows each (48 tokens of 16)
+    for k, u in enumerate(units):
+        u.mass[:3] = [float(x) for x in vals[f"mass {k}"]]
+        u.pert[:3] = [float(x) for x in vals[f"pert {k}"]]
+    O.route_global(units, int(vals["F"][0]), int(vals["Q"][0]), float(vals["alpha"][0]))
+    letter = {O.FULL: "F", O.INT2: "Q", O.EVICTED: "E"}
+    for k, u in enumerate(units):
+        assert [letter[int(t)] for t in u.tier[:3]] == vals[f"tiers {k}"]
+
+
+def test_route_global_one_unit_is_the_unit_routing():
+    r = _rng(301)
+    a, b = _scored_units(1, 302, n0=160)[0], _scored_units(1, 302, n0=160)[0]
+    for u in (a, b):
+        u.mass[:10] = r.random(10) if u is a else a.mass[:10]
+        u.pert[:10] = r.random(10) if u is a else a.pert[:10]
+    a.pert[:10] = b.pert[:10] = r.random(10)
+    b.mass[:10] = a.mass[:10]
+    a.F = b.F = 3
+    a.Q = b.Q = 4
+    a.route()
+    O.route_global([b], 3, 4, 0.5)
+    np.testing.assert_array_equal(a.tier, b.tier)
+
+
+def test_route_global_budget_covers_everything_and_ties():
+    units = _scored_units(3, 310)
+    for u in units:
+        u.mass[:3] = 1.0
+        u.pert[:3] = 1.0
+    # budgets for all 9 live windows: nothing evicted, all full
+    O.route_global(units, 9, 0, 0.5)
+    assert all((u.tier[:3] == O.FULL).all() for u in units)
+    # equal scores everywhere: the lower flat ids (earlier units) win both stages
+    units = _scored_units(3, 320)
+    for u in units:
+        u.mass[:3] = 0.5
+        u.pert[:3] = 0.5
+    O.route_global(units, 4, 3, 0.5)
+    assert units[0].tier[:3].tolist() == [O.FULL] * 3 and units[1].tier[0] == O.FULL
+    assert units[1].tier[1:3].tolist() == [O.INT2] * 2 and units[2].tier[0] == O.INT2
+    assert units[2].tier[1:3].tolist() == [O.EVICTED] * 2
