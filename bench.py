@@ -798,6 +798,133 @@ def run_diag(args):
     print(json.dumps(line), flush=True)
 
 
+LAYERS = 32
+
+
+def run_layers(args):
+    """32 layers of the c2 shape decoded together, routed under budgets shared by all layers
+    and kv heads of each sequence (qe_route_windows_global every 16 steps)."""
+    import torch
+
+    from kv_cache_eviction_gqa_b200 import binding as Bd
+    cfg = CFG
+    Lr, B, Hq, Hkv, D, w, G = LAYERS, cfg.B, cfg.Hq, cfg.Hkv, cfg.D, cfg.window, cfg.G
+    dev = torch.device("cuda", 0)
+    t = torch.bfloat16
+    hbm, hbm_kind = measured_peaks()
+    K_steps, W_steps = min(args.steps, 64), max(3, min(args.warmup, 16))
+    F_total = cfg.full_windows * Hkv * Lr
+    Q_total = cfg.int2_windows * Hkv * Lr
+    max_ctx = cfg.ctx + W_steps + K_steps + 1
+    n_win = -(-max_ctx // w)
+    cpu = None
+    if not args.no_cpu_baseline:
+        c2 = cpu_baseline(cfg)
+        cpu = dict(c2, value=c2["value"] / Lr,
+                   sample=c2["sample"] + f"; divided by {Lr} layers (the oracle's per-unit routing stands in "
+                                         "for the global selection, a small part of the step)")
+    g = torch.Generator(device=dev)
+    ctxs, Wos, qs, ks, vs = [], [], [], [], []
+    for l in range(Lr):
+        g.manual_seed(cfg.seed * 104729 + l)
+        Wo = (torch.randn((Hq * D, cfg.hidden), generator=g, device=dev, dtype=torch.float32)
+              / math.sqrt(Hq * D)).to(t)
+        # 4 outlier channels x8 on K and V per (batch, kv head), as in the c2 recipe
+        scale = torch.ones((B, Hkv, 1, D), device=dev)
+        ch = torch.rand((B, Hkv, D), generator=g, device=dev).argsort(dim=-1)[..., :4]
+        scale.scatter_(-1, ch.unsqueeze(2), 8.0)
+        K = (torch.randn((B, Hkv, cfg.ctx, D), generator=g, device=dev, dtype=t) * scale.to(t))
+        V = (torch.randn((B, Hkv, cfg.ctx, D), generator=g, device=dev, dtype=t) * scale.to(t))
+        shape = Bd.ContextShape(B, Hq, Hkv, D, w, cfg.full_windows, cfg.int2_windows, 0, cfg.hidden, max_ctx,
+                                cfg.alpha, slots_per_unit=n_win)
+        c = Bd.QEvictContext(shape, Wo)
+        c.load_prefill(K, V)
+        del K, V
+        ctxs.append(c)
+        Wos.append(Wo)
+        n_s = W_steps + K_steps
+        qs.append(torch.randn((n_s, B, Hq, D), generator=g, device=dev, dtype=t))
+        ks.append(torch.randn((n_s, B, Hkv, D), generator=g, device=dev, dtype=t))
+        vs.append(torch.randn((n_s, B, Hkv, D), generator=g, device=dev, dtype=t))
+    torch.cuda.synchronize()
+    outs = [torch.empty((B, Hq, D), dtype=torch.float32, device=dev) for _ in range(Lr)]
+    Wmax = ctxs[0].layout.max_windows
+    scratch = torch.empty(Bd.route_global_scratch_bytes(Lr, B, Hkv, Wmax), dtype=torch.uint8, device=dev)
+    st = torch.cuda.current_stream()
+    # the calls a serving loop makes, with their arguments marshalled once (shapes were checked
+    # when the tensors were made): the host must not be what paces 32 launches per step
+    lib, sp = Bd.lib(), Bd._stream()
+    call_args = [[(ctxs[l]._h, Bd._ptr(qs[l][s]), Bd._ptr(ks[l][s]), Bd._ptr(vs[l][s]), Bd._ptr(outs[l]), sp)
+                  for l in range(Lr)] for s in range(W_steps + K_steps)]
+
+    def step(s):
+        for a in call_args[s]:
+            rc = lib.qe_decode_step(*a)
+            if rc:
+                raise RuntimeError(f"qe_decode_step failed: {Bd.strerror(rc)}")
+        if s % cfg.route_every == 0:
+            Bd.route_windows_global(ctxs, F_total, Q_total, cfg.alpha, scratch)
+
+    def step_bytes():
+        tot = 0
+        for c in ctxs:
+            sk = c.state()["stacks"].cpu().numpy()
+            nf, nq = int(sk[:, 2].sum()), int(sk[:, 3].sum())
+            tail = c.length - (c.length // w) * w
+            tot += (nf * w * (4 * D + 4 * G) + nq * w * (D + 4 * G) + c.units * tail * 4 * D
+                    + c.units * (G * D * 6 + (nf + nq) // c.units * 16))
+        return tot
+
+    for s in range(W_steps):
+        step(s)
+    torch.cuda.synchronize()
+    for l, c in enumerate(ctxs):
+        if c.status() != (0, 0):
+            raise RuntimeError(f"layer {l}: device status {c.status()} after warm-up")
+    bytes0 = step_bytes()
+    ms = []
+    with ClockSampler(0) as clk:
+        for s in range(W_steps, W_steps + K_steps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(st)
+            step(s)
+            b.record(st)
+            b.synchronize()
+            ms.append(a.elapsed_time(b))
+    bytes1 = step_bytes()
+    for l, c in enumerate(ctxs):
+        if c.status() != (0, 0):
+            raise RuntimeError(f"layer {l}: device status {c.status()}")
+    step_s = sum(ms) / 1e3 / K_steps
+    alg = (bytes0 + bytes1) / 2
+    route_ms = [m for i, m in enumerate(ms) if (W_steps + i) % cfg.route_every == 0]
+    plain_ms = [m for i, m in enumerate(ms) if (W_steps + i) % cfg.route_every]
+    nf_u = [int(x) for x in ctxs[0].state()["stacks"][:, 2].cpu().tolist()]
+    line = {
+        "metric": f"{Lr}-layer decode steps/sec with global routing (32K ctx, batch 8); achieved HBM GB/s vs peak",
+        "value": 1.0 / step_s, "unit": "steps/s", "n_gpus": 1, "steps": K_steps, "warmup": W_steps,
+        "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{Lr} layers of {cfg.name} (B={B}, Hq={Hq}, Hkv={Hkv}, D={D}, 32K prefill, window "
+                               f"{w}); per sequence one budget over all layers and kv heads: {F_total} full + "
+                               f"{Q_total} INT2 windows (the c2 per-head share x {Hkv * Lr}); global routing every "
+                               f"{cfg.route_every} steps; K/V N(0,1) with 4 outlier channels x8 drawn on the "
+                               "device with a seeded generator",
+                   "l2": f"not flushed: the {Lr}-layer working set (about 45 GB) is far larger than L2"},
+        "roofline": {"kernel": "whole step (32 fused decode launches + global routing events)", "bound": "hbm",
+                     "achieved": alg / step_s / 1e9, "peak": hbm, "unit": "GB/s", "frac": alg / step_s / 1e9 / hbm,
+                     "peak_kind": f"{hbm_kind} (MEASURED_PEAKS.json hbm_gbs)", "traffic": None,
+                     "algorithmic_bytes": alg},
+        "secondary": {"routing_step_ms": statistics.mean(route_ms) if route_ms else None,
+                      "plain_step_ms": statistics.mean(plain_ms) if plain_ms else None,
+                      "layer0_full_windows_per_unit_min_max": [min(nf_u), max(nf_u)]},
+        "cpu_baseline": cpu,
+        "clocks": clk.summary(),
+        "gpu_launches": K_steps * Lr + (len(route_ms) * (3 * Lr + 1)),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
@@ -807,9 +934,10 @@ def main():
     ap.add_argument("--max-splits", type=int, default=32)
     ap.add_argument("--e2e-steps", type=int, default=640)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["c2", "c3", "c4", "diag"], default="c2",
+    ap.add_argument("--workload", choices=["c2", "c3", "c4", "diag", "layers"], default="c2",
                     help="c2: tiered decode (the default bench); c3: CriticalKV selection; c4: DBTrimKV trim; "
-                         "diag: QEvict diagnostics (future missed mass, churn, LIR) at the c2 shape")
+                         "diag: QEvict diagnostics (future missed mass, churn, LIR) at the c2 shape; "
+                         "layers: 32 c2-shaped layers under one global budget per sequence")
     ap.add_argument("--profile-steps", type=int, default=0,
                     help="run only this many eager decode steps after the prefill, then exit")
     args = ap.parse_args()
@@ -823,7 +951,7 @@ def main():
         return
     if args.workload != "c2":
         if rank == 0:
-            {"c3": run_c3, "c4": run_c4, "diag": run_diag}[args.workload](args)
+            {"c3": run_c3, "c4": run_c4, "diag": run_diag, "layers": run_layers}[args.workload](args)
         return
     if world > 1:
         import datetime

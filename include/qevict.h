@@ -71,7 +71,7 @@ typedef struct {
   int full_windows;           /* F: full-precision budget per unit (windows)              */
   int int2_windows;           /* Q: INT2 budget per unit (windows)                        */
   float alpha;                /* stage-1 share of each budget (0.5 on the pages)          */
-  int route_every;            /* R: route after attention on decode steps s % R == 0      */
+  int route_every;            /* R: route after attention on decode steps s % R == 0; 0: qe_decode_step never routes (the caller does, e.g. qe_route_windows_global) */
   int hidden;                 /* columns of W_O                                           */
   int max_ctx;                /* capacity in tokens per unit (prefill + decode)           */
   int pages_per_unit;         /* page-pool capacity per unit (>= ceil(prefill/16) + margin)*/
@@ -179,6 +179,32 @@ QE_API int qe_decode_attend_and_score_noalloc(qe_ctx* ctx, const void* q, float*
  * dequant(ledger) rounded to the cache dtype into fresh pages and keep the entry.
  * Per-unit counts of the event land in the layout's route_stats array. */
 QE_API int qe_route_windows(qe_ctx* ctx, qe_stream_t stream);
+
+/* qe_route_windows_global - one routing event under budgets shared by every layer and kv head
+ * of a sequence ("Make Each Token Count", Metodologia 3: Orçamento Global, applied to the
+ * window tiers of "Resumo Técnico: QEvict", Metodologia). For each batch element b, the live
+ * complete windows of all contexts (one per layer, in the order given) and all kv heads compete:
+ *   Full = TwoStage(L_b, full_windows); INT2 = TwoStage(L_b \ Full, int2_windows); the rest
+ *   is evicted. Window w of kv head h of layer l has the flat position (l*Hkv + h)*W + w
+ *   (W = max_windows); equal scores go to the lower position. TwoStage is the rule of
+ *   qe_route_windows with alpha given here. Each context then applies its transitions exactly
+ *   as qe_route_windows does (write-once quantisation, promotion, page and ledger reuse).
+ *   ctxs [host]: n_layers distinct loaded contexts with equal B, Hkv and max_windows; their own
+ *     full_windows / int2_windows are not used. Give each context page and ledger pools large
+ *     enough for the share a unit may receive (e.g. slots_per_unit = max_windows); a unit whose
+ *     pool runs out records QE_ERR_POOL_EXHAUSTED / QE_ERR_LEDGER_FULL in its context's status.
+ *   scratch [dev]: qe_route_global_scratch_bytes(n_layers, B, Hkv, max_windows) bytes,
+ *     256-byte aligned, not shared by concurrent calls.
+ * Host-side errors: QE_ERR_INVALID_ARG (null, repeated or mismatched contexts, negative
+ * budgets, alpha outside [0, 1]), QE_ERR_STATE (a context not loaded), QE_ERR_UNSUPPORTED_SHAPE
+ * (B * n_layers * Hkv * max_windows >= 2^31), QE_ERR_WORKSPACE (small or misaligned scratch).
+ * Use route_every = 0 in the contexts so that qe_decode_step leaves routing to this call.
+ * After it, qe_list_counts gives upper bounds of the per-unit tier sizes. Asynchronous on
+ * `stream`; allocates nothing. */
+QE_API size_t qe_route_global_scratch_bytes(int n_layers, int B, int Hkv, int max_windows);
+QE_API int qe_route_windows_global(qe_ctx* const* ctxs, int n_layers, int full_windows,
+                                   int int2_windows, float alpha, void* scratch,
+                                   size_t scratch_bytes, qe_stream_t stream);
 
 /* qe_decode_step - one whole decode step: kv_append, decode_attend_and_score and, on steps
  * s % R == 0 (s counted from the prefill), route_windows. Arguments as above. */
@@ -334,7 +360,8 @@ QE_API int qe_status(qe_ctx* ctx, int* detail);
 /* qe_step_index - decode steps taken since the last prefill; qe_length - tokens per unit. */
 QE_API int qe_step_index(const qe_ctx* ctx);
 QE_API int qe_length(const qe_ctx* ctx);
-/* qe_list_counts - full-tier and INT2-tier window counts (identical for every unit). */
+/* qe_list_counts - full-tier and INT2-tier window counts (identical for every unit under
+ * per-unit routing; upper bounds over units after qe_route_windows_global). */
 QE_API int qe_list_counts(const qe_ctx* ctx, int* n_full, int* n_int2);
 
 /* qe_strerror - static message for a QE_* code. */

@@ -69,6 +69,8 @@ def lib():
             "qe_trim_scratch_bytes": (sz, [i, i]),
             "qe_trim_global_topm": (i, [vp, vp, vp, vp, i, i, i, i, i, i, ll, vp, vp, vp, vp, vp,
                                         vp, sz, vp]),
+            "qe_route_global_scratch_bytes": (sz, [i, i, i, i]),
+            "qe_route_windows_global": (i, [vp, i, i, i, f, vp, sz, vp]),
             "qe_diag_tiers": (i, [vp, vp, vp, i, i, i, vp, vp]),
             "qe_diag_fmm_scratch_bytes": (sz, [i, i]),
             "qe_diag_fmm": (i, [vp, vp, ll, i, vp, i, i, i, i, i, i, i, vp, vp, sz, vp]),
@@ -460,3 +462,26 @@ def diag_fmm(q: torch.Tensor, K_ghost: torch.Tensor, n: int, tiers: torch.Tensor
                              Hkv, D, dtype_code(q.dtype), _ptr(out), _ptr(scratch), scratch.numel(),
                              _stream(stream)), "qe_diag_fmm")
     return out, scratch
+
+
+def route_global_scratch_bytes(n_layers: int, B: int, Hkv: int, max_windows: int) -> int:
+    return int(lib().qe_route_global_scratch_bytes(n_layers, B, Hkv, max_windows))
+
+
+def route_windows_global(ctxs, full_windows: int, int2_windows: int, alpha: float = 0.5, scratch=None,
+                         stream=None):
+    """One routing event under budgets shared by every layer (context) and kv head of each
+    sequence (qe_route_windows_global). ``ctxs``: the layers' QEvictContext, in layer order.
+    Returns the scratch buffer (reuse it across events)."""
+    if not ctxs:
+        raise ValueError("no contexts")
+    c0 = ctxs[0]
+    W = c0.layout.max_windows
+    if scratch is None:
+        nbytes = route_global_scratch_bytes(len(ctxs), c0.shape.B, c0.shape.Hkv, W)
+        scratch = torch.empty(nbytes, dtype=torch.uint8, device=c0.workspace.device)
+    arr = (C.c_void_p * len(ctxs))(*[c._h.value for c in ctxs])
+    _check(lib().qe_route_windows_global(arr, len(ctxs), int(full_windows), int(int2_windows), float(alpha),
+                                         _ptr(scratch), scratch.numel(), _stream(stream)),
+           "qe_route_windows_global")
+    return scratch

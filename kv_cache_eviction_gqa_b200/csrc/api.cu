@@ -20,7 +20,7 @@ int check_config(const qe_config* c) {
   if (c->window != 16 && c->window != 32 && c->window != 64) return QE_ERR_UNSUPPORTED_SHAPE;
   if (c->full_windows < 0 || c->int2_windows < 0) return QE_ERR_INVALID_ARG;
   if (!(c->alpha >= 0.f && c->alpha <= 1.f)) return QE_ERR_INVALID_ARG;
-  if (c->route_every < 1) return QE_ERR_INVALID_ARG;
+  if (c->route_every < 0) return QE_ERR_INVALID_ARG;  // 0: the caller routes
   if (c->hidden < 1 || c->hidden % 64) return QE_ERR_UNSUPPORTED_SHAPE;
   if (c->max_ctx < c->window) return QE_ERR_INVALID_ARG;
   if (c->pages_per_unit < c->window / QE_PAGE) return QE_ERR_INVALID_ARG;
@@ -230,7 +230,7 @@ QE_API int qe_decode_step(qe_ctx* c, const void* q, const void* k, const void* v
   }
   c->last_stream = st;
   if (c->n - c->complete * c->cfg.window == c->cfg.window && (e = finalize_tail(c, st))) return e;
-  if (c->step % c->cfg.route_every == 0) {
+  if (c->cfg.route_every > 0 && c->step % c->cfg.route_every == 0) {
     e = qe_route_windows(c, s);
     if (e) return e;
   }

@@ -215,6 +215,9 @@ int launch_decode(qe_ctx* c, const void* q, float* out, cudaStream_t st, const v
                   const void* v_new = nullptr);
 int launch_finalize(qe_ctx* c, int tail_win, cudaStream_t st);
 int launch_route(qe_ctx* c, cudaStream_t st);
+// route with the tier of every candidate window given: window w of unit (b, kvh) takes
+// decided[b * dec_stride + kvh * max_windows + w] (QE_TIER_FULL, _INT2 or _EVICTED)
+int launch_route_decided(qe_ctx* c, const uint8_t* decided, size_t dec_stride, cudaStream_t st);
 int launch_set_tier(qe_ctx* c, int unit, const int32_t* ids_host, int n, int tier, cudaStream_t st);
 int launch_vwo(const void* V, int n_groups, int rows, int D, int dtype, const void* W_O, int Hq,
                int Hkv, int hidden, float* out, long long out_group_stride, int32_t* status,

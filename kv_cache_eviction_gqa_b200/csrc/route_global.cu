@@ -1,0 +1,263 @@
+// Window routing under budgets shared by every layer and kv head of a sequence.
+//
+// "Make Each Token Count" - Metodologia 3 (Orçamento Global): one budget over all layers and
+// heads instead of a fixed share per head, applied here to the window tiers of "Resumo Técnico:
+// QEvict" - Metodologia (full / INT2 / evicted), with the two-stage selection of "Resumo
+// Técnico: CriticalKV" - Algoritmo (Etapa 1: floor(alpha * b) by attention mass, Etapa 2: the
+// rest by the perturbation score).
+//
+// One routing event: (1) for every layer (one context each) a kernel copies each live window's
+// cumulative mass and perturbation into the sequence's candidate arrays at the flat position
+// (layer, kv head, window); (2) one CTA per sequence selects Full = TwoStage(L, F) and
+// INT2 = TwoStage(L minus Full, Q) over all candidates by exact radix selections on 64-bit keys
+// (the score's order-preserving bits, then the complement of the flat position, so equal scores
+// go to the lower position); (3) each layer's route kernel applies its part - page and ledger
+// allocation, write-once quantisation, promotion - exactly as for per-unit routing.
+#include <math.h>
+
+#include "qe_internal.cuh"
+
+namespace {
+
+constexpr int kSelThreadsG = 1024;
+constexpr uint8_t kValid = 1, kPick = 2, kFull = 4, kInt2 = 8;
+
+struct GlobArgs {
+  float* mass;       // [B][n] cumulative attention mass of each candidate
+  float* pert;       // [B][n] cumulative perturbation score
+  uint8_t* flag;     // [B][n] kValid | kPick | kFull | kInt2
+  uint8_t* decided;  // [B][n] QE_TIER_* after the selection
+  int n;             // candidates per sequence: layers * Hkv * max_windows
+};
+
+__device__ __forceinline__ uint32_t order_bits(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// higher score first, then the lower flat position; never 0 for a candidate
+__device__ __forceinline__ unsigned long long cand_key(float score, int i) {
+  return ((unsigned long long)order_bits(score) << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)i);
+}
+
+__global__ void glob_keygen_kernel(DevState st, int layer, GlobArgs g) {
+  const int u = blockIdx.x;
+  const int b = u / st.Hkv, kvh = u % st.Hkv;
+  const int nf = st.stacks[u * 4 + 2], nq = st.stacks[u * 4 + 3];
+  const size_t ub = (size_t)u * st.Wmax;
+  const size_t base = (size_t)b * g.n + ((size_t)layer * st.Hkv + kvh) * st.Wmax;
+  for (int i = threadIdx.x; i < nf + nq; i += blockDim.x) {
+    const int win = i < nf ? st.full_list[ub + i] : st.int2_list[ub + i - nf];
+    if (win < 0 || win >= st.Wmax) {
+      qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
+      continue;
+    }
+    g.mass[base + win] = st.mass[ub + win];
+    g.pert[base + win] = st.pert[ub + win];
+    g.flag[base + win] = kValid;
+  }
+}
+
+struct SelSh {
+  unsigned int hist[256];
+  int ctl[3];
+  int red[kSelThreadsG / 32];
+};
+
+__device__ int block_count(int v, SelSh& sh) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if ((threadIdx.x & 31) == 0) sh.red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  int t = 0;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += sh.red[w];
+  __syncthreads();
+  return t;
+}
+
+// Threshold of the k largest keys (1 <= k <= number of non-zero keys; non-zero keys distinct):
+// key(i) is among them iff key(i) != 0 and (key(i) >> shift) >= (prefix >> shift). Most
+// significant 8-bit digit first; a pass ends the search when the digit that holds the k-th key
+// holds exactly the keys still needed.
+template <typename KeyFn>
+__device__ void topk_threshold(int n, int k, KeyFn key, SelSh& sh, unsigned long long* prefix_out, int* shift_out) {
+  unsigned long long prefix = 0;
+  int shift = 64;
+  for (int pass = 0; pass < 8; ++pass) {
+    const int sft = 56 - 8 * pass;
+    for (int d = threadIdx.x; d < 256; d += blockDim.x) sh.hist[d] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const unsigned long long kk = key(i);
+      if (kk != 0 && (shift == 64 || (kk >> shift) == (prefix >> shift)))
+        atomicAdd(&sh.hist[(kk >> sft) & 255], 1u);
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      // lane l owns digits 255 - 8l .. 248 - 8l, highest first
+      const int l = threadIdx.x;
+      uint32_t c[8], loc = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        c[j] = sh.hist[255 - 8 * l - j];
+        loc += c[j];
+      }
+      uint32_t inc = loc;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (l >= o) inc += y;
+      }
+      long long above = (long long)(inc - loc);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (above < k && above + c[j] >= k) {
+          sh.ctl[0] = 255 - 8 * l - j;
+          sh.ctl[1] = (int)above;
+          sh.ctl[2] = (int)c[j];
+        }
+        above += c[j];
+      }
+    }
+    __syncthreads();
+    k -= sh.ctl[1];
+    prefix |= (unsigned long long)sh.ctl[0] << sft;
+    shift = sft;
+    const bool done = sh.ctl[2] == k;
+    __syncthreads();
+    if (done) break;
+  }
+  *prefix_out = prefix;
+  *shift_out = shift;
+}
+
+// TwoStage(members, b) with stage-1 share b1: the chosen candidates get `out` in their flag
+template <typename MemberFn>
+__device__ void two_stage_global(int n, int b, int b1, MemberFn member, const float* mass, const float* pert,
+                                 uint8_t* flag, uint8_t out, SelSh& sh) {
+  int cnt_local = 0;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) cnt_local += member(i) ? 1 : 0;
+  const int cnt = block_count(cnt_local, sh);
+  if (cnt <= b) {
+    for (int i = threadIdx.x; i < n; i += blockDim.x)
+      if (member(i)) flag[i] |= out;
+    __syncthreads();
+    return;
+  }
+  unsigned long long P;
+  int S;
+  if (b1 > 0) {
+    auto k1 = [&](int i) -> unsigned long long { return member(i) ? cand_key(mass[i], i) : 0ull; };
+    topk_threshold(n, b1, k1, sh, &P, &S);
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const unsigned long long kk = k1(i);
+      if (kk != 0 && (kk >> S) >= (P >> S)) flag[i] |= kPick;
+    }
+    __syncthreads();
+  }
+  if (b - b1 > 0) {
+    auto k2 = [&](int i) -> unsigned long long {
+      return (member(i) && !(flag[i] & kPick)) ? cand_key(pert[i], i) : 0ull;
+    };
+    topk_threshold(n, b - b1, k2, sh, &P, &S);
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const unsigned long long kk = k2(i);
+      if (kk != 0 && (kk >> S) >= (P >> S)) flag[i] |= out;
+    }
+    __syncthreads();
+  }
+  for (int i = threadIdx.x; i < n; i += blockDim.x)
+    if (flag[i] & kPick) flag[i] = (uint8_t)((flag[i] & ~kPick) | out);
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kSelThreadsG) glob_select_kernel(GlobArgs g, int F, int F1, int Q, int Q1) {
+  __shared__ SelSh sh;
+  const size_t base = (size_t)blockIdx.x * g.n;
+  const float* mass = g.mass + base;
+  const float* pert = g.pert + base;
+  uint8_t* flag = g.flag + base;
+  uint8_t* decided = g.decided + base;
+  const int n = g.n;
+  two_stage_global(n, F, F1, [&](int i) { return (flag[i] & kValid) != 0; }, mass, pert, flag, kFull, sh);
+  two_stage_global(n, Q, Q1, [&](int i) { return (flag[i] & (kValid | kFull)) == kValid; }, mass, pert, flag,
+                   kInt2, sh);
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const uint8_t f = flag[i];
+    decided[i] = (f & kFull) ? QE_TIER_FULL : ((f & kInt2) ? QE_TIER_INT2 : QE_TIER_EVICTED);
+  }
+}
+
+struct GlobLayout {
+  size_t mass, pert, flag, decided, total;
+};
+
+GlobLayout glob_layout(int n_layers, int B, int Hkv, int max_windows) {
+  const size_t n = (size_t)n_layers * Hkv * max_windows * B;
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  GlobLayout L{};
+  L.mass = 0;
+  L.pert = up(L.mass + n * 4);
+  L.flag = up(L.pert + n * 4);
+  L.decided = up(L.flag + n);
+  L.total = up(L.decided + n);
+  return L;
+}
+
+}  // namespace
+
+extern "C" QE_API size_t qe_route_global_scratch_bytes(int n_layers, int B, int Hkv, int max_windows) {
+  if (n_layers < 1 || B < 1 || Hkv < 1 || max_windows < 1) return 0;
+  return glob_layout(n_layers, B, Hkv, max_windows).total;
+}
+
+extern "C" QE_API int qe_route_windows_global(qe_ctx* const* ctxs, int n_layers, int full_windows,
+                                              int int2_windows, float alpha, void* scratch,
+                                              size_t scratch_bytes, qe_stream_t stream) {
+  if (!ctxs || n_layers < 1 || !scratch || full_windows < 0 || int2_windows < 0) return QE_ERR_INVALID_ARG;
+  if (!(alpha >= 0.f && alpha <= 1.f)) return QE_ERR_INVALID_ARG;
+  const qe_ctx* c0 = ctxs[0];
+  for (int l = 0; l < n_layers; ++l) {
+    const qe_ctx* c = ctxs[l];
+    if (!c) return QE_ERR_INVALID_ARG;
+    if (!c->loaded) return QE_ERR_STATE;
+    if (c->cfg.B != c0->cfg.B || c->cfg.Hkv != c0->cfg.Hkv || c->lay.max_windows != c0->lay.max_windows)
+      return QE_ERR_INVALID_ARG;
+    for (int m = 0; m < l; ++m)
+      if (ctxs[m] == c) return QE_ERR_INVALID_ARG;  // a layer listed twice
+  }
+  const int B = c0->cfg.B, Hkv = c0->cfg.Hkv, Wmax = c0->lay.max_windows;
+  const long long n = (long long)n_layers * Hkv * Wmax;
+  if (n * B >= (1ll << 31)) return QE_ERR_UNSUPPORTED_SHAPE;
+  const GlobLayout L = glob_layout(n_layers, B, Hkv, Wmax);
+  if (!qe_aligned(scratch, 256) || scratch_bytes < L.total) return QE_ERR_WORKSPACE;
+  uint8_t* base = static_cast<uint8_t*>(scratch);
+  GlobArgs g{};
+  g.mass = reinterpret_cast<float*>(base + L.mass);
+  g.pert = reinterpret_cast<float*>(base + L.pert);
+  g.flag = base + L.flag;
+  g.decided = base + L.decided;
+  g.n = (int)n;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int F1 = (int)floor((double)alpha * full_windows);
+  const int Q1 = (int)floor((double)alpha * int2_windows);
+  QE_CUDA_TRY(cudaMemsetAsync(g.flag, 0, (size_t)n * B, st));
+  for (int l = 0; l < n_layers; ++l) {
+    const DevState s = make_state(ctxs[l]);
+    glob_keygen_kernel<<<s.U, 256, 0, st>>>(s, l, g);
+    QE_CUDA_TRY(cudaGetLastError());
+  }
+  glob_select_kernel<<<B, kSelThreadsG, 0, st>>>(g, full_windows, F1, int2_windows, Q1);
+  QE_CUDA_TRY(cudaGetLastError());
+  for (int l = 0; l < n_layers; ++l) {
+    qe_ctx* c = ctxs[l];
+    const int e = launch_route_decided(c, g.decided + (size_t)l * Hkv * Wmax, (size_t)n, st);
+    if (e) return e;
+    // per-unit tier sizes are no longer equal across units: keep upper bounds
+    const int tot = c->n_full_max + c->n_int2_max;
+    c->n_full_max = tot < full_windows ? tot : full_windows;
+    c->n_int2_max = tot < int2_windows ? tot : int2_windows;
+    c->last_stream = st;
+  }
+  return QE_OK;
+}

@@ -168,11 +168,14 @@ struct RouteArgs {
   int32_t* plist;   // [U][Wmax] windows to promote
   int32_t* xcount;  // [U][4]
   int F, Q, F1, Q1; // budgets and their stage-1 shares floor(alpha*b)
-  int mode;         // 0: two-stage routing; 1: explicit targets for one unit
+  int mode;         // 0: two-stage routing; 1: explicit targets for one unit; 2: decided tiers
   int unit;         // mode 1
   const int32_t* ids;  // mode 1: window ids
   int n_ids;           // mode 1
   int target;          // mode 1: QE_TIER_INT2 or QE_TIER_FULL
+  // mode 2: new tier of window w of unit (b, kvh) at decided[b * dec_stride + kvh * Wmax + w]
+  const uint8_t* decided;
+  size_t dec_stride;
 };
 
 // Sort N 64-bit keys in shared memory in descending order (bitonic network, N a power of 2).
@@ -291,6 +294,18 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
     two_stage_select(n, N, cand, km, kp, inset, sel, s1, a.Q, a.Q1, ibuf, key);
     for (int i = threadIdx.x; i < n; i += blockDim.x)
       if (sel[i]) newt[i] = QE_TIER_INT2;
+  } else if (a.mode == 2) {
+    // tiers decided by a selection over several contexts (global budgets)
+    const uint8_t* dec = a.decided + (size_t)(u / st.Hkv) * a.dec_stride + (size_t)(u % st.Hkv) * st.Wmax;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const int t = dec[cand[i]];
+      if (t == QE_TIER_FULL || t == QE_TIER_INT2 || t == QE_TIER_EVICTED) {
+        newt[i] = (uint8_t)t;
+      } else {
+        newt[i] = oldt[i];
+        qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
+      }
+    }
   } else {
     for (int i = threadIdx.x; i < n; i += blockDim.x) newt[i] = oldt[i];
     __syncthreads();
@@ -668,6 +683,24 @@ int launch_route(qe_ctx* c, cudaStream_t s) {
   a.Q1 = (int)floor((double)c->cfg.alpha * a.Q);
   a.mode = 0;
   a.unit = -1;
+  const size_t smem = route_smem(st);
+  if (int e = route_smem_attr(smem, st.Wmax)) return e;
+  route_kernel<<<st.U, kRouteThreads, smem, s>>>(a);
+  QE_CUDA_TRY(cudaGetLastError());
+  return apply_dispatch(c, st, -1, s);
+}
+
+int launch_route_decided(qe_ctx* c, const uint8_t* decided, size_t dec_stride, cudaStream_t s) {
+  DevState st = make_state(c);
+  RouteArgs a{};
+  a.st = st;
+  a.xlist = c->xlist;
+  a.plist = c->plist;
+  a.xcount = c->xcount;
+  a.mode = 2;
+  a.unit = -1;
+  a.decided = decided;
+  a.dec_stride = dec_stride;
   const size_t smem = route_smem(st);
   if (int e = route_smem_attr(smem, st.Wmax)) return e;
   route_kernel<<<st.U, kRouteThreads, smem, s>>>(a);

@@ -340,7 +340,8 @@ def route_global(units, full_windows: int, int2_windows: int, alpha: float):
     Full = TwoStage(L, F); INT2 = TwoStage(L minus Full, Q); the rest is evicted, and each unit
     applies its part with the write-once ledger. ``units`` are the QEvictUnit of one sequence
     in flat order (layer-major, then kv head); window w of unit k has the flat id k * W + w
-    (W windows per unit), and ties go to the lower flat id. Returns the per-unit assignments.
+    (W windows per unit), and ties go to the lower flat id. Returns the per-unit assignments
+    and the selection itself (candidates, the picks of each stage, the flat scores).
     """
     W = len(units[0].tier)
     mass = np.concatenate([u.mass for u in units])
@@ -359,7 +360,7 @@ def route_global(units, full_windows: int, int2_windows: int, alpha: float):
         per_unit[j // W][j % W] = t
     for k, u in enumerate(units):
         u.apply(per_unit[k])
-    return per_unit
+    return per_unit, dict(L=L, full=(f1, f2), int2=(q1, q2), mass=mass, pert=pert, W=W)
 
 
 # ---------------------------------------------------------------------------

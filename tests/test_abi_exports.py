@@ -66,3 +66,7 @@ def test_host_side_argument_errors_need_no_device(libpath):
     assert L.qe_diag_tiers(None, None, None, 1, 1, 0, None, None) == B.QE_ERR_INVALID_ARG
     assert L.qe_diag_fmm(None, None, 1, 0, None, 1, 1, 1, 1, 1, 128, B.QE_BF16, None, None, 0,
                          None) == B.QE_ERR_INVALID_ARG
+    # global routing: sizes and argument checks on the host
+    assert L.qe_route_global_scratch_bytes(32, 8, 8, 1025) >= 32 * 8 * 8 * 1025 * 10
+    assert L.qe_route_global_scratch_bytes(0, 8, 8, 1025) == 0
+    assert L.qe_route_windows_global(None, 1, 1, 1, 0.5, None, 0, None) == B.QE_ERR_INVALID_ARG
