@@ -166,3 +166,39 @@ def test_global_budget_covering_everything_evicts_nothing():
         route_windows_global([ctxs[0], c3], 4, 4)
     with pytest.raises(RuntimeError, match="invalid"):
         route_windows_global([ctxs[0], ctxs[0]], 4, 4)
+
+
+def test_one_layer_one_kv_head_equals_per_unit_routing():
+    """With one layer and one kv head per sequence the global candidates are exactly one unit's
+    windows, so qe_route_windows_global must reproduce qe_route_windows tier for tier."""
+    from kv_cache_eviction_gqa_b200.binding import ContextShape, QEvictContext, route_windows_global
+    cfg = W.C2.scaled(name="one", B=3, Hkv=1, Hq=4, ctx=1500, full_windows=7, int2_windows=12, steps=24,
+                      hidden=512, seed=2500)
+    inp = W.draw_decode_inputs(cfg)
+    t = torch.bfloat16
+    K = torch.from_numpy(inp.K).view(cfg.B, 1, cfg.ctx, cfg.D).to("cuda", t)
+    V = torch.from_numpy(inp.V).view(cfg.B, 1, cfg.ctx, cfg.D).to("cuda", t)
+    Wo = torch.from_numpy(inp.W_O).to("cuda", t)
+    ctxs = []
+    for _ in range(2):
+        shape = ContextShape(cfg.B, cfg.Hq, 1, cfg.D, cfg.window, cfg.full_windows, cfg.int2_windows, 0,
+                             cfg.hidden, cfg.ctx + cfg.steps, slots_per_unit=80)
+        c = QEvictContext(shape, Wo)
+        c.workspace.zero_()
+        c.load_prefill(K, V)
+        ctxs.append(c)
+    local, glob = ctxs
+    for s in range(cfg.steps):
+        q = torch.from_numpy(inp.q[s]).to("cuda", t)
+        k = torch.from_numpy(inp.k_new[s]).to("cuda", t)
+        v = torch.from_numpy(inp.v_new[s]).to("cuda", t)
+        o1, o2 = local.decode_step(q, k, v), glob.decode_step(q, k, v)
+        if s % 4 == 0:
+            local.route_windows()
+            route_windows_global([glob], cfg.full_windows, cfg.int2_windows, cfg.alpha)
+        torch.cuda.synchronize()
+        assert local.status() == (0, 0) and glob.status() == (0, 0)
+        assert torch.equal(o1, o2), f"step {s}: outputs differ"
+        sl, sg = local.state(), glob.state()
+        for name in ("win_tier", "win_slot", "mass", "pert", "stacks"):
+            assert torch.equal(sl[name], sg[name]), f"step {s}: {name} differs"
