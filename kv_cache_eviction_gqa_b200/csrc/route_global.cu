@@ -6,13 +6,15 @@
 // Técnico: CriticalKV" - Algoritmo (Etapa 1: floor(alpha * b) by attention mass, Etapa 2: the
 // rest by the perturbation score).
 //
-// One routing event: (1) for every layer (one context each) a kernel copies each live window's
-// cumulative mass and perturbation into the sequence's candidate arrays at the flat position
-// (layer, kv head, window); (2) one CTA per sequence selects Full = TwoStage(L, F) and
-// INT2 = TwoStage(L minus Full, Q) over all candidates by exact radix selections on 64-bit keys
-// (the score's order-preserving bits, then the complement of the flat position, so equal scores
-// go to the lower position); (3) each layer's route kernel applies its part - page and ledger
-// allocation, write-once quantisation, promotion - exactly as for per-unit routing.
+// One routing event: (1) for every layer (one context each) a kernel appends each live window's
+// cumulative mass, perturbation and flat position (layer, kv head, window) to its sequence's
+// candidate list (a unit claims its range with one atomic add, so the list holds live windows
+// only, in no particular order); (2) one CTA per sequence selects Full = TwoStage(L, F) and
+// INT2 = TwoStage(L minus Full, Q) over the list by exact radix selections on 64-bit keys (the
+// score's order-preserving bits, then the complement of the flat position, so equal scores go to
+// the lower position and the result does not depend on the list order) and writes each chosen
+// tier at the window's flat position; (3) each layer's route kernel applies its part - page and
+// ledger allocation, write-once quantisation, promotion - exactly as for per-unit routing.
 #include <math.h>
 
 #include "qe_internal.cuh"
@@ -20,14 +22,16 @@
 namespace {
 
 constexpr int kSelThreadsG = 1024;
-constexpr uint8_t kValid = 1, kPick = 2, kFull = 4, kInt2 = 8;
+constexpr uint8_t kPick = 2, kFull = 4, kInt2 = 8;
 
 struct GlobArgs {
-  float* mass;       // [B][n] cumulative attention mass of each candidate
-  float* pert;       // [B][n] cumulative perturbation score
-  uint8_t* flag;     // [B][n] kValid | kPick | kFull | kInt2
-  uint8_t* decided;  // [B][n] QE_TIER_* after the selection
-  int n;             // candidates per sequence: layers * Hkv * max_windows
+  float* mass;       // [B][n] candidate list: cumulative attention mass,
+  float* pert;       // [B][n] cumulative perturbation score,
+  int32_t* pos;      // [B][n] flat position (layer * Hkv + kv head) * max_windows + window,
+  uint8_t* flag;     // [B][n] kPick | kFull | kInt2
+  int32_t* count;    // [B] list lengths
+  uint8_t* decided;  // [B][n] QE_TIER_* by flat position (EVICTED where not chosen)
+  int n;             // flat positions per sequence: layers * Hkv * max_windows
 };
 
 __device__ __forceinline__ uint32_t order_bits(float f) {
@@ -45,16 +49,27 @@ __global__ void glob_keygen_kernel(DevState st, int layer, GlobArgs g) {
   const int b = u / st.Hkv, kvh = u % st.Hkv;
   const int nf = st.stacks[u * 4 + 2], nq = st.stacks[u * 4 + 3];
   const size_t ub = (size_t)u * st.Wmax;
-  const size_t base = (size_t)b * g.n + ((size_t)layer * st.Hkv + kvh) * st.Wmax;
-  for (int i = threadIdx.x; i < nf + nq; i += blockDim.x) {
-    const int win = i < nf ? st.full_list[ub + i] : st.int2_list[ub + i - nf];
+  const int pos0 = (layer * st.Hkv + kvh) * st.Wmax;
+  // a unit never holds more than max_windows live windows; anything else is a corrupted count
+  const bool sane = nf >= 0 && nq >= 0 && nf + nq <= st.Wmax;
+  const int cnt = sane ? nf + nq : 0;
+  __shared__ int s_base;
+  if (threadIdx.x == 0) {
+    if (!sane) qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
+    s_base = atomicAdd(&g.count[b], cnt);
+  }
+  __syncthreads();
+  const size_t base = (size_t)b * g.n + s_base;
+  for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
+    int win = i < nf ? st.full_list[ub + i] : st.int2_list[ub + i - nf];
     if (win < 0 || win >= st.Wmax) {
       qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
-      continue;
+      win = 0;  // keeps the list well formed; the status word reports the fault
     }
-    g.mass[base + win] = st.mass[ub + win];
-    g.pert[base + win] = st.pert[ub + win];
-    g.flag[base + win] = kValid;
+    g.mass[base + i] = st.mass[ub + win];
+    g.pert[base + i] = st.pert[ub + win];
+    g.pos[base + i] = pos0 + win;
+    g.flag[base + i] = 0;
   }
 }
 
@@ -134,7 +149,7 @@ __device__ void topk_threshold(int n, int k, KeyFn key, SelSh& sh, unsigned long
 // TwoStage(members, b) with stage-1 share b1: the chosen candidates get `out` in their flag
 template <typename MemberFn>
 __device__ void two_stage_global(int n, int b, int b1, MemberFn member, const float* mass, const float* pert,
-                                 uint8_t* flag, uint8_t out, SelSh& sh) {
+                                 const int32_t* pos, uint8_t* flag, uint8_t out, SelSh& sh) {
   int cnt_local = 0;
   for (int i = threadIdx.x; i < n; i += blockDim.x) cnt_local += member(i) ? 1 : 0;
   const int cnt = block_count(cnt_local, sh);
@@ -147,7 +162,7 @@ __device__ void two_stage_global(int n, int b, int b1, MemberFn member, const fl
   unsigned long long P;
   int S;
   if (b1 > 0) {
-    auto k1 = [&](int i) -> unsigned long long { return member(i) ? cand_key(mass[i], i) : 0ull; };
+    auto k1 = [&](int i) -> unsigned long long { return member(i) ? cand_key(mass[i], pos[i]) : 0ull; };
     topk_threshold(n, b1, k1, sh, &P, &S);
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
       const unsigned long long kk = k1(i);
@@ -157,7 +172,7 @@ __device__ void two_stage_global(int n, int b, int b1, MemberFn member, const fl
   }
   if (b - b1 > 0) {
     auto k2 = [&](int i) -> unsigned long long {
-      return (member(i) && !(flag[i] & kPick)) ? cand_key(pert[i], i) : 0ull;
+      return (member(i) && !(flag[i] & kPick)) ? cand_key(pert[i], pos[i]) : 0ull;
     };
     topk_threshold(n, b - b1, k2, sh, &P, &S);
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
@@ -176,20 +191,21 @@ __global__ void __launch_bounds__(kSelThreadsG) glob_select_kernel(GlobArgs g, i
   const size_t base = (size_t)blockIdx.x * g.n;
   const float* mass = g.mass + base;
   const float* pert = g.pert + base;
+  const int32_t* pos = g.pos + base;
   uint8_t* flag = g.flag + base;
   uint8_t* decided = g.decided + base;
-  const int n = g.n;
-  two_stage_global(n, F, F1, [&](int i) { return (flag[i] & kValid) != 0; }, mass, pert, flag, kFull, sh);
-  two_stage_global(n, Q, Q1, [&](int i) { return (flag[i] & (kValid | kFull)) == kValid; }, mass, pert, flag,
-                   kInt2, sh);
+  const int n = g.count[blockIdx.x];  // the list holds live windows only
+  two_stage_global(n, F, F1, [&](int) { return true; }, mass, pert, pos, flag, kFull, sh);
+  two_stage_global(n, Q, Q1, [&](int i) { return (flag[i] & kFull) == 0; }, mass, pert, pos, flag, kInt2, sh);
+  // chosen tiers by flat position (every other position was set to EVICTED beforehand)
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
     const uint8_t f = flag[i];
-    decided[i] = (f & kFull) ? QE_TIER_FULL : ((f & kInt2) ? QE_TIER_INT2 : QE_TIER_EVICTED);
+    decided[pos[i]] = (f & kFull) ? QE_TIER_FULL : ((f & kInt2) ? QE_TIER_INT2 : QE_TIER_EVICTED);
   }
 }
 
 struct GlobLayout {
-  size_t mass, pert, flag, decided, total;
+  size_t mass, pert, pos, flag, count, decided, total;
 };
 
 GlobLayout glob_layout(int n_layers, int B, int Hkv, int max_windows) {
@@ -198,8 +214,10 @@ GlobLayout glob_layout(int n_layers, int B, int Hkv, int max_windows) {
   GlobLayout L{};
   L.mass = 0;
   L.pert = up(L.mass + n * 4);
-  L.flag = up(L.pert + n * 4);
-  L.decided = up(L.flag + n);
+  L.pos = up(L.pert + n * 4);
+  L.flag = up(L.pos + n * 4);
+  L.count = up(L.flag + n);
+  L.decided = up(L.count + (size_t)B * 4);
   L.total = up(L.decided + n);
   return L;
 }
@@ -235,13 +253,17 @@ extern "C" QE_API int qe_route_windows_global(qe_ctx* const* ctxs, int n_layers,
   GlobArgs g{};
   g.mass = reinterpret_cast<float*>(base + L.mass);
   g.pert = reinterpret_cast<float*>(base + L.pert);
+  g.pos = reinterpret_cast<int32_t*>(base + L.pos);
   g.flag = base + L.flag;
+  g.count = reinterpret_cast<int32_t*>(base + L.count);
   g.decided = base + L.decided;
   g.n = (int)n;
   cudaStream_t st = (cudaStream_t)stream;
   const int F1 = (int)floor((double)alpha * full_windows);
   const int Q1 = (int)floor((double)alpha * int2_windows);
-  QE_CUDA_TRY(cudaMemsetAsync(g.flag, 0, (size_t)n * B, st));
+  static_assert(QE_TIER_EVICTED == 0, "decided is cleared to EVICTED with a zero fill");
+  QE_CUDA_TRY(cudaMemsetAsync(g.count, 0, (size_t)B * 4, st));
+  QE_CUDA_TRY(cudaMemsetAsync(g.decided, 0, (size_t)n * B, st));
   for (int l = 0; l < n_layers; ++l) {
     const DevState s = make_state(ctxs[l]);
     glob_keygen_kernel<<<s.U, 256, 0, st>>>(s, l, g);
