@@ -70,3 +70,19 @@ def test_host_side_argument_errors_need_no_device(libpath):
     assert L.qe_route_global_scratch_bytes(32, 8, 8, 1025) >= 32 * 8 * 8 * 1025 * 10
     assert L.qe_route_global_scratch_bytes(0, 8, 8, 1025) == 0
     assert L.qe_route_windows_global(None, 1, 1, 1, 0.5, None, 0, None) == B.QE_ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="gcc not available")
+def test_header_is_plain_c(tmp_path):
+    """include/qevict.h is a C header: it compiles as strict C99 (no torch or C++ types)."""
+    src = tmp_path / "use.c"
+    src.write_text('#include "qevict.h"\n'
+                   "int main(void) {\n"
+                   "  qe_config c; qe_layout l; (void)c; (void)l;\n"
+                   "  return (int)qe_diag_fmm_scratch_bytes(1, 4) + (int)qe_route_global_scratch_bytes(1, 1, 1, 1)\n"
+                   "         + (int)qe_trim_scratch_bytes(1, 1);\n"
+                   "}\n")
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
+                        os.path.join(ROOT, "include"), "-c", str(src), "-o", str(tmp_path / "use.o")],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
