@@ -28,6 +28,9 @@ Functions and where they come from (page title, section):
   (Orçamento Global), 4 (Implementação, paged variable-length heads).
 * ``output_perturbation`` -- L = ||o - o_hat||_1; "Resumo Técnico: CriticalKV",
   Framework Teórico (Definição de Perturbação). Diagnostic only.
+* ``sekv_segment`` / ``sekv_summaries`` / ``sekv_gates`` / ``sekv_attend`` -- SEKV's
+  entropy-guided spans, surprisal-weighted span summaries and mixed-resolution attention
+  with the size correction; "Resumo Técnico: SEKV", Metodologia 1-3.
 * ``tier_diagnostics`` / ``future_missed_mass`` -- selection churn, global
   latent importance reactivation and future missed mass; "Resumo Técnico:
   QEvict", Principais Contribuições 1.

@@ -32,6 +32,10 @@ Pins (tests that tie each function to something other than itself):
 * route_global -- one unit reduces to the unit's own routing; budgets covering
   every window evict nothing; equal scores across units go to the earlier unit;
   a hand-worked two-unit case (``tests/golden/route_global.txt``).
+* sekv_segment / sekv_summaries / sekv_attend -- a hand-worked segmentation and a
+  hand-worked weighted mean; a span of identical tokens, summarised with its size
+  correction, gives exactly the attention of its tokens; every span expanded, or every
+  token an anchor, is plain attention; a zero-surprisal span falls back to the plain mean.
 * tier_diagnostics -- hand-worked two-unit event sequence in
   ``tests/golden/diag_tiers.txt``; a constant sequence has no change and no exit;
   a window alternating FULL/INT2 counts every exit and re-entry once per event and
@@ -515,3 +519,91 @@ def future_missed_mass(qG: np.ndarray, K: np.ndarray, tiers: np.ndarray, window:
         _, p = attend(np.asarray(qG[h], dtype=np.float64), K, K)
         total += p[evicted].sum()
     return total / G
+
+
+# ---------------------------------------------------------------------------
+# SEKV mixed-resolution attention ("Resumo Técnico: SEKV", Metodologia 1-3)
+# ---------------------------------------------------------------------------
+
+
+def sekv_segment(H: np.ndarray, tau: float):
+    """Entropy-guided segmentation (Metodologia 1): tokens whose surprisal H_t >= tau are
+    anchors (kept at full resolution); every maximal run of non-anchor tokens is a span.
+    Returns (anchor positions, spans as (start, end) pairs, end exclusive)."""
+    H = np.asarray(H, dtype=np.float32)
+    anchor = H >= np.float32(tau)
+    anchors = np.nonzero(anchor)[0]
+    spans = []
+    t, n = 0, len(H)
+    while t < n:
+        if anchor[t]:
+            t += 1
+            continue
+        s = t
+        while t < n and not anchor[t]:
+            t += 1
+        spans.append((s, t))
+    return anchors, spans
+
+
+def sekv_summaries(K: np.ndarray, V: np.ndarray, H: np.ndarray, spans):
+    """Span summaries (Metodologia 2, GPU-side coarse representation): the surprisal-weighted,
+    normalised mean of the span's keys, k_S = sum_t H_t K_t / sum_t H_t, and the same mean of
+    its values; the plain mean when the span's surprisal sums to 0. Returns (kbar, vbar, sizes)."""
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    H = np.asarray(H, dtype=np.float64)
+    kbar = np.zeros((len(spans), K.shape[1]))
+    vbar = np.zeros_like(kbar)
+    sizes = np.array([e - s for s, e in spans], dtype=np.int64)
+    for i, (s, e) in enumerate(spans):
+        w = H[s:e]
+        if w.sum() == 0:
+            w = np.ones(e - s)
+        kbar[i] = w @ K[s:e] / w.sum()
+        vbar[i] = w @ V[s:e] / w.sum()
+    return kbar, vbar, sizes
+
+
+def sekv_gates(qG: np.ndarray, kbar: np.ndarray) -> np.ndarray:
+    """Relevance of each span to the step's query heads (Metodologia 3, Roteamento): the
+    largest q_h . k_S / sqrt(D) over the G heads of the kv head."""
+    qG = np.asarray(qG, dtype=np.float64)
+    if len(kbar) == 0:
+        return np.zeros(0)
+    return (qG @ kbar.T / math.sqrt(qG.shape[1])).max(axis=0)
+
+
+def sekv_attend(qG, K, V, H, tau: float, theta: float, expand=None):
+    """Mixed-resolution attention (Metodologia 3, Atenção de Resolução Mista) of the G query
+    heads of one kv head: anchors contribute their K/V; a span whose gate reaches theta is
+    expanded and contributes its tokens; every other span contributes its summary with the
+    size correction ln|S| added to its score (it stands for |S| tokens). ``expand`` may give
+    the expansion decisions instead of the gate. Returns (o [G][D], expanded [n_spans])."""
+    qG = np.asarray(qG, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    anchors, spans = sekv_segment(H, tau)
+    kbar, vbar, sizes = sekv_summaries(K, V, H, spans)
+    if expand is None:
+        expand = sekv_gates(qG, kbar) >= theta
+    expand = np.asarray(expand, dtype=bool)
+    keys, vals, bias = [K[anchors]], [V[anchors]], [np.zeros(len(anchors))]
+    for i, (s, e) in enumerate(spans):
+        if expand[i]:
+            keys.append(K[s:e])
+            vals.append(V[s:e])
+            bias.append(np.zeros(e - s))
+        else:
+            keys.append(kbar[i:i + 1])
+            vals.append(vbar[i:i + 1])
+            bias.append(np.array([math.log(sizes[i])]))
+    Kx, Vx, bx = np.concatenate(keys), np.concatenate(vals), np.concatenate(bias)
+    D = qG.shape[1]
+    o = np.empty((len(qG), D))
+    for h, q in enumerate(qG):
+        s = Kx @ q / math.sqrt(D) + bx
+        s = s - s.max()
+        p = np.exp(s)
+        o[h] = (p / p.sum()) @ Vx
+    return o, expand

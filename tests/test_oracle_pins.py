@@ -595,3 +595,66 @@ def test_route_global_budget_covers_everything_and_ties():
     assert units[0].tier[:3].tolist() == [O.FULL] * 3 and units[1].tier[0] == O.FULL
     assert units[1].tier[1:3].tolist() == [O.INT2] * 2 and units[2].tier[0] == O.INT2
     assert units[2].tier[1:3].tolist() == [O.EVICTED] * 2
+
+
+# ---------------------------------------------------------------------------
+# SEKV mixed-resolution attention ("Resumo Técnico: SEKV", Metodologia 1-3)
+# ---------------------------------------------------------------------------
+
+
+def test_sekv_segmentation_hand_worked():
+    # surprisal 5 0 0 7 1 2 9 0 with tau = 5: anchors at 0, 3, 6; spans [1, 3), [4, 6), [7, 8)
+    anchors, spans = O.sekv_segment(np.array([5, 0, 0, 7, 1, 2, 9, 0], np.float32), 5.0)
+    assert anchors.tolist() == [0, 3, 6] and spans == [(1, 3), (4, 6), (7, 8)]
+    # no anchor: one span over everything; every token an anchor: no span
+    assert O.sekv_segment(np.zeros(5, np.float32), 1.0)[1] == [(0, 5)]
+    assert O.sekv_segment(np.ones(4, np.float32), 0.5)[1] == []
+
+
+def test_sekv_summary_weighted_mean_and_zero_fallback():
+    K = np.array([[1.0, 0.0], [3.0, 4.0], [0.0, 8.0]])
+    V = np.array([[2.0, 2.0], [6.0, -2.0], [1.0, 1.0]])
+    # weights 1 and 3 over tokens 0..1: (k0 + 3 k1) / 4 = (2.5, 3.0); (v0 + 3 v1) / 4 = (5.0, -1.0)
+    kb, vb, sz = O.sekv_summaries(K, V, np.array([1.0, 3.0, 0.0]), [(0, 2), (2, 3)])
+    assert np.allclose(kb[0], [2.5, 3.0]) and np.allclose(vb[0], [5.0, -1.0]) and sz.tolist() == [2, 1]
+    # zero surprisal over a span: the plain mean
+    kb, vb, _ = O.sekv_summaries(K, V, np.zeros(3), [(0, 3)])
+    assert np.allclose(kb[0], K.mean(axis=0)) and np.allclose(vb[0], V.mean(axis=0))
+
+
+def test_sekv_identical_span_summary_is_exact():
+    """A span of w identical tokens summarised with ln w added to its score carries exactly
+    the attention of its w tokens: w e^s = e^(s + ln w)."""
+    r = _rng(401)
+    D, G = 16, 3
+    K = r.standard_normal((12, D))
+    V = r.standard_normal((12, D))
+    K[4:9] = K[4]
+    V[4:9] = V[4]
+    H = np.full(12, 9.0, np.float32)
+    H[4:9] = r.random(5).astype(np.float32)  # tokens 4..8 below tau: one span
+    q = r.standard_normal((G, D))
+    o, exp_ = O.sekv_attend(q, K, V, H, 5.0, np.inf)
+    assert exp_.tolist() == [False]
+    for h in range(G):
+        o_full, _ = O.attend(q[h], K, V)
+        assert np.allclose(o[h], o_full, rtol=1e-12, atol=1e-12)
+
+
+def test_sekv_everything_expanded_or_anchored_is_plain_attention():
+    r = _rng(402)
+    D, G, n = 16, 2, 40
+    K = r.standard_normal((n, D))
+    V = r.standard_normal((n, D))
+    H = r.exponential(size=n).astype(np.float32)
+    q = r.standard_normal((G, D))
+    for tau, theta in ((1.0, -np.inf), (-1.0, 0.0)):
+        o, _ = O.sekv_attend(q, K, V, H, tau, theta)
+        for h in range(G):
+            o_full, _ = O.attend(q[h], K, V)
+            assert np.allclose(o[h], o_full, rtol=1e-12, atol=1e-12)
+    # the gate of a span is the largest scaled score over the heads
+    _, spans = O.sekv_segment(H, 1.0)
+    kb, _, _ = O.sekv_summaries(K, V, H, spans)
+    g = O.sekv_gates(q, kb)
+    assert np.allclose(g, np.max(q @ kb.T, axis=0) / math.sqrt(D))
