@@ -971,6 +971,119 @@ def run_layers(args):
     print(json.dumps(line), flush=True)
 
 
+SEKV_THETA = 1.5
+
+
+def run_sekv(args):
+    """SEKV mixed-resolution attention at the c2 shape: entropy-guided spans over a 32K
+    context (built once), then per step the span gates and one softmax over anchors, span
+    summaries (size-corrected) and the tokens of expanded spans."""
+    import torch
+
+    from kv_cache_eviction_gqa_b200 import binding as Bd
+    import oracle as O
+    cfg = CFG
+    B, Hq, Hkv, D, G, n = cfg.B, cfg.Hq, cfg.Hkv, cfg.D, cfg.G, cfg.ctx
+    dev = torch.device("cuda", 0)
+    t = torch.bfloat16
+    hbm, hbm_kind = measured_peaks()
+    H = W.draw_surprisal(cfg, n)
+    cpu = None
+    if not args.no_cpu_baseline:
+        K0, V0 = W.draw_unit_cache(cfg, 0, 0)
+        q0 = W.draw_step_inputs(cfg.scaled(steps=1))[0][0][0, :G]
+        t0 = time.perf_counter()
+        reps = 0
+        while time.perf_counter() - t0 < 10.0:
+            O.sekv_attend(q0, K0, V0, H[0], W.SEKV_TAU, SEKV_THETA)
+            reps += 1
+        per_unit = (time.perf_counter() - t0) / reps
+        cpu = {"value": 1.0 / (per_unit * cfg.units), "unit": "steps/s", "kind": "oracle",
+               "cores": len(os.sched_getaffinity(0)), "blas_threads": blas_threads(),
+               "sample": f"float64 oracle on 1 of {cfg.units} units ({reps} runs of segmentation, summaries and "
+                         "mixed attention), scaled to all units"}
+    g = torch.Generator(device=dev)
+    g.manual_seed(cfg.seed * 7877)
+    scale = torch.ones((B, Hkv, 1, D), device=dev)
+    ch = torch.rand((B, Hkv, D), generator=g, device=dev).argsort(dim=-1)[..., :4]
+    scale.scatter_(-1, ch.unsqueeze(2), 8.0)
+    K = torch.randn((B, Hkv, n, D), generator=g, device=dev, dtype=t) * scale.to(t)
+    V = torch.randn((B, Hkv, n, D), generator=g, device=dev, dtype=t) * scale.to(t)
+    q = torch.randn((B, Hq, D), generator=g, device=dev, dtype=t)
+    Hd = torch.from_numpy(H).to(dev)
+    st = torch.cuda.current_stream()
+    flush = L2Flush(dev)
+    state = Bd.sekv_build(K, V, Hd, W.SEKV_TAU, Hq)
+    build_ms = _timed(lambda: Bd.sekv_build(K, V, Hd, W.SEKV_TAU, Hq, state), 5, flush, st)
+    out = Bd.sekv_attend(q, K, V, SEKV_THETA, state)
+    torch.cuda.synchronize()
+    cap = torch.cuda.Stream()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr, stream=cap):
+        Bd.sekv_attend(q, K, V, SEKV_THETA, state, out)
+    for _ in range(args.warmup):
+        gr.replay()
+    torch.cuda.synchronize()
+    with ClockSampler(0) as clk:
+        ms = _timed(gr.replay, args.steps, flush, st)
+    step_s = statistics.mean(ms) / 1e3
+    views = Bd.sekv_views(state, B, Hq, Hkv, n, D)
+    counts = views["counts"].cpu().numpy()
+    ss, se = views["span_start"].cpu().numpy(), views["span_end"].cpu().numpy()
+    exp_ = views["expanded"].cpu().numpy()
+    alg, n_exp, n_spans = 0, 0, 0
+    for b in range(B):
+        A, NS = int(counts[b, 0]), int(counts[b, 1])
+        lens = se[b, :NS] - ss[b, :NS]
+        for h in range(Hkv):
+            e = exp_[b, h, :NS].astype(bool)
+            n_exp += int(e.sum())
+            n_spans += NS
+            alg += (A * 2 * D * 2 + NS * D * 4 + int((~e).sum()) * 2 * D * 4 + int(lens[e].sum()) * 2 * D * 2
+                    + G * D * 2 + G * D * 4)
+    # e2e: q from pinned host memory, output back
+    qh = q.cpu().pin_memory()
+    oh = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    ge = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(ge, stream=cap):
+        q.copy_(qh, non_blocking=True)
+        Bd.sekv_attend(q, K, V, SEKV_THETA, state, out)
+        oh.copy_(out, non_blocking=True)
+    e2e_ms = []
+    for _ in range(min(args.steps, 64)):
+        flush.zero_()
+        torch.cuda.synchronize()
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        ge.replay()
+        b_.record(st)
+        b_.synchronize()
+        e2e_ms.append(a.elapsed_time(b_))
+    line = {
+        "metric": "SEKV mixed-resolution attention steps/sec (32K ctx, batch 8); achieved HBM GB/s vs peak",
+        "value": 1.0 / step_s, "unit": "steps/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"sekv at the {cfg.name} shape: B={B}, Hq={Hq}, Hkv={Hkv}, D={D}, n={n}; surprisal "
+                               f"Exponential(1) per token, anchors at H >= ln 10 (about 10 %), expansion threshold "
+                               f"{SEKV_THETA}; K/V N(0,1) with 4 outlier channels x8 drawn on the device",
+                   "l2": FLUSH_NOTE},
+        "roofline": {"kernel": "one step: gate, mixed attention and combine (one graph)", "bound": "hbm",
+                     "achieved": alg / step_s / 1e9, "peak": hbm, "unit": "GB/s", "frac": alg / step_s / 1e9 / hbm,
+                     "peak_kind": f"{hbm_kind} (MEASURED_PEAKS.json hbm_gbs)", "traffic": None,
+                     "algorithmic_bytes": alg},
+        "secondary": {"build_ms": statistics.mean(build_ms), "anchors_per_sequence": float(counts[:, 0].mean()),
+                      "spans_per_sequence": float(counts[:, 1].mean()),
+                      "expanded_fraction": n_exp / max(n_spans, 1)},
+        "cpu_baseline": cpu,
+        "e2e": {"value": len(e2e_ms) / (sum(e2e_ms) / 1e3), "unit": "steps/s", "h2d_bytes_per_step": q.numel() * 2,
+                "d2h_bytes_per_step": out.numel() * 4, "steps": len(e2e_ms)},
+        "clocks": clk.summary(),
+        "gpu_launches": args.steps * 3,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
@@ -980,10 +1093,11 @@ def main():
     ap.add_argument("--max-splits", type=int, default=32)
     ap.add_argument("--e2e-steps", type=int, default=640)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["c2", "c3", "c4", "diag", "layers"], default="c2",
+    ap.add_argument("--workload", choices=["c2", "c3", "c4", "diag", "layers", "sekv"], default="c2",
                     help="c2: tiered decode (the default bench); c3: CriticalKV selection; c4: DBTrimKV trim; "
                          "diag: QEvict diagnostics (future missed mass, churn, LIR) at the c2 shape; "
-                         "layers: 32 c2-shaped layers under one global budget per sequence")
+                         "layers: 32 c2-shaped layers under one global budget per sequence; "
+                         "sekv: SEKV mixed-resolution attention at the c2 shape")
     ap.add_argument("--profile-steps", type=int, default=0,
                     help="run only this many eager decode steps after the prefill, then exit")
     args = ap.parse_args()
@@ -997,7 +1111,8 @@ def main():
         return
     if args.workload != "c2":
         if rank == 0:
-            {"c3": run_c3, "c4": run_c4, "diag": run_diag, "layers": run_layers}[args.workload](args)
+            {"c3": run_c3, "c4": run_c4, "diag": run_diag, "layers": run_layers,
+             "sekv": run_sekv}[args.workload](args)
         return
     if world > 1:
         import datetime

@@ -352,6 +352,38 @@ QE_API int qe_diag_fmm(const void* q, const void* K_ghost, long long n_stride, i
                        int dtype, float* fmm_out, void* scratch, size_t scratch_bytes,
                        qe_stream_t stream);
 
+/* SEKV-style mixed-resolution attention ("Resumo Técnico: SEKV", Metodologia 1-3).
+ * qe_sekv_build (once per cache): for each sequence b, tokens with surprisal H[b][t] >= tau are
+ *   anchors (full resolution) and every maximal run of non-anchor tokens is a span; for each
+ *   (b, kv head) and span S the summary key is sum_{t in S} H_t K_t / sum_{t in S} H_t (the
+ *   plain mean when that sum is 0) and the summary value the same mean of V, in float32.
+ * qe_sekv_attend (every step): span S of kv head h is expanded when
+ *   max over the G query heads of h of q . kbar_S / sqrt(D) >= theta; the output of query head
+ *   (b, hq) is the softmax attention over the anchors' K/V, the tokens of expanded spans and
+ *   the summaries of the other spans, a summary's score raised by ln|S| (it stands for |S|
+ *   tokens). The trained routing projections and thresholds and the CPU low-rank rebuild are
+ *   not part of this call: theta stands for the learned threshold and an expanded span
+ *   contributes the tokens in K/V.
+ *   q [dev]: [B][Hq][D]; K, V [dev]: [B][Hkv][n][D] (16-byte aligned), fp16 or bf16 (dtype);
+ *   H [dev, float]: [B][n] surprisal per token; out [dev, float]: [B][Hq][D].
+ *   state [dev]: qe_sekv_state_bytes(B, Hq, Hkv, n, D) bytes, 256-byte aligned, written by
+ *   build and read (expansion flags and partials written) by attend; qe_sekv_state_offsets
+ *   gives the byte offsets of its arrays: [0] counts [B][2] int32 (anchors, spans), [1] anchor
+ *   positions [B][n] int32, [2] span starts, [3] span ends (exclusive) [B][cap] int32, [4] summary
+ *   keys, [5] summary values [B][Hkv][cap][D] float, [6] expansion flags [B][Hkv][cap] uint8,
+ *   and [7] cap = (n + 1) / 2.
+ * Errors (returned, nothing launched): QE_ERR_INVALID_ARG (null or misaligned pointer, n < 1,
+ * Hq not a multiple of Hkv, bad dtype), QE_ERR_UNSUPPORTED_SHAPE (D not in {64, 128}, G not in
+ * {1, 2, 4, 5, 8}, n > 500000), QE_ERR_WORKSPACE (small state). Asynchronous; allocates nothing. */
+QE_API size_t qe_sekv_state_bytes(int B, int Hq, int Hkv, int n, int D);
+QE_API int qe_sekv_state_offsets(int B, int Hq, int Hkv, int n, int D, size_t* offsets);
+QE_API int qe_sekv_build(const void* K, const void* V, const float* H, int B, int Hq, int Hkv, int n,
+                         int D, int dtype, float tau, void* state, size_t state_bytes,
+                         qe_stream_t stream);
+QE_API int qe_sekv_attend(const void* q, const void* K, const void* V, int B, int Hq, int Hkv, int n,
+                          int D, int dtype, float theta, void* state, size_t state_bytes,
+                          float* out, qe_stream_t stream);
+
 /* qe_status - copy the device status word to the host (synchronises the context's last
  * stream) and return the first recorded error, or QE_OK. *detail (may be NULL) receives the
  * failing index or unit. */

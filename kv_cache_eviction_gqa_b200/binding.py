@@ -71,6 +71,10 @@ def lib():
                                         vp, sz, vp]),
             "qe_route_global_scratch_bytes": (sz, [i, i, i, i]),
             "qe_route_windows_global": (i, [vp, i, i, i, f, vp, sz, vp]),
+            "qe_sekv_state_bytes": (sz, [i, i, i, i, i]),
+            "qe_sekv_state_offsets": (i, [i, i, i, i, i, C.POINTER(C.c_size_t)]),
+            "qe_sekv_build": (i, [vp, vp, vp, i, i, i, i, i, i, f, vp, sz, vp]),
+            "qe_sekv_attend": (i, [vp, vp, vp, i, i, i, i, i, i, f, vp, sz, vp, vp]),
             "qe_diag_tiers": (i, [vp, vp, vp, i, i, i, vp, vp]),
             "qe_diag_fmm_scratch_bytes": (sz, [i, i]),
             "qe_diag_fmm": (i, [vp, vp, ll, i, vp, i, i, i, i, i, i, i, vp, vp, sz, vp]),
@@ -485,3 +489,59 @@ def route_windows_global(ctxs, full_windows: int, int2_windows: int, alpha: floa
                                          _ptr(scratch), scratch.numel(), _stream(stream)),
            "qe_route_windows_global")
     return scratch
+
+
+def sekv_state_bytes(B: int, Hq: int, Hkv: int, n: int, D: int) -> int:
+    return int(lib().qe_sekv_state_bytes(B, Hq, Hkv, n, D))
+
+
+def sekv_build(K: torch.Tensor, V: torch.Tensor, H: torch.Tensor, tau: float, Hq: int, state=None, stream=None):
+    """SEKV segmentation and span summaries (qe_sekv_build). K, V [B][Hkv][n][D] fp16/bf16,
+    H [B][n] float32 surprisal. Returns the state buffer for sekv_attend."""
+    _need(K, "K")
+    B, Hkv, n, D = K.shape
+    _need(V, "V", K.dtype, K.shape)
+    _need(H, "H", torch.float32, (B, n))
+    nbytes = sekv_state_bytes(B, Hq, Hkv, n, D)
+    if nbytes == 0:
+        raise ValueError("unsupported SEKV shape")
+    if state is None:
+        state = torch.empty(nbytes, dtype=torch.uint8, device=K.device)
+    _check(lib().qe_sekv_build(_ptr(K), _ptr(V), _ptr(H), B, Hq, Hkv, n, D, dtype_code(K.dtype), float(tau),
+                               _ptr(state), state.numel(), _stream(stream)), "qe_sekv_build")
+    return state
+
+
+def sekv_attend(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, theta: float, state: torch.Tensor, out=None,
+                stream=None):
+    """SEKV mixed-resolution attention of one step (qe_sekv_attend). q [B][Hq][D]; K, V and
+    state as given to sekv_build. Returns out [B][Hq][D] float32."""
+    _need(q, "q", K.dtype)
+    B, Hq, D = q.shape
+    _, Hkv, n, _ = K.shape
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.float32, (B, Hq, D))
+    _check(lib().qe_sekv_attend(_ptr(q), _ptr(K), _ptr(V), B, Hq, Hkv, n, D, dtype_code(q.dtype), float(theta),
+                                _ptr(state), state.numel(), _ptr(out), _stream(stream)), "qe_sekv_attend")
+    return out
+
+
+def sekv_views(state: torch.Tensor, B: int, Hq: int, Hkv: int, n: int, D: int) -> dict:
+    """Views of the SEKV state arrays (counts, anchors, span bounds, summaries, expansion flags)."""
+    off = (C.c_size_t * 8)()
+    _check(lib().qe_sekv_state_offsets(B, Hq, Hkv, n, D, off), "qe_sekv_state_offsets")
+    cap = int(off[7])
+
+    def view(o, count, dtype, shape):
+        nb = count * torch.tensor([], dtype=dtype).element_size()
+        return state[o:o + nb].view(dtype).view(*shape)
+
+    return {"counts": view(off[0], B * 2, torch.int32, (B, 2)),
+            "anchor_pos": view(off[1], B * n, torch.int32, (B, n)),
+            "span_start": view(off[2], B * cap, torch.int32, (B, cap)),
+            "span_end": view(off[3], B * cap, torch.int32, (B, cap)),
+            "kbar": view(off[4], B * Hkv * cap * D, torch.float32, (B, Hkv, cap, D)),
+            "vbar": view(off[5], B * Hkv * cap * D, torch.float32, (B, Hkv, cap, D)),
+            "expanded": view(off[6], B * Hkv * cap, torch.uint8, (B, Hkv, cap)),
+            "cap": cap}

@@ -462,3 +462,19 @@ def draw_ghost_keys(cfg: DiagConfig, b: int, kvh: int) -> np.ndarray:
 def draw_diag_queries(cfg: DiagConfig) -> np.ndarray:
     """The step's queries [B][Hq][D]: the first decode step's q of ``base``."""
     return draw_step_inputs(cfg.base.scaled(steps=1))[0][0]
+
+
+# --------------------------------------------------------------------------
+# SEKV workloads (surprisal per token)
+# --------------------------------------------------------------------------
+
+# anchor threshold for Exponential(1) surprisal: P(H >= ln 10) = 1/10, so about 10 % of the
+# tokens are anchors and spans average about 9 tokens
+SEKV_TAU = math.log(10.0)
+
+
+def draw_surprisal(cfg: DecodeConfig, n: int) -> np.ndarray:
+    """Per-token surprisal [B][n] float32, Exponential(1): a stand-in for -log p(x_t | x_<t)
+    of a language model, which needs trained weights."""
+    r = _rng(cfg.seed, 0x5E4B)
+    return r.exponential(size=(cfg.B, n)).astype(np.float32)
