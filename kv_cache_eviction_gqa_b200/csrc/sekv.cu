@@ -25,6 +25,7 @@ namespace {
 constexpr int kSekvWarps = 4;      // warps per CTA (gate, summarize, attend)
 constexpr int kSekvMaxSplits = 32;
 constexpr int kSekvTargetCtas = 1184;  // 148 SMs x 8
+constexpr int kSekvSpanBlocks = 64;    // CTAs per unit for the per-span kernels (grid-stride over spans)
 
 struct SekvLayout {
   size_t counts, anchor_pos, span_start, span_end, kbar, vbar, expanded, part_ml, part_o, total;
@@ -145,32 +146,33 @@ __global__ void __launch_bounds__(kSekvWarps * 32)
   constexpr int D = 32 * DPL;
   const int u = blockIdx.x, b = u / Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int i = blockIdx.y * kSekvWarps + warp;
-  if (i >= counts[b * 2 + 1]) return;
-  const int s = span_start[(size_t)b * cap + i], e = span_end[(size_t)b * cap + i];
-  float ak[DPL] = {}, av[DPL] = {}, pk[DPL] = {}, pv[DPL] = {};
-  float ws = 0.f;
-  for (int t = s; t < e; ++t) {
-    const float w = H[(size_t)b * n + t];
-    float kx[DPL], vx[DPL];
-    load_dims<T, DPL>(K + ((size_t)u * n + t) * D, lane, kx);
-    load_dims<T, DPL>(V + ((size_t)u * n + t) * D, lane, vx);
-#pragma unroll
-    for (int j = 0; j < DPL; ++j) {
-      ak[j] = fmaf(w, kx[j], ak[j]);
-      av[j] = fmaf(w, vx[j], av[j]);
-      pk[j] += kx[j];
-      pv[j] += vx[j];
+  const int nspans = counts[b * 2 + 1];
+  for (int i = blockIdx.y * kSekvWarps + warp; i < nspans; i += gridDim.y * kSekvWarps) {
+    const int s = span_start[(size_t)b * cap + i], e = span_end[(size_t)b * cap + i];
+    float ak[DPL] = {}, av[DPL] = {}, pk[DPL] = {}, pv[DPL] = {};
+    float ws = 0.f;
+    for (int t = s; t < e; ++t) {
+      const float w = H[(size_t)b * n + t];
+      float kx[DPL], vx[DPL];
+      load_dims<T, DPL>(K + ((size_t)u * n + t) * D, lane, kx);
+      load_dims<T, DPL>(V + ((size_t)u * n + t) * D, lane, vx);
+  #pragma unroll
+      for (int j = 0; j < DPL; ++j) {
+        ak[j] = fmaf(w, kx[j], ak[j]);
+        av[j] = fmaf(w, vx[j], av[j]);
+        pk[j] += kx[j];
+        pv[j] += vx[j];
+      }
+      ws += w;
     }
-    ws += w;
-  }
-  const float inv = ws > 0.f ? 1.f / ws : 1.f / (float)(e - s);
-  float* kr = kbar + ((size_t)u * cap + i) * D + lane * DPL;
-  float* vr = vbar + ((size_t)u * cap + i) * D + lane * DPL;
-#pragma unroll
-  for (int j = 0; j < DPL; ++j) {
-    kr[j] = (ws > 0.f ? ak[j] : pk[j]) * inv;
-    vr[j] = (ws > 0.f ? av[j] : pv[j]) * inv;
+    const float inv = ws > 0.f ? 1.f / ws : 1.f / (float)(e - s);
+    float* kr = kbar + ((size_t)u * cap + i) * D + lane * DPL;
+    float* vr = vbar + ((size_t)u * cap + i) * D + lane * DPL;
+  #pragma unroll
+    for (int j = 0; j < DPL; ++j) {
+      kr[j] = (ws > 0.f ? ak[j] : pk[j]) * inv;
+      vr[j] = (ws > 0.f ? av[j] : pv[j]) * inv;
+    }
   }
 }
 
@@ -182,20 +184,22 @@ __global__ void __launch_bounds__(kSekvWarps * 32)
   constexpr int D = 32 * DPL;
   const int u = blockIdx.x, b = u / Hkv, kvh = u % Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int i = blockIdx.y * kSekvWarps + warp;
-  if (i >= counts[b * 2 + 1]) return;
-  const float* kr = kbar + ((size_t)u * cap + i) * D + lane * DPL;
-  float g = -INFINITY;
+  const int nspans = counts[b * 2 + 1];
+  float qx[G][DPL];
 #pragma unroll
-  for (int h = 0; h < G; ++h) {
-    float qx[DPL];
-    load_dims<T, DPL>(q + ((size_t)b * Hq + (size_t)kvh * G + h) * D, lane, qx);
-    float d = 0.f;
+  for (int h = 0; h < G; ++h) load_dims<T, DPL>(q + ((size_t)b * Hq + (size_t)kvh * G + h) * D, lane, qx[h]);
+  for (int i = blockIdx.y * kSekvWarps + warp; i < nspans; i += gridDim.y * kSekvWarps) {
+    const float* kr = kbar + ((size_t)u * cap + i) * D + lane * DPL;
+    float g = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < DPL; ++j) d = fmaf(qx[j], kr[j], d);
-    g = fmaxf(g, warp_allsum(d) * scale);
+    for (int h = 0; h < G; ++h) {
+      float d = 0.f;
+#pragma unroll
+      for (int j = 0; j < DPL; ++j) d = fmaf(qx[h][j], kr[j], d);
+      g = fmaxf(g, warp_allsum(d) * scale);
+    }
+    if (lane == 0) expanded[(size_t)u * cap + i] = g >= theta ? 1 : 0;
   }
-  if (lane == 0) expanded[(size_t)u * cap + i] = g >= theta ? 1 : 0;
 }
 
 struct SekvAttendArgs {
@@ -352,7 +356,8 @@ int launch_build(const void* K, const void* V, const float* H, int B, int Hkv, i
   sekv_segment_kernel<<<B, 1024, 0, s>>>(H, n, tau, L.cap, counts, reinterpret_cast<int32_t*>(st + L.anchor_pos),
                                          sst, sen);
   QE_CUDA_TRY(cudaGetLastError());
-  const dim3 grid(B * Hkv, (L.cap + kSekvWarps - 1) / kSekvWarps);
+  const int ny = (L.cap + kSekvWarps - 1) / kSekvWarps;
+  const dim3 grid(B * Hkv, ny < kSekvSpanBlocks ? ny : kSekvSpanBlocks);
   sekv_summarize_kernel<T, DPL><<<grid, kSekvWarps * 32, 0, s>>>(
       static_cast<const T*>(K), static_cast<const T*>(V), H, n, Hkv, L.cap, counts, sst, sen,
       reinterpret_cast<float*>(st + L.kbar), reinterpret_cast<float*>(st + L.vbar));
@@ -368,7 +373,8 @@ int launch_attend(const void* q, const void* K, const void* V, int B, int Hq, in
   const int32_t* counts = reinterpret_cast<const int32_t*>(st + L.counts);
   const float* kbar = reinterpret_cast<const float*>(st + L.kbar);
   uint8_t* expanded = st + L.expanded;
-  const dim3 ggrid(U, (L.cap + kSekvWarps - 1) / kSekvWarps);
+  const int ny = (L.cap + kSekvWarps - 1) / kSekvWarps;
+  const dim3 ggrid(U, ny < kSekvSpanBlocks ? ny : kSekvSpanBlocks);
   sekv_gate_kernel<T, DPL, G><<<ggrid, kSekvWarps * 32, 0, s>>>(static_cast<const T*>(q), Hq, Hkv, L.cap, counts,
                                                                 kbar, (float)(1.0 / sqrt((double)D)), theta,
                                                                 expanded);

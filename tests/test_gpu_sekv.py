@@ -65,9 +65,9 @@ def run_case(base, n, tau, theta_mode):
             ref[b, h] = (spans, kb)
     # theta: a fixed value, or the 90th percentile of the oracle's gates (about 10 % expanded)
     if theta_mode == "q90":
-        gates = np.concatenate([O.sekv_gates(q[b, h * G:(h + 1) * G], ref[b, h][1])
-                                for b in range(B) for h in range(Hkv) if len(ref[b, h][1])])
-        theta = float(np.quantile(gates, 0.9)) if len(gates) else 0.0
+        gates = [O.sekv_gates(q[b, h * G:(h + 1) * G], ref[b, h][1])
+                 for b in range(B) for h in range(Hkv) if len(ref[b, h][1])]
+        theta = float(np.quantile(np.concatenate(gates), 0.9)) if gates else 0.0
     else:
         theta = float(theta_mode)
     out = Bd.sekv_attend(torch.from_numpy(q).to("cuda", t), K, V, theta, state)
