@@ -86,3 +86,21 @@ def test_header_is_plain_c(tmp_path):
                         os.path.join(ROOT, "include"), "-c", str(src), "-o", str(tmp_path / "use.o")],
                        capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_sekv_host_side_sizes_and_errors(libpath):
+    from kv_cache_eviction_gqa_b200 import binding as B
+    L = B.lib()
+    # the state holds summaries for up to (n + 1) / 2 spans per (sequence, kv head) in float32
+    n, D = 32768, 128
+    assert L.qe_sekv_state_bytes(8, 32, 8, n, D) >= 8 * 8 * ((n + 1) // 2) * D * 4 * 2
+    assert L.qe_sekv_state_bytes(1, 4, 1, n, 96) == 0          # D = 96 unsupported
+    assert L.qe_sekv_state_bytes(1, 6, 4, n, 128) == 0         # Hq not a multiple of Hkv
+    assert L.qe_sekv_state_bytes(1, 4, 1, 0, 128) == 0         # no token
+    import ctypes as C
+    off = (C.c_size_t * 8)()
+    assert L.qe_sekv_state_offsets(2, 8, 2, 1001, 64, off) == B.QE_OK and off[7] == 501
+    assert list(off[:7]) == sorted(off[:7])
+    assert L.qe_sekv_build(None, None, None, 1, 4, 1, 16, 128, B.QE_BF16, 1.0, None, 0, None) == B.QE_ERR_INVALID_ARG
+    assert L.qe_sekv_attend(None, None, None, 1, 4, 1, 16, 128, B.QE_BF16, 1.0, None, 0, None,
+                            None) == B.QE_ERR_INVALID_ARG
