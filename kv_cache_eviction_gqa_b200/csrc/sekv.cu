@@ -323,27 +323,25 @@ __global__ void __launch_bounds__(kSekvWarps * 32) sekv_attend_kernel(SekvAttend
   }
 }
 
-// out[b][kvh*G + h][d] = sum_s O_s 2^(M_s - M) / sum_s L_s 2^(M_s - M)
+// out[b][kvh*G + h][d] = sum_s O_s 2^(M_s - M) / sum_s L_s 2^(M_s - M); one CTA per (unit, head)
 __global__ void sekv_combine_kernel(const float* __restrict__ part_ml, const float* __restrict__ part_o, int S, int G,
                                     int D, int Hq, int Hkv, float* out) {
-  const int u = blockIdx.x, b = u / Hkv, kvh = u % Hkv;
-  for (int h = 0; h < G; ++h) {
-    const size_t p0 = (size_t)u * S * G;
-    float M = -1e30f;
-    for (int s = 0; s < S; ++s) M = fmaxf(M, part_ml[(p0 + (size_t)s * G + h) * 2]);
-    float L = 0.f;
+  const int u = blockIdx.x, h = blockIdx.y, b = u / Hkv, kvh = u % Hkv;
+  const size_t p0 = (size_t)u * S * G;
+  float M = -1e30f;
+  for (int s = 0; s < S; ++s) M = fmaxf(M, part_ml[(p0 + (size_t)s * G + h) * 2]);
+  float L = 0.f;
+  for (int s = 0; s < S; ++s) {
+    const size_t pi = p0 + (size_t)s * G + h;
+    L = fmaf(part_ml[pi * 2 + 1], ex2s(part_ml[pi * 2] - M), L);
+  }
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float O = 0.f;
     for (int s = 0; s < S; ++s) {
       const size_t pi = p0 + (size_t)s * G + h;
-      L = fmaf(part_ml[pi * 2 + 1], ex2s(part_ml[pi * 2] - M), L);
+      O = fmaf(part_o[pi * D + d], ex2s(part_ml[pi * 2] - M), O);
     }
-    for (int d = threadIdx.x; d < D; d += blockDim.x) {
-      float O = 0.f;
-      for (int s = 0; s < S; ++s) {
-        const size_t pi = p0 + (size_t)s * G + h;
-        O = fmaf(part_o[pi * D + d], ex2s(part_ml[pi * 2] - M), O);
-      }
-      out[((size_t)b * Hq + (size_t)kvh * G + h) * D + d] = L > 0.f ? O / L : 0.f;
-    }
+    out[((size_t)b * Hq + (size_t)kvh * G + h) * D + d] = L > 0.f ? O / L : 0.f;
   }
 }
 
@@ -400,7 +398,7 @@ int launch_attend(const void* q, const void* K, const void* V, int B, int Hq, in
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
   sekv_attend_kernel<T, DPL, G><<<U * S, kSekvWarps * 32, 0, s>>>(a);
   QE_CUDA_TRY(cudaGetLastError());
-  sekv_combine_kernel<<<U, 128, 0, s>>>(a.part_ml, a.part_o, S, G, D, Hq, Hkv, out);
+  sekv_combine_kernel<<<dim3(U, G), 128, 0, s>>>(a.part_ml, a.part_o, S, G, D, Hq, Hkv, out);
   QE_CUDA_TRY(cudaGetLastError());
   return QE_OK;
 }
