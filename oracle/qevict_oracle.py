@@ -208,7 +208,7 @@ class QEvictUnit:
     Per token: the values attention uses (``Keff``/``Veff``), the values the
     full tier stores (``Kst``/``Vst``) and the projected-value norms n[h].
 
-    Readings where the pages are silent (each listed in the design doc):
+    Readings where the pages are silent:
     the tail (newest, incomplete) window is always full precision, outside the
     budget and not routed; scores accumulate undecayed from step 0; evicted
     windows never return; routing runs after attention on steps s % R == 0;
