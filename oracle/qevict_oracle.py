@@ -22,20 +22,24 @@ Pins (tests that tie each function to something other than itself):
   routing fixture in ``tests/golden/two_stage.txt``.
 * QEvictUnit -- per-step mass invariant (sum over live windows = G);
   write-once ledger (demote -> promote -> demote yields identical codes);
-  with budgets covering every window it reduces to plain attention.
+  with budgets covering every window it reduces to plain attention; a hand-worked
+  two-head, two-window step with a different W_O slice per head fixes the mass and the
+  perturbation accumulation (``tests/golden/qevict_pert.txt``).
 * observation_mass -- brute force; sum over keys of A = G * n_obs.
 * trim_global_topm -- closed forms: constant beta keeps the most recent
   entries, equal age keeps the larger beta, beta = 1 everywhere ties and keeps
   the lowest flat indices; compared with ``np.argsort`` on tiny sets.
-* output_perturbation -- diagnostic only (parity unpinned: the pages give no
-  value for it and the bound theta is not printed).
+* output_perturbation -- a hand-worked three-token case, unprojected and projected
+  through W_O^h (``tests/golden/output_perturbation.txt``); the full set gives 0.
 * route_global -- one unit reduces to the unit's own routing; budgets covering
   every window evict nothing; equal scores across units go to the earlier unit;
   a hand-worked two-unit case (``tests/golden/route_global.txt``).
 * sekv_segment / sekv_summaries / sekv_attend -- a hand-worked segmentation and a
   hand-worked weighted mean; a span of identical tokens, summarised with its size
   correction, gives exactly the attention of its tokens; every span expanded, or every
-  token an anchor, is plain attention; a zero-surprisal span falls back to the plain mean.
+  token an anchor, is plain attention; a zero-surprisal span falls back to the plain mean;
+  sekv_gates -- a hand-worked two-head case where the maximum over heads, the mean and
+  the 1/sqrt(D) scale all differ (``tests/golden/sekv_gates.txt``).
 * tier_diagnostics -- hand-worked two-unit event sequence in
   ``tests/golden/diag_tiers.txt``; a constant sequence has no change and no exit;
   a window alternating FULL/INT2 counts every exit and re-entry once per event and

@@ -658,3 +658,68 @@ def test_sekv_everything_expanded_or_anchored_is_plain_attention():
     kb, _, _ = O.sekv_summaries(K, V, H, spans)
     g = O.sekv_gates(q, kb)
     assert np.allclose(g, np.max(q @ kb.T, axis=0) / math.sqrt(D))
+
+
+# ---------------------------------------------------------------------------
+# hand-worked pins of the unit's perturbation accumulation, the SEKV gate and the
+# output perturbation (fixtures carry the citation and the arithmetic)
+# ---------------------------------------------------------------------------
+
+
+def _read_kv_golden(golden_dir, name):
+    vals = {}
+    with open(os.path.join(golden_dir, name)) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            k, v = [t.strip() for t in line.split("|")]
+            vals[k] = np.array([float(x) for x in v.split()])
+    return vals
+
+
+def test_unit_perturbation_golden(golden_dir):
+    g = _read_kv_golden(golden_dir, "qevict_pert.txt")
+    K0 = np.stack([np.log(g["a"]), np.log(g["b"])], axis=1)
+    V0 = g["V"].reshape(4, 2)
+    W_O = g["W_O"].reshape(4, 2)
+    u = O.QEvictUnit(K0, V0, W_O, 0, 2, 2, 8, 8, 0.5, "fp16", 8)
+    # the two windows of the prefill are full precision and every token is live
+    assert list(u.tier[:2]) == [O.FULL, O.FULL]
+    qG = np.array([[math.sqrt(2), 0.0], [0.0, math.sqrt(2)]])
+    _, step_mass = u.attend_and_score(qG)
+    np.testing.assert_allclose(step_mass[:2], g["mass_step"], rtol=1e-12)
+    np.testing.assert_allclose(u.pert[:2], g["pert_step"], rtol=1e-12)
+    # undecayed sums: a second identical step doubles both scores
+    u.attend_and_score(qG)
+    np.testing.assert_allclose(u.mass[:2], 2 * g["mass_step"], rtol=1e-12)
+    np.testing.assert_allclose(u.pert[:2], 2 * g["pert_step"], rtol=1e-12)
+
+
+def test_sekv_gates_golden(golden_dir):
+    g = _read_kv_golden(golden_dir, "sekv_gates.txt")
+    q = g["q"].reshape(2, 4)
+    kbar = g["kbar"].reshape(2, 4)
+    np.testing.assert_allclose(O.sekv_gates(q, kbar), g["gates"], rtol=1e-15)
+    # the gate decides expansion inside sekv_attend: with surprisal (0, 5, 0) and tau = 1 the
+    # middle token is an anchor and the other two are one-token spans whose summaries are
+    # exactly kbar_0 and kbar_1
+    H = np.array([0.0, 5.0, 0.0])
+    anchors, spans = O.sekv_segment(H, 1.0)
+    assert list(anchors) == [1] and [tuple(s) for s in spans] == [(0, 1), (2, 3)]
+    K3 = np.stack([kbar[0], np.zeros(4), kbar[1]])
+    V3 = np.eye(3, 4)
+    _, expanded = O.sekv_attend(q, K3, V3, H, 1.0, g["theta"][0])
+    np.testing.assert_array_equal(expanded.astype(int), g["expanded"].astype(int))
+
+
+def test_output_perturbation_golden(golden_dir):
+    g = _read_kv_golden(golden_dir, "output_perturbation.txt")
+    K = np.stack([np.log(g["a"]), np.zeros(3)], axis=1)
+    V = g["V"].reshape(3, 2)
+    q = np.array([math.sqrt(2), 0.0])
+    subset = g["subset"].astype(int)
+    assert O.output_perturbation(q, K, V, subset) == pytest.approx(g["L"][0], rel=1e-12)
+    W = g["W_O_h"].reshape(2, 2)
+    assert O.output_perturbation(q, K, V, subset, W) == pytest.approx(g["L_projected"][0], rel=1e-12)
+    # the full set perturbs nothing
+    assert O.output_perturbation(q, K, V, np.arange(3), W) == pytest.approx(0.0, abs=1e-15)
