@@ -232,6 +232,20 @@ QE_API int qe_promote(qe_ctx* ctx, int unit, const int32_t* win_ids, int n,
 QE_API int qe_int2_quantize(const void* x, int T, int D, int dtype, uint8_t* codes,
                             uint32_t* meta, qe_stream_t stream);
 
+/* qe_ledger_read - the write-once INT2 ledger entry of one window ("Resumo Técnico: QEvict",
+ * Hierarquia Recuperável: Livro de Registro de Quantização de Escrita Única), in the row-major
+ * form of qe_int2_quantize. Inside the workspace an entry is stored in 16-token blocks arranged
+ * for the decode kernel's tensor-core operands; this call is how a caller inspects it.
+ *   unit in [0, B*Hkv), win in [0, max_windows).
+ *   codes_k, codes_v [dev]: [window][D/4] bytes (element 4j+e of a token in bits 2e of byte j).
+ *   meta_k, meta_v [dev]: [window][D/16] u32 = fp16 scale (low half) | fp16 zero (high half).
+ *   found [dev, int32]: 1 when the window has a ledger entry (the outputs are then written),
+ *     0 when it has none (nothing else is written).
+ * QE_ERR_INVALID_ARG for a null or misaligned pointer or an index out of range; QE_ERR_STATE
+ * before the prefill. Asynchronous on `stream`; allocates nothing. */
+QE_API int qe_ledger_read(qe_ctx* ctx, int unit, int win, uint8_t* codes_k, uint32_t* meta_k,
+                          uint8_t* codes_v, uint32_t* meta_v, int32_t* found, qe_stream_t stream);
+
 /* qe_vwo_l1norm - N[g][r][j] = || V[g][r][:] @ W_O^{h} ||_1 with h = (g % Hkv)*G + j, on
  * tensor cores (tcgen05, accumulators in TMEM).
  *   V [dev]: [n_groups][rows][D] dtype. W_O [dev]: [Hq*D][hidden] dtype.

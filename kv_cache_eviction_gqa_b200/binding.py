@@ -78,6 +78,7 @@ def lib():
             "qe_diag_tiers": (i, [vp, vp, vp, i, i, i, vp, vp]),
             "qe_diag_fmm_scratch_bytes": (sz, [i, i]),
             "qe_diag_fmm": (i, [vp, vp, ll, i, vp, i, i, i, i, i, i, i, vp, vp, sz, vp]),
+            "qe_ledger_read": (i, [vp, i, i, vp, vp, vp, vp, vp, vp]),
             "qe_status": (i, [vp, C.POINTER(C.c_int)]),
             "qe_step_index": (i, [vp]),
             "qe_length": (i, [vp]),
@@ -269,31 +270,38 @@ class QEvictContext:
             "route_stats": self._view(L.route_stats, U * 8, torch.int32, (U, 8)),
         }
 
-    def ledger_entry(self, unit: int, win: int):
-        """Decode one window's INT2 ledger entry into (codes_K, s_K, z_K, codes_V, s_V, z_V).
-
-        Layout of an entry (window w, head dim D): codes K [w][D/4] bytes | codes V | meta K
-        [w][D/16] u32 (fp16 scale low, fp16 zero high) | meta V.
-        """
-        st = self.state()
-        slot = int(st["win_slot"][unit, win])
-        if slot < 0:
-            return None
-        w, D = self.shape.window, self.shape.D
-        raw = st["slots"][unit, slot].cpu().numpy()
+    def ledger_entry(self, unit: int, win: int, stream=None):
+        """One window's INT2 ledger entry as (codes_K, s_K, z_K, codes_V, s_V, z_V) NumPy arrays
+        (codes [window][D] in 0..3, scales and zeros [window][D/16] float16), read through
+        qe_ledger_read; None when the window has no entry."""
         import numpy as np
+        w, D = self.shape.window, self.shape.D
+        dev = self.workspace.device
+        ck = torch.empty((w, D // 4), dtype=torch.uint8, device=dev)
+        cv = torch.empty_like(ck)
+        mk = torch.empty((w, D // 16), dtype=torch.int32, device=dev)
+        mv = torch.empty_like(mk)
+        found = torch.zeros(1, dtype=torch.int32, device=dev)
+        _check(lib().qe_ledger_read(self._h, unit, win, _ptr(ck), _ptr(mk), _ptr(cv), _ptr(mv), _ptr(found),
+                                    _stream(stream)), "qe_ledger_read")
+        if stream is None:
+            torch.cuda.synchronize(dev)
+        else:
+            stream.synchronize()
+        if int(found.item()) == 0:
+            return None
+
         def codes(b):
-            b = b.reshape(w, D // 4)
+            b = b.cpu().numpy()
             return np.stack([(b >> (2 * e)) & 3 for e in range(4)], -1).reshape(w, D)
-        def meta(b):
-            m = b.view(np.uint32).reshape(w, D // 16)
+
+        def meta(m):
+            m = m.cpu().numpy().view(np.uint32)
             return ((m & 0xFFFF).astype(np.uint16).view(np.float16),
                     (m >> 16).astype(np.uint16).view(np.float16))
-        n = w * D // 4
-        ck, cv = codes(raw[:n]), codes(raw[n:2 * n])
-        sk, zk = meta(raw[2 * n:3 * n])
-        sv, zv = meta(raw[3 * n:4 * n])
-        return ck, sk, zk, cv, sv, zv
+        sk, zk = meta(mk)
+        sv, zv = meta(mv)
+        return codes(ck), sk, zk, codes(cv), sv, zv
 
 
 # ---------------------------------------------------------------------------------

@@ -289,6 +289,16 @@ QE_API int qe_vwo_l1norm(const void* V, int n_groups, int rows, int D, int dtype
                     (cudaStream_t)s);
 }
 
+QE_API int qe_ledger_read(qe_ctx* c, int unit, int win, uint8_t* codes_k, uint32_t* meta_k, uint8_t* codes_v,
+                          uint32_t* meta_v, int32_t* found, qe_stream_t s) {
+  if (!c || !codes_k || !meta_k || !codes_v || !meta_v || !found) return QE_ERR_INVALID_ARG;
+  if (!c->loaded) return QE_ERR_STATE;
+  if (unit < 0 || unit >= c->lay.units || win < 0 || win >= c->lay.max_windows) return QE_ERR_INVALID_ARG;
+  if (!qe_aligned(meta_k, 4) || !qe_aligned(meta_v, 4) || !qe_aligned(found, 4)) return QE_ERR_INVALID_ARG;
+  c->last_stream = (cudaStream_t)s;
+  return launch_ledger_read(c, unit, win, codes_k, meta_k, codes_v, meta_v, found, (cudaStream_t)s);
+}
+
 QE_API int qe_status(qe_ctx* c, int* detail) {
   if (!c) return QE_ERR_INVALID_ARG;
   int32_t h[4] = {0, 0, 0, 0};

@@ -63,7 +63,8 @@ __device__ __forceinline__ void append_token(const DevState& st, int u, int pos,
 }
 
 // The same append run by one warp (lanes 0..31, D/8 <= 32), synchronising the warp only.
-__device__ __forceinline__ void append_token_warp(const DevState& st, int u, int pos, const uint4* k_new,
+// Returns (in every lane) the page that received the token, -1 if none could be taken.
+__device__ __forceinline__ int append_token_warp(const DevState& st, int u, int pos, const uint4* k_new,
                                                   const uint4* v_new, uint4* tailV) {
   const int lane = threadIdx.x & 31;
   const int b = u / st.Hkv, kvh = u % st.Hkv;
@@ -111,4 +112,5 @@ __device__ __forceinline__ void append_token_warp(const DevState& st, int u, int
   }
   asm volatile("fence.proxy.async.global;" ::: "memory");
   __syncwarp();
+  return page;
 }

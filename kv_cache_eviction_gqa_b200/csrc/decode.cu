@@ -6,49 +6,45 @@
 // readable by attention (Metodologia 2); GQA decode path (Implementação).
 // "Resumo Técnico: CriticalKV" - Etapa 2: the perturbation score A_i * ||V_i W_O||_1.
 //
-// Work split. Per unit u = (b, g) the live windows are [full windows | INT2 windows | tail].
+// Work split. Per unit u = (b, g) the live windows are [full windows | tail | INT2 windows].
 // The unit's S CTAs form one thread-block cluster; CTA s takes the s-th S-th of the full
 // windows and of the INT2 windows (the tail counts as one more INT2 window of the last CTA),
-// so every SM streams the same mix of bandwidth-heavy full pages and arithmetic-heavy INT2
-// entries. Inside a CTA each warp takes whole windows round-robin and streams them through
-// its own ring of shared-memory stages (completion on an mbarrier per stage): a full page
-// arrives as 128-byte-swizzled TMA boxes from a tensor map over the page pool, an INT2
-// ledger entry or a tail page as one 1-D bulk copy, each with its tokens' projected-value norms.
+// so every SM streams the same mix of bandwidth-heavy full pages and compact INT2 entries.
+// Inside a CTA each warp takes whole windows round-robin and streams them through its own
+// ring of shared-memory stages (completion on an mbarrier per stage): a full or tail page
+// arrives as 128-byte-swizzled TMA boxes from a tensor map over the page pool, an INT2 ledger
+// entry as one 1-D bulk copy, each with its tokens' projected-value norms.
 //
-// Full-precision windows run on the warp-level tensor cores (m16n8k16, f32 accumulate):
-// S = Q K^T with the G query rows padded to 16, then O^T = V^T P^T with P split into two
-// 16-bit parts so the product keeps float32 accuracy. A decode step has G <= 8 query rows per
-// KV head; a tcgen05 tile (M >= 64) would be mostly padding and its TMEM round trip buys
-// nothing on a path that HBM bounds, so these pages stay on mma.sync.
+// Every tier runs on the warp-level tensor cores (mma.sync, f32 accumulate) in one register
+// layout: the G query heads of the group are the rows of S = Q K^T (padded to 16), 16 tokens
+// are its columns, so lane (r, t) holds head r's scores of tokens 2t, 2t+1, 8+2t, 9+2t - which
+// is exactly the B fragment of O^T = V^T P^T. A decode step has G <= 8 query rows per KV head;
+// a tcgen05 tile (M >= 64) would be mostly padding and its TMEM round trip buys nothing on a
+// path that HBM bounds, so the decode stays on mma.sync.
 //
-// INT2 and tail windows run on the CUDA cores. A token is handled by LPT = D / DPL lanes; lane
-// `sub` owns the DPL contiguous head-dim elements [DPL*sub, DPL*sub + DPL), i.e. one INT2
-// group (DPL = 16) or half of one (DPL = 8), so it needs one scale/zero per token. With
-// DPL = 16 the two 8-element chunks of a lane are loaded in a lane-dependent order (register
-// chunk c holds memory chunk c ^ sw) so that every 16-byte shared-memory load instruction of
-// the warp touches each bank once. A warp works on TPS = 32 / LPT tokens at a time; q and the
-// accumulators of the G query heads stay in registers as float pairs and all multiply-adds
-// are packed (f32x2). A token's G dot products are summed over its lanes with a butterfly, so
-// every lane of the group holds the scores and no weight broadcast is needed. Each lane group
-// keeps its own online-softmax state (log2 domain); the accumulators are rescaled only when
-// the running maximum grows by more than 2^8.
+// Full-precision pages: S from ldmatrix K tiles, P split into two 16-bit parts of the cache
+// dtype (hi + residual) so O keeps float32 accuracy, V^T by ldmatrix.trans.
 //
-// INT2 decoding without float conversions: a pair of 2-bit codes (even element E, odd E+1)
-// is shifted once into the mantissas of 4.0 and 1.0, giving x = 4 + c_E/4 and 1 + c_(E+1)/4
-// exactly; the affine map k = c*s + z is folded into the per-token scale (4s) and a per-pair
-// offset, so a score is 4s (q . x) + z sum(q) - 4s (4 sum(q_even) + sum(q_odd)).
+// INT2 blocks (16 tokens, layout in int2_block.cuh): a K or V value is c*s + z with a 2-bit code
+// c and an fp16 scale s and zero z per 16-element group. The codes enter the MMA exactly as
+// fp16 subnormals c * 4^i * 2^-24 (one mask per register); per group g
+//   S += s_g * (Q_g . C_g)  (one MMA per 8 tokens, then an f32x2 FMA by the token scales),
+//   S += Z (sum of q over each group)  (one m16n8k8 MMA per 8 tokens, q sums split hi + lo),
+//   O_g^T += C_g^T (P * s_g)  (one MMA per group; P * s rounded once to fp16),
+//   O^T += Z^T P  (one MMA per 16 tokens, P split hi + lo).
+// The powers 4^i and 2^-24 are folded into q, the staged scales and the accumulator. The
+// block's scales are converted to float32 once per warp into a small staging area.
 //
-// Scoring without a second pass: at the end of each window every lane group records its
-// (max, sum_i 2^(s_i-max), sum_i 2^(s_i-max) n_i) per head in its own slot. After the pass the
-// cluster merges the CTA partials through distributed shared memory into the unit's log-sum-
-// exp; each CTA writes its share of the output and adds the exact attention mass and
-// perturbation of the windows it streamed to the cumulative scores. The tail window's norms
-// are not known yet; its per-token attention is accumulated instead (tail_p) and folded in
-// when the window completes.
+// Scoring without a second pass: at the end of each window the warp records its
+// (max, sum_i 2^(s_i-max), sum_i 2^(s_i-max) n_i) per head. After the pass the cluster merges
+// the CTA partials through distributed shared memory into the unit's log-sum-exp; each CTA
+// writes its share of the output and adds the exact attention mass and perturbation of the
+// windows it streamed to the cumulative scores. The tail window's norms are not known yet;
+// its per-token attention is accumulated instead (tail_p) and folded in when it completes.
 #include <math.h>
 
 #include "append.cuh"
-#include "int2.cuh"
+#include "int2_block.cuh"
 #include "qe_internal.cuh"
 #include "tc_common.cuh"
 #include "warp_mma.cuh"
@@ -64,44 +60,26 @@ namespace {
 #ifndef QE_DECODE_MINB
 #define QE_DECODE_MINB 4
 #endif
-#ifndef QE_DECODE_FULL_LAST
-#define QE_DECODE_FULL_LAST 0  // 1: odd warps stream their full-precision windows last
-#endif
-#ifndef QE_DECODE_SB
-#define QE_DECODE_SB 4
-#endif
 constexpr int kNW = QE_DECODE_NW;    // warps per CTA
 #define QE_MAX_SPLITS_CLUSTER 16          // CTAs per unit (one cluster, non-portable size)
 constexpr int kNST = QE_DECODE_NST;  // stages per warp
 constexpr float kRescale = 8.f;  // rescale the accumulators when the max grows by > 2^8
 
-// Per-window score partials: one slot per lane group of {max, sum p, sum p n} x G heads,
-// weights 2^(s - max) relative to the slot's max; an unused slot holds max -1e30 and zeros.
 struct DecodeArgs {
   DevState st;
   const void* q;     // [B][Hq][D]
   float* out;        // [B][Hq][D]
-  float* win_part;   // [U][Wmax][win_part_floats(D, G)]
+  float* win_part;   // [U][Wmax][3 G]: {max, sum p, sum p n} per head
   float* tail_s;     // [U][window][G]
   int splits;        // CTAs per unit = cluster size
   int tail_win, tail_len;
   float scale_log2;  // log2(e) / sqrt(D)
   // optional fused append of the step's token at position append_pos (k_new != nullptr): the
-  // CTA that streams the tail window writes it before its first copy
+  // warp that streams the tail window writes it before issuing the tail's copies
   const uint4* k_new;
   const uint4* v_new;
   uint4* tailV;
   int append_pos;
-};
-
-template <int D, int G>
-struct Map {
-  static constexpr int DPL = decode_dpl(G);    // head-dim elements per lane
-  static constexpr int LPT = D / DPL;          // lanes per token
-  static constexpr int TPS = 32 / LPT;         // tokens per warp step
-  static constexpr int SB = (16 / TPS) < QE_DECODE_SB ? (16 / TPS) : QE_DECODE_SB;  // tokens per group per batch
-  static constexpr int SBT = SB * TPS;         // tokens per batch (divides 16)
-  static constexpr int NP = DPL / 2;           // float pairs per lane
 };
 
 // 2^x with the hardware approximation (relative error about 2^-22; results below 2^-126
@@ -131,107 +109,86 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// Chunk order of a lane (DPL = 16): register chunk c holds memory chunk c ^ sw. It may
-// depend on `sub` only: lanes with the same `sub` in different token groups must hold the
-// same elements in the same registers, since the groups are summed register by register.
-// At D = 64 a row is one bank cycle and no lane-only order helps; those loads stay 2-way.
-template <int D, int DPL>
-__device__ __forceinline__ int chunk_swap(int sub, int grp) {
-  (void)grp;
-  if constexpr (DPL == 16 && D == 128) return (sub >> 2) & 1;
-  else return 0;
-}
-
-template <typename T>
-__device__ __forceinline__ void cvt8(const uint4 w, float2* x) {
-  x[0] = make_float2(Elem<T>::lo(w.x), Elem<T>::hi(w.x));
-  x[1] = make_float2(Elem<T>::lo(w.y), Elem<T>::hi(w.y));
-  x[2] = make_float2(Elem<T>::lo(w.z), Elem<T>::hi(w.z));
-  x[3] = make_float2(Elem<T>::lo(w.w), Elem<T>::hi(w.w));
-}
-
-// the lane's DPL elements of a row as float pairs
-template <typename T, int DPL>
-__device__ __forceinline__ void load_row(const T* row, int sub, int sw, float2 (&x)[DPL / 2]) {
-  const uint4* p = reinterpret_cast<const uint4*>(row + DPL * sub);
-  if constexpr (DPL == 16) {
-    cvt8<T>(p[sw], x);
-    cvt8<T>(p[sw ^ 1], x + 4);
-  } else {
-    cvt8<T>(p[0], x);
-  }
-}
-
-// Codes E (even) and E+1 from one shift: the pair {4 + c_E/4, 1 + c_(E+1)/4}. Code E lands in
-// mantissa bits 19-20 of 4.0 (4 * (1 + c/16)) and code E+1 in bits 21-22 of 1.0, so both
-// values are exact and the code's contribution is c/4 in either case; only the constant part
-// differs (4 for even elements, 1 for odd ones).
-template <int E>
-__device__ __forceinline__ float2 code_pair(uint32_t bits) {
-  constexpr int sh = 19 - 2 * E;
-  const uint32_t v = sh >= 0 ? (bits << (sh >= 0 ? sh : 0)) : (bits >> (sh < 0 ? -sh : 0));
-  return make_float2(__uint_as_float((v & 0x00180000u) | 0x40800000u),
-                     __uint_as_float((v & 0x00600000u) | 0x3f800000u));
-}
-
-template <int NP>
-__device__ __forceinline__ void decode_codes(uint32_t bits, float2 (&x)[NP]) {
-  x[0] = code_pair<0>(bits);
-  x[1] = code_pair<2>(bits);
-  x[2] = code_pair<4>(bits);
-  x[3] = code_pair<6>(bits);
-  if constexpr (NP == 8) {
-    x[4] = code_pair<8>(bits);
-    x[5] = code_pair<10>(bits);
-    x[6] = code_pair<12>(bits);
-    x[7] = code_pair<14>(bits);
-  }
-}
-
-// the lane's codes of one row, with register chunk c = memory chunk c ^ sw in bits 16c..
-template <int DPL>
-__device__ __forceinline__ uint32_t load_codes(const uint8_t* row, int sub, int sw) {
-  if constexpr (DPL == 16) {
-    const uint32_t b = reinterpret_cast<const uint32_t*>(row)[sub];
-    return sw ? __funnelshift_l(b, b, 16) : b;
-  } else {
-    return reinterpret_cast<const uint16_t*>(row)[sub];
-  }
-}
-
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
-// Shared-memory stage of one task (1024-byte aligned). A full-precision page arrives as TMA
-// boxes of 16 rows x 64 elements with the 128-byte swizzle (box (part, x) at
-// (part * D/64 + x) * 2048, part 0 = K rows, 1 = V rows), so the 8 rows of every ldmatrix
-// tile sit in distinct banks; tail pages and INT2 ledger entries are 1-D bulk copies in their
-// contiguous layout. Up to 64 tokens' norms follow at PAGE_BYTES.
-template <int D, int G>
+// {lo, hi} rounded to an fp16 pair (lo in the low half)
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ float h_lo(uint32_t x) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(x & 0xffffu)));
+}
+__device__ __forceinline__ float h_hi(uint32_t x) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(x >> 16)));
+}
+
+// fp16 MMAs with f32 accumulate: m16n8k16 (A 4 regs, B 2 regs) and m16n8k8 (A 2 regs, B 1 reg)
+__device__ __forceinline__ void mma_h16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                        uint32_t b0, uint32_t b1) {
+  MmaOp<__half>::run(c, a0, a1, a2, a3, b0, b1);
+}
+__device__ __forceinline__ void mma_h8(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5}, {%6}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(b0));
+}
+
+// Register i (0..3) of a packed code word: the codes at bits [2i, 2i+1] of each 16-bit half as
+// the fp16 subnormals c * 4^i * 2^-24.
+template <int I>
+__device__ __forceinline__ uint32_t code_reg(uint32_t x) {
+  return x & (0x00030003u << (2 * I));
+}
+
+// Shared memory of a warp: a ring of kNST page stages (1024-byte aligned) and, elsewhere, a ring
+// of kNST norm stages and the INT2 scale staging. A full-precision or tail page arrives as TMA
+// boxes of 16 rows x 64 elements with the 128-byte swizzle (box (part, x) at (part * D/64 + x) *
+// 2048, part 0 = K rows, 1 = V rows), so the 8 rows of every ldmatrix tile sit in distinct
+// banks; an INT2 ledger entry is a 1-D bulk copy (w/16 blocks of 16*D bytes, at most a page).
+// A norm stage holds the task's tokens' norms (window * G floats, runtime size).
+template <int D>
 struct StageLayout {
   static constexpr int PAGE_BYTES = 2 * QE_PAGE * D * 2;            // K rows then V rows
-  static constexpr int RAW = PAGE_BYTES + 64 * G * 4;
-  static constexpr int BYTES = (RAW + 1023) / 1024 * 1024;
+  static constexpr int BYTES = (PAGE_BYTES + 1023) / 1024 * 1024;
 };
+// Per-warp staging of one INT2 block's scales in float32: [K, V][t (0..3)][group][4 tokens
+// 2t, 2t+1, 8+2t, 9+2t], rows padded by 4 floats so the four t rows sit in distinct banks.
+template <int D>
+struct ScaleStage {
+  static constexpr int ROW = (D / 16) * 4 + 4;  // floats per t row
+  static constexpr int FLOATS = 2 * 4 * ROW;
+  static constexpr int BYTES = FLOATS * 4;
+};
+// bytes of one norm stage for a window of w tokens (16-byte multiple)
+__host__ __device__ constexpr int norm_stage_bytes(int w, int G) { return (w * G * 4 + 15) / 16 * 16; }
+// per-warp auxiliary area (norm ring, then scale staging) and the whole dynamic shared memory
+template <int D>
+__host__ __device__ constexpr int aux_bytes(int w, int G) { return 3 * norm_stage_bytes(w, G) + ScaleStage<D>::BYTES; }
 
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
     decode_kernel(const __grid_constant__ CUtensorMap tmP, DecodeArgs a) {
-  using M = Map<D, G>;
-  constexpr int DPL = M::DPL, LPT = M::LPT, TPS = M::TPS, SB = M::SB, SBT = M::SBT, NP = M::NP;
-  using SL = StageLayout<D, G>;
+  using BL = Int2Block<D>;
+  constexpr int G8 = BL::G8, WPL = BL::WPL;
+  using SL = StageLayout<D>;
   constexpr int PAGE_BYTES = SL::PAGE_BYTES;
   constexpr int STAGE = SL::BYTES;
+  constexpr int SROW = ScaleStage<D>::ROW;
+  static_assert(kNST == 3, "aux_bytes assumes three stages");
   extern __shared__ __align__(128) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const DevState& st = a.st;
   const int u = blockIdx.x / a.splits, split = blockIdx.x % a.splits;
   const int b = u / st.Hkv, kvh = u % st.Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int grp = lane / LPT, sub = lane % LPT;
-  const int sw = chunk_swap<D, DPL>(sub, grp);
+  const int g8 = lane >> 2, t4 = lane & 3;
   const int w = st.window, ppw = st.ppw;
   const size_t ub = (size_t)u * st.Wmax;
-  const int gi = DPL * sub / 16;  // this lane's INT2 group within a row
+  const float sl = a.scale_log2;
 
   // this split's share of each tier
   const int nf = st.stacks[u * 4 + 2], nq = st.stacks[u * 4 + 3];
@@ -242,48 +199,30 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
   const int q0 = (int)((long long)nqv * split / a.splits);
   const int q1 = min(nq, (int)((long long)nqv * (split + 1) / a.splits));
   const int has_tail = (a.tail_len > 0 && split == a.splits - 1) ? 1 : 0;
-  const int nF = f1 - f0, nQ = q1 - q0, nJ = nF + nQ + has_tail;
-  // fused append: the warp that streams the tail window writes the new token first (its tail
-  // task comes last, after this warp's own fence); the other warp starts at once
-  if (a.k_new != nullptr && has_tail && warp == (nJ - 1) % kNW)
-    append_token_warp(st, u, a.append_pos, a.k_new, a.v_new, a.tailV);
+  const int nF = f1 - f0, nQ = q1 - q0, nJ = nF + has_tail + nQ;
 
+  const int NSB = norm_stage_bytes(w, G);
   uint8_t* ring = smem + warp * kNST * STAGE;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kNW * kNST * STAGE) + warp * kNST;
+  uint8_t* aux = smem + kNW * kNST * STAGE + kNW * kNST * 8 + warp * aux_bytes<D>(w, G);
+  uint8_t* nring = aux;                                           // [kNST][NSB]
+  float* sst = reinterpret_cast<float*>(aux + kNST * NSB);        // scale staging
   if (lane == 0) {
     for (int s = 0; s < kNST; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
   }
   __syncwarp();
 
-  // SIMT state for the INT2 and tail windows (set up after the full-precision phase): the G
-  // query heads of this group, this lane's DPL elements, in the log2 domain; per lane-group
-  // online-softmax state; lw/nw: sums of the current window
-  float2 q[G][NP];
-  float qsum[G];   // sum of the lane's q elements
-  float qsum2[G];  // 4 * (sum over even elements) + (sum over odd elements): the constant part of q . x
-  float2 acc[G][NP];
-  float2 zacc[G];  // INT2 value offsets (even, odd element) weighted by p * ...
-  float m[G], lsum[G], lw[G], nw[G];
-
-  // virtual index j of this split -> (kind, list index)
-  auto kind_of = [&](int j) { return j < nF ? 0 : (j < nF + nQ ? 1 : 2); };  // full, int2, tail
-  auto list_idx = [&](int j) { return j < nF ? f0 + j : nf + q0 + (j - nF); };
+  // virtual index j of this split: [0, nF) full, nF the tail (when present), then INT2
+  auto kind_of = [&](int j) { return j < nF ? 0 : (j < nF + has_tail ? 2 : 1); };  // full, int2, tail
+  auto list_idx = [&](int j) { return j < nF ? f0 + j : nf + q0 + (j - nF - has_tail); };
   auto n_tasks = [&](int j) {
     const int k = kind_of(j);
     return k == 0 ? ppw : (k == 1 ? 1 : (a.tail_len + QE_PAGE - 1) / QE_PAGE);
   };
-  // This warp's windows are j = warp + kNW * r, r < n_own; the first n_own_full are
-  // full-precision. With QE_DECODE_FULL_LAST, odd warps stream their full-precision windows
-  // last (measured: no gain at c2, so off). Tasks are addressed by the ordinal o of the window
-  // in this warp's order.
+  // This warp's windows are j = warp + kNW * o, o < n_own (kinds in the order above).
   const int n_own = nJ > warp ? (nJ - warp + kNW - 1) / kNW : 0;
-  const int n_own_full = nF > warp ? (nF - warp + kNW - 1) / kNW : 0;
-  const bool full_last = QE_DECODE_FULL_LAST && (warp & 1) && n_own_full > 0 && n_own_full < n_own;
-  auto jmap = [&](int o) {
-    const int r = !full_last ? o : (o < n_own - n_own_full ? n_own_full + o : o - (n_own - n_own_full));
-    return warp + kNW * r;
-  };
+  auto jmap = [&](int o) { return warp + kNW * o; };
   auto advance = [&](int& o, int& pg) {
     if (++pg >= n_tasks(jmap(o))) {
       pg = 0;
@@ -303,7 +242,7 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
     if (jj < nJ) {
       const int kd = kind_of(jj);
       const int win = kd == 0 ? st.full_list[ub + f0 + jj]
-                              : (kd == 1 ? st.int2_list[ub + q0 + (jj - nF)] : a.tail_win);
+                              : (kd == 1 ? st.int2_list[ub + q0 + (jj - nF - has_tail)] : a.tail_win);
       if (win >= 0 && win < st.Wmax) {
         e_win = win;
         if (kd == 1) {
@@ -316,6 +255,8 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
       }
     }
   };
+  // fused append: page of the step's token (written by this warp just before the tail's copies)
+  int app_pg = -1, app_page = -1;
   // issue the copies of task (window ordinal r, page pg) into stage s (all lanes call)
   auto issue = [&](int r, int pg, int s) {
     const int j = jmap(r);
@@ -323,20 +264,27 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
     const int src = r - rb;
     const int win = __shfl_sync(0xffffffffu, e_win, src);
     const int sel = pg == 0 ? e_id[0] : (pg == 1 ? e_id[1] : (pg == 2 ? e_id[2] : e_id[3]));
-    const int id = __shfl_sync(0xffffffffu, sel, src);
+    int id = __shfl_sync(0xffffffffu, sel, src);
     uint8_t* dst = ring + s * STAGE;
+    uint8_t* ndst = nring + s * NSB;
     uint64_t* bar = &bars[s];
     const int k = kind_of(j);
+    if (k == 2 && pg == 0 && a.k_new != nullptr) {
+      // the step's token goes into the tail window before its pages are copied
+      app_page = append_token_warp(st, u, a.append_pos, a.k_new, a.v_new, a.tailV);
+      app_pg = (a.append_pos % w) / QE_PAGE;
+    }
+    if (k == 2 && pg == app_pg) id = app_page;
     fence_proxy_async_smem();
     if (lane != 0) return;
-    if (k == 0) {
-      // full-precision page: 2 * D/64 swizzled TMA boxes, then the page's norms
+    if (k != 1) {
+      // full-precision or tail page: 2 * D/64 swizzled TMA boxes (+ the page's norms)
       if (win < 0 || id < 0 || id >= st.P) {
         qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
         mbar_arrive_expect_tx(bar, 0);
         return;
       }
-      const uint32_t nb = QE_PAGE * G * 4;
+      const uint32_t nb = k == 0 ? QE_PAGE * G * 4 : 0;
       mbar_arrive_expect_tx(bar, PAGE_BYTES + nb);
       const int row0 = (u * st.P + id) * 2 * QE_PAGE;
 #pragma unroll
@@ -344,126 +292,87 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
 #pragma unroll
         for (int xb = 0; xb < D / 64; ++xb)
           tc::tma_load_2d(dst + (part * (D / 64) + xb) * 2048, &tmP, xb * 64, row0 + part * QE_PAGE, bar);
-      bulk_g2s(dst + PAGE_BYTES, st.norms + ((size_t)u * st.norm_pitch + (size_t)win * w + pg * QE_PAGE) * G, nb,
-               bar);
+      if (k == 0)
+        bulk_g2s(ndst, st.norms + ((size_t)u * st.norm_pitch + (size_t)win * w + pg * QE_PAGE) * G, nb, bar);
       return;
     }
-    if (k == 1) {
-      if (win < 0 || id < 0 || id >= st.S) {
-        qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
-        mbar_arrive_expect_tx(bar, 0);
-        return;
-      }
-      const uint32_t nb = (uint32_t)(w * G * 4);
-      mbar_arrive_expect_tx(bar, (uint32_t)st.slot_bytes + nb);
-      bulk_g2s(dst, st.slots + ((size_t)u * st.S + id) * st.slot_bytes, (uint32_t)st.slot_bytes, bar);
-      bulk_g2s(dst + PAGE_BYTES, st.norms + ((size_t)u * st.norm_pitch + (size_t)win * w) * G, nb, bar);
-    } else {
-      if (win < 0 || id < 0 || id >= st.P) {
-        qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
-        mbar_arrive_expect_tx(bar, 0);
-        return;
-      }
-      const uint8_t* src_p = st.pages + ((size_t)u * st.P + id) * st.page_bytes;
-      {
-        mbar_arrive_expect_tx(bar, PAGE_BYTES);
-        bulk_g2s(dst, src_p, PAGE_BYTES, bar);
-      }
+    if (win < 0 || id < 0 || id >= st.S) {
+      qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
+      mbar_arrive_expect_tx(bar, 0);
+      return;
     }
+    const uint32_t nb = (uint32_t)(w * G * 4);
+    mbar_arrive_expect_tx(bar, (uint32_t)st.slot_bytes + nb);
+    bulk_g2s(dst, st.slots + ((size_t)u * st.S + id) * st.slot_bytes, (uint32_t)st.slot_bytes, bar);
+    bulk_g2s(ndst, st.norms + ((size_t)u * st.norm_pitch + (size_t)win * w) * G, nb, bar);
   };
 
-  // softmax bookkeeping for one batch: s[i][h] are the scores of the group's SB tokens
-  // (-inf where invalid); on return they hold the weights 2^(s - m). The running max m
-  // starts at a finite -1e30 so that 2^(-inf - m) = 0 needs no guard. One rarely taken
-  // branch per batch covers every head.
-  auto online = [&](float (&s)[SB][G]) {
-    float mb[G];
-    bool grow = false;
+  // online softmax state of head g8 (lanes g8 >= G carry padding rows): running max (log2
+  // domain), sum of weights, and the current window's sums of weights and weighted norms
+  float mh = -1e30f, lh = 0.f, lwh = 0.f, nwh = 0.f;
+  const float hmask = g8 < G ? 1.f : 0.f;
+  // O^T accumulators: oacc[m] holds rows (head-dim elements) 16m + g8 (c0, c1) and 16m + 8 + g8
+  // (c2, c3), columns (heads) 2 t4 and 2 t4 + 1. zacc: the INT2 zero-point part, rows = groups.
+  float oacc[G8][4];
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      mb[h] = s[0][h];
+  for (int m = 0; m < G8; ++m) oacc[m][0] = oacc[m][1] = oacc[m][2] = oacc[m][3] = 0.f;
+  float zacc[4] = {0.f, 0.f, 0.f, 0.f};
+
+  // Softmax bookkeeping of one 16-token task: s holds head g8's log2-domain scores of tokens
+  // 2t4, 2t4+1, 8+2t4, 9+2t4 (-inf where absent); p receives their weights 2^(s - max). The
+  // running max starts at a finite -1e30 so that 2^(-inf - m) = 0 needs no guard; one rarely
+  // taken branch rescales the accumulators when the max grows by more than 2^kRescale.
+  auto softmax = [&](const float (&s)[4], float (&p)[4], const float* nrm) {
+    float mx = fmaxf(fmaxf(s[0], s[1]), fmaxf(s[2], s[3]));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const bool grow = mx > mh + kRescale;
+    if (__any_sync(0xffffffffu, grow)) {
+      const float mn = grow ? mx : mh;
+      const float f = ex2(mh - mn);
+      lh *= f;
+      lwh *= f;
+      nwh *= f;
+      mh = mn;
+      // O^T columns 2 t4, 2 t4 + 1 belong to the heads of lanes 8 t4 and 8 t4 + 4
+      const float fa = __shfl_sync(0xffffffffu, f, 8 * t4);
+      const float fb = __shfl_sync(0xffffffffu, f, 8 * t4 + 4);
 #pragma unroll
-      for (int i = 1; i < SB; ++i) mb[h] = fmaxf(mb[h], s[i][h]);
-      grow |= mb[h] > m[h] + kRescale;
-    }
-    if (grow) {
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float mn = mb[h] > m[h] + kRescale ? mb[h] : m[h];
-        const float f = ex2(m[h] - mn);
-        const float2 f2 = make_float2(f, f);
-#pragma unroll
-        for (int e = 0; e < NP; ++e) acc[h][e] = __fmul2_rn(acc[h][e], f2);
-        zacc[h] = __fmul2_rn(zacc[h], f2);
-        lsum[h] *= f;
-        lw[h] *= f;
-        nw[h] *= f;
-        m[h] = mn;
+      for (int m = 0; m < G8; ++m) {
+        oacc[m][0] *= fa;
+        oacc[m][1] *= fb;
+        oacc[m][2] *= fa;
+        oacc[m][3] *= fb;
       }
+      zacc[0] *= fa;
+      zacc[1] *= fb;
     }
 #pragma unroll
-    for (int i = 0; i < SB; ++i)
-#pragma unroll
-      for (int h = 0; h < G; ++h) s[i][h] = ex2(s[i][h] - m[h]);
-  };
-
-  // sum every score over the LPT lanes of its token (pairs of heads added as f32x2)
-  auto butterfly = [&](float (&s)[SB][G]) {
-#pragma unroll
-    for (int o = LPT / 2; o; o >>= 1)
-#pragma unroll
-      for (int i = 0; i < SB; ++i) {
-#pragma unroll
-        for (int h = 0; h + 1 < G; h += 2) {
-          const float2 r = make_float2(__shfl_xor_sync(0xffffffffu, s[i][h], o),
-                                       __shfl_xor_sync(0xffffffffu, s[i][h + 1], o));
-          const float2 v = __fadd2_rn(make_float2(s[i][h], s[i][h + 1]), r);
-          s[i][h] = v.x;
-          s[i][h + 1] = v.y;
-        }
-        if constexpr (G % 2) s[i][G - 1] += __shfl_xor_sync(0xffffffffu, s[i][G - 1], o);
-      }
-  };
-
-  // window sums of one token: lw += p, nw += p * n (pairs of heads as f32x2)
-  auto window_sums = [&](const float (&p)[G], const float* n) {
-#pragma unroll
-    for (int h = 0; h + 1 < G; h += 2) {
-      const float2 pp = make_float2(p[h], p[h + 1]);
-      const float2 l2 = __fadd2_rn(make_float2(lw[h], lw[h + 1]), pp);
-      // n + h is 8-byte aligned only when G is even (n = norms + t * G)
-      const float2 nn = G % 2 == 0 ? *reinterpret_cast<const float2*>(n + h) : make_float2(n[h], n[h + 1]);
-      const float2 n2 = ffma2(pp, nn, make_float2(nw[h], nw[h + 1]));
-      lw[h] = l2.x;
-      lw[h + 1] = l2.y;
-      nw[h] = n2.x;
-      nw[h + 1] = n2.y;
-    }
-    if constexpr (G % 2) {
-      lw[G - 1] += p[G - 1];
-      nw[G - 1] = fmaf(p[G - 1], n[G - 1], nw[G - 1]);
+    for (int i = 0; i < 4; ++i) p[i] = hmask * ex2(s[i] - mh);
+    const float psum = (p[0] + p[1]) + (p[2] + p[3]);
+    lh += psum;
+    lwh += psum;
+    if (nrm != nullptr && g8 < G) {
+      nwh = fmaf(p[0], nrm[(2 * t4) * G + g8], nwh);
+      nwh = fmaf(p[1], nrm[(2 * t4 + 1) * G + g8], nwh);
+      nwh = fmaf(p[2], nrm[(8 + 2 * t4) * G + g8], nwh);
+      nwh = fmaf(p[3], nrm[(9 + 2 * t4) * G + g8], nwh);
     }
   };
-
-  // QK of one row of K for every head
-  auto qk_row = [&](const float2 (&kx)[NP], float (&out)[G]) {
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float2 d2 = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int e = 0; e < NP; ++e) d2 = ffma2(q[h][e], kx[e], d2);
-      out[h] = d2.x + d2.y;
+  // end of a window: its partial (max, sum p, sum p n) per head into the window's slot
+  auto window_end = [&](int li) {
+    float l2 = lwh + __shfl_xor_sync(0xffffffffu, lwh, 1);
+    l2 += __shfl_xor_sync(0xffffffffu, l2, 2);
+    float n2 = nwh + __shfl_xor_sync(0xffffffffu, nwh, 1);
+    n2 += __shfl_xor_sync(0xffffffffu, n2, 2);
+    if (t4 == 0 && g8 < G) {
+      float* wp = a.win_part + (ub + li) * win_part_floats(D, G) + g8;
+      wp[0] = mh;
+      wp[G] = l2;
+      wp[2 * G] = n2;
     }
-  };
-
-  // PV of one row of V for every head: acc[h] += p[h] * v
-  auto pv_row = [&](const float2 (&vx)[NP], const float (&p)[G]) {
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float2 p2 = make_float2(p[h], p[h]);
-#pragma unroll
-      for (int e = 0; e < NP; ++e) acc[h][e] = ffma2(p2, vx[e], acc[h][e]);
-    }
+    lwh = 0.f;
+    nwh = 0.f;
   };
 
   int o = 0, pg = 0;                  // window ordinal and page being computed
@@ -475,198 +384,130 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
   }
   int k = 0;
   bool ok = true;
-  const int g8 = lane >> 2, t4 = lane & 3;
 
-  // ---- full-precision pages on the tensor cores ----
-  // S = Q K^T with A = the G query rows (padded to 16, raw q), B = 8-token tiles of K
-  // (ldmatrix); lane (g8, t4) then holds head g8's scores of tokens 2t4, 2t4+1, 8+2t4, 9+2t4.
-  // O^T = V^T P^T with A = V^T (ldmatrix.trans) and B = P^T taken straight from those
-  // registers, split into two 16-bit parts so the product keeps float32 accuracy. At the end
-  // the partial (per head: max, sum of weights, O as [G][D]) goes to the stage consumed last
-  // (the next copy targets it only after the merge below).
-  auto mma_phase = [&]() -> const float* {
-      uint32_t qa[D / 16][2];
-      {
-        const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
-            reinterpret_cast<const T*>(a.q) + ((size_t)b * st.Hq + (size_t)kvh * G + (g8 < G ? g8 : 0)) * D);
-  #pragma unroll
-        for (int kc = 0; kc < D / 16; ++kc) {
-          qa[kc][0] = g8 < G ? qrow[kc * 8 + t4] : 0u;
-          qa[kc][1] = g8 < G ? qrow[kc * 8 + 4 + t4] : 0u;
-        }
-      }
-      float oacc[D / 16][4];
-  #pragma unroll
-      for (int mt = 0; mt < D / 16; ++mt) oacc[mt][0] = oacc[mt][1] = oacc[mt][2] = oacc[mt][3] = 0.f;
-      float mh = -1e30f, lh = 0.f, lwh = 0.f, nwh = 0.f;  // head g8: running max, sums
-      const float hmask = g8 < G ? 1.f : 0.f;
-      while (o < n_own && kind_of(jmap(o)) == 0) {
-        if (io < n_own) {
-          issue(io, ipg, issued % kNST);
-          advance(io, ipg);
-          ++issued;
-        }
-        const int s = k % kNST;
-        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[s], (k / kNST) & 1, st.status, 1000 + u));
-        if (!ok) break;
-        const uint8_t* stage = ring + s * STAGE;
-        const float* nrm = reinterpret_cast<const float*>(stage + PAGE_BYTES);
-        float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
-  #pragma unroll
-        for (int kc2 = 0; kc2 < D / 32; ++kc2) {
-          uint32_t kb[4];
-          ldsm_x4(kb, stage + swz<D>(0, lane & 7, kc2 * 32 + (lane >> 3) * 8));
-          MmaOp<T>::run(c0, qa[2 * kc2][0], 0u, qa[2 * kc2][1], 0u, kb[0], kb[1]);
-          MmaOp<T>::run(c0, qa[2 * kc2 + 1][0], 0u, qa[2 * kc2 + 1][1], 0u, kb[2], kb[3]);
-          ldsm_x4(kb, stage + swz<D>(0, 8 + (lane & 7), kc2 * 32 + (lane >> 3) * 8));
-          MmaOp<T>::run(c1, qa[2 * kc2][0], 0u, qa[2 * kc2][1], 0u, kb[0], kb[1]);
-          MmaOp<T>::run(c1, qa[2 * kc2 + 1][0], 0u, qa[2 * kc2 + 1][1], 0u, kb[2], kb[3]);
-        }
-        float mx = fmaxf(fmaxf(c0[0], c0[1]), fmaxf(c1[0], c1[1]));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        const float ms = mx * a.scale_log2;
-        const bool grow = ms > mh + kRescale;
-        if (__any_sync(0xffffffffu, grow)) {
-          const float mn = grow ? ms : mh;
-          const float f = ex2(mh - mn);
-          lh *= f;
-          lwh *= f;
-          nwh *= f;
-          mh = mn;
-          // O^T column pair (2 t4, 2 t4 + 1) belongs to heads held by lanes 8 t4 and 8 t4 + 4
-          const float fa = __shfl_sync(0xffffffffu, f, 8 * t4);
-          const float fb = __shfl_sync(0xffffffffu, f, 8 * t4 + 4);
-  #pragma unroll
-          for (int mt = 0; mt < D / 16; ++mt) {
-            oacc[mt][0] *= fa;
-            oacc[mt][1] *= fb;
-            oacc[mt][2] *= fa;
-            oacc[mt][3] *= fb;
-          }
-        }
-        const float p0 = hmask * ex2(fmaf(c0[0], a.scale_log2, -mh));
-        const float p1 = hmask * ex2(fmaf(c0[1], a.scale_log2, -mh));
-        const float p2 = hmask * ex2(fmaf(c1[0], a.scale_log2, -mh));
-        const float p3 = hmask * ex2(fmaf(c1[1], a.scale_log2, -mh));
-        const float psum = (p0 + p1) + (p2 + p3);
-        lh += psum;
-        lwh += psum;
-        if (g8 < G) {
-          nwh = fmaf(p0, nrm[(2 * t4) * G + g8], nwh);
-          nwh = fmaf(p1, nrm[(2 * t4 + 1) * G + g8], nwh);
-          nwh = fmaf(p2, nrm[(8 + 2 * t4) * G + g8], nwh);
-          nwh = fmaf(p3, nrm[(9 + 2 * t4) * G + g8], nwh);
-        }
-        uint32_t ph0, pl0, ph1, pl1;
-        MmaOp<T>::split(p0, p1, ph0, pl0);
-        MmaOp<T>::split(p2, p3, ph1, pl1);
-  #pragma unroll
-        for (int mt = 0; mt < D / 16; ++mt) {
-          uint32_t va[4];
-          ldsm_x4_t(va, stage + swz<D>(1, ((lane >> 4) << 3) + (lane & 7), mt * 16 + ((lane >> 3) & 1) * 8));
-          MmaOp<T>::run(oacc[mt], va[0], va[1], va[2], va[3], ph0, ph1);
-          MmaOp<T>::run(oacc[mt], va[0], va[1], va[2], va[3], pl0, pl1);
-        }
-        __syncwarp();
-        if (pg + 1 >= ppw) {
-          // end of a window: its partial (m, sum p, sum p n) per head
-          float l2 = lwh + __shfl_xor_sync(0xffffffffu, lwh, 1);
-          l2 += __shfl_xor_sync(0xffffffffu, l2, 2);
-          float n2 = nwh + __shfl_xor_sync(0xffffffffu, nwh, 1);
-          n2 += __shfl_xor_sync(0xffffffffu, n2, 2);
-          if (g8 < G) {
-            // slot 0 holds the window's partial, the other lanes mark the remaining slots unused
-            float* wp = a.win_part + (ub + list_idx(jmap(o))) * win_part_floats(D, G) + g8;
+  // q fragments (A operand, cache dtype): head g8's elements 16m + 2t4, +1 and 16m + 8 + 2t4, +1
+  uint32_t qa[G8][2];
+  {
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+        reinterpret_cast<const T*>(a.q) + ((size_t)b * st.Hq + (size_t)kvh * G + (g8 < G ? g8 : 0)) * D);
 #pragma unroll
-            for (int slot = t4; slot < TPS; slot += 4) {
-              wp[slot * 3 * G] = slot == 0 ? mh : -1e30f;
-              wp[slot * 3 * G + G] = slot == 0 ? l2 : 0.f;
-              wp[slot * 3 * G + 2 * G] = slot == 0 ? n2 : 0.f;
-            }
-          }
-          lwh = 0.f;
-          nwh = 0.f;
-        }
-        advance(o, pg);
-        ++k;
+    for (int m = 0; m < G8; ++m) {
+      qa[m][0] = g8 < G ? qrow[m * 8 + t4] : 0u;
+      qa[m][1] = g8 < G ? qrow[m * 8 + 4 + t4] : 0u;
+    }
+  }
+
+  // ---- phase 1: full-precision windows, then the tail, from swizzled TMA pages ----
+  while (o < n_own && kind_of(jmap(o)) != 1) {
+    if (io < n_own) {
+      issue(io, ipg, issued % kNST);
+      advance(io, ipg);
+      ++issued;
+    }
+    const int s = k % kNST;
+    ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[s], (k / kNST) & 1, st.status, 1000 + u));
+    if (!ok) break;
+    uint8_t* stage = ring + s * STAGE;
+    const int j = jmap(o);
+    const bool tail = kind_of(j) == 2;
+    const int valid = tail ? min(QE_PAGE, a.tail_len - pg * QE_PAGE) : QE_PAGE;
+    if (valid < QE_PAGE) {
+      // rows past the tail's last token hold stale data: zero their V rows (weight 0 must not
+      // meet a NaN) and mask their scores below
+      for (int i = lane; i < (QE_PAGE - valid) * (D / 64) * 8; i += 32) {
+        const int row = valid + i / ((D / 64) * 8), rest = i % ((D / 64) * 8);
+        *reinterpret_cast<uint4*>(stage + ((D / 64) + rest / 8) * 2048 + row * 128 + (rest % 8) * 16) =
+            make_uint4(0u, 0u, 0u, 0u);
       }
-    lh += __shfl_xor_sync(0xffffffffu, lh, 1);
-    lh += __shfl_xor_sync(0xffffffffu, lh, 2);
-    float* fo = reinterpret_cast<float*>(ring + ((k + kNST - 1) % kNST) * STAGE);
+      __syncwarp();
+    }
+    float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int mt = 0; mt < D / 16; ++mt) {
-      if (2 * t4 < G) {
-        fo[(2 * t4) * D + mt * 16 + g8] = oacc[mt][0];
-        fo[(2 * t4) * D + mt * 16 + g8 + 8] = oacc[mt][2];
-      }
-      if (2 * t4 + 1 < G) {
-        fo[(2 * t4 + 1) * D + mt * 16 + g8] = oacc[mt][1];
-        fo[(2 * t4 + 1) * D + mt * 16 + g8 + 8] = oacc[mt][3];
+    for (int kc2 = 0; kc2 < D / 32; ++kc2) {
+      uint32_t kb[4];
+      ldsm_x4(kb, stage + swz<D>(0, lane & 7, kc2 * 32 + (lane >> 3) * 8));
+      MmaOp<T>::run(c0, qa[2 * kc2][0], 0u, qa[2 * kc2][1], 0u, kb[0], kb[1]);
+      MmaOp<T>::run(c0, qa[2 * kc2 + 1][0], 0u, qa[2 * kc2 + 1][1], 0u, kb[2], kb[3]);
+      ldsm_x4(kb, stage + swz<D>(0, 8 + (lane & 7), kc2 * 32 + (lane >> 3) * 8));
+      MmaOp<T>::run(c1, qa[2 * kc2][0], 0u, qa[2 * kc2][1], 0u, kb[0], kb[1]);
+      MmaOp<T>::run(c1, qa[2 * kc2 + 1][0], 0u, qa[2 * kc2 + 1][1], 0u, kb[2], kb[3]);
+    }
+    float sc[4] = {c0[0] * sl, c0[1] * sl, c1[0] * sl, c1[1] * sl};
+    if (tail) {
+      const int tk[4] = {2 * t4, 2 * t4 + 1, 8 + 2 * t4, 9 + 2 * t4};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (tk[i] >= valid) sc[i] = -INFINITY;
+        else if (g8 < G) a.tail_s[((size_t)u * w + pg * QE_PAGE + tk[i]) * G + g8] = sc[i];
       }
     }
-    if (t4 == 0 && g8 < G) {
-      fo[G * D + g8] = mh;
-      fo[G * D + G + g8] = lh;
+    float p[4];
+    softmax(sc, p, tail ? nullptr : reinterpret_cast<const float*>(nring + s * NSB));
+    uint32_t ph0, pl0, ph1, pl1;
+    MmaOp<T>::split(p[0], p[1], ph0, pl0);
+    MmaOp<T>::split(p[2], p[3], ph1, pl1);
+#pragma unroll
+    for (int m = 0; m < G8; ++m) {
+      uint32_t va[4];
+      ldsm_x4_t(va, stage + swz<D>(1, ((lane >> 4) << 3) + (lane & 7), m * 16 + ((lane >> 3) & 1) * 8));
+      MmaOp<T>::run(oacc[m], va[0], va[1], va[2], va[3], ph0, ph1);
+      MmaOp<T>::run(oacc[m], va[0], va[1], va[2], va[3], pl0, pl1);
     }
     __syncwarp();
-    return fo;
-  };
+    if (tail) {
+      // the tail's mass is formed at the end from its token scores; its sums belong to no slot
+      lwh = 0.f;
+      nwh = 0.f;
+    } else if (pg + 1 >= ppw) {
+      window_end(list_idx(j));
+    }
+    advance(o, pg);
+    ++k;
+  }
 
-  // ---- SIMT state for the INT2 and tail windows ----
-  auto load_q = [&]() {
-    const T* qb = reinterpret_cast<const T*>(a.q) + ((size_t)b * st.Hq + (size_t)kvh * G) * D;
-    const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
+  // ---- phase 2: INT2 ledger entries ----
+  // From here on the accumulators hold O^T * 2^-24 in rows g8 and O^T * 2^-20 in rows 8 + g8
+  // (the scale of the subnormal code operands); the zero-point part stays unscaled in zacc.
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      load_row<T, DPL>(qb + (size_t)h * D, sub, sw, q[h]);
-      float2 s2 = make_float2(0.f, 0.f);
+  for (int m = 0; m < G8; ++m) {
+    oacc[m][0] *= 0x1p-24f;
+    oacc[m][1] *= 0x1p-24f;
+    oacc[m][2] *= 0x1p-20f;
+    oacc[m][3] *= 0x1p-20f;
+  }
+  if (ok && o < n_own) {
+    // q as fp16 with the elements 8 + 2t4, 9 + 2t4 of each group quartered (their codes carry
+    // 4x), and head g8's sum of q over groups 2t4, 2t4 + 1 in the log2 domain, split hi + lo
+    uint32_t qh[G8][2];
+    float qs[G8];
 #pragma unroll
-      for (int e = 0; e < NP; ++e) {
-        q[h][e] = __fmul2_rn(q[h][e], sc2);
-        s2 = __fadd2_rn(s2, q[h][e]);
-      }
-      qsum[h] = s2.x + s2.y;
-      qsum2[h] = fmaf(4.f, s2.x, s2.y);
+    for (int m = 0; m < G8; ++m) {
+      const float x0 = Elem<T>::lo(qa[m][0]), x1 = Elem<T>::hi(qa[m][0]);
+      const float x2 = Elem<T>::lo(qa[m][1]), x3 = Elem<T>::hi(qa[m][1]);
+      qh[m][0] = pack_h2(x0, x1);
+      qh[m][1] = pack_h2(0.25f * x2, 0.25f * x3);
+      float t = (x0 + x1) + (x2 + x3);
+      t += __shfl_xor_sync(0xffffffffu, t, 1);
+      t += __shfl_xor_sync(0xffffffffu, t, 2);
+      qs[m] = t * sl;
     }
-  };
-  auto simt_empty = [&]() {
+    float qg0 = 0.f, qg1 = 0.f;
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      zacc[h] = make_float2(0.f, 0.f);
-      m[h] = -1e30f;
-      lsum[h] = 0.f;
-      lw[h] = 0.f;
-      nw[h] = 0.f;
-#pragma unroll
-      for (int e = 0; e < NP; ++e) acc[h][e] = make_float2(0.f, 0.f);
+    for (int m = 0; m < G8; ++m) {
+      if (m == 2 * t4) qg0 = qs[m];
+      if (m == 2 * t4 + 1) qg1 = qs[m];
     }
-  };
-  // merge a tensor-core partial (at a window boundary) into the SIMT state; lane group 0
-  // takes its values, every lane group rescales to the common maximum
-  auto merge = [&](const float* fo) {
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float mf = fo[G * D + h], lf = fo[G * D + G + h];
-      const float M = fmaxf(m[h], mf);
-      const float fs = ex2(m[h] - M), ff = grp == 0 ? ex2(mf - M) : 0.f;
-      const float2 fs2 = make_float2(fs, fs), ff2 = make_float2(ff, ff);
-      lsum[h] = fmaf(lsum[h], fs, lf * ff);
-      zacc[h] = __fmul2_rn(zacc[h], fs2);
-#pragma unroll
-      for (int e = 0; e < NP; ++e) {
-        // register pair e of chunk c = e / 4 sits in memory chunk c ^ sw
-        const int d = DPL * sub + 8 * ((e / 4) ^ sw) + 2 * (e % 4);
-        acc[h][e] = ffma2(make_float2(fo[h * D + d], fo[h * D + d + 1]), ff2, __fmul2_rn(acc[h][e], fs2));
-      }
-      m[h] = M;
-    }
-    __syncwarp();
-  };
+    const uint32_t qgh = pack_h2(qg0, qg1);
+    const uint32_t qgl = pack_h2(qg0 - h_lo(qgh), qg1 - h_hi(qgh));
+    // staged scale factors: K scores of tokens 0..7 carry 2^-24, of tokens 8..15 16 * 2^-24;
+    // V rows 8..15 of the block carry 4x in their codes, so their P * s is quartered
+    const int stk = lane & 15, kvsel = lane >> 4;
+    const float sfac = kvsel == 0 ? (stk < 8 ? 0x1p24f * sl : 0x1p20f * sl) : (stk < 8 ? 1.f : 0.25f);
+    float* sdst = sst + kvsel * 4 * SROW + ((stk & 7) >> 1) * SROW + ((stk & 1) + 2 * (stk >> 3));
+    const float* sk = sst + t4 * SROW;
+    const float* sv = sst + 4 * SROW + t4 * SROW;
 
-  // ---- INT2 ledger entries and the tail window on the CUDA cores ----
-  auto simt_phase = [&]() {
-    while (ok && o < n_own && kind_of(jmap(o)) != 0) {
+    while (o < n_own) {
       if (io < n_own) {
         issue(io, ipg, issued % kNST);
         advance(io, ipg);
@@ -676,168 +517,115 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
       ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[s], (k / kNST) & 1, st.status, 1000 + u));
       if (!ok) break;
       const uint8_t* stage = ring + s * STAGE;
-      const int j = jmap(o);
-      const int kind = kind_of(j);
-      const float* nrm = reinterpret_cast<const float*>(stage + PAGE_BYTES);
-      if (kind == 2) {
-        // ---- a page of the tail window: mask tokens past its length, keep raw scores ----
-        const T* Ks = reinterpret_cast<const T*>(stage);
-        const T* Vs = Ks + QE_PAGE * D;
-        const int valid = min(QE_PAGE, a.tail_len - pg * QE_PAGE);
-        for (int t0 = 0; t0 < valid; t0 += SBT) {
-          float sc[SB][G];
-  #pragma unroll
-          for (int i = 0; i < SB; ++i) {
-            float2 kx[NP];
-            load_row<T, DPL>(Ks + (size_t)(t0 + i * TPS + grp) * D, sub, sw, kx);
-            qk_row(kx, sc[i]);
-          }
-          butterfly(sc);
-  #pragma unroll
-          for (int i = 0; i < SB; ++i) {
-            const int t = t0 + i * TPS + grp;
-            if (t >= valid) {
-  #pragma unroll
-              for (int h = 0; h < G; ++h) sc[i][h] = -INFINITY;
-            } else if (sub == 0) {
-  #pragma unroll
-              for (int h = 0; h < G; ++h) a.tail_s[((size_t)u * w + pg * QE_PAGE + t) * G + h] = sc[i][h];
-            }
-          }
-          online(sc);
-  #pragma unroll
-          for (int i = 0; i < SB; ++i) {
-            const int t = t0 + i * TPS + grp;
-  #pragma unroll
-            for (int h = 0; h < G; ++h) lw[h] += sc[i][h];
-            if (t < valid) {
-              float2 vx[NP];
-              load_row<T, DPL>(Vs + (size_t)t * D, sub, sw, vx);
-              pv_row(vx, sc[i]);
-            }
-          }
-        }
-      } else {
-        // ---- INT2 ledger entry: codes K [w][D/4] | codes V | meta K [w][D/16] | meta V ----
-        const uint8_t* kc = stage;
-        const uint8_t* vc = stage + w * D / 4;
-        const uint32_t* km = reinterpret_cast<const uint32_t*>(stage + w * D / 2);
-        const uint32_t* vm = km + w * D / 16;
-        for (int t0 = 0; t0 < w; t0 += SBT) {
-          float sc[SB][G];
-  #pragma unroll
-          for (int i = 0; i < SB; ++i) {
-            const int t = t0 + i * TPS + grp;
-            float2 x[NP];
-            decode_codes<NP>(load_codes<DPL>(kc + t * (D / 4), sub, sw), x);
-            const uint32_t mt = km[t * (D / 16) + gi];
-            const float s4 = 4.f * meta_scale(mt), z = meta_zero(mt);
-            float d[G];
-            qk_row(x, d);
-            // q . x = qsum2 + (q . c) / 4, so q . k = s (q . c) + z qsum = 4s (q . x) + z qsum - 4s qsum2
-  #pragma unroll
-            for (int h = 0; h + 1 < G; h += 2) {
-              const float2 c0 = ffma2(make_float2(z, z), make_float2(qsum[h], qsum[h + 1]),
-                                      __fmul2_rn(make_float2(-s4, -s4), make_float2(qsum2[h], qsum2[h + 1])));
-              const float2 r = ffma2(make_float2(s4, s4), make_float2(d[h], d[h + 1]), c0);
-              sc[i][h] = r.x;
-              sc[i][h + 1] = r.y;
-            }
-            if constexpr (G % 2)
-              sc[i][G - 1] = fmaf(s4, d[G - 1], fmaf(z, qsum[G - 1], -s4 * qsum2[G - 1]));
-          }
-          butterfly(sc);
-          online(sc);
-  #pragma unroll
-          for (int i = 0; i < SB; ++i) {
-            const int t = t0 + i * TPS + grp;
-            window_sums(sc[i], nrm + t * G);
-            float2 x[NP];
-            decode_codes<NP>(load_codes<DPL>(vc + t * (D / 4), sub, sw), x);
-            const uint32_t mt = vm[t * (D / 16) + gi];
-            const float s4 = 4.f * meta_scale(mt), z = meta_zero(mt);
-            // v = 4s * x + (z - 16s) for even elements (x = 4 + c/4), 4s * x + (z - 4s) for odd
-            // ones (x = 1 + c/4): acc += (p * 4s) * x, zacc += p * (z - 16s, z - 4s)
-            const float2 zz = make_float2(fmaf(-4.f, s4, z), z - s4);
-            float ps[G];
-  #pragma unroll
-            for (int h = 0; h < G; ++h) {
-              ps[h] = sc[i][h] * s4;
-              zacc[h] = ffma2(make_float2(sc[i][h], sc[i][h]), zz, zacc[h]);
-            }
-            pv_row(x, ps);
-          }
-        }
-      }
-      __syncwarp();
-      if (pg + 1 >= n_tasks(j)) {
-        // end of a window: each lane group's leader records its (max, sum p, sum p n) per head
-        // in its own slot (no cross-group reduction here: the score update folds the slots)
-        if (kind != 2 && sub == 0) {
-          float* ws = a.win_part + (ub + list_idx(j)) * win_part_floats(D, G) + grp * 3 * G;
-          if constexpr (G == 4) {
-            reinterpret_cast<float4*>(ws)[0] = make_float4(m[0], m[1], m[2], m[3]);
-            reinterpret_cast<float4*>(ws + G)[0] = make_float4(lw[0], lw[1], lw[2], lw[3]);
-            reinterpret_cast<float4*>(ws + 2 * G)[0] = make_float4(nw[0], nw[1], nw[2], nw[3]);
-          } else {
+      const float* nrm = reinterpret_cast<const float*>(nring + s * NSB);
+      for (int bk = 0; bk < w / 16; ++bk) {
+        const uint8_t* blk = stage + bk * BL::BYTES;
+        {  // stage this block's scales: lanes 0-15 the K scales of token lane, 16-31 the V scales
+          const __half* srow = reinterpret_cast<const __half*>(blk + (kvsel ? BL::VS : BL::KS)) + stk * G8;
 #pragma unroll
-            for (int h = 0; h < G; ++h) {
-              ws[h] = m[h];
-              ws[G + h] = lw[h];
-              ws[2 * G + h] = nw[h];
-            }
+          for (int m = 0; m < G8; ++m) sdst[m * 4] = __half2float(srow[m]) * sfac;
+        }
+        __syncwarp();
+        // ---- K side: scores of tokens 2t4, 2t4+1 (tile A) and 8+2t4, 9+2t4 (tile B) ----
+        float sc[4];
+        {
+          const uint32_t zA = 2 * t4 < G8 ? *reinterpret_cast<const uint32_t*>(blk + BL::KZ + (g8 * G8 + 2 * t4) * 2) : 0u;
+          const uint32_t zB =
+              2 * t4 < G8 ? *reinterpret_cast<const uint32_t*>(blk + BL::KZ + ((8 + g8) * G8 + 2 * t4) * 2) : 0u;
+          float za[4] = {0.f, 0.f, 0.f, 0.f}, zb[4] = {0.f, 0.f, 0.f, 0.f};
+          mma_h8(za, qgh, 0u, zA);
+          mma_h8(za, qgl, 0u, zA);
+          mma_h8(zb, qgh, 0u, zB);
+          mma_h8(zb, qgl, 0u, zB);
+          sc[0] = za[0];
+          sc[1] = za[1];
+          sc[2] = zb[0];
+          sc[3] = zb[1];
+        }
+        uint32_t kw[WPL];
+        if constexpr (WPL == 4) {
+          const uint4 v4 = *reinterpret_cast<const uint4*>(blk + BL::KC + lane * 16);
+          kw[0] = v4.x; kw[1] = v4.y; kw[2] = v4.z; kw[3] = v4.w;
+        } else {
+          const uint2 v2 = *reinterpret_cast<const uint2*>(blk + BL::KC + lane * 8);
+          kw[0] = v2.x; kw[1] = v2.y;
+        }
+#pragma unroll
+        for (int jj = 0; jj < WPL; ++jj) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int m = 2 * jj + e;
+            const uint32_t x = e ? (kw[jj] >> 8) : kw[jj];
+            float cA[4] = {0.f, 0.f, 0.f, 0.f}, cB[4] = {0.f, 0.f, 0.f, 0.f};
+            mma_h16(cA, qh[m][0], 0u, qh[m][1], 0u, code_reg<0>(x), code_reg<1>(x));
+            mma_h16(cB, qh[m][0], 0u, qh[m][1], 0u, code_reg<2>(x), code_reg<3>(x));
+            const float4 s4 = *reinterpret_cast<const float4*>(sk + m * 4);
+            const float2 ra = ffma2(make_float2(s4.x, s4.y), make_float2(cA[0], cA[1]), make_float2(sc[0], sc[1]));
+            const float2 rb = ffma2(make_float2(s4.z, s4.w), make_float2(cB[0], cB[1]), make_float2(sc[2], sc[3]));
+            sc[0] = ra.x;
+            sc[1] = ra.y;
+            sc[2] = rb.x;
+            sc[3] = rb.y;
           }
         }
-  #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          lsum[h] += lw[h];
-          lw[h] = 0.f;
-          nw[h] = 0.f;
+        float p[4];
+        softmax(sc, p, nrm + bk * 16 * G);
+        // ---- V side ----
+        {
+          uint32_t ph0, pl0, ph1, pl1;
+          MmaOp<__half>::split(p[0], p[1], ph0, pl0);
+          MmaOp<__half>::split(p[2], p[3], ph1, pl1);
+          const uint32_t za0 = g8 < G8 ? *reinterpret_cast<const uint32_t*>(blk + BL::VZ + (g8 * 16 + 2 * t4) * 2) : 0u;
+          const uint32_t za2 =
+              g8 < G8 ? *reinterpret_cast<const uint32_t*>(blk + BL::VZ + (g8 * 16 + 8 + 2 * t4) * 2) : 0u;
+          mma_h16(zacc, za0, 0u, za2, 0u, ph0, ph1);
+          mma_h16(zacc, za0, 0u, za2, 0u, pl0, pl1);
         }
+        uint32_t vw[WPL];
+        if constexpr (WPL == 4) {
+          const uint4 v4 = *reinterpret_cast<const uint4*>(blk + BL::VC + lane * 16);
+          vw[0] = v4.x; vw[1] = v4.y; vw[2] = v4.z; vw[3] = v4.w;
+        } else {
+          const uint2 v2 = *reinterpret_cast<const uint2*>(blk + BL::VC + lane * 8);
+          vw[0] = v2.x; vw[1] = v2.y;
+        }
+#pragma unroll
+        for (int jj = 0; jj < WPL; ++jj) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int m = 2 * jj + e;
+            const uint32_t x = e ? (vw[jj] >> 8) : vw[jj];
+            const float4 s4 = *reinterpret_cast<const float4*>(sv + m * 4);
+            const uint32_t b0 = pack_h2(p[0] * s4.x, p[1] * s4.y);
+            const uint32_t b1 = pack_h2(p[2] * s4.z, p[3] * s4.w);
+            mma_h16(oacc[m], code_reg<0>(x), code_reg<2>(x), code_reg<1>(x), code_reg<3>(x), b0, b1);
+          }
+        }
+        __syncwarp();  // the next block restages the scales
       }
+      window_end(list_idx(jmap(o)));
       advance(o, pg);
       ++k;
-    }
-  };
-
-  // at most two segments (full then the rest, or the rest then full); each phase has one call
-  // site so that it is inlined and its state stays in registers
-  simt_empty();
-  for (int seg = 0; seg < 2 && ok && o < n_own; ++seg) {
-    if (kind_of(jmap(o)) == 0) {
-      merge(mma_phase());
-    } else {
-      load_q();
-      simt_phase();
     }
   }
   if (!ok) {  // drain copies still in flight if a wait gave up
     for (; k < issued; ++k) mbar_wait_bounded(&bars[k % kNST], (k / kNST) & 1, st.status, 2000 + u);
   }
-
-  // ---- merge lane groups, then warps, into the CTA's partial ----
+  // back to O^T: undo the code scales and add the zero-point part of each element's group
 #pragma unroll
-  for (int h = 0; h < G; ++h) {
-    float mx = m[h];
-#pragma unroll
-    for (int o = LPT; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    const float f = ex2(m[h] - mx);
-    lsum[h] *= f;
-    const float2 f2 = make_float2(f, f);
-#pragma unroll
-    for (int e = 0; e < NP; ++e) acc[h][e] = __fmul2_rn(__fadd2_rn(acc[h][e], zacc[h]), f2);
-#pragma unroll
-    for (int o = LPT; o < 32; o <<= 1) {
-      lsum[h] += __shfl_xor_sync(0xffffffffu, lsum[h], o);
-#pragma unroll
-      for (int e = 0; e < NP; ++e) {
-        acc[h][e].x += __shfl_xor_sync(0xffffffffu, acc[h][e].x, o);
-        acc[h][e].y += __shfl_xor_sync(0xffffffffu, acc[h][e].y, o);
-      }
-    }
-    m[h] = mx;
+  for (int m = 0; m < G8; ++m) {
+    const float z0 = __shfl_sync(0xffffffffu, zacc[0], 4 * m + t4);
+    const float z1 = __shfl_sync(0xffffffffu, zacc[1], 4 * m + t4);
+    oacc[m][0] = fmaf(oacc[m][0], 0x1p24f, z0);
+    oacc[m][1] = fmaf(oacc[m][1], 0x1p24f, z1);
+    oacc[m][2] = fmaf(oacc[m][2], 0x1p20f, z0);
+    oacc[m][3] = fmaf(oacc[m][3], 0x1p20f, z1);
   }
-  __syncthreads();
+  lh += __shfl_xor_sync(0xffffffffu, lh, 1);
+  lh += __shfl_xor_sync(0xffffffffu, lh, 2);
+
+  // ---- merge the warps into the CTA's partial ----
+  const bool cta_ok = __syncthreads_and(ok ? 1 : 0) != 0;  // also: every warp is done with its ring
   float* mw = reinterpret_cast<float*>(smem);  // [kNW][G]
   float* lwv = mw + kNW * G;                   // [kNW][G]
   float* aw = lwv + kNW * G;                   // [kNW][G][D]
@@ -850,22 +638,24 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
   float* gl = pf + QE_MAX_SPLITS_CLUSTER * QE_MAX_G;  // [G] unit sum of weights
   float* lse = gl + QE_MAX_G;                         // [G] unit log2-sum-exp
   float* red = lse + QE_MAX_G;                        // [kNW]
-  if (lane < LPT) {
+  float* okv = red + kNW;                             // [1] this CTA finished every wait
+  if (t4 == 0 && g8 < G) {
+    mw[warp * G + g8] = mh;
+    lwv[warp * G + g8] = lh;
+  }
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      if (lane == 0) {
-        mw[warp * G + h] = m[h];
-        lwv[warp * G + h] = lsum[h];
-      }
-#pragma unroll
-      for (int e = 0; e < NP; ++e) {
-        // register pair e of chunk c = e / 4 sits in memory chunk c ^ sw
-        const int d = DPL * sub + 8 * ((e / 4) ^ sw) + 2 * (e % 4);
-        aw[((size_t)warp * G + h) * D + d] = acc[h][e].x;
-        aw[((size_t)warp * G + h) * D + d + 1] = acc[h][e].y;
-      }
+  for (int m = 0; m < G8; ++m) {
+    float* a0 = aw + (size_t)warp * G * D;
+    if (2 * t4 < G) {
+      a0[(2 * t4) * D + m * 16 + g8] = oacc[m][0];
+      a0[(2 * t4) * D + m * 16 + 8 + g8] = oacc[m][2];
+    }
+    if (2 * t4 + 1 < G) {
+      a0[(2 * t4 + 1) * D + m * 16 + g8] = oacc[m][1];
+      a0[(2 * t4 + 1) * D + m * 16 + 8 + g8] = oacc[m][3];
     }
   }
+  if (threadIdx.x == 0) okv[0] = cta_ok ? 1.f : 0.f;
   __syncthreads();
   for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
     const int h = i / D;
@@ -894,6 +684,10 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
     pm[i] = ld_cluster(cm + i % G, (uint32_t)(i / G));
     pl[i] = ld_cluster(cl + i % G, (uint32_t)(i / G));
   }
+  // every CTA of the unit must have finished its waits: a CTA that gave up holds partials of
+  // a part of its windows, and window partials it never wrote may be stale
+  float all_ok = 1.f;
+  for (int r = 0; r < S; ++r) all_ok = fminf(all_ok, ld_cluster(okv, (uint32_t)r));
   __syncthreads();
   if (threadIdx.x < G) {
     const int h = threadIdx.x;
@@ -919,42 +713,41 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
       a.out[((size_t)b * st.Hq + (size_t)kvh * G + h) * D + i % D] = A / gl[h];
     }
   }
-  // exact attention mass and perturbation of this step for the windows this CTA streamed
-  for (int jj = threadIdx.x; jj < nF + nQ; jj += blockDim.x) {
-    const int li = list_idx(jj);
-    const int win = jj < nF ? st.full_list[ub + li] : st.int2_list[ub + li - nf];
-    if (win < 0 || win >= st.Wmax) continue;
-    float dm = 0.f, dp = 0.f;
-    const float* wp = a.win_part + (ub + li) * win_part_floats(D, G);
-#pragma unroll
-    for (int slot = 0; slot < TPS; ++slot) {
-      const float* ws = wp + slot * 3 * G;
+  if (all_ok > 0.f) {
+    // exact attention mass and perturbation of this step for the windows this CTA streamed
+    for (int jj = threadIdx.x; jj < nF + nQ; jj += blockDim.x) {
+      const int vj = jj < nF ? jj : jj + has_tail;
+      const int li = list_idx(vj);
+      const int win = jj < nF ? st.full_list[ub + li] : st.int2_list[ub + li - nf];
+      if (win < 0 || win >= st.Wmax) continue;
+      const float* wp = a.win_part + (ub + li) * win_part_floats(D, G);
+      float dm = 0.f, dp = 0.f;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float f = ex2(ws[h] - lse[h]);
-        dm = fmaf(ws[G + h], f, dm);
-        dp = fmaf(ws[2 * G + h], f, dp);
+        const float f = ex2(wp[h] - lse[h]);
+        dm = fmaf(wp[G + h], f, dm);
+        dp = fmaf(wp[2 * G + h], f, dp);
       }
+      st.mass[ub + win] += dm;
+      st.pert[ub + win] += dp;
     }
-    st.mass[ub + win] += dm;
-    st.pert[ub + win] += dp;
-  }
-  // tail tokens (last CTA of the cluster): cumulative per-token attention and window mass
-  if (has_tail) {
-    float tm = 0.f;
-    for (int i = threadIdx.x; i < a.tail_len * G; i += blockDim.x) {
-      const int h = i % G;
-      const float pv = ex2(a.tail_s[(size_t)u * w * G + i] - lse[h]);
-      st.tail_p[(size_t)u * w * G + i] += pv;
-      tm += pv;
-    }
-    tm = warp_sum(tm);
-    if (lane == 0) red[warp] = tm;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float s2 = 0.f;
-      for (int x = 0; x < kNW; ++x) s2 += red[x];
-      st.mass[ub + a.tail_win] += s2;
+    // tail tokens (last CTA of the cluster): cumulative per-token attention and window mass
+    if (has_tail) {
+      float tm = 0.f;
+      for (int i = threadIdx.x; i < a.tail_len * G; i += blockDim.x) {
+        const int h = i % G;
+        const float pv = ex2(a.tail_s[(size_t)u * w * G + i] - lse[h]);
+        st.tail_p[(size_t)u * w * G + i] += pv;
+        tm += pv;
+      }
+      tm = warp_sum(tm);
+      if (lane == 0) red[warp] = tm;
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        float s2 = 0.f;
+        for (int x = 0; x < kNW; ++x) s2 += red[x];
+        st.mass[ub + a.tail_win] += s2;
+      }
     }
   }
   cluster_sync();  // keep this CTA's partial alive until every CTA of the cluster has read it
@@ -963,43 +756,49 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
 template <typename T, int D, int G>
 int launch_decode_t(qe_ctx* c, const void* q, float* out, cudaStream_t s, const void* k_new,
                     const void* v_new) {
-  constexpr int STAGE = StageLayout<D, G>::BYTES;
-  const size_t smem = 1024 + (size_t)kNW * kNST * STAGE + kNW * kNST * 8;  // + alignment slack
+  constexpr int STAGE = StageLayout<D>::BYTES;
+  auto smem_for = [](int w) {
+    return (size_t)1024 + (size_t)kNW * kNST * STAGE + kNW * kNST * 8 + (size_t)kNW * aux_bytes<D>(w, G);
+  };
   static_assert((size_t)(kNW * G * (D + 2) + 2 * QE_MAX_G + G * D + 3 * QE_MAX_SPLITS_CLUSTER * QE_MAX_G +
-                         2 * QE_MAX_G + kNW) * 4 <= (size_t)kNW * kNST * STAGE,
+                         2 * QE_MAX_G + kNW + 1) * 4 <= (size_t)kNW * kNST * STAGE,
                 "merge area");
   auto kern = decode_kernel<T, D, G>;
   // One-time set-up per instantiation and device (kept out of the per-step path and of graph
-  // capture): clusters[S] = how many clusters of S CTAs can be resident at once.
+  // capture): clusters[wi][S] = how many clusters of S CTAs can be resident at once with the
+  // shared memory of window size 16 << wi.
   static QeOnce once;
-  static int clusters_of[QE_MAX_DEVICES][QE_MAX_SPLITS_CLUSTER + 1];
+  static int clusters_of[QE_MAX_DEVICES][3][QE_MAX_SPLITS_CLUSTER + 1];
   int dev = 0;
   const int se = qe_once_per_device(once, &dev, [&](int d) {
-    QE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    QE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_for(64)));
     QE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
-    for (int S = 1; S <= QE_MAX_SPLITS_CLUSTER; ++S) {
-      cudaLaunchConfig_t qc = {};
-      cudaLaunchAttribute qa[1];
-      qa[0].id = cudaLaunchAttributeClusterDimension;
-      qa[0].val.clusterDim.x = S;
-      qa[0].val.clusterDim.y = 1;
-      qa[0].val.clusterDim.z = 1;
-      qc.gridDim = dim3(S);
-      qc.blockDim = dim3(kNW * 32);
-      qc.dynamicSmemBytes = smem;
-      qc.attrs = qa;
-      qc.numAttrs = 1;
-      int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, kern, &qc) != cudaSuccess) {
-        (void)cudaGetLastError();
-        n = 0;
+    for (int wi = 0; wi < 3; ++wi)
+      for (int S = 1; S <= QE_MAX_SPLITS_CLUSTER; ++S) {
+        cudaLaunchConfig_t qc = {};
+        cudaLaunchAttribute qa[1];
+        qa[0].id = cudaLaunchAttributeClusterDimension;
+        qa[0].val.clusterDim.x = S;
+        qa[0].val.clusterDim.y = 1;
+        qa[0].val.clusterDim.z = 1;
+        qc.gridDim = dim3(S);
+        qc.blockDim = dim3(kNW * 32);
+        qc.dynamicSmemBytes = smem_for(16 << wi);
+        qc.attrs = qa;
+        qc.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &qc) != cudaSuccess) {
+          (void)cudaGetLastError();
+          n = 0;
+        }
+        clusters_of[d][wi][S] = n;
       }
-      clusters_of[d][S] = n;
-    }
     return QE_OK;
   });
   if (se) return se;
-  const int* clusters = clusters_of[dev];
+  const int wi = c->cfg.window == 16 ? 0 : (c->cfg.window == 32 ? 1 : 2);
+  const size_t smem = smem_for(c->cfg.window);
+  const int* clusters = clusters_of[dev][wi];
   DecodeArgs a{};
   a.st = make_state(c);
   // the page pool as a 2-D tensor [units * P * 32 rows][D] for the swizzled TMA page loads

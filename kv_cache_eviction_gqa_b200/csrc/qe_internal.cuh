@@ -14,16 +14,9 @@
 
 #define QE_PAGE 16
 
-// Lane mapping of the decode kernel's CUDA-core path: head-dim elements per lane, and lane
-// groups (tokens processed side by side) per warp. The per-window score partials keep one
-// slot per lane group.
-#ifndef QE_DECODE_DPL4
-#define QE_DECODE_DPL4 16
-#endif
-__host__ __device__ constexpr int decode_dpl(int G) { return G <= 4 ? QE_DECODE_DPL4 : 8; }
-__host__ __device__ constexpr int decode_groups(int D, int G) { return 32 / (D / decode_dpl(G)); }
-// floats of one window's score partials: [lane-group slot][max, sum p, sum p n][G]
-__host__ __device__ constexpr int win_part_floats(int D, int G) { return decode_groups(D, G) * 3 * G; }
+// floats of one window's score partials in the decode kernel's scratch: {max, sum p, sum p n}
+// per query head of the group, relative to that max
+__host__ __device__ constexpr int win_part_floats(int D, int G) { return (void)D, 3 * G; }
 #define QE_MAX_G 8
 #define QE_MAX_SPLITS 64
 
@@ -227,3 +220,5 @@ int launch_vwo_tc(const void* V, int n_groups, int rows, int D, int dtype, const
                   cudaStream_t st);
 int launch_int2_quantize(const void* x, int T, int D, int dtype, uint8_t* codes, uint32_t* meta,
                          cudaStream_t st);
+int launch_ledger_read(qe_ctx* c, int unit, int win, uint8_t* codes_k, uint32_t* meta_k, uint8_t* codes_v,
+                       uint32_t* meta_v, int32_t* found, cudaStream_t st);

@@ -14,6 +14,7 @@
 
 #include "append.cuh"
 #include "int2.cuh"
+#include "int2_block.cuh"
 #include "qe_internal.cuh"
 
 namespace {
@@ -478,13 +479,20 @@ __global__ void __launch_bounds__(256) apply_kernel(DevState st, const int32_t* 
                                                     const int32_t* xcount, int unit_only) {
   constexpr int DPL = D / 32;
   using R = Int2Row<DPL>;
+  using BL = Int2Block<D>;
   using Wd = typename RowWord<DPL>::type;
+  // per warp: the block as it sits in the ledger, then the row-major K and V codes
+  constexpr int NAT = QE_PAGE * D / 4;
+  __shared__ __align__(16) uint8_t sm_all[8][BL::BYTES + 2 * NAT];
   const int u = unit_only >= 0 ? unit_only : blockIdx.x;
   const int lane = threadIdx.x & 31;
+  uint8_t* img = sm_all[threadIdx.x >> 5];
+  uint8_t* natk = img + BL::BYTES;
+  uint8_t* natv = natk + NAT;
   const int warps = blockDim.x >> 5, gw = blockIdx.y * warps + (threadIdx.x >> 5);
   const int nx = xcount[u * 4 + 0], np = xcount[u * 4 + 1];
   const size_t ub = (size_t)u * st.Wmax;
-  const int w = st.window, ppw = st.ppw;
+  const int ppw = st.ppw;
   for (int it = gw; it < (nx + np) * ppw; it += gridDim.y * warps) {
     const int item = it / ppw, pg = it % ppw;
     const bool quant = item < nx;
@@ -499,14 +507,12 @@ __global__ void __launch_bounds__(256) apply_kernel(DevState st, const int32_t* 
       if (lane == 0) qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
       continue;
     }
-    uint8_t* sl = st.slots + ((size_t)u * st.S + slot) * st.slot_bytes;
-    uint8_t* kc = sl;
-    uint8_t* vc = sl + (size_t)w * D / 4;
-    uint32_t* km = reinterpret_cast<uint32_t*>(sl + (size_t)w * D / 2);
-    uint32_t* vm = km + (size_t)w * D / 16;
+    // block pg of the window's ledger entry holds the page's 16 tokens
+    uint4* gblk = reinterpret_cast<uint4*>(st.slots + ((size_t)u * st.S + slot) * st.slot_bytes +
+                                           (size_t)pg * BL::BYTES);
     Wd* krows = reinterpret_cast<Wd*>(st.pages + ((size_t)u * st.P + page) * st.page_bytes);
     Wd* vrows = krows + QE_PAGE * 32;  // 32 words per row
-    const int t0 = pg * QE_PAGE;       // first token of the page in its window
+    __syncwarp();  // the previous item is done with this warp's shared memory
     if (quant) {
       Wd kw[QE_PAGE], vw[QE_PAGE];
 #pragma unroll
@@ -516,39 +522,67 @@ __global__ void __launch_bounds__(256) apply_kernel(DevState st, const int32_t* 
       }
 #pragma unroll
       for (int r = 0; r < QE_PAGE; ++r) {
-        const int t = t0 + r;
         float xk[DPL], xv[DPL];
         word_to_f<T>(kw[r], xk);
         word_to_f<T>(vw[r], xv);
         uint32_t mk, mv;
         const uint32_t bk = R::quantize(xk, &mk);
         const uint32_t bv = R::quantize(xv, &mv);
-        R::store_codes(kc + (size_t)t * D / 4, bk, lane);
-        R::store_codes(vc + (size_t)t * D / 4, bv, lane);
+        R::store_codes(natk + r * (D / 4), bk, lane);
+        R::store_codes(natv + r * (D / 4), bv, lane);
         if (lane % R::LPG == 0) {
-          km[(size_t)t * D / 16 + R::group_of(lane)] = mk;
-          vm[(size_t)t * D / 16 + R::group_of(lane)] = mv;
+          const int g = R::group_of(lane);
+          uint16_t* ks = reinterpret_cast<uint16_t*>(img + BL::KS);
+          uint16_t* kz = reinterpret_cast<uint16_t*>(img + BL::KZ);
+          uint16_t* vs = reinterpret_cast<uint16_t*>(img + BL::VS);
+          uint16_t* vz = reinterpret_cast<uint16_t*>(img + BL::VZ);
+          ks[r * BL::G8 + g] = static_cast<uint16_t>(mk & 0xffffu);
+          kz[r * BL::G8 + g] = static_cast<uint16_t>(mk >> 16);
+          vs[r * BL::G8 + g] = static_cast<uint16_t>(mv & 0xffffu);
+          vz[g * QE_PAGE + r] = static_cast<uint16_t>(mv >> 16);
         }
       }
-    } else {
-      uint32_t bk[QE_PAGE], bv[QE_PAGE], mk[QE_PAGE], mv[QE_PAGE];
+      __syncwarp();
+      uint32_t pk[BL::WPL], pv[BL::WPL];
+      BL::template pack<false>(natk, lane, pk);
+      BL::template pack<true>(natv, lane, pv);
+      uint32_t* kc = reinterpret_cast<uint32_t*>(img + BL::KC) + lane * BL::WPL;
+      uint32_t* vc = reinterpret_cast<uint32_t*>(img + BL::VC) + lane * BL::WPL;
 #pragma unroll
-      for (int r = 0; r < QE_PAGE; ++r) {
-        const int t = t0 + r;
-        bk[r] = R::load_codes(kc + (size_t)t * D / 4, lane);
-        bv[r] = R::load_codes(vc + (size_t)t * D / 4, lane);
-        mk[r] = km[(size_t)t * D / 16 + R::group_of(lane)];
-        mv[r] = vm[(size_t)t * D / 16 + R::group_of(lane)];
+      for (int j = 0; j < BL::WPL; ++j) {
+        kc[j] = pk[j];
+        vc[j] = pv[j];
       }
+      __syncwarp();
+      const uint4* src = reinterpret_cast<const uint4*>(img);
+      for (int i = lane; i < BL::BYTES / 16; i += 32) gblk[i] = src[i];
+    } else {
+      uint4* dst = reinterpret_cast<uint4*>(img);
+      for (int i = lane; i < BL::BYTES / 16; i += 32) dst[i] = gblk[i];
+      __syncwarp();
+      const uint32_t* kc = reinterpret_cast<const uint32_t*>(img + BL::KC);
+      const uint32_t* vc = reinterpret_cast<const uint32_t*>(img + BL::VC);
+      for (int n = lane; n < NAT; n += 32) {
+        natk[n] = BL::template unpack_byte<false>(kc, n);
+        natv[n] = BL::template unpack_byte<true>(vc, n);
+      }
+      __syncwarp();
+      const uint16_t* ks = reinterpret_cast<const uint16_t*>(img + BL::KS);
+      const uint16_t* kz = reinterpret_cast<const uint16_t*>(img + BL::KZ);
+      const uint16_t* vs = reinterpret_cast<const uint16_t*>(img + BL::VS);
+      const uint16_t* vz = reinterpret_cast<const uint16_t*>(img + BL::VZ);
+      const int g = R::group_of(lane);
 #pragma unroll
       for (int r = 0; r < QE_PAGE; ++r) {
-        const float sk = meta_scale(mk[r]), zk = meta_zero(mk[r]);
-        const float sv = meta_scale(mv[r]), zv = meta_zero(mv[r]);
+        const uint32_t bk = R::load_codes(natk + r * (D / 4), lane);
+        const uint32_t bv = R::load_codes(natv + r * (D / 4), lane);
+        const float sk = meta_scale(ks[r * BL::G8 + g]), zk = meta_scale(kz[r * BL::G8 + g]);
+        const float sv = meta_scale(vs[r * BL::G8 + g]), zv = meta_scale(vz[g * QE_PAGE + r]);
         float xk[DPL], xv[DPL];
 #pragma unroll
         for (int e = 0; e < DPL; ++e) {
-          xk[e] = fmaf((float)((bk[r] >> (2 * e)) & 3u), sk, zk);
-          xv[e] = fmaf((float)((bv[r] >> (2 * e)) & 3u), sv, zv);
+          xk[e] = fmaf((float)((bk >> (2 * e)) & 3u), sk, zk);
+          xv[e] = fmaf((float)((bv >> (2 * e)) & 3u), sv, zv);
         }
         Wd ok, ov;
         f_to_word<T>(xk, ok);
@@ -556,6 +590,48 @@ __global__ void __launch_bounds__(256) apply_kernel(DevState st, const int32_t* 
         krows[r * 32 + lane] = ok;
         vrows[r * 32 + lane] = ov;
       }
+    }
+  }
+}
+
+// A window's ledger entry in the row-major form of qe_int2_quantize: one warp per 16-token
+// block. found[0] = 1 when the window has an entry, else 0 (and nothing else is written).
+template <int D>
+__global__ void __launch_bounds__(128) ledger_read_kernel(DevState st, int u, int win, uint8_t* codes_k,
+                                                          uint32_t* meta_k, uint8_t* codes_v, uint32_t* meta_v,
+                                                          int32_t* found) {
+  using BL = Int2Block<D>;
+  constexpr int NAT = QE_PAGE * D / 4;
+  __shared__ __align__(16) uint8_t sm_all[4][BL::BYTES];
+  const int lane = threadIdx.x & 31, wq = threadIdx.x >> 5;
+  const int slot = st.win_slot[(size_t)u * st.Wmax + win];
+  if (slot < 0 || slot >= st.S) {
+    if (threadIdx.x == 0) found[0] = 0;
+    return;
+  }
+  if (threadIdx.x == 0) found[0] = 1;
+  uint8_t* img = sm_all[wq];
+  for (int bk = wq; bk < st.window / QE_PAGE; bk += 4) {
+    const uint4* g = reinterpret_cast<const uint4*>(st.slots + ((size_t)u * st.S + slot) * st.slot_bytes +
+                                                    (size_t)bk * BL::BYTES);
+    __syncwarp();
+    for (int i = lane; i < BL::BYTES / 16; i += 32) reinterpret_cast<uint4*>(img)[i] = g[i];
+    __syncwarp();
+    const uint32_t* kc = reinterpret_cast<const uint32_t*>(img + BL::KC);
+    const uint32_t* vc = reinterpret_cast<const uint32_t*>(img + BL::VC);
+    for (int n = lane; n < NAT; n += 32) {
+      codes_k[(size_t)bk * NAT + n] = BL::template unpack_byte<false>(kc, n);
+      codes_v[(size_t)bk * NAT + n] = BL::template unpack_byte<true>(vc, n);
+    }
+    const uint16_t* ks = reinterpret_cast<const uint16_t*>(img + BL::KS);
+    const uint16_t* kz = reinterpret_cast<const uint16_t*>(img + BL::KZ);
+    const uint16_t* vs = reinterpret_cast<const uint16_t*>(img + BL::VS);
+    const uint16_t* vz = reinterpret_cast<const uint16_t*>(img + BL::VZ);
+    for (int i = lane; i < QE_PAGE * BL::G8; i += 32) {
+      const int t = i / BL::G8, gg = i % BL::G8;
+      const size_t o = ((size_t)bk * QE_PAGE + t) * BL::G8 + gg;
+      meta_k[o] = (uint32_t)ks[t * BL::G8 + gg] | ((uint32_t)kz[t * BL::G8 + gg] << 16);
+      meta_v[o] = (uint32_t)vs[t * BL::G8 + gg] | ((uint32_t)vz[gg * QE_PAGE + t] << 16);
     }
   }
 }
@@ -726,6 +802,17 @@ int launch_set_tier(qe_ctx* c, int unit, const int32_t* ids, int n, int tier, cu
   route_kernel<<<1, kRouteThreads, smem, s>>>(a);
   QE_CUDA_TRY(cudaGetLastError());
   return apply_dispatch(c, st, unit, s);
+}
+
+int launch_ledger_read(qe_ctx* c, int unit, int win, uint8_t* codes_k, uint32_t* meta_k, uint8_t* codes_v,
+                       uint32_t* meta_v, int32_t* found, cudaStream_t s) {
+  const DevState st = make_state(c);
+  if (c->cfg.D == 128)
+    ledger_read_kernel<128><<<1, 128, 0, s>>>(st, unit, win, codes_k, meta_k, codes_v, meta_v, found);
+  else
+    ledger_read_kernel<64><<<1, 128, 0, s>>>(st, unit, win, codes_k, meta_k, codes_v, meta_v, found);
+  QE_CUDA_TRY(cudaGetLastError());
+  return QE_OK;
 }
 
 int launch_int2_quantize(const void* x, int T, int D, int dtype, uint8_t* codes, uint32_t* meta,
