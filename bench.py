@@ -41,9 +41,27 @@ METRIC = "decode attn+routing steps/sec; achieved HBM GB/s vs peak at 32K ctx, b
 CFG = W.C2
 FALLBACK_HBM_GBS = 6650.0
 # DRAM read + write of one steady decode launch (decode step 2 of the sequence) from an ncu
-# capture of the current decode kernel (profiles/decode_kernel_c2_llama8b_32k_b8.md); set to
-# None whenever the kernel changes until it is captured again.
-DECODE_TRAFFIC_BYTES = 108.958464e6 + 4.140032e6
+# capture, and the digest of the decode kernel's sources it was taken with: the bench reports
+# the traffic only while the sources still hash to that digest.
+DECODE_TRAFFIC_BYTES = None
+DECODE_TRAFFIC_SOURCES_SHA = None
+DECODE_SOURCES = ("decode.cu", "int2_block.cuh", "append.cuh", "qe_internal.cuh", "warp_mma.cuh", "tc_common.cuh")
+
+
+def decode_sources_sha() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for name in DECODE_SOURCES:
+        with open(os.path.join(ROOT, "kv_cache_eviction_gqa_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def decode_traffic():
+    """ncu DRAM traffic of a steady decode launch, or None when the kernel changed since."""
+    if DECODE_TRAFFIC_BYTES is None or decode_sources_sha() != DECODE_TRAFFIC_SOURCES_SHA:
+        return None
+    return DECODE_TRAFFIC_BYTES
 
 
 def max_over_ranks(value: float, device) -> float:
@@ -208,6 +226,10 @@ def cpu_baseline(cfg, target_s=10.0):
 
 
 def run_reference(args, rank):
+    """The oracle as it stands, on the host cores. A timed step is a bounded sample of the
+    batch's decode step: the decode step of one (batch, kv-head) unit (units are independent).
+    ms_per_step is that measured sample time; value is the whole-batch rate it implies
+    (units_per_step samples make one batch step)."""
     if rank != 0:
         return
     cfg = CFG
@@ -228,16 +250,19 @@ def run_reference(args, rank):
         t0 = time.perf_counter()
         oracle_step(cfg, u, s, b, h, q, k, v)
         t += time.perf_counter() - t0
-    per_step_full = t / args.steps * cfg.units  # one decode step of the whole batch
-    value = 1.0 / per_step_full
+    sample_s = t / args.steps               # measured: one unit's decode step
+    value = 1.0 / (sample_s * cfg.units)    # whole-batch decode steps per second
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": per_step_full * 1e3, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": sample_s * 1e3, "units_per_step": cfg.units, "units_per_sample": 1,
+            "step_note": f"a timed step is one sampled unit's decode step (measured); a batch step is "
+                         f"{cfg.units} such units, so value = 1 / ({cfg.units} x ms_per_step)",
+            "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": workload_config(cfg),
             "cpu_baseline": {"value": value, "unit": "steps/s", "kind": "oracle",
                              "cores": len(os.sched_getaffinity(0)), "blas_threads": blas_threads(),
-                             "sample": f"each step: 1 of {cfg.units} units (b=0, kv-head 0) of the "
-                                       f"decode step, scaled to the whole batch"},
+                             "sample": f"each timed step: the decode step of unit (b=0, kv-head 0), 1 of "
+                                       f"{cfg.units}; {args.steps} steps in {t:.2f} s"},
             "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -411,7 +436,10 @@ def run_ours(args, rank, world, local_rank):
     st_bytes = sum(decode_bytes(cfg, *meta[i % S][:3]) for i in steady)
     st_dec_ms = sum(dec_ms[i] for i in steady)
 
-    # end to end through the public API with host buffers (H2D inputs, D2H output)
+    # end to end through the public API with host buffers (H2D inputs, D2H output): each step
+    # as a serving loop runs it - the step's inputs copied in from pinned host memory, the C-ABI
+    # decode-step call (qe_decode_step through the binding), the output read back, the host
+    # waiting for it; host wall time per step
     q_h = torch.empty((S, cfg.B, cfg.Hq, cfg.D), dtype=tdt, pin_memory=True)
     k_h = torch.empty((S, cfg.B, cfg.Hkv, cfg.D), dtype=tdt, pin_memory=True)
     v_h = torch.empty_like(k_h, pin_memory=True)
@@ -423,10 +451,29 @@ def run_ours(args, rank, world, local_rank):
     h2d = q_d.numel() * 2 + k_d.numel() * 2 + v_d.numel() * 2
     d2h = out.numel() * 4
     e2e_steps = min(K_steps, args.e2e_steps)
+    wall_s = 0.0
+    host_ms = []
+    for i in range(e2e_steps):
+        s = i % S
+        if s == 0:  # a fresh sequence: the context's host and device state back to the prefill
+            ctx.load_prefill(K, V, norms)
+        flush.zero_()
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        q_d.copy_(q_h[s], non_blocking=True)
+        k_d.copy_(k_h[s], non_blocking=True)
+        v_d.copy_(v_h[s], non_blocking=True)
+        ctx.decode_step(q_d, k_d, v_d, out)
+        out_h.copy_(out, non_blocking=True)
+        stream.synchronize()
+        dt = time.perf_counter() - t0
+        wall_s += dt
+        host_ms.append(dt * 1e3)
+    wall_ms = max_over_ranks(wall_s * 1e3, dev)
+    e2e_call_value = whole_job_rate(e2e_steps, world, wall_ms)
+    # the same step, captured once per step index as a CUDA graph and replayed from an idle host
+    # (what a serving loop that replays graphs gets); reported beside the per-call number
     e2e_ms = 0.0
-    # each step as a serving loop runs it: the step's inputs copied in from pinned host memory,
-    # the public decode-step call, the output read back - captured once per step index as a
-    # CUDA graph and replayed from an idle host that waits for the step's output
     ctx.load_prefill(K, V, norms)
     torch.cuda.synchronize()
     g_e2e = []
@@ -481,16 +528,21 @@ def run_ours(args, rank, world, local_rank):
             "roofline": {"kernel": "decode_kernel (split-K GQA decode + window scoring)",
                          "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
-                         "traffic": DECODE_TRAFFIC_BYTES, "launches_counted": n_l,
+                         "traffic": decode_traffic(), "launches_counted": n_l,
+                         "traffic_sources_sha": decode_sources_sha(),
                          "traffic_launch": "decode step 2 (steady), ncu dram__bytes_read.sum + write.sum",
                          "algorithmic_bytes_traffic_launch": decode_bytes(cfg, *meta[2 % S][:3]),
                          "bytes_per_launch_avg": b_sum / max(n_l, 1)},
             "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": h2d,
+            "e2e": {"value": e2e_call_value, "unit": "steps/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-                    "path": "per step: H2D of q, k, v from pinned host memory, qe_decode_step through the "
-                            "Python binding, D2H of the output, captured once per step index as a CUDA graph "
-                            "and replayed from an idle host that waits for each step's output"},
+                    "median_step_ms": statistics.median(host_ms),
+                    "path": "per step, host wall time: H2D of q, k, v from pinned host memory, "
+                            "qe_decode_step called through the C ABI (ctypes binding), D2H of the output, "
+                            "host waits for it (no graph)",
+                    "graph_replay": {"value": e2e_value, "unit": "steps/s",
+                                     "path": "the same step captured once per step index as a CUDA graph "
+                                             "and replayed from an idle host"}},
             "clocks": clocks,
             "gpu_launches": launches,
         }

@@ -163,6 +163,7 @@ QE_API int qe_load_prefill(qe_ctx* c, const void* K, const void* V, int ctx_len,
   c->loaded = 1;
   c->n_full_max = ctx_len / c->cfg.window;
   c->n_int2_max = 0;
+  c->counts_exact = 1;
   c->last_stream = st;
   return QE_OK;
 }
@@ -248,6 +249,7 @@ QE_API int qe_quantize_once(qe_ctx* c, int unit, const int32_t* ids, int n, qe_s
   int e = launch_set_tier(c, unit, ids, n, QE_TIER_INT2, (cudaStream_t)s);
   if (e) return e;
   c->n_int2_max += n;
+  c->counts_exact = 0;
   c->last_stream = (cudaStream_t)s;
   return QE_OK;
 }
@@ -262,6 +264,7 @@ QE_API int qe_promote(qe_ctx* c, int unit, const int32_t* ids, int n, qe_stream_
   int e = launch_set_tier(c, unit, ids, n, QE_TIER_FULL, (cudaStream_t)s);
   if (e) return e;
   c->n_full_max += n;
+  c->counts_exact = 0;
   c->last_stream = (cudaStream_t)s;
   return QE_OK;
 }

@@ -10,10 +10,11 @@
 // The unit's S CTAs form one thread-block cluster; CTA s takes the s-th S-th of the full
 // windows and of the INT2 windows (the tail counts as one more INT2 window of the last CTA),
 // so every SM streams the same mix of bandwidth-heavy full pages and compact INT2 entries.
-// Inside a CTA each warp takes whole windows round-robin and streams them through its own
-// ring of shared-memory stages (completion on an mbarrier per stage): a full or tail page
-// arrives as 128-byte-swizzled TMA boxes from a tensor map over the page pool, an INT2 ledger
-// entry as one 1-D bulk copy, each with its tokens' projected-value norms.
+// Inside a CTA each warp takes whole windows round-robin and streams them as tasks of at most
+// 16*D*2 bytes through its own ring of shared-memory stages (completion on an mbarrier per
+// stage): the K rows of a full or tail page, its V rows (128-byte-swizzled TMA boxes from a
+// tensor map over the page pool), or a chunk of up to 32 tokens of an INT2 ledger entry (one
+// 1-D bulk copy), each with its tokens' projected-value norms.
 //
 // Every tier runs on the warp-level tensor cores (mma.sync, f32 accumulate) in one register
 // layout: the G query heads of the group are the rows of S = Q K^T (padded to 16), 16 tokens
@@ -22,8 +23,9 @@
 // a tcgen05 tile (M >= 64) would be mostly padding and its TMEM round trip buys nothing on a
 // path that HBM bounds, so the decode stays on mma.sync.
 //
-// Full-precision pages: S from ldmatrix K tiles, P split into two 16-bit parts of the cache
-// dtype (hi + residual) so O keeps float32 accuracy, V^T by ldmatrix.trans.
+// Full-precision pages: S from ldmatrix K tiles (four independent accumulator chains), P split
+// into two 16-bit parts of the cache dtype (hi + residual) so O keeps float32 accuracy, V^T by
+// ldmatrix.trans.
 //
 // INT2 blocks (16 tokens, layout in int2_block.cuh): a K or V value is c*s + z with a 2-bit code
 // c and an fp16 scale s and zero z per 16-element group. The codes enter the MMA exactly as
@@ -32,8 +34,9 @@
 //   S += Z (sum of q over each group)  (one m16n8k8 MMA per 8 tokens, q sums split hi + lo),
 //   O_g^T += C_g^T (P * s_g)  (one MMA per group; P * s rounded once to fp16),
 //   O^T += Z^T P  (one MMA per 16 tokens, P split hi + lo).
-// The powers 4^i and 2^-24 are folded into q, the staged scales and the accumulator. The
-// block's scales are converted to float32 once per warp into a small staging area.
+// The token scales reach the lanes that need them as float32 through one more MMA per group
+// (the group's scales times a 0/1 selection matrix), so no conversion or staging is needed.
+// The powers 4^i and 2^-24 are folded into q, the selection matrix and the accumulator.
 //
 // Scoring without a second pass: at the end of each window the warp records its
 // (max, sum_i 2^(s_i-max), sum_i 2^(s_i-max) n_i) per head. After the pass the cluster merges
@@ -52,18 +55,26 @@
 namespace {
 
 #ifndef QE_DECODE_NW
-#define QE_DECODE_NW 2
-#endif
-#ifndef QE_DECODE_NST
-#define QE_DECODE_NST 3
+#define QE_DECODE_NW 3
 #endif
 #ifndef QE_DECODE_MINB
 #define QE_DECODE_MINB 4
 #endif
 constexpr int kNW = QE_DECODE_NW;    // warps per CTA
-#define QE_MAX_SPLITS_CLUSTER 16          // CTAs per unit (one cluster, non-portable size)
-constexpr int kNST = QE_DECODE_NST;  // stages per warp
-constexpr float kRescale = 8.f;  // rescale the accumulators when the max grows by > 2^8
+#define QE_MAX_SPLITS_CLUSTER 16     // CTAs per unit (one cluster, non-portable size)
+constexpr float kRescale = 8.f;      // rescale the accumulators when the max grows by > 2^8
+
+// stages per warp (fewer for wide groups, whose norm slots are larger)
+__host__ __device__ constexpr int nst_of(int G) { return G <= 4 ? 4 : 3; }
+// bytes of one stage: the K (or V) rows of a page, or an INT2 chunk of up to 32 tokens
+template <int D>
+__host__ __device__ constexpr int stage_bytes() { return (QE_PAGE * D * 2 + 1023) / 1024 * 1024; }
+// bytes of one norm slot: the norms of up to 32 tokens
+__host__ __device__ constexpr int norm_slot_bytes(int G) { return 32 * G * 4; }
+template <int D, int G>
+__host__ __device__ constexpr size_t decode_smem_bytes() {
+  return 1024 + (size_t)kNW * nst_of(G) * (stage_bytes<D>() + norm_slot_bytes(G) + 8);
+}
 
 struct DecodeArgs {
   DevState st;
@@ -72,6 +83,7 @@ struct DecodeArgs {
   float* win_part;   // [U][Wmax][3 G]: {max, sum p, sum p n} per head
   float* tail_s;     // [U][window][G]
   int splits;        // CTAs per unit = cluster size
+  int nf, nq;        // full / INT2 windows of every unit, or -1: read them from the device state
   int tail_win, tail_len;
   float scale_log2;  // log2(e) / sqrt(D)
   // optional fused append of the step's token at position append_pos (k_new != nullptr): the
@@ -91,7 +103,8 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // thread-block cluster helpers: barrier over the cluster's CTAs, and a load from the shared
-// memory of CTA `rank` of the cluster at the address of a local shared variable
+// memory of CTA `rank` of the cluster at the address of a local shared variable (issued after
+// a cluster barrier; the barrier orders it)
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
@@ -99,7 +112,7 @@ __device__ __forceinline__ float ld_cluster(const float* local, uint32_t rank) {
   uint32_t a;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(local)), "r"(rank));
   float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a));
   return v;
 }
 
@@ -130,11 +143,18 @@ __device__ __forceinline__ void mma_h16(float (&c)[4], uint32_t a0, uint32_t a1,
   MmaOp<__half>::run(c, a0, a1, a2, a3, b0, b1);
 }
 __device__ __forceinline__ void mma_h8(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5}, {%6}, "
       "{%0, %1, %2, %3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(b0));
+}
+
+// fp16 pair product, round to nearest
+__device__ __forceinline__ uint32_t __hmul2_u32(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
 }
 
 // Register i (0..3) of a packed code word: the codes at bits [2i, 2i+1] of each 16-bit half as
@@ -144,41 +164,19 @@ __device__ __forceinline__ uint32_t code_reg(uint32_t x) {
   return x & (0x00030003u << (2 * I));
 }
 
-// Shared memory of a warp: a ring of kNST page stages (1024-byte aligned) and, elsewhere, a ring
-// of kNST norm stages and the INT2 scale staging. A full-precision or tail page arrives as TMA
-// boxes of 16 rows x 64 elements with the 128-byte swizzle (box (part, x) at (part * D/64 + x) *
-// 2048, part 0 = K rows, 1 = V rows), so the 8 rows of every ldmatrix tile sit in distinct
-// banks; an INT2 ledger entry is a 1-D bulk copy (w/16 blocks of 16*D bytes, at most a page).
-// A norm stage holds the task's tokens' norms (window * G floats, runtime size).
-template <int D>
-struct StageLayout {
-  static constexpr int PAGE_BYTES = 2 * QE_PAGE * D * 2;            // K rows then V rows
-  static constexpr int BYTES = (PAGE_BYTES + 1023) / 1024 * 1024;
-};
-// Per-warp staging of one INT2 block's scales in float32: [K, V][t (0..3)][group][4 tokens
-// 2t, 2t+1, 8+2t, 9+2t], rows padded by 4 floats so the four t rows sit in distinct banks.
-template <int D>
-struct ScaleStage {
-  static constexpr int ROW = (D / 16) * 4 + 4;  // floats per t row
-  static constexpr int FLOATS = 2 * 4 * ROW;
-  static constexpr int BYTES = FLOATS * 4;
-};
-// bytes of one norm stage for a window of w tokens (16-byte multiple)
-__host__ __device__ constexpr int norm_stage_bytes(int w, int G) { return (w * G * 4 + 15) / 16 * 16; }
-// per-warp auxiliary area (norm ring, then scale staging) and the whole dynamic shared memory
-template <int D>
-__host__ __device__ constexpr int aux_bytes(int w, int G) { return 3 * norm_stage_bytes(w, G) + ScaleStage<D>::BYTES; }
-
-template <typename T, int D, int G>
+template <typename T, int D, int G, int W>
 __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
     decode_kernel(const __grid_constant__ CUtensorMap tmP, DecodeArgs a) {
   using BL = Int2Block<D>;
   constexpr int G8 = BL::G8, WPL = BL::WPL;
-  using SL = StageLayout<D>;
-  constexpr int PAGE_BYTES = SL::PAGE_BYTES;
-  constexpr int STAGE = SL::BYTES;
-  constexpr int SROW = ScaleStage<D>::ROW;
-  static_assert(kNST == 3, "aux_bytes assumes three stages");
+  constexpr int NST = nst_of(G);
+  constexpr int PPW = W / QE_PAGE;               // pages per window
+  constexpr int BPC = W >= 32 ? 2 : 1;           // INT2 blocks per chunk task
+  constexpr int CPW = W / (QE_PAGE * BPC);       // INT2 chunk tasks per window
+  constexpr int HALF = QE_PAGE * D * 2;          // bytes of a page's K (or V) rows
+  constexpr int STAGE = stage_bytes<D>();
+  constexpr int NSB = norm_slot_bytes(G);
+  constexpr int NB = D / 64;                     // TMA boxes per K or V half
   extern __shared__ __align__(128) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const DevState& st = a.st;
@@ -186,12 +184,12 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
   const int b = u / st.Hkv, kvh = u % st.Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g8 = lane >> 2, t4 = lane & 3;
-  const int w = st.window, ppw = st.ppw;
   const size_t ub = (size_t)u * st.Wmax;
   const float sl = a.scale_log2;
 
   // this split's share of each tier
-  const int nf = st.stacks[u * 4 + 2], nq = st.stacks[u * 4 + 3];
+  const int nf = a.nf >= 0 ? a.nf : st.stacks[u * 4 + 2];
+  const int nq = a.nq >= 0 ? a.nq : st.stacks[u * 4 + 3];
   const int f0 = (int)((long long)nf * split / a.splits), f1 = (int)((long long)nf * (split + 1) / a.splits);
   // the last split also streams the tail window (and appends the new token): it counts as one
   // INT2 window of that split's share
@@ -200,45 +198,34 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
   const int q1 = min(nq, (int)((long long)nqv * (split + 1) / a.splits));
   const int has_tail = (a.tail_len > 0 && split == a.splits - 1) ? 1 : 0;
   const int nF = f1 - f0, nQ = q1 - q0, nJ = nF + has_tail + nQ;
+  const int tail_pages = (a.tail_len + QE_PAGE - 1) / QE_PAGE;
 
-  const int NSB = norm_stage_bytes(w, G);
-  uint8_t* ring = smem + warp * kNST * STAGE;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kNW * kNST * STAGE) + warp * kNST;
-  uint8_t* aux = smem + kNW * kNST * STAGE + kNW * kNST * 8 + warp * aux_bytes<D>(w, G);
-  uint8_t* nring = aux;                                           // [kNST][NSB]
-  float* sst = reinterpret_cast<float*>(aux + kNST * NSB);        // scale staging
+  uint8_t* ring = smem + warp * NST * STAGE;
+  uint8_t* nring = smem + kNW * NST * STAGE + warp * NST * NSB;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kNW * NST * (STAGE + NSB)) + warp * NST;
   if (lane == 0) {
-    for (int s = 0; s < kNST; ++s) mbar_init(&bars[s], 1);
+    for (int s = 0; s < NST; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
   }
   __syncwarp();
 
-  // virtual index j of this split: [0, nF) full, nF the tail (when present), then INT2
+  // virtual index j of this split: [0, nF) full, nF the tail (when present), then INT2.
+  // This warp's windows are j = warp + kNW * o, o < n_own (kinds in that order); each window is
+  // a run of tasks i: full and tail windows K, V of every page; INT2 windows their chunks.
+  const int n_own = nJ > warp ? (nJ - warp + kNW - 1) / kNW : 0;
   auto kind_of = [&](int j) { return j < nF ? 0 : (j < nF + has_tail ? 2 : 1); };  // full, int2, tail
   auto list_idx = [&](int j) { return j < nF ? f0 + j : nf + q0 + (j - nF - has_tail); };
-  auto n_tasks = [&](int j) {
-    const int k = kind_of(j);
-    return k == 0 ? ppw : (k == 1 ? 1 : (a.tail_len + QE_PAGE - 1) / QE_PAGE);
-  };
-  // This warp's windows are j = warp + kNW * o, o < n_own (kinds in the order above).
-  const int n_own = nJ > warp ? (nJ - warp + kNW - 1) / kNW : 0;
-  auto jmap = [&](int o) { return warp + kNW * o; };
-  auto advance = [&](int& o, int& pg) {
-    if (++pg >= n_tasks(jmap(o))) {
-      pg = 0;
-      ++o;
-    }
-  };
+  auto n_sub = [&](int kind) { return kind == 0 ? 2 * PPW : (kind == 1 ? CPW : 2 * tail_pages); };
   // Index prefetch: lane l holds the window id and the page ids (full, tail) or the ledger
   // slot (INT2) of this warp's window of ordinal rb + l, so issuing a copy never waits on a
   // dependent global load. Reloaded every 32 windows.
-  int e_win = -1, e_id[4] = {-1, -1, -1, -1}, rb = -32;
+  int e_win = -1, e_id[PPW], rb = -32;
   auto load_ids = [&](int base) {
     rb = base;
-    const int jj = base + lane < n_own ? jmap(base + lane) : nJ;
+    const int jj = base + lane < n_own ? warp + kNW * (base + lane) : nJ;
     e_win = -1;
 #pragma unroll
-    for (int p = 0; p < 4; ++p) e_id[p] = -1;
+    for (int p = 0; p < PPW; ++p) e_id[p] = -1;
     if (jj < nJ) {
       const int kd = kind_of(jj);
       const int win = kd == 0 ? st.full_list[ub + f0 + jj]
@@ -249,51 +236,53 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
           e_id[0] = st.win_slot[ub + win];
         } else {
 #pragma unroll
-          for (int p = 0; p < 4; ++p)
-            if (p < ppw) e_id[p] = st.win_pages[(ub + win) * ppw + p];
+          for (int p = 0; p < PPW; ++p) e_id[p] = st.win_pages[(ub + win) * PPW + p];
         }
       }
     }
   };
   // fused append: page of the step's token (written by this warp just before the tail's copies)
   int app_pg = -1, app_page = -1;
-  // issue the copies of task (window ordinal r, page pg) into stage s (all lanes call)
-  auto issue = [&](int r, int pg, int s) {
-    const int j = jmap(r);
+  // issue the copies of task (window ordinal r, task i) into stage s (all lanes call)
+  auto issue = [&](int r, int i, int s) {
+    const int j = warp + kNW * r;
     if (r - rb >= 32) load_ids(r - r % 32);
     const int src = r - rb;
-    const int win = __shfl_sync(0xffffffffu, e_win, src);
-    const int sel = pg == 0 ? e_id[0] : (pg == 1 ? e_id[1] : (pg == 2 ? e_id[2] : e_id[3]));
-    int id = __shfl_sync(0xffffffffu, sel, src);
-    uint8_t* dst = ring + s * STAGE;
-    uint8_t* ndst = nring + s * NSB;
-    uint64_t* bar = &bars[s];
     const int k = kind_of(j);
-    if (k == 2 && pg == 0 && a.k_new != nullptr) {
+    const int pg = k == 1 ? 0 : (i >> 1);
+    int sel = e_id[0];
+#pragma unroll
+    for (int p = 1; p < PPW; ++p)
+      if (pg == p) sel = e_id[p];
+    const int win = __shfl_sync(0xffffffffu, e_win, src);
+    int id = __shfl_sync(0xffffffffu, sel, src);
+    if (k == 2 && i == 0 && a.k_new != nullptr) {
       // the step's token goes into the tail window before its pages are copied
       app_page = append_token_warp(st, u, a.append_pos, a.k_new, a.v_new, a.tailV);
-      app_pg = (a.append_pos % w) / QE_PAGE;
+      app_pg = (a.append_pos % W) / QE_PAGE;
     }
     if (k == 2 && pg == app_pg) id = app_page;
     fence_proxy_async_smem();
     if (lane != 0) return;
+    uint8_t* dst = ring + s * STAGE;
+    uint64_t* bar = &bars[s];
     if (k != 1) {
-      // full-precision or tail page: 2 * D/64 swizzled TMA boxes (+ the page's norms)
+      // the K (i even) or V (i odd) rows of a full-precision or tail page: D/64 swizzled TMA
+      // boxes; a full page's K task also brings the page's norms
       if (win < 0 || id < 0 || id >= st.P) {
         qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
         mbar_arrive_expect_tx(bar, 0);
         return;
       }
-      const uint32_t nb = k == 0 ? QE_PAGE * G * 4 : 0;
-      mbar_arrive_expect_tx(bar, PAGE_BYTES + nb);
-      const int row0 = (u * st.P + id) * 2 * QE_PAGE;
+      const bool nrm = k == 0 && (i & 1) == 0;
+      const uint32_t nb = nrm ? QE_PAGE * G * 4 : 0;
+      mbar_arrive_expect_tx(bar, HALF + nb);
+      const int row0 = (u * st.P + id) * 2 * QE_PAGE + (i & 1) * QE_PAGE;
 #pragma unroll
-      for (int part = 0; part < 2; ++part)
-#pragma unroll
-        for (int xb = 0; xb < D / 64; ++xb)
-          tc::tma_load_2d(dst + (part * (D / 64) + xb) * 2048, &tmP, xb * 64, row0 + part * QE_PAGE, bar);
-      if (k == 0)
-        bulk_g2s(ndst, st.norms + ((size_t)u * st.norm_pitch + (size_t)win * w + pg * QE_PAGE) * G, nb, bar);
+      for (int xb = 0; xb < NB; ++xb) tc::tma_load_2d(dst + xb * 2048, &tmP, xb * 64, row0, bar);
+      if (nrm)
+        bulk_g2s(nring + s * NSB, st.norms + ((size_t)u * st.norm_pitch + (size_t)win * W + pg * QE_PAGE) * G, nb,
+                 bar);
       return;
     }
     if (win < 0 || id < 0 || id >= st.S) {
@@ -301,168 +290,243 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
       mbar_arrive_expect_tx(bar, 0);
       return;
     }
-    const uint32_t nb = (uint32_t)(w * G * 4);
-    mbar_arrive_expect_tx(bar, (uint32_t)st.slot_bytes + nb);
-    bulk_g2s(dst, st.slots + ((size_t)u * st.S + id) * st.slot_bytes, (uint32_t)st.slot_bytes, bar);
-    bulk_g2s(ndst, st.norms + ((size_t)u * st.norm_pitch + (size_t)win * w) * G, nb, bar);
+    constexpr uint32_t cb = BPC * BL::BYTES, nb = BPC * QE_PAGE * G * 4;
+    mbar_arrive_expect_tx(bar, cb + nb);
+    bulk_g2s(dst, st.slots + ((size_t)u * st.S + id) * st.slot_bytes + (size_t)i * cb, cb, bar);
+    bulk_g2s(nring + s * NSB, st.norms + ((size_t)u * st.norm_pitch + (size_t)win * W + i * BPC * QE_PAGE) * G, nb,
+             bar);
   };
 
-  // online softmax state of head g8 (lanes g8 >= G carry padding rows): running max (log2
-  // domain), sum of weights, and the current window's sums of weights and weighted norms
-  float mh = -1e30f, lh = 0.f, lwh = 0.f, nwh = 0.f;
-  const float hmask = g8 < G ? 1.f : 0.f;
+  // Scores come out of S^T = K Q^T with tokens as MMA rows and heads as columns: lane (g8, t4)
+  // holds the scores of tokens g8 and 8 + g8 for heads 2 t4 and 2 t4 + 1 (slots 0, 1 and 2, 3
+  // of every 16-token block). Each lane keeps the online-softmax state of its two heads: running
+  // max (log2 domain), sum of weights, and the current window's sums of weights and weighted
+  // norms (per-lane partial sums over its tokens, reduced over the eight token rows when used).
+  const int h0 = 2 * t4, h1 = 2 * t4 + 1;
+  const float hm0 = h0 < G ? 1.f : 0.f, hm1 = h1 < G ? 1.f : 0.f;
+  float m0 = -1e30f, m1 = -1e30f, l0 = 0.f, l1 = 0.f, lw0 = 0.f, lw1 = 0.f, nw0 = 0.f, nw1 = 0.f;
   // O^T accumulators: oacc[m] holds rows (head-dim elements) 16m + g8 (c0, c1) and 16m + 8 + g8
-  // (c2, c3), columns (heads) 2 t4 and 2 t4 + 1. zacc: the INT2 zero-point part, rows = groups.
+  // (c2, c3), columns (heads) h0 and h1. zacc: the INT2 zero-point part, rows = groups.
   float oacc[G8][4];
 #pragma unroll
   for (int m = 0; m < G8; ++m) oacc[m][0] = oacc[m][1] = oacc[m][2] = oacc[m][3] = 0.f;
   float zacc[4] = {0.f, 0.f, 0.f, 0.f};
 
-  // Softmax bookkeeping of one 16-token task: s holds head g8's log2-domain scores of tokens
-  // 2t4, 2t4+1, 8+2t4, 9+2t4 (-inf where absent); p receives their weights 2^(s - max). The
-  // running max starts at a finite -1e30 so that 2^(-inf - m) = 0 needs no guard; one rarely
-  // taken branch rescales the accumulators when the max grows by more than 2^kRescale.
-  auto softmax = [&](const float (&s)[4], float (&p)[4], const float* nrm) {
-    float mx = fmaxf(fmaxf(s[0], s[1]), fmaxf(s[2], s[3]));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    const bool grow = mx > mh + kRescale;
+  // Softmax bookkeeping of N/4 16-token blocks: s holds this lane's log2-domain scores (slots
+  // 4b + {0: token g8 head h0, 1: token g8 head h1, 2: token 8+g8 head h0, 3: token 8+g8 head h1},
+  // -inf where absent); p receives the weights 2^(s - max). The running max starts at a finite
+  // -1e30 so that 2^(-inf - m) = 0 needs no guard; one rarely taken branch rescales the
+  // accumulators when a head's max grows by more than 2^kRescale. nrm (may be null): the blocks'
+  // norms, [16 N/4 tokens][G].
+  auto softmax = [&](auto& s, auto& p, const float* nrm) {
+    constexpr int N = sizeof(s) / sizeof(float);
+    float x0 = s[0], x1 = s[1];
+#pragma unroll
+    for (int i = 2; i < N; i += 2) {
+      x0 = fmaxf(x0, s[i]);
+      x1 = fmaxf(x1, s[i + 1]);
+    }
+    // a head's max grows past m + kRescale exactly when one of its lanes sees such a score; only
+    // then is the max reduced over the eight token rows
+    const bool grow = x0 > m0 + kRescale || x1 > m1 + kRescale;
     if (__any_sync(0xffffffffu, grow)) {
-      const float mn = grow ? mx : mh;
-      const float f = ex2(mh - mn);
-      lh *= f;
-      lwh *= f;
-      nwh *= f;
-      mh = mn;
-      // O^T columns 2 t4, 2 t4 + 1 belong to the heads of lanes 8 t4 and 8 t4 + 4
-      const float fa = __shfl_sync(0xffffffffu, f, 8 * t4);
-      const float fb = __shfl_sync(0xffffffffu, f, 8 * t4 + 4);
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, o));
+        x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, o));
+      }
+      const float n0 = x0 > m0 + kRescale ? x0 : m0, n1 = x1 > m1 + kRescale ? x1 : m1;
+      const float f0 = ex2(m0 - n0), f1 = ex2(m1 - n1);
+      l0 *= f0;
+      lw0 *= f0;
+      nw0 *= f0;
+      l1 *= f1;
+      lw1 *= f1;
+      nw1 *= f1;
+      m0 = n0;
+      m1 = n1;
 #pragma unroll
       for (int m = 0; m < G8; ++m) {
-        oacc[m][0] *= fa;
-        oacc[m][1] *= fb;
-        oacc[m][2] *= fa;
-        oacc[m][3] *= fb;
+        oacc[m][0] *= f0;
+        oacc[m][1] *= f1;
+        oacc[m][2] *= f0;
+        oacc[m][3] *= f1;
       }
-      zacc[0] *= fa;
-      zacc[1] *= fb;
+      zacc[0] *= f0;
+      zacc[1] *= f1;
     }
+    float ps0 = 0.f, ps1 = 0.f;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) p[i] = hmask * ex2(s[i] - mh);
-    const float psum = (p[0] + p[1]) + (p[2] + p[3]);
-    lh += psum;
-    lwh += psum;
-    if (nrm != nullptr && g8 < G) {
-      nwh = fmaf(p[0], nrm[(2 * t4) * G + g8], nwh);
-      nwh = fmaf(p[1], nrm[(2 * t4 + 1) * G + g8], nwh);
-      nwh = fmaf(p[2], nrm[(8 + 2 * t4) * G + g8], nwh);
-      nwh = fmaf(p[3], nrm[(9 + 2 * t4) * G + g8], nwh);
+    for (int i = 0; i < N; i += 2) {
+      p[i] = hm0 * ex2(s[i] - m0);
+      p[i + 1] = hm1 * ex2(s[i + 1] - m1);
+      ps0 += p[i];
+      ps1 += p[i + 1];
+    }
+    l0 += ps0;
+    l1 += ps1;
+    lw0 += ps0;
+    lw1 += ps1;
+    if (nrm != nullptr) {
+#pragma unroll
+      for (int i = 0; i < N; i += 2) {
+        const int tok = 16 * (i >> 2) + g8 + 8 * ((i >> 1) & 1);
+        const float* nr = nrm + tok * G;
+        float a0, a1;
+        if constexpr (G % 2 == 0) {
+          const float2 v = *reinterpret_cast<const float2*>(nr + (h0 < G ? h0 : 0));
+          a0 = v.x;
+          a1 = v.y;
+        } else {
+          a0 = nr[h0 < G ? h0 : 0];
+          a1 = nr[h1 < G ? h1 : 0];
+        }
+        nw0 = fmaf(p[i], a0, nw0);
+        nw1 = fmaf(p[i + 1], a1, nw1);
+      }
     }
   };
   // end of a window: its partial (max, sum p, sum p n) per head into the window's slot
   auto window_end = [&](int li) {
-    float l2 = lwh + __shfl_xor_sync(0xffffffffu, lwh, 1);
-    l2 += __shfl_xor_sync(0xffffffffu, l2, 2);
-    float n2 = nwh + __shfl_xor_sync(0xffffffffu, nwh, 1);
-    n2 += __shfl_xor_sync(0xffffffffu, n2, 2);
-    if (t4 == 0 && g8 < G) {
-      float* wp = a.win_part + (ub + li) * win_part_floats(D, G) + g8;
-      wp[0] = mh;
-      wp[G] = l2;
-      wp[2 * G] = n2;
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      lw0 += __shfl_xor_sync(0xffffffffu, lw0, o);
+      lw1 += __shfl_xor_sync(0xffffffffu, lw1, o);
+      nw0 += __shfl_xor_sync(0xffffffffu, nw0, o);
+      nw1 += __shfl_xor_sync(0xffffffffu, nw1, o);
     }
-    lwh = 0.f;
-    nwh = 0.f;
+    if (g8 == 0) {
+      float* wp = a.win_part + (ub + li) * win_part_floats(D, G);
+      if (h0 < G) {
+        wp[h0] = m0;
+        wp[G + h0] = lw0;
+        wp[2 * G + h0] = nw0;
+      }
+      if (h1 < G) {
+        wp[h1] = m1;
+        wp[G + h1] = lw1;
+        wp[2 * G + h1] = nw1;
+      }
+    }
+    lw0 = lw1 = nw0 = nw1 = 0.f;
+  };
+  // P of one 16-token block as the B fragment of O^T = V^T P^T (tokens 2t4, 2t4+1 | 8+2t4,
+  // 9+2t4 of head g8): the 16-bit pairs of the score layout, transposed 8x8 by movmatrix
+  auto transpose_pair = [&](uint32_t x) {
+    uint32_t y;
+    asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
   };
 
-  int o = 0, pg = 0;                  // window ordinal and page being computed
-  int io = 0, ipg = 0, issued = 0;    // next task to copy
-  for (int s = 0; s < kNST - 1 && io < n_own; ++s) {
-    issue(io, ipg, s);
-    advance(io, ipg);
+  int o = 0, ti = 0;                  // window ordinal and task being computed
+  int io = 0, ii = 0, issued = 0;     // next task to copy
+  auto advance = [&](int& r, int& i) {
+    if (++i >= n_sub(kind_of(warp + kNW * r))) {
+      i = 0;
+      ++r;
+    }
+  };
+  for (int s = 0; s < NST - 1 && io < n_own; ++s) {
+    issue(io, ii, s);
+    advance(io, ii);
     ++issued;
   }
   int k = 0;
   bool ok = true;
+  // wait for the task computed next, after issuing the one NST - 1 ahead
+  auto next_stage = [&]() -> int {
+    if (io < n_own) {
+      issue(io, ii, issued % NST);
+      advance(io, ii);
+      ++issued;
+    }
+    const int s = k % NST;
+    ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[s], (k / NST) & 1, st.status, 1000 + u));
+    return s;
+  };
 
-  // q fragments (A operand, cache dtype): head g8's elements 16m + 2t4, +1 and 16m + 8 + 2t4, +1
-  uint32_t qa[G8][2];
+  // q as the B operand of S^T = K Q^T (cache dtype): head g8's elements 16m + 2t4, +1 (qb[m][0])
+  // and 16m + 8 + 2t4, +1 (qb[m][1]); zero for padding heads
+  uint32_t qb[G8][2];
   {
     const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
         reinterpret_cast<const T*>(a.q) + ((size_t)b * st.Hq + (size_t)kvh * G + (g8 < G ? g8 : 0)) * D);
 #pragma unroll
     for (int m = 0; m < G8; ++m) {
-      qa[m][0] = g8 < G ? qrow[m * 8 + t4] : 0u;
-      qa[m][1] = g8 < G ? qrow[m * 8 + 4 + t4] : 0u;
+      qb[m][0] = g8 < G ? qrow[m * 8 + t4] : 0u;
+      qb[m][1] = g8 < G ? qrow[m * 8 + 4 + t4] : 0u;
     }
   }
 
-  // ---- phase 1: full-precision windows, then the tail, from swizzled TMA pages ----
-  while (o < n_own && kind_of(jmap(o)) != 1) {
-    if (io < n_own) {
-      issue(io, ipg, issued % kNST);
-      advance(io, ipg);
-      ++issued;
-    }
-    const int s = k % kNST;
-    ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[s], (k / kNST) & 1, st.status, 1000 + u));
-    if (!ok) break;
-    uint8_t* stage = ring + s * STAGE;
-    const int j = jmap(o);
-    const bool tail = kind_of(j) == 2;
-    const int valid = tail ? min(QE_PAGE, a.tail_len - pg * QE_PAGE) : QE_PAGE;
-    if (valid < QE_PAGE) {
-      // rows past the tail's last token hold stale data: zero their V rows (weight 0 must not
-      // meet a NaN) and mask their scores below
-      for (int i = lane; i < (QE_PAGE - valid) * (D / 64) * 8; i += 32) {
-        const int row = valid + i / ((D / 64) * 8), rest = i % ((D / 64) * 8);
-        *reinterpret_cast<uint4*>(stage + ((D / 64) + rest / 8) * 2048 + row * 128 + (rest % 8) * 16) =
-            make_uint4(0u, 0u, 0u, 0u);
+  // ---- phase 1: full-precision windows, then the tail: K task (scores, softmax), V task ----
+  {
+    uint32_t ph0 = 0, pl0 = 0, ph1 = 0, pl1 = 0;  // P^T of the last K task, for its V task
+    int valid = QE_PAGE;
+    while (o < n_own && kind_of(warp + kNW * o) != 1) {
+      const int s = next_stage();
+      if (!ok) break;
+      uint8_t* stage = ring + s * STAGE;
+      const int j = warp + kNW * o;
+      const bool tail = kind_of(j) == 2;
+      if ((ti & 1) == 0) {
+        // K rows: S^T = K Q^T over 16 tokens, two independent chains
+        valid = tail ? min(QE_PAGE, a.tail_len - (ti >> 1) * QE_PAGE) : QE_PAGE;
+        float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int m = 0; m < G8; ++m) {
+          uint32_t ka[4];
+          ldsm_x4(ka, stage + swz<D>(0, ((lane >> 3) & 1) * 8 + (lane & 7), m * 16 + (lane >> 4) * 8));
+          if (m & 1) MmaOp<T>::run(c1, ka[0], ka[1], ka[2], ka[3], qb[m][0], qb[m][1]);
+          else MmaOp<T>::run(c0, ka[0], ka[1], ka[2], ka[3], qb[m][0], qb[m][1]);
+        }
+        float sc[4] = {(c0[0] + c1[0]) * sl, (c0[1] + c1[1]) * sl, (c0[2] + c1[2]) * sl, (c0[3] + c1[3]) * sl};
+        if (tail) {
+          const int pg = ti >> 1;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int tk = g8 + 8 * (i >> 1), hh = 2 * t4 + (i & 1);
+            if (tk >= valid) sc[i] = -INFINITY;
+            else if (hh < G) a.tail_s[((size_t)u * W + pg * QE_PAGE + tk) * G + hh] = sc[i];
+          }
+        }
+        float p[4];
+        softmax(sc, p, tail ? nullptr : reinterpret_cast<const float*>(nring + s * NSB));
+        uint32_t x0, y0, x1, y1;
+        MmaOp<T>::split(p[0], p[1], x0, y0);
+        MmaOp<T>::split(p[2], p[3], x1, y1);
+        ph0 = transpose_pair(x0);
+        pl0 = transpose_pair(y0);
+        ph1 = transpose_pair(x1);
+        pl1 = transpose_pair(y1);
+        if (tail) {
+          // the tail's mass is formed at the end from its token scores; its sums belong to no slot
+          lw0 = lw1 = nw0 = nw1 = 0.f;
+        }
+      } else {
+        // V rows: O^T += V^T P^T
+        if (valid < QE_PAGE) {
+          // rows past the tail's last token hold stale data: zero them (weight 0 must not meet
+          // a NaN)
+          for (int i = lane; i < (QE_PAGE - valid) * NB * 8; i += 32) {
+            const int row = valid + i / (NB * 8), rest = i % (NB * 8);
+            *reinterpret_cast<uint4*>(stage + (rest / 8) * 2048 + row * 128 + (rest % 8) * 16) =
+                make_uint4(0u, 0u, 0u, 0u);
+          }
+          __syncwarp();
+        }
+#pragma unroll
+        for (int m = 0; m < G8; ++m) {
+          uint32_t va[4];
+          ldsm_x4_t(va, stage + swz<D>(0, ((lane >> 4) << 3) + (lane & 7), m * 16 + ((lane >> 3) & 1) * 8));
+          MmaOp<T>::run(oacc[m], va[0], va[1], va[2], va[3], ph0, ph1);
+          MmaOp<T>::run(oacc[m], va[0], va[1], va[2], va[3], pl0, pl1);
+        }
+        if (!tail && ti == 2 * PPW - 1) window_end(list_idx(j));
       }
       __syncwarp();
+      advance(o, ti);
+      ++k;
     }
-    float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int kc2 = 0; kc2 < D / 32; ++kc2) {
-      uint32_t kb[4];
-      ldsm_x4(kb, stage + swz<D>(0, lane & 7, kc2 * 32 + (lane >> 3) * 8));
-      MmaOp<T>::run(c0, qa[2 * kc2][0], 0u, qa[2 * kc2][1], 0u, kb[0], kb[1]);
-      MmaOp<T>::run(c0, qa[2 * kc2 + 1][0], 0u, qa[2 * kc2 + 1][1], 0u, kb[2], kb[3]);
-      ldsm_x4(kb, stage + swz<D>(0, 8 + (lane & 7), kc2 * 32 + (lane >> 3) * 8));
-      MmaOp<T>::run(c1, qa[2 * kc2][0], 0u, qa[2 * kc2][1], 0u, kb[0], kb[1]);
-      MmaOp<T>::run(c1, qa[2 * kc2 + 1][0], 0u, qa[2 * kc2 + 1][1], 0u, kb[2], kb[3]);
-    }
-    float sc[4] = {c0[0] * sl, c0[1] * sl, c1[0] * sl, c1[1] * sl};
-    if (tail) {
-      const int tk[4] = {2 * t4, 2 * t4 + 1, 8 + 2 * t4, 9 + 2 * t4};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        if (tk[i] >= valid) sc[i] = -INFINITY;
-        else if (g8 < G) a.tail_s[((size_t)u * w + pg * QE_PAGE + tk[i]) * G + g8] = sc[i];
-      }
-    }
-    float p[4];
-    softmax(sc, p, tail ? nullptr : reinterpret_cast<const float*>(nring + s * NSB));
-    uint32_t ph0, pl0, ph1, pl1;
-    MmaOp<T>::split(p[0], p[1], ph0, pl0);
-    MmaOp<T>::split(p[2], p[3], ph1, pl1);
-#pragma unroll
-    for (int m = 0; m < G8; ++m) {
-      uint32_t va[4];
-      ldsm_x4_t(va, stage + swz<D>(1, ((lane >> 4) << 3) + (lane & 7), m * 16 + ((lane >> 3) & 1) * 8));
-      MmaOp<T>::run(oacc[m], va[0], va[1], va[2], va[3], ph0, ph1);
-      MmaOp<T>::run(oacc[m], va[0], va[1], va[2], va[3], pl0, pl1);
-    }
-    __syncwarp();
-    if (tail) {
-      // the tail's mass is formed at the end from its token scores; its sums belong to no slot
-      lwh = 0.f;
-      nwh = 0.f;
-    } else if (pg + 1 >= ppw) {
-      window_end(list_idx(j));
-    }
-    advance(o, pg);
-    ++k;
   }
 
   // ---- phase 2: INT2 ledger entries ----
@@ -478,69 +542,45 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
   if (ok && o < n_own) {
     // q as fp16 with the elements 8 + 2t4, 9 + 2t4 of each group quartered (their codes carry
     // 4x), and head g8's sum of q over groups 2t4, 2t4 + 1 in the log2 domain, split hi + lo
+    // (the B operand of the zero-point product Z Q_g)
     uint32_t qh[G8][2];
-    float qs[G8];
+    float qg0 = 0.f, qg1 = 0.f;
 #pragma unroll
     for (int m = 0; m < G8; ++m) {
-      const float x0 = Elem<T>::lo(qa[m][0]), x1 = Elem<T>::hi(qa[m][0]);
-      const float x2 = Elem<T>::lo(qa[m][1]), x3 = Elem<T>::hi(qa[m][1]);
+      const float x0 = Elem<T>::lo(qb[m][0]), x1 = Elem<T>::hi(qb[m][0]);
+      const float x2 = Elem<T>::lo(qb[m][1]), x3 = Elem<T>::hi(qb[m][1]);
       qh[m][0] = pack_h2(x0, x1);
       qh[m][1] = pack_h2(0.25f * x2, 0.25f * x3);
       float t = (x0 + x1) + (x2 + x3);
       t += __shfl_xor_sync(0xffffffffu, t, 1);
       t += __shfl_xor_sync(0xffffffffu, t, 2);
-      qs[m] = t * sl;
-    }
-    float qg0 = 0.f, qg1 = 0.f;
-#pragma unroll
-    for (int m = 0; m < G8; ++m) {
-      if (m == 2 * t4) qg0 = qs[m];
-      if (m == 2 * t4 + 1) qg1 = qs[m];
+      if (m == 2 * t4) qg0 = t * sl;
+      if (m == 2 * t4 + 1) qg1 = t * sl;
     }
     const uint32_t qgh = pack_h2(qg0, qg1);
     const uint32_t qgl = pack_h2(qg0 - h_lo(qgh), qg1 - h_hi(qgh));
-    // staged scale factors: K scores of tokens 0..7 carry 2^-24, of tokens 8..15 16 * 2^-24;
-    // V rows 8..15 of the block carry 4x in their codes, so their P * s is quartered
-    const int stk = lane & 15, kvsel = lane >> 4;
-    const float sfac = kvsel == 0 ? (stk < 8 ? 0x1p24f * sl : 0x1p20f * sl) : (stk < 8 ? 1.f : 0.25f);
-    float* sdst = sst + kvsel * 4 * SROW + ((stk & 7) >> 1) * SROW + ((stk & 1) + 2 * (stk >> 3));
-    const float* sk = sst + t4 * SROW;
-    const float* sv = sst + 4 * SROW + t4 * SROW;
+    // selection matrix that deals a token's K scale to both head columns: row 0 picks all
+    const uint32_t sel0 = t4 == 0 ? 0x3c00u : 0u;
+    const float2 fa = make_float2(0x1p24f * sl, 0x1p24f * sl), fb = make_float2(0x1p20f * sl, 0x1p20f * sl);
+    constexpr uint32_t kQuarter2 = 0x34003400u;  // fp16 pair {0.25, 0.25}
 
     while (o < n_own) {
-      if (io < n_own) {
-        issue(io, ipg, issued % kNST);
-        advance(io, ipg);
-        ++issued;
-      }
-      const int s = k % kNST;
-      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[s], (k / kNST) & 1, st.status, 1000 + u));
+      const int s = next_stage();
       if (!ok) break;
       const uint8_t* stage = ring + s * STAGE;
-      const float* nrm = reinterpret_cast<const float*>(nring + s * NSB);
-      for (int bk = 0; bk < w / 16; ++bk) {
-        const uint8_t* blk = stage + bk * BL::BYTES;
-        {  // stage this block's scales: lanes 0-15 the K scales of token lane, 16-31 the V scales
-          const __half* srow = reinterpret_cast<const __half*>(blk + (kvsel ? BL::VS : BL::KS)) + stk * G8;
+      float sc[4 * BPC], p[4 * BPC];
 #pragma unroll
-          for (int m = 0; m < G8; ++m) sdst[m * 4] = __half2float(srow[m]) * sfac;
-        }
-        __syncwarp();
-        // ---- K side: scores of tokens 2t4, 2t4+1 (tile A) and 8+2t4, 9+2t4 (tile B) ----
-        float sc[4];
+      for (int bk = 0; bk < BPC; ++bk) {
+        // ---- K side: S^T = (C s + Z) Q^T for tokens g8, 8 + g8 and heads h0, h1 ----
+        const uint8_t* blk = stage + bk * BL::BYTES;
+        float zs[4] = {0.f, 0.f, 0.f, 0.f};
         {
-          const uint32_t zA = 2 * t4 < G8 ? *reinterpret_cast<const uint32_t*>(blk + BL::KZ + (g8 * G8 + 2 * t4) * 2) : 0u;
+          const uint32_t zA =
+              2 * t4 < G8 ? *reinterpret_cast<const uint32_t*>(blk + BL::KZ + (g8 * G8 + 2 * t4) * 2) : 0u;
           const uint32_t zB =
               2 * t4 < G8 ? *reinterpret_cast<const uint32_t*>(blk + BL::KZ + ((8 + g8) * G8 + 2 * t4) * 2) : 0u;
-          float za[4] = {0.f, 0.f, 0.f, 0.f}, zb[4] = {0.f, 0.f, 0.f, 0.f};
-          mma_h8(za, qgh, 0u, zA);
-          mma_h8(za, qgl, 0u, zA);
-          mma_h8(zb, qgh, 0u, zB);
-          mma_h8(zb, qgl, 0u, zB);
-          sc[0] = za[0];
-          sc[1] = za[1];
-          sc[2] = zb[0];
-          sc[3] = zb[1];
+          mma_h8(zs, zA, zB, qgh);
+          mma_h8(zs, zA, zB, qgl);
         }
         uint32_t kw[WPL];
         if constexpr (WPL == 4) {
@@ -550,37 +590,48 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
           const uint2 v2 = *reinterpret_cast<const uint2*>(blk + BL::KC + lane * 8);
           kw[0] = v2.x; kw[1] = v2.y;
         }
+        float2 sA = make_float2(0.f, 0.f), sB = make_float2(0.f, 0.f);
 #pragma unroll
         for (int jj = 0; jj < WPL; ++jj) {
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int m = 2 * jj + e;
             const uint32_t x = e ? (kw[jj] >> 8) : kw[jj];
-            float cA[4] = {0.f, 0.f, 0.f, 0.f}, cB[4] = {0.f, 0.f, 0.f, 0.f};
-            mma_h16(cA, qh[m][0], 0u, qh[m][1], 0u, code_reg<0>(x), code_reg<1>(x));
-            mma_h16(cB, qh[m][0], 0u, qh[m][1], 0u, code_reg<2>(x), code_reg<3>(x));
-            const float4 s4 = *reinterpret_cast<const float4*>(sk + m * 4);
-            const float2 ra = ffma2(make_float2(s4.x, s4.y), make_float2(cA[0], cA[1]), make_float2(sc[0], sc[1]));
-            const float2 rb = ffma2(make_float2(s4.z, s4.w), make_float2(cB[0], cB[1]), make_float2(sc[2], sc[3]));
-            sc[0] = ra.x;
-            sc[1] = ra.y;
-            sc[2] = rb.x;
-            sc[3] = rb.y;
+            // this lane's token scales s(g8), s(8 + g8) as float32 in both head columns
+            const uint32_t sp = *reinterpret_cast<const uint32_t*>(blk + BL::KS + (m * QE_PAGE + 2 * g8) * 2);
+            float cs[4] = {0.f, 0.f, 0.f, 0.f}, cc[4] = {0.f, 0.f, 0.f, 0.f};
+            mma_h8(cs, sp, __byte_perm(sp, 0u, 0x1032), sel0);
+            mma_h16(cc, code_reg<0>(x), code_reg<2>(x), code_reg<1>(x), code_reg<3>(x), qh[m][0], qh[m][1]);
+            sA = ffma2(make_float2(cs[0], cs[1]), make_float2(cc[0], cc[1]), sA);
+            sB = ffma2(make_float2(cs[2], cs[3]), make_float2(cc[2], cc[3]), sB);
           }
         }
-        float p[4];
-        softmax(sc, p, nrm + bk * 16 * G);
-        // ---- V side ----
+        sA = ffma2(sA, fa, make_float2(zs[0], zs[1]));
+        sB = ffma2(sB, fb, make_float2(zs[2], zs[3]));
+        sc[4 * bk + 0] = sA.x;
+        sc[4 * bk + 1] = sA.y;
+        sc[4 * bk + 2] = sB.x;
+        sc[4 * bk + 3] = sB.y;
+      }
+      softmax(sc, p, reinterpret_cast<const float*>(nring + s * NSB));
+#pragma unroll
+      for (int bk = 0; bk < BPC; ++bk) {
+        // ---- V side: O^T += V^T (P^T s) per group, zero points Z^T P^T ----
+        const uint8_t* blk = stage + bk * BL::BYTES;
+        const float* pb = p + 4 * bk;
+        uint32_t x0, y0, x1, y1;
+        MmaOp<__half>::split(pb[0], pb[1], x0, y0);
+        MmaOp<__half>::split(pb[2], pb[3], x1, y1);
+        const uint32_t ph0 = transpose_pair(x0), pl0 = transpose_pair(y0);
+        const uint32_t ph1 = transpose_pair(x1), pl1 = transpose_pair(y1);
         {
-          uint32_t ph0, pl0, ph1, pl1;
-          MmaOp<__half>::split(p[0], p[1], ph0, pl0);
-          MmaOp<__half>::split(p[2], p[3], ph1, pl1);
-          const uint32_t za0 = g8 < G8 ? *reinterpret_cast<const uint32_t*>(blk + BL::VZ + (g8 * 16 + 2 * t4) * 2) : 0u;
-          const uint32_t za2 =
-              g8 < G8 ? *reinterpret_cast<const uint32_t*>(blk + BL::VZ + (g8 * 16 + 8 + 2 * t4) * 2) : 0u;
-          mma_h16(zacc, za0, 0u, za2, 0u, ph0, ph1);
-          mma_h16(zacc, za0, 0u, za2, 0u, pl0, pl1);
+          uint2 zg = make_uint2(0u, 0u);
+          if (g8 < G8) zg = *reinterpret_cast<const uint2*>(blk + BL::VZ + (g8 * QE_PAGE + 4 * t4) * 2);
+          mma_h16(zacc, zg.x, 0u, zg.y, 0u, ph0, ph1);
+          mma_h16(zacc, zg.x, 0u, zg.y, 0u, pl0, pl1);
         }
+        // the codes of tokens 8..15 carry 4x: their weights are quartered (exact)
+        const uint32_t pq1 = __hmul2_u32(ph1, kQuarter2);
         uint32_t vw[WPL];
         if constexpr (WPL == 4) {
           const uint4 v4 = *reinterpret_cast<const uint4*>(blk + BL::VC + lane * 16);
@@ -595,21 +646,20 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
           for (int e = 0; e < 2; ++e) {
             const int m = 2 * jj + e;
             const uint32_t x = e ? (vw[jj] >> 8) : vw[jj];
-            const float4 s4 = *reinterpret_cast<const float4*>(sv + m * 4);
-            const uint32_t b0 = pack_h2(p[0] * s4.x, p[1] * s4.y);
-            const uint32_t b1 = pack_h2(p[2] * s4.z, p[3] * s4.w);
-            mma_h16(oacc[m], code_reg<0>(x), code_reg<2>(x), code_reg<1>(x), code_reg<3>(x), b0, b1);
+            const uint2 sg = *reinterpret_cast<const uint2*>(blk + BL::VS + (m * QE_PAGE + 4 * t4) * 2);
+            mma_h16(oacc[m], code_reg<0>(x), code_reg<2>(x), code_reg<1>(x), code_reg<3>(x),
+                    __hmul2_u32(ph0, sg.x), __hmul2_u32(pq1, sg.y));
           }
         }
-        __syncwarp();  // the next block restages the scales
       }
-      window_end(list_idx(jmap(o)));
-      advance(o, pg);
+      __syncwarp();
+      if (ti == CPW - 1) window_end(list_idx(warp + kNW * o));
+      advance(o, ti);
       ++k;
     }
   }
   if (!ok) {  // drain copies still in flight if a wait gave up
-    for (; k < issued; ++k) mbar_wait_bounded(&bars[k % kNST], (k / kNST) & 1, st.status, 2000 + u);
+    for (; k < issued; ++k) mbar_wait_bounded(&bars[k % NST], (k / NST) & 1, st.status, 2000 + u);
   }
   // back to O^T: undo the code scales and add the zero-point part of each element's group
 #pragma unroll
@@ -621,11 +671,36 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
     oacc[m][2] = fmaf(oacc[m][2], 0x1p20f, z0);
     oacc[m][3] = fmaf(oacc[m][3], 0x1p20f, z1);
   }
-  lh += __shfl_xor_sync(0xffffffffu, lh, 1);
-  lh += __shfl_xor_sync(0xffffffffu, lh, 2);
+#pragma unroll
+  for (int o2 = 4; o2 < 32; o2 <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, o2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, o2);
+  }
 
   // ---- merge the warps into the CTA's partial ----
   const bool cta_ok = __syncthreads_and(ok ? 1 : 0) != 0;  // also: every warp is done with its ring
+  // the window scores this CTA updates: fetch their ids, partials and cumulative values now so
+  // that the loads overlap the merges below (one window per thread and pass)
+  constexpr int kPre = 1;
+  int pw_win[kPre];
+  float pw_m[kPre], pw_p[kPre], pw_part[kPre][3 * G];
+#pragma unroll
+  for (int x = 0; x < kPre; ++x) {
+    const int jj = threadIdx.x + x * kNW * 32;
+    pw_win[x] = -1;
+    if (jj < nF + nQ) {
+      const int li = list_idx(jj < nF ? jj : jj + has_tail);
+      const int win = jj < nF ? st.full_list[ub + li] : st.int2_list[ub + li - nf];
+      if (win >= 0 && win < st.Wmax) {
+        pw_win[x] = win;
+        pw_m[x] = st.mass[ub + win];
+        pw_p[x] = st.pert[ub + win];
+        const float* wp = a.win_part + (ub + li) * win_part_floats(D, G);
+#pragma unroll
+        for (int h = 0; h < 3 * G; ++h) pw_part[x][h] = wp[h];
+      }
+    }
+  }
   float* mw = reinterpret_cast<float*>(smem);  // [kNW][G]
   float* lwv = mw + kNW * G;                   // [kNW][G]
   float* aw = lwv + kNW * G;                   // [kNW][G][D]
@@ -639,20 +714,29 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
   float* lse = gl + QE_MAX_G;                         // [G] unit log2-sum-exp
   float* red = lse + QE_MAX_G;                        // [kNW]
   float* okv = red + kNW;                             // [1] this CTA finished every wait
-  if (t4 == 0 && g8 < G) {
-    mw[warp * G + g8] = mh;
-    lwv[warp * G + g8] = lh;
-  }
-#pragma unroll
-  for (int m = 0; m < G8; ++m) {
-    float* a0 = aw + (size_t)warp * G * D;
-    if (2 * t4 < G) {
-      a0[(2 * t4) * D + m * 16 + g8] = oacc[m][0];
-      a0[(2 * t4) * D + m * 16 + 8 + g8] = oacc[m][2];
+  float* oks = okv + 1;                               // [S] every CTA's flag
+  if (g8 == 0) {
+    if (h0 < G) {
+      mw[warp * G + h0] = m0;
+      lwv[warp * G + h0] = l0;
     }
-    if (2 * t4 + 1 < G) {
-      a0[(2 * t4 + 1) * D + m * 16 + g8] = oacc[m][1];
-      a0[(2 * t4 + 1) * D + m * 16 + 8 + g8] = oacc[m][3];
+    if (h1 < G) {
+      mw[warp * G + h1] = m1;
+      lwv[warp * G + h1] = l1;
+    }
+  }
+  {
+    float* a0 = aw + (size_t)warp * G * D;
+#pragma unroll
+    for (int m = 0; m < G8; ++m) {
+      if (2 * t4 < G) {
+        a0[(2 * t4) * D + m * 16 + g8] = oacc[m][0];
+        a0[(2 * t4) * D + m * 16 + 8 + g8] = oacc[m][2];
+      }
+      if (2 * t4 + 1 < G) {
+        a0[(2 * t4 + 1) * D + m * 16 + g8] = oacc[m][1];
+        a0[(2 * t4 + 1) * D + m * 16 + 8 + g8] = oacc[m][3];
+      }
     }
   }
   if (threadIdx.x == 0) okv[0] = cta_ok ? 1.f : 0.f;
@@ -681,14 +765,17 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
   const int S = a.splits;
   cluster_sync();
   for (int i = threadIdx.x; i < S * G; i += blockDim.x) {
-    pm[i] = ld_cluster(cm + i % G, (uint32_t)(i / G));
-    pl[i] = ld_cluster(cl + i % G, (uint32_t)(i / G));
+    const float vm = ld_cluster(cm + i % G, (uint32_t)(i / G));
+    const float vl = ld_cluster(cl + i % G, (uint32_t)(i / G));
+    pm[i] = vm;
+    pl[i] = vl;
   }
   // every CTA of the unit must have finished its waits: a CTA that gave up holds partials of
   // a part of its windows, and window partials it never wrote may be stale
-  float all_ok = 1.f;
-  for (int r = 0; r < S; ++r) all_ok = fminf(all_ok, ld_cluster(okv, (uint32_t)r));
+  if (threadIdx.x < S) oks[threadIdx.x] = ld_cluster(okv, (uint32_t)threadIdx.x);
   __syncthreads();
+  float all_ok = 1.f;
+  for (int r = 0; r < S; ++r) all_ok = fminf(all_ok, oks[r]);
   if (threadIdx.x < G) {
     const int h = threadIdx.x;
     float M = pm[h];
@@ -708,19 +795,20 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
     const int i1 = min((split + 1) * per, G * D);
     for (int i = split * per + threadIdx.x; i < i1; i += blockDim.x) {
       const int h = i / D;
+      float v[QE_MAX_SPLITS_CLUSTER];
+#pragma unroll
+      for (int r = 0; r < QE_MAX_SPLITS_CLUSTER; ++r)
+        if (r < S) v[r] = ld_cluster(ca + i, (uint32_t)r);
       float A = 0.f;
-      for (int r = 0; r < S; ++r) A = fmaf(ld_cluster(ca + i, (uint32_t)r), pf[r * G + h], A);
+#pragma unroll
+      for (int r = 0; r < QE_MAX_SPLITS_CLUSTER; ++r)
+        if (r < S) A = fmaf(v[r], pf[r * G + h], A);
       a.out[((size_t)b * st.Hq + (size_t)kvh * G + h) * D + i % D] = A / gl[h];
     }
   }
   if (all_ok > 0.f) {
     // exact attention mass and perturbation of this step for the windows this CTA streamed
-    for (int jj = threadIdx.x; jj < nF + nQ; jj += blockDim.x) {
-      const int vj = jj < nF ? jj : jj + has_tail;
-      const int li = list_idx(vj);
-      const int win = jj < nF ? st.full_list[ub + li] : st.int2_list[ub + li - nf];
-      if (win < 0 || win >= st.Wmax) continue;
-      const float* wp = a.win_part + (ub + li) * win_part_floats(D, G);
+    auto update = [&](int win, float m0, float p0, const float* wp) {
       float dm = 0.f, dp = 0.f;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
@@ -728,16 +816,25 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
         dm = fmaf(wp[G + h], f, dm);
         dp = fmaf(wp[2 * G + h], f, dp);
       }
-      st.mass[ub + win] += dm;
-      st.pert[ub + win] += dp;
+      st.mass[ub + win] = m0 + dm;
+      st.pert[ub + win] = p0 + dp;
+    };
+#pragma unroll
+    for (int x = 0; x < kPre; ++x)
+      if (pw_win[x] >= 0) update(pw_win[x], pw_m[x], pw_p[x], pw_part[x]);
+    for (int jj = threadIdx.x + kPre * kNW * 32; jj < nF + nQ; jj += blockDim.x) {
+      const int li = list_idx(jj < nF ? jj : jj + has_tail);
+      const int win = jj < nF ? st.full_list[ub + li] : st.int2_list[ub + li - nf];
+      if (win >= 0 && win < st.Wmax)
+        update(win, st.mass[ub + win], st.pert[ub + win], a.win_part + (ub + li) * win_part_floats(D, G));
     }
     // tail tokens (last CTA of the cluster): cumulative per-token attention and window mass
     if (has_tail) {
       float tm = 0.f;
       for (int i = threadIdx.x; i < a.tail_len * G; i += blockDim.x) {
         const int h = i % G;
-        const float pv = ex2(a.tail_s[(size_t)u * w * G + i] - lse[h]);
-        st.tail_p[(size_t)u * w * G + i] += pv;
+        const float pv = ex2(a.tail_s[(size_t)u * W * G + i] - lse[h]);
+        st.tail_p[(size_t)u * W * G + i] += pv;
         tm += pv;
       }
       tm = warp_sum(tm);
@@ -753,52 +850,46 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
   cluster_sync();  // keep this CTA's partial alive until every CTA of the cluster has read it
 }
 
-template <typename T, int D, int G>
-int launch_decode_t(qe_ctx* c, const void* q, float* out, cudaStream_t s, const void* k_new,
+template <typename T, int D, int G, int W>
+int launch_decode_w(qe_ctx* c, const void* q, float* out, cudaStream_t s, const void* k_new,
                     const void* v_new) {
-  constexpr int STAGE = StageLayout<D>::BYTES;
-  auto smem_for = [](int w) {
-    return (size_t)1024 + (size_t)kNW * kNST * STAGE + kNW * kNST * 8 + (size_t)kNW * aux_bytes<D>(w, G);
-  };
+  constexpr size_t smem = decode_smem_bytes<D, G>();
   static_assert((size_t)(kNW * G * (D + 2) + 2 * QE_MAX_G + G * D + 3 * QE_MAX_SPLITS_CLUSTER * QE_MAX_G +
-                         2 * QE_MAX_G + kNW + 1) * 4 <= (size_t)kNW * kNST * STAGE,
+                         2 * QE_MAX_G + kNW + 1 + QE_MAX_SPLITS_CLUSTER) * 4 <=
+                    (size_t)kNW * nst_of(G) * stage_bytes<D>(),
                 "merge area");
-  auto kern = decode_kernel<T, D, G>;
+  auto kern = decode_kernel<T, D, G, W>;
   // One-time set-up per instantiation and device (kept out of the per-step path and of graph
-  // capture): clusters[wi][S] = how many clusters of S CTAs can be resident at once with the
-  // shared memory of window size 16 << wi.
+  // capture): clusters[S] = how many clusters of S CTAs can be resident at once.
   static QeOnce once;
-  static int clusters_of[QE_MAX_DEVICES][3][QE_MAX_SPLITS_CLUSTER + 1];
+  static int clusters_of[QE_MAX_DEVICES][QE_MAX_SPLITS_CLUSTER + 1];
   int dev = 0;
   const int se = qe_once_per_device(once, &dev, [&](int d) {
-    QE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_for(64)));
+    QE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     QE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
-    for (int wi = 0; wi < 3; ++wi)
-      for (int S = 1; S <= QE_MAX_SPLITS_CLUSTER; ++S) {
-        cudaLaunchConfig_t qc = {};
-        cudaLaunchAttribute qa[1];
-        qa[0].id = cudaLaunchAttributeClusterDimension;
-        qa[0].val.clusterDim.x = S;
-        qa[0].val.clusterDim.y = 1;
-        qa[0].val.clusterDim.z = 1;
-        qc.gridDim = dim3(S);
-        qc.blockDim = dim3(kNW * 32);
-        qc.dynamicSmemBytes = smem_for(16 << wi);
-        qc.attrs = qa;
-        qc.numAttrs = 1;
-        int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, kern, &qc) != cudaSuccess) {
-          (void)cudaGetLastError();
-          n = 0;
-        }
-        clusters_of[d][wi][S] = n;
+    for (int S = 1; S <= QE_MAX_SPLITS_CLUSTER; ++S) {
+      cudaLaunchConfig_t qc = {};
+      cudaLaunchAttribute qa[1];
+      qa[0].id = cudaLaunchAttributeClusterDimension;
+      qa[0].val.clusterDim.x = S;
+      qa[0].val.clusterDim.y = 1;
+      qa[0].val.clusterDim.z = 1;
+      qc.gridDim = dim3(S);
+      qc.blockDim = dim3(kNW * 32);
+      qc.dynamicSmemBytes = smem;
+      qc.attrs = qa;
+      qc.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &qc) != cudaSuccess) {
+        (void)cudaGetLastError();
+        n = 0;
       }
+      clusters_of[d][S] = n;
+    }
     return QE_OK;
   });
   if (se) return se;
-  const int wi = c->cfg.window == 16 ? 0 : (c->cfg.window == 32 ? 1 : 2);
-  const size_t smem = smem_for(c->cfg.window);
-  const int* clusters = clusters_of[dev][wi];
+  const int* clusters = clusters_of[dev];
   DecodeArgs a{};
   a.st = make_state(c);
   // the page pool as a 2-D tensor [units * P * 32 rows][D] for the swizzled TMA page loads
@@ -813,6 +904,8 @@ int launch_decode_t(qe_ctx* c, const void* q, float* out, cudaStream_t s, const 
   a.out = out;
   a.win_part = c->win_part;
   a.tail_s = c->tail_s;
+  a.nf = c->counts_exact ? c->n_full_max : -1;
+  a.nq = c->counts_exact ? c->n_int2_max : -1;
   a.tail_win = c->complete;
   a.tail_len = c->n - c->complete * c->cfg.window;
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
@@ -845,6 +938,16 @@ int launch_decode_t(qe_ctx* c, const void* q, float* out, cudaStream_t s, const 
   lc.numAttrs = 1;
   QE_CUDA_TRY(cudaLaunchKernelEx(&lc, kern, tmP, a));
   return QE_OK;
+}
+
+template <typename T, int D, int G>
+int launch_decode_t(qe_ctx* c, const void* q, float* out, cudaStream_t s, const void* k, const void* v) {
+  switch (c->cfg.window) {
+    case 16: return launch_decode_w<T, D, G, 16>(c, q, out, s, k, v);
+    case 32: return launch_decode_w<T, D, G, 32>(c, q, out, s, k, v);
+    case 64: return launch_decode_w<T, D, G, 64>(c, q, out, s, k, v);
+    default: return QE_ERR_UNSUPPORTED_SHAPE;
+  }
 }
 
 template <typename T, int D>

@@ -11,8 +11,14 @@
 //   KC [32 lanes][D/32 u32]  K codes, each lane's words in the order its mma.sync B fragments
 //                            take them (S = Q K^T, query heads as rows, tokens as columns)
 //   VC [32 lanes][D/32 u32]  V codes, in the order of the A fragments of O^T = V^T P^T
-//   KS [16 tokens][D/16]     fp16 K scales     KZ [16][D/16] fp16 K zeros
-//   VS [16 tokens][D/16]     fp16 V scales     VZ [D/16][16] fp16 V zeros (group-major)
+//   KS [D/16][16]            fp16 K scales, group-major, tokens in pair order (below)
+//   KZ [16 tokens][D/16]     fp16 K zeros, token-major
+//   VS [D/16][16]            fp16 V scales, group-major, fragment order
+//   VZ [D/16][16]            fp16 V zeros, group-major, fragment order
+// Pair order of a group's 16 tokens: position 2r + j holds token r + 8j, so one 4-byte load
+// gives lane (r, t) the scales of the two tokens of its score rows. Fragment order: position
+// 4t + j holds token 2t, 2t+1, 8+2t, 9+2t for j = 0..3, so one 8-byte load gives lane (r, t)
+// the pairs its P^T fragments need.
 //
 // Code placement. Word j of a lane holds the codes of groups 2j (bytes 0 and 2) and 2j+1
 // (bytes 1 and 3); within a 16-bit half, bits [2i, 2i+1] of each byte feed register i of the
@@ -37,6 +43,12 @@ struct Int2Block {
   static constexpr int VS = 12 * D;
   static constexpr int VZ = 14 * D;
   static constexpr int BYTES = 16 * D;
+
+  // position of token t (0..15) in the fragment order / pair order of a group-major array
+  static __host__ __device__ __forceinline__ int fpos(int t) {
+    return 4 * ((t & 7) >> 1) + (t & 1) + 2 * (t >> 3);
+  }
+  static __host__ __device__ __forceinline__ int ppos(int t) { return 2 * (t & 7) + (t >> 3); }
 
   // (lane, word, bit) of the K / V code of token t (0..15), element d (0..D-1)
   static __host__ __device__ __forceinline__ void kpos(int t, int d, int& lane, int& word, int& bit) {

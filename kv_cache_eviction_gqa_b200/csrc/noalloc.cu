@@ -12,9 +12,13 @@
 //
 // The array is a file-scope __device__ object of kStaticScratchBytes: every GPU that loads
 // this library holds that much memory until the process exits. All calls on one GPU share
-// it; every value a call reads from it was written earlier in the same call, so nothing needs
-// clearing, but two calls whose kernels overlap on the same GPU (for example two contexts on
-// two streams) race on it: issue them one after the other. A config whose scratch needs more
+// it, and it keeps whatever the last call left. Nothing needs clearing: a call folds a window
+// partial into the cumulative scores only if every CTA of the window's unit finished all its
+// waits, and each such partial was written earlier in the same call; when a bounded wait gives
+// up (QE_ERR_TIMEOUT in the status word) the step's score update is skipped for that unit, so
+// values left by another call are never read into the scores. Two calls whose kernels overlap
+// on the same GPU (for example two contexts on two streams) race on the array: issue them one
+// after the other. A config whose scratch needs more
 // than kStaticScratchBytes is rejected with QE_ERR_INVALID_ARG before anything is enqueued.
 // The first call on a device looks up the array's device address (cudaGetSymbolAddress with
 // that device current) and caches it; make that first call before any stream capture.

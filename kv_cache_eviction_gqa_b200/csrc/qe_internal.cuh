@@ -40,6 +40,9 @@ struct qe_ctx {
   int loaded;           // prefill done
   int n_full_max;       // upper bound of full-tier windows over units
   int n_int2_max;       // upper bound of INT2-tier windows over units
+  int counts_exact;     // every unit holds exactly n_full_max / n_int2_max windows (per-unit
+                        // routing keeps the units in step; host-given transitions and the
+                        // global budget do not)
   cudaStream_t last_stream;
   // scratch sub-buffers [dev]
   float* win_part;      // [U][max_windows][win_part_floats(D, G)]
@@ -119,12 +122,15 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+// One test of an mbarrier phase. The thread may be suspended in it until the phase completes
+// or about a millisecond has passed (the suspend-time hint), so a waiting warp takes no issue
+// slots from the others while its copy is in flight.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
       : "memory");
   return ok != 0;
 }

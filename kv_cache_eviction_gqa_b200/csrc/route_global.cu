@@ -279,6 +279,7 @@ extern "C" QE_API int qe_route_windows_global(qe_ctx* const* ctxs, int n_layers,
     const int tot = c->n_full_max + c->n_int2_max;
     c->n_full_max = tot < full_windows ? tot : full_windows;
     c->n_int2_max = tot < int2_windows ? tot : int2_windows;
+    c->counts_exact = 0;
     c->last_stream = st;
   }
   return QE_OK;

@@ -536,10 +536,10 @@ __global__ void __launch_bounds__(256) apply_kernel(DevState st, const int32_t* 
           uint16_t* kz = reinterpret_cast<uint16_t*>(img + BL::KZ);
           uint16_t* vs = reinterpret_cast<uint16_t*>(img + BL::VS);
           uint16_t* vz = reinterpret_cast<uint16_t*>(img + BL::VZ);
-          ks[r * BL::G8 + g] = static_cast<uint16_t>(mk & 0xffffu);
+          ks[g * QE_PAGE + BL::ppos(r)] = static_cast<uint16_t>(mk & 0xffffu);
           kz[r * BL::G8 + g] = static_cast<uint16_t>(mk >> 16);
-          vs[r * BL::G8 + g] = static_cast<uint16_t>(mv & 0xffffu);
-          vz[g * QE_PAGE + r] = static_cast<uint16_t>(mv >> 16);
+          vs[g * QE_PAGE + BL::fpos(r)] = static_cast<uint16_t>(mv & 0xffffu);
+          vz[g * QE_PAGE + BL::fpos(r)] = static_cast<uint16_t>(mv >> 16);
         }
       }
       __syncwarp();
@@ -576,8 +576,8 @@ __global__ void __launch_bounds__(256) apply_kernel(DevState st, const int32_t* 
       for (int r = 0; r < QE_PAGE; ++r) {
         const uint32_t bk = R::load_codes(natk + r * (D / 4), lane);
         const uint32_t bv = R::load_codes(natv + r * (D / 4), lane);
-        const float sk = meta_scale(ks[r * BL::G8 + g]), zk = meta_scale(kz[r * BL::G8 + g]);
-        const float sv = meta_scale(vs[r * BL::G8 + g]), zv = meta_scale(vz[g * QE_PAGE + r]);
+        const float sk = meta_scale(ks[g * QE_PAGE + BL::ppos(r)]), zk = meta_scale(kz[r * BL::G8 + g]);
+        const float sv = meta_scale(vs[g * QE_PAGE + BL::fpos(r)]), zv = meta_scale(vz[g * QE_PAGE + BL::fpos(r)]);
         float xk[DPL], xv[DPL];
 #pragma unroll
         for (int e = 0; e < DPL; ++e) {
@@ -630,8 +630,9 @@ __global__ void __launch_bounds__(128) ledger_read_kernel(DevState st, int u, in
     for (int i = lane; i < QE_PAGE * BL::G8; i += 32) {
       const int t = i / BL::G8, gg = i % BL::G8;
       const size_t o = ((size_t)bk * QE_PAGE + t) * BL::G8 + gg;
-      meta_k[o] = (uint32_t)ks[t * BL::G8 + gg] | ((uint32_t)kz[t * BL::G8 + gg] << 16);
-      meta_v[o] = (uint32_t)vs[t * BL::G8 + gg] | ((uint32_t)vz[gg * QE_PAGE + t] << 16);
+      const int fp = BL::fpos(t);
+      meta_k[o] = (uint32_t)ks[gg * QE_PAGE + BL::ppos(t)] | ((uint32_t)kz[t * BL::G8 + gg] << 16);
+      meta_v[o] = (uint32_t)vs[gg * QE_PAGE + fp] | ((uint32_t)vz[gg * QE_PAGE + fp] << 16);
     }
   }
 }

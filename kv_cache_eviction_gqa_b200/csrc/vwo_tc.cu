@@ -40,7 +40,7 @@ struct VwoArgs {
   int mpairs;           // ceil(rows / 256)
   int nsplit;           // N-tile ranges per (group, row block)
   int ntot;             // G * ntiles_per_head
-  int atomic;           // several CTAs add into one output element
+  int atomic;           // several CTAs add into one output element (never set: splits are whole heads)
   int32_t* status;
 };
 
@@ -209,14 +209,17 @@ int launch_tc(const void* V, int n_groups, int rows, const void* W, int Hq, int 
   a.mpairs = (rows + kMT * kBM - 1) / (kMT * kBM);
   a.ntot = a.G * a.ntiles_per_head;
   const long long items = (long long)n_groups * a.mpairs;
+  // Few row blocks: split the columns over several CTAs, at whole query heads only (a divisor
+  // of G), so that every output element is written by one CTA and results do not depend on
+  // the order in which CTAs finish.
+  int want = 1;
+  if (items < 2ll * sms) want = (int)((2ll * sms + items - 1) / items);
   int nsplit = 1;
-  if (items < 2ll * sms) nsplit = (int)((2ll * sms + items - 1) / items);
-  if (nsplit > a.ntot) nsplit = a.ntot;
+  for (int d = 1; d <= a.G; ++d)
+    if (a.G % d == 0 && d <= want) nsplit = d;
   a.nsplit = nsplit;
-  a.atomic = nsplit > 1;
+  a.atomic = 0;
   a.status = status;
-  if (a.atomic)
-    QE_CUDA_TRY(cudaMemset2DAsync(out, (size_t)ogs * 4, 0, (size_t)rows * a.G * 4, n_groups, s));
   kern<<<(unsigned)(items * nsplit), kThreads, SMEM, s>>>(tmV, tmW, a);
   return cudaGetLastError() == cudaSuccess ? QE_OK : QE_ERR_CUDA;
 }

@@ -172,9 +172,7 @@ def test_one_layer_one_kv_head_equals_per_unit_routing():
     """With one layer and one kv head per sequence the global candidates are exactly one unit's
     windows, so qe_route_windows_global must reproduce qe_route_windows tier for tier. Both
     contexts get the same prefill norms and no window completes during the run (the tail holds
-    one token at the start), so every score is bit-identical: the tensor-core norm GEMM adds
-    split pieces with float atomics, so two contexts computing their own norms agree to
-    rounding only."""
+    one token at the start), so every score is bit-identical."""
     from kv_cache_eviction_gqa_b200.binding import ContextShape, QEvictContext, route_windows_global, vwo_l1norm
     cfg = W.C2.scaled(name="one", B=3, Hkv=1, Hq=4, ctx=46 * 32 + 1, full_windows=7, int2_windows=12, steps=24,
                       hidden=512, seed=2500)
