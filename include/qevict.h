@@ -360,6 +360,18 @@ QE_API int qe_diag_tiers(const uint8_t* tiers, uint8_t* prev, uint8_t* flags, in
  * QE_ERR_UNSUPPORTED_SHAPE for D not in {64, 128}, G not in {1, 2, 4, 5, 8} or
  * B * Hkv * n_stride + 16 >= 2^31; QE_ERR_WORKSPACE for a small scratch. Asynchronous on `stream`;
  * allocates nothing. */
+/* qe_diag_summary - the pooled diagnostics of qe_diag_tiers' counters ("Resumo Técnico: QEvict",
+ * Principais Contribuições 1): sums over units of the six counters, churn = changed / live_prev
+ * and LIR = windows_reentered / windows_exited (NaN when the denominator is 0).
+ *   counters [dev, int64]: [units][6] as qe_diag_tiers keeps them. out [host]: filled.
+ * Synchronises `stream` (the counters are read back). QE_ERR_INVALID_ARG for a null pointer or
+ * units < 1; QE_ERR_CUDA when the copy fails. */
+typedef struct {
+  long long live_prev, changed, exits, reentries, windows_exited, windows_reentered;
+  double churn, lir;
+} qe_diag_stats;
+QE_API int qe_diag_summary(const long long* counters, int units, qe_diag_stats* out, qe_stream_t stream);
+
 QE_API size_t qe_diag_fmm_scratch_bytes(int units, int G);
 QE_API int qe_diag_fmm(const void* q, const void* K_ghost, long long n_stride, int n,
                        const uint8_t* tiers, int W, int window, int B, int Hq, int Hkv, int D,
@@ -397,6 +409,29 @@ QE_API int qe_sekv_build(const void* K, const void* V, const float* H, int B, in
 QE_API int qe_sekv_attend(const void* q, const void* K, const void* V, int B, int Hq, int Hkv, int n,
                           int D, int dtype, float theta, void* state, size_t state_bytes,
                           float* out, qe_stream_t stream);
+
+/* qe_state_bytes / qe_state_export / qe_state_import - checkpoint and restore of one context:
+ * the persistent state the pages describe ("Resumo Técnico: QEvict", Hierarquia Recuperável:
+ * the write-once INT2 ledger; Pontuação Cumulativa: the cumulative window scores), together with
+ * the page pool, page tables, tier map, tier lists and free stacks that give it meaning, and the
+ * host-side counters (tokens, decode steps, complete windows).
+ * Format: a 256-byte header (magic "QEVS", version, the qe_config, the host counters, the byte
+ * count that follows) and then the whole workspace verbatim (qe_layout.total bytes: the state
+ * arrays, and the scratch region, which also carries the V rows of the incomplete tail window
+ * that its norms are computed from when it completes).
+ *   qe_state_bytes: bytes of a checkpoint of this context (0 for a NULL context).
+ *   qe_state_export: dst [host or dev] of at least qe_state_bytes(ctx) bytes; asynchronous on
+ *     `stream` for device memory and pinned host memory (the caller keeps dst alive and reads it
+ *     after synchronising); the state copied is the one every earlier call on `stream` leaves.
+ *     QE_ERR_STATE before the prefill, QE_ERR_WORKSPACE for a small buffer.
+ *   qe_state_import: src [host or dev] of a checkpoint taken from a context with an equal
+ *     qe_config (and the same W_O, which is not part of the checkpoint). Reads the header
+ *     (synchronising `stream`), checks it, then copies the state into this context's workspace
+ *     on `stream` and restores the host counters. QE_ERR_INVALID_ARG for a bad magic, version or
+ *     config (nothing is changed then); QE_ERR_WORKSPACE for a small buffer. */
+QE_API size_t qe_state_bytes(const qe_ctx* ctx);
+QE_API int qe_state_export(qe_ctx* ctx, void* dst, size_t bytes, qe_stream_t stream);
+QE_API int qe_state_import(qe_ctx* ctx, const void* src, size_t bytes, qe_stream_t stream);
 
 /* qe_status - copy the device status word to the host (synchronises the context's last
  * stream) and return the first recorded error, or QE_OK. *detail (may be NULL) receives the

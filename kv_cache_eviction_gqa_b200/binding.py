@@ -31,6 +31,11 @@ class QeConfig(C.Structure):
                                         "slots_per_unit", "max_splits")]
 
 
+class QeDiagStats(C.Structure):
+    _fields_ = [(n, C.c_longlong) for n in ("live_prev", "changed", "exits", "reentries", "windows_exited",
+                                            "windows_reentered")] + [("churn", C.c_double), ("lir", C.c_double)]
+
+
 class QeLayout(C.Structure):
     _fields_ = [(n, C.c_size_t) for n in ("total", "pages", "page_free", "win_pages", "win_tier",
                                            "win_slot", "slots", "slot_free", "mass", "pert", "norms",
@@ -79,6 +84,10 @@ def lib():
             "qe_diag_fmm_scratch_bytes": (sz, [i, i]),
             "qe_diag_fmm": (i, [vp, vp, ll, i, vp, i, i, i, i, i, i, i, vp, vp, sz, vp]),
             "qe_ledger_read": (i, [vp, i, i, vp, vp, vp, vp, vp, vp]),
+            "qe_state_bytes": (sz, [vp]),
+            "qe_state_export": (i, [vp, vp, sz, vp]),
+            "qe_state_import": (i, [vp, vp, sz, vp]),
+            "qe_diag_summary": (i, [vp, i, C.POINTER(QeDiagStats), vp]),
             "qe_status": (i, [vp, C.POINTER(C.c_int)]),
             "qe_step_index": (i, [vp]),
             "qe_length": (i, [vp]),
@@ -270,6 +279,25 @@ class QEvictContext:
             "route_stats": self._view(L.route_stats, U * 8, torch.int32, (U, 8)),
         }
 
+    def state_bytes(self) -> int:
+        return int(lib().qe_state_bytes(self._h))
+
+    def export_state(self, dst: torch.Tensor = None, stream=None) -> torch.Tensor:
+        """Checkpoint of the context (qe_state_export) into a uint8 tensor (host or device)."""
+        n = self.state_bytes()
+        if dst is None:
+            dst = torch.empty(n, dtype=torch.uint8, device=self.workspace.device)
+        if dst.dtype != torch.uint8 or not dst.is_contiguous() or dst.numel() < n:
+            raise ValueError(f"dst must be a contiguous uint8 tensor of at least {n} bytes")
+        _check(lib().qe_state_export(self._h, _ptr(dst), n, _stream(stream)), "qe_state_export")
+        return dst
+
+    def import_state(self, src: torch.Tensor, stream=None):
+        """Restore a checkpoint taken from a context of the same configuration (qe_state_import)."""
+        if src.dtype != torch.uint8 or not src.is_contiguous():
+            raise ValueError("src must be a contiguous uint8 tensor")
+        _check(lib().qe_state_import(self._h, _ptr(src), src.numel(), _stream(stream)), "qe_state_import")
+
     def ledger_entry(self, unit: int, win: int, stream=None):
         """One window's INT2 ledger entry as (codes_K, s_K, z_K, codes_V, s_V, z_V) NumPy arrays
         (codes [window][D] in 0..3, scales and zeros [window][D/16] float16), read through
@@ -435,14 +463,13 @@ class TierDiagnostics:
                "qe_diag_tiers")
         self.events += 1
 
-    def summary(self) -> dict:
-        """Pooled counts and the two ratios (nan when a denominator is 0); synchronises."""
-        c = self.counters.sum(dim=0).cpu().tolist()
-        keys = ("live_prev", "changed", "exits", "reentries", "windows_exited", "windows_reentered")
-        out = dict(zip(keys, c))
-        out["churn"] = c[1] / c[0] if c[0] else float("nan")
-        out["lir"] = c[5] / c[4] if c[4] else float("nan")
-        return out
+    def summary(self, stream=None) -> dict:
+        """Pooled counts and the two ratios (nan when a denominator is 0), from qe_diag_summary;
+        synchronises."""
+        st = QeDiagStats()
+        _check(lib().qe_diag_summary(_ptr(self.counters), self.units, C.byref(st), _stream(stream)),
+               "qe_diag_summary")
+        return {name: getattr(st, name) for name, _ in QeDiagStats._fields_}
 
 
 def diag_fmm_scratch_bytes(units: int, G: int) -> int:

@@ -302,6 +302,69 @@ QE_API int qe_ledger_read(qe_ctx* c, int unit, int win, uint8_t* codes_k, uint32
   return launch_ledger_read(c, unit, win, codes_k, meta_k, codes_v, meta_v, found, (cudaStream_t)s);
 }
 
+// ---- checkpoint of a context ----
+namespace {
+struct StateHeader {  // 256 bytes, little endian as the host
+  char magic[4];      // "QEVS"
+  int32_t version;    // 1
+  qe_config cfg;
+  int32_t n, step, complete, n_full_max, n_int2_max, counts_exact;
+  uint64_t state_bytes;  // bytes of workspace that follow the header (all of it)
+};
+constexpr size_t kHeaderBytes = 256;
+static_assert(sizeof(StateHeader) <= kHeaderBytes, "state header");
+constexpr int32_t kStateVersion = 1;
+bool same_config(const qe_config& a, const qe_config& b) { return memcmp(&a, &b, sizeof(qe_config)) == 0; }
+}  // namespace
+
+QE_API size_t qe_state_bytes(const qe_ctx* c) { return c ? kHeaderBytes + c->lay.total : 0; }
+
+QE_API int qe_state_export(qe_ctx* c, void* dst, size_t bytes, qe_stream_t s) {
+  if (!c || !dst) return QE_ERR_INVALID_ARG;
+  if (!c->loaded) return QE_ERR_STATE;
+  if (bytes < qe_state_bytes(c)) return QE_ERR_WORKSPACE;
+  StateHeader h;
+  memset(&h, 0, sizeof(h));
+  memcpy(h.magic, "QEVS", 4);
+  h.version = kStateVersion;
+  h.cfg = c->cfg;
+  h.n = c->n;
+  h.step = c->step;
+  h.complete = c->complete;
+  h.n_full_max = c->n_full_max;
+  h.n_int2_max = c->n_int2_max;
+  h.counts_exact = c->counts_exact;
+  h.state_bytes = c->lay.total;
+  cudaStream_t st = (cudaStream_t)s;
+  // the header from pageable host memory: the copy consumes it before returning
+  QE_CUDA_TRY(cudaMemcpyAsync(dst, &h, sizeof(h), cudaMemcpyDefault, st));
+  QE_CUDA_TRY(cudaMemcpyAsync((uint8_t*)dst + kHeaderBytes, c->ws, c->lay.total, cudaMemcpyDefault, st));
+  c->last_stream = st;
+  return QE_OK;
+}
+
+QE_API int qe_state_import(qe_ctx* c, const void* src, size_t bytes, qe_stream_t s) {
+  if (!c || !src) return QE_ERR_INVALID_ARG;
+  if (bytes < kHeaderBytes) return QE_ERR_WORKSPACE;
+  cudaStream_t st = (cudaStream_t)s;
+  StateHeader h;
+  QE_CUDA_TRY(cudaMemcpyAsync(&h, src, sizeof(h), cudaMemcpyDefault, st));
+  QE_CUDA_TRY(cudaStreamSynchronize(st));
+  if (memcmp(h.magic, "QEVS", 4) != 0 || h.version != kStateVersion) return QE_ERR_INVALID_ARG;
+  if (!same_config(h.cfg, c->cfg) || h.state_bytes != c->lay.total) return QE_ERR_INVALID_ARG;
+  if (bytes < kHeaderBytes + h.state_bytes) return QE_ERR_WORKSPACE;
+  QE_CUDA_TRY(cudaMemcpyAsync(c->ws, (const uint8_t*)src + kHeaderBytes, h.state_bytes, cudaMemcpyDefault, st));
+  c->n = h.n;
+  c->step = h.step;
+  c->complete = h.complete;
+  c->n_full_max = h.n_full_max;
+  c->n_int2_max = h.n_int2_max;
+  c->counts_exact = h.counts_exact;
+  c->loaded = 1;
+  c->last_stream = st;
+  return QE_OK;
+}
+
 QE_API int qe_status(qe_ctx* c, int* detail) {
   if (!c) return QE_ERR_INVALID_ARG;
   int32_t h[4] = {0, 0, 0, 0};

@@ -23,6 +23,8 @@
 
 #include <type_traits>
 
+#include <stdlib.h>
+
 #include "qe_internal.cuh"
 #include "tc_common.cuh"
 #include "warp_mma.cuh"
@@ -355,6 +357,33 @@ extern "C" QE_API int qe_diag_tiers(const uint8_t* tiers, uint8_t* prev, uint8_t
   tier_diag_kernel<<<units, kTierThreads, 0, (cudaStream_t)stream>>>(tiers, prev, flags, W, first ? 1 : 0,
                                                                     counters);
   return cudaGetLastError() == cudaSuccess ? QE_OK : QE_ERR_CUDA;
+}
+
+extern "C" QE_API int qe_diag_summary(const long long* counters, int units, qe_diag_stats* out,
+                                      qe_stream_t s) {
+  if (!counters || !out || units < 1) return QE_ERR_INVALID_ARG;
+  long long* h = (long long*)malloc(sizeof(long long) * 6 * (size_t)units);
+  if (!h) return QE_ERR_INVALID_ARG;
+  const bool okc = cudaMemcpyAsync(h, counters, sizeof(long long) * 6 * (size_t)units, cudaMemcpyDeviceToHost,
+                                   (cudaStream_t)s) == cudaSuccess &&
+                   cudaStreamSynchronize((cudaStream_t)s) == cudaSuccess;
+  if (!okc) {
+    free(h);
+    return QE_ERR_CUDA;
+  }
+  long long sum[6] = {0, 0, 0, 0, 0, 0};
+  for (int u = 0; u < units; ++u)
+    for (int i = 0; i < 6; ++i) sum[i] += h[(size_t)u * 6 + i];
+  free(h);
+  out->live_prev = sum[0];
+  out->changed = sum[1];
+  out->exits = sum[2];
+  out->reentries = sum[3];
+  out->windows_exited = sum[4];
+  out->windows_reentered = sum[5];
+  out->churn = sum[0] ? (double)sum[1] / (double)sum[0] : NAN;
+  out->lir = sum[4] ? (double)sum[5] / (double)sum[4] : NAN;
+  return QE_OK;
 }
 
 extern "C" QE_API size_t qe_diag_fmm_scratch_bytes(int units, int G) {

@@ -86,8 +86,13 @@ def _near_tie(unit: O.QEvictUnit, w: int) -> bool:
 
 
 def run_decode_parity(cfg: W.DecodeConfig, check_units=None, steps=None, max_splits=32,
-                      check_every=1, verbose=False, diag=False) -> ParityReport:
+                      check_every=1, verbose=False, diag=False, fused=False) -> ParityReport:
     """Decode sequence on the GPU and in the oracle, compared step by step.
+
+    With fused=True every step is one qe_decode_step call (the step's append inside the decode
+    launch, routing on s % R == 0 in the same call): the call the bench times. The routing
+    checks then take the candidates and the tiers before the event from the oracle's unit
+    (the two sides' tiers agree before every event, which the previous event's checks assert).
 
     With diag=True the QEvict diagnostics ride along: after every routing event the context's
     tier map goes to qe_diag_tiers (the oracle's own tier history to tier_diagnostics, counts
@@ -135,8 +140,12 @@ def run_decode_parity(cfg: W.DecodeConfig, check_units=None, steps=None, max_spl
         k = torch.from_numpy(inp.k_new[s]).to(dev, tdt)
         v = torch.from_numpy(inp.v_new[s]).to(dev, tdt)
         # scores before routing, for the selection-property check
-        ctx.kv_append(k, v)
-        out = ctx.decode_attend_and_score(q)
+        routing = s % cfg.route_every == 0
+        if fused:
+            out = ctx.decode_step(q, k, v)
+        else:
+            ctx.kv_append(k, v)
+            out = ctx.decode_attend_and_score(q)
         if diag:
             ghost[:, :, cfg.ctx + s] = k
             fmm_g, fscr = diag_fmm(q, ghost, cfg.ctx + s + 1, st["win_tier"], cfg.window)
@@ -144,11 +153,10 @@ def run_decode_parity(cfg: W.DecodeConfig, check_units=None, steps=None, max_spl
         if diag:
             assert trim_status(fscr) == (0, 0)
             fmm_g = fmm_g.cpu().numpy()
-        routing = s % cfg.route_every == 0
         g_mass = st["mass"].cpu().numpy().copy()
         g_pert = st["pert"].cpu().numpy().copy()
         g_tier_before = st["win_tier"].cpu().numpy().copy()
-        if routing:
+        if routing and not fused:
             ctx.route_windows()
         torch.cuda.synchronize()
         rc, det = ctx.status()
@@ -185,6 +193,11 @@ def run_decode_parity(cfg: W.DecodeConfig, check_units=None, steps=None, max_spl
                         f"at window {lp[rp.argmax()]}"
             if routing:
                 rep.route_events += 1
+                if fused:
+                    # tiers before the event, as the oracle holds them (routing already ran on the GPU)
+                    tb = np.where(unit.tier == O.FULL, TIER_FULL, np.where(unit.tier == O.INT2, TIER_INT2,
+                                  np.where(unit.tier == O.TAIL, TIER_TAIL, TIER_EVICTED)))
+                    g_tier_before[u, :tb.size] = tb
                 cands = np.nonzero((g_tier_before[u] == TIER_FULL) | (g_tier_before[u] == TIER_INT2))[0]
                 # property: the GPU decision is the two-stage selection of its own scores
                 full_g = _select_two_stage(cands, g_mass[u].astype(np.float64),

@@ -104,3 +104,23 @@ def test_sekv_host_side_sizes_and_errors(libpath):
     assert L.qe_sekv_build(None, None, None, 1, 4, 1, 16, 128, B.QE_BF16, 1.0, None, 0, None) == B.QE_ERR_INVALID_ARG
     assert L.qe_sekv_attend(None, None, None, 1, 4, 1, 16, 128, B.QE_BF16, 1.0, None, 0, None,
                             None) == B.QE_ERR_INVALID_ARG
+
+
+def test_state_checkpoint_host_checks():
+    """qe_state_bytes is the header plus the whole workspace; export before a prefill is out of
+    order and touches nothing (stand-in device addresses)."""
+    import ctypes as C
+    from kv_cache_eviction_gqa_b200 import binding as Bd
+    assert Bd.lib().qe_state_bytes(None) == 0
+    cfg = Bd.QeConfig(2, 8, 2, 64, Bd.QE_FP16, 16, 16, 8, 8, 0.5, 4, 512, 2048, 2048 // 16 + 4, 16, 16)
+    lay = Bd.QeLayout()
+    assert Bd.lib().qe_plan(C.byref(cfg), C.byref(lay)) == 0
+    h = C.c_void_p()
+    fake = C.c_void_p(1 << 40)
+    assert Bd.lib().qe_create(C.byref(cfg), fake, C.c_size_t(lay.total), fake, C.byref(h)) == 0
+    try:
+        n = Bd.lib().qe_state_bytes(h)
+        assert n == 256 + lay.total
+        assert Bd.lib().qe_state_export(h, fake, C.c_size_t(n), None) == Bd.QE_ERR_STATE
+    finally:
+        Bd.lib().qe_destroy(h)

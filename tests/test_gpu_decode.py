@@ -40,21 +40,26 @@ def test_small_sequences(cfg):
     print(rep)
 
 
-# full sizes, in the launch configuration the bench uses; the oracle follows sampled units
+# full sizes, through the call and launch configuration the bench times (qe_decode_step: the
+# append inside the decode launch, routing in the same call); the oracle follows sampled units
 @pytest.mark.slow
 def test_c2_full_size_sampled_units():
     cfg = W.C2
     units = [0, cfg.units - 1]
-    rep = run_decode_parity(cfg, check_units=units)
+    rep = run_decode_parity(cfg, check_units=units, fused=True)
     assert rep.steps == cfg.steps and rep.route_events == 4 * len(units) and rep.codes_checked > 0
     print(rep)
 
 
 @pytest.mark.slow
-def test_c5_full_size_sampled_unit():
+def test_c5_full_size_sampled_units():
+    """All 256 drift steps of the long-context stress (16 routing events, 8 focus rotations that
+    force repeated promotions and demotions through the write-once ledger) on two kv heads."""
     cfg = W.C5
-    rep = run_decode_parity(cfg, check_units=[3], steps=80)
-    assert rep.steps == 80 and rep.route_events == 5 and rep.codes_checked > 0
+    units = [3, 6]
+    rep = run_decode_parity(cfg, check_units=units, fused=True)
+    assert rep.steps == cfg.steps == 256 and rep.route_events == 16 * len(units)
+    assert rep.codes_checked > 0 and rep.promoted_checked > 0
     print(rep)
 
 
