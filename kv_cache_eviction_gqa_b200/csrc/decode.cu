@@ -156,6 +156,20 @@ __device__ __forceinline__ uint32_t __hmul2_u32(uint32_t a, uint32_t b) {
   asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
   return r;
 }
+// fp16 pair a * b + c, one rounding
+__device__ __forceinline__ uint32_t __hfma2_u32(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t r;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+// The weight-times-scale product w s of a pair, where w = wh + wl (fp16 high and low parts), as
+// an unevaluated fp16 sum hi + lo: hi = fl(wh s); lo = fl(fl(wh s - hi) + wl s), where wh s - hi
+// (the rounding error of a product) is exact in fp16 barring underflow, so hi + lo carries
+// w s to about 2^-20 relative, where the single product wh s (dropping wl) is off by up to 2^-10.
+__device__ __forceinline__ void ws_split(uint32_t wh, uint32_t wl, uint32_t sc, uint32_t& hi, uint32_t& lo) {
+  hi = __hmul2_u32(wh, sc);
+  lo = __hfma2_u32(wl, sc, __hfma2_u32(wh, sc, hi ^ 0x80008000u));
+}
 
 // Register i (0..3) of a packed code word: the codes at bits [2i, 2i+1] of each 16-bit half as
 // the fp16 subnormals c * 4^i * 2^-24.
@@ -180,6 +194,7 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
   extern __shared__ __align__(128) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const DevState& st = a.st;
+  if (threadIdx.x == 0) asm volatile("prefetch.tensormap [%0];" ::"l"(&tmP) : "memory");
   const int u = blockIdx.x / a.splits, split = blockIdx.x % a.splits;
   const int b = u / st.Hkv, kvh = u % st.Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -209,27 +224,57 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
   }
   __syncwarp();
 
-  // virtual index j of this split: [0, nF) full, nF the tail (when present), then INT2.
-  // This warp's windows are j = warp + kNW * o, o < n_own (kinds in that order); each window is
-  // a run of tasks i: full and tail windows K, V of every page; INT2 windows their chunks.
-  const int n_own = nJ > warp ? (nJ - warp + kNW - 1) / kNW : 0;
-  auto kind_of = [&](int j) { return j < nF ? 0 : (j < nF + has_tail ? 2 : 1); };  // full, int2, tail
-  auto list_idx = [&](int j) { return j < nF ? f0 + j : nf + q0 + (j - nF - has_tail); };
+  // Windows of this split in the order [tail (when present) | full | INT2]; warp w takes
+  // windows j = w + kNW * o' (each window a run of tasks: full and tail windows K, V of every
+  // page; INT2 windows their chunks). Even warps walk their windows in that order, odd warps
+  // start with their INT2 windows (o' = o + their number of tail and full windows, mod n_own),
+  // so that at any time some warps of the SM stream full-precision pages while others do the
+  // INT2 tier's dequantising arithmetic, and warp 0 starts with the tail and its append.
+  auto kind_of = [&](int j) { return j < has_tail ? 2 : (j < has_tail + nF ? 0 : 1); };  // full 0, INT2 1, tail 2
+  // position in the full list, or nf + position in the INT2 list (the window-partial slot)
+  auto list_idx = [&](int j) {
+    const int v = j - has_tail;
+    return v < nF ? f0 + v : nf + q0 + (v - nF);
+  };
   auto n_sub = [&](int kind) { return kind == 0 ? 2 * PPW : (kind == 1 ? CPW : 2 * tail_pages); };
+  const int n_own = nJ > warp ? (nJ - warp + kNW - 1) / kNW : 0;
+  const int n_ft = has_tail + nF;
+  const int rot = (warp & 1) && n_ft > warp ? (n_ft - warp + kNW - 1) / kNW : 0;
+  auto j_of = [&](int o) {
+    int oo = o + rot;
+    if (oo >= n_own) oo -= n_own;
+    return warp + kNW * oo;
+  };
+  struct Cursor {
+    int o, i;  // window ordinal of this warp, task within the window
+  };
+  auto cur_kind = [&](const Cursor& c) { return kind_of(j_of(c.o)); };
+  auto cur_set = [&](Cursor& c, int o) {
+    c.o = o;
+    c.i = 0;
+  };
+  // next task; a new window when the current one is done
+  auto cur_next = [&](Cursor& c) {
+    if (++c.i >= n_sub(cur_kind(c))) {
+      c.i = 0;
+      ++c.o;
+    }
+  };
+  auto cur_list_idx = [&](const Cursor& c) { return list_idx(j_of(c.o)); };
   // Index prefetch: lane l holds the window id and the page ids (full, tail) or the ledger
   // slot (INT2) of this warp's window of ordinal rb + l, so issuing a copy never waits on a
   // dependent global load. Reloaded every 32 windows.
   int e_win = -1, e_id[PPW], rb = -32;
   auto load_ids = [&](int base) {
     rb = base;
-    const int jj = base + lane < n_own ? warp + kNW * (base + lane) : nJ;
+    const int jj = base + lane < n_own ? j_of(base + lane) : nJ;
     e_win = -1;
 #pragma unroll
     for (int p = 0; p < PPW; ++p) e_id[p] = -1;
     if (jj < nJ) {
       const int kd = kind_of(jj);
-      const int win = kd == 0 ? st.full_list[ub + f0 + jj]
-                              : (kd == 1 ? st.int2_list[ub + q0 + (jj - nF - has_tail)] : a.tail_win);
+      const int li = kd == 2 ? 0 : list_idx(jj);
+      const int win = kd == 0 ? st.full_list[ub + li] : (kd == 1 ? st.int2_list[ub + li - nf] : a.tail_win);
       if (win >= 0 && win < st.Wmax) {
         e_win = win;
         if (kd == 1) {
@@ -244,11 +289,10 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
   // fused append: page of the step's token (written by this warp just before the tail's copies)
   int app_pg = -1, app_page = -1;
   // issue the copies of task (window ordinal r, task i) into stage s (all lanes call)
-  auto issue = [&](int r, int i, int s) {
-    const int j = warp + kNW * r;
+  auto issue = [&](const Cursor& c, int s) {
+    const int r = c.o, i = c.i, k = cur_kind(c);
     if (r - rb >= 32) load_ids(r - r % 32);
     const int src = r - rb;
-    const int k = kind_of(j);
     const int pg = k == 1 ? 0 : (i >> 1);
     int sel = e_id[0];
 #pragma unroll
@@ -418,26 +462,22 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
     return y;
   };
 
-  int o = 0, ti = 0;                  // window ordinal and task being computed
-  int io = 0, ii = 0, issued = 0;     // next task to copy
-  auto advance = [&](int& r, int& i) {
-    if (++i >= n_sub(kind_of(warp + kNW * r))) {
-      i = 0;
-      ++r;
-    }
-  };
-  for (int s = 0; s < NST - 1 && io < n_own; ++s) {
-    issue(io, ii, s);
-    advance(io, ii);
+  Cursor cc, ci;  // the task being computed, the next task to copy
+  cur_set(cc, 0);
+  cur_set(ci, 0);
+  int issued = 0;
+  for (int s = 0; s < NST - 1 && ci.o < n_own; ++s) {
+    issue(ci, s);
+    cur_next(ci);
     ++issued;
   }
   int k = 0;
   bool ok = true;
   // wait for the task computed next, after issuing the one NST - 1 ahead
   auto next_stage = [&]() -> int {
-    if (io < n_own) {
-      issue(io, ii, issued % NST);
-      advance(io, ii);
+    if (ci.o < n_own) {
+      issue(ci, issued % NST);
+      cur_next(ci);
       ++issued;
     }
     const int s = k % NST;
@@ -458,16 +498,58 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
     }
   }
 
-  // ---- phase 1: full-precision windows, then the tail: K task (scores, softmax), V task ----
-  {
-    uint32_t ph0 = 0, pl0 = 0, ph1 = 0, pl1 = 0;  // P^T of the last K task, for its V task
-    int valid = QE_PAGE;
-    while (o < n_own && kind_of(warp + kNW * o) != 1) {
-      const int s = next_stage();
-      if (!ok) break;
+  // INT2 operands, computed once:
+  // q as fp16 with the elements 8 + 2t4, 9 + 2t4 of each group quartered (their codes carry
+  // 4x), and head g8's sum of q over groups 2t4, 2t4 + 1 in the log2 domain, split hi + lo
+  // (the B operand of the zero-point product Z Q_g)
+  uint32_t qh[G8][2];
+  float qg0 = 0.f, qg1 = 0.f;
+#pragma unroll
+  for (int m = 0; m < G8; ++m) {
+    const float x0 = Elem<T>::lo(qb[m][0]), x1 = Elem<T>::hi(qb[m][0]);
+    const float x2 = Elem<T>::lo(qb[m][1]), x3 = Elem<T>::hi(qb[m][1]);
+    qh[m][0] = pack_h2(x0, x1);
+    qh[m][1] = pack_h2(0.25f * x2, 0.25f * x3);
+    float t = (x0 + x1) + (x2 + x3);
+    t += __shfl_xor_sync(0xffffffffu, t, 1);
+    t += __shfl_xor_sync(0xffffffffu, t, 2);
+    if (m == 2 * t4) qg0 = t * sl;
+    if (m == 2 * t4 + 1) qg1 = t * sl;
+  }
+  const uint32_t qgh = pack_h2(qg0, qg1);
+  const uint32_t qgl = pack_h2(qg0 - h_lo(qgh), qg1 - h_hi(qgh));
+  // selection matrix that deals a token's K scale to both head columns: row 0 picks all
+  const uint32_t sel0 = t4 == 0 ? 0x3c00u : 0u;
+  const float2 fa = make_float2(0x1p24f * sl, 0x1p24f * sl), fb = make_float2(0x1p20f * sl, 0x1p20f * sl);
+  constexpr uint32_t kQuarter2 = 0x34003400u;  // fp16 pair {0.25, 0.25}
+
+  // The accumulators hold O^T while full-precision and tail pages are streamed, and O^T * 2^-24
+  // in rows g8 / O^T * 2^-20 in rows 8 + g8 (the scale of the subnormal code operands) while INT2
+  // chunks are; they are rescaled at every switch (the zero-point part stays unscaled in zacc).
+  auto to_units = [&](bool int2) {
+    const float lo = int2 ? 0x1p-24f : 0x1p24f, hi = int2 ? 0x1p-20f : 0x1p20f;
+#pragma unroll
+    for (int m = 0; m < G8; ++m) {
+      oacc[m][0] *= lo;
+      oacc[m][1] *= lo;
+      oacc[m][2] *= hi;
+      oacc[m][3] *= hi;
+    }
+  };
+  bool int2_units = false;
+  uint32_t ph0 = 0, pl0 = 0, ph1 = 0, pl1 = 0;  // P^T of the last K task, for its V task
+  int valid = QE_PAGE;
+  while (cc.o < n_own) {
+    const int s = next_stage();
+    if (!ok) break;
+    const int kd = cur_kind(cc), ti = cc.i;
+    if ((kd == 1) != int2_units) {
+      int2_units = kd == 1;
+      to_units(int2_units);
+    }
+    if (kd != 1) {
       uint8_t* stage = ring + s * STAGE;
-      const int j = warp + kNW * o;
-      const bool tail = kind_of(j) == 2;
+      const bool tail = kd == 2;
       if ((ti & 1) == 0) {
         // K rows: S^T = K Q^T over 16 tokens, two independent chains
         valid = tail ? min(QE_PAGE, a.tail_len - (ti >> 1) * QE_PAGE) : QE_PAGE;
@@ -521,52 +603,9 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
           MmaOp<T>::run(oacc[m], va[0], va[1], va[2], va[3], ph0, ph1);
           MmaOp<T>::run(oacc[m], va[0], va[1], va[2], va[3], pl0, pl1);
         }
-        if (!tail && ti == 2 * PPW - 1) window_end(list_idx(j));
+        if (!tail && ti == 2 * PPW - 1) window_end(cur_list_idx(cc));
       }
-      __syncwarp();
-      advance(o, ti);
-      ++k;
-    }
-  }
-
-  // ---- phase 2: INT2 ledger entries ----
-  // From here on the accumulators hold O^T * 2^-24 in rows g8 and O^T * 2^-20 in rows 8 + g8
-  // (the scale of the subnormal code operands); the zero-point part stays unscaled in zacc.
-#pragma unroll
-  for (int m = 0; m < G8; ++m) {
-    oacc[m][0] *= 0x1p-24f;
-    oacc[m][1] *= 0x1p-24f;
-    oacc[m][2] *= 0x1p-20f;
-    oacc[m][3] *= 0x1p-20f;
-  }
-  if (ok && o < n_own) {
-    // q as fp16 with the elements 8 + 2t4, 9 + 2t4 of each group quartered (their codes carry
-    // 4x), and head g8's sum of q over groups 2t4, 2t4 + 1 in the log2 domain, split hi + lo
-    // (the B operand of the zero-point product Z Q_g)
-    uint32_t qh[G8][2];
-    float qg0 = 0.f, qg1 = 0.f;
-#pragma unroll
-    for (int m = 0; m < G8; ++m) {
-      const float x0 = Elem<T>::lo(qb[m][0]), x1 = Elem<T>::hi(qb[m][0]);
-      const float x2 = Elem<T>::lo(qb[m][1]), x3 = Elem<T>::hi(qb[m][1]);
-      qh[m][0] = pack_h2(x0, x1);
-      qh[m][1] = pack_h2(0.25f * x2, 0.25f * x3);
-      float t = (x0 + x1) + (x2 + x3);
-      t += __shfl_xor_sync(0xffffffffu, t, 1);
-      t += __shfl_xor_sync(0xffffffffu, t, 2);
-      if (m == 2 * t4) qg0 = t * sl;
-      if (m == 2 * t4 + 1) qg1 = t * sl;
-    }
-    const uint32_t qgh = pack_h2(qg0, qg1);
-    const uint32_t qgl = pack_h2(qg0 - h_lo(qgh), qg1 - h_hi(qgh));
-    // selection matrix that deals a token's K scale to both head columns: row 0 picks all
-    const uint32_t sel0 = t4 == 0 ? 0x3c00u : 0u;
-    const float2 fa = make_float2(0x1p24f * sl, 0x1p24f * sl), fb = make_float2(0x1p20f * sl, 0x1p20f * sl);
-    constexpr uint32_t kQuarter2 = 0x34003400u;  // fp16 pair {0.25, 0.25}
-
-    while (o < n_own) {
-      const int s = next_stage();
-      if (!ok) break;
+    } else {
       const uint8_t* stage = ring + s * STAGE;
       float sc[4 * BPC], p[4 * BPC];
 #pragma unroll
@@ -631,7 +670,7 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
           mma_h16(zacc, zg.x, 0u, zg.y, 0u, pl0, pl1);
         }
         // the codes of tokens 8..15 carry 4x: their weights are quartered (exact)
-        const uint32_t pq1 = __hmul2_u32(ph1, kQuarter2);
+        const uint32_t pq1 = __hmul2_u32(ph1, kQuarter2), pql1 = __hmul2_u32(pl1, kQuarter2);
         uint32_t vw[WPL];
         if constexpr (WPL == 4) {
           const uint4 v4 = *reinterpret_cast<const uint4*>(blk + BL::VC + lane * 16);
@@ -647,29 +686,34 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
             const int m = 2 * jj + e;
             const uint32_t x = e ? (vw[jj] >> 8) : vw[jj];
             const uint2 sg = *reinterpret_cast<const uint2*>(blk + BL::VS + (m * QE_PAGE + 4 * t4) * 2);
-            mma_h16(oacc[m], code_reg<0>(x), code_reg<2>(x), code_reg<1>(x), code_reg<3>(x),
-                    __hmul2_u32(ph0, sg.x), __hmul2_u32(pq1, sg.y));
+            uint32_t h0, l0, h1, l1;
+            ws_split(ph0, pl0, sg.x, h0, l0);
+            ws_split(pq1, pql1, sg.y, h1, l1);
+            const uint32_t c0 = code_reg<0>(x), c1 = code_reg<1>(x), c2 = code_reg<2>(x), c3 = code_reg<3>(x);
+            mma_h16(oacc[m], c0, c2, c1, c3, h0, h1);
+            mma_h16(oacc[m], c0, c2, c1, c3, l0, l1);
           }
         }
       }
-      __syncwarp();
-      if (ti == CPW - 1) window_end(list_idx(warp + kNW * o));
-      advance(o, ti);
-      ++k;
+      if (ti == CPW - 1) window_end(cur_list_idx(cc));
     }
+    __syncwarp();
+    cur_next(cc);
+    ++k;
   }
+  if (int2_units) to_units(false);
   if (!ok) {  // drain copies still in flight if a wait gave up
     for (; k < issued; ++k) mbar_wait_bounded(&bars[k % NST], (k / NST) & 1, st.status, 2000 + u);
   }
-  // back to O^T: undo the code scales and add the zero-point part of each element's group
+  // add the zero-point part of each element's group
 #pragma unroll
   for (int m = 0; m < G8; ++m) {
     const float z0 = __shfl_sync(0xffffffffu, zacc[0], 4 * m + t4);
     const float z1 = __shfl_sync(0xffffffffu, zacc[1], 4 * m + t4);
-    oacc[m][0] = fmaf(oacc[m][0], 0x1p24f, z0);
-    oacc[m][1] = fmaf(oacc[m][1], 0x1p24f, z1);
-    oacc[m][2] = fmaf(oacc[m][2], 0x1p20f, z0);
-    oacc[m][3] = fmaf(oacc[m][3], 0x1p20f, z1);
+    oacc[m][0] += z0;
+    oacc[m][1] += z1;
+    oacc[m][2] += z0;
+    oacc[m][3] += z1;
   }
 #pragma unroll
   for (int o2 = 4; o2 < 32; o2 <<= 1) {
@@ -689,7 +733,7 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
     const int jj = threadIdx.x + x * kNW * 32;
     pw_win[x] = -1;
     if (jj < nF + nQ) {
-      const int li = list_idx(jj < nF ? jj : jj + has_tail);
+      const int li = jj < nF ? f0 + jj : nf + q0 + (jj - nF);
       const int win = jj < nF ? st.full_list[ub + li] : st.int2_list[ub + li - nf];
       if (win >= 0 && win < st.Wmax) {
         pw_win[x] = win;
@@ -823,7 +867,7 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
     for (int x = 0; x < kPre; ++x)
       if (pw_win[x] >= 0) update(pw_win[x], pw_m[x], pw_p[x], pw_part[x]);
     for (int jj = threadIdx.x + kPre * kNW * 32; jj < nF + nQ; jj += blockDim.x) {
-      const int li = list_idx(jj < nF ? jj : jj + has_tail);
+      const int li = jj < nF ? f0 + jj : nf + q0 + (jj - nF);
       const int win = jj < nF ? st.full_list[ub + li] : st.int2_list[ub + li - nf];
       if (win >= 0 && win < st.Wmax)
         update(win, st.mass[ub + win], st.pert[ub + win], a.win_part + (ub + li) * win_part_floats(D, G));

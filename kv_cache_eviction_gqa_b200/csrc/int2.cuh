@@ -10,6 +10,43 @@
 #pragma once
 #include "qe_internal.cuh"
 
+// The parameters of one group from its exact min and max: s = fp16((max - min) / 3) with the
+// quotient correctly rounded in float32 (the correction for division by a known constant,
+// Markstein; Brisebarre, Muller and Raina: q0 = RN(d * RN(1/3)), r = d - 3 q0 exact with an FMA,
+// q = RN(q0 + r * RN(1/3)); checked against IEEE division for every non-negative finite float32
+// and +inf, which passes through), z = fp16(min); the float values of s and z and an
+// approximate reciprocal of s (0 when s == 0).
+struct Int2Group {
+  __half sh, zh;
+  float s, z, rs;
+  __device__ __forceinline__ Int2Group(float mn, float mx) {
+    const float d3 = __fsub_rn(mx, mn);
+    const float third = 0.333333343267440796f;  // RN(1/3)
+    float q3 = __fmul_rn(d3, third);
+    q3 = __fmaf_rn(__fmaf_rn(-3.f, q3, d3), third, q3);
+    if (isinf(d3)) q3 = d3;
+    sh = __float2half_rn(q3);
+    zh = __float2half_rn(mn);
+    s = __half2float(sh);
+    z = __half2float(zh);
+    rs = 0.f;
+    if (s != 0.f) asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rs) : "f"(s));
+  }
+  // code = rint(f32(x - z) / s) clamped to [0, 3]: the quotient is formed with the approximate
+  // reciprocal (relative error about 2^-23, far below 1e-3); within 1e-3 of a half-integer the
+  // correctly rounded division decides instead, so the result is that of rint of the IEEE
+  // quotient in every case. s == 0 gives 0; negative values and NaN convert to 0.
+  __device__ __forceinline__ uint32_t code(float x) const {
+    const float d = __fsub_rn(x, z);
+    float qv = __fmul_rn(d, rs);
+    if (fabsf(qv - rintf(qv)) > 0.499f) qv = __fdiv_rn(d, s);
+    return min(__float2uint_rn(qv), 3u);
+  }
+  __device__ __forceinline__ uint32_t meta() const {
+    return static_cast<uint32_t>(__half_as_ushort(sh)) | (static_cast<uint32_t>(__half_as_ushort(zh)) << 16);
+  }
+};
+
 template <int DPL>
 struct Int2Row {
   static constexpr int LPG = 16 / DPL;  // lanes per 16-element group
@@ -28,35 +65,11 @@ struct Int2Row {
       mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     }
-    // (max - min) / 3 correctly rounded in float32, by the correction for division by a
-    // known constant (Markstein; Brisebarre, Muller and Raina): q0 = RN(d * RN(1/3)),
-    // r = d - 3 q0 (exact with an FMA), q = RN(q0 + r * RN(1/3)). Checked against IEEE
-    // division for every non-negative finite float32 and +inf (which passes through).
-    const float d3 = __fsub_rn(mx, mn);
-    const float third = 0.333333343267440796f;  // RN(1/3)
-    float q3 = __fmul_rn(d3, third);
-    q3 = __fmaf_rn(__fmaf_rn(-3.f, q3, d3), third, q3);
-    if (isinf(d3)) q3 = d3;
-    const __half sh = __float2half_rn(q3);
-    const __half zh = __float2half_rn(mn);
-    const float s = __half2float(sh), z = __half2float(zh);
-    // code = rint(f32(x - z) / s): the quotient is formed with an approximate reciprocal
-    // (relative error about 2^-23, far below 1e-3); within 1e-3 of a half-integer the correctly
-    // rounded division decides instead, so the result is that of rint of the IEEE quotient in
-    // every case. s == 0 gives 0 for every element; negative values and NaN convert to 0.
-    float rs = 0.f;
-    if (s != 0.f) asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rs) : "f"(s));
+    const Int2Group q(mn, mx);
     uint32_t bits = 0;
 #pragma unroll
-    for (int e = 0; e < DPL; ++e) {
-      const float d = __fsub_rn(x[e], z);
-      float qv = __fmul_rn(d, rs);
-      if (fabsf(qv - rintf(qv)) > 0.499f) qv = __fdiv_rn(d, s);
-      const uint32_t c = min(__float2uint_rn(qv), 3u);
-      bits |= c << (2 * e);
-    }
-    *meta = static_cast<uint32_t>(__half_as_ushort(sh)) |
-            (static_cast<uint32_t>(__half_as_ushort(zh)) << 16);
+    for (int e = 0; e < DPL; ++e) bits |= q.code(x[e]) << (2 * e);
+    *meta = q.meta();
     return bits;
   }
 

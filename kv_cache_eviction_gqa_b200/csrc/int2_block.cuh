@@ -64,35 +64,8 @@ struct Int2Block {
     bit = 16 * (t & 1) + 8 * (g & 1) + 2 * ((t >> 3) + 2 * (r >> 3));
   }
 
-  // Row-major codes of one 16-token block (nat[t * D/4 + d/4], element d in bits 2(d%4)) ->
-  // this lane's WPL packed words. V selects the V placement.
-  template <bool V>
-  static __device__ __forceinline__ void pack(const uint8_t* nat, int lane, uint32_t (&w)[WPL]) {
-    const int r = lane >> 2, t4 = lane & 3;
-#pragma unroll
-    for (int j = 0; j < WPL; ++j) {
-      uint32_t x = 0;
-#pragma unroll
-      for (int slot = 0; slot < 16; ++slot) {
-        const int e = slot >> 3, eg = (slot >> 2) & 1, i = slot & 3;
-        const int g = 2 * j + eg;
-        int t, d;
-        if (!V) {
-          t = r + 8 * (i >> 1);
-          d = 16 * g + 2 * t4 + e + 8 * (i & 1);
-        } else {
-          t = 2 * t4 + e + 8 * (i & 1);
-          d = 16 * g + r + 8 * (i >> 1);
-        }
-        const uint32_t c = (nat[t * (D / 4) + (d >> 2)] >> (2 * (d & 3))) & 3u;
-        x |= c << (16 * e + 8 * eg + 2 * i);
-      }
-      w[j] = x;
-    }
-  }
-
-  // Inverse of pack: the packed words of a block (all lanes, words[lane * WPL + j]) -> byte n
-  // (0 .. 16*D/4 - 1) of the row-major codes.
+  // The packed words of a block (all lanes, words[lane * WPL + j]) -> byte n (0 .. 16*D/4 - 1)
+  // of the row-major codes (nat[t * D/4 + d/4], element d in bits 2(d%4)).
   template <bool V>
   static __device__ __forceinline__ uint8_t unpack_byte(const uint32_t* words, int n) {
     const int t = n / (D / 4), d0 = 4 * (n % (D / 4));

@@ -20,6 +20,7 @@
 namespace {
 
 constexpr int kRouteThreads = 512;
+constexpr int kRankMax = 384;  // candidate sets up to this size are ranked by counting
 
 // ---------------------------------------------------------------------------
 // block helpers
@@ -179,36 +180,96 @@ struct RouteArgs {
   size_t dec_stride;
 };
 
-// Sort N 64-bit keys in shared memory in descending order (bitonic network, N a power of 2).
-__device__ void bitonic_desc(unsigned long long* key, int N) {
-  for (int k = 2; k <= N; k <<= 1)
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = threadIdx.x; i < N; i += blockDim.x) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const unsigned long long x = key[i], y = key[ixj];
-          if (((i & k) == 0) ? (x < y) : (x > y)) {
-            key[i] = y;
-            key[ixj] = x;
-          }
-        }
-      }
-      __syncthreads();
-    }
-}
-
 // Selection key: higher score first, then the lower window id; the candidate index rides in
-// the low 12 bits (window ids < 2^20, candidates < 4096). Every real key is non-zero.
+// the low 12 bits (window ids < 2^20, candidates < 4096). Every real key is non-zero and keys
+// of distinct candidates differ.
 __device__ __forceinline__ unsigned long long sel_key(float score, int win, int idx) {
   return ((unsigned long long)ordered_bits(score) << 32) |
          ((unsigned long long)(0xFFFFFu - (uint32_t)win) << 12) | (uint32_t)idx;
 }
 
+// Number of keys in key[0..n) larger than x. A warp scans together and stops once every lane's
+// count has reached `stop` (those candidates are out either way).
+__device__ __forceinline__ int rank_of(const unsigned long long* key, int n, unsigned long long x, int stop) {
+  int r = 0;
+  for (int j0 = 0; j0 < n; j0 += 64) {
+    const int j1 = min(n, j0 + 64);
+    for (int j = j0; j < j1; ++j) r += key[j] > x ? 1 : 0;
+    if (__all_sync(0xffffffffu, r >= stop)) break;
+  }
+  return r;
+}
+
+// Marks mark[i] |= 1 for the b largest of the non-zero keys key[0..n) (keys distinct), by a radix
+// select from the most significant byte: a 256-bin histogram of the next byte among the keys
+// that share the digits chosen so far, the bin where the count from the top reaches b, and so on
+// until that bin holds exactly the keys still needed. hist: 256 ints of shared memory.
+__device__ void radix_top(const unsigned long long* key, int n, int b, uint8_t* mark, int* hist) {
+  __shared__ int s_digit, s_above, s_in;
+  unsigned long long prefix = 0ull, mask = 0ull;
+  int remaining = b;
+  bool inclusive = false;
+  for (int shift = 56; shift >= 0 && remaining > 0; shift -= 8) {
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const unsigned long long k = key[i];
+      if (k != 0ull && (k & mask) == prefix) atomicAdd(&hist[(int)((k >> shift) & 255ull)], 1);
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      // lane l sums bins 255 - 8l .. 248 - 8l (top down); the first lane whose running total from
+      // the top reaches `remaining` holds the crossing bin
+      const int l = threadIdx.x;
+      int part = 0;
+      for (int q = 0; q < 8; ++q) part += hist[255 - 8 * l - q];
+      int incl = part;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (l >= o) incl += v;
+      }
+      const unsigned hit = __ballot_sync(0xffffffffu, incl >= remaining);
+      const int lw = __ffs(hit) - 1;
+      if (l == lw) {
+        int above = incl - part;
+        for (int q = 0; q < 8; ++q) {
+          const int d = 255 - 8 * l - q, c = hist[d];
+          if (above + c >= remaining) {
+            s_digit = d;
+            s_above = above;
+            s_in = c;
+            break;
+          }
+          above += c;
+        }
+      }
+    }
+    __syncthreads();
+    const int d = s_digit, above = s_above, in = s_in;
+    __syncthreads();
+    prefix |= (unsigned long long)d << shift;
+    mask |= 255ull << shift;
+    remaining -= above;
+    if (remaining == in) {  // the crossing bin holds exactly the keys still needed
+      inclusive = true;
+      break;
+    }
+  }
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const unsigned long long k = key[i], km = k & mask;
+    if (k != 0ull && (km > prefix || (inclusive && km == prefix))) mark[i] = 1;
+  }
+  __syncthreads();
+}
+
 // Two-stage selection among candidates with inset[i]; selected ones get sel[i] = 1 and the
-// stage-1 picks s1mark[i] = 1. `key` holds N >= n 64-bit keys (N a power of two).
-__device__ void two_stage_select(int n, int N, const int32_t* cand, const float* k1, const float* k2,
+// stage-1 picks s1mark[i] = 1. A candidate's rank in a set is the number of members with a
+// larger key, so stage 1 keeps the inset members of rank < b1 by k1 and stage 2 the members of
+// the rest of rank < b - b1 by k2: exactly the top-b1 and top-(b - b1) (keys are distinct).
+// `key` holds at least n 64-bit keys.
+__device__ void two_stage_select(int n, const int32_t* cand, const float* k1, const float* k2,
                                  const uint8_t* inset, uint8_t* sel, uint8_t* s1mark, int b, int b1,
-                                 int* ibuf, unsigned long long* key) {
+                                 int* ibuf, unsigned long long* key, int* hist) {
   int cnt_local = 0;
   for (int i = threadIdx.x; i < n; i += blockDim.x) cnt_local += inset[i];
   int cnt;
@@ -221,23 +282,41 @@ __device__ void two_stage_select(int n, int N, const int32_t* cand, const float*
     __syncthreads();
     return;
   }
-  // stage 1: the b1 largest k1 among inset
-  for (int i = threadIdx.x; i < N; i += blockDim.x) {
-    key[i] = (i < n && inset[i]) ? sel_key(k1[i], cand[i], i) : 0ull;
-    if (i < n) s1mark[i] = 0;
+  if (n > kRankMax) {
+    // many candidates: radix select (a few histogram passes) instead of n^2 rank counts
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      key[i] = inset[i] ? sel_key(k1[i], cand[i], i) : 0ull;
+      s1mark[i] = 0;
+    }
+    __syncthreads();
+    if (b1 > 0) radix_top(key, n, b1, s1mark, hist);
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      key[i] = (inset[i] && !s1mark[i]) ? sel_key(k2[i], cand[i], i) : 0ull;
+      sel[i] = s1mark[i];
+    }
+    __syncthreads();
+    if (b - b1 > 0) radix_top(key, n, b - b1, sel, hist);
+    return;
   }
+  // stage 1: the b1 largest k1 among inset
+  for (int i = threadIdx.x; i < n; i += blockDim.x) key[i] = inset[i] ? sel_key(k1[i], cand[i], i) : 0ull;
   __syncthreads();
-  bitonic_desc(key, N);
-  for (int r = threadIdx.x; r < b1; r += blockDim.x) s1mark[key[r] & 0xFFFu] = 1;
+  const int nn = (n + 31) / 32 * 32;  // whole warps take part in every rank scan
+  for (int i = threadIdx.x; i < nn; i += blockDim.x) {
+    const unsigned long long x = i < n ? key[i] : 0ull;
+    const int r = rank_of(key, n, x, b1);
+    if (i < n) s1mark[i] = (x != 0ull && r < b1) ? 1 : 0;
+  }
   __syncthreads();
   // stage 2: the b - b1 largest k2 among inset minus stage 1
-  for (int i = threadIdx.x; i < N; i += blockDim.x) {
-    key[i] = (i < n && inset[i] && !s1mark[i]) ? sel_key(k2[i], cand[i], i) : 0ull;
-    if (i < n) sel[i] = s1mark[i];
-  }
+  for (int i = threadIdx.x; i < n; i += blockDim.x)
+    key[i] = (inset[i] && !s1mark[i]) ? sel_key(k2[i], cand[i], i) : 0ull;
   __syncthreads();
-  bitonic_desc(key, N);
-  for (int r = threadIdx.x; r < b - b1; r += blockDim.x) sel[key[r] & 0xFFFu] = 1;
+  for (int i = threadIdx.x; i < nn; i += blockDim.x) {
+    const unsigned long long x = i < n ? key[i] : 0ull;
+    const int r = rank_of(key, n, x, b - b1);
+    if (i < n) sel[i] = s1mark[i] | ((x != 0ull && r < b - b1) ? 1 : 0);
+  }
   __syncthreads();
 }
 
@@ -248,8 +327,6 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
   const int nf = st.stacks[u * 4 + 2], nq = st.stacks[u * 4 + 3], n = nf + nq;
   int NW = 1;  // key buffer capacity (power of two >= Wmax)
   while (NW < st.Wmax) NW <<= 1;
-  int N = 1;   // sort size: power of two >= the candidate count
-  while (N < n) N <<= 1;
   unsigned long long* key = reinterpret_cast<unsigned long long*>(sm);
   int32_t* cand = reinterpret_cast<int32_t*>(key + NW);
   float* km = reinterpret_cast<float*>(cand + st.Wmax);
@@ -261,6 +338,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
   uint8_t* s1 = sel + st.Wmax;
   __shared__ int ibuf[33];
   __shared__ float fbuf[32];
+  __shared__ int hist[256];
   __shared__ int s_abort;
   if (threadIdx.x == 0) s_abort = 0;
   if (n > st.Wmax) {
@@ -282,7 +360,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
   if (a.mode == 0) {
     for (int i = threadIdx.x; i < n; i += blockDim.x) inset[i] = 1;
     __syncthreads();
-    two_stage_select(n, N, cand, km, kp, inset, sel, s1, a.F, a.F1, ibuf, key);
+    two_stage_select(n, cand, km, kp, inset, sel, s1, a.F, a.F1, ibuf, key, hist);
     float s1m = 0.f, am = 0.f;
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
       if (sel[i]) newt[i] = QE_TIER_FULL;
@@ -292,7 +370,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
     }
     stage1_mass = block_sum(s1m, fbuf);
     all_mass = block_sum(am, fbuf);
-    two_stage_select(n, N, cand, km, kp, inset, sel, s1, a.Q, a.Q1, ibuf, key);
+    two_stage_select(n, cand, km, kp, inset, sel, s1, a.Q, a.Q1, ibuf, key, hist);
     for (int i = threadIdx.x; i < n; i += blockDim.x)
       if (sel[i]) newt[i] = QE_TIER_INT2;
   } else if (a.mode == 2) {
@@ -437,59 +515,40 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// quantise (first demotion only) and promote, one warp per (window, page)
+// quantise (first demotion only) and promote
 // ---------------------------------------------------------------------------
-// A lane owns DPL = D/32 consecutive elements of a row (one 4- or 8-byte word). The window's
-// ledger slot and the page are looked up once per 16 tokens; every row load of the page is
-// issued before the first one is used.
-template <int DPL> struct RowWord;
-template <> struct RowWord<4> { using type = uint2; };
-template <> struct RowWord<2> { using type = uint32_t; };
-
-template <typename T>
-__device__ __forceinline__ void word_to_f(uint2 w, float (&x)[4]) {
-  x[0] = Elem<T>::lo(w.x);
-  x[1] = Elem<T>::hi(w.x);
-  x[2] = Elem<T>::lo(w.y);
-  x[3] = Elem<T>::hi(w.y);
-}
-template <typename T>
-__device__ __forceinline__ void word_to_f(uint32_t w, float (&x)[2]) {
-  x[0] = Elem<T>::lo(w);
-  x[1] = Elem<T>::hi(w);
-}
 template <typename T>
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
   const T lo = Elem<T>::from_f(a), hi = Elem<T>::from_f(b);
   return static_cast<uint32_t>(*reinterpret_cast<const unsigned short*>(&lo)) |
          (static_cast<uint32_t>(*reinterpret_cast<const unsigned short*>(&hi)) << 16);
 }
-template <typename T>
-__device__ __forceinline__ void f_to_word(const float (&x)[4], uint2& w) {
-  w.x = pack2<T>(x[0], x[1]);
-  w.y = pack2<T>(x[2], x[3]);
-}
-template <typename T>
-__device__ __forceinline__ void f_to_word(const float (&x)[2], uint32_t& w) {
-  w = pack2<T>(x[0], x[1]);
-}
-
+// One warp per (window, page) = one 16-token block of the window's ledger entry. Lane (r, t)
+// works directly in the block's placement (int2_block.cuh): for K it quantises the elements
+// 16g + 2t + {0, 1, 8, 9} of tokens r and 8 + r (a group's 16 elements of a token sit in the
+// four lanes of a quad: min and max by two shuffles), for V the elements 16g + r and 16g + 8 + r
+// of tokens 2t, 2t+1, 8+2t, 9+2t (a group's elements sit in the eight lanes of a column), and
+// packs its own code words; promotion reverses this. The page and the block pass through shared
+// memory so that both move with coalesced 16-byte accesses.
 template <typename T, int D>
-__global__ void __launch_bounds__(256) apply_kernel(DevState st, const int32_t* xlist, const int32_t* plist,
+__global__ void __launch_bounds__(128) apply_kernel(DevState st, const int32_t* xlist, const int32_t* plist,
                                                     const int32_t* xcount, int unit_only) {
-  constexpr int DPL = D / 32;
-  using R = Int2Row<DPL>;
   using BL = Int2Block<D>;
-  using Wd = typename RowWord<DPL>::type;
-  // per warp: the block as it sits in the ledger, then the row-major K and V codes
-  constexpr int NAT = QE_PAGE * D / 4;
-  __shared__ __align__(16) uint8_t sm_all[8][BL::BYTES + 2 * NAT];
+  constexpr int G8 = BL::G8, WPL = BL::WPL;
+  constexpr int PAGEB = 2 * QE_PAGE * D * 2;  // K rows then V rows
+  __shared__ __align__(16) uint8_t sm_all[4][PAGEB + BL::BYTES];
   const int u = unit_only >= 0 ? unit_only : blockIdx.x;
-  const int lane = threadIdx.x & 31;
-  uint8_t* img = sm_all[threadIdx.x >> 5];
-  uint8_t* natk = img + BL::BYTES;
-  uint8_t* natv = natk + NAT;
-  const int warps = blockDim.x >> 5, gw = blockIdx.y * warps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31, wq = threadIdx.x >> 5;
+  const int r = lane >> 2, t4 = lane & 3;
+  uint8_t* pg_s = sm_all[wq];
+  uint8_t* img = pg_s + PAGEB;
+  T* Ks = reinterpret_cast<T*>(pg_s);
+  T* Vs = Ks + QE_PAGE * D;
+  uint16_t* ks = reinterpret_cast<uint16_t*>(img + BL::KS);
+  uint16_t* kz = reinterpret_cast<uint16_t*>(img + BL::KZ);
+  uint16_t* vs = reinterpret_cast<uint16_t*>(img + BL::VS);
+  uint16_t* vz = reinterpret_cast<uint16_t*>(img + BL::VZ);
+  const int warps = blockDim.x >> 5, gw = blockIdx.y * warps + wq;
   const int nx = xcount[u * 4 + 0], np = xcount[u * 4 + 1];
   const size_t ub = (size_t)u * st.Wmax;
   const int ppw = st.ppw;
@@ -507,89 +566,107 @@ __global__ void __launch_bounds__(256) apply_kernel(DevState st, const int32_t* 
       if (lane == 0) qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
       continue;
     }
-    // block pg of the window's ledger entry holds the page's 16 tokens
     uint4* gblk = reinterpret_cast<uint4*>(st.slots + ((size_t)u * st.S + slot) * st.slot_bytes +
                                            (size_t)pg * BL::BYTES);
-    Wd* krows = reinterpret_cast<Wd*>(st.pages + ((size_t)u * st.P + page) * st.page_bytes);
-    Wd* vrows = krows + QE_PAGE * 32;  // 32 words per row
+    uint4* gpage = reinterpret_cast<uint4*>(st.pages + ((size_t)u * st.P + page) * st.page_bytes);
     __syncwarp();  // the previous item is done with this warp's shared memory
     if (quant) {
-      Wd kw[QE_PAGE], vw[QE_PAGE];
+      for (int i = lane; i < PAGEB / 16; i += 32) reinterpret_cast<uint4*>(pg_s)[i] = gpage[i];
+      __syncwarp();
+      uint32_t kw[WPL], vw[WPL];
 #pragma unroll
-      for (int r = 0; r < QE_PAGE; ++r) {
-        kw[r] = krows[r * 32 + lane];
-        vw[r] = vrows[r * 32 + lane];
-      }
+      for (int j = 0; j < WPL; ++j) kw[j] = vw[j] = 0u;
 #pragma unroll
-      for (int r = 0; r < QE_PAGE; ++r) {
-        float xk[DPL], xv[DPL];
-        word_to_f<T>(kw[r], xk);
-        word_to_f<T>(vw[r], xv);
-        uint32_t mk, mv;
-        const uint32_t bk = R::quantize(xk, &mk);
-        const uint32_t bv = R::quantize(xv, &mv);
-        R::store_codes(natk + r * (D / 4), bk, lane);
-        R::store_codes(natv + r * (D / 4), bv, lane);
-        if (lane % R::LPG == 0) {
-          const int g = R::group_of(lane);
-          uint16_t* ks = reinterpret_cast<uint16_t*>(img + BL::KS);
-          uint16_t* kz = reinterpret_cast<uint16_t*>(img + BL::KZ);
-          uint16_t* vs = reinterpret_cast<uint16_t*>(img + BL::VS);
-          uint16_t* vz = reinterpret_cast<uint16_t*>(img + BL::VZ);
-          ks[g * QE_PAGE + BL::ppos(r)] = static_cast<uint16_t>(mk & 0xffffu);
-          kz[r * BL::G8 + g] = static_cast<uint16_t>(mk >> 16);
-          vs[g * QE_PAGE + BL::fpos(r)] = static_cast<uint16_t>(mv & 0xffffu);
-          vz[g * QE_PAGE + BL::fpos(r)] = static_cast<uint16_t>(mv >> 16);
+      for (int tb = 0; tb < 2; ++tb) {
+        const int t = r + 8 * tb;
+        const uint32_t* row = reinterpret_cast<const uint32_t*>(Ks + t * D);
+#pragma unroll
+        for (int g = 0; g < G8; ++g) {
+          const uint32_t a = row[8 * g + t4], b = row[8 * g + 4 + t4];
+          const float x0 = Elem<T>::lo(a), x1 = Elem<T>::hi(a), x2 = Elem<T>::lo(b), x3 = Elem<T>::hi(b);
+          float mn = fminf(fminf(x0, x1), fminf(x2, x3)), mx = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
+#pragma unroll
+          for (int o = 1; o < 4; o <<= 1) {
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          }
+          const Int2Group q(mn, mx);
+          const int base = 8 * (g & 1) + 4 * tb;  // register i = 2 tb + h at bit 2i of each half
+          kw[g >> 1] |= (q.code(x0) << base) | (q.code(x1) << (16 + base)) | (q.code(x2) << (base + 2)) |
+                        (q.code(x3) << (16 + base + 2));
+          if (t4 == 0) {
+            ks[g * QE_PAGE + BL::ppos(t)] = __half_as_ushort(q.sh);
+            kz[t * G8 + g] = __half_as_ushort(q.zh);
+          }
         }
       }
-      __syncwarp();
-      uint32_t pk[BL::WPL], pv[BL::WPL];
-      BL::template pack<false>(natk, lane, pk);
-      BL::template pack<true>(natv, lane, pv);
-      uint32_t* kc = reinterpret_cast<uint32_t*>(img + BL::KC) + lane * BL::WPL;
-      uint32_t* vc = reinterpret_cast<uint32_t*>(img + BL::VC) + lane * BL::WPL;
 #pragma unroll
-      for (int j = 0; j < BL::WPL; ++j) {
-        kc[j] = pk[j];
-        vc[j] = pv[j];
+      for (int kk = 0; kk < 4; ++kk) {
+        const int tk = 2 * t4 + (kk & 1) + 8 * (kk >> 1);
+        const int e = kk & 1, kh = kk >> 1;
+#pragma unroll
+        for (int g = 0; g < G8; ++g) {
+          const float x0 = Elem<T>::to_f(Vs[tk * D + 16 * g + r]), x1 = Elem<T>::to_f(Vs[tk * D + 16 * g + 8 + r]);
+          float mn = fminf(x0, x1), mx = fmaxf(x0, x1);
+#pragma unroll
+          for (int o = 4; o < 32; o <<= 1) {
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          }
+          const Int2Group q(mn, mx);
+          const int base = 16 * e + 8 * (g & 1) + 2 * kh;  // register i = 2 rh + kh
+          vw[g >> 1] |= (q.code(x0) << base) | (q.code(x1) << (base + 4));
+          if (r == 0) {
+            vs[g * QE_PAGE + BL::fpos(tk)] = __half_as_ushort(q.sh);
+            vz[g * QE_PAGE + BL::fpos(tk)] = __half_as_ushort(q.zh);
+          }
+        }
+      }
+      uint32_t* kc = reinterpret_cast<uint32_t*>(img + BL::KC) + lane * WPL;
+      uint32_t* vc = reinterpret_cast<uint32_t*>(img + BL::VC) + lane * WPL;
+#pragma unroll
+      for (int j = 0; j < WPL; ++j) {
+        kc[j] = kw[j];
+        vc[j] = vw[j];
       }
       __syncwarp();
-      const uint4* src = reinterpret_cast<const uint4*>(img);
-      for (int i = lane; i < BL::BYTES / 16; i += 32) gblk[i] = src[i];
+      for (int i = lane; i < BL::BYTES / 16; i += 32) gblk[i] = reinterpret_cast<const uint4*>(img)[i];
     } else {
-      uint4* dst = reinterpret_cast<uint4*>(img);
-      for (int i = lane; i < BL::BYTES / 16; i += 32) dst[i] = gblk[i];
+      for (int i = lane; i < BL::BYTES / 16; i += 32) reinterpret_cast<uint4*>(img)[i] = gblk[i];
       __syncwarp();
-      const uint32_t* kc = reinterpret_cast<const uint32_t*>(img + BL::KC);
-      const uint32_t* vc = reinterpret_cast<const uint32_t*>(img + BL::VC);
-      for (int n = lane; n < NAT; n += 32) {
-        natk[n] = BL::template unpack_byte<false>(kc, n);
-        natv[n] = BL::template unpack_byte<true>(vc, n);
-      }
-      __syncwarp();
-      const uint16_t* ks = reinterpret_cast<const uint16_t*>(img + BL::KS);
-      const uint16_t* kz = reinterpret_cast<const uint16_t*>(img + BL::KZ);
-      const uint16_t* vs = reinterpret_cast<const uint16_t*>(img + BL::VS);
-      const uint16_t* vz = reinterpret_cast<const uint16_t*>(img + BL::VZ);
-      const int g = R::group_of(lane);
+      const uint32_t* kc = reinterpret_cast<const uint32_t*>(img + BL::KC) + lane * WPL;
+      const uint32_t* vc = reinterpret_cast<const uint32_t*>(img + BL::VC) + lane * WPL;
 #pragma unroll
-      for (int r = 0; r < QE_PAGE; ++r) {
-        const uint32_t bk = R::load_codes(natk + r * (D / 4), lane);
-        const uint32_t bv = R::load_codes(natv + r * (D / 4), lane);
-        const float sk = meta_scale(ks[g * QE_PAGE + BL::ppos(r)]), zk = meta_scale(kz[r * BL::G8 + g]);
-        const float sv = meta_scale(vs[g * QE_PAGE + BL::fpos(r)]), zv = meta_scale(vz[g * QE_PAGE + BL::fpos(r)]);
-        float xk[DPL], xv[DPL];
+      for (int tb = 0; tb < 2; ++tb) {
+        const int t = r + 8 * tb;
+        uint32_t* row = reinterpret_cast<uint32_t*>(Ks + t * D);
 #pragma unroll
-        for (int e = 0; e < DPL; ++e) {
-          xk[e] = fmaf((float)((bk >> (2 * e)) & 3u), sk, zk);
-          xv[e] = fmaf((float)((bv >> (2 * e)) & 3u), sv, zv);
+        for (int g = 0; g < G8; ++g) {
+          const uint32_t x = kc[g >> 1];
+          const int base = 8 * (g & 1) + 4 * tb;
+          const float sc = meta_scale(ks[g * QE_PAGE + BL::ppos(t)]), zc = meta_scale(kz[t * G8 + g]);
+          const float v0 = fmaf((float)((x >> base) & 3u), sc, zc), v1 = fmaf((float)((x >> (16 + base)) & 3u), sc, zc);
+          const float v2 = fmaf((float)((x >> (base + 2)) & 3u), sc, zc);
+          const float v3 = fmaf((float)((x >> (16 + base + 2)) & 3u), sc, zc);
+          row[8 * g + t4] = pack2<T>(v0, v1);
+          row[8 * g + 4 + t4] = pack2<T>(v2, v3);
         }
-        Wd ok, ov;
-        f_to_word<T>(xk, ok);
-        f_to_word<T>(xv, ov);
-        krows[r * 32 + lane] = ok;
-        vrows[r * 32 + lane] = ov;
       }
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const int tk = 2 * t4 + (kk & 1) + 8 * (kk >> 1);
+        const int e = kk & 1, kh = kk >> 1;
+#pragma unroll
+        for (int g = 0; g < G8; ++g) {
+          const uint32_t x = vc[g >> 1];
+          const int base = 16 * e + 8 * (g & 1) + 2 * kh;
+          const float sc = meta_scale(vs[g * QE_PAGE + BL::fpos(tk)]), zc = meta_scale(vz[g * QE_PAGE + BL::fpos(tk)]);
+          Vs[tk * D + 16 * g + r] = Elem<T>::from_f(fmaf((float)((x >> base) & 3u), sc, zc));
+          Vs[tk * D + 16 * g + 8 + r] = Elem<T>::from_f(fmaf((float)((x >> (base + 4)) & 3u), sc, zc));
+        }
+      }
+      __syncwarp();
+      for (int i = lane; i < PAGEB / 16; i += 32) gpage[i] = reinterpret_cast<const uint4*>(pg_s)[i];
     }
   }
 }
@@ -661,10 +738,22 @@ void launch_apply(const DevState& st, const qe_ctx* c, int unit_only, cudaStream
   // windows into a new tier (host-given transitions at most Wmax)
   int wins = unit_only >= 0 ? st.Wmax : c->cfg.full_windows + c->cfg.int2_windows;
   if (wins > st.Wmax) wins = st.Wmax;
-  int per_unit = (wins * st.ppw + 7) / 8;
+  // 4 warps per block, one (window, page) item per warp at a time; a routing event moves at most
+  // F + Q windows into a new tier (host-given transitions at most Wmax). The blocks of a unit
+  // loop over its items, so one wave of about four blocks per SM covers any event.
+  int per_unit = (wins * st.ppw + 3) / 4;
+  static QeOnce once;
+  static int sms_of[QE_MAX_DEVICES];
+  int dev = 0;
+  if (qe_once_per_device(once, &dev, [](int d) {
+        QE_CUDA_TRY(cudaDeviceGetAttribute(&sms_of[d], cudaDevAttrMultiProcessorCount, d));
+        return QE_OK;
+      }) != QE_OK)
+    sms_of[dev] = 148;
+  const int wave = (4 * sms_of[dev] + units - 1) / units;
+  if (per_unit > wave) per_unit = wave;
   if (per_unit < 1) per_unit = 1;
-  if (per_unit > 1024) per_unit = 1024;
-  apply_kernel<T, D><<<dim3(units, per_unit), 256, 0, s>>>(st, c->xlist, c->plist, c->xcount,
+  apply_kernel<T, D><<<dim3(units, per_unit), 128, 0, s>>>(st, c->xlist, c->plist, c->xcount,
                                                             unit_only);
 }
 

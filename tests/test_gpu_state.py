@@ -67,8 +67,9 @@ def test_export_import_continues_like_the_original_and_the_oracle(where):
         assert restored.status() == (0, 0)
         assert torch.equal(o1, o2), f"step {s}: outputs differ after the restore"
         sa, sb = a.state(), restored.state()
-        for name in sa:
-            assert torch.equal(sa[name], sb[name]), f"step {s}: {name} differs after the restore"
+        for name in sa:  # bitwise: free pages and slots hold whatever the allocator left (NaN too)
+            assert torch.equal(sa[name].contiguous().view(torch.uint8), sb[name].contiguous().view(torch.uint8)), \
+                f"step {s}: {name} differs after the restore"
         # the restored context against the oracle (routing on this unit matches: no near-ties)
         og = o2.cpu().numpy()[b, h * G:(h + 1) * G]
         err = (np.abs(og - o_ref).max(axis=-1) / np.abs(o_ref).max(axis=-1)).max()
