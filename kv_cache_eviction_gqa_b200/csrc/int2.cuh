@@ -24,13 +24,14 @@ struct Int2Group {
     const float third = 0.333333343267440796f;  // RN(1/3)
     float q3 = __fmul_rn(d3, third);
     q3 = __fmaf_rn(__fmaf_rn(-3.f, q3, d3), third, q3);
-    if (isinf(d3)) q3 = d3;
+    q3 = isinf(d3) ? d3 : q3;
     sh = __float2half_rn(q3);
     zh = __float2half_rn(mn);
     s = __half2float(sh);
     z = __half2float(zh);
-    rs = 0.f;
-    if (s != 0.f) asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rs) : "f"(s));
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(s));
+    rs = s != 0.f ? r : 0.f;
   }
   // code = rint(f32(x - z) / s) clamped to [0, 3]: the quotient is formed with the approximate
   // reciprocal (relative error about 2^-23, far below 1e-3); within 1e-3 of a half-integer the
@@ -42,10 +43,60 @@ struct Int2Group {
     if (fabsf(qv - rintf(qv)) > 0.499f) qv = __fdiv_rn(d, s);
     return min(__float2uint_rn(qv), 3u);
   }
+  // Parameters (rs, -z) of the fast code path: q = f32(f32(x - z) * rs), with the approximate
+  // reciprocal rs (relative error below 2^-22), is within 2^-20 of the IEEE quotient
+  // f32(x - z) / s for q < 4, and stays within (-0.5, 3.5) for every x of the group when
+  // |min - z| * rs < 0.45. Groups outside that bound (or with s subnormal or infinite in fp16,
+  // or z infinite) get -1 in place of rs: the exact path decides. s == 0 gives rs = 0, so every
+  // q is 0.
+  __device__ __forceinline__ float2 fast_params(float mn) const {
+    const bool ok = (s == 0.f || (s >= 0x1p-14f && s <= 65504.f)) && fabsf(z) <= 65504.f &&
+                    fabsf(__fsub_rn(mn, z)) * rs < 0.45f;
+    return make_float2(ok ? rs : -1.f, -z);
+  }
   __device__ __forceinline__ uint32_t meta() const {
     return static_cast<uint32_t>(__half_as_ushort(sh)) | (static_cast<uint32_t>(__half_as_ushort(zh)) << 16);
   }
 };
+
+// code = clamp(rint(f32(x - z) / s), 0, 3) by IEEE division; 0 when s == 0 (the definition the
+// fast path below falls back on).
+__device__ __forceinline__ uint32_t int2_code_exact(float x, float s, float z) {
+  if (s == 0.f) return 0u;
+  return min(__float2uint_rn(__fdiv_rn(__fsub_rn(x, z), s)), 3u);
+}
+
+// The 16 codes of one group, element e at bits 2e of n, from its elements as eight pairs of
+// 16-bit values (e2[i] holds elements 2i, 2i + 1) and fast parameters p = (rs, -z), rs >= 0.
+// Each q = f32(f32(x - z) * rs) is rounded to an integer by adding 1.5 * 2^23: the sum's bits are
+// 0x4B400000 + rint(q) (ties to even, q in (-0.5, 3.5)), so the codes accumulate by shifted
+// adds of the raw bits, less the same sum of the constant part. Returns the mask of elements
+// whose q lies within 2^-16 of a half-integer (bit e), where q could round the other way than
+// the exact quotient (they differ by less than 2^-20): those take the exact path.
+template <typename T>
+__device__ __forceinline__ uint32_t int2_group_codes_fast(const uint32_t (&e2)[8], float2 p, uint32_t& n) {
+  constexpr float kMagic = 12582912.f;  // 1.5 * 2^23, bits 0x4B400000
+  constexpr float kNear = 0.5f - 0x1p-16f;
+  constexpr uint32_t kBias = [] {
+    uint32_t b = 0u;
+    for (int e = 0; e < 16; ++e) b += 0x4B400000u << (2 * e);
+    return b;
+  }();
+  const float2 r2 = make_float2(p.x, p.x), nz2 = make_float2(p.y, p.y);
+  uint32_t acc = 0u, near = 0u;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float2 x = make_float2(Elem<T>::lo(e2[i]), Elem<T>::hi(e2[i]));
+    const float2 q = __fmul2_rn(__fadd2_rn(x, nz2), r2);
+    const float2 t = __fadd2_rn(q, make_float2(kMagic, kMagic));
+    const float2 e = __ffma2_rn(q, make_float2(-1.f, -1.f), __fadd2_rn(t, make_float2(-kMagic, -kMagic)));
+    near |= (fabsf(e.x) > kNear ? 1u : 0u) << (2 * i);
+    near |= (fabsf(e.y) > kNear ? 1u : 0u) << (2 * i + 1);
+    acc += (__float_as_uint(t.x) << (4 * i)) + (__float_as_uint(t.y) << (4 * i + 2));
+  }
+  n = acc - kBias;
+  return near;
+}
 
 template <int DPL>
 struct Int2Row {

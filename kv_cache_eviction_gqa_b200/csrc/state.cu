@@ -523,152 +523,347 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
   return static_cast<uint32_t>(*reinterpret_cast<const unsigned short*>(&lo)) |
          (static_cast<uint32_t>(*reinterpret_cast<const unsigned short*>(&hi)) << 16);
 }
-// One warp per (window, page) = one 16-token block of the window's ledger entry. Lane (r, t)
-// works directly in the block's placement (int2_block.cuh): for K it quantises the elements
-// 16g + 2t + {0, 1, 8, 9} of tokens r and 8 + r (a group's 16 elements of a token sit in the
-// four lanes of a quad: min and max by two shuffles), for V the elements 16g + r and 16g + 8 + r
-// of tokens 2t, 2t+1, 8+2t, 9+2t (a group's elements sit in the eight lanes of a column), and
-// packs its own code words; promotion reverses this. The page and the block pass through shared
-// memory so that both move with coalesced 16-byte accesses.
+// Quantise (first demotion) and promote, one item = one (window, page) = one 16-token block of
+// the window's ledger entry. The items of all units form one list (unit u's nx quantisations
+// then np promotions, ppw pages each); block b of the grid takes items b, b + gridDim, ... .
+// Each block is a pair of warps, warp 0 on the item's K rows and warp 1 on its V rows; the item's
+// source arrives and its result leaves by bulk copies, the next item's copy overlapping the
+// store of the current one, and many blocks per SM keep enough copies in flight.
+//
+// Quantisation, pass A (natural layout): lane l takes the (token, group) pairs l, l + 32, ...
+// of its warp's tensor, reads the group's 16 elements, forms min and max with packed 16-bit
+// min/max and builds the group's parameters once: fp16 scale and zero into the block's meta
+// arrays, (-z, 1/s) for pass B. Pass B (block placement, int2_block.cuh): lane (r, t) computes
+// the codes of its own positions with int2_code2_fast and stores its code words; positions the
+// fast path cannot decide are marked in a bit mask and recomputed afterwards by IEEE division.
+// Promotion: pass A turns each group's fp16 (s, z) into floats once; pass B rebuilds each element
+// as f32(code * s + z) rounded to the cache dtype, in row-major page order.
+constexpr int kApplyThreads = 64;
+
+__device__ __forceinline__ void bulk_s2g(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_u32(src)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+template <typename T> __device__ __forceinline__ uint32_t min2_u32(uint32_t a, uint32_t b);
+template <typename T> __device__ __forceinline__ uint32_t max2_u32(uint32_t a, uint32_t b);
+template <> __device__ __forceinline__ uint32_t min2_u32<__nv_bfloat16>(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("min.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+template <> __device__ __forceinline__ uint32_t max2_u32<__nv_bfloat16>(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+template <> __device__ __forceinline__ uint32_t min2_u32<__half>(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("min.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+template <> __device__ __forceinline__ uint32_t max2_u32<__half>(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// A page's 32 rows (16 K then 16 V) sit in shared memory with a stride of D + 8 elements, so that
+// the placement passes (lanes of one quad column on eight different rows) hit distinct banks;
+// the group parameters use a stride of D/16 + 1 per token for the same reason.
+template <int D>
+constexpr int apply_row() { return D + 8; }
+template <int D>
+constexpr size_t apply_buf_bytes() {  // a padded page image (a block image is smaller)
+  return (size_t)2 * QE_PAGE * apply_row<D>() * 2;
+}
+template <int D>
+size_t apply_smem_bytes(int units) {
+  return 2 * apply_buf_bytes<D>() + 2 * QE_PAGE * (D / 16 + 1) * 8 + 32 + 4 * (size_t)(units + 1);
+}
+
+// Replace the codes of the elements marked in mask (bit e; elements 0..7 in a, 8..15 in b, pairs
+// of 16-bit values) in n by IEEE division: the path taken where the fast one cannot decide.
+template <typename T>
+__device__ __noinline__ uint32_t int2_group_codes_exact(uint32_t n, uint32_t mask, uint4 a, uint4 b, float s,
+                                                        float z) {
+  const uint32_t e2[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  for (int e = 0; e < 16; ++e) {
+    if (!((mask >> e) & 1u)) continue;
+    const uint32_t w = e2[e >> 1];
+    const float x = (e & 1) ? Elem<T>::hi(w) : Elem<T>::lo(w);
+    n = (n & ~(3u << (2 * e))) | (int2_code_exact(x, s, z) << (2 * e));
+  }
+  return n;
+}
+
 template <typename T, int D>
-__global__ void __launch_bounds__(128) apply_kernel(DevState st, const int32_t* xlist, const int32_t* plist,
-                                                    const int32_t* xcount, int unit_only) {
+__global__ void __launch_bounds__(kApplyThreads) apply_kernel(DevState st, const int32_t* xlist,
+                                                              const int32_t* plist, const int32_t* xcount,
+                                                              int unit_only) {
   using BL = Int2Block<D>;
   constexpr int G8 = BL::G8, WPL = BL::WPL;
-  constexpr int PAGEB = 2 * QE_PAGE * D * 2;  // K rows then V rows
-  __shared__ __align__(16) uint8_t sm_all[4][PAGEB + BL::BYTES];
-  const int u = unit_only >= 0 ? unit_only : blockIdx.x;
-  const int lane = threadIdx.x & 31, wq = threadIdx.x >> 5;
+  constexpr int RS = apply_row<D>();          // row stride in shared memory (elements)
+  constexpr int PAGES = (int)apply_buf_bytes<D>();  // a padded page image
+  constexpr int NG = QE_PAGE * G8;            // groups per tensor and block
+  constexpr int PS = G8 + 1;                  // parameter stride per token
+  extern __shared__ __align__(16) uint8_t sm[];
+  const int lane = threadIdx.x & 31, wq = threadIdx.x >> 5;  // wq: 0 K rows, 1 V rows
   const int r = lane >> 2, t4 = lane & 3;
-  uint8_t* pg_s = sm_all[wq];
-  uint8_t* img = pg_s + PAGEB;
-  T* Ks = reinterpret_cast<T*>(pg_s);
-  T* Vs = Ks + QE_PAGE * D;
-  uint16_t* ks = reinterpret_cast<uint16_t*>(img + BL::KS);
-  uint16_t* kz = reinterpret_cast<uint16_t*>(img + BL::KZ);
-  uint16_t* vs = reinterpret_cast<uint16_t*>(img + BL::VS);
-  uint16_t* vz = reinterpret_cast<uint16_t*>(img + BL::VZ);
-  const int warps = blockDim.x >> 5, gw = blockIdx.y * warps + wq;
-  const int nx = xcount[u * 4 + 0], np = xcount[u * 4 + 1];
-  const size_t ub = (size_t)u * st.Wmax;
+  float2* prm = reinterpret_cast<float2*>(sm + 2 * PAGES) + wq * QE_PAGE * PS;  // this warp's [16][PS]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + 2 * PAGES + 2 * QE_PAGE * PS * 8);
+  int* info = reinterpret_cast<int*>(bars + 1);  // kind of the item in IN
+  int* pre = reinterpret_cast<int*>(sm + 2 * PAGES + 2 * QE_PAGE * PS * 8 + 32);  // [units + 1]
+  const int units = unit_only >= 0 ? 1 : st.U;
   const int ppw = st.ppw;
-  for (int it = gw; it < (nx + np) * ppw; it += gridDim.y * warps) {
-    const int item = it / ppw, pg = it % ppw;
-    const bool quant = item < nx;
-    const int win = quant ? xlist[ub + item] : plist[ub + item - nx];
+
+  // item prefix over units
+  if (wq == 0) {
+    int carry = 0;
+    for (int c0 = 0; c0 < units; c0 += 32) {
+      const int uu = c0 + lane;
+      const int uid = unit_only >= 0 ? unit_only : uu;
+      int v = uu < units ? (xcount[uid * 4 + 0] + xcount[uid * 4 + 1]) * ppw : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += y;
+      }
+      if (uu < units) pre[uu + 1] = carry + v;
+      carry += __shfl_sync(0xffffffffu, v, 31);
+    }
+    if (lane == 0) {
+      pre[0] = 0;
+      mbar_init(&bars[0], 1);
+      fence_mbar_init();
+    }
+  }
+  __syncthreads();
+  const int total = pre[units];
+  const int n_items = (int)blockIdx.x < total ? (total - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+
+  // Warp 0's lane l holds the addresses of the block's item kb + l (reloaded every 32 items):
+  // kind (0 quantise, 1 promote, -1 invalid), the page and the block.
+  int e_kind = -1;
+  uint4* e_page = nullptr;
+  uint4* e_blk = nullptr;
+  int kb = -32;
+  auto load_items = [&](int base) {
+    kb = base;
+    e_kind = -1;
+    if (base + lane >= n_items) return;
+    const int it = (int)blockIdx.x + (base + lane) * (int)gridDim.x;
+    int lo = 0, hi = units;  // pre[lo] <= it < pre[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (pre[mid] <= it) lo = mid;
+      else hi = mid;
+    }
+    const int u = unit_only >= 0 ? unit_only : lo;
+    const int local = it - pre[lo], item = local / ppw, pg = local % ppw;
+    const int nx = xcount[u * 4 + 0];
+    const size_t ub = (size_t)u * st.Wmax;
+    const int win = item < nx ? xlist[ub + item] : plist[ub + item - nx];
     if (win < 0 || win >= st.Wmax) {
-      if (lane == 0) qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
-      continue;
+      qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
+      return;
     }
     const int slot = st.win_slot[ub + win];
     const int page = st.win_pages[(ub + win) * ppw + pg];
     if (slot < 0 || slot >= st.S || page < 0 || page >= st.P) {
-      if (lane == 0) qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
+      qe_record_error(st.status, QE_ERR_DEVICE_FAULT, u);
+      return;
+    }
+    e_kind = item < nx ? 0 : 1;
+    e_blk = reinterpret_cast<uint4*>(st.slots + ((size_t)u * st.S + slot) * st.slot_bytes + (size_t)pg * BL::BYTES);
+    e_page = reinterpret_cast<uint4*>(st.pages + ((size_t)u * st.P + page) * st.page_bytes);
+  };
+  // Two buffers: IN receives the item's source by bulk copy (the page to quantise, row by row
+  // into the padded layout, or the ledger block to dequantise), OUT holds its result (the block,
+  // or the padded page) until the bulk store has read it. The next item's copy into IN is
+  // issued as soon as both warps are done with the current one, so it overlaps the store.
+  uint4* dst = nullptr;  // warp 0: where the item in OUT goes
+  uint4* dst_next = nullptr;
+  uint32_t par = 0u;     // barrier parity (every thread; the control flow is uniform)
+  bool pend = false;     // warp 0: a copy into IN is in flight
+  uint8_t* in_b = sm;
+  uint8_t* out_b = sm + PAGES;
+  auto issue = [&](int k) {  // warp 0
+    if (k - kb >= 32) load_items(k - k % 32);
+    const int src = k - kb;
+    const int kind = __shfl_sync(0xffffffffu, e_kind, src);
+    uint4* pgp = reinterpret_cast<uint4*>(__shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(e_page), src));
+    uint4* blp = reinterpret_cast<uint4*>(__shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(e_blk), src));
+    dst_next = kind == 0 ? blp : pgp;
+    if (lane == 0) info[0] = kind;
+    if (kind < 0) return;
+    pend = true;
+    fence_proxy_async_smem();
+    if (kind == 0) {
+      if (lane == 0) mbar_arrive_expect_tx(&bars[0], 2 * QE_PAGE * D * 2);
+      __syncwarp();
+      bulk_g2s(in_b + lane * RS * 2, reinterpret_cast<const uint8_t*>(pgp) + lane * D * 2, D * 2, &bars[0]);
+    } else if (lane == 0) {
+      mbar_arrive_expect_tx(&bars[0], BL::BYTES);
+      bulk_g2s(in_b, blp, BL::BYTES, &bars[0]);
+    }
+  };
+
+  if (wq == 0 && n_items > 0) issue(0);
+  bool ok = true;
+  for (int k = 0; k < n_items; ++k) {
+    __syncthreads();  // info[0] of item k is visible; both warps are past item k - 1
+    const int kind = info[0];
+    if (kind < 0) {  // uniform
+      __syncthreads();  // every thread has read info[0] before the next issue rewrites it
+      if (wq == 0 && k + 1 < n_items) issue(k + 1);
       continue;
     }
-    uint4* gblk = reinterpret_cast<uint4*>(st.slots + ((size_t)u * st.S + slot) * st.slot_bytes +
-                                           (size_t)pg * BL::BYTES);
-    uint4* gpage = reinterpret_cast<uint4*>(st.pages + ((size_t)u * st.P + page) * st.page_bytes);
-    __syncwarp();  // the previous item is done with this warp's shared memory
-    if (quant) {
-      for (int i = lane; i < PAGEB / 16; i += 32) reinterpret_cast<uint4*>(pg_s)[i] = gpage[i];
+    const bool okw = mbar_wait_bounded(&bars[0], par, st.status, 3000);
+    if (wq == 0) bulk_wait_read_all();  // OUT is free: the store of item k - 1 has read it
+    ok = __syncthreads_and(okw ? 1 : 0) != 0;
+    if (!ok) break;
+    par ^= 1u;
+    pend = false;
+    dst = dst_next;
+    uint8_t* pg_s = kind == 0 ? in_b : out_b;  // the page image (read or written)
+    uint8_t* img = kind == 0 ? out_b : in_b;   // the block image (written or read)
+    T* rows = reinterpret_cast<T*>(pg_s) + wq * QE_PAGE * RS;  // this warp's 16 rows
+    uint16_t* msc = reinterpret_cast<uint16_t*>(img + (wq ? BL::VS : BL::KS));  // scales
+    uint16_t* mzr = reinterpret_cast<uint16_t*>(img + (wq ? BL::VZ : BL::KZ));  // zeros
+    // position of a (token, group) scale / zero in the block's meta arrays
+    auto s_at = [&](int tok, int g) { return g * QE_PAGE + (wq ? BL::fpos(tok) : BL::ppos(tok)); };
+    auto z_at = [&](int tok, int g) { return wq ? g * QE_PAGE + BL::fpos(tok) : tok * G8 + g; };
+    uint32_t* words = reinterpret_cast<uint32_t*>(img + (wq ? BL::VC : BL::KC)) + lane * WPL;
+    if (kind == 0) {
+      // ---- pass A: each group's min, max, parameters and 16 codes (natural order: element e
+      // at bits 2e of the group's word), once ----
+      uint32_t* nat = reinterpret_cast<uint32_t*>(prm);  // [16 tokens][PS] code words
+#pragma unroll
+      for (int k2 = 0; k2 < NG / 32; ++k2) {
+        const int p = lane + 32 * k2, tok = p / G8, g = p % G8;
+        // the two 16-byte halves, upper half first for g >= G8/2 so that a quarter-warp's loads
+        // fall on distinct banks
+        const uint4* src = reinterpret_cast<const uint4*>(rows + tok * RS + 16 * g);
+        const int h = g >= G8 / 2 ? 1 : 0;
+        const uint4 ha = src[h], hb = src[h ^ 1];
+        const uint4 a = h ? hb : ha, b = h ? ha : hb;  // elements 0..7, 8..15
+        const uint32_t mn = min2_u32<T>(min2_u32<T>(min2_u32<T>(a.x, a.y), min2_u32<T>(a.z, a.w)),
+                                        min2_u32<T>(min2_u32<T>(b.x, b.y), min2_u32<T>(b.z, b.w)));
+        const uint32_t mx = max2_u32<T>(max2_u32<T>(max2_u32<T>(a.x, a.y), max2_u32<T>(a.z, a.w)),
+                                        max2_u32<T>(max2_u32<T>(b.x, b.y), max2_u32<T>(b.z, b.w)));
+        const float fmn = fminf(Elem<T>::lo(mn), Elem<T>::hi(mn)), fmx = fmaxf(Elem<T>::lo(mx), Elem<T>::hi(mx));
+        const Int2Group q(fmn, fmx);
+        msc[s_at(tok, g)] = __half_as_ushort(q.sh);
+        mzr[z_at(tok, g)] = __half_as_ushort(q.zh);
+        const float2 pm = q.fast_params(fmn);
+        const uint32_t e2[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        uint32_t n;
+        uint32_t near = int2_group_codes_fast<T>(e2, pm, n);
+        if (pm.x < 0.f) near = 0xFFFFu;
+        if (near) n = int2_group_codes_exact<T>(n, near, a, b, q.s, q.z);
+        nat[tok * PS + g] = n;
+      }
       __syncwarp();
-      uint32_t kw[WPL], vw[WPL];
+      // ---- pass B: the code words in block placement ----
+      uint32_t w[WPL];
 #pragma unroll
-      for (int j = 0; j < WPL; ++j) kw[j] = vw[j] = 0u;
+      for (int j = 0; j < WPL; ++j) w[j] = 0u;
+      if (wq == 0) {
+        // K: tokens r, 8 + r; elements 2t, 2t + 1, 8 + 2t, 9 + 2t of each group go to bits base,
+        // 16 + base, base + 2, 18 + base of the word of the group pair
 #pragma unroll
-      for (int tb = 0; tb < 2; ++tb) {
-        const int t = r + 8 * tb;
-        const uint32_t* row = reinterpret_cast<const uint32_t*>(Ks + t * D);
+        for (int tb = 0; tb < 2; ++tb) {
 #pragma unroll
-        for (int g = 0; g < G8; ++g) {
-          const uint32_t a = row[8 * g + t4], b = row[8 * g + 4 + t4];
-          const float x0 = Elem<T>::lo(a), x1 = Elem<T>::hi(a), x2 = Elem<T>::lo(b), x3 = Elem<T>::hi(b);
-          float mn = fminf(fminf(x0, x1), fminf(x2, x3)), mx = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
-#pragma unroll
-          for (int o = 1; o < 4; o <<= 1) {
-            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          for (int g = 0; g < G8; ++g) {
+            const uint32_t x = nat[(r + 8 * tb) * PS + g] >> (4 * t4);
+            const uint32_t v = (x & 0x3u) | ((x >> 14) & 0xCu) | ((x << 14) & 0x30000u) | (x & 0xC0000u);
+            w[g >> 1] |= v << (8 * (g & 1) + 4 * tb);
           }
-          const Int2Group q(mn, mx);
-          const int base = 8 * (g & 1) + 4 * tb;  // register i = 2 tb + h at bit 2i of each half
-          kw[g >> 1] |= (q.code(x0) << base) | (q.code(x1) << (16 + base)) | (q.code(x2) << (base + 2)) |
-                        (q.code(x3) << (16 + base + 2));
-          if (t4 == 0) {
-            ks[g * QE_PAGE + BL::ppos(t)] = __half_as_ushort(q.sh);
-            kz[t * G8 + g] = __half_as_ushort(q.zh);
+        }
+      } else {
+        // V: tokens 2t + e + 8 kh; elements r, 8 + r of each group go to bits base, base + 4
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const int tk = 2 * t4 + (kk & 1) + 8 * (kk >> 1);
+#pragma unroll
+          for (int g = 0; g < G8; ++g) {
+            const uint32_t y = (nat[tk * PS + g] >> (2 * r)) & 0x00030003u;
+            w[g >> 1] |= ((y | (y >> 12)) & 0x33u) << (16 * (kk & 1) + 8 * (g & 1) + 2 * (kk >> 1));
           }
         }
       }
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const int tk = 2 * t4 + (kk & 1) + 8 * (kk >> 1);
-        const int e = kk & 1, kh = kk >> 1;
-#pragma unroll
-        for (int g = 0; g < G8; ++g) {
-          const float x0 = Elem<T>::to_f(Vs[tk * D + 16 * g + r]), x1 = Elem<T>::to_f(Vs[tk * D + 16 * g + 8 + r]);
-          float mn = fminf(x0, x1), mx = fmaxf(x0, x1);
-#pragma unroll
-          for (int o = 4; o < 32; o <<= 1) {
-            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-          }
-          const Int2Group q(mn, mx);
-          const int base = 16 * e + 8 * (g & 1) + 2 * kh;  // register i = 2 rh + kh
-          vw[g >> 1] |= (q.code(x0) << base) | (q.code(x1) << (base + 4));
-          if (r == 0) {
-            vs[g * QE_PAGE + BL::fpos(tk)] = __half_as_ushort(q.sh);
-            vz[g * QE_PAGE + BL::fpos(tk)] = __half_as_ushort(q.zh);
-          }
-        }
-      }
-      uint32_t* kc = reinterpret_cast<uint32_t*>(img + BL::KC) + lane * WPL;
-      uint32_t* vc = reinterpret_cast<uint32_t*>(img + BL::VC) + lane * WPL;
-#pragma unroll
-      for (int j = 0; j < WPL; ++j) {
-        kc[j] = kw[j];
-        vc[j] = vw[j];
-      }
-      __syncwarp();
-      for (int i = lane; i < BL::BYTES / 16; i += 32) gblk[i] = reinterpret_cast<const uint4*>(img)[i];
+      for (int j = 0; j < WPL; ++j) words[j] = w[j];
     } else {
-      for (int i = lane; i < BL::BYTES / 16; i += 32) reinterpret_cast<uint4*>(img)[i] = gblk[i];
-      __syncwarp();
-      const uint32_t* kc = reinterpret_cast<const uint32_t*>(img + BL::KC) + lane * WPL;
-      const uint32_t* vc = reinterpret_cast<const uint32_t*>(img + BL::VC) + lane * WPL;
+      // ---- pass A: each group's (s, z) as floats, once ----
 #pragma unroll
-      for (int tb = 0; tb < 2; ++tb) {
-        const int t = r + 8 * tb;
-        uint32_t* row = reinterpret_cast<uint32_t*>(Ks + t * D);
-#pragma unroll
-        for (int g = 0; g < G8; ++g) {
-          const uint32_t x = kc[g >> 1];
-          const int base = 8 * (g & 1) + 4 * tb;
-          const float sc = meta_scale(ks[g * QE_PAGE + BL::ppos(t)]), zc = meta_scale(kz[t * G8 + g]);
-          const float v0 = fmaf((float)((x >> base) & 3u), sc, zc), v1 = fmaf((float)((x >> (16 + base)) & 3u), sc, zc);
-          const float v2 = fmaf((float)((x >> (base + 2)) & 3u), sc, zc);
-          const float v3 = fmaf((float)((x >> (16 + base + 2)) & 3u), sc, zc);
-          row[8 * g + t4] = pack2<T>(v0, v1);
-          row[8 * g + 4 + t4] = pack2<T>(v2, v3);
-        }
-      }
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const int tk = 2 * t4 + (kk & 1) + 8 * (kk >> 1);
-        const int e = kk & 1, kh = kk >> 1;
-#pragma unroll
-        for (int g = 0; g < G8; ++g) {
-          const uint32_t x = vc[g >> 1];
-          const int base = 16 * e + 8 * (g & 1) + 2 * kh;
-          const float sc = meta_scale(vs[g * QE_PAGE + BL::fpos(tk)]), zc = meta_scale(vz[g * QE_PAGE + BL::fpos(tk)]);
-          Vs[tk * D + 16 * g + r] = Elem<T>::from_f(fmaf((float)((x >> base) & 3u), sc, zc));
-          Vs[tk * D + 16 * g + 8 + r] = Elem<T>::from_f(fmaf((float)((x >> (base + 4)) & 3u), sc, zc));
-        }
+      for (int k2 = 0; k2 < NG / 32; ++k2) {
+        const int p = lane + 32 * k2, tok = p / G8, g = p % G8;
+        prm[tok * PS + g] = make_float2(meta_scale(msc[s_at(tok, g)]), meta_scale(mzr[z_at(tok, g)]));
       }
       __syncwarp();
-      for (int i = lane; i < PAGEB / 16; i += 32) gpage[i] = reinterpret_cast<const uint4*>(pg_s)[i];
+      // ---- pass B: f32(code * s + z) in the cache dtype, row-major ----
+      // two codes c as floats: the low bits of 2^23 + c, minus 2^23
+      auto cf2 = [](uint32_t x, int b0, int b1) {
+        return __fadd2_rn(make_float2(__uint_as_float(0x4B000000u | ((x >> b0) & 3u)),
+                                      __uint_as_float(0x4B000000u | ((x >> b1) & 3u))),
+                          make_float2(-8388608.f, -8388608.f));
+      };
+      if (wq == 0) {
+#pragma unroll
+        for (int tb = 0; tb < 2; ++tb) {
+          const int t = r + 8 * tb;
+          uint32_t* row = reinterpret_cast<uint32_t*>(rows + t * RS);
+#pragma unroll
+          for (int g = 0; g < G8; ++g) {
+            const uint32_t x = words[g >> 1];
+            const int base = 8 * (g & 1) + 4 * tb;
+            const float2 pm = prm[t * PS + g];
+            const float2 s2 = make_float2(pm.x, pm.x), z2 = make_float2(pm.y, pm.y);
+            const float2 va = __ffma2_rn(cf2(x, base, 16 + base), s2, z2);
+            const float2 vb = __ffma2_rn(cf2(x, base + 2, 16 + base + 2), s2, z2);
+            row[8 * g + t4] = pack2<T>(va.x, va.y);
+            row[8 * g + 4 + t4] = pack2<T>(vb.x, vb.y);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const int tk = 2 * t4 + (kk & 1) + 8 * (kk >> 1);
+          const int e = kk & 1, kh = kk >> 1;
+#pragma unroll
+          for (int g = 0; g < G8; ++g) {
+            const uint32_t x = words[g >> 1];
+            const int base = 16 * e + 8 * (g & 1) + 2 * kh;
+            const float2 pm = prm[tk * PS + g];
+            const float2 v = __ffma2_rn(cf2(x, base, base + 4), make_float2(pm.x, pm.x), make_float2(pm.y, pm.y));
+            rows[tk * RS + 16 * g + r] = Elem<T>::from_f(v.x);
+            rows[tk * RS + 16 * g + 8 + r] = Elem<T>::from_f(v.y);
+          }
+        }
+      }
+    }
+    // the result leaves by bulk stores once both warps' writes are visible to the async proxy;
+    // then IN is free for the next item's copy
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (wq == 0) {
+      if (kind == 0) {
+        if (lane == 0) bulk_s2g(dst, img, BL::BYTES);
+      } else {
+        bulk_s2g(reinterpret_cast<uint8_t*>(dst) + lane * D * 2, pg_s + lane * RS * 2, D * 2);
+      }
+      bulk_commit();
+      if (k + 1 < n_items) issue(k + 1);
     }
   }
+  if (!ok && wq == 0 && pend) mbar_wait_bounded(&bars[0], par, st.status, 3001);  // a copy still in flight
+  bulk_wait_all();
 }
 
 // A window's ledger entry in the row-major form of qe_int2_quantize: one warp per 16-token
@@ -734,27 +929,29 @@ __global__ void int2_quantize_kernel(const T* x, int rows, uint8_t* codes, uint3
 template <typename T, int D>
 void launch_apply(const DevState& st, const qe_ctx* c, int unit_only, cudaStream_t s) {
   const int units = unit_only >= 0 ? 1 : st.U;
-  // 8 warps per block, one warp per (window, page); a routing event moves at most F + Q
-  // windows into a new tier (host-given transitions at most Wmax)
+  // a routing event moves at most F + Q windows of a unit into a new tier (host-given
+  // transitions at most Wmax): that bounds the items; the grid is one wave of resident blocks
   int wins = unit_only >= 0 ? st.Wmax : c->cfg.full_windows + c->cfg.int2_windows;
   if (wins > st.Wmax) wins = st.Wmax;
-  // 4 warps per block, one (window, page) item per warp at a time; a routing event moves at most
-  // F + Q windows into a new tier (host-given transitions at most Wmax). The blocks of a unit
-  // loop over its items, so one wave of about four blocks per SM covers any event.
-  int per_unit = (wins * st.ppw + 3) / 4;
+  const size_t smem = apply_smem_bytes<D>(units);
   static QeOnce once;
-  static int sms_of[QE_MAX_DEVICES];
+  static int wave_of[QE_MAX_DEVICES];
   int dev = 0;
   if (qe_once_per_device(once, &dev, [](int d) {
-        QE_CUDA_TRY(cudaDeviceGetAttribute(&sms_of[d], cudaDevAttrMultiProcessorCount, d));
+        QE_CUDA_TRY(cudaFuncSetAttribute(apply_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         96 * 1024));
+        int sms = 0, per_sm = 0;
+        QE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, d));
+        QE_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, apply_kernel<T, D>, kApplyThreads,
+                                                                  apply_smem_bytes<D>(64)));
+        wave_of[d] = sms * (per_sm > 0 ? per_sm : 1);
         return QE_OK;
       }) != QE_OK)
-    sms_of[dev] = 148;
-  const int wave = (4 * sms_of[dev] + units - 1) / units;
-  if (per_unit > wave) per_unit = wave;
-  if (per_unit < 1) per_unit = 1;
-  apply_kernel<T, D><<<dim3(units, per_unit), 128, 0, s>>>(st, c->xlist, c->plist, c->xcount,
-                                                            unit_only);
+    wave_of[dev] = 148 * 8;
+  const long long max_items = (long long)units * wins * st.ppw;
+  int blocks = (int)(max_items < wave_of[dev] ? max_items : wave_of[dev]);
+  if (blocks < 1) blocks = 1;
+  apply_kernel<T, D><<<blocks, kApplyThreads, smem, s>>>(st, c->xlist, c->plist, c->xcount, unit_only);
 }
 
 int apply_dispatch(const qe_ctx* c, const DevState& st, int unit_only, cudaStream_t s) {
