@@ -9,7 +9,7 @@
 // One routing event: (1) for every layer (one context each) a kernel appends each live window's
 // cumulative mass, perturbation and flat position (layer, kv head, window) to its sequence's
 // candidate list (a unit claims its range with one atomic add, so the list holds live windows
-// only, in no particular order); (2) one CTA per sequence selects Full = TwoStage(L, F) and
+// only, in no particular order); (2) one thread-block cluster per sequence selects Full = TwoStage(L, F) and
 // INT2 = TwoStage(L minus Full, Q) over the list by exact radix selections on 64-bit keys (the
 // score's order-preserving bits, then the complement of the flat position, so equal scores go to
 // the lower position and the result does not depend on the list order) and writes each chosen
@@ -21,7 +21,6 @@
 
 namespace {
 
-constexpr int kSelThreadsG = 1024;
 constexpr uint8_t kPick = 2, kFull = 4, kInt2 = 8;
 
 struct GlobArgs {
@@ -73,39 +72,85 @@ __global__ void glob_keygen_kernel(DevState st, int layer, GlobArgs g) {
   }
 }
 
+// The selection of one sequence runs on one thread-block cluster of C CTAs (C up to 16): CTA r
+// owns the r-th C-th of the candidate list. Every count and radix histogram is formed per CTA in
+// shared memory and summed over the cluster through distributed shared memory, so every CTA
+// takes the same decisions; flags are read and written only by the CTA that owns the entry.
+constexpr int kSelThreadsG = 512;
+constexpr int kSelMaxCluster = 16;
+
 struct SelSh {
-  unsigned int hist[256];
+  unsigned int hist[256];  // this CTA's histogram of the current digit (read by the cluster)
+  unsigned int tot[256];   // the cluster's histogram
+  int cnt;                 // this CTA's member count (read by the cluster)
   int ctl[3];
   int red[kSelThreadsG / 32];
 };
 
-__device__ int block_count(int v, SelSh& sh) {
+__device__ __forceinline__ void sel_cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t sel_ld_cluster(const uint32_t* local, uint32_t rank) {
+  uint32_t a, v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(local)), "r"(rank));
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t sel_cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t sel_cluster_size() {
+  uint32_t n;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(n));
+  return n;
+}
+
+// the cluster-wide sum of v over every thread of every CTA
+__device__ int cluster_count(int v, SelSh& sh) {
 #pragma unroll
   for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   if ((threadIdx.x & 31) == 0) sh.red[threadIdx.x >> 5] = v;
   __syncthreads();
+  if (threadIdx.x == 0) {
+    int t = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += sh.red[w];
+    sh.cnt = t;
+  }
+  sel_cluster_sync();
   int t = 0;
-  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += sh.red[w];
-  __syncthreads();
+  const uint32_t C = sel_cluster_size();
+  for (uint32_t r = 0; r < C; ++r) t += (int)sel_ld_cluster(reinterpret_cast<const uint32_t*>(&sh.cnt), r);
+  sel_cluster_sync();  // every CTA has read the counts before they change
   return t;
 }
 
-// Threshold of the k largest keys (1 <= k <= number of non-zero keys; non-zero keys distinct):
-// key(i) is among them iff key(i) != 0 and (key(i) >> shift) >= (prefix >> shift). Most
-// significant 8-bit digit first; a pass ends the search when the digit that holds the k-th key
-// holds exactly the keys still needed.
+// Threshold of the k largest keys over the cluster's entries (1 <= k <= number of non-zero
+// keys; non-zero keys distinct): key(i) is among them iff key(i) != 0 and
+// (key(i) >> shift) >= (prefix >> shift). Most significant 8-bit digit first; a pass ends the
+// search when the digit that holds the k-th key holds exactly the keys still needed. [i0, i1)
+// are this CTA's entries.
 template <typename KeyFn>
-__device__ void topk_threshold(int n, int k, KeyFn key, SelSh& sh, unsigned long long* prefix_out, int* shift_out) {
+__device__ void topk_threshold(int i0, int i1, int k, KeyFn key, SelSh& sh, unsigned long long* prefix_out,
+                               int* shift_out) {
   unsigned long long prefix = 0;
   int shift = 64;
+  const uint32_t C = sel_cluster_size();
   for (int pass = 0; pass < 8; ++pass) {
     const int sft = 56 - 8 * pass;
     for (int d = threadIdx.x; d < 256; d += blockDim.x) sh.hist[d] = 0;
     __syncthreads();
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) {
       const unsigned long long kk = key(i);
       if (kk != 0 && (shift == 64 || (kk >> shift) == (prefix >> shift)))
         atomicAdd(&sh.hist[(kk >> sft) & 255], 1u);
+    }
+    sel_cluster_sync();
+    for (int d = threadIdx.x; d < 256; d += blockDim.x) {
+      uint32_t t = 0;
+      for (uint32_t r = 0; r < C; ++r) t += sel_ld_cluster(&sh.hist[d], r);
+      sh.tot[d] = t;
     }
     __syncthreads();
     if (threadIdx.x < 32) {
@@ -114,7 +159,7 @@ __device__ void topk_threshold(int n, int k, KeyFn key, SelSh& sh, unsigned long
       uint32_t c[8], loc = 0;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        c[j] = sh.hist[255 - 8 * l - j];
+        c[j] = sh.tot[255 - 8 * l - j];
         loc += c[j];
       }
       uint32_t inc = loc;
@@ -139,7 +184,7 @@ __device__ void topk_threshold(int n, int k, KeyFn key, SelSh& sh, unsigned long
     prefix |= (unsigned long long)sh.ctl[0] << sft;
     shift = sft;
     const bool done = sh.ctl[2] == k;
-    __syncthreads();
+    sel_cluster_sync();  // every CTA has read the histograms before the next pass clears them
     if (done) break;
   }
   *prefix_out = prefix;
@@ -148,13 +193,13 @@ __device__ void topk_threshold(int n, int k, KeyFn key, SelSh& sh, unsigned long
 
 // TwoStage(members, b) with stage-1 share b1: the chosen candidates get `out` in their flag
 template <typename MemberFn>
-__device__ void two_stage_global(int n, int b, int b1, MemberFn member, const float* mass, const float* pert,
-                                 const int32_t* pos, uint8_t* flag, uint8_t out, SelSh& sh) {
+__device__ void two_stage_global(int i0, int i1, int b, int b1, MemberFn member, const float* mass,
+                                 const float* pert, const int32_t* pos, uint8_t* flag, uint8_t out, SelSh& sh) {
   int cnt_local = 0;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) cnt_local += member(i) ? 1 : 0;
-  const int cnt = block_count(cnt_local, sh);
+  for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) cnt_local += member(i) ? 1 : 0;
+  const int cnt = cluster_count(cnt_local, sh);
   if (cnt <= b) {
-    for (int i = threadIdx.x; i < n; i += blockDim.x)
+    for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x)
       if (member(i)) flag[i] |= out;
     __syncthreads();
     return;
@@ -163,8 +208,8 @@ __device__ void two_stage_global(int n, int b, int b1, MemberFn member, const fl
   int S;
   if (b1 > 0) {
     auto k1 = [&](int i) -> unsigned long long { return member(i) ? cand_key(mass[i], pos[i]) : 0ull; };
-    topk_threshold(n, b1, k1, sh, &P, &S);
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    topk_threshold(i0, i1, b1, k1, sh, &P, &S);
+    for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) {
       const unsigned long long kk = k1(i);
       if (kk != 0 && (kk >> S) >= (P >> S)) flag[i] |= kPick;
     }
@@ -174,34 +219,74 @@ __device__ void two_stage_global(int n, int b, int b1, MemberFn member, const fl
     auto k2 = [&](int i) -> unsigned long long {
       return (member(i) && !(flag[i] & kPick)) ? cand_key(pert[i], pos[i]) : 0ull;
     };
-    topk_threshold(n, b - b1, k2, sh, &P, &S);
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    topk_threshold(i0, i1, b - b1, k2, sh, &P, &S);
+    for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) {
       const unsigned long long kk = k2(i);
       if (kk != 0 && (kk >> S) >= (P >> S)) flag[i] |= out;
     }
     __syncthreads();
   }
-  for (int i = threadIdx.x; i < n; i += blockDim.x)
+  for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x)
     if (flag[i] & kPick) flag[i] = (uint8_t)((flag[i] & ~kPick) | out);
   __syncthreads();
 }
 
+// one cluster per sequence: grid = B * C CTAs, cluster size C
 __global__ void __launch_bounds__(kSelThreadsG) glob_select_kernel(GlobArgs g, int F, int F1, int Q, int Q1) {
   __shared__ SelSh sh;
-  const size_t base = (size_t)blockIdx.x * g.n;
+  const uint32_t C = sel_cluster_size(), rank = sel_cluster_rank();
+  const int seq = blockIdx.x / C;
+  const size_t base = (size_t)seq * g.n;
   const float* mass = g.mass + base;
   const float* pert = g.pert + base;
   const int32_t* pos = g.pos + base;
   uint8_t* flag = g.flag + base;
   uint8_t* decided = g.decided + base;
-  const int n = g.count[blockIdx.x];  // the list holds live windows only
-  two_stage_global(n, F, F1, [&](int) { return true; }, mass, pert, pos, flag, kFull, sh);
-  two_stage_global(n, Q, Q1, [&](int i) { return (flag[i] & kFull) == 0; }, mass, pert, pos, flag, kInt2, sh);
+  const int n = g.count[seq];  // the list holds live windows only
+  const int i0 = (int)((long long)n * rank / C), i1 = (int)((long long)n * (rank + 1) / C);
+  two_stage_global(i0, i1, F, F1, [&](int) { return true; }, mass, pert, pos, flag, kFull, sh);
+  two_stage_global(i0, i1, Q, Q1, [&](int i) { return (flag[i] & kFull) == 0; }, mass, pert, pos, flag, kInt2, sh);
   // chosen tiers by flat position (every other position was set to EVICTED beforehand)
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+  for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) {
     const uint8_t f = flag[i];
     decided[pos[i]] = (f & kFull) ? QE_TIER_FULL : ((f & kInt2) ? QE_TIER_INT2 : QE_TIER_EVICTED);
   }
+}
+
+// Cluster size of the selection: the largest C <= 16 whose B clusters can be resident at once
+// (all of them, when possible), at least 1. Found once per device.
+int glob_select_cluster(int B) {
+  static QeOnce once;
+  static int resident[QE_MAX_DEVICES][kSelMaxCluster + 1];
+  int dev = 0;
+  if (qe_once_per_device(once, &dev, [](int d) {
+        QE_CUDA_TRY(cudaFuncSetAttribute(glob_select_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+        for (int C = 1; C <= kSelMaxCluster; ++C) {
+          cudaLaunchConfig_t qc = {};
+          cudaLaunchAttribute qa[1];
+          qa[0].id = cudaLaunchAttributeClusterDimension;
+          qa[0].val.clusterDim.x = C;
+          qa[0].val.clusterDim.y = 1;
+          qa[0].val.clusterDim.z = 1;
+          qc.gridDim = dim3(C);
+          qc.blockDim = dim3(kSelThreadsG);
+          qc.attrs = qa;
+          qc.numAttrs = 1;
+          int nc = 0;
+          if (cudaOccupancyMaxActiveClusters(&nc, glob_select_kernel, &qc) != cudaSuccess) {
+            (void)cudaGetLastError();
+            nc = 0;
+          }
+          resident[d][C] = nc;
+        }
+        return QE_OK;
+      }) != QE_OK)
+    return 1;
+  for (int C = kSelMaxCluster; C > 1; --C)
+    if (resident[dev][C] >= B) return C;
+  for (int C = kSelMaxCluster; C > 1; --C)
+    if (resident[dev][C] >= 1) return C;
+  return 1;
 }
 
 struct GlobLayout {
@@ -269,8 +354,21 @@ extern "C" QE_API int qe_route_windows_global(qe_ctx* const* ctxs, int n_layers,
     glob_keygen_kernel<<<s.U, 256, 0, st>>>(s, l, g);
     QE_CUDA_TRY(cudaGetLastError());
   }
-  glob_select_kernel<<<B, kSelThreadsG, 0, st>>>(g, full_windows, F1, int2_windows, Q1);
-  QE_CUDA_TRY(cudaGetLastError());
+  {
+    const int C = glob_select_cluster(B);
+    cudaLaunchConfig_t lc = {};
+    cudaLaunchAttribute la[1];
+    la[0].id = cudaLaunchAttributeClusterDimension;
+    la[0].val.clusterDim.x = C;
+    la[0].val.clusterDim.y = 1;
+    la[0].val.clusterDim.z = 1;
+    lc.gridDim = dim3(B * C);
+    lc.blockDim = dim3(kSelThreadsG);
+    lc.stream = st;
+    lc.attrs = la;
+    lc.numAttrs = 1;
+    QE_CUDA_TRY(cudaLaunchKernelEx(&lc, glob_select_kernel, g, full_windows, F1, int2_windows, Q1));
+  }
   for (int l = 0; l < n_layers; ++l) {
     qe_ctx* c = ctxs[l];
     const int e = launch_route_decided(c, g.decided + (size_t)l * Hkv * Wmax, (size_t)n, st);
