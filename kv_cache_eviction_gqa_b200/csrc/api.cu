@@ -45,7 +45,7 @@ void scratch_sizes(const qe_config* c, size_t (&sz)[kScratchParts]) {
   sz[4] = U * 4 * 4;
   sz[5] = Wmax * 4;
   sz[6] = (size_t)c->Hkv * c->B * w * D * 2;
-  sz[7] = (size_t)c->Hkv * c->B * w * G * 4;
+  sz[7] = (size_t)kTailNormParts * c->Hkv * c->B * w * G * 4;
 }
 
 int finalize_tail(qe_ctx* c, cudaStream_t st) {

@@ -17,6 +17,8 @@
 // floats of one window's score partials in the decode kernel's scratch: {max, sum p, sum p n}
 // per query head of the group, relative to that max
 __host__ __device__ constexpr int win_part_floats(int D, int G) { return (void)D, 3 * G; }
+// column parts of a completed window's V W_O norms (partial row sums, added by finalize)
+constexpr int kTailNormParts = 8;
 #define QE_MAX_G 8
 #define QE_MAX_SPLITS 64
 
@@ -52,7 +54,7 @@ struct qe_ctx {
   int32_t* xcount;      // [U][4] counts: quantise, promote
   int32_t* host_ids;    // [max_windows] staging for host-given window ids
   uint8_t* tailV;       // [Hkv][B][window][D] dtype: V of the tail window (for its norms)
-  float* tail_norm;     // [Hkv][B*window][G] norms of a just-completed window
+  float* tail_norm;     // [kTailNormParts][Hkv][B*window][G] partial norms of a just-completed window
   // typed views of the state arrays
   template <typename T> T* at(size_t off) const { return reinterpret_cast<T*>(ws + off); }
 };
@@ -223,7 +225,9 @@ int launch_vwo(const void* V, int n_groups, int rows, int D, int dtype, const vo
                cudaStream_t st);
 int launch_vwo_tc(const void* V, int n_groups, int rows, int D, int dtype, const void* W_O, int Hq,
                   int Hkv, int hidden, float* out, long long out_group_stride, int32_t* status,
-                  cudaStream_t st);
+                  cudaStream_t st, int nparts = 1, long long part_stride = 0);
+// column parts for the tensor-core launch of few rows (1 when the launch already fills the GPU)
+int vwo_tc_parts(int n_groups, int rows, int Hq, int Hkv, int hidden, int max_parts, int sms);
 int launch_int2_quantize(const void* x, int T, int D, int dtype, uint8_t* codes, uint32_t* meta,
                          cudaStream_t st);
 int launch_ledger_read(qe_ctx* c, int unit, int win, uint8_t* codes_k, uint32_t* meta_k, uint8_t* codes_v,

@@ -134,13 +134,16 @@ __global__ void append_kernel(DevState st, const uint4* k_new, const uint4* v_ne
 // the tail window completed: store its norms, fold the deferred perturbation score,
 // and move it into the full tier as a routing candidate
 // ---------------------------------------------------------------------------
-__global__ void finalize_kernel(DevState st, const float* tail_norm, int tw) {
+__global__ void finalize_kernel(DevState st, const float* tail_norm, int nparts, long long pstride, int tw) {
   const int u = blockIdx.x, b = u / st.Hkv, kvh = u % st.Hkv, w = st.window, G = st.G;
   __shared__ float red[32];
   float acc = 0.f;
   for (int i = threadIdx.x; i < w * G; i += blockDim.x) {
     const int t = i / G, h = i % G;
-    const float nrm = tail_norm[(((size_t)kvh * st.B + b) * w + t) * G + h];
+    // the column parts' partial row sums, added in part order
+    const float* tn = tail_norm + (((size_t)kvh * st.B + b) * w + t) * G + h;
+    float nrm = tn[0];
+    for (int pp = 1; pp < nparts; ++pp) nrm += tn[pp * pstride];
     st.norms[((size_t)u * st.norm_pitch + (size_t)tw * w + t) * G + h] = nrm;
     float* tp = st.tail_p + (size_t)u * w * G + i;
     acc += *tp * nrm;
@@ -1026,10 +1029,28 @@ int launch_append(qe_ctx* c, const void* k, const void* v, cudaStream_t s) {
 int launch_finalize(qe_ctx* c, int tw, cudaStream_t s) {
   DevState st = make_state(c);
   const int rows = c->cfg.B * c->cfg.window;
-  int e = launch_vwo(c->tailV, c->cfg.Hkv, rows, c->cfg.D, c->cfg.dtype, c->W_O, c->cfg.Hq,
-                     c->cfg.Hkv, c->cfg.hidden, c->tail_norm, (long long)rows * c->G, st.status, s);
+  const long long gstride = (long long)rows * c->G, pstride = (long long)c->cfg.Hkv * gstride;
+  // A completed window is a few row blocks: on the tensor-core path each head's hidden columns
+  // are split into parts so that the launch covers the SMs; finalize adds the parts in order.
+  int nparts = 1, e;
+  if (c->cfg.hidden % 128 == 0) {
+    static QeOnce once;
+    static int sms_of[QE_MAX_DEVICES];
+    int dev = 0;
+    if (qe_once_per_device(once, &dev, [](int d) {
+          QE_CUDA_TRY(cudaDeviceGetAttribute(&sms_of[d], cudaDevAttrMultiProcessorCount, d));
+          return QE_OK;
+        }) != QE_OK)
+      sms_of[dev] = 148;
+    nparts = vwo_tc_parts(c->cfg.Hkv, rows, c->cfg.Hq, c->cfg.Hkv, c->cfg.hidden, kTailNormParts, sms_of[dev]);
+    e = launch_vwo_tc(c->tailV, c->cfg.Hkv, rows, c->cfg.D, c->cfg.dtype, c->W_O, c->cfg.Hq, c->cfg.Hkv,
+                      c->cfg.hidden, c->tail_norm, gstride, st.status, s, nparts, pstride);
+  } else {
+    e = launch_vwo(c->tailV, c->cfg.Hkv, rows, c->cfg.D, c->cfg.dtype, c->W_O, c->cfg.Hq, c->cfg.Hkv,
+                   c->cfg.hidden, c->tail_norm, gstride, st.status, s);
+  }
   if (e) return e;
-  finalize_kernel<<<st.U, 128, 0, s>>>(st, c->tail_norm, tw);
+  finalize_kernel<<<st.U, 128, 0, s>>>(st, c->tail_norm, nparts, pstride, tw);
   return cudaGetLastError() == cudaSuccess ? QE_OK : QE_ERR_CUDA;
 }
 

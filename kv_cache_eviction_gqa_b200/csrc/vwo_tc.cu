@@ -40,6 +40,8 @@ struct VwoArgs {
   int mpairs;           // ceil(rows / 256)
   int nsplit;           // N-tile ranges per (group, row block)
   int ntot;             // G * ntiles_per_head
+  int nparts;           // column parts per head (each writes its own partial row sums)
+  long long pstride;    // elements between the partial outputs of consecutive parts
   int atomic;           // several CTAs add into one output element (never set: splits are whole heads)
   int32_t* status;
 };
@@ -160,7 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (n % a.ntiles_per_head == a.ntiles_per_head - 1 || i == NT - 1) {
         const int j = n / a.ntiles_per_head;
         if (r < a.rows) {
-          float* o = a.out + (size_t)g * a.ogs + (size_t)r * a.G + j;
+          float* o = a.out + (size_t)(split % a.nparts) * a.pstride + (size_t)g * a.ogs + (size_t)r * a.G + j;
           if (a.atomic) atomicAdd(o, rowsum);
           else *o = rowsum;
         }
@@ -178,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D, bool BF16>
 int launch_tc(const void* V, int n_groups, int rows, const void* W, int Hq, int Hkv, int hidden, float* out,
-              long long ogs, int32_t* status, cudaStream_t s) {
+              long long ogs, int nparts, long long pstride, int32_t* status, cudaStream_t s) {
   constexpr int KB = D / 64;
   // at least 120 KB so that two CTAs never share an SM (each holds all 512 TMEM columns)
   constexpr size_t SMEM_USE = 1024 + (size_t)kMT * KB * kBM * 128 + (size_t)kNST * (kBN / 64) * D * 128 + 256;
@@ -217,7 +219,14 @@ int launch_tc(const void* V, int n_groups, int rows, const void* W, int Hq, int 
   int nsplit = 1;
   for (int d = 1; d <= a.G; ++d)
     if (a.G % d == 0 && d <= want) nsplit = d;
+  // with column parts, every head's tiles are split into nparts ranges of their own
+  if (nparts > 1) {
+    if (a.ntiles_per_head % nparts) return QE_ERR_UNSUPPORTED_SHAPE;
+    nsplit = a.G * nparts;
+  }
   a.nsplit = nsplit;
+  a.nparts = nparts > 1 ? nparts : 1;
+  a.pstride = pstride;
   a.atomic = 0;
   a.status = status;
   kern<<<(unsigned)(items * nsplit), kThreads, SMEM, s>>>(tmV, tmW, a);
@@ -228,13 +237,25 @@ int launch_tc(const void* V, int n_groups, int rows, const void* W, int Hq, int 
 
 // Tensor-core path for hidden % 128 == 0; status may be NULL (errors then go nowhere).
 int launch_vwo_tc(const void* V, int n_groups, int rows, int D, int dtype, const void* W_O, int Hq, int Hkv,
-                  int hidden, float* out, long long ogs, int32_t* status, cudaStream_t s) {
+                  int hidden, float* out, long long ogs, int32_t* status, cudaStream_t s, int nparts,
+                  long long pstride) {
   if (hidden % kBN) return QE_ERR_UNSUPPORTED_SHAPE;
   if ((long long)n_groups * rows > 0x7fffffffll) return QE_ERR_UNSUPPORTED_SHAPE;
   const bool bf = dtype == QE_BF16;
   if (D == 128)
-    return bf ? launch_tc<128, true>(V, n_groups, rows, W_O, Hq, Hkv, hidden, out, ogs, status, s)
-              : launch_tc<128, false>(V, n_groups, rows, W_O, Hq, Hkv, hidden, out, ogs, status, s);
-  return bf ? launch_tc<64, true>(V, n_groups, rows, W_O, Hq, Hkv, hidden, out, ogs, status, s)
-            : launch_tc<64, false>(V, n_groups, rows, W_O, Hq, Hkv, hidden, out, ogs, status, s);
+    return bf ? launch_tc<128, true>(V, n_groups, rows, W_O, Hq, Hkv, hidden, out, ogs, nparts, pstride, status, s)
+              : launch_tc<128, false>(V, n_groups, rows, W_O, Hq, Hkv, hidden, out, ogs, nparts, pstride, status, s);
+  return bf ? launch_tc<64, true>(V, n_groups, rows, W_O, Hq, Hkv, hidden, out, ogs, nparts, pstride, status, s)
+            : launch_tc<64, false>(V, n_groups, rows, W_O, Hq, Hkv, hidden, out, ogs, nparts, pstride, status, s);
+}
+
+// Column parts for a launch of few row blocks: the largest power of two that divides the
+// hidden tiles of a head and keeps items * G * parts within one wave of the SMs.
+int vwo_tc_parts(int n_groups, int rows, int Hq, int Hkv, int hidden, int max_parts, int sms) {
+  if (hidden % kBN) return 1;
+  const long long items = (long long)n_groups * ((rows + kMT * kBM - 1) / (kMT * kBM));
+  const int G = Hq / Hkv, tph = hidden / kBN;
+  int P = 1;
+  while (2 * P <= max_parts && tph % (2 * P) == 0 && items * G * 2 * P <= sms) P *= 2;
+  return P;
 }
