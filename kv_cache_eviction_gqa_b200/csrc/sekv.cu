@@ -241,52 +241,140 @@ __global__ void __launch_bounds__(kSekvWarps * 32) sekv_attend_kernel(SekvAttend
 #pragma unroll
     for (int j = 0; j < DPL; ++j) acc[h][j] = 0.f;
   }
-  // one key/value pair with its log2-domain score offset
-  auto take = [&](const float (&kx)[DPL], const float (&vx)[DPL], float bias2) {
+  // KB keys at a time: the lane's partial dot products of the G x KB (head, key) pairs are
+  // summed over the warp by a reduce-scatter (a lane ends with one full sum) followed by an
+  // all-gather (every lane then holds every score), NP - 1 shuffles each instead of five per
+  // pair; then every lane updates the same online-softmax state of each head once per batch.
+  // bias: the log2-domain score offset of each key (-inf for an unused slot).
+  constexpr int KB = 4, NPAIR = G * KB;
+  constexpr int NP = NPAIR <= 4 ? 4 : (NPAIR <= 8 ? 8 : (NPAIR <= 16 ? 16 : 32));
+  static_assert(NPAIR <= 32, "at most 32 (head, key) pairs per batch");
+  auto take_batch = [&](const float (&kx)[KB][DPL], const float (&vx)[KB][DPL], const float (&bias)[KB]) {
+    float d[NP];
+#pragma unroll
+    for (int v = 0; v < NP; ++v) {
+      float t = 0.f;
+      if (v < NPAIR) {
+#pragma unroll
+        for (int j = 0; j < DPL; ++j) t = fmaf(qv[v / KB][j], kx[v % KB][j], t);
+      }
+      d[v] = t;
+    }
+    // reduce-scatter: at the level of partner distance o the lane keeps the lower or upper half
+    // of its block (by bit o of its lane index) and adds the partner's copy of that half
+#pragma unroll
+    for (int lvl = 0; lvl < 5; ++lvl) {
+      const int o = 16 >> lvl, width = NP >> lvl;
+      if (width > 1) {
+        const int half = width >> 1;
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < half; ++i) {
+          const float send = up ? d[i] : d[i + half];
+          const float keep = up ? d[i + half] : d[i];
+          d[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+      } else {
+        d[0] += __shfl_xor_sync(0xffffffffu, d[0], o);
+      }
+    }
+    // all-gather, the same levels in reverse: blocks double until every lane holds all NP sums
+#pragma unroll
+    for (int lvl = 4; lvl >= 0; --lvl) {
+      const int o = 16 >> lvl, width = NP >> lvl;
+      if (width > 1) {
+        const int half = width >> 1;
+        const bool up = (lane & o) != 0;
+        float r[NP / 2];
+#pragma unroll
+        for (int i = 0; i < half; ++i) r[i] = __shfl_xor_sync(0xffffffffu, d[i], o);
+#pragma unroll
+        for (int i = 0; i < half; ++i) {
+          const float mine = d[i];
+          d[i] = up ? r[i] : mine;
+          d[i + half] = up ? mine : r[i];
+        }
+      }
+    }
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      float d = 0.f;
+      float sc[KB], mx = m[h];
 #pragma unroll
-      for (int j = 0; j < DPL; ++j) d = fmaf(qv[h][j], kx[j], d);
-      const float s = fmaf(warp_allsum(d), a.scale_log2, bias2);
-      if (s > m[h]) {
-        const float f = ex2s(m[h] - s);
-        l[h] *= f;
-#pragma unroll
-        for (int j = 0; j < DPL; ++j) acc[h][j] *= f;
-        m[h] = s;
+      for (int k = 0; k < KB; ++k) {
+        sc[k] = fmaf(d[h * KB + k], a.scale_log2, bias[k]);
+        mx = fmaxf(mx, sc[k]);
       }
-      const float p = ex2s(s - m[h]);
-      l[h] += p;
+      const float f = ex2s(m[h] - mx);
+      float p[KB], ps = 0.f;
 #pragma unroll
-      for (int j = 0; j < DPL; ++j) acc[h][j] = fmaf(p, vx[j], acc[h][j]);
+      for (int k = 0; k < KB; ++k) {
+        p[k] = ex2s(sc[k] - mx);
+        ps += p[k];
+      }
+      l[h] = fmaf(l[h], f, ps);
+#pragma unroll
+      for (int j = 0; j < DPL; ++j) {
+        float t = acc[h][j] * f;
+#pragma unroll
+        for (int k = 0; k < KB; ++k) t = fmaf(p[k], vx[k][j], t);
+        acc[h][j] = t;
+      }
+      m[h] = mx;
     }
   };
-  auto take_token = [&](int t) {
-    float kx[DPL], vx[DPL];
-    load_dims<T, DPL>(Kb + (size_t)t * D, lane, kx);
-    load_dims<T, DPL>(Vb + (size_t)t * D, lane, vx);
-    take(kx, vx, 0.f);
+  auto clear_slot = [&](float (&kx)[DPL], float (&vx)[DPL], float& bias) {
+#pragma unroll
+    for (int j = 0; j < DPL; ++j) kx[j] = vx[j] = 0.f;
+    bias = -INFINITY;
   };
-  for (int it = i0 + warp; it < i1; it += kSekvWarps) {
-    if (it < A) {
-      take_token(a.anchor_pos[(size_t)b * a.n + it]);
-    } else {
-      const int i = it - A;
-      const int s = a.span_start[(size_t)b * a.cap + i], e = a.span_end[(size_t)b * a.cap + i];
-      if (a.expanded[(size_t)u * a.cap + i]) {
-        for (int t = s; t < e; ++t) take_token(t);
+  // pass 1: the single-key items (anchors, summaries of spans that are not expanded), KB of
+  // the warp's items per batch
+  for (int base = i0 + warp; base < i1; base += KB * kSekvWarps) {
+    float kx[KB][DPL], vx[KB][DPL], bias[KB];
+#pragma unroll
+    for (int k = 0; k < KB; ++k) {
+      clear_slot(kx[k], vx[k], bias[k]);
+      const int it = base + k * kSekvWarps;
+      if (it >= i1) continue;
+      if (it < A) {
+        const int t = a.anchor_pos[(size_t)b * a.n + it];
+        load_dims<T, DPL>(Kb + (size_t)t * D, lane, kx[k]);
+        load_dims<T, DPL>(Vb + (size_t)t * D, lane, vx[k]);
+        bias[k] = 0.f;
       } else {
-        float kx[DPL], vx[DPL];
+        const int i = it - A;
+        if (a.expanded[(size_t)u * a.cap + i]) continue;
+        const int s = a.span_start[(size_t)b * a.cap + i], e = a.span_end[(size_t)b * a.cap + i];
         const float* kr = a.kbar + ((size_t)u * a.cap + i) * D + lane * DPL;
         const float* vr = a.vbar + ((size_t)u * a.cap + i) * D + lane * DPL;
 #pragma unroll
         for (int j = 0; j < DPL; ++j) {
-          kx[j] = kr[j];
-          vx[j] = vr[j];
+          kx[k][j] = kr[j];
+          vx[k][j] = vr[j];
         }
-        take(kx, vx, log2f((float)(e - s)));  // the summary stands for e - s tokens
+        bias[k] = log2f((float)(e - s));  // the summary stands for e - s tokens
       }
+    }
+    take_batch(kx, vx, bias);
+  }
+  // pass 2: the tokens of the warp's expanded spans, KB per batch
+  for (int it = i0 + warp; it < i1; it += kSekvWarps) {
+    if (it < A) continue;
+    const int i = it - A;
+    if (!a.expanded[(size_t)u * a.cap + i]) continue;
+    const int s = a.span_start[(size_t)b * a.cap + i], e = a.span_end[(size_t)b * a.cap + i];
+    for (int t0 = s; t0 < e; t0 += KB) {
+      float kx[KB][DPL], vx[KB][DPL], bias[KB];
+#pragma unroll
+      for (int k = 0; k < KB; ++k) {
+        clear_slot(kx[k], vx[k], bias[k]);
+        if (t0 + k < e) {
+          load_dims<T, DPL>(Kb + (size_t)(t0 + k) * D, lane, kx[k]);
+          load_dims<T, DPL>(Vb + (size_t)(t0 + k) * D, lane, vx[k]);
+          bias[k] = 0.f;
+        }
+      }
+      take_batch(kx, vx, bias);
     }
   }
   // merge the warps into the CTA partial

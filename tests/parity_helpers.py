@@ -6,6 +6,8 @@ every decode step the checked units are compared:
 * attention output: max |o_gpu - o_ref| / max |o_ref| per (batch, query head) <= 2e-3;
 * cumulative window mass and perturbation: |d| / max(|ref|, 1e-30) <= 1e-4 per window
   (the tail window's perturbation is folded in when it completes, so it is compared then);
+* routing: per-event counters (promotions, first and reused demotions, evictions, tier sizes,
+  stage-1 share of the mass) equal those of the oracle's transitions;
 * routing: tier decisions must match, except items whose score lies within 1e-4 relative
   of a selection boundary (near-ties: counted and reported). When every mismatch is a
   near-tie the oracle adopts the GPU's tiers for those windows so histories stay aligned;
@@ -40,6 +42,7 @@ def torch_dtype(name):
 class ParityReport:
     steps: int = 0
     max_out_err: float = 0.0
+    stats_checked: int = 0
     max_mass_err: float = 0.0
     max_pert_err: float = 0.0
     route_events: int = 0
@@ -210,6 +213,7 @@ def run_decode_parity(cfg: W.DecodeConfig, check_units=None, steps=None, max_spl
                 assert got_full == full_g, f"step {s} unit {u}: full tier is not the two-stage pick"
                 assert got_int2 == int2_g, f"step {s} unit {u}: INT2 tier is not the two-stage pick"
                 ledger_before = set(unit.ledger.keys())
+                tier_o_before = unit.tier.copy()
                 new = unit.route()
                 mism = [w for w, t in new.items() if int(g_tier[u, w]) != t]
                 if mism:
@@ -247,6 +251,34 @@ def run_decode_parity(cfg: W.DecodeConfig, check_units=None, steps=None, max_spl
                         rep.promoted_checked += 1
                 if diag:
                     o_hist[u].append(unit.tier.copy())
+                # the event's counters (qe_route_windows' per-unit route_stats) against the
+                # oracle's transitions: promotions, first demotions, demotions that reuse a
+                # ledger entry, evictions, tier sizes, and the stage-1 share of the candidates'
+                # mass (x 1e6) when the selection had no near-tie
+                rs = st["route_stats"][u].cpu().numpy()
+                ob, oa = tier_o_before, unit.tier
+                live_b = (ob == O.FULL) | (ob == O.INT2)
+                demoted = np.nonzero((ob == O.FULL) & (oa == O.INT2))[0]
+                exp_stats = {
+                    "promoted": int(np.sum((ob == O.INT2) & (oa == O.FULL))),
+                    "first demotions": int(sum(1 for w in demoted if int(w) not in ledger_before)),
+                    "reused demotions": int(sum(1 for w in demoted if int(w) in ledger_before)),
+                    "evicted": int(np.sum(live_b & (oa == O.EVICTED))),
+                    "full windows": int(np.sum(oa == O.FULL)),
+                    "int2 windows": int(np.sum(oa == O.INT2)),
+                }
+                got_stats = dict(zip(exp_stats, (int(rs[0]), int(rs[1]), int(rs[2]), int(rs[3]), int(rs[4]),
+                                                 int(rs[5]))))
+                assert got_stats == exp_stats, f"step {s} unit {u}: route_stats {got_stats} vs {exp_stats}"
+                if not mism:
+                    L_ = unit.last_route["L"]
+                    f1_ = unit.last_route["full"][0]
+                    tot = float(np.sum(unit.mass[L_]))
+                    share = round(1e6 * float(np.sum(unit.mass[f1_])) / tot) if tot > 0 else 0
+                    # float32 sums of masses that match the oracle's to ~1e-6 relative
+                    assert abs(int(rs[7]) - share) <= 2 + 1e-5 * share, \
+                        f"step {s} unit {u}: stage-1 share {rs[7]} vs {share}"
+                rep.stats_checked += 1
                 # tiers agree after replay
                 live_o = {int(w): int(unit.tier[w]) for w in np.nonzero(unit.tier != O.EVICTED)[0]}
                 for w, t in live_o.items():
