@@ -54,6 +54,36 @@ __device__ int block_excl_scan(int v, int* buf, int* total) {
   return r;
 }
 
+// Exclusive prefix sums of N per-thread counts at once (one pass of barriers for all of them);
+// buf holds at least N * 33 ints.
+template <int N>
+__device__ void block_excl_scan_n(const int (&v)[N], int* buf, int (&excl)[N], int (&total)[N]) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int inc[N];
+#pragma unroll
+  for (int j = 0; j < N; ++j) {
+    inc[j] = warp_incl_scan(v[j], lane);
+    if (lane == 31) buf[j * 33 + warp] = inc[j];
+  }
+  __syncthreads();
+  if (warp == 0) {
+#pragma unroll
+    for (int j = 0; j < N; ++j) {
+      const int x = lane < nw ? buf[j * 33 + lane] : 0;
+      const int xi = warp_incl_scan(x, lane);
+      if (lane < nw) buf[j * 33 + lane] = xi - x;
+      if (lane == 31) buf[j * 33 + 32] = xi;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < N; ++j) {
+    excl[j] = buf[j * 33 + warp] + inc[j] - v[j];
+    total[j] = buf[j * 33 + 32];
+  }
+  __syncthreads();
+}
+
 __device__ float block_sum(float v, float* buf) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
 #pragma unroll
@@ -340,6 +370,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
   uint8_t* sel = inset + st.Wmax;
   uint8_t* s1 = sel + st.Wmax;
   __shared__ int ibuf[33];
+  __shared__ int sbuf[9 * 33];
   __shared__ float fbuf[32];
   __shared__ int hist[256];
   __shared__ int s_abort;
@@ -409,26 +440,27 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
   // each thread owns a contiguous run of candidates so prefix sums stay in candidate order
   const int per = (n + blockDim.x - 1) / blockDim.x;
   const int i0 = threadIdx.x * per, i1 = min(n, i0 + per);
-  int c_tp = 0, c_ts = 0, c_gp = 0, c_gs = 0, c_pr = 0, c_nf = 0, c_nq = 0;
+  // counts per thread: pages taken, new ledger slots, pages given back, slots given back,
+  // promotions, full, INT2, demotions (first or reused), evictions
+  int cnt[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
   for (int i = i0; i < i1; ++i) {
     const int o = oldt[i], t = newt[i];
     const int slot = st.win_slot[ub + cand[i]];
-    c_tp += (o == QE_TIER_INT2 && t == QE_TIER_FULL) ? st.ppw : 0;
-    c_ts += (o == QE_TIER_FULL && t == QE_TIER_INT2 && slot < 0);
-    c_gp += (o == QE_TIER_FULL && t != QE_TIER_FULL) ? st.ppw : 0;
-    c_gs += (t == QE_TIER_EVICTED && slot >= 0);
-    c_pr += (o == QE_TIER_INT2 && t == QE_TIER_FULL);
-    c_nf += (t == QE_TIER_FULL);
-    c_nq += (t == QE_TIER_INT2);
+    cnt[0] += (o == QE_TIER_INT2 && t == QE_TIER_FULL) ? st.ppw : 0;
+    cnt[1] += (o == QE_TIER_FULL && t == QE_TIER_INT2 && slot < 0);
+    cnt[2] += (o == QE_TIER_FULL && t != QE_TIER_FULL) ? st.ppw : 0;
+    cnt[3] += (t == QE_TIER_EVICTED && slot >= 0);
+    cnt[4] += (o == QE_TIER_INT2 && t == QE_TIER_FULL);
+    cnt[5] += (t == QE_TIER_FULL);
+    cnt[6] += (t == QE_TIER_INT2);
+    cnt[7] += (o == QE_TIER_FULL && t == QE_TIER_INT2);
+    cnt[8] += (t == QE_TIER_EVICTED);
   }
-  int T_tp, T_ts, T_gp, T_gs, T_pr, T_nf, T_nq;
-  int o_tp = block_excl_scan(c_tp, ibuf, &T_tp);
-  int o_ts = block_excl_scan(c_ts, ibuf, &T_ts);
-  int o_gp = block_excl_scan(c_gp, ibuf, &T_gp);
-  int o_gs = block_excl_scan(c_gs, ibuf, &T_gs);
-  int o_pr = block_excl_scan(c_pr, ibuf, &T_pr);
-  int o_nf = block_excl_scan(c_nf, ibuf, &T_nf);
-  int o_nq = block_excl_scan(c_nq, ibuf, &T_nq);
+  int ex[9], tot[9];
+  block_excl_scan_n<9>(cnt, sbuf, ex, tot);
+  const int o_tp = ex[0], o_ts = ex[1], o_gp = ex[2], o_gs = ex[3], o_pr = ex[4], o_nf = ex[5], o_nq = ex[6];
+  const int T_tp = tot[0], T_ts = tot[1], T_gp = tot[2], T_gs = tot[3], T_pr = tot[4], T_nf = tot[5],
+            T_nq = tot[6], T_re = tot[7], T_ev = tot[8];
   const int ptop = st.stacks[u * 4 + 0], stop = st.stacks[u * 4 + 1];
   if (threadIdx.x == 0) {
     if (T_tp > ptop) {
@@ -503,14 +535,6 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
     rs[7] = all_mass > 0.f ? (int)llrintf(1e6f * stage1_mass / all_mass) : 0;
   }
   // demotions that reused an entry, evictions
-  int c_re = 0, c_ev = 0;
-  for (int i = i0; i < i1; ++i) {
-    c_re += (oldt[i] == QE_TIER_FULL && newt[i] == QE_TIER_INT2);
-    c_ev += (newt[i] == QE_TIER_EVICTED);
-  }
-  int T_re, T_ev;
-  block_excl_scan(c_re, ibuf, &T_re);
-  block_excl_scan(c_ev, ibuf, &T_ev);
   if (threadIdx.x == 0) {
     st.route_stats[u * 8 + 2] = T_re - T_ts;
     st.route_stats[u * 8 + 3] = T_ev;
