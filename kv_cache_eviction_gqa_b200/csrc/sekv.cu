@@ -19,16 +19,16 @@
 #include <math.h>
 
 #include "qe_internal.cuh"
+#include "warp_mma.cuh"
 
 namespace {
 
 constexpr int kSekvWarps = 4;      // warps per CTA (gate, summarize, attend)
 constexpr int kSekvMaxSplits = 32;
-constexpr int kSekvTargetCtas = 1184;  // 148 SMs x 8
 constexpr int kSekvSpanBlocks = 64;    // CTAs per unit for the per-span kernels (grid-stride over spans)
 
 struct SekvLayout {
-  size_t counts, anchor_pos, span_start, span_end, kbar, vbar, expanded, part_ml, part_o, total;
+  size_t counts, anchor_pos, span_start, span_end, kbar, vbar, expanded, part_ml, part_o, tok, sums, lcount, total;
   int cap;  // spans per sequence at most: (n + 1) / 2 (two spans are separated by an anchor)
 };
 
@@ -46,14 +46,13 @@ SekvLayout sekv_layout(int B, int Hkv, int n, int D, int G) {
   L.expanded = up(L.vbar + U * L.cap * D * 4);
   L.part_ml = up(L.expanded + U * L.cap);
   L.part_o = up(L.part_ml + U * kSekvMaxSplits * G * 2 * 4);
-  L.total = up(L.part_o + U * kSekvMaxSplits * G * (size_t)D * 4);
+  L.tok = up(L.part_o + U * kSekvMaxSplits * G * (size_t)D * 4);  // [U][n] tokens attended one by one
+  L.sums = up(L.tok + U * (size_t)n * 4);                          // [U][cap] spans attended by summary
+  L.lcount = up(L.sums + U * (size_t)L.cap * 4);                   // [U][2] their counts
+  L.total = up(L.lcount + U * 2 * 4);
   return L;
 }
 
-int sekv_splits(int U) {
-  int S = (kSekvTargetCtas + U - 1) / U;
-  return S < 1 ? 1 : (S > kSekvMaxSplits ? kSekvMaxSplits : S);
-}
 
 __device__ __forceinline__ float ex2s(float x) {
   float y;
@@ -87,6 +86,35 @@ __device__ int block_scan01(int v, int* wsum, int* total) {
   }
   __syncthreads();
   const int r = wsum[warp] + in_warp;
+  *total = wsum[32];
+  __syncthreads();
+  return r;
+}
+
+// exclusive prefix sum of a non-negative int over the block (blockDim.x = 1024); *total gets the sum
+__device__ int block_scan_int(int v, int* wsum, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  if (lane == 31) wsum[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    const int x = lane < (int)(blockDim.x >> 5) ? wsum[lane] : 0;
+    int xi = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, xi, o);
+      if (lane >= o) xi += y;
+    }
+    wsum[lane] = xi - x;
+    if (lane == 31) wsum[32] = xi;
+  }
+  __syncthreads();
+  const int r = wsum[warp] + inc - v;
   *total = wsum[32];
   __syncthreads();
   return r;
@@ -202,6 +230,50 @@ __global__ void __launch_bounds__(kSekvWarps * 32)
   }
 }
 
+// Per step, one CTA per unit: the tokens attended one by one (the anchors, then every token of
+// each expanded span, in position order within a span) and the spans attended by their summary.
+__global__ void __launch_bounds__(1024) sekv_lists_kernel(const int32_t* __restrict__ counts,
+                                                          const int32_t* __restrict__ anchor_pos,
+                                                          const int32_t* __restrict__ span_start,
+                                                          const int32_t* __restrict__ span_end,
+                                                          const uint8_t* __restrict__ expanded, int n, int cap,
+                                                          int Hkv, int32_t* tok, int32_t* sums, int32_t* lcount) {
+  const int u = blockIdx.x, b = u / Hkv;
+  const int A = counts[b * 2 + 0], NS = counts[b * 2 + 1];
+  int32_t* tl = tok + (size_t)u * n;
+  int32_t* sl = sums + (size_t)u * cap;
+  for (int i = threadIdx.x; i < A; i += blockDim.x) tl[i] = anchor_pos[(size_t)b * n + i];
+  __shared__ int wsum[33];
+  int carry_t = A, carry_s = 0;
+  for (int base = 0; base < NS; base += blockDim.x) {
+    const int i = base + threadIdx.x;
+    const bool in = i < NS;
+    const bool ex = in && expanded[(size_t)u * cap + i];
+    const int s0 = ex ? span_start[(size_t)b * cap + i] : 0, e0 = ex ? span_end[(size_t)b * cap + i] : 0;
+    int tt, ts;
+    const int it = block_scan_int(e0 - s0, wsum, &tt);
+    const int is = block_scan01(in && !ex ? 1 : 0, wsum, &ts);
+    for (int t = s0; t < e0; ++t) tl[carry_t + it + (t - s0)] = t;
+    if (in && !ex) sl[carry_s + is] = i;
+    carry_t += tt;
+    carry_s += ts;
+  }
+  if (threadIdx.x == 0) {
+    lcount[u * 2 + 0] = carry_t;
+    lcount[u * 2 + 1] = carry_s;
+  }
+}
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, int bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 struct SekvAttendArgs {
   const void* q;
   const void* K;
@@ -215,24 +287,154 @@ struct SekvAttendArgs {
   const uint8_t* expanded;
   float* part_ml;  // [U][S][G][2]
   float* part_o;   // [U][S][G][D]
+  const int32_t* tok;     // [U][n] tokens attended one by one
+  const int32_t* sums;    // [U][cap] spans attended by summary
+  const int32_t* lcount;  // [U][2]
   int n, cap, Hq, Hkv, S;
   float scale_log2;
 };
 
+// One split of a unit: its share of the unit's tokens attended one by one, 16 per tile on the
+// warp-level tensor cores, and its share of the unit's span summaries on the CUDA cores.
+// Tokens: a warp gathers the K and V rows of 16 tokens with cp.async into a 128-byte-swizzled
+// tile (two stages, the next tile's gather overlapping the current one), S^T = K Q^T with the
+// tokens as MMA rows and the query heads as columns, an online softmax per lane for its two
+// heads, P split into a 16-bit high part and its residual and turned by movmatrix into the B
+// fragment of O^T = V^T P^T. Summaries: four per warp step, the G x 4 (head, summary) dot
+// products summed over the warp by a reduce-scatter and an all-gather, the score raised by
+// log2|S|. The two partial states of a warp are merged, then the warps, then (next kernel) the
+// splits.
 template <typename T, int DPL, int G>
 __global__ void __launch_bounds__(kSekvWarps * 32) sekv_attend_kernel(SekvAttendArgs a) {
-  constexpr int D = 32 * DPL;
+  constexpr int D = 32 * DPL, G8 = D / 16;
+  constexpr int TILE = 2 * QE_PAGE * D * 2;  // K rows, then V rows, of 16 tokens
+  constexpr int CPR = D / 8;                 // 16-byte chunks per row
+  static_assert(G <= 8, "a warp's MMA columns hold at most 8 query heads");
+  extern __shared__ __align__(128) uint8_t sekv_smem[];
   const int u = blockIdx.x / a.S, split = blockIdx.x % a.S;
   const int b = u / a.Hkv, kvh = u % a.Hkv;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int A = a.counts[b * 2 + 0], NS = a.counts[b * 2 + 1], I = A + NS;
-  const int i0 = (int)((long long)I * split / a.S), i1 = (int)((long long)I * (split + 1) / a.S);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g8 = lane >> 2, t4 = lane & 3;
+  const int ntok = a.lcount[u * 2 + 0], nsum = a.lcount[u * 2 + 1];
+  const int NT = (ntok + 15) / 16;
+  const int ta = (int)((long long)NT * split / a.S), tbn = (int)((long long)NT * (split + 1) / a.S);
+  const int sa = (int)((long long)nsum * split / a.S), sbn = (int)((long long)nsum * (split + 1) / a.S);
   const T* Kb = reinterpret_cast<const T*>(a.K) + (size_t)u * a.n * D;
   const T* Vb = reinterpret_cast<const T*>(a.V) + (size_t)u * a.n * D;
+  const int32_t* tl = a.tok + (size_t)u * a.n;
+  const T* qbase = reinterpret_cast<const T*>(a.q) + ((size_t)b * a.Hq + (size_t)kvh * G) * D;
+  // q for the summaries: lane l holds elements l*DPL .. of every head
   float qv[G][DPL];
 #pragma unroll
-  for (int h = 0; h < G; ++h)
-    load_dims<T, DPL>(reinterpret_cast<const T*>(a.q) + ((size_t)b * a.Hq + (size_t)kvh * G + h) * D, lane, qv[h]);
+  for (int h = 0; h < G; ++h) load_dims<T, DPL>(qbase + (size_t)h * D, lane, qv[h]);
+  // q as the B operand of S^T = K Q^T: head g8's elements 16m + 2t4, +1 and 16m + 8 + 2t4, +1
+  uint32_t qb[G8][2];
+  {
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(qbase + (size_t)(g8 < G ? g8 : 0) * D);
+#pragma unroll
+    for (int m = 0; m < G8; ++m) {
+      qb[m][0] = g8 < G ? qrow[m * 8 + t4] : 0u;
+      qb[m][1] = g8 < G ? qrow[m * 8 + 4 + t4] : 0u;
+    }
+  }
+
+  // ---- tokens on the tensor cores ----
+  const int h0 = 2 * t4, h1 = 2 * t4 + 1;
+  const float hm0 = h0 < G ? 1.f : 0.f, hm1 = h1 < G ? 1.f : 0.f;
+  float m0 = -1e30f, m1 = -1e30f, l0 = 0.f, l1 = 0.f;
+  float oacc[G8][4];
+#pragma unroll
+  for (int m = 0; m < G8; ++m) oacc[m][0] = oacc[m][1] = oacc[m][2] = oacc[m][3] = 0.f;
+  uint8_t* ring = sekv_smem + warp * 2 * TILE;
+  // gather tile t into stage st: row r is token tl[16 t + r]; rows past the list are zero-filled
+  auto gather = [&](int t, int st) {
+    const int row = t * 16 + (lane & 15);
+    const int pos = (lane < 16 && row < ntok) ? tl[row] : -1;
+    uint8_t* dst = ring + st * TILE;
+#pragma unroll
+    for (int k = 0; k < 16 * CPR / 32; ++k) {
+      const int c = lane + 32 * k, r = c / CPR, cc = c % CPR;
+      const int p = __shfl_sync(0xffffffffu, pos, r);
+      const size_t off = (size_t)(p >= 0 ? p : 0) * D + cc * 8;
+      const int bytes = p >= 0 ? 16 : 0;
+      cp_async16(dst + swz<D>(0, r, cc * 8), Kb + off, bytes);
+      cp_async16(dst + swz<D>(1, r, cc * 8), Vb + off, bytes);
+    }
+    cp_async_commit();
+  };
+  auto transpose_pair = [](uint32_t x) {
+    uint32_t y;
+    asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+  };
+  const float sl2 = a.scale_log2;
+  int stg = 0;
+  if (ta + warp < tbn) gather(ta + warp, 0);
+  for (int t = ta + warp; t < tbn; t += kSekvWarps, stg ^= 1) {
+    if (t + kSekvWarps < tbn) {
+      gather(t + kSekvWarps, stg ^ 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncwarp();
+    const uint8_t* tile = ring + stg * TILE;
+    const int valid = min(16, ntok - t * 16);
+    float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int m = 0; m < G8; ++m) {
+      uint32_t ka[4];
+      ldsm_x4(ka, tile + swz<D>(0, ((lane >> 3) & 1) * 8 + (lane & 7), m * 16 + (lane >> 4) * 8));
+      if (m & 1) MmaOp<T>::run(c1, ka[0], ka[1], ka[2], ka[3], qb[m][0], qb[m][1]);
+      else MmaOp<T>::run(c0, ka[0], ka[1], ka[2], ka[3], qb[m][0], qb[m][1]);
+    }
+    // lane (g8, t4): tokens g8 (slots 0, 1) and 8 + g8 (slots 2, 3), heads h0 (0, 2) and h1 (1, 3)
+    float sc[4] = {(c0[0] + c1[0]) * sl2, (c0[1] + c1[1]) * sl2, (c0[2] + c1[2]) * sl2, (c0[3] + c1[3]) * sl2};
+    if (g8 >= valid) sc[0] = sc[1] = -INFINITY;
+    if (g8 + 8 >= valid) sc[2] = sc[3] = -INFINITY;
+    float x0 = fmaxf(sc[0], sc[2]), x1 = fmaxf(sc[1], sc[3]);
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, o));
+      x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, o));
+    }
+    const float n0 = fmaxf(m0, x0), n1 = fmaxf(m1, x1);
+    const float f0 = ex2s(m0 - n0), f1 = ex2s(m1 - n1);
+    l0 *= f0;
+    l1 *= f1;
+#pragma unroll
+    for (int m = 0; m < G8; ++m) {
+      oacc[m][0] *= f0;
+      oacc[m][1] *= f1;
+      oacc[m][2] *= f0;
+      oacc[m][3] *= f1;
+    }
+    m0 = n0;
+    m1 = n1;
+    const float p0 = hm0 * ex2s(sc[0] - m0), p1 = hm1 * ex2s(sc[1] - m1);
+    const float p2 = hm0 * ex2s(sc[2] - m0), p3 = hm1 * ex2s(sc[3] - m1);
+    l0 += p0 + p2;
+    l1 += p1 + p3;
+    uint32_t xh0, xl0, xh1, xl1;
+    MmaOp<T>::split(p0, p1, xh0, xl0);
+    MmaOp<T>::split(p2, p3, xh1, xl1);
+    const uint32_t ph0 = transpose_pair(xh0), pl0 = transpose_pair(xl0);
+    const uint32_t ph1 = transpose_pair(xh1), pl1 = transpose_pair(xl1);
+#pragma unroll
+    for (int m = 0; m < G8; ++m) {
+      uint32_t va[4];
+      ldsm_x4_t(va, tile + swz<D>(1, ((lane >> 4) << 3) + (lane & 7), m * 16 + ((lane >> 3) & 1) * 8));
+      MmaOp<T>::run(oacc[m], va[0], va[1], va[2], va[3], ph0, ph1);
+      MmaOp<T>::run(oacc[m], va[0], va[1], va[2], va[3], pl0, pl1);
+    }
+    __syncwarp();
+  }
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+  }
+
+  // ---- span summaries on the CUDA cores ----
   float m[G], l[G], acc[G][DPL];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
@@ -327,80 +529,73 @@ __global__ void __launch_bounds__(kSekvWarps * 32) sekv_attend_kernel(SekvAttend
     for (int j = 0; j < DPL; ++j) kx[j] = vx[j] = 0.f;
     bias = -INFINITY;
   };
-  // pass 1: the single-key items (anchors, summaries of spans that are not expanded), KB of
-  // the warp's items per batch
-  for (int base = i0 + warp; base < i1; base += KB * kSekvWarps) {
+  for (int base = sa + warp; base < sbn; base += KB * kSekvWarps) {
     float kx[KB][DPL], vx[KB][DPL], bias[KB];
 #pragma unroll
     for (int k = 0; k < KB; ++k) {
       clear_slot(kx[k], vx[k], bias[k]);
       const int it = base + k * kSekvWarps;
-      if (it >= i1) continue;
-      if (it < A) {
-        const int t = a.anchor_pos[(size_t)b * a.n + it];
-        load_dims<T, DPL>(Kb + (size_t)t * D, lane, kx[k]);
-        load_dims<T, DPL>(Vb + (size_t)t * D, lane, vx[k]);
-        bias[k] = 0.f;
-      } else {
-        const int i = it - A;
-        if (a.expanded[(size_t)u * a.cap + i]) continue;
-        const int s = a.span_start[(size_t)b * a.cap + i], e = a.span_end[(size_t)b * a.cap + i];
-        const float* kr = a.kbar + ((size_t)u * a.cap + i) * D + lane * DPL;
-        const float* vr = a.vbar + ((size_t)u * a.cap + i) * D + lane * DPL;
+      if (it >= sbn) continue;
+      const int i = a.sums[(size_t)u * a.cap + it];
+      const int s0 = a.span_start[(size_t)b * a.cap + i], e0 = a.span_end[(size_t)b * a.cap + i];
+      const float* kr = a.kbar + ((size_t)u * a.cap + i) * D + lane * DPL;
+      const float* vr = a.vbar + ((size_t)u * a.cap + i) * D + lane * DPL;
 #pragma unroll
-        for (int j = 0; j < DPL; ++j) {
-          kx[k][j] = kr[j];
-          vx[k][j] = vr[j];
-        }
-        bias[k] = log2f((float)(e - s));  // the summary stands for e - s tokens
+      for (int j = 0; j < DPL; ++j) {
+        kx[k][j] = kr[j];
+        vx[k][j] = vr[j];
       }
+      bias[k] = log2f((float)(e0 - s0));  // the summary stands for e0 - s0 tokens
     }
     take_batch(kx, vx, bias);
   }
-  // pass 2: the tokens of the warp's expanded spans, KB per batch
-  for (int it = i0 + warp; it < i1; it += kSekvWarps) {
-    if (it < A) continue;
-    const int i = it - A;
-    if (!a.expanded[(size_t)u * a.cap + i]) continue;
-    const int s = a.span_start[(size_t)b * a.cap + i], e = a.span_end[(size_t)b * a.cap + i];
-    for (int t0 = s; t0 < e; t0 += KB) {
-      float kx[KB][DPL], vx[KB][DPL], bias[KB];
-#pragma unroll
-      for (int k = 0; k < KB; ++k) {
-        clear_slot(kx[k], vx[k], bias[k]);
-        if (t0 + k < e) {
-          load_dims<T, DPL>(Kb + (size_t)(t0 + k) * D, lane, kx[k]);
-          load_dims<T, DPL>(Vb + (size_t)(t0 + k) * D, lane, vx[k]);
-          bias[k] = 0.f;
-        }
-      }
-      take_batch(kx, vx, bias);
-    }
-  }
-  // merge the warps into the CTA partial
-  __shared__ float wm[kSekvWarps][G], wl[kSekvWarps][G];
-  __shared__ float wo[kSekvWarps][G][D];
+
+  // ---- merge the warp's two partial states, then the warps, into the CTA partial ----
+  __syncthreads();  // every warp is done with its gather ring, which now holds the merge
+  float* wm = reinterpret_cast<float*>(sekv_smem);  // [kSekvWarps][G]
+  float* wl = wm + kSekvWarps * G;                   // [kSekvWarps][G]
+  float* wo = wl + kSekvWarps * G;                   // [kSekvWarps][G][D]
+  float* my = wo + (size_t)warp * G * D;
+  float fa0 = 0.f, fa1 = 0.f;
 #pragma unroll
   for (int h = 0; h < G; ++h) {
+    const float mA = __shfl_sync(0xffffffffu, (h & 1) ? m1 : m0, h >> 1);
+    const float lA = __shfl_sync(0xffffffffu, (h & 1) ? l1 : l0, h >> 1);
+    const float M = fmaxf(mA, m[h]);
+    const float fA = ex2s(mA - M), fB = ex2s(m[h] - M);
     if (lane == 0) {
-      wm[warp][h] = m[h];
-      wl[warp][h] = l[h];
+      wm[warp * G + h] = M;
+      wl[warp * G + h] = lA * fA + l[h] * fB;
     }
 #pragma unroll
-    for (int j = 0; j < DPL; ++j) wo[warp][h][lane * DPL + j] = acc[h][j];
+    for (int j = 0; j < DPL; ++j) my[h * D + lane * DPL + j] = acc[h][j] * fB;
+    if (h == h0) fa0 = fA;
+    if (h == h1) fa1 = fA;
+  }
+  __syncwarp();
+#pragma unroll
+  for (int mm = 0; mm < G8; ++mm) {
+    if (h0 < G) {
+      my[h0 * D + mm * 16 + g8] += oacc[mm][0] * fa0;
+      my[h0 * D + mm * 16 + 8 + g8] += oacc[mm][2] * fa0;
+    }
+    if (h1 < G) {
+      my[h1 * D + mm * 16 + g8] += oacc[mm][1] * fa1;
+      my[h1 * D + mm * 16 + 8 + g8] += oacc[mm][3] * fa1;
+    }
   }
   __syncthreads();
   for (int x = threadIdx.x; x < G * D; x += blockDim.x) {
     const int h = x / D, d = x % D;
-    float M = wm[0][h];
+    float M = wm[h];
 #pragma unroll
-    for (int w = 1; w < kSekvWarps; ++w) M = fmaxf(M, wm[w][h]);
+    for (int w = 1; w < kSekvWarps; ++w) M = fmaxf(M, wm[w * G + h]);
     float L = 0.f, O = 0.f;
 #pragma unroll
     for (int w = 0; w < kSekvWarps; ++w) {
-      const float f = ex2s(wm[w][h] - M);
-      L = fmaf(wl[w][h], f, L);
-      O = fmaf(wo[w][h][d], f, O);
+      const float f = ex2s(wm[w * G + h] - M);
+      L = fmaf(wl[w * G + h], f, L);
+      O = fmaf(wo[((size_t)w * G + h) * D + d], f, O);
     }
     const size_t pi = ((size_t)u * a.S + split) * G + h;
     a.part_o[pi * D + d] = O;
@@ -455,7 +650,26 @@ template <typename T, int DPL, int G>
 int launch_attend(const void* q, const void* K, const void* V, int B, int Hq, int Hkv, int n, float theta,
                   uint8_t* st, const SekvLayout& L, float* out, cudaStream_t s) {
   constexpr int D = 32 * DPL;
-  const int U = B * Hkv, S = sekv_splits(U);
+  constexpr size_t SMEM = (size_t)kSekvWarps * 2 * (2 * QE_PAGE * D * 2);  // two gather stages per warp
+  static_assert((2 + D) * kSekvWarps * G * 4 <= SMEM, "the warp merge fits in the gather rings");
+  const int U = B * Hkv;
+  // one wave of resident CTAs over the units (found once per instantiation and device)
+  static QeOnce once;
+  static int resident_of[QE_MAX_DEVICES];
+  int dev = 0;
+  if (int e = qe_once_per_device(once, &dev, [](int d) {
+        QE_CUDA_TRY(cudaFuncSetAttribute(sekv_attend_kernel<T, DPL, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)SMEM));
+        int sms = 0, per_sm = 0;
+        QE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, d));
+        QE_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sekv_attend_kernel<T, DPL, G>,
+                                                                  kSekvWarps * 32, SMEM));
+        resident_of[d] = sms * (per_sm > 0 ? per_sm : 1);
+        return QE_OK;
+      }))
+    return e;
+  int S = resident_of[dev] / U;
+  S = S < 1 ? 1 : (S > kSekvMaxSplits ? kSekvMaxSplits : S);
   const int32_t* counts = reinterpret_cast<const int32_t*>(st + L.counts);
   const float* kbar = reinterpret_cast<const float*>(st + L.kbar);
   uint8_t* expanded = st + L.expanded;
@@ -465,7 +679,18 @@ int launch_attend(const void* q, const void* K, const void* V, int B, int Hq, in
                                                                 kbar, (float)(1.0 / sqrt((double)D)), theta,
                                                                 expanded);
   QE_CUDA_TRY(cudaGetLastError());
+  int32_t* tok = reinterpret_cast<int32_t*>(st + L.tok);
+  int32_t* sums = reinterpret_cast<int32_t*>(st + L.sums);
+  int32_t* lcount = reinterpret_cast<int32_t*>(st + L.lcount);
+  sekv_lists_kernel<<<U, 1024, 0, s>>>(counts, reinterpret_cast<const int32_t*>(st + L.anchor_pos),
+                                       reinterpret_cast<const int32_t*>(st + L.span_start),
+                                       reinterpret_cast<const int32_t*>(st + L.span_end), expanded, n, L.cap, Hkv,
+                                       tok, sums, lcount);
+  QE_CUDA_TRY(cudaGetLastError());
   SekvAttendArgs a{};
+  a.tok = tok;
+  a.sums = sums;
+  a.lcount = lcount;
   a.q = q;
   a.K = K;
   a.V = V;
@@ -484,7 +709,7 @@ int launch_attend(const void* q, const void* K, const void* V, int B, int Hq, in
   a.Hkv = Hkv;
   a.S = S;
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
-  sekv_attend_kernel<T, DPL, G><<<U * S, kSekvWarps * 32, 0, s>>>(a);
+  sekv_attend_kernel<T, DPL, G><<<U * S, kSekvWarps * 32, SMEM, s>>>(a);
   QE_CUDA_TRY(cudaGetLastError());
   sekv_combine_kernel<<<dim3(U, G), 128, 0, s>>>(a.part_ml, a.part_o, S, G, D, Hq, Hkv, out);
   QE_CUDA_TRY(cudaGetLastError());
