@@ -60,10 +60,45 @@ __device__ __forceinline__ float ex2s(float x) {
   return y;
 }
 
-__device__ __forceinline__ float warp_allsum(float v) {
+// NP (a power of two, 4..32) values per lane summed over the warp: a reduce-scatter (at partner
+// distance o the lane keeps the lower or upper half of its block, by bit o of its index, and adds
+// the partner's copy of that half) and then an all-gather (the same levels in reverse), so every
+// lane ends with all NP sums; NP - 1 shuffles each way instead of five per value.
+template <int NP>
+__device__ __forceinline__ void warp_sum_all(float (&d)[NP], int lane) {
 #pragma unroll
-  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
+  for (int lvl = 0; lvl < 5; ++lvl) {
+    const int o = 16 >> lvl, width = NP >> lvl;
+    if (width > 1) {
+      const int half = width >> 1;
+      const bool up = (lane & o) != 0;
+#pragma unroll
+      for (int i = 0; i < half; ++i) {
+        const float send = up ? d[i] : d[i + half];
+        const float keep = up ? d[i + half] : d[i];
+        d[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      }
+    } else {
+      d[0] += __shfl_xor_sync(0xffffffffu, d[0], o);
+    }
+  }
+#pragma unroll
+  for (int lvl = 4; lvl >= 0; --lvl) {
+    const int o = 16 >> lvl, width = NP >> lvl;
+    if (width > 1) {
+      const int half = width >> 1;
+      const bool up = (lane & o) != 0;
+      float r[NP / 2];
+#pragma unroll
+      for (int i = 0; i < half; ++i) r[i] = __shfl_xor_sync(0xffffffffu, d[i], o);
+#pragma unroll
+      for (int i = 0; i < half; ++i) {
+        const float mine = d[i];
+        d[i] = up ? r[i] : mine;
+        d[i + half] = up ? mine : r[i];
+      }
+    }
+  }
 }
 
 // exclusive prefix sum of a 0/1 flag over the block (blockDim.x = 1024); *total gets the sum
@@ -204,29 +239,48 @@ __global__ void __launch_bounds__(kSekvWarps * 32)
   }
 }
 
-// one warp per (kv head, span): expanded = max_h q_h . kbar / sqrt(D) >= theta
+// one warp per four (kv head, span) pairs at a time: expanded = max_h q_h . kbar / sqrt(D) >= theta
 template <typename T, int DPL, int G>
 __global__ void __launch_bounds__(kSekvWarps * 32)
     sekv_gate_kernel(const T* __restrict__ q, int Hq, int Hkv, int cap, const int32_t* counts,
                      const float* __restrict__ kbar, float scale, float theta, uint8_t* expanded) {
-  constexpr int D = 32 * DPL;
+  constexpr int D = 32 * DPL, KB = 4, NPAIR = G * KB;
+  constexpr int NP = NPAIR <= 4 ? 4 : (NPAIR <= 8 ? 8 : (NPAIR <= 16 ? 16 : 32));
   const int u = blockIdx.x, b = u / Hkv, kvh = u % Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nspans = counts[b * 2 + 1];
   float qx[G][DPL];
 #pragma unroll
   for (int h = 0; h < G; ++h) load_dims<T, DPL>(q + ((size_t)b * Hq + (size_t)kvh * G + h) * D, lane, qx[h]);
-  for (int i = blockIdx.y * kSekvWarps + warp; i < nspans; i += gridDim.y * kSekvWarps) {
-    const float* kr = kbar + ((size_t)u * cap + i) * D + lane * DPL;
-    float g = -INFINITY;
+  const int stride = gridDim.y * kSekvWarps;
+  for (int base = blockIdx.y * kSekvWarps + warp; base < nspans; base += KB * stride) {
+    float kx[KB][DPL];
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float d = 0.f;
+    for (int k = 0; k < KB; ++k) {
+      const int i = base + k * stride;
+      const float* kr = kbar + ((size_t)u * cap + (i < nspans ? i : 0)) * D + lane * DPL;
 #pragma unroll
-      for (int j = 0; j < DPL; ++j) d = fmaf(qx[h][j], kr[j], d);
-      g = fmaxf(g, warp_allsum(d) * scale);
+      for (int j = 0; j < DPL; ++j) kx[k][j] = i < nspans ? kr[j] : 0.f;
     }
-    if (lane == 0) expanded[(size_t)u * cap + i] = g >= theta ? 1 : 0;
+    float d[NP];
+#pragma unroll
+    for (int v = 0; v < NP; ++v) {
+      float t = 0.f;
+      if (v < NPAIR) {
+#pragma unroll
+        for (int j = 0; j < DPL; ++j) t = fmaf(qx[v / KB][j], kx[v % KB][j], t);
+      }
+      d[v] = t;
+    }
+    warp_sum_all<NP>(d, lane);
+#pragma unroll
+    for (int k = 0; k < KB; ++k) {
+      const int i = base + k * stride;
+      float g = -INFINITY;
+#pragma unroll
+      for (int h = 0; h < G; ++h) g = fmaxf(g, d[h * KB + k] * scale);
+      if (lane == k && i < nspans) expanded[(size_t)u * cap + i] = g >= theta ? 1 : 0;
+    }
   }
 }
 
@@ -462,42 +516,7 @@ __global__ void __launch_bounds__(kSekvWarps * 32) sekv_attend_kernel(SekvAttend
       }
       d[v] = t;
     }
-    // reduce-scatter: at the level of partner distance o the lane keeps the lower or upper half
-    // of its block (by bit o of its lane index) and adds the partner's copy of that half
-#pragma unroll
-    for (int lvl = 0; lvl < 5; ++lvl) {
-      const int o = 16 >> lvl, width = NP >> lvl;
-      if (width > 1) {
-        const int half = width >> 1;
-        const bool up = (lane & o) != 0;
-#pragma unroll
-        for (int i = 0; i < half; ++i) {
-          const float send = up ? d[i] : d[i + half];
-          const float keep = up ? d[i + half] : d[i];
-          d[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-        }
-      } else {
-        d[0] += __shfl_xor_sync(0xffffffffu, d[0], o);
-      }
-    }
-    // all-gather, the same levels in reverse: blocks double until every lane holds all NP sums
-#pragma unroll
-    for (int lvl = 4; lvl >= 0; --lvl) {
-      const int o = 16 >> lvl, width = NP >> lvl;
-      if (width > 1) {
-        const int half = width >> 1;
-        const bool up = (lane & o) != 0;
-        float r[NP / 2];
-#pragma unroll
-        for (int i = 0; i < half; ++i) r[i] = __shfl_xor_sync(0xffffffffu, d[i], o);
-#pragma unroll
-        for (int i = 0; i < half; ++i) {
-          const float mine = d[i];
-          d[i] = up ? r[i] : mine;
-          d[i + half] = up ? mine : r[i];
-        }
-      }
-    }
+    warp_sum_all<NP>(d, lane);
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       float sc[KB], mx = m[h];
