@@ -44,7 +44,7 @@ FALLBACK_HBM_GBS = 6650.0
 # capture, and the digest of the decode kernel's sources it was taken with: the bench reports
 # the traffic only while the sources still hash to that digest.
 DECODE_TRAFFIC_BYTES = 108935680 + 4205056
-DECODE_TRAFFIC_SOURCES_SHA = "518e020e94bf65e8"
+DECODE_TRAFFIC_SOURCES_SHA = "2478175b16d07d0d"
 DECODE_SOURCES = ("decode.cu", "int2_block.cuh", "append.cuh", "qe_internal.cuh", "warp_mma.cuh", "tc_common.cuh")
 
 

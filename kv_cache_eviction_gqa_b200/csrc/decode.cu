@@ -6,37 +6,42 @@
 // readable by attention (Metodologia 2); GQA decode path (Implementação).
 // "Resumo Técnico: CriticalKV" - Etapa 2: the perturbation score A_i * ||V_i W_O||_1.
 //
-// Work split. Per unit u = (b, g) the live windows are [full windows | tail | INT2 windows].
+// Work split. Per unit u = (b, g) the live windows are [tail | full windows | INT2 windows].
 // The unit's S CTAs form one thread-block cluster; CTA s takes the s-th S-th of the full
 // windows and of the INT2 windows (the tail counts as one more INT2 window of the last CTA),
 // so every SM streams the same mix of bandwidth-heavy full pages and compact INT2 entries.
-// Inside a CTA each warp takes whole windows round-robin and streams them as tasks of at most
-// 16*D*2 bytes through its own ring of shared-memory stages (completion on an mbarrier per
-// stage): the K rows of a full or tail page, its V rows (128-byte-swizzled TMA boxes from a
-// tensor map over the page pool), or a chunk of up to 32 tokens of an INT2 ledger entry (one
-// 1-D bulk copy), each with its tokens' projected-value norms.
+// Inside a CTA warp w takes windows w, w + kNW, ...; even warps walk them in list order, odd
+// warps start with their INT2 windows, so some warps of an SM stream full pages while others
+// do the INT2 arithmetic. A warp streams its windows as tasks of 16*D*2 bytes through its own
+// ring of shared-memory stages (completion on an mbarrier per stage): the K rows of a full or
+// tail page, its V rows (128-byte-swizzled TMA boxes from a tensor map over the page pool), or
+// a chunk of up to 32 tokens of an INT2 ledger entry (one 1-D bulk copy), each with its
+// tokens' projected-value norms.
 //
-// Every tier runs on the warp-level tensor cores (mma.sync, f32 accumulate) in one register
-// layout: the G query heads of the group are the rows of S = Q K^T (padded to 16), 16 tokens
-// are its columns, so lane (r, t) holds head r's scores of tokens 2t, 2t+1, 8+2t, 9+2t - which
-// is exactly the B fragment of O^T = V^T P^T. A decode step has G <= 8 query rows per KV head;
-// a tcgen05 tile (M >= 64) would be mostly padding and its TMEM round trip buys nothing on a
-// path that HBM bounds, so the decode stays on mma.sync.
+// Every tier runs on the warp-level tensor cores (mma.sync, f32 accumulate) with the tokens
+// as MMA rows: S^T = K Q^T takes 16 tokens as the A operand and the G <= 8 query heads of the
+// group as the B columns (no padding rows), so lane (r, t) holds the scores of tokens r and
+// 8 + r for heads 2t and 2t + 1; P^T goes through movmatrix into the B fragment of
+// O^T = V^T P^T. A decode step has G <= 8 query heads per KV head; a tcgen05 tile (M >= 64)
+// would be mostly padding and its TMEM round trip buys nothing on a path that HBM bounds, so
+// the decode stays on mma.sync.
 //
-// Full-precision pages: S from ldmatrix K tiles (four independent accumulator chains), P split
+// Full-precision pages: S^T from ldmatrix K tiles (two independent accumulator chains), P split
 // into two 16-bit parts of the cache dtype (hi + residual) so O keeps float32 accuracy, V^T by
 // ldmatrix.trans.
 //
 // INT2 blocks (16 tokens, layout in int2_block.cuh): a K or V value is c*s + z with a 2-bit code
 // c and an fp16 scale s and zero z per 16-element group. The codes enter the MMA exactly as
 // fp16 subnormals c * 4^i * 2^-24 (one mask per register); per group g
-//   S += s_g * (Q_g . C_g)  (one MMA per 8 tokens, then an f32x2 FMA by the token scales),
-//   S += Z (sum of q over each group)  (one m16n8k8 MMA per 8 tokens, q sums split hi + lo),
-//   O_g^T += C_g^T (P * s_g)  (one MMA per group; P * s rounded once to fp16),
-//   O^T += Z^T P  (one MMA per 16 tokens, P split hi + lo).
+//   S^T += s_g * (C_g Q_g^T)  (one MMA per 16 tokens, then an f32x2 FMA by the token scales),
+//   S^T += Z (sum of q over each group)  (m16n8k8 MMAs, q sums split hi + lo),
+//   O_g^T += C_g^T (P^T s_g)  (two MMAs per group: the weight-times-scale operand carried as
+//                              an exact fp16 sum hi + lo),
+//   O^T += Z^T P^T  (one MMA per 16 tokens and 16-bit part of P).
 // The token scales reach the lanes that need them as float32 through one more MMA per group
 // (the group's scales times a 0/1 selection matrix), so no conversion or staging is needed.
-// The powers 4^i and 2^-24 are folded into q, the selection matrix and the accumulator.
+// The powers 4^i and 2^-24 are folded into q, the selection matrix and the accumulator, which
+// holds O^T scaled by 2^-24 (rows 0-7) and 2^-20 (rows 8-15) while INT2 chunks stream.
 //
 // Scoring without a second pass: at the end of each window the warp records its
 // (max, sum_i 2^(s_i-max), sum_i 2^(s_i-max) n_i) per head. After the pass the cluster merges
