@@ -543,31 +543,67 @@ __global__ void __launch_bounds__(kSekvWarps * 32) sekv_attend_kernel(SekvAttend
       m[h] = mx;
     }
   };
-  auto clear_slot = [&](float (&kx)[DPL], float (&vx)[DPL], float& bias) {
+  // The warp's batches of KB summaries flow through its gather ring (now idle), split into four
+  // slots of KB key rows and KB value rows, three batches in flight ahead of the one computed.
+  // Batch c holds the warp's summaries base_c + k * kSekvWarps (k < KB), base_c = sa + warp +
+  // c * KB * kSekvWarps; a slot's rows are float32, lane l reading its DPL elements.
+  constexpr int SROW = D * 4;                 // one float32 row
+  constexpr int SLOT = 2 * KB * SROW;         // KB key rows, then KB value rows
+  static_assert(4 * SLOT <= 2 * TILE, "four summary slots fit in a warp's gather ring");
+  __shared__ float sbias[kSekvWarps][4][KB];
+  const int nbatch = sbn > sa + warp ? (sbn - sa - warp + KB * kSekvWarps - 1) / (KB * kSekvWarps) : 0;
+  auto sgather = [&](int c) {
+    if (c < nbatch) {
+      const int base = sa + warp + c * KB * kSekvWarps;
+      uint8_t* slot = ring + (c & 3) * SLOT;
+      // lane k < KB: the k-th summary's span index and its log2-size bias (-inf when absent)
+      int i = -1;
+      if (lane < KB) {
+        const int it = base + lane * kSekvWarps;
+        if (it < sbn) {
+          i = a.sums[(size_t)u * a.cap + it];
+          const int s0 = a.span_start[(size_t)b * a.cap + i], e0 = a.span_end[(size_t)b * a.cap + i];
+          sbias[warp][c & 3][lane] = log2f((float)(e0 - s0));  // the summary stands for e0 - s0 tokens
+        } else {
+          sbias[warp][c & 3][lane] = -INFINITY;
+        }
+      }
 #pragma unroll
-    for (int j = 0; j < DPL; ++j) kx[j] = vx[j] = 0.f;
-    bias = -INFINITY;
+      for (int x = 0; x < 2 * KB * SROW / 16 / 32; ++x) {
+        const int ch = lane + 32 * x;           // 16-byte chunk of the slot
+        const int row = ch / (SROW / 16);       // 0..KB-1 keys, KB..2KB-1 values
+        const int k = row % KB, w16 = ch % (SROW / 16);
+        const int ik = __shfl_sync(0xffffffffu, i, k);
+        const float* src = (row < KB ? a.kbar : a.vbar) + ((size_t)u * a.cap + (ik >= 0 ? ik : 0)) * D + w16 * 4;
+        cp_async16(slot + row * SROW + w16 * 16, src, ik >= 0 ? 16 : 0);
+      }
+    }
+    cp_async_commit();  // one group per batch index, empty past the end, so the waits below line up
   };
-  for (int base = sa + warp; base < sbn; base += KB * kSekvWarps) {
+  sgather(0);
+  sgather(1);
+  sgather(2);
+  for (int c = 0; c < nbatch; ++c) {
+    cp_async_wait<2>();
+    __syncwarp();
+    const uint8_t* slot = ring + (c & 3) * SLOT;
     float kx[KB][DPL], vx[KB][DPL], bias[KB];
 #pragma unroll
     for (int k = 0; k < KB; ++k) {
-      clear_slot(kx[k], vx[k], bias[k]);
-      const int it = base + k * kSekvWarps;
-      if (it >= sbn) continue;
-      const int i = a.sums[(size_t)u * a.cap + it];
-      const int s0 = a.span_start[(size_t)b * a.cap + i], e0 = a.span_end[(size_t)b * a.cap + i];
-      const float* kr = a.kbar + ((size_t)u * a.cap + i) * D + lane * DPL;
-      const float* vr = a.vbar + ((size_t)u * a.cap + i) * D + lane * DPL;
+      const float* kr = reinterpret_cast<const float*>(slot + k * SROW) + lane * DPL;
+      const float* vr = reinterpret_cast<const float*>(slot + (KB + k) * SROW) + lane * DPL;
 #pragma unroll
       for (int j = 0; j < DPL; ++j) {
         kx[k][j] = kr[j];
         vx[k][j] = vr[j];
       }
-      bias[k] = log2f((float)(e0 - s0));  // the summary stands for e0 - s0 tokens
+      bias[k] = sbias[warp][c & 3][k];
     }
     take_batch(kx, vx, bias);
+    __syncwarp();  // the slot is read before the next gather into it
+    sgather(c + 3);
   }
+  cp_async_wait<0>();
 
   // ---- merge the warp's two partial states, then the warps, into the CTA partial ----
   __syncthreads();  // every warp is done with its gather ring, which now holds the merge
