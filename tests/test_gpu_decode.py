@@ -44,8 +44,11 @@ def test_small_sequences(cfg):
 # append inside the decode launch, routing in the same call); the oracle follows sampled units
 @pytest.mark.slow
 def test_c2_full_size_sampled_units():
+    """The benched call (qe_decode_step: append fused into the decode launch, routing every 16
+    steps) at full c2 size, all 64 steps, on eight units spread over every batch row and kv head
+    (unit 9k: batch k, kv head k mod 8)."""
     cfg = W.C2
-    units = [0, cfg.units - 1]
+    units = [9 * k for k in range(8) if 9 * k < cfg.units]
     rep = run_decode_parity(cfg, check_units=units, fused=True)
     assert rep.steps == cfg.steps and rep.route_events == 4 * len(units) and rep.codes_checked > 0
     print(rep)
