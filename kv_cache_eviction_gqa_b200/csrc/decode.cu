@@ -113,6 +113,15 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
 __device__ __forceinline__ float ld_cluster(const float* local, uint32_t rank) {
   uint32_t a;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(local)), "r"(rank));
@@ -171,9 +180,14 @@ __device__ __forceinline__ uint32_t __hfma2_u32(uint32_t a, uint32_t b, uint32_t
 // an unevaluated fp16 sum hi + lo: hi = fl(wh s); lo = fl(fl(wh s - hi) + wl s), where wh s - hi
 // (the rounding error of a product) is exact in fp16 barring underflow, so hi + lo carries
 // w s to about 2^-20 relative, where the single product wh s (dropping wl) is off by up to 2^-10.
+// The error term is one fused multiply-add with a negated addend (the negation folds into it).
 __device__ __forceinline__ void ws_split(uint32_t wh, uint32_t wl, uint32_t sc, uint32_t& hi, uint32_t& lo) {
   hi = __hmul2_u32(wh, sc);
-  lo = __hfma2_u32(wl, sc, __hfma2_u32(wh, sc, hi ^ 0x80008000u));
+  uint32_t e;
+  asm("{\n\t.reg .b32 n;\n\tneg.f16x2 n, %2;\n\tfma.rn.f16x2 %0, %1, %3, n;\n\t}"
+      : "=r"(e)
+      : "r"(wh), "r"(hi), "r"(sc));
+  lo = __hfma2_u32(wl, sc, e);
 }
 
 // Register i (0..3) of a packed code word: the codes at bits [2i, 2i+1] of each 16-bit half as
@@ -470,8 +484,11 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
   Cursor cc, ci;  // the task being computed, the next task to copy
   cur_set(cc, 0);
   cur_set(ci, 0);
+  // The first task's copies go out at once; the rest of the prologue's copies only after the
+  // query operands are set up, so that at launch, when every warp of the grid asks for its
+  // stages together, the first stages are not queued behind the later ones.
   int issued = 0;
-  for (int s = 0; s < NST - 1 && ci.o < n_own; ++s) {
+  for (int s = 0; s < 1 && ci.o < n_own; ++s) {
     issue(ci, s);
     cur_next(ci);
     ++issued;
@@ -541,6 +558,11 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
       oacc[m][3] *= hi;
     }
   };
+  for (int s = issued; s < NST - 1 && ci.o < n_own; ++s) {
+    issue(ci, s);
+    cur_next(ci);
+    ++issued;
+  }
   bool int2_units = false;
   uint32_t ph0 = 0, pl0 = 0, ph1 = 0, pl1 = 0;  // P^T of the last K task, for its V task
   int valid = QE_PAGE;
@@ -726,30 +748,41 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
     l1 += __shfl_xor_sync(0xffffffffu, l1, o2);
   }
 
-  // ---- merge the warps into the CTA's partial ----
-  const bool cta_ok = __syncthreads_and(ok ? 1 : 0) != 0;  // also: every warp is done with its ring
-  // the window scores this CTA updates: fetch their ids, partials and cumulative values now so
-  // that the loads overlap the merges below (one window per thread and pass)
+  // the window scores this CTA updates (one window per thread and pass): their ids and
+  // cumulative values are fetched before the CTA barrier, so that the loads overlap the wait for
+  // the slowest warp; their step partials (written by any warp of the CTA) after it
   constexpr int kPre = 1;
-  int pw_win[kPre];
+  int pw_win[kPre], pw_li[kPre];
   float pw_m[kPre], pw_p[kPre], pw_part[kPre][3 * G];
 #pragma unroll
   for (int x = 0; x < kPre; ++x) {
     const int jj = threadIdx.x + x * kNW * 32;
     pw_win[x] = -1;
+    pw_li[x] = 0;
     if (jj < nF + nQ) {
       const int li = jj < nF ? f0 + jj : nf + q0 + (jj - nF);
       const int win = jj < nF ? st.full_list[ub + li] : st.int2_list[ub + li - nf];
       if (win >= 0 && win < st.Wmax) {
         pw_win[x] = win;
+        pw_li[x] = li;
         pw_m[x] = st.mass[ub + win];
         pw_p[x] = st.pert[ub + win];
-        const float* wp = a.win_part + (ub + li) * win_part_floats(D, G);
-#pragma unroll
-        for (int h = 0; h < 3 * G; ++h) pw_part[x][h] = wp[h];
       }
     }
   }
+  // the tail's cumulative per-token attention, read at the end
+  if (has_tail)
+    for (int i = threadIdx.x * 32; i < a.tail_len * G; i += blockDim.x * 32)
+      prefetch_l2(st.tail_p + (size_t)u * W * G + i);
+  // ---- merge the warps into the CTA's partial ----
+  const bool cta_ok = __syncthreads_and(ok ? 1 : 0) != 0;  // also: every warp is done with its ring
+#pragma unroll
+  for (int x = 0; x < kPre; ++x)
+    if (pw_win[x] >= 0) {
+      const float* wp = a.win_part + (ub + pw_li[x]) * win_part_floats(D, G);
+#pragma unroll
+      for (int h = 0; h < 3 * G; ++h) pw_part[x][h] = wp[h];
+    }
   float* mw = reinterpret_cast<float*>(smem);  // [kNW][G]
   float* lwv = mw + kNW * G;                   // [kNW][G]
   float* aw = lwv + kNW * G;                   // [kNW][G][D]
@@ -812,7 +845,18 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
   // ---- the unit's S CTAs form one cluster: merge the partials through distributed
   // shared memory; each CTA writes its share of the output and the scores of its windows ----
   const int S = a.splits;
+  const int per = (G * D + S - 1) / S;
+  const int o1 = min((split + 1) * per, G * D);
+  const int i_first = split * per + threadIdx.x;
   cluster_sync();
+  // this thread's first output element: its S partials are fetched in the same round as the
+  // CTA maxima and sums
+  float vfirst[QE_MAX_SPLITS_CLUSTER];
+  if (i_first < o1) {
+#pragma unroll
+    for (int r = 0; r < QE_MAX_SPLITS_CLUSTER; ++r)
+      if (r < S) vfirst[r] = ld_cluster(ca + i_first, (uint32_t)r);
+  }
   for (int i = threadIdx.x; i < S * G; i += blockDim.x) {
     const float vm = ld_cluster(cm + i % G, (uint32_t)(i / G));
     const float vl = ld_cluster(cl + i % G, (uint32_t)(i / G));
@@ -839,10 +883,16 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
     lse[h] = M + log2f(L);
   }
   __syncthreads();
+  if (i_first < o1) {
+    const int h = i_first / D;
+    float A = 0.f;
+#pragma unroll
+    for (int r = 0; r < QE_MAX_SPLITS_CLUSTER; ++r)
+      if (r < S) A = fmaf(vfirst[r], pf[r * G + h], A);
+    a.out[((size_t)b * st.Hq + (size_t)kvh * G + h) * D + i_first % D] = A / gl[h];
+  }
   {
-    const int per = (G * D + S - 1) / S;
-    const int i1 = min((split + 1) * per, G * D);
-    for (int i = split * per + threadIdx.x; i < i1; i += blockDim.x) {
+    for (int i = i_first + blockDim.x; i < o1; i += blockDim.x) {
       const int h = i / D;
       float v[QE_MAX_SPLITS_CLUSTER];
 #pragma unroll
@@ -855,6 +905,9 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
       a.out[((size_t)b * st.Hq + (size_t)kvh * G + h) * D + i % D] = A / gl[h];
     }
   }
+  // this CTA has read every partial it needs from the cluster: signal it now, and wait for the
+  // other CTAs (which may still read this CTA's partial) only before exiting
+  cluster_arrive();
   if (all_ok > 0.f) {
     // exact attention mass and perturbation of this step for the windows this CTA streamed
     auto update = [&](int win, float m0, float p0, const float* wp) {
@@ -896,7 +949,7 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
       }
     }
   }
-  cluster_sync();  // keep this CTA's partial alive until every CTA of the cluster has read it
+  cluster_wait();  // keep this CTA's partial alive until every CTA of the cluster has read it
 }
 
 template <typename T, int D, int G, int W>
