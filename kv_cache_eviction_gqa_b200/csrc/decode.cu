@@ -113,14 +113,11 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void cluster_arrive() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 __device__ __forceinline__ float ld_cluster(const float* local, uint32_t rank) {
   uint32_t a;
@@ -770,12 +767,25 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
       }
     }
   }
-  // the tail's cumulative per-token attention, read at the end
-  if (has_tail)
-    for (int i = threadIdx.x * 32; i < a.tail_len * G; i += blockDim.x * 32)
-      prefetch_l2(st.tail_p + (size_t)u * W * G + i);
+  float tail_m0 = 0.f;  // the tail window's cumulative mass
+  if (has_tail && threadIdx.x == 0) tail_m0 = st.mass[ub + a.tail_win];
   // ---- merge the warps into the CTA's partial ----
   const bool cta_ok = __syncthreads_and(ok ? 1 : 0) != 0;  // also: every warp is done with its ring
+  // the tail tokens' scores (written by a warp of this CTA during the pass) and cumulative
+  // attention, fetched now so that the loads overlap the merges
+  constexpr int kTailPer = (W * G + kNW * 32 - 1) / (kNW * 32);
+  float t_s[kTailPer], t_p[kTailPer];
+  if (has_tail) {
+#pragma unroll
+    for (int x = 0; x < kTailPer; ++x) {
+      const int i = threadIdx.x + x * kNW * 32;
+      t_s[x] = t_p[x] = 0.f;
+      if (i < a.tail_len * G) {
+        t_s[x] = a.tail_s[(size_t)u * W * G + i];
+        t_p[x] = st.tail_p[(size_t)u * W * G + i];
+      }
+    }
+  }
 #pragma unroll
   for (int x = 0; x < kPre; ++x)
     if (pw_win[x] >= 0) {
@@ -905,9 +915,10 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
       a.out[((size_t)b * st.Hq + (size_t)kvh * G + h) * D + i % D] = A / gl[h];
     }
   }
-  // this CTA has read every partial it needs from the cluster: signal it now, and wait for the
-  // other CTAs (which may still read this CTA's partial) only before exiting
-  cluster_arrive();
+  // this CTA has read every partial it needs from the cluster (the values are in registers,
+  // there is nothing to order): signal it now, and wait for the other CTAs, which may still read
+  // this CTA's partial, only before exiting
+  cluster_arrive_relaxed();
   if (all_ok > 0.f) {
     // exact attention mass and perturbation of this step for the windows this CTA streamed
     auto update = [&](int win, float m0, float p0, const float* wp) {
@@ -933,11 +944,14 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
     // tail tokens (last CTA of the cluster): cumulative per-token attention and window mass
     if (has_tail) {
       float tm = 0.f;
-      for (int i = threadIdx.x; i < a.tail_len * G; i += blockDim.x) {
-        const int h = i % G;
-        const float pv = ex2(a.tail_s[(size_t)u * W * G + i] - lse[h]);
-        st.tail_p[(size_t)u * W * G + i] += pv;
-        tm += pv;
+#pragma unroll
+      for (int x = 0; x < kTailPer; ++x) {
+        const int i = threadIdx.x + x * kNW * 32;
+        if (i < a.tail_len * G) {
+          const float pv = ex2(t_s[x] - lse[i % G]);
+          st.tail_p[(size_t)u * W * G + i] = t_p[x] + pv;
+          tm += pv;
+        }
       }
       tm = warp_sum(tm);
       if (lane == 0) red[warp] = tm;
@@ -945,7 +959,7 @@ __global__ void __launch_bounds__(kNW * 32, QE_DECODE_MINB)
       if (threadIdx.x == 0) {
         float s2 = 0.f;
         for (int x = 0; x < kNW; ++x) s2 += red[x];
-        st.mass[ub + a.tail_win] += s2;
+        st.mass[ub + a.tail_win] = tail_m0 + s2;
       }
     }
   }
