@@ -610,7 +610,7 @@ constexpr size_t apply_buf_bytes() {  // a padded page image (a block image is s
 }
 template <int D>
 size_t apply_smem_bytes(int units) {
-  return 2 * apply_buf_bytes<D>() + 2 * QE_PAGE * (D / 16 + 1) * 8 + 32 + 4 * (size_t)(units + 1);
+  return apply_buf_bytes<D>() + Int2Block<D>::BYTES + 2 * QE_PAGE * (D / 16 + 1) * 8 + 32 + 4 * (size_t)(units + 1);
 }
 
 // Replace the codes of the elements marked in mask (bit e; elements 0..7 in a, 8..15 in b, pairs
@@ -641,10 +641,11 @@ __global__ void __launch_bounds__(kApplyThreads) apply_kernel(DevState st, const
   extern __shared__ __align__(16) uint8_t sm[];
   const int lane = threadIdx.x & 31, wq = threadIdx.x >> 5;  // wq: 0 K rows, 1 V rows
   const int r = lane >> 2, t4 = lane & 3;
-  float2* prm = reinterpret_cast<float2*>(sm + 2 * PAGES) + wq * QE_PAGE * PS;  // this warp's [16][PS]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + 2 * PAGES + 2 * QE_PAGE * PS * 8);
-  int* info = reinterpret_cast<int*>(bars + 1);  // kind of the item in IN
-  int* pre = reinterpret_cast<int*>(sm + 2 * PAGES + 2 * QE_PAGE * PS * 8 + 32);  // [units + 1]
+  constexpr int BUFS = PAGES + BL::BYTES;      // the page image, then the block image
+  float2* prm = reinterpret_cast<float2*>(sm + BUFS) + wq * QE_PAGE * PS;  // this warp's [16][PS]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + BUFS + 2 * QE_PAGE * PS * 8);
+  int* info = reinterpret_cast<int*>(bars + 1);  // kind of the item whose source is being copied
+  int* pre = reinterpret_cast<int*>(sm + BUFS + 2 * QE_PAGE * PS * 8 + 32);  // [units + 1]
   const int units = unit_only >= 0 ? 1 : st.U;
   const int ppw = st.ppw;
 
@@ -709,16 +710,19 @@ __global__ void __launch_bounds__(kApplyThreads) apply_kernel(DevState st, const
     e_blk = reinterpret_cast<uint4*>(st.slots + ((size_t)u * st.S + slot) * st.slot_bytes + (size_t)pg * BL::BYTES);
     e_page = reinterpret_cast<uint4*>(st.pages + ((size_t)u * st.P + page) * st.page_bytes);
   };
-  // Two buffers: IN receives the item's source by bulk copy (the page to quantise, row by row
-  // into the padded layout, or the ledger block to dequantise), OUT holds its result (the block,
-  // or the padded page) until the bulk store has read it. The next item's copy into IN is
-  // issued as soon as both warps are done with the current one, so it overlaps the store.
-  uint4* dst = nullptr;  // warp 0: where the item in OUT goes
+  // Two buffers, a padded page image and a block image: an item's source arrives by bulk copy in
+  // one (the page to quantise, row by row into the padded layout, or the ledger block to
+  // dequantise) and its result is built in the other, which the bulk store then reads. The next
+  // item's copy is issued as soon as both warps are done with the current item, so it overlaps
+  // the store; when its source buffer is the one the store is reading (the kinds differ), it
+  // first waits for the store to have read it.
+  uint4* dst = nullptr;  // warp 0: where the item's result goes
   uint4* dst_next = nullptr;
   uint32_t par = 0u;     // barrier parity (every thread; the control flow is uniform)
-  bool pend = false;     // warp 0: a copy into IN is in flight
-  uint8_t* in_b = sm;
-  uint8_t* out_b = sm + PAGES;
+  bool pend = false;     // warp 0: a copy is in flight
+  int store_kind = -1;   // warp 0: kind of the item whose store may still read its buffer
+  uint8_t* pg_s = sm;           // the page image
+  uint8_t* img = sm + PAGES;    // the block image
   auto issue = [&](int k) {  // warp 0
     if (k - kb >= 32) load_items(k - k % 32);
     const int src = k - kb;
@@ -728,15 +732,16 @@ __global__ void __launch_bounds__(kApplyThreads) apply_kernel(DevState st, const
     dst_next = kind == 0 ? blp : pgp;
     if (lane == 0) info[0] = kind;
     if (kind < 0) return;
+    if (store_kind >= 0 && store_kind != kind) bulk_wait_read_all();  // the source buffer is free
     pend = true;
     fence_proxy_async_smem();
     if (kind == 0) {
       if (lane == 0) mbar_arrive_expect_tx(&bars[0], 2 * QE_PAGE * D * 2);
       __syncwarp();
-      bulk_g2s(in_b + lane * RS * 2, reinterpret_cast<const uint8_t*>(pgp) + lane * D * 2, D * 2, &bars[0]);
+      bulk_g2s(pg_s + lane * RS * 2, reinterpret_cast<const uint8_t*>(pgp) + lane * D * 2, D * 2, &bars[0]);
     } else if (lane == 0) {
       mbar_arrive_expect_tx(&bars[0], BL::BYTES);
-      bulk_g2s(in_b, blp, BL::BYTES, &bars[0]);
+      bulk_g2s(img, blp, BL::BYTES, &bars[0]);
     }
   };
 
@@ -751,14 +756,12 @@ __global__ void __launch_bounds__(kApplyThreads) apply_kernel(DevState st, const
       continue;
     }
     const bool okw = mbar_wait_bounded(&bars[0], par, st.status, 3000);
-    if (wq == 0) bulk_wait_read_all();  // OUT is free: the store of item k - 1 has read it
+    if (wq == 0) bulk_wait_read_all();  // the result buffer is free: the store of item k - 1 has read it
     ok = __syncthreads_and(okw ? 1 : 0) != 0;
     if (!ok) break;
     par ^= 1u;
     pend = false;
     dst = dst_next;
-    uint8_t* pg_s = kind == 0 ? in_b : out_b;  // the page image (read or written)
-    uint8_t* img = kind == 0 ? out_b : in_b;   // the block image (written or read)
     T* rows = reinterpret_cast<T*>(pg_s) + wq * QE_PAGE * RS;  // this warp's 16 rows
     uint16_t* msc = reinterpret_cast<uint16_t*>(img + (wq ? BL::VS : BL::KS));  // scales
     uint16_t* mzr = reinterpret_cast<uint16_t*>(img + (wq ? BL::VZ : BL::KZ));  // zeros
@@ -876,7 +879,7 @@ __global__ void __launch_bounds__(kApplyThreads) apply_kernel(DevState st, const
       }
     }
     // the result leaves by bulk stores once both warps' writes are visible to the async proxy;
-    // then IN is free for the next item's copy
+    // then the source buffer is free for the next item's copy
     fence_proxy_async_smem();
     __syncthreads();
     if (wq == 0) {
@@ -886,6 +889,7 @@ __global__ void __launch_bounds__(kApplyThreads) apply_kernel(DevState st, const
         bulk_s2g(reinterpret_cast<uint8_t*>(dst) + lane * D * 2, pg_s + lane * RS * 2, D * 2);
       }
       bulk_commit();
+      store_kind = kind;
       if (k + 1 < n_items) issue(k + 1);
     }
   }
