@@ -1130,7 +1130,7 @@ def run_sekv(args):
         "e2e": {"value": len(e2e_ms) / (sum(e2e_ms) / 1e3), "unit": "steps/s", "h2d_bytes_per_step": q.numel() * 2,
                 "d2h_bytes_per_step": out.numel() * 4, "steps": len(e2e_ms)},
         "clocks": clk.summary(),
-        "gpu_launches": args.steps * 3,
+        "gpu_launches": args.steps * 4,  # gate, lists, attend, combine
     }
     print(json.dumps(line), flush=True)
 
